@@ -1,0 +1,249 @@
+/*
+ * halo_oracle.c -- plain, slow, double-precision CPU oracle for HaloNet's
+ * blocked local self-attention with haloing.
+ *
+ * TEST INFRASTRUCTURE ONLY.  Only the test suite, the package's smoke() check
+ * and the benchmark's CPU-baseline leg may load this library.  It shares no
+ * code, header, table or helper with the CUDA path and the CUDA path never
+ * calls it.
+ *
+ * What it computes (HaloNet, "Scaling Local Self-Attention for Parameter
+ * Efficient Visual Backbones"):
+ *   - Section 2.2 and Figure 1: the H x W map is cut into non-overlapping
+ *     b x b query blocks; each block shares one (b+2h) x (b+2h) neighbourhood
+ *     made of the block plus an h-pixel halo, padded at the image border.
+ *   - Section 2.1: each logit is a content-content term q.k plus a
+ *     content-geometry term q.r with r indexed by relative position; the
+ *     relative embedding is shared by all heads (footnote 1).
+ *   - Appendix A: the relative embedding is factorised along height and
+ *     width.  Following the blog page's RelPosEmb module, two full-width
+ *     tables rel_h, rel_w of shape [2w-1, d] are summed.
+ *   - Blog page, HaloAttention.forward: q is scaled by d^-1/2 before both the
+ *     content and the relative logits, keys outside the image are removed from
+ *     the softmax, softmax over the window, then the weighted sum of v.
+ *   - Section 2.2 and Figure 2: the stride-2 variant subsamples the queries
+ *     like a strided convolution and keeps the stride-1 neighbourhood.
+ *
+ * Readings where the pages are silent or garbled:
+ *   relative index  = (key window coordinate) - (query in-block coordinate)
+ *                     + w - 1, rows -> rel_h, columns -> rel_w (the blog's
+ *                     rel_to_abs recipe, pinned by a test that restates it);
+ *   out-of-image keys get weight exactly 0 (the blog's printed mask polarity
+ *                     is inverted; the paper pads the border);
+ *   stride 2        = queries at even in-block offsets 0,2,..,b-2; the
+ *                     relative index uses the pixel's in-block offset.
+ *
+ * For each output pixel and head the oracle evaluates the defining formula
+ * directly: every window key's logit, the maximum over in-image keys, the
+ * exponentials, their sum and the weighted sum of v, all in double precision,
+ * from the stored input values (float32, or bf16 widened exactly).
+ *
+ * Build: gcc -O2 -fopenmp -shared -fPIC halo_oracle.c -o liboracle.so -lm
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stddef.h>
+#include <string.h>
+#ifdef _OPENMP
+#include <omp.h>
+#endif
+
+/* dtype codes of the stored inputs */
+#define ORACLE_F32 0
+#define ORACLE_BF16 1
+
+/* Read element i of a float32 or bf16 array as a double (exact widening). */
+static double read_elem(const void *base, size_t i, int dtype)
+{
+    if (dtype == ORACLE_F32) {
+        return (double)((const float *)base)[i];
+    }
+    uint32_t bits = ((uint32_t)((const uint16_t *)base)[i]) << 16;
+    float f;
+    memcpy(&f, &bits, sizeof f);
+    return (double)f;
+}
+
+typedef struct {
+    const void *q, *k, *v, *rel_h, *rel_w;
+    int N, H, W, heads, d, b, h, S, dtype;
+} oracle_args;
+
+/*
+ * One output pixel (n, oy, ox), one head: writes d doubles to out_vec.
+ * Scratch z must hold w*w doubles, valid w*w chars.
+ */
+static void one_pixel_head(const oracle_args *a, int n, int oy, int ox, int head,
+                           double *z, char *valid, double *out_vec)
+{
+    const int w = a->b + 2 * a->h;
+    const int C = a->heads * a->d;
+    const double s = 1.0 / sqrt((double)a->d);
+
+    /* the query pixel and its block */
+    const int y = a->S * oy, x = a->S * ox;
+    const int by = y / a->b, bx = x / a->b;
+    const int qy = y - by * a->b, qx = x - bx * a->b;
+    /* the window's top-left corner in image coordinates */
+    const int y0 = by * a->b - a->h, x0 = bx * a->b - a->h;
+
+    const size_t qoff = (((size_t)n * a->H + y) * a->W + x) * C + (size_t)head * a->d;
+
+    /* logits over the whole window; out-of-image keys are marked invalid */
+    double m = -INFINITY;
+    for (int kr = 0; kr < w; ++kr) {
+        for (int kc = 0; kc < w; ++kc) {
+            const int Y = y0 + kr, X = x0 + kc;
+            const int j = kr * w + kc;
+            if (Y < 0 || Y >= a->H || X < 0 || X >= a->W) {
+                valid[j] = 0;
+                z[j] = 0.0;
+                continue;
+            }
+            valid[j] = 1;
+            const size_t koff = (((size_t)n * a->H + Y) * a->W + X) * C + (size_t)head * a->d;
+            const size_t rh = (size_t)(kr - qy + w - 1) * a->d;
+            const size_t rw = (size_t)(kc - qx + w - 1) * a->d;
+            double acc = 0.0;
+            for (int e = 0; e < a->d; ++e) {
+                const double qe = read_elem(a->q, qoff + e, a->dtype);
+                const double ke = read_elem(a->k, koff + e, a->dtype);
+                const double he = read_elem(a->rel_h, rh + e, a->dtype);
+                const double we = read_elem(a->rel_w, rw + e, a->dtype);
+                acc += qe * (ke + he + we);
+            }
+            z[j] = s * acc;
+            if (z[j] > m) m = z[j];
+        }
+    }
+
+    /* softmax over the in-image keys, then the weighted sum of v */
+    double Z = 0.0;
+    for (int j = 0; j < w * w; ++j) {
+        if (valid[j]) {
+            z[j] = exp(z[j] - m);
+            Z += z[j];
+        }
+    }
+    for (int e = 0; e < a->d; ++e) out_vec[e] = 0.0;
+    for (int kr = 0; kr < w; ++kr) {
+        for (int kc = 0; kc < w; ++kc) {
+            const int j = kr * w + kc;
+            if (!valid[j]) continue;
+            const int Y = y0 + kr, X = x0 + kc;
+            const size_t voff = (((size_t)n * a->H + Y) * a->W + X) * C + (size_t)head * a->d;
+            for (int e = 0; e < a->d; ++e) {
+                out_vec[e] += z[j] * read_elem(a->v, voff + e, a->dtype);
+            }
+        }
+    }
+    for (int e = 0; e < a->d; ++e) out_vec[e] /= Z;
+}
+
+static int check_args(const oracle_args *a)
+{
+    if (!a->q || !a->k || !a->v || !a->rel_h || !a->rel_w) return -1;
+    if (a->N <= 0 || a->H <= 0 || a->W <= 0 || a->heads <= 0 || a->d <= 0 || a->b <= 0 || a->h < 0)
+        return -2;
+    if (a->H % a->b || a->W % a->b) return -3;
+    if (a->S != 1 && a->S != 2) return -4;
+    if (a->b % a->S) return -3;
+    if (a->dtype != ORACLE_F32 && a->dtype != ORACLE_BF16) return -9;
+    if (a->b + 2 * a->h > 4096) return -2;
+    return 0;
+}
+
+/*
+ * Full output: out is [N, H/S, W/S, heads*d] doubles.  threads <= 0 uses the
+ * OpenMP default.  Returns 0, or a negative code for invalid arguments.
+ */
+int halo_oracle_f64(const void *q, const void *k, const void *v,
+                    const void *rel_h, const void *rel_w, double *out,
+                    int N, int H, int W, int heads, int dim_head,
+                    int block, int halo, int stride, int dtype, int threads)
+{
+    oracle_args a = {q, k, v, rel_h, rel_w, N, H, W, heads, dim_head, block, halo, stride, dtype};
+    int rc = check_args(&a);
+    if (rc) return rc;
+    if (!out) return -1;
+    const int OH = H / stride, OW = W / stride, C = heads * dim_head;
+    const int w = block + 2 * halo;
+    const long total = (long)N * heads * OH * OW;
+#ifdef _OPENMP
+    if (threads > 0) omp_set_num_threads(threads);
+#else
+    (void)threads;
+#endif
+#pragma omp parallel
+    {
+        double *z = (double *)__builtin_alloca(sizeof(double) * (size_t)w * w);
+        char *valid = (char *)__builtin_alloca((size_t)w * w);
+        double *vec = (double *)__builtin_alloca(sizeof(double) * (size_t)dim_head);
+#pragma omp for schedule(static)
+        for (long u = 0; u < total; ++u) {
+            /* unit u = (n, head, oy, ox) */
+            long t = u;
+            const int ox = (int)(t % OW); t /= OW;
+            const int oy = (int)(t % OH); t /= OH;
+            const int head = (int)(t % heads); t /= heads;
+            const int n = (int)t;
+            one_pixel_head(&a, n, oy, ox, head, z, valid, vec);
+            double *dst = out + (((size_t)n * OH + oy) * OW + ox) * C + (size_t)head * dim_head;
+            for (int e = 0; e < dim_head; ++e) dst[e] = vec[e];
+        }
+    }
+    return 0;
+}
+
+/*
+ * Sampled output pixels: samples holds nsamples (n, oy, ox) triples; out is
+ * [nsamples, heads*d] doubles.  Used for parity at full sizes, where the whole
+ * output would take the oracle too long.
+ */
+int halo_oracle_samples_f64(const void *q, const void *k, const void *v,
+                            const void *rel_h, const void *rel_w,
+                            const int *samples, int nsamples, double *out,
+                            int N, int H, int W, int heads, int dim_head,
+                            int block, int halo, int stride, int dtype, int threads)
+{
+    oracle_args a = {q, k, v, rel_h, rel_w, N, H, W, heads, dim_head, block, halo, stride, dtype};
+    int rc = check_args(&a);
+    if (rc) return rc;
+    if (!samples || !out) return -1;
+    const int OH = H / stride, OW = W / stride, C = heads * dim_head;
+    const int w = block + 2 * halo;
+    for (int i = 0; i < nsamples; ++i) {
+        const int n = samples[3 * i], oy = samples[3 * i + 1], ox = samples[3 * i + 2];
+        if (n < 0 || n >= N || oy < 0 || oy >= OH || ox < 0 || ox >= OW) return -2;
+    }
+    const long total = (long)nsamples * heads;
+#ifdef _OPENMP
+    if (threads > 0) omp_set_num_threads(threads);
+#else
+    (void)threads;
+#endif
+#pragma omp parallel
+    {
+        double *z = (double *)__builtin_alloca(sizeof(double) * (size_t)w * w);
+        char *valid = (char *)__builtin_alloca((size_t)w * w);
+        double *vec = (double *)__builtin_alloca(sizeof(double) * (size_t)dim_head);
+#pragma omp for schedule(static)
+        for (long u = 0; u < total; ++u) {
+            const int i = (int)(u / heads), head = (int)(u % heads);
+            one_pixel_head(&a, samples[3 * i], samples[3 * i + 1], samples[3 * i + 2], head, z, valid, vec);
+            double *dst = out + (size_t)i * C + (size_t)head * dim_head;
+            for (int e = 0; e < dim_head; ++e) dst[e] = vec[e];
+        }
+    }
+    return 0;
+}
+
+/* Number of OpenMP threads a parallel region would use (for reporting). */
+int halo_oracle_max_threads(void)
+{
+#ifdef _OPENMP
+    return omp_get_max_threads();
+#else
+    return 1;
+#endif
+}
