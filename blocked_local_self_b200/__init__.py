@@ -1,0 +1,116 @@
+"""blocked_local_self_b200 -- HaloNet blocked local self-attention with
+haloing on NVIDIA B200 (sm_100a).
+
+The computation runs entirely in ``libhalo.so`` (hand-written CUDA, C ABI in
+``include/halo.h``).  This module only marshals torch tensors (device memory
+and streams) into that ABI.
+
+    out = attn(q, k, v, rel_h, rel_w, block=8, halo=3, stride=1)
+
+q, k, v: NHWC ``[N, H, W, heads*dim_head]`` CUDA tensors (bf16 or float32),
+rel_h, rel_w: ``[2*(block+2*halo)-1, dim_head]`` of the same dtype.
+Returns ``[N, H/stride, W/stride, heads*dim_head]``.
+"""
+from __future__ import annotations
+
+import torch
+
+from . import _native
+from ._native import HaloError, HALO_BF16, HALO_F32
+
+__all__ = ["attn", "attn_host", "kernel_for", "get_last_error", "debug_wait_timeout", "version", "HaloError",
+           "load"]
+
+
+def load():
+    """Load libhalo.so (raises ImportError when it has not been built)."""
+    return _native.lib()
+
+
+def _dtype_code(t: torch.Tensor) -> int:
+    if t.dtype == torch.bfloat16:
+        return HALO_BF16
+    if t.dtype == torch.float32:
+        return HALO_F32
+    raise TypeError(f"unsupported dtype {t.dtype}; expected bfloat16 or float32")
+
+
+def _sizes(q: torch.Tensor, rel_h: torch.Tensor, heads: int | None):
+    if q.dim() != 4 or rel_h.dim() != 2:
+        raise ValueError("q must be [N, H, W, C] and rel_h [2w-1, dim_head]")
+    N, H, W, C = q.shape
+    d = rel_h.shape[1]
+    if heads is None:
+        if C % d:
+            raise ValueError(f"channels {C} not a multiple of dim_head {d}")
+        heads = C // d
+    return N, H, W, heads, d
+
+
+def _stream_ptr(stream) -> int:
+    if stream is None:
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(stream, torch.cuda.Stream):
+        return stream.cuda_stream
+    return int(stream)
+
+
+def attn(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, rel_h: torch.Tensor, rel_w: torch.Tensor,
+         block: int, halo: int, stride: int = 1, heads: int | None = None, out: torch.Tensor | None = None,
+         stream=None) -> torch.Tensor:
+    """Blocked local self-attention with haloing on device tensors (asynchronous
+    on ``stream``, default: torch's current stream)."""
+    tensors = (q, k, v, rel_h, rel_w)
+    for t in tensors:
+        if not t.is_cuda:
+            raise ValueError("attn expects CUDA tensors; use attn_host for host buffers")
+        if not t.is_contiguous():
+            raise ValueError("tensors must be contiguous")
+    N, H, W, heads, d = _sizes(q, rel_h, heads)
+    code = _dtype_code(q)
+    if out is None:
+        out = torch.empty((N, H // stride, W // stride, heads * d), dtype=q.dtype, device=q.device)
+    rc = _native.lib().halo_attn(q.data_ptr(), k.data_ptr(), v.data_ptr(), rel_h.data_ptr(), rel_w.data_ptr(),
+                                 out.data_ptr(), N, H, W, heads, d, block, halo, stride, code, _stream_ptr(stream))
+    if rc != 0:
+        raise HaloError(rc)
+    return out
+
+
+def attn_host(q_h: torch.Tensor, k_h: torch.Tensor, v_h: torch.Tensor, rel_h_h: torch.Tensor,
+              rel_w_h: torch.Tensor, out_h: torch.Tensor, staging: dict, block: int, halo: int, stride: int = 1,
+              heads: int | None = None, stream=None) -> torch.Tensor:
+    """End-to-end form on host tensors: copies in, kernel, copy out, all queued
+    on ``stream`` by libhalo.  ``staging`` holds caller-allocated device tensors
+    ``q, k, v, rel_h, rel_w, out`` of matching sizes.  Synchronise the stream
+    before reading ``out_h``."""
+    N, H, W, heads, d = _sizes(q_h, rel_h_h, heads)
+    code = _dtype_code(q_h)
+    s = staging
+    rc = _native.lib().halo_attn_host(
+        q_h.data_ptr(), k_h.data_ptr(), v_h.data_ptr(), rel_h_h.data_ptr(), rel_w_h.data_ptr(), out_h.data_ptr(),
+        s["q"].data_ptr(), s["k"].data_ptr(), s["v"].data_ptr(), s["rel_h"].data_ptr(), s["rel_w"].data_ptr(),
+        s["out"].data_ptr(), N, H, W, heads, d, block, halo, stride, code, _stream_ptr(stream))
+    if rc != 0:
+        raise HaloError(rc, "halo_attn_host")
+    return out_h
+
+
+def kernel_for(N: int, H: int, W: int, heads: int, dim_head: int, block: int, halo: int, stride: int,
+               dtype: torch.dtype) -> str:
+    """Name of the kernel ``attn`` launches for a shape: "tc_bf16", "simt_f32" or "none"."""
+    code = HALO_BF16 if dtype == torch.bfloat16 else HALO_F32
+    k = _native.lib().halo_kernel_for(N, H, W, heads, dim_head, block, halo, stride, code)
+    return {0: "none", 1: "simt_f32", 2: "tc_bf16"}[k]
+
+
+def get_last_error() -> int:
+    return _native.lib().halo_get_last_error()
+
+
+def debug_wait_timeout(limit_us: int, stream=None) -> int:
+    return _native.lib().halo_debug_wait_timeout(limit_us, _stream_ptr(stream))
+
+
+def version() -> int:
+    return _native.lib().halo_version()

@@ -1,0 +1,359 @@
+// halo_api.cu -- host side of libhalo: argument checks, kernel selection,
+// TMA descriptor encoding, launches, error reporting.  See include/halo.h for
+// the contract of every entry point.
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include "../../include/halo.h"
+#include "halo_simt.cuh"
+#include "halo_tc.cuh"
+
+namespace {
+
+constexpr int kVersion = 100;                 // 0.1.0
+constexpr int kMaxDynSmem = 227 * 1024;       // sm_100 opt-in limit per block
+
+const char* status_text(int code) {
+  switch (code) {
+    case HALO_OK: return "ok";
+    case HALO_ERR_NULL: return "a required pointer is NULL";
+    case HALO_ERR_DIMS: return "a size is non-positive or too large";
+    case HALO_ERR_DIVISIBILITY: return "H and W must be multiples of block, and block a multiple of stride";
+    case HALO_ERR_STRIDE: return "stride must be 1 or 2";
+    case HALO_ERR_ALIGN: return "pointers must be 16-byte aligned and heads*dim_head rows a multiple of 16 bytes";
+    case HALO_ERR_UNSUPPORTED: return "no kernel of this library handles this shape";
+    case HALO_ERR_CUDA: return "a CUDA call or kernel launch failed";
+    case HALO_ERR_TIMEOUT: return "a bounded device-side wait ran out";
+    case HALO_ERR_DTYPE: return "dtype must be HALO_F32 or HALO_BF16";
+    case HALO_ERR_ALIAS: return "out overlaps an input";
+    case HALO_ERR_DEVICE: return "the current device is not an sm_100 GPU";
+    default: return "unknown status code";
+  }
+}
+
+struct Shape {
+  int N, H, W, heads, d, block, halo, stride, dtype;
+  size_t elem() const { return dtype == HALO_F32 ? 4 : 2; }
+  size_t in_bytes() const { return static_cast<size_t>(N) * H * W * heads * d * elem(); }
+  size_t out_bytes() const { return static_cast<size_t>(N) * (H / stride) * (W / stride) * heads * d * elem(); }
+  size_t rel_bytes() const { return static_cast<size_t>(2 * (block + 2 * halo) - 1) * d * elem(); }
+};
+
+// Checks that need no pointers.  Order: dtype, sizes, stride, divisibility, row alignment.
+int check_shape(const Shape& s) {
+  if (s.dtype != HALO_F32 && s.dtype != HALO_BF16) return HALO_ERR_DTYPE;
+  if (s.N <= 0 || s.H <= 0 || s.W <= 0 || s.heads <= 0 || s.d <= 0 || s.block <= 0 || s.halo < 0)
+    return HALO_ERR_DIMS;
+  const long long C = static_cast<long long>(s.heads) * s.d;
+  const long long elems = static_cast<long long>(s.N) * s.H * s.W * C;
+  if (C > (1 << 20) || elems >= (1LL << 40) || s.block + 2 * s.halo > 4096 || s.H > (1 << 24) ||
+      s.W > (1 << 24))
+    return HALO_ERR_DIMS;
+  if (s.stride != 1 && s.stride != 2) return HALO_ERR_STRIDE;
+  if (s.H % s.block || s.W % s.block || s.block % s.stride) return HALO_ERR_DIVISIBILITY;
+  if ((C * static_cast<long long>(s.elem())) % 16 != 0) return HALO_ERR_ALIGN;
+  return HALO_OK;
+}
+
+// ----------------------------------------------------------------------------
+// Tensor-core kernel table: (d, window, stride) -> instantiation
+// ----------------------------------------------------------------------------
+using TcKernel = void (*)(const CUtensorMap, const CUtensorMap, const CUtensorMap, const halo::tc::Params);
+
+struct TcEntry {
+  int d, win, stride;
+  TcKernel fn;
+  int (*smem)(int);
+  int stage_bytes;
+  int parts;
+};
+
+template <int D, int WIN, int STRIDE>
+int tc_smem(int stages) { return halo::tc::smem_bytes<D, WIN, STRIDE>(stages); }
+
+#define HALO_TC_ENTRY(D, WIN, S)                                                                 \
+  TcEntry {                                                                                      \
+    D, WIN, S, halo::tc::halo_fwd_tc<D, WIN, S>, tc_smem<D, WIN, S>,                             \
+        halo::tc::Cfg<D, WIN, S>::STAGE_BYTES, halo::tc::Cfg<D, WIN, S>::PARTS                   \
+  }
+#define HALO_TC_WINS(D, S) \
+  HALO_TC_ENTRY(D, 8, S), HALO_TC_ENTRY(D, 10, S), HALO_TC_ENTRY(D, 12, S), HALO_TC_ENTRY(D, 14, S), \
+      HALO_TC_ENTRY(D, 16, S)
+
+const TcEntry kTcTable[] = {
+    HALO_TC_WINS(16, 1), HALO_TC_WINS(32, 1), HALO_TC_WINS(64, 1),
+    HALO_TC_WINS(16, 2), HALO_TC_WINS(32, 2), HALO_TC_WINS(64, 2),
+};
+
+const TcEntry* find_tc(const Shape& s) {
+  if (s.dtype != HALO_BF16 || s.block != halo::tc::kBlock) return nullptr;
+  const int win = s.block + 2 * s.halo;
+  for (const TcEntry& e : kTcTable)
+    if (e.d == s.d && e.win == win && e.stride == s.stride && s.heads % e.parts == 0) return &e;
+  return nullptr;
+}
+
+int select_kernel(const Shape& s) {
+  if (check_shape(s) != HALO_OK) return HALO_KERNEL_NONE;
+  if (find_tc(s)) return HALO_KERNEL_TC_BF16;
+  if (s.d <= 128) return HALO_KERNEL_SIMT_F32;
+  return HALO_KERNEL_NONE;
+}
+
+// ----------------------------------------------------------------------------
+// Device properties and TMA descriptor encoding
+// ----------------------------------------------------------------------------
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+std::mutex g_mutex;
+EncodeTiledFn g_encode = nullptr;
+constexpr int kMaxDevices = 64;
+int g_sm_count[kMaxDevices];
+int g_dev_ok[kMaxDevices];  // 0 unknown, 1 sm_100, -1 other
+
+int device_info(int* sm_count) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return HALO_ERR_CUDA;
+  std::lock_guard<std::mutex> lock(g_mutex);
+  if (g_dev_ok[dev] == 0) {
+    int major = 0, sms = 0;
+    if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+      return HALO_ERR_CUDA;
+    g_dev_ok[dev] = (major == 10) ? 1 : -1;
+    g_sm_count[dev] = sms;
+  }
+  if (g_dev_ok[dev] != 1) return HALO_ERR_DEVICE;
+  *sm_count = g_sm_count[dev];
+  return HALO_OK;
+}
+
+EncodeTiledFn encoder() {
+  std::lock_guard<std::mutex> lock(g_mutex);
+  if (!g_encode) {
+    void* fn = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      g_encode = reinterpret_cast<EncodeTiledFn>(fn);
+  }
+  return g_encode;
+}
+
+// 4-D map over an NHWC bf16 tensor {C, W, H, N}; box {d, bw, bh, 1}.
+bool encode_nhwc(CUtensorMap* m, const void* base, const Shape& s, int bw, int bh, int estride) {
+  EncodeTiledFn enc = encoder();
+  if (!enc) return false;
+  const cuuint64_t C = static_cast<cuuint64_t>(s.heads) * s.d;
+  cuuint64_t dims[4] = {C, static_cast<cuuint64_t>(s.W), static_cast<cuuint64_t>(s.H),
+                        static_cast<cuuint64_t>(s.N)};
+  cuuint64_t strides[3] = {C * 2, C * 2 * s.W, C * 2 * s.W * s.H};
+  cuuint32_t box[4] = {static_cast<cuuint32_t>(s.d), static_cast<cuuint32_t>(bw), static_cast<cuuint32_t>(bh), 1};
+  cuuint32_t es[4] = {1, static_cast<cuuint32_t>(estride), static_cast<cuuint32_t>(estride), 1};
+  const CUtensorMapSwizzle sw = s.d == 16 ? CU_TENSOR_MAP_SWIZZLE_32B
+                                          : (s.d == 32 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_128B);
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, strides, box, es,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+bool overlaps(const void* a, size_t na, const void* b, size_t nb) {
+  const uintptr_t x = reinterpret_cast<uintptr_t>(a), y = reinterpret_cast<uintptr_t>(b);
+  return x < y + nb && y < x + na;
+}
+
+int check_pointers(const void* q, const void* k, const void* v, const void* rel_h, const void* rel_w,
+                   const void* out, const Shape& s) {
+  if (!q || !k || !v || !rel_h || !rel_w || !out) return HALO_ERR_NULL;
+  const void* ptrs[6] = {q, k, v, rel_h, rel_w, out};
+  for (const void* ptr : ptrs)
+    if (reinterpret_cast<uintptr_t>(ptr) % 16) return HALO_ERR_ALIGN;
+  const size_t ob = s.out_bytes(), ib = s.in_bytes(), rb = s.rel_bytes();
+  if (overlaps(out, ob, q, ib) || overlaps(out, ob, k, ib) || overlaps(out, ob, v, ib) ||
+      overlaps(out, ob, rel_h, rb) || overlaps(out, ob, rel_w, rb))
+    return HALO_ERR_ALIAS;
+  return HALO_OK;
+}
+
+template <typename T, int DMAX>
+cudaError_t launch_simt_t(const void* q, const void* k, const void* v, const void* rh, const void* rw, void* out,
+                          const Shape& s, cudaStream_t st) {
+  const long long total = static_cast<long long>(s.N) * (s.H / s.stride) * (s.W / s.stride) * s.heads;
+  const long long blocks = (total + halo::simt::kThreads - 1) / halo::simt::kThreads;
+  if (blocks > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
+  halo::simt::halo_fwd_simt<T, DMAX><<<static_cast<unsigned>(blocks), halo::simt::kThreads, 0, st>>>(
+      static_cast<const T*>(q), static_cast<const T*>(k), static_cast<const T*>(v), static_cast<const T*>(rh),
+      static_cast<const T*>(rw), static_cast<T*>(out), s.N, s.H, s.W, s.heads, s.d, s.block, s.halo, s.stride,
+      1.0f / std::sqrt(static_cast<float>(s.d)));
+  return cudaGetLastError();
+}
+
+template <typename T>
+cudaError_t launch_simt(const void* q, const void* k, const void* v, const void* rh, const void* rw, void* out,
+                        const Shape& s, cudaStream_t st) {
+  if (s.d <= 16) return launch_simt_t<T, 16>(q, k, v, rh, rw, out, s, st);
+  if (s.d <= 32) return launch_simt_t<T, 32>(q, k, v, rh, rw, out, s, st);
+  if (s.d <= 64) return launch_simt_t<T, 64>(q, k, v, rh, rw, out, s, st);
+  return launch_simt_t<T, 128>(q, k, v, rh, rw, out, s, st);
+}
+
+int launch_tc(const TcEntry& e, const void* q, const void* k, const void* v, const void* rh, const void* rw,
+              void* out, const Shape& s, int sm_count, cudaStream_t st) {
+  const int win = s.block + 2 * s.halo;
+  CUtensorMap mq, mk, mv;
+  if (!encode_nhwc(&mq, q, s, halo::tc::kBlock, halo::tc::kBlock, s.stride) ||
+      !encode_nhwc(&mk, k, s, halo::tc::kRowKeys, win, 1) || !encode_nhwc(&mv, v, s, halo::tc::kRowKeys, win, 1))
+    return HALO_ERR_CUDA;
+  // The kernel moves registers between its warpgroups with setmaxnreg; that is
+  // only safe if the launch allocation covers the split (otherwise the
+  // increase would wait forever).  Refuse to launch when it does not.
+  cudaFuncAttributes attr;
+  if (cudaFuncGetAttributes(&attr, reinterpret_cast<const void*>(e.fn)) != cudaSuccess) return HALO_ERR_CUDA;
+  if (256 * halo::tc::kSoftmaxRegs + 128 * halo::tc::kProducerRegs > halo::tc::kThreads * attr.numRegs)
+    return HALO_ERR_UNSUPPORTED;
+  // dynamic shared memory budget: the per-block opt-in limit minus the
+  // kernel's static shared memory (mbarriers and flags)
+  int optin = 0, dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) != cudaSuccess)
+    return HALO_ERR_CUDA;
+  const int budget = (optin < kMaxDynSmem ? optin : kMaxDynSmem) - static_cast<int>(attr.sharedSizeBytes);
+  int stages = 8;
+  while (stages > 1 && e.smem(stages) > budget) --stages;
+  const int smem = e.smem(stages);
+  if (smem > budget) return HALO_ERR_UNSUPPORTED;
+  if (cudaFuncSetAttribute(reinterpret_cast<const void*>(e.fn), cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           smem) != cudaSuccess)
+    return HALO_ERR_CUDA;
+  halo::tc::Params p;
+  p.rel_h = static_cast<const __nv_bfloat16*>(rh);
+  p.rel_w = static_cast<const __nv_bfloat16*>(rw);
+  p.out = static_cast<__nv_bfloat16*>(out);
+  p.N = s.N;
+  p.H = s.H;
+  p.W = s.W;
+  p.heads = s.heads;
+  p.halo = s.halo;
+  p.nbx = s.W / halo::tc::kBlock;
+  p.nby = s.H / halo::tc::kBlock;
+  p.heads_per_item = e.parts;
+  const long long items = static_cast<long long>(s.N) * p.nbx * p.nby * (s.heads / e.parts);
+  if (items > 0x7fffffffLL) return HALO_ERR_DIMS;
+  p.num_items = static_cast<int>(items);
+  p.stages = stages;
+  p.OH = s.H / s.stride;
+  p.OW = s.W / s.stride;
+  p.c = 1.4426950408889634f / std::sqrt(static_cast<float>(s.d));
+  const int grid = static_cast<int>(items < sm_count ? items : sm_count);
+  e.fn<<<grid, halo::tc::kThreads, smem, st>>>(mq, mk, mv, p);
+  return cudaGetLastError() == cudaSuccess ? HALO_OK : HALO_ERR_CUDA;
+}
+
+int attn_device(const void* q, const void* k, const void* v, const void* rel_h, const void* rel_w, void* out,
+                const Shape& s, cudaStream_t st) {
+  int rc = check_shape(s);
+  if (rc != HALO_OK) return rc;
+  rc = check_pointers(q, k, v, rel_h, rel_w, out, s);
+  if (rc != HALO_OK) return rc;
+  const int kind = select_kernel(s);
+  if (kind == HALO_KERNEL_NONE) return HALO_ERR_UNSUPPORTED;
+  int sm_count = 0;
+  rc = device_info(&sm_count);
+  if (rc != HALO_OK) return rc;
+  if (kind == HALO_KERNEL_TC_BF16) return launch_tc(*find_tc(s), q, k, v, rel_h, rel_w, out, s, sm_count, st);
+  cudaError_t err = (s.dtype == HALO_F32) ? launch_simt<float>(q, k, v, rel_h, rel_w, out, s, st)
+                                          : launch_simt<__nv_bfloat16>(q, k, v, rel_h, rel_w, out, s, st);
+  return err == cudaSuccess ? HALO_OK : HALO_ERR_CUDA;
+}
+
+__global__ void wait_timeout_kernel(unsigned long long limit_ns) {
+  __shared__ __align__(8) uint64_t bar;
+  if (threadIdx.x == 0) {
+    halo::sm100::mbar_init(&bar, 1);
+    halo::sm100::fence_mbar_init();
+    // nothing ever arrives on `bar`: the wait must end by its time limit
+    if (!halo::sm100::mbar_wait(&bar, 0, limit_ns)) atomicExch(&halo::g_halo_error, HALO_ERR_TIMEOUT);
+  }
+}
+
+}  // namespace
+
+extern "C" {
+
+int halo_attn(const void* q, const void* k, const void* v, const void* rel_h, const void* rel_w, void* out, int N,
+              int H, int W, int heads, int dim_head, int block, int halo, int stride, int dtype, void* stream) {
+  const Shape s{N, H, W, heads, dim_head, block, halo, stride, dtype};
+  return attn_device(q, k, v, rel_h, rel_w, out, s, static_cast<cudaStream_t>(stream));
+}
+
+int halo_attn_host(const void* q_h, const void* k_h, const void* v_h, const void* rel_h_h, const void* rel_w_h,
+                   void* out_h, void* q_d, void* k_d, void* v_d, void* rel_h_d, void* rel_w_d, void* out_d, int N,
+                   int H, int W, int heads, int dim_head, int block, int halo, int stride, int dtype,
+                   void* stream) {
+  const Shape s{N, H, W, heads, dim_head, block, halo, stride, dtype};
+  int rc = check_shape(s);
+  if (rc != HALO_OK) return rc;
+  if (!q_h || !k_h || !v_h || !rel_h_h || !rel_w_h || !out_h) return HALO_ERR_NULL;
+  rc = check_pointers(q_d, k_d, v_d, rel_h_d, rel_w_d, out_d, s);
+  if (rc != HALO_OK) return rc;
+  if (select_kernel(s) == HALO_KERNEL_NONE) return HALO_ERR_UNSUPPORTED;
+  int sm_count = 0;
+  rc = device_info(&sm_count);
+  if (rc != HALO_OK) return rc;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const size_t ib = s.in_bytes(), rb = s.rel_bytes();
+  if (cudaMemcpyAsync(q_d, q_h, ib, cudaMemcpyHostToDevice, st) != cudaSuccess ||
+      cudaMemcpyAsync(k_d, k_h, ib, cudaMemcpyHostToDevice, st) != cudaSuccess ||
+      cudaMemcpyAsync(v_d, v_h, ib, cudaMemcpyHostToDevice, st) != cudaSuccess ||
+      cudaMemcpyAsync(rel_h_d, rel_h_h, rb, cudaMemcpyHostToDevice, st) != cudaSuccess ||
+      cudaMemcpyAsync(rel_w_d, rel_w_h, rb, cudaMemcpyHostToDevice, st) != cudaSuccess)
+    return HALO_ERR_CUDA;
+  rc = attn_device(q_d, k_d, v_d, rel_h_d, rel_w_d, out_d, s, st);
+  if (rc != HALO_OK) return rc;
+  if (cudaMemcpyAsync(out_h, out_d, s.out_bytes(), cudaMemcpyDeviceToHost, st) != cudaSuccess) return HALO_ERR_CUDA;
+  return HALO_OK;
+}
+
+int halo_kernel_for(int N, int H, int W, int heads, int dim_head, int block, int halo, int stride, int dtype) {
+  const Shape s{N, H, W, heads, dim_head, block, halo, stride, dtype};
+  return select_kernel(s);
+}
+
+const char* halo_strerror(int code) { return status_text(code); }
+
+int halo_get_last_error(void) {
+  if (cudaDeviceSynchronize() != cudaSuccess) return HALO_ERR_CUDA;
+  int flag = 0;
+  const int zero = 0;
+  if (cudaMemcpyFromSymbol(&flag, halo::g_halo_error, sizeof(int)) != cudaSuccess) return HALO_ERR_CUDA;
+  if (cudaMemcpyToSymbol(halo::g_halo_error, &zero, sizeof(int)) != cudaSuccess) return HALO_ERR_CUDA;
+  return flag;
+}
+
+int halo_debug_wait_timeout(int limit_us, void* stream) {
+  if (limit_us < 1 || limit_us > 1000000) return HALO_ERR_DIMS;
+  int sm_count = 0;
+  const int rc = device_info(&sm_count);
+  if (rc != HALO_OK) return rc;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  wait_timeout_kernel<<<1, 32, 0, st>>>(static_cast<unsigned long long>(limit_us) * 1000ull);
+  if (cudaGetLastError() != cudaSuccess || cudaStreamSynchronize(st) != cudaSuccess) return HALO_ERR_CUDA;
+  int flag = 0;
+  const int zero = 0;
+  if (cudaMemcpyFromSymbol(&flag, halo::g_halo_error, sizeof(int)) != cudaSuccess ||
+      cudaMemcpyToSymbol(halo::g_halo_error, &zero, sizeof(int)) != cudaSuccess)
+    return HALO_ERR_CUDA;
+  return flag;
+}
+
+int halo_version(void) { return kVersion; }
+
+}  // extern "C"

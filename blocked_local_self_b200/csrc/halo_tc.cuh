@@ -1,0 +1,530 @@
+// halo_tc.cuh -- fused bf16 blocked local self-attention with haloing for
+// sm_100a: TMA window loads, tcgen05 tensor-core QK^T / relative logits / PV
+// with TMEM accumulators, masked softmax on the CUDA cores.
+//
+// Operation (HaloNet, "Scaling Local Self-Attention for Parameter Efficient
+// Visual Backbones", sections 2.1-2.2 and appendix A; index conventions of the
+// blog page's RelPosEmb / HaloAttention modules):
+//   z[q, key] = s * q . (k[key] + rel_h[kr - qy + w - 1] + rel_w[kc - qx + w - 1])
+//   out[q]    = sum over in-image window keys of softmax(z) * v[key]
+//
+// Design (one CTA per SM, persistent over work items):
+//   * item = one 8x8 query block and one head (stride 1: 64 query rows), or
+//     one block and PARTS heads (stride 2: 16 query rows per head, head p in
+//     rows 16p..16p+15 of a 64-row MMA tile).
+//   * warp 8 (one lane) streams items with TMA: the query tile and, per head,
+//     the w x 16 window of K and of V (w = 8 + 2*halo rows; the window row is
+//     padded from w to 16 keys so every window row is one 32-byte swizzle
+//     chunk of the P operand).  Keys outside the image arrive as zeros.
+//   * warp 9 (one lane) issues tcgen05.mma: S = Q K^T (M=64, N=16w, bf16 in,
+//     f32 in TMEM), G = Q R^T with R = [rel_h; rel_w] (the 2(2w-1) relative
+//     dot products of every query), and after the softmax O = P V (and, for
+//     d = 16, the row sums through a ones tile appended to V).
+//   * warps 0-3 and 4-7 are two softmax warpgroups that take alternate items;
+//     each owns one half of every TMEM lane quadrant (lanes 0-15 or 16-31), so
+//     the MMAs of one item overlap the softmax of the other.  A query row is
+//     split over two threads (tcgen05.ld 16x32bx2): the thread with lane < 16
+//     takes the even window rows, its partner the odd ones.
+//   * per row: gather the relative logits that apply to this query from G,
+//     add them, mask out-of-image keys, exact row max, exponentials (part on
+//     the MUFU unit, part as a cubic polynomial on the FMA pipe), bf16 P into
+//     shared memory, then normalise O and store bf16 NHWC directly.
+//   Nothing but q, k, v, the tables and out touches global memory.
+#pragma once
+
+#include <cstdint>
+#include <cuda.h>
+#include <cuda_bf16.h>
+
+#include "sm100.cuh"
+
+namespace halo {
+
+__device__ int g_halo_error;  // sticky device error flag (HALO_ERR_TIMEOUT)
+
+namespace tc {
+
+using namespace sm100;
+
+constexpr int kBlock = 8;         // query block side handled by this kernel
+constexpr int kRowKeys = 16;      // window row pitch in keys (w padded to 16)
+constexpr int kThreads = 384;     // 2 softmax warpgroups + 1 producer warpgroup
+constexpr int kTmaWarp = 8;       // producer warpgroup: warp 8 TMA, warp 9 MMA,
+constexpr int kMmaWarp = 9;       // warps 10-11 idle
+// Register split (setmaxnreg): the kernel launches with kLaunchRegs per thread
+// (3 warps per SM sub-partition cap it at 168); the producer warpgroup gives
+// registers back and the softmax warpgroups take more.  The sum stays within
+// the launch allocation: 256*216 + 128*56 = 62464 <= 384*168 = 64512.
+constexpr int kLaunchRegs = 168;
+constexpr int kSoftmaxRegs = 216;
+constexpr int kProducerRegs = 56;
+static_assert(256 * kSoftmaxRegs + 128 * kProducerRegs <= kThreads * kLaunchRegs, "register split");
+constexpr uint32_t kTmemCols = 512;
+constexpr uint32_t kTmemS = 0;    // S: columns [0, 16w)
+constexpr uint32_t kTmemG = 256;  // G: columns [256, 320)
+constexpr uint32_t kTmemO = 320;  // O (+ row sums): columns [320, 448)
+constexpr int kGCols = 64;        // rel_h logits at [0, 2w-1), rel_w logits at [32, 32+2w-1)
+constexpr uint64_t kWaitNs = 1000000000ull;  // 1 s bound on every wait
+
+struct Params {
+  const __nv_bfloat16* rel_h;
+  const __nv_bfloat16* rel_w;
+  __nv_bfloat16* out;
+  int N, H, W, heads, halo;
+  int nbx, nby;            // blocks along x and y
+  int num_items;           // total work items
+  int heads_per_item;      // PARTS
+  int stages;              // TMA pipeline depth
+  int OH, OW;
+  float c;                 // log2(e) / sqrt(d)
+};
+
+template <int D, int WIN, int STRIDE>
+struct Cfg {
+  static constexpr int ROWB = D * 2;                      // bytes of one pixel's head slice
+  static constexpr int PARTS = (STRIDE == 1) ? 1 : (D == 16 ? 4 : (D == 32 ? 2 : 1));
+  static constexpr int QROWS_PER_HEAD = (STRIDE == 1) ? 64 : 16;
+  // stride 1: 64-row Q tile.  stride 2: zero-gap buffer so that the 64-row view
+  // of head p holds its 16 queries in rows 16p..16p+15 and zeros elsewhere.
+  static constexpr int QBUF_ROWS = (STRIDE == 1) ? 64 : (112 + 48 * (PARTS - 1));
+  static constexpr int KEYS = WIN * kRowKeys;             // S columns / PV K extent
+  static constexpr int KV_TILE = KEYS * ROWB;             // bytes of one head's K (or V) window
+  static constexpr int Q_BYTES = QBUF_ROWS * ROWB;
+  static constexpr int STAGE_BYTES = Q_BYTES + 2 * PARTS * KV_TILE;
+  static constexpr int TX_BYTES = PARTS * (QROWS_PER_HEAD * ROWB + 2 * KV_TILE);
+  static constexpr int P_TILE = WIN * 2048;               // 64 rows x 16 keys x 2 B per window row
+  static constexpr int R_TILE = kGCols * ROWB;            // [rel_h; rel_w] B operand
+  static constexpr bool SUM_BY_MMA = (D == 16);           // row sums through a ones tile in PV
+  static constexpr int ONES_TILE = SUM_BY_MMA ? KEYS * ROWB : 0;
+  static constexpr int O_COLS = SUM_BY_MMA ? 2 * D : D;   // PV N
+  static constexpr SmemSwizzle SW = (ROWB == 32) ? SW_32B : (ROWB == 64 ? SW_64B : SW_128B);
+  static constexpr uint32_t SBO = 8 * ROWB;               // 8-row core-matrix group stride
+  static constexpr int NROW = WIN / 2;                    // window rows per thread
+  static_assert(WIN % 2 == 0 && WIN <= 16 && WIN >= 8, "window must be even, 8..16");
+  static_assert(D == 16 || D == 32 || D == 64, "dim_head must be 16, 32 or 64");
+  static_assert(PARTS * O_COLS <= 128, "O region");
+};
+
+// Bytes of dynamic shared memory for a given stage count (plus 1 KB alignment slack).
+template <int D, int WIN, int STRIDE>
+__host__ __device__ constexpr int smem_bytes(int stages) {
+  using C = Cfg<D, WIN, STRIDE>;
+  return 1024 + 2 * C::P_TILE + C::R_TILE + C::ONES_TILE + stages * C::STAGE_BYTES;
+}
+
+// Swizzled byte offset of 16-byte unit u of row r in a K-major tile whose
+// rows are ROWB bytes (the TMA / tcgen05 32B, 64B and 128B swizzle patterns).
+template <int ROWB>
+__device__ __forceinline__ uint32_t swz(int r, int u) {
+  if (ROWB == 32) return r * 32 + ((u ^ ((r >> 2) & 1)) << 4);
+  if (ROWB == 64) return r * 64 + ((u ^ ((r >> 1) & 3)) << 4);
+  return r * 128 + ((u ^ (r & 7)) << 4);
+}
+
+// 2^x for x <= 0 on the FMA pipe: x = j + f with j = floor(x), f in [0, 1);
+// 2^f by a cubic fitted to the relative error on [0, 1) with p(0) = 1
+// (max relative error 8.6e-5), and 2^j added to the exponent field.
+// x is clamped at -127 so that masked (-inf) logits give a value < 2^-126.
+__device__ __forceinline__ float exp2_poly(float x) {
+  x = fmaxf(x, -127.0f);
+  const float magic = 12582912.0f;  // 1.5 * 2^23: adding it rounds to an integer
+  float t;
+  asm("add.rm.f32 %0, %1, %2;" : "=f"(t) : "f"(x), "f"(magic));
+  const float j = t - magic;
+  const float f = x - j;
+  float p = fmaf(f, 0.0770670548f, 0.2276449651f);
+  p = fmaf(p, f, 0.6951168180f);
+  p = fmaf(p, f, 1.0f);
+  return __int_as_float(__float_as_int(p) + (__float_as_int(t) << 23));
+}
+
+__device__ __forceinline__ float exp2_mufu(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+  uint32_t r;
+  asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
+  return r;
+}
+
+__device__ __forceinline__ void record_timeout(int* abort_flag) {
+  atomicExch(&g_halo_error, -8);  // HALO_ERR_TIMEOUT
+  *(volatile int*)abort_flag = 1;
+}
+
+template <int D, int WIN, int STRIDE>
+__global__ void __launch_bounds__(kThreads, 1)
+    halo_fwd_tc(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__ CUtensorMap tmap_k,
+                const __grid_constant__ CUtensorMap tmap_v, const Params p) {
+  using C = Cfg<D, WIN, STRIDE>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* sP = smem;                               // 2 x P_TILE (one per warpgroup)
+  uint8_t* sR = sP + 2 * C::P_TILE;                 // R tile
+  uint8_t* sStage = sR + C::R_TILE;                 // stages x STAGE_BYTES
+  // ones tile (d = 16) after the stages: the PV B descriptor reaches it with a
+  // positive leading byte offset from any V tile
+  uint8_t* sOnes = sStage + p.stages * C::STAGE_BYTES;
+
+  __shared__ __align__(8) uint64_t bar_full[8];
+  __shared__ __align__(8) uint64_t bar_empty[8];
+  __shared__ __align__(8) uint64_t bar_sfull[2];
+  __shared__ __align__(8) uint64_t bar_pfull[2];
+  __shared__ __align__(8) uint64_t bar_ofull[2];
+  __shared__ __align__(8) uint64_t bar_tfree[2];
+  __shared__ __align__(8) uint64_t bar_done;
+  __shared__ uint32_t tmem_base_sh;
+  __shared__ int abort_flag;
+
+  const int tid = threadIdx.x;
+  const int warp = tid >> 5;
+  const int lane = tid & 31;
+  const int S = p.stages;
+
+  // ---------------------------------------------------------------- set-up
+  if (tid == 0) {
+    for (int i = 0; i < S; ++i) {
+      mbar_init(&bar_full[i], 1);
+      mbar_init(&bar_empty[i], 1);
+    }
+    for (int g = 0; g < 2; ++g) {
+      mbar_init(&bar_sfull[g], 1);
+      mbar_init(&bar_pfull[g], 4);
+      mbar_init(&bar_ofull[g], 1);
+      mbar_init(&bar_tfree[g], 4);
+    }
+    mbar_init(&bar_done, 1);
+    abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == kTmaWarp && lane == 0) {
+    prefetch_tensormap(&tmap_q);
+    prefetch_tensormap(&tmap_k);
+    prefetch_tensormap(&tmap_v);
+  }
+  // R tile: rows [0, 2w-1) = rel_h, rows [32, 32+2w-1) = rel_w, other rows 0.
+  for (int idx = tid; idx < kGCols * (D / 8); idx += kThreads) {
+    const int r = idx / (D / 8), u = idx % (D / 8);
+    uint4 val = make_uint4(0, 0, 0, 0);
+    if (r < 2 * WIN - 1) val = *reinterpret_cast<const uint4*>(p.rel_h + r * D + u * 8);
+    else if (r >= 32 && r < 32 + 2 * WIN - 1) val = *reinterpret_cast<const uint4*>(p.rel_w + (r - 32) * D + u * 8);
+    *reinterpret_cast<uint4*>(sR + swz<C::ROWB>(r, u)) = val;
+  }
+  if constexpr (C::SUM_BY_MMA) {
+    // ones tile in the same MN-major layout as a V tile: every element 1.0
+    for (int idx = tid; idx < C::ONES_TILE / 16; idx += kThreads)
+      reinterpret_cast<uint4*>(sOnes)[idx] = make_uint4(0x3f803f80u, 0x3f803f80u, 0x3f803f80u, 0x3f803f80u);
+  }
+  if constexpr (STRIDE == 2) {
+    // zero the query buffers: the TMA only ever writes the 16-row head slots
+    for (int s = 0; s < S; ++s)
+      for (int idx = tid; idx < C::Q_BYTES / 16; idx += kThreads)
+        reinterpret_cast<uint4*>(sStage + s * C::STAGE_BYTES)[idx] = make_uint4(0, 0, 0, 0);
+  }
+  fence_proxy_async_smem();
+  if (warp == 0) {
+    tmem_alloc(&tmem_base_sh, kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = tmem_base_sh;
+
+  // Items of this CTA: k = 0, 1, ...; global item = blockIdx.x + k * gridDim.x
+  // ordered so that concurrently running CTAs work on neighbouring blocks.
+  const int groups = p.heads / C::PARTS;
+  const int my_items = (p.num_items > (int)blockIdx.x)
+                           ? (p.num_items - 1 - (int)blockIdx.x) / (int)gridDim.x + 1 : 0;
+
+  if (warp >= 8) {
+  // Producer warpgroup.  Each role ends in its own copy of the teardown
+  // barrier so that no code is shared between the two register budgets.
+  asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kProducerRegs));
+  if (warp == kTmaWarp) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      int issued = 0;
+      for (int k = 0; k < my_items; ++k) {
+        const int s = k % S;
+        if (k >= S && !mbar_wait(&bar_empty[s], ((k / S) - 1) & 1, kWaitNs, &abort_flag)) {
+          if (!abort_flag) record_timeout(&abort_flag);
+          break;
+        }
+        const int item = blockIdx.x + k * gridDim.x;
+        const int grp = item % groups;
+        const int blk = item / groups;
+        const int bx = blk % p.nbx, by = (blk / p.nbx) % p.nby, n = blk / (p.nbx * p.nby);
+        uint8_t* st = sStage + s * C::STAGE_BYTES;
+        mbar_arrive_expect_tx(&bar_full[s], C::TX_BYTES);
+        for (int part = 0; part < C::PARTS; ++part) {
+          const int head = grp * C::PARTS + part;
+          uint8_t* qdst = st + ((STRIDE == 1) ? 0 : (48 + 64 * part) * C::ROWB);
+          tma_load_4d(qdst, &tmap_q, &bar_full[s], head * D, bx * kBlock, by * kBlock, n);
+          uint8_t* kdst = st + C::Q_BYTES + part * C::KV_TILE;
+          uint8_t* vdst = st + C::Q_BYTES + (C::PARTS + part) * C::KV_TILE;
+          tma_load_4d(kdst, &tmap_k, &bar_full[s], head * D, bx * kBlock - p.halo, by * kBlock - p.halo, n);
+          tma_load_4d(vdst, &tmap_v, &bar_full[s], head * D, bx * kBlock - p.halo, by * kBlock - p.halo, n);
+        }
+        issued = k + 1;
+      }
+      if (abort_flag) {
+        // let loads that are still in flight land before the CTA exits
+        for (int k = (issued > S ? issued - S : 0); k < issued; ++k)
+          mbar_wait(&bar_full[k % S], (k / S) & 1, kWaitNs);
+      }
+    }
+  } else if (warp == kMmaWarp) {
+    // ------------------------------------------------------------ MMA issue
+    if (lane == 0) {
+      const uint32_t idS = idesc_bf16_f32(64, C::KEYS, false);
+      const uint32_t idG = idesc_bf16_f32(64, kGCols, false);
+      const uint32_t idO = idesc_bf16_f32(64, C::O_COLS, true);
+      auto issue_s = [&](int k) -> bool {
+        const int s = k % S, g = k & 1;
+        if (!mbar_wait(&bar_full[s], (k / S) & 1, kWaitNs, &abort_flag)) return false;
+        if (k >= 2 && !mbar_wait(&bar_tfree[g], ((k >> 1) - 1) & 1, kWaitNs, &abort_flag)) return false;
+        tc_fence_after();
+        const uint32_t half = static_cast<uint32_t>(g * 16) << 16;
+        const uint8_t* st = sStage + s * C::STAGE_BYTES;
+        for (int part = 0; part < C::PARTS; ++part) {
+          const uint32_t qa = smem_addr(st + ((STRIDE == 1) ? 0 : (48 + 48 * part) * C::ROWB));
+          const uint32_t ka = smem_addr(st + C::Q_BYTES + part * C::KV_TILE);
+          for (int ks = 0; ks < D / 16; ++ks) {
+            mma_f16_ss(tmem + half + kTmemS, smem_desc(qa + 32 * ks, 16, C::SBO, C::SW),
+                       smem_desc(ka + 32 * ks, 16, C::SBO, C::SW), idS, (part | ks) != 0);
+          }
+        }
+        const uint32_t ra = smem_addr(sR);
+        for (int part = 0; part < C::PARTS; ++part) {
+          const uint32_t qa = smem_addr(st + ((STRIDE == 1) ? 0 : (48 + 48 * part) * C::ROWB));
+          for (int ks = 0; ks < D / 16; ++ks) {
+            mma_f16_ss(tmem + half + kTmemG, smem_desc(qa + 32 * ks, 16, C::SBO, C::SW),
+                       smem_desc(ra + 32 * ks, 16, C::SBO, C::SW), idG, (part | ks) != 0);
+          }
+        }
+        mma_commit(&bar_sfull[g]);
+        return true;
+      };
+      auto issue_o = [&](int k) -> bool {
+        const int s = k % S, g = k & 1;
+        if (!mbar_wait(&bar_pfull[g], (k >> 1) & 1, kWaitNs, &abort_flag)) return false;
+        tc_fence_after();
+        const uint32_t half = static_cast<uint32_t>(g * 16) << 16;
+        const uint8_t* st = sStage + s * C::STAGE_BYTES;
+        const uint32_t pa = smem_addr(sP + g * C::P_TILE);
+        for (int part = 0; part < C::PARTS; ++part) {
+          const uint32_t va = smem_addr(st + C::Q_BYTES + (C::PARTS + part) * C::KV_TILE);
+          // with the ones tile the B operand spans two swizzle atoms along N:
+          // V (D columns) then ones (D columns) at leading byte offset LBO
+          const uint32_t lbo = C::SUM_BY_MMA ? (smem_addr(sOnes) - va) : 16u;
+          for (int kk = 0; kk < C::KEYS / 16; ++kk) {
+            mma_f16_ss(tmem + half + kTmemO + part * C::O_COLS, smem_desc(pa + kk * 2048, 16, 256, SW_32B),
+                       smem_desc(va + kk * 16 * C::ROWB, lbo, C::SBO, C::SW), idO, kk != 0);
+          }
+        }
+        mma_commit(&bar_ofull[g]);
+        mma_commit(&bar_empty[s]);
+        return true;
+      };
+      bool ok = true;
+      if (my_items > 0) ok = issue_s(0);
+      for (int k = 0; ok && k < my_items; ++k) {
+        if (k + 1 < my_items) ok = issue_s(k + 1);
+        if (ok) ok = issue_o(k);
+      }
+      if (!ok && !abort_flag) record_timeout(&abort_flag);
+      // all issued MMAs complete before the CTA frees TMEM
+      mma_commit(&bar_done);
+      mbar_wait(&bar_done, 0, kWaitNs);
+    }
+  }
+  __syncwarp();  // reconverge lane 0 with its warp before the aligned barrier
+  tc_fence_before();
+  named_bar_sync(1, kThreads);
+  return;
+  }
+
+  asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kSoftmaxRegs));
+  {
+    // ------------------------------------------------------------ softmax warpgroups
+    const int g = warp >> 2;          // warpgroup 0 or 1
+    const int wq = warp & 3;          // TMEM lane quadrant
+    const int half = lane >> 4;       // 0: even window rows, 1: odd window rows
+    const int r16 = lane & 15;        // row within the quadrant
+    const bool active = (STRIDE == 1) || (wq < C::PARTS);
+    const uint32_t tq = tmem + (static_cast<uint32_t>(32 * wq + 16 * g) << 16);
+    uint8_t* pt = sP + g * C::P_TILE;
+    // this thread's query row within the 64-row tile, and its in-block offset
+    const int row = 16 * wq + r16;
+    const int qy = (STRIDE == 1) ? (row >> 3) : 2 * (r16 >> 2);
+    const int qx = (STRIDE == 1) ? (row & 7) : 2 * (r16 & 3);
+    const float c = p.c;
+    const int C_all = p.heads * D;
+
+    int j = 0;
+    for (int k = g; k < my_items; k += 2, ++j) {
+      if (!mbar_wait(&bar_sfull[g], j & 1, kWaitNs, &abort_flag)) {
+        if (!abort_flag) record_timeout(&abort_flag);
+        break;
+      }
+      tc_fence_after();
+      const int item = blockIdx.x + k * gridDim.x;
+      const int grp = item % groups;
+      const int blk = item / groups;
+      const int bx = blk % p.nbx, by = (blk / p.nbx) % p.nby, n = blk / (p.nbx * p.nby);
+      const int head = grp * C::PARTS + ((STRIDE == 1) ? 0 : wq);
+      const int y0 = by * kBlock - p.halo, x0 = bx * kBlock - p.halo;
+
+      float l = 0.f;
+      if (active) {
+        // ---- relative logits: G row -> this warp's scratch (inside its P rows)
+        {
+          uint32_t gr[32];
+          tmem_ld_16x32bx2_x32<32>(tq + kTmemG, gr);
+          tmem_wait_ld();
+          // scratch float j of row r16 lives at chunk j/8, P row (16*wq + r16), byte 4*(j%8)
+#pragma unroll
+          for (int cc = 0; cc < 4; ++cc) {
+            uint8_t* dst = pt + (half * 4 + cc) * 2048 + row * 32;
+            reinterpret_cast<uint4*>(dst)[0] = make_uint4(gr[8 * cc + 0], gr[8 * cc + 1], gr[8 * cc + 2], gr[8 * cc + 3]);
+            reinterpret_cast<uint4*>(dst)[1] = make_uint4(gr[8 * cc + 4], gr[8 * cc + 5], gr[8 * cc + 6], gr[8 * cc + 7]);
+          }
+        }
+        __syncwarp();
+        auto scratch = [&](int jj) -> float {
+          return *reinterpret_cast<const float*>(pt + (jj >> 3) * 2048 + row * 32 + (jj & 7) * 4);
+        };
+        float rh[C::NROW];
+        float rw[WIN];
+#pragma unroll
+        for (int i = 0; i < C::NROW; ++i) {
+          const int kr = 2 * i + half;
+          const int Y = y0 + kr;
+          rh[i] = (Y >= 0 && Y < p.H) ? scratch(kr - qy + WIN - 1) : -INFINITY;
+        }
+#pragma unroll
+        for (int kc = 0; kc < WIN; ++kc) {
+          const int X = x0 + kc;
+          rw[kc] = (X >= 0 && X < p.W) ? scratch(32 + kc - qx + WIN - 1) : -INFINITY;
+        }
+        __syncwarp();
+
+        // ---- S rows of this thread: window rows 2i + half
+        float sv[C::NROW][16];
+#pragma unroll
+        for (int i = 0; i < C::NROW; ++i) {
+          tmem_ld_16x32bx2_x16<16>(tq + kTmemS + 32 * i, *reinterpret_cast<uint32_t(*)[16]>(&sv[i][0]));
+        }
+        tmem_wait_ld();
+        tc_fence_before();
+
+        // ---- exact row max of z = S + rel_h + rel_w over in-image keys
+        float m = -INFINITY;
+#pragma unroll
+        for (int i = 0; i < C::NROW; ++i) {
+          float mi = -INFINITY;
+#pragma unroll
+          for (int kc = 0; kc < WIN; ++kc) {
+            sv[i][kc] += rw[kc];
+            mi = fmaxf(mi, sv[i][kc]);
+          }
+          m = fmaxf(m, mi + rh[i]);
+        }
+        m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 16));
+        const float mc = m * c;
+
+        // ---- p = 2^(c*z - c*m); bf16 P into the swizzled operand tile
+#pragma unroll
+        for (int i = 0; i < C::NROW; ++i) {
+          const float bias = fmaf(rh[i], c, -mc);
+          float e[16];
+#pragma unroll
+          for (int kc = 0; kc < 16; ++kc) {
+            if (kc < WIN) {
+              const float x = fmaf(sv[i][kc], c, bias);
+              // about 40% of the exponentials run on the FMA pipe
+              e[kc] = (kc % 5 == 1 || kc % 5 == 3) ? exp2_poly(x) : exp2_mufu(x);
+            } else {
+              e[kc] = 0.f;
+            }
+          }
+          uint32_t pk[8];
+#pragma unroll
+          for (int t = 0; t < 8; ++t) pk[t] = pack_bf16x2(e[2 * t], e[2 * t + 1]);
+          if constexpr (!C::SUM_BY_MMA) {
+#pragma unroll
+            for (int kc = 0; kc < WIN; ++kc) l += e[kc];
+          }
+          const int kr = 2 * i + half;
+          uint8_t* dst = pt + kr * 2048 + row * 32;
+          const int sw = (row >> 2) & 1;
+          *reinterpret_cast<uint4*>(dst + (sw << 4)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+          *reinterpret_cast<uint4*>(dst + ((sw ^ 1) << 4)) = make_uint4(pk[4], pk[5], pk[6], pk[7]);
+        }
+        if constexpr (!C::SUM_BY_MMA) l += __shfl_xor_sync(0xffffffffu, l, 16);
+        fence_proxy_async_smem();
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bar_pfull[g]);
+
+      // ---- O = P V, normalise, store
+      if (!mbar_wait(&bar_ofull[g], j & 1, kWaitNs, &abort_flag)) {
+        if (!abort_flag) record_timeout(&abort_flag);
+        break;
+      }
+      tc_fence_after();
+      if (active) {
+        const uint32_t oaddr = tq + kTmemO + ((STRIDE == 1) ? 0 : wq * C::O_COLS);
+        float o[D / 2];
+        if constexpr (D == 16) {
+          uint32_t r[8];
+          tmem_ld_16x32bx2_x8<8>(oaddr, r);
+          uint32_t rs[8];
+          tmem_ld_16x32bx2_x8<8>(oaddr + D, rs);  // row sums (ones tile): every column holds the sum
+          tmem_wait_ld();
+#pragma unroll
+          for (int t = 0; t < 8; ++t) o[t] = __uint_as_float(r[t]);
+          l = __uint_as_float(rs[0]);
+        } else if constexpr (D == 32) {
+          uint32_t r[16];
+          tmem_ld_16x32bx2_x16<16>(oaddr, r);
+          tmem_wait_ld();
+#pragma unroll
+          for (int t = 0; t < 16; ++t) o[t] = __uint_as_float(r[t]);
+        } else {
+          uint32_t r[32];
+          tmem_ld_16x32bx2_x32<32>(oaddr, r);
+          tmem_wait_ld();
+#pragma unroll
+          for (int t = 0; t < 32; ++t) o[t] = __uint_as_float(r[t]);
+        }
+        const float inv = 1.0f / l;
+        uint32_t pk[D / 4];
+#pragma unroll
+        for (int t = 0; t < D / 4; ++t) pk[t] = pack_bf16x2(o[2 * t] * inv, o[2 * t + 1] * inv);
+        const int y = by * kBlock + qy, x = bx * kBlock + qx;
+        const int oy = y / STRIDE, ox = x / STRIDE;
+        __nv_bfloat16* dst = p.out + ((static_cast<size_t>(n) * p.OH + oy) * p.OW + ox) * C_all + head * D + half * (D / 2);
+#pragma unroll
+        for (int t = 0; t < D / 16; ++t)
+          reinterpret_cast<uint4*>(dst)[t] = make_uint4(pk[4 * t], pk[4 * t + 1], pk[4 * t + 2], pk[4 * t + 3]);
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bar_tfree[g]);
+    }
+  }
+
+  // ---------------------------------------------------------------- teardown
+  tc_fence_before();
+  named_bar_sync(1, kThreads);
+  tc_fence_after();
+  if (warp == 0) tmem_dealloc(tmem, kTmemCols);
+}
+
+}  // namespace tc
+}  // namespace halo

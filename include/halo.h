@@ -1,0 +1,135 @@
+/*
+ * halo.h -- C ABI of libhalo: HaloNet blocked local self-attention with
+ * haloing on NVIDIA B200 (sm_100a).
+ *
+ * The operation ("Scaling Local Self-Attention for Parameter Efficient Visual
+ * Backbones", sections 2.1-2.2, Figures 1-2, Appendix A; the blog page's
+ * HaloAttention / RelPosEmb modules for the concrete index conventions):
+ *
+ *   The H x W map is cut into non-overlapping block x block query blocks.
+ *   Block (by, bx) attends to the w x w window (w = block + 2*halo) whose top
+ *   left pixel is (by*block - halo, bx*block - halo); window keys outside the
+ *   image are removed from the softmax.  For query pixel (y, x) with in-block
+ *   offset (qy, qx) and window key (kr, kc) at image pixel (Y, X), per head:
+ *
+ *     z = s * q[y,x] . ( k[Y,X] + rel_h[kr - qy + w - 1] + rel_w[kc - qx + w - 1] )
+ *     out[y/stride, x/stride] = sum_keys softmax(z) * v[Y,X]          s = dim_head^-1/2
+ *
+ *   stride 2 takes the queries at even in-block offsets (0, 2, .., block-2)
+ *   and keeps the stride-1 window (section 2.2, Figure 2).
+ *
+ * Layouts (all row-major, contiguous, no padding):
+ *   q, k, v : [N, H, W, heads*dim_head]  (NHWC; channel = head*dim_head + e)
+ *   rel_h, rel_w : [2*w - 1, dim_head]   (shared by all heads)
+ *   out     : [N, H/stride, W/stride, heads*dim_head]
+ *
+ * Conventions shared by every entry point:
+ *   - Return value: HALO_OK (0) or a negative halo_status code; nothing is
+ *     launched when an argument check fails.
+ *   - Device-pointer calls are asynchronous on `stream` (a cudaStream_t; NULL
+ *     means the legacy default stream).  The library allocates no device
+ *     memory for them and keeps no pointer after the call returns.  The caller
+ *     owns every buffer and must keep it alive until the stream work is done.
+ *   - `out` must not overlap any input.
+ *   - Thread safety: calls from several host threads are safe.  TMA
+ *     descriptors are encoded on the host for every call (kernel parameters);
+ *     the only process-wide state is a mutex-guarded table of per-device
+ *     properties and the driver entry point used for the encoding.
+ */
+#ifndef HALO_H_
+#define HALO_H_
+
+#include <stddef.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  HALO_F32 = 0,  /* float32 inputs and output, float32 arithmetic */
+  HALO_BF16 = 1  /* bfloat16 inputs and output, float32 accumulation */
+} halo_dtype_t;
+
+typedef enum {
+  HALO_OK = 0,
+  HALO_ERR_NULL = -1,          /* a required pointer is NULL */
+  HALO_ERR_DIMS = -2,          /* a size is non-positive, or too large */
+  HALO_ERR_DIVISIBILITY = -3,  /* H or W not a multiple of block, or block not a multiple of stride */
+  HALO_ERR_STRIDE = -4,        /* stride not 1 or 2 */
+  HALO_ERR_ALIGN = -5,         /* a pointer is not 16-byte aligned, or a row of C channels is not a multiple of 16 bytes */
+  HALO_ERR_UNSUPPORTED = -6,   /* a shape no kernel of this library handles (see halo_kernel_for) */
+  HALO_ERR_CUDA = -7,          /* a CUDA runtime call or kernel launch failed */
+  HALO_ERR_TIMEOUT = -8,       /* a bounded device-side wait ran out (reported by halo_get_last_error) */
+  HALO_ERR_DTYPE = -9,         /* dtype is not a halo_dtype_t value */
+  HALO_ERR_ALIAS = -10,        /* out overlaps an input */
+  HALO_ERR_DEVICE = -11        /* the current device is not an sm_100 GPU */
+} halo_status;
+
+/* Which kernel halo_attn would launch for a shape (halo_kernel_for). */
+typedef enum {
+  HALO_KERNEL_NONE = 0,       /* the shape is rejected */
+  HALO_KERNEL_SIMT_F32 = 1,   /* CUDA-core kernel (float32 arithmetic); all float32 shapes, and bf16 shapes the tensor-core kernel does not cover */
+  HALO_KERNEL_TC_BF16 = 2     /* TMA + tcgen05/TMEM tensor-core kernel for bf16 */
+} halo_kernel_t;
+
+/*
+ * halo_attn -- the fused operation on device buffers.
+ *
+ * q, k, v, rel_h, rel_w, out: device pointers in the layouts above, all of
+ * dtype `dtype`, each 16-byte aligned.  N, H, W, heads, dim_head, block > 0,
+ * halo >= 0 (halo 0 is attention on isolated blocks, section 4.3),
+ * H % block == 0, W % block == 0, stride in {1, 2}, block % stride == 0.
+ * heads*dim_head*sizeof(dtype) must be a multiple of 16 bytes.
+ *
+ * Asynchronous: returns after the launch is queued on `stream`.  Errors found
+ * by the device (a bounded wait that ran out) are recorded in a device flag
+ * that halo_get_last_error() reads.
+ */
+int halo_attn(const void* q, const void* k, const void* v, const void* rel_h, const void* rel_w, void* out,
+              int N, int H, int W, int heads, int dim_head, int block, int halo, int stride, int dtype,
+              void* stream);
+
+/*
+ * halo_attn_host -- the same operation on HOST buffers (end-to-end form).
+ *
+ * q_h .. rel_w_h: host input pointers (pinned memory is fastest), out_h: host
+ * output pointer.  q_d .. out_d: caller-owned device buffers of the same sizes
+ * that the call uses as staging; the library allocates nothing.  The call
+ * queues host->device copies of the five inputs, the kernel and the
+ * device->host copy of the output on `stream` and returns without waiting;
+ * synchronise `stream` before reading out_h.
+ */
+int halo_attn_host(const void* q_h, const void* k_h, const void* v_h, const void* rel_h_h, const void* rel_w_h,
+                   void* out_h, void* q_d, void* k_d, void* v_d, void* rel_h_d, void* rel_w_d, void* out_d,
+                   int N, int H, int W, int heads, int dim_head, int block, int halo, int stride, int dtype,
+                   void* stream);
+
+/* Which kernel halo_attn would launch for these arguments (halo_kernel_t),
+ * or HALO_KERNEL_NONE when the shape is rejected.  No device work. */
+int halo_kernel_for(int N, int H, int W, int heads, int dim_head, int block, int halo, int stride, int dtype);
+
+/* Static description of a status code; never NULL. */
+const char* halo_strerror(int code);
+
+/* Reads and clears the device error flag of the current device (HALO_OK or
+ * HALO_ERR_TIMEOUT).  Synchronises the device. */
+int halo_get_last_error(void);
+
+/*
+ * halo_debug_wait_timeout -- failure-detection self test.  Launches one tiny
+ * kernel that waits on an mbarrier nobody arrives at, with a limit of
+ * `limit_us` microseconds (1 .. 1000000); when the limit runs out the kernel
+ * records HALO_ERR_TIMEOUT in the device flag and returns normally.  Returns
+ * the flag's value (it synchronises `stream`), so a working timeout path
+ * returns HALO_ERR_TIMEOUT.  Touches no caller memory.
+ */
+int halo_debug_wait_timeout(int limit_us, void* stream);
+
+/* Library version: major*10000 + minor*100 + patch. */
+int halo_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* HALO_H_ */

@@ -1,0 +1,114 @@
+"""The C ABI: libhalo.so loads without a GPU, exports every entry point that
+include/halo.h declares, and rejects invalid arguments before touching the
+device (no kernel is launched by these tests)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "halo.h")
+
+
+def _declared_functions():
+    src = open(HEADER).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"^\s*(?:const\s+)?\w+\*?\s+\*?(halo_\w+)\s*\(", src, flags=re.M)))
+
+
+def _lib():
+    from blocked_local_self_b200 import _native
+    return _native.lib()
+
+
+def test_header_declares_the_boundary():
+    names = _declared_functions()
+    for expected in ("halo_attn", "halo_attn_host", "halo_kernel_for", "halo_strerror", "halo_get_last_error",
+                     "halo_debug_wait_timeout", "halo_version"):
+        assert expected in names
+
+
+def test_library_exports_every_declared_symbol():
+    lib = _lib()
+    for name in _declared_functions():
+        assert hasattr(lib, name), f"libhalo.so does not export {name}"
+
+
+def test_binding_mirrors_header():
+    from blocked_local_self_b200 import _native
+    assert sorted(_native.SIGNATURES) == _declared_functions()
+
+
+def test_status_codes_match_header():
+    from blocked_local_self_b200 import _native
+    src = open(HEADER).read()
+    for name, val in re.findall(r"(HALO_(?:OK|ERR_\w+))\s*=\s*(-?\d+)", src):
+        assert getattr(_native, name) == int(val), name
+
+
+def test_strerror_covers_codes():
+    lib = _lib()
+    for code in range(0, -12, -1):
+        text = lib.halo_strerror(code).decode()
+        assert text and text != "unknown status code"
+    assert lib.halo_strerror(-99).decode() == "unknown status code"
+
+
+def test_version():
+    assert _lib().halo_version() >= 100
+
+
+ARGS = dict(N=1, H=16, W=16, heads=2, d=16, block=8, halo=3, stride=1, dtype=1)
+
+
+def _call(ptrs=(16,) * 6, **over):
+    a = dict(ARGS, **over)
+    return _lib().halo_attn(*ptrs, a["N"], a["H"], a["W"], a["heads"], a["d"], a["block"], a["halo"],
+                            a["stride"], a["dtype"], None)
+
+
+@pytest.mark.parametrize("over,code", [
+    (dict(dtype=7), -9),
+    (dict(N=0), -2), (dict(H=-8), -2), (dict(heads=0), -2), (dict(d=0), -2), (dict(block=0), -2),
+    (dict(halo=-1), -2),
+    (dict(stride=3), -4),
+    (dict(H=12), -3), (dict(W=20), -3), (dict(block=3, stride=2, H=9, W=9), -3),
+    (dict(heads=1, d=4), -5),
+])
+def test_shape_checks(over, code):
+    assert _call(**over) == code
+
+
+def test_pointer_checks():
+    assert _call(ptrs=(16, 16, 0, 16, 16, 16)) == -1
+    assert _call(ptrs=(16, 16, 24, 16, 16, 4096)) == -5
+    # out overlapping q: q at 1<<20, out 256 bytes later
+    assert _call(ptrs=(1 << 20, 1 << 22, 1 << 23, 1 << 24, 1 << 25, (1 << 20) + 256)) == -10
+
+
+def test_kernel_selection_is_host_only():
+    lib = _lib()
+    # the stage-1 HaloNet layer goes to the tensor-core kernel
+    assert lib.halo_kernel_for(32, 64, 64, 8, 16, 8, 3, 1, 1) == 2
+    assert lib.halo_kernel_for(64, 32, 32, 8, 64, 8, 3, 1, 1) == 2
+    assert lib.halo_kernel_for(64, 64, 64, 8, 32, 8, 3, 2, 1) == 2
+    # float32 goes to the CUDA-core kernel, invalid shapes to none
+    assert lib.halo_kernel_for(1, 16, 16, 2, 32, 4, 1, 1, 0) == 1
+    assert lib.halo_kernel_for(1, 16, 16, 2, 32, 5, 1, 1, 0) == 0
+
+
+def test_host_entry_checks_before_any_copy():
+    lib = _lib()
+    a = ARGS
+    rc = lib.halo_attn_host(*([16] * 5 + [None]), *([16] * 6), a["N"], a["H"], a["W"], a["heads"], a["d"],
+                            a["block"], a["halo"], a["stride"], a["dtype"], None)
+    assert rc == -1
+
+
+def test_missing_library_fails_loudly(tmp_path, monkeypatch):
+    from blocked_local_self_b200 import _native
+    monkeypatch.setattr(_native, "LIB_PATH", str(tmp_path / "libhalo.so"))
+    monkeypatch.setattr(_native, "_lib", None)
+    with pytest.raises(ImportError):
+        _native.lib()
