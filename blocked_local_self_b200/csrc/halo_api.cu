@@ -83,8 +83,7 @@ int tc_smem(int stages) { return halo::tc::smem_bytes<D, WIN, STRIDE>(stages); }
         halo::tc::Cfg<D, WIN, S>::STAGE_BYTES, halo::tc::Cfg<D, WIN, S>::PARTS                   \
   }
 #define HALO_TC_WINS(D, S) \
-  HALO_TC_ENTRY(D, 8, S), HALO_TC_ENTRY(D, 10, S), HALO_TC_ENTRY(D, 12, S), HALO_TC_ENTRY(D, 14, S), \
-      HALO_TC_ENTRY(D, 16, S)
+  HALO_TC_ENTRY(D, 8, S), HALO_TC_ENTRY(D, 10, S), HALO_TC_ENTRY(D, 12, S), HALO_TC_ENTRY(D, 14, S)
 
 const TcEntry kTcTable[] = {
     HALO_TC_WINS(16, 1), HALO_TC_WINS(32, 1), HALO_TC_WINS(64, 1),
@@ -210,7 +209,7 @@ int launch_tc(const TcEntry& e, const void* q, const void* k, const void* v, con
   const int win = s.block + 2 * s.halo;
   CUtensorMap mq, mk, mv;
   if (!encode_nhwc(&mq, q, s, halo::tc::kBlock, halo::tc::kBlock, s.stride) ||
-      !encode_nhwc(&mk, k, s, halo::tc::kRowKeys, win, 1) || !encode_nhwc(&mv, v, s, halo::tc::kRowKeys, win, 1))
+      !encode_nhwc(&mk, k, s, win, win, 1) || !encode_nhwc(&mv, v, s, halo::tc::kRowKeys, win, 1))
     return HALO_ERR_CUDA;
   // The kernel moves registers between its warpgroups with setmaxnreg; that is
   // only safe if the launch allocation covers the split (otherwise the

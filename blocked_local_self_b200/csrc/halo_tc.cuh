@@ -47,23 +47,27 @@ namespace tc {
 using namespace sm100;
 
 constexpr int kBlock = 8;         // query block side handled by this kernel
-constexpr int kRowKeys = 16;      // window row pitch in keys (w padded to 16)
+constexpr int kRowKeys = 16;      // P / V window row pitch in keys (w padded to 16)
 constexpr int kThreads = 384;     // 2 softmax warpgroups + 1 producer warpgroup
 constexpr int kTmaWarp = 8;       // producer warpgroup: warp 8 TMA, warp 9 MMA,
 constexpr int kMmaWarp = 9;       // warps 10-11 idle
 // Register split (setmaxnreg): the kernel launches with kLaunchRegs per thread
 // (3 warps per SM sub-partition cap it at 168); the producer warpgroup gives
 // registers back and the softmax warpgroups take more.  The sum stays within
-// the launch allocation: 256*216 + 128*56 = 62464 <= 384*168 = 64512.
+// the launch allocation: 256*208 + 128*72 = 62464 <= 384*168 = 64512.
 constexpr int kLaunchRegs = 168;
-constexpr int kSoftmaxRegs = 216;
-constexpr int kProducerRegs = 56;
+constexpr int kSoftmaxRegs = 208;
+constexpr int kProducerRegs = 72;
 static_assert(256 * kSoftmaxRegs + 128 * kProducerRegs <= kThreads * kLaunchRegs, "register split");
+// TMEM: 512 columns x 128 lanes.  Warpgroup g owns lanes 16g..16g+15 of every
+// 32-lane quadrant (the two M=64 accumulator halves) and, inside that, two
+// item slots of 256 columns: S at [0, 200), G at [200, 256); O (and the row
+// sums) overwrite the first S columns once P has been taken from S.
 constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kTmemS = 0;    // S: columns [0, 16w)
-constexpr uint32_t kTmemG = 256;  // G: columns [256, 320)
-constexpr uint32_t kTmemO = 320;  // O (+ row sums): columns [320, 448)
-constexpr int kGCols = 64;        // rel_h logits at [0, 2w-1), rel_w logits at [32, 32+2w-1)
+constexpr uint32_t kSlotCols = 256;
+constexpr uint32_t kTmemG = 200;
+constexpr int kGCols = 56;        // rel_h logits at [0, 2w-1), rel_w logits at [28, 28+2w-1)
+constexpr int kGRelW = 28;
 constexpr uint64_t kWaitNs = 1000000000ull;  // 1 s bound on every wait
 
 struct Params {
@@ -87,29 +91,38 @@ struct Cfg {
   // stride 1: 64-row Q tile.  stride 2: zero-gap buffer so that the 64-row view
   // of head p holds its 16 queries in rows 16p..16p+15 and zeros elsewhere.
   static constexpr int QBUF_ROWS = (STRIDE == 1) ? 64 : (112 + 48 * (PARTS - 1));
-  static constexpr int KEYS = WIN * kRowKeys;             // S columns / PV K extent
-  static constexpr int KV_TILE = KEYS * ROWB;             // bytes of one head's K (or V) window
+  static constexpr int KS = WIN * WIN;                    // keys of the window (K tile rows written)
+  static constexpr int NS = (KS + 7) / 8 * 8;             // S columns (QK^T N); rows KS..NS-1 zero
+  static constexpr int KP = WIN * kRowKeys;               // PV K extent (V tile rows, P columns)
+  static constexpr int K_TILE = NS * ROWB;
+  static constexpr int V_TILE = KP * ROWB;
   static constexpr int Q_BYTES = QBUF_ROWS * ROWB;
-  static constexpr int STAGE_BYTES = Q_BYTES + 2 * PARTS * KV_TILE;
-  static constexpr int TX_BYTES = PARTS * (QROWS_PER_HEAD * ROWB + 2 * KV_TILE);
+  static constexpr int STAGE_RAW = Q_BYTES + PARTS * (K_TILE + V_TILE);
+  static constexpr int STAGE_BYTES = (STAGE_RAW + 1023) / 1024 * 1024;
+  static constexpr int TX_BYTES = PARTS * (QROWS_PER_HEAD * ROWB + (KS + KP) * ROWB);
   static constexpr int P_TILE = WIN * 2048;               // 64 rows x 16 keys x 2 B per window row
-  static constexpr int R_TILE = kGCols * ROWB;            // [rel_h; rel_w] B operand
+  static constexpr int R_TILE = kGCols * ROWB;            // [rel_h; 0; rel_w; 0] B operand
+  static constexpr int SCRATCH_LINE = 36;                 // floats per (row, half) line of the gather scratch
+  static constexpr int SCRATCH = 8 * 32 * SCRATCH_LINE * 4;
   static constexpr bool SUM_BY_MMA = (D == 16);           // row sums through a ones tile in PV
-  static constexpr int ONES_TILE = SUM_BY_MMA ? KEYS * ROWB : 0;
+  static constexpr int ONES_TILE = SUM_BY_MMA ? KP * ROWB : 0;
   static constexpr int O_COLS = SUM_BY_MMA ? 2 * D : D;   // PV N
   static constexpr SmemSwizzle SW = (ROWB == 32) ? SW_32B : (ROWB == 64 ? SW_64B : SW_128B);
   static constexpr uint32_t SBO = 8 * ROWB;               // 8-row core-matrix group stride
   static constexpr int NROW = WIN / 2;                    // window rows per thread
-  static_assert(WIN % 2 == 0 && WIN <= 16 && WIN >= 8, "window must be even, 8..16");
+  static_assert(WIN % 2 == 0 && WIN <= 14 && WIN >= 8, "window must be even, 8..14");
   static_assert(D == 16 || D == 32 || D == 64, "dim_head must be 16, 32 or 64");
-  static_assert(PARTS * O_COLS <= 128, "O region");
+  static_assert(NS <= (int)kTmemG, "S must fit below G in a TMEM slot");
+  static_assert(2 * WIN - 1 <= kGRelW, "relative table rows");
+  static_assert(PARTS * O_COLS <= (int)kTmemG, "O region below the G columns");
 };
 
 // Bytes of dynamic shared memory for a given stage count (plus 1 KB alignment slack).
 template <int D, int WIN, int STRIDE>
 __host__ __device__ constexpr int smem_bytes(int stages) {
   using C = Cfg<D, WIN, STRIDE>;
-  return 1024 + 2 * C::P_TILE + C::R_TILE + C::ONES_TILE + stages * C::STAGE_BYTES;
+  return 1024 + 2 * C::P_TILE + C::SCRATCH + ((C::R_TILE + 1023) / 1024) * 1024 + stages * C::STAGE_BYTES +
+         C::ONES_TILE;
 }
 
 // Swizzled byte offset of 16-byte unit u of row r in a K-major tile whose
@@ -155,6 +168,20 @@ __device__ __forceinline__ void record_timeout(int* abort_flag) {
   *(volatile int*)abort_flag = 1;
 }
 
+struct ItemCoord {
+  int n, by, bx, grp;
+};
+
+__device__ __forceinline__ ItemCoord item_coord(int item, int groups, int nbx, int nby) {
+  ItemCoord c;
+  c.grp = item % groups;
+  const int blk = item / groups;
+  c.bx = blk % nbx;
+  c.by = (blk / nbx) % nby;
+  c.n = blk / (nbx * nby);
+  return c;
+}
+
 template <int D, int WIN, int STRIDE>
 __global__ void __launch_bounds__(kThreads, 1)
     halo_fwd_tc(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__ CUtensorMap tmap_k,
@@ -162,19 +189,20 @@ __global__ void __launch_bounds__(kThreads, 1)
   using C = Cfg<D, WIN, STRIDE>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint8_t* sP = smem;                               // 2 x P_TILE (one per warpgroup)
-  uint8_t* sR = sP + 2 * C::P_TILE;                 // R tile
-  uint8_t* sStage = sR + C::R_TILE;                 // stages x STAGE_BYTES
+  uint8_t* sP = smem;                                          // 2 x P_TILE (one per warpgroup)
+  float* sScratch = reinterpret_cast<float*>(sP + 2 * C::P_TILE);  // relative-logit gather scratch
+  uint8_t* sR = sP + 2 * C::P_TILE + C::SCRATCH;               // R tile (1 KB aligned)
+  uint8_t* sStage = sR + ((C::R_TILE + 1023) / 1024) * 1024;   // stages x STAGE_BYTES
   // ones tile (d = 16) after the stages: the PV B descriptor reaches it with a
   // positive leading byte offset from any V tile
   uint8_t* sOnes = sStage + p.stages * C::STAGE_BYTES;
 
   __shared__ __align__(8) uint64_t bar_full[8];
   __shared__ __align__(8) uint64_t bar_empty[8];
-  __shared__ __align__(8) uint64_t bar_sfull[2];
-  __shared__ __align__(8) uint64_t bar_pfull[2];
-  __shared__ __align__(8) uint64_t bar_ofull[2];
-  __shared__ __align__(8) uint64_t bar_tfree[2];
+  __shared__ __align__(8) uint64_t bar_sfull[4];   // index 2*g + slot
+  __shared__ __align__(8) uint64_t bar_pfull[4];
+  __shared__ __align__(8) uint64_t bar_ofull[4];
+  __shared__ __align__(8) uint64_t bar_tfree[4];
   __shared__ __align__(8) uint64_t bar_done;
   __shared__ uint32_t tmem_base_sh;
   __shared__ int abort_flag;
@@ -190,11 +218,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&bar_full[i], 1);
       mbar_init(&bar_empty[i], 1);
     }
-    for (int g = 0; g < 2; ++g) {
-      mbar_init(&bar_sfull[g], 1);
-      mbar_init(&bar_pfull[g], 4);
-      mbar_init(&bar_ofull[g], 1);
-      mbar_init(&bar_tfree[g], 4);
+    for (int b = 0; b < 4; ++b) {
+      mbar_init(&bar_sfull[b], 1);
+      mbar_init(&bar_pfull[b], 4);
+      mbar_init(&bar_ofull[b], 1);
+      mbar_init(&bar_tfree[b], 4);
     }
     mbar_init(&bar_done, 1);
     abort_flag = 0;
@@ -205,12 +233,13 @@ __global__ void __launch_bounds__(kThreads, 1)
     prefetch_tensormap(&tmap_k);
     prefetch_tensormap(&tmap_v);
   }
-  // R tile: rows [0, 2w-1) = rel_h, rows [32, 32+2w-1) = rel_w, other rows 0.
+  // R tile: rows [0, 2w-1) = rel_h, rows [28, 28+2w-1) = rel_w, other rows 0.
   for (int idx = tid; idx < kGCols * (D / 8); idx += kThreads) {
     const int r = idx / (D / 8), u = idx % (D / 8);
     uint4 val = make_uint4(0, 0, 0, 0);
     if (r < 2 * WIN - 1) val = *reinterpret_cast<const uint4*>(p.rel_h + r * D + u * 8);
-    else if (r >= 32 && r < 32 + 2 * WIN - 1) val = *reinterpret_cast<const uint4*>(p.rel_w + (r - 32) * D + u * 8);
+    else if (r >= kGRelW && r < kGRelW + 2 * WIN - 1)
+      val = *reinterpret_cast<const uint4*>(p.rel_w + (r - kGRelW) * D + u * 8);
     *reinterpret_cast<uint4*>(sR + swz<C::ROWB>(r, u)) = val;
   }
   if constexpr (C::SUM_BY_MMA) {
@@ -218,11 +247,21 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int idx = tid; idx < C::ONES_TILE / 16; idx += kThreads)
       reinterpret_cast<uint4*>(sOnes)[idx] = make_uint4(0x3f803f80u, 0x3f803f80u, 0x3f803f80u, 0x3f803f80u);
   }
-  if constexpr (STRIDE == 2) {
-    // zero the query buffers: the TMA only ever writes the 16-row head slots
-    for (int s = 0; s < S; ++s)
+  // Zero what the TMA never writes: the K tile rows KS..NS-1 (read by the
+  // N = NS MMA) and, at stride 2, the query buffer outside the head slots.
+  for (int s = 0; s < S; ++s) {
+    uint8_t* st = sStage + s * C::STAGE_BYTES;
+    if constexpr (STRIDE == 2) {
       for (int idx = tid; idx < C::Q_BYTES / 16; idx += kThreads)
-        reinterpret_cast<uint4*>(sStage + s * C::STAGE_BYTES)[idx] = make_uint4(0, 0, 0, 0);
+        reinterpret_cast<uint4*>(st)[idx] = make_uint4(0, 0, 0, 0);
+    }
+    if constexpr (C::NS > C::KS) {
+      constexpr int tail = (C::NS - C::KS) * C::ROWB / 16;
+      for (int idx = tid; idx < C::PARTS * tail; idx += kThreads) {
+        uint8_t* kt = st + C::Q_BYTES + (idx / tail) * C::K_TILE + C::KS * C::ROWB;
+        reinterpret_cast<uint4*>(kt)[idx % tail] = make_uint4(0, 0, 0, 0);
+      }
+    }
   }
   fence_proxy_async_smem();
   if (warp == 0) {
@@ -236,6 +275,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   // Items of this CTA: k = 0, 1, ...; global item = blockIdx.x + k * gridDim.x
   // ordered so that concurrently running CTAs work on neighbouring blocks.
+  // Item k belongs to warpgroup k & 1 as its (k >> 1)-th item, which uses
+  // TMEM slot (k >> 1) & 1 of that warpgroup.
   const int groups = p.heads / C::PARTS;
   const int my_items = (p.num_items > (int)blockIdx.x)
                            ? (p.num_items - 1 - (int)blockIdx.x) / (int)gridDim.x + 1 : 0;
@@ -245,7 +286,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   // barrier so that no code is shared between the two register budgets.
   asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kProducerRegs));
   if (warp == kTmaWarp) {
-    // ------------------------------------------------------------ producer
+    // ------------------------------------------------------------ TMA producer
     if (lane == 0) {
       int issued = 0;
       for (int k = 0; k < my_items; ++k) {
@@ -254,20 +295,20 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (!abort_flag) record_timeout(&abort_flag);
           break;
         }
-        const int item = blockIdx.x + k * gridDim.x;
-        const int grp = item % groups;
-        const int blk = item / groups;
-        const int bx = blk % p.nbx, by = (blk / p.nbx) % p.nby, n = blk / (p.nbx * p.nby);
+        const ItemCoord ic = item_coord(blockIdx.x + k * gridDim.x, groups, p.nbx, p.nby);
         uint8_t* st = sStage + s * C::STAGE_BYTES;
         mbar_arrive_expect_tx(&bar_full[s], C::TX_BYTES);
+#pragma unroll 1
         for (int part = 0; part < C::PARTS; ++part) {
-          const int head = grp * C::PARTS + part;
+          const int head = ic.grp * C::PARTS + part;
           uint8_t* qdst = st + ((STRIDE == 1) ? 0 : (48 + 64 * part) * C::ROWB);
-          tma_load_4d(qdst, &tmap_q, &bar_full[s], head * D, bx * kBlock, by * kBlock, n);
-          uint8_t* kdst = st + C::Q_BYTES + part * C::KV_TILE;
-          uint8_t* vdst = st + C::Q_BYTES + (C::PARTS + part) * C::KV_TILE;
-          tma_load_4d(kdst, &tmap_k, &bar_full[s], head * D, bx * kBlock - p.halo, by * kBlock - p.halo, n);
-          tma_load_4d(vdst, &tmap_v, &bar_full[s], head * D, bx * kBlock - p.halo, by * kBlock - p.halo, n);
+          tma_load_4d(qdst, &tmap_q, &bar_full[s], head * D, ic.bx * kBlock, ic.by * kBlock, ic.n);
+          uint8_t* kdst = st + C::Q_BYTES + part * C::K_TILE;
+          uint8_t* vdst = st + C::Q_BYTES + C::PARTS * C::K_TILE + part * C::V_TILE;
+          tma_load_4d(kdst, &tmap_k, &bar_full[s], head * D, ic.bx * kBlock - p.halo, ic.by * kBlock - p.halo,
+                      ic.n);
+          tma_load_4d(vdst, &tmap_v, &bar_full[s], head * D, ic.bx * kBlock - p.halo, ic.by * kBlock - p.halo,
+                      ic.n);
         }
         issued = k + 1;
       }
@@ -280,63 +321,86 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else if (warp == kMmaWarp) {
     // ------------------------------------------------------------ MMA issue
     if (lane == 0) {
-      const uint32_t idS = idesc_bf16_f32(64, C::KEYS, false);
+      const uint32_t idS = idesc_bf16_f32(64, C::NS, false);
       const uint32_t idG = idesc_bf16_f32(64, kGCols, false);
       const uint32_t idO = idesc_bf16_f32(64, C::O_COLS, true);
-      auto issue_s = [&](int k) -> bool {
-        const int s = k % S, g = k & 1;
-        if (!mbar_wait(&bar_full[s], (k / S) & 1, kWaitNs, &abort_flag)) return false;
-        if (k >= 2 && !mbar_wait(&bar_tfree[g], ((k >> 1) - 1) & 1, kWaitNs, &abort_flag)) return false;
-        tc_fence_after();
-        const uint32_t half = static_cast<uint32_t>(g * 16) << 16;
+      // S(k): QK^T and the relative dot products of item k into its TMEM slot.
+      auto issue_s = [&](int k) {
+        const int s = k % S, g = k & 1, sl = (k >> 1) & 1;
+        const uint32_t dst = tmem + (static_cast<uint32_t>(g * 16) << 16) + sl * kSlotCols;
         const uint8_t* st = sStage + s * C::STAGE_BYTES;
+#pragma unroll 1
         for (int part = 0; part < C::PARTS; ++part) {
           const uint32_t qa = smem_addr(st + ((STRIDE == 1) ? 0 : (48 + 48 * part) * C::ROWB));
-          const uint32_t ka = smem_addr(st + C::Q_BYTES + part * C::KV_TILE);
+          const uint32_t ka = smem_addr(st + C::Q_BYTES + part * C::K_TILE);
           for (int ks = 0; ks < D / 16; ++ks) {
-            mma_f16_ss(tmem + half + kTmemS, smem_desc(qa + 32 * ks, 16, C::SBO, C::SW),
-                       smem_desc(ka + 32 * ks, 16, C::SBO, C::SW), idS, (part | ks) != 0);
+            mma_f16_ss(dst, smem_desc(qa + 32 * ks, 16, C::SBO, C::SW), smem_desc(ka + 32 * ks, 16, C::SBO, C::SW),
+                       idS, (part | ks) != 0);
           }
         }
         const uint32_t ra = smem_addr(sR);
+#pragma unroll 1
         for (int part = 0; part < C::PARTS; ++part) {
           const uint32_t qa = smem_addr(st + ((STRIDE == 1) ? 0 : (48 + 48 * part) * C::ROWB));
           for (int ks = 0; ks < D / 16; ++ks) {
-            mma_f16_ss(tmem + half + kTmemG, smem_desc(qa + 32 * ks, 16, C::SBO, C::SW),
+            mma_f16_ss(dst + kTmemG, smem_desc(qa + 32 * ks, 16, C::SBO, C::SW),
                        smem_desc(ra + 32 * ks, 16, C::SBO, C::SW), idG, (part | ks) != 0);
           }
         }
-        mma_commit(&bar_sfull[g]);
-        return true;
+        mma_commit(&bar_sfull[2 * g + sl]);
       };
-      auto issue_o = [&](int k) -> bool {
-        const int s = k % S, g = k & 1;
-        if (!mbar_wait(&bar_pfull[g], (k >> 1) & 1, kWaitNs, &abort_flag)) return false;
-        tc_fence_after();
-        const uint32_t half = static_cast<uint32_t>(g * 16) << 16;
+      // O(k): P V of item k once its warpgroup has written P; frees stage k.
+      auto issue_o = [&](int k) {
+        const int s = k % S, g = k & 1, sl = (k >> 1) & 1;
+        const uint32_t dst = tmem + (static_cast<uint32_t>(g * 16) << 16) + sl * kSlotCols;
         const uint8_t* st = sStage + s * C::STAGE_BYTES;
         const uint32_t pa = smem_addr(sP + g * C::P_TILE);
+#pragma unroll 1
         for (int part = 0; part < C::PARTS; ++part) {
-          const uint32_t va = smem_addr(st + C::Q_BYTES + (C::PARTS + part) * C::KV_TILE);
+          const uint32_t va = smem_addr(st + C::Q_BYTES + C::PARTS * C::K_TILE + part * C::V_TILE);
           // with the ones tile the B operand spans two swizzle atoms along N:
           // V (D columns) then ones (D columns) at leading byte offset LBO
           const uint32_t lbo = C::SUM_BY_MMA ? (smem_addr(sOnes) - va) : 16u;
-          for (int kk = 0; kk < C::KEYS / 16; ++kk) {
-            mma_f16_ss(tmem + half + kTmemO + part * C::O_COLS, smem_desc(pa + kk * 2048, 16, 256, SW_32B),
-                       smem_desc(va + kk * 16 * C::ROWB, lbo, C::SBO, C::SW), idO, kk != 0);
+#pragma unroll 1
+          for (int kk = 0; kk < WIN; ++kk) {
+            mma_f16_ss(dst + part * C::O_COLS, smem_desc(pa + kk * 2048, 16, 256, SW_32B),
+                       smem_desc(va + kk * kRowKeys * C::ROWB, lbo, C::SBO, C::SW), idO, kk != 0);
           }
         }
-        mma_commit(&bar_ofull[g]);
+        mma_commit(&bar_ofull[2 * g + sl]);
         mma_commit(&bar_empty[s]);
-        return true;
       };
-      bool ok = true;
-      if (my_items > 0) ok = issue_s(0);
-      for (int k = 0; ok && k < my_items; ++k) {
-        if (k + 1 < my_items) ok = issue_s(k + 1);
-        if (ok) ok = issue_o(k);
+      // Issue whichever step is ready (O first: it releases a waiting
+      // warpgroup).  S(k) needs its stage loaded and the slot's previous
+      // item (k - 4) consumed; O(k) needs P(k).
+      int ns = 0, no = 0;
+      uint64_t idle_since = global_timer_ns();
+      uint32_t polls = 0;
+      while (no < my_items) {
+        bool did = false;
+        if (no < ns && mbar_test(&bar_pfull[2 * (no & 1) + ((no >> 1) & 1)], (no >> 2) & 1)) {
+          tc_fence_after();
+          issue_o(no);
+          ++no;
+          did = true;
+        } else if (ns < my_items && mbar_test(&bar_full[ns % S], (ns / S) & 1) &&
+                   (ns < 4 || mbar_test(&bar_tfree[2 * (ns & 1) + ((ns >> 1) & 1)], ((ns >> 2) - 1) & 1))) {
+          tc_fence_after();
+          issue_s(ns);
+          ++ns;
+          did = true;
+        }
+        if (did) {
+          polls = 0;
+          idle_since = global_timer_ns();
+        } else if ((++polls & 15u) == 0) {
+          if (*(volatile int*)&abort_flag) break;
+          if (global_timer_ns() - idle_since > kWaitNs) {
+            record_timeout(&abort_flag);
+            break;
+          }
+        }
       }
-      if (!ok && !abort_flag) record_timeout(&abort_flag);
       // all issued MMAs complete before the CTA frees TMEM
       mma_commit(&bar_done);
       mbar_wait(&bar_done, 0, kWaitNs);
@@ -358,6 +422,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const bool active = (STRIDE == 1) || (wq < C::PARTS);
     const uint32_t tq = tmem + (static_cast<uint32_t>(32 * wq + 16 * g) << 16);
     uint8_t* pt = sP + g * C::P_TILE;
+    float* scr = sScratch + (warp * 32) * C::SCRATCH_LINE;  // this warp's 32 lines
     // this thread's query row within the 64-row tile, and its in-block offset
     const int row = 16 * wq + r16;
     const int qy = (STRIDE == 1) ? (row >> 3) : 2 * (r16 >> 2);
@@ -365,65 +430,114 @@ __global__ void __launch_bounds__(kThreads, 1)
     const float c = p.c;
     const int C_all = p.heads * D;
 
-    int j = 0;
-    for (int k = g; k < my_items; k += 2, ++j) {
-      if (!mbar_wait(&bar_sfull[g], j & 1, kWaitNs, &abort_flag)) {
+    // Epilogue of a finished item: O (and row sums) from its TMEM slot,
+    // normalise, bf16, store; then hand the slot back to the MMA warp.
+    auto epilogue = [&](int jj, const ItemCoord& ic, float l) -> bool {
+      const int b = 2 * g + (jj & 1);
+      if (!mbar_wait(&bar_ofull[b], (jj >> 1) & 1, kWaitNs, &abort_flag)) {
         if (!abort_flag) record_timeout(&abort_flag);
+        return false;
+      }
+      tc_fence_after();
+      if (active) {
+        const int head = ic.grp * C::PARTS + ((STRIDE == 1) ? 0 : wq);
+        const uint32_t oaddr = tq + (jj & 1) * kSlotCols + ((STRIDE == 1) ? 0 : wq * C::O_COLS);
+        float o[D / 2];
+        if constexpr (D == 16) {
+          uint32_t r[8];
+          tmem_ld_16x32bx2_x8<8>(oaddr, r);
+          uint32_t rs[8];
+          tmem_ld_16x32bx2_x8<8>(oaddr + D, rs);  // row sums (ones tile): every column holds the sum
+          tmem_wait_ld();
+#pragma unroll
+          for (int t = 0; t < 8; ++t) o[t] = __uint_as_float(r[t]);
+          l = __uint_as_float(rs[0]);
+        } else if constexpr (D == 32) {
+          uint32_t r[16];
+          tmem_ld_16x32bx2_x16<16>(oaddr, r);
+          tmem_wait_ld();
+#pragma unroll
+          for (int t = 0; t < 16; ++t) o[t] = __uint_as_float(r[t]);
+        } else {
+          uint32_t r[32];
+          tmem_ld_16x32bx2_x32<32>(oaddr, r);
+          tmem_wait_ld();
+#pragma unroll
+          for (int t = 0; t < 32; ++t) o[t] = __uint_as_float(r[t]);
+        }
+        const float inv = 1.0f / l;
+        uint32_t pk[D / 4];
+#pragma unroll
+        for (int t = 0; t < D / 4; ++t) pk[t] = pack_bf16x2(o[2 * t] * inv, o[2 * t + 1] * inv);
+        const int y = ic.by * kBlock + qy, x = ic.bx * kBlock + qx;
+        const int oy = y / STRIDE, ox = x / STRIDE;
+        __nv_bfloat16* dst =
+            p.out + ((static_cast<size_t>(ic.n) * p.OH + oy) * p.OW + ox) * C_all + head * D + half * (D / 2);
+#pragma unroll
+        for (int t = 0; t < D / 16; ++t)
+          reinterpret_cast<uint4*>(dst)[t] = make_uint4(pk[4 * t], pk[4 * t + 1], pk[4 * t + 2], pk[4 * t + 3]);
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bar_tfree[b]);
+      return true;
+    };
+
+    ItemCoord prev_ic{0, 0, 0, 0};
+    float prev_l = 0.f;
+    int j = 0;
+    bool ok = true;
+    for (int k = g; k < my_items; k += 2, ++j) {
+      const int sl = j & 1;
+      const int b = 2 * g + sl;
+      if (!mbar_wait(&bar_sfull[b], (j >> 1) & 1, kWaitNs, &abort_flag)) {
+        if (!abort_flag) record_timeout(&abort_flag);
+        ok = false;
         break;
       }
       tc_fence_after();
-      const int item = blockIdx.x + k * gridDim.x;
-      const int grp = item % groups;
-      const int blk = item / groups;
-      const int bx = blk % p.nbx, by = (blk / p.nbx) % p.nby, n = blk / (p.nbx * p.nby);
-      const int head = grp * C::PARTS + ((STRIDE == 1) ? 0 : wq);
-      const int y0 = by * kBlock - p.halo, x0 = bx * kBlock - p.halo;
+      const ItemCoord ic = item_coord(blockIdx.x + k * gridDim.x, groups, p.nbx, p.nby);
+      const int y0 = ic.by * kBlock - p.halo, x0 = ic.bx * kBlock - p.halo;
+      const uint32_t ts = tq + sl * kSlotCols;
 
-      float l = 0.f;
+      float rh[C::NROW];
+      float rw[WIN];
+      float sv[C::NROW][16];
+      float m = -INFINITY;
       if (active) {
-        // ---- relative logits: G row -> this warp's scratch (inside its P rows)
+        // ---- relative logits: this query's G row -> scratch line -> gather
         {
           uint32_t gr[32];
-          tmem_ld_16x32bx2_x32<32>(tq + kTmemG, gr);
+          tmem_ld_16x32bx2_x32<24>(ts + kTmemG, gr);  // half 0: rel_h part, half 1: rel_w part (from col 24)
           tmem_wait_ld();
-          // scratch float j of row r16 lives at chunk j/8, P row (16*wq + r16), byte 4*(j%8)
+          float* line = scr + (2 * r16 + half) * C::SCRATCH_LINE;
 #pragma unroll
-          for (int cc = 0; cc < 4; ++cc) {
-            uint8_t* dst = pt + (half * 4 + cc) * 2048 + row * 32;
-            reinterpret_cast<uint4*>(dst)[0] = make_uint4(gr[8 * cc + 0], gr[8 * cc + 1], gr[8 * cc + 2], gr[8 * cc + 3]);
-            reinterpret_cast<uint4*>(dst)[1] = make_uint4(gr[8 * cc + 4], gr[8 * cc + 5], gr[8 * cc + 6], gr[8 * cc + 7]);
-          }
+          for (int t = 0; t < 8; ++t)
+            reinterpret_cast<uint4*>(line)[t] =
+                make_uint4(gr[4 * t + 0], gr[4 * t + 1], gr[4 * t + 2], gr[4 * t + 3]);
         }
         __syncwarp();
-        auto scratch = [&](int jj) -> float {
-          return *reinterpret_cast<const float*>(pt + (jj >> 3) * 2048 + row * 32 + (jj & 7) * 4);
-        };
-        float rh[C::NROW];
-        float rw[WIN];
+        const float* lh = scr + (2 * r16) * C::SCRATCH_LINE;                        // rel_h logits
+        const float* lw = scr + (2 * r16 + 1) * C::SCRATCH_LINE + (kGRelW - 24);   // rel_w logits
 #pragma unroll
         for (int i = 0; i < C::NROW; ++i) {
           const int kr = 2 * i + half;
           const int Y = y0 + kr;
-          rh[i] = (Y >= 0 && Y < p.H) ? scratch(kr - qy + WIN - 1) : -INFINITY;
+          rh[i] = (Y >= 0 && Y < p.H) ? lh[kr - qy + WIN - 1] : -INFINITY;
         }
 #pragma unroll
         for (int kc = 0; kc < WIN; ++kc) {
           const int X = x0 + kc;
-          rw[kc] = (X >= 0 && X < p.W) ? scratch(32 + kc - qx + WIN - 1) : -INFINITY;
+          rw[kc] = (X >= 0 && X < p.W) ? lw[kc - qx + WIN - 1] : -INFINITY;
         }
-        __syncwarp();
 
-        // ---- S rows of this thread: window rows 2i + half
-        float sv[C::NROW][16];
+        // ---- S rows of this thread: window rows 2i + half (WIN keys each)
 #pragma unroll
-        for (int i = 0; i < C::NROW; ++i) {
-          tmem_ld_16x32bx2_x16<16>(tq + kTmemS + 32 * i, *reinterpret_cast<uint32_t(*)[16]>(&sv[i][0]));
-        }
+        for (int i = 0; i < C::NROW; ++i)
+          tmem_ld_16x32bx2_x16<WIN>(ts + 2 * WIN * i, *reinterpret_cast<uint32_t(*)[16]>(&sv[i][0]));
         tmem_wait_ld();
-        tc_fence_before();
 
         // ---- exact row max of z = S + rel_h + rel_w over in-image keys
-        float m = -INFINITY;
 #pragma unroll
         for (int i = 0; i < C::NROW; ++i) {
           float mi = -INFINITY;
@@ -435,8 +549,20 @@ __global__ void __launch_bounds__(kThreads, 1)
           m = fmaxf(m, mi + rh[i]);
         }
         m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 16));
-        const float mc = m * c;
+      }
+      tc_fence_before();
 
+      // ---- finish the previous item while this one's P is not yet written:
+      // its PV has had the whole gather + max to complete, and P(j-1) must be
+      // consumed before P(j) overwrites the warpgroup's P tile.
+      if (j >= 1 && !epilogue(j - 1, prev_ic, prev_l)) {
+        ok = false;
+        break;
+      }
+
+      float l = 0.f;
+      if (active) {
+        const float mc = m * c;
         // ---- p = 2^(c*z - c*m); bf16 P into the swizzled operand tile
 #pragma unroll
         for (int i = 0; i < C::NROW; ++i) {
@@ -469,54 +595,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         fence_proxy_async_smem();
       }
       __syncwarp();
-      if (lane == 0) mbar_arrive(&bar_pfull[g]);
-
-      // ---- O = P V, normalise, store
-      if (!mbar_wait(&bar_ofull[g], j & 1, kWaitNs, &abort_flag)) {
-        if (!abort_flag) record_timeout(&abort_flag);
-        break;
-      }
-      tc_fence_after();
-      if (active) {
-        const uint32_t oaddr = tq + kTmemO + ((STRIDE == 1) ? 0 : wq * C::O_COLS);
-        float o[D / 2];
-        if constexpr (D == 16) {
-          uint32_t r[8];
-          tmem_ld_16x32bx2_x8<8>(oaddr, r);
-          uint32_t rs[8];
-          tmem_ld_16x32bx2_x8<8>(oaddr + D, rs);  // row sums (ones tile): every column holds the sum
-          tmem_wait_ld();
-#pragma unroll
-          for (int t = 0; t < 8; ++t) o[t] = __uint_as_float(r[t]);
-          l = __uint_as_float(rs[0]);
-        } else if constexpr (D == 32) {
-          uint32_t r[16];
-          tmem_ld_16x32bx2_x16<16>(oaddr, r);
-          tmem_wait_ld();
-#pragma unroll
-          for (int t = 0; t < 16; ++t) o[t] = __uint_as_float(r[t]);
-        } else {
-          uint32_t r[32];
-          tmem_ld_16x32bx2_x32<32>(oaddr, r);
-          tmem_wait_ld();
-#pragma unroll
-          for (int t = 0; t < 32; ++t) o[t] = __uint_as_float(r[t]);
-        }
-        const float inv = 1.0f / l;
-        uint32_t pk[D / 4];
-#pragma unroll
-        for (int t = 0; t < D / 4; ++t) pk[t] = pack_bf16x2(o[2 * t] * inv, o[2 * t + 1] * inv);
-        const int y = by * kBlock + qy, x = bx * kBlock + qx;
-        const int oy = y / STRIDE, ox = x / STRIDE;
-        __nv_bfloat16* dst = p.out + ((static_cast<size_t>(n) * p.OH + oy) * p.OW + ox) * C_all + head * D + half * (D / 2);
-#pragma unroll
-        for (int t = 0; t < D / 16; ++t)
-          reinterpret_cast<uint4*>(dst)[t] = make_uint4(pk[4 * t], pk[4 * t + 1], pk[4 * t + 2], pk[4 * t + 3]);
-      }
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&bar_tfree[g]);
+      if (lane == 0) mbar_arrive(&bar_pfull[b]);
+      prev_ic = ic;
+      prev_l = l;
     }
+    if (ok && j >= 1) epilogue(j - 1, prev_ic, prev_l);
   }
 
   // ---------------------------------------------------------------- teardown

@@ -100,7 +100,7 @@ def test_kernel_selection(name, kernel):
 
 CASES = []
 for d in (16, 32, 64):
-    for halo in (1, 2, 3, 4):
+    for halo in (0, 1, 2, 3):
         for stride in (1, 2):
             CASES.append(dict(N=2, H=24, W=40, heads=8 if d < 64 else 4, dim_head=d, block=8, halo=halo,
                               stride=stride))
@@ -109,7 +109,7 @@ CASES += [
     dict(N=1, H=8, W=8, heads=2, dim_head=32, block=8, halo=3, stride=1),    # block = map, halo all outside
     dict(N=3, H=16, W=8, heads=4, dim_head=64, block=8, halo=0, stride=2),   # isolated blocks, stride 2
     dict(N=5, H=8, W=56, heads=8, dim_head=16, block=8, halo=3, stride=1),   # one block row, ragged items
-    dict(N=1, H=64, W=8, heads=2, dim_head=32, block=8, halo=4, stride=2),   # one block column
+    dict(N=1, H=64, W=8, heads=2, dim_head=32, block=8, halo=3, stride=2),   # one block column
 ]
 
 
@@ -132,6 +132,7 @@ SIMT_CASES = [
     dict(N=1, H=32, W=32, heads=2, dim_head=128, block=16, halo=2, stride=1, dtype="f32"),
     dict(N=2, H=32, W=32, heads=4, dim_head=32, block=16, halo=4, stride=1, dtype="bf16"),
     dict(N=1, H=16, W=16, heads=1, dim_head=16, block=8, halo=3, stride=2, dtype="bf16"),
+    dict(N=2, H=24, W=16, heads=4, dim_head=16, block=8, halo=4, stride=1, dtype="bf16"),
 ]
 
 
