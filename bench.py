@@ -35,7 +35,8 @@ import torch  # noqa: E402
 import workloads  # noqa: E402
 
 METRIC = "halo-attention output pixels/s and TFLOP/s, % of bf16 tensor/HBM roofline"
-KERNEL_SOURCES = ["blocked_local_self_b200/csrc/halo_tc.cuh", "blocked_local_self_b200/csrc/sm100.cuh"]
+KERNEL_SOURCES = ["blocked_local_self_b200/csrc/halo_tc.cuh", "blocked_local_self_b200/csrc/halo_tc2.cuh",
+                  "blocked_local_self_b200/csrc/sm100.cuh"]
 TRAFFIC_FILE = os.path.join(ROOT, "profiles", "traffic_halo_fwd_tc.json")
 L2_BYTES = 126 * 1024 * 1024
 

@@ -13,6 +13,7 @@
 #include "../../include/halo.h"
 #include "halo_simt.cuh"
 #include "halo_tc.cuh"
+#include "halo_tc2.cuh"
 
 namespace {
 
@@ -90,6 +91,30 @@ const TcEntry kTcTable[] = {
     HALO_TC_WINS(16, 2), HALO_TC_WINS(32, 2), HALO_TC_WINS(64, 2),
 };
 
+// Stride-1 kernel with two heads per 128-row tile: (d, window) -> instantiation.
+using Tc2Kernel = void (*)(const CUtensorMap, const CUtensorMap, const CUtensorMap, const halo::tc2::Params);
+struct Tc2Entry {
+  int d, win;
+  Tc2Kernel fn;
+  int (*smem)(int);
+};
+template <int D, int WIN>
+int tc2_smem(int stages) { return halo::tc2::smem_bytes<D, WIN>(stages); }
+#define HALO_TC2_ENTRY(D, WIN) \
+  Tc2Entry { D, WIN, halo::tc2::halo_fwd_tc2<D, WIN>, tc2_smem<D, WIN> }
+const Tc2Entry kTc2Table[] = {
+    HALO_TC2_ENTRY(16, 8),  HALO_TC2_ENTRY(16, 10), HALO_TC2_ENTRY(16, 12), HALO_TC2_ENTRY(16, 14),
+    HALO_TC2_ENTRY(32, 8),  HALO_TC2_ENTRY(32, 10), HALO_TC2_ENTRY(32, 12), HALO_TC2_ENTRY(32, 14),
+};
+
+const Tc2Entry* find_tc2(const Shape& s) {
+  if (s.dtype != HALO_BF16 || s.block != halo::tc2::kBlock || s.stride != 1 || s.heads % 2) return nullptr;
+  const int win = s.block + 2 * s.halo;
+  for (const Tc2Entry& e : kTc2Table)
+    if (e.d == s.d && e.win == win) return &e;
+  return nullptr;
+}
+
 const TcEntry* find_tc(const Shape& s) {
   if (s.dtype != HALO_BF16 || s.block != halo::tc::kBlock) return nullptr;
   const int win = s.block + 2 * s.halo;
@@ -100,7 +125,7 @@ const TcEntry* find_tc(const Shape& s) {
 
 int select_kernel(const Shape& s) {
   if (check_shape(s) != HALO_OK) return HALO_KERNEL_NONE;
-  if (find_tc(s)) return HALO_KERNEL_TC_BF16;
+  if (find_tc2(s) || find_tc(s)) return HALO_KERNEL_TC_BF16;
   if (s.d <= 128) return HALO_KERNEL_SIMT_F32;
   return HALO_KERNEL_NONE;
 }
@@ -256,6 +281,50 @@ int launch_tc(const TcEntry& e, const void* q, const void* k, const void* v, con
   return cudaGetLastError() == cudaSuccess ? HALO_OK : HALO_ERR_CUDA;
 }
 
+int launch_tc2(const Tc2Entry& e, const void* q, const void* k, const void* v, const void* rh, const void* rw,
+               void* out, const Shape& s, int sm_count, cudaStream_t st) {
+  const int win = s.block + 2 * s.halo;
+  CUtensorMap mq, mk, mv;
+  if (!encode_nhwc(&mq, q, s, halo::tc2::kBlock, halo::tc2::kBlock, 1) || !encode_nhwc(&mk, k, s, win, win, 1) ||
+      !encode_nhwc(&mv, v, s, win, win, 1))
+    return HALO_ERR_CUDA;
+  cudaFuncAttributes attr;
+  if (cudaFuncGetAttributes(&attr, reinterpret_cast<const void*>(e.fn)) != cudaSuccess) return HALO_ERR_CUDA;
+  if (256 * halo::tc2::kSoftmaxRegs + 128 * halo::tc2::kProducerRegs > halo::tc2::kThreads * attr.numRegs)
+    return HALO_ERR_UNSUPPORTED;
+  int optin = 0, dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) != cudaSuccess)
+    return HALO_ERR_CUDA;
+  const int budget = (optin < kMaxDynSmem ? optin : kMaxDynSmem) - static_cast<int>(attr.sharedSizeBytes);
+  int stages = 8;
+  while (stages > 1 && e.smem(stages) > budget) --stages;
+  const int smem = e.smem(stages);
+  if (smem > budget) return HALO_ERR_UNSUPPORTED;
+  if (cudaFuncSetAttribute(reinterpret_cast<const void*>(e.fn), cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           smem) != cudaSuccess)
+    return HALO_ERR_CUDA;
+  halo::tc2::Params p;
+  p.rel_h = static_cast<const __nv_bfloat16*>(rh);
+  p.rel_w = static_cast<const __nv_bfloat16*>(rw);
+  p.out = static_cast<__nv_bfloat16*>(out);
+  p.N = s.N;
+  p.H = s.H;
+  p.W = s.W;
+  p.heads = s.heads;
+  p.halo = s.halo;
+  p.nbx = s.W / halo::tc2::kBlock;
+  p.nby = s.H / halo::tc2::kBlock;
+  const long long items = static_cast<long long>(s.N) * p.nbx * p.nby * (s.heads / 2);
+  if (items > 0x7fffffffLL) return HALO_ERR_DIMS;
+  p.num_items = static_cast<int>(items);
+  p.stages = stages;
+  p.c = 1.4426950408889634f / std::sqrt(static_cast<float>(s.d));
+  const int grid = static_cast<int>(items < sm_count ? items : sm_count);
+  e.fn<<<grid, halo::tc2::kThreads, smem, st>>>(mq, mk, mv, p);
+  return cudaGetLastError() == cudaSuccess ? HALO_OK : HALO_ERR_CUDA;
+}
+
 int attn_device(const void* q, const void* k, const void* v, const void* rel_h, const void* rel_w, void* out,
                 const Shape& s, cudaStream_t st) {
   int rc = check_shape(s);
@@ -267,7 +336,10 @@ int attn_device(const void* q, const void* k, const void* v, const void* rel_h, 
   int sm_count = 0;
   rc = device_info(&sm_count);
   if (rc != HALO_OK) return rc;
-  if (kind == HALO_KERNEL_TC_BF16) return launch_tc(*find_tc(s), q, k, v, rel_h, rel_w, out, s, sm_count, st);
+  if (kind == HALO_KERNEL_TC_BF16) {
+    if (const Tc2Entry* e2 = find_tc2(s)) return launch_tc2(*e2, q, k, v, rel_h, rel_w, out, s, sm_count, st);
+    return launch_tc(*find_tc(s), q, k, v, rel_h, rel_w, out, s, sm_count, st);
+  }
   cudaError_t err = (s.dtype == HALO_F32) ? launch_simt<float>(q, k, v, rel_h, rel_w, out, s, st)
                                           : launch_simt<__nv_bfloat16>(q, k, v, rel_h, rel_w, out, s, st);
   return err == cudaSuccess ? HALO_OK : HALO_ERR_CUDA;
