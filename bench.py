@@ -36,8 +36,8 @@ import workloads  # noqa: E402
 
 METRIC = "halo-attention output pixels/s and TFLOP/s, % of bf16 tensor/HBM roofline"
 KERNEL_SOURCES = ["blocked_local_self_b200/csrc/halo_tc.cuh", "blocked_local_self_b200/csrc/halo_tc2.cuh",
-                  "blocked_local_self_b200/csrc/sm100.cuh"]
-TRAFFIC_FILE = os.path.join(ROOT, "profiles", "traffic_halo_fwd_tc.json")
+                  "blocked_local_self_b200/csrc/halo_tc3.cuh", "blocked_local_self_b200/csrc/sm100.cuh"]
+PROFILES = os.path.join(ROOT, "profiles")
 L2_BYTES = 126 * 1024 * 1024
 
 
@@ -183,17 +183,21 @@ def kernel_source_hash() -> str:
 
 
 def ncu_traffic(workload: str):
-    """DRAM bytes per launch from the committed ncu summary, only while the
-    kernel source still matches the one that was profiled."""
-    try:
-        with open(TRAFFIC_FILE) as f:
-            d = json.load(f)
-    except (OSError, ValueError):
-        return None
-    entry = d.get(workload)
-    if not entry or entry.get("kernel_source_sha") != kernel_source_hash():
-        return None
-    return entry.get("dram_bytes_per_launch")
+    """DRAM bytes per launch (dram__bytes_read.sum + dram__bytes_write.sum)
+    from a committed ncu summary under profiles/ that names this workload,
+    only while the kernel sources still hash to the value it records."""
+    import glob
+    import re
+    for path in sorted(glob.glob(os.path.join(PROFILES, "*.md"))):
+        with open(path) as f:
+            text = f.read()
+        fields = dict(re.findall(r"^- (\w+): `?([^`\n]+?)`?\s*$", text, flags=re.M))
+        if fields.get("workload") != workload or "dram_bytes_per_launch" not in fields:
+            continue
+        if fields.get("kernel_source_sha") != kernel_source_hash():
+            return None
+        return float(fields["dram_bytes_per_launch"])
+    return None
 
 
 # ---------------------------------------------------------------------------
@@ -280,8 +284,8 @@ def main():
         s = sets[i % n_sets]
         halo.attn(*s, block=wl.block, halo=wl.halo, stride=wl.stride, out=outs[i % n_sets], stream=stream)
 
-    kernel = halo.kernel_for(wl.N, wl.H, wl.W, wl.heads, wl.dim_head, wl.block, wl.halo, wl.stride,
-                             wl.torch_dtype)
+    kernel = halo.kernel_name(wl.N, wl.H, wl.W, wl.heads, wl.dim_head, wl.block, wl.halo, wl.stride,
+                              wl.torch_dtype)
     for i in range(args.warmup):
         step(i)
     torch.cuda.synchronize()

@@ -18,7 +18,7 @@ import torch
 from . import _native
 from ._native import HaloError, HALO_BF16, HALO_F32
 
-__all__ = ["attn", "attn_host", "kernel_for", "get_last_error", "debug_wait_timeout", "version", "HaloError",
+__all__ = ["attn", "attn_host", "kernel_for", "kernel_name", "get_last_error", "debug_wait_timeout", "version", "HaloError",
            "load"]
 
 
@@ -102,6 +102,13 @@ def kernel_for(N: int, H: int, W: int, heads: int, dim_head: int, block: int, ha
     code = HALO_BF16 if dtype == torch.bfloat16 else HALO_F32
     k = _native.lib().halo_kernel_for(N, H, W, heads, dim_head, block, halo, stride, code)
     return {0: "none", 1: "simt_f32", 2: "tc_bf16"}[k]
+
+
+def kernel_name(N: int, H: int, W: int, heads: int, dim_head: int, block: int, halo: int, stride: int,
+                dtype: torch.dtype) -> str:
+    """Instantiation ``attn`` launches for a shape, e.g. "halo_fwd_tc2<16,14>", or "none"."""
+    code = HALO_BF16 if dtype == torch.bfloat16 else HALO_F32
+    return _native.lib().halo_kernel_name(N, H, W, heads, dim_head, block, halo, stride, code).decode()
 
 
 def get_last_error() -> int:

@@ -40,6 +40,7 @@ SIGNATURES = {
     "halo_attn": (_i, [_vp] * 6 + [_i] * 9 + [_vp]),
     "halo_attn_host": (_i, [_vp] * 12 + [_i] * 9 + [_vp]),
     "halo_kernel_for": (_i, [_i] * 9),
+    "halo_kernel_name": (ctypes.c_char_p, [_i] * 9),
     "halo_strerror": (ctypes.c_char_p, [_i]),
     "halo_get_last_error": (_i, []),
     "halo_debug_wait_timeout": (_i, [_i, _vp]),

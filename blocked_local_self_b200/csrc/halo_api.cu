@@ -7,6 +7,7 @@
 
 #include <cmath>
 #include <cstdint>
+#include <cstdio>
 #include <cstring>
 #include <mutex>
 
@@ -14,6 +15,7 @@
 #include "halo_simt.cuh"
 #include "halo_tc.cuh"
 #include "halo_tc2.cuh"
+#include "halo_tc3.cuh"
 
 namespace {
 
@@ -115,6 +117,30 @@ const Tc2Entry* find_tc2(const Shape& s) {
   return nullptr;
 }
 
+// Stride-1 kernel for 16x16 query blocks: (d, window) -> instantiation.
+using Tc3Kernel = void (*)(const CUtensorMap, const CUtensorMap, const CUtensorMap, const halo::tc3::Params);
+struct Tc3Entry {
+  int d, win;
+  Tc3Kernel fn;
+  int (*smem)(int);
+};
+template <int D, int WIN>
+int tc3_smem(int stages) { return halo::tc3::smem_bytes<D, WIN>(stages); }
+#define HALO_TC3_ENTRY(D, WIN) \
+  Tc3Entry { D, WIN, halo::tc3::halo_fwd_tc3<D, WIN>, tc3_smem<D, WIN> }
+#define HALO_TC3_WINS(D)                                                                   \
+  HALO_TC3_ENTRY(D, 16), HALO_TC3_ENTRY(D, 18), HALO_TC3_ENTRY(D, 20), HALO_TC3_ENTRY(D, 22), \
+      HALO_TC3_ENTRY(D, 24)
+const Tc3Entry kTc3Table[] = {HALO_TC3_WINS(16), HALO_TC3_WINS(32)};
+
+const Tc3Entry* find_tc3(const Shape& s) {
+  if (s.dtype != HALO_BF16 || s.block != halo::tc3::kBlock || s.stride != 1) return nullptr;
+  const int win = s.block + 2 * s.halo;
+  for (const Tc3Entry& e : kTc3Table)
+    if (e.d == s.d && e.win == win) return &e;
+  return nullptr;
+}
+
 const TcEntry* find_tc(const Shape& s) {
   if (s.dtype != HALO_BF16 || s.block != halo::tc::kBlock) return nullptr;
   const int win = s.block + 2 * s.halo;
@@ -125,7 +151,7 @@ const TcEntry* find_tc(const Shape& s) {
 
 int select_kernel(const Shape& s) {
   if (check_shape(s) != HALO_OK) return HALO_KERNEL_NONE;
-  if (find_tc2(s) || find_tc(s)) return HALO_KERNEL_TC_BF16;
+  if (find_tc2(s) || find_tc(s) || find_tc3(s)) return HALO_KERNEL_TC_BF16;
   if (s.d <= 128) return HALO_KERNEL_SIMT_F32;
   return HALO_KERNEL_NONE;
 }
@@ -325,6 +351,50 @@ int launch_tc2(const Tc2Entry& e, const void* q, const void* k, const void* v, c
   return cudaGetLastError() == cudaSuccess ? HALO_OK : HALO_ERR_CUDA;
 }
 
+int launch_tc3(const Tc3Entry& e, const void* q, const void* k, const void* v, const void* rh, const void* rw,
+               void* out, const Shape& s, int sm_count, cudaStream_t st) {
+  const int win = s.block + 2 * s.halo;
+  CUtensorMap mq, mk, mv;
+  if (!encode_nhwc(&mq, q, s, halo::tc3::kBlock, halo::tc3::kBlock, 1) || !encode_nhwc(&mk, k, s, win, win, 1) ||
+      !encode_nhwc(&mv, v, s, win, win, 1))
+    return HALO_ERR_CUDA;
+  cudaFuncAttributes attr;
+  if (cudaFuncGetAttributes(&attr, reinterpret_cast<const void*>(e.fn)) != cudaSuccess) return HALO_ERR_CUDA;
+  if (256 * halo::tc3::kSoftmaxRegs + 128 * halo::tc3::kProducerRegs > halo::tc3::kThreads * attr.numRegs)
+    return HALO_ERR_UNSUPPORTED;
+  int optin = 0, dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) != cudaSuccess)
+    return HALO_ERR_CUDA;
+  const int budget = (optin < kMaxDynSmem ? optin : kMaxDynSmem) - static_cast<int>(attr.sharedSizeBytes);
+  int stages = 4;  // the kernel has four stage barriers
+  while (stages > 1 && e.smem(stages) > budget) --stages;
+  const int smem = e.smem(stages);
+  if (smem > budget) return HALO_ERR_UNSUPPORTED;
+  if (cudaFuncSetAttribute(reinterpret_cast<const void*>(e.fn), cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           smem) != cudaSuccess)
+    return HALO_ERR_CUDA;
+  halo::tc3::Params p;
+  p.rel_h = static_cast<const __nv_bfloat16*>(rh);
+  p.rel_w = static_cast<const __nv_bfloat16*>(rw);
+  p.out = static_cast<__nv_bfloat16*>(out);
+  p.N = s.N;
+  p.H = s.H;
+  p.W = s.W;
+  p.heads = s.heads;
+  p.halo = s.halo;
+  p.nbx = s.W / halo::tc3::kBlock;
+  p.nby = s.H / halo::tc3::kBlock;
+  const long long items = static_cast<long long>(s.N) * p.nbx * p.nby * s.heads;
+  if (items > 0x7fffffffLL) return HALO_ERR_DIMS;
+  p.num_items = static_cast<int>(items);
+  p.stages = stages;
+  p.c = 1.4426950408889634f / std::sqrt(static_cast<float>(s.d));
+  const int grid = static_cast<int>(items < sm_count ? items : sm_count);
+  e.fn<<<grid, halo::tc3::kThreads, smem, st>>>(mq, mk, mv, p);
+  return cudaGetLastError() == cudaSuccess ? HALO_OK : HALO_ERR_CUDA;
+}
+
 int attn_device(const void* q, const void* k, const void* v, const void* rel_h, const void* rel_w, void* out,
                 const Shape& s, cudaStream_t st) {
   int rc = check_shape(s);
@@ -338,6 +408,7 @@ int attn_device(const void* q, const void* k, const void* v, const void* rel_h, 
   if (rc != HALO_OK) return rc;
   if (kind == HALO_KERNEL_TC_BF16) {
     if (const Tc2Entry* e2 = find_tc2(s)) return launch_tc2(*e2, q, k, v, rel_h, rel_w, out, s, sm_count, st);
+    if (const Tc3Entry* e3 = find_tc3(s)) return launch_tc3(*e3, q, k, v, rel_h, rel_w, out, s, sm_count, st);
     return launch_tc(*find_tc(s), q, k, v, rel_h, rel_w, out, s, sm_count, st);
   }
   cudaError_t err = (s.dtype == HALO_F32) ? launch_simt<float>(q, k, v, rel_h, rel_w, out, s, st)
@@ -396,6 +467,27 @@ int halo_attn_host(const void* q_h, const void* k_h, const void* v_h, const void
 int halo_kernel_for(int N, int H, int W, int heads, int dim_head, int block, int halo, int stride, int dtype) {
   const Shape s{N, H, W, heads, dim_head, block, halo, stride, dtype};
   return select_kernel(s);
+}
+
+const char* halo_kernel_name(int N, int H, int W, int heads, int dim_head, int block, int halo, int stride,
+                             int dtype) {
+  thread_local char name[64];
+  const Shape s{N, H, W, heads, dim_head, block, halo, stride, dtype};
+  const int kind = select_kernel(s);
+  if (kind == HALO_KERNEL_NONE) {
+    std::snprintf(name, sizeof(name), "none");
+  } else if (kind == HALO_KERNEL_TC_BF16) {
+    if (const Tc2Entry* e = find_tc2(s)) std::snprintf(name, sizeof(name), "halo_fwd_tc2<%d,%d>", e->d, e->win);
+    else if (const Tc3Entry* e = find_tc3(s)) std::snprintf(name, sizeof(name), "halo_fwd_tc3<%d,%d>", e->d, e->win);
+    else {
+      const TcEntry* t = find_tc(s);
+      std::snprintf(name, sizeof(name), "halo_fwd_tc<%d,%d,%d>", t->d, t->win, t->stride);
+    }
+  } else {
+    const int dmax = s.d <= 16 ? 16 : s.d <= 32 ? 32 : s.d <= 64 ? 64 : 128;
+    std::snprintf(name, sizeof(name), "halo_fwd_simt<%s,%d>", s.dtype == HALO_F32 ? "float" : "bf16", dmax);
+  }
+  return name;
 }
 
 const char* halo_strerror(int code) { return status_text(code); }

@@ -394,6 +394,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           polls = 0;
           idle_since = global_timer_ns();
         } else if ((++polls & 15u) == 0) {
+          __nanosleep(200);  // back off instead of spinning on the issue slots
           if (*(volatile int*)&abort_flag) break;
           if (global_timer_ns() - idle_since > kWaitNs) {
             record_timeout(&abort_flag);

@@ -13,7 +13,7 @@
 // or 32 the A.V product is a long chain of such small MMAs, so this kernel
 // (a) packs two heads into every 128-row tile, (b) folds the relative dot
 // products into the QK^T MMA as 56 extra B rows (N = 256), and (c) splits the
-// A.V chain over the four warps of the softmax warpgroup, each issuing its own
+// A.V chain over the warps of the softmax warpgroup, each issuing its own
 // K-step range into its own accumulator.
 //
 // Work item = one 8x8 query block and a pair of heads (a, b):
@@ -25,15 +25,18 @@
 //     L holds one query row of one head: columns [0, w*w) are q.k, columns
 //     [200, 256) the relative dot products q.rel_h[.] and q.rel_w[.].
 //   * softmax warpgroup (one thread per TMEM lane = one query row): gather the
-//     14 + 14 relative logits of its query, then the window keys in two
-//     chunks, each with its own exact maximum; exponentials part on MUFU,
-//     part as a cubic polynomial on the FMA pipe; bf16 P written back into
-//     the same TMEM lane (tcgen05.st) over the consumed S columns.
-//   * A.V (issued by the softmax warps): O_s = P[:, keys of stream s] [V_a|V_b],
-//     M=128 with P read from TMEM, N = 2d (head a's rows use the V_a columns,
-//     head b's the V_b columns), one accumulator per stream.
-//   * epilogue: O = sum over chunks of 2^(c(m_chunk - m)) * O_chunk, divided
-//     by the same combination of the chunk row sums, bf16, stored NHWC.
+//     14 + 14 relative logits of its query, then the window keys in three
+//     (d = 16) or two (d = 32) chunks of whole K-steps, each with its own
+//     exact maximum; exponentials part on MUFU, part as a cubic polynomial on
+//     the FMA pipe; bf16 P written back into the same TMEM lane (tcgen05.st)
+//     over the consumed S columns.
+//   * A.V (warp q of the warpgroup issues chunk q): O_q = P[:, keys of chunk q]
+//     [V_a | V_b | 1], M=128 with P read from TMEM, N = 3d for d = 16 (the
+//     ones block yields the chunk's row sum of the bf16 P) or N = 2d for
+//     d = 32 (row sums added on the CUDA cores); head a's rows use the V_a
+//     columns, head b's the V_b columns.
+//   * epilogue: O = sum over chunks of 2^(c(m_q - m)) * O_q, divided by the
+//     same combination of the chunk row sums, bf16, stored NHWC.
 // Two softmax warpgroups work on alternate items, each in its own half of
 // TMEM.  Every wait is bounded and reports HALO_ERR_TIMEOUT.
 #pragma once
@@ -41,6 +44,7 @@
 #include <cstdint>
 #include <cuda.h>
 #include <cuda_bf16.h>
+#include <utility>
 
 #include "halo_tc.cuh"
 #include "sm100.cuh"
@@ -86,16 +90,21 @@ struct Cfg {
   static constexpr int KS = WIN * WIN;                    // window keys
   static constexpr int KSTEPS = (KS + 15) / 16;           // A.V K-steps
   static constexpr int KP = KSTEPS * 16;                  // keys incl. zero padding
-  static constexpr int C1STEPS = KSTEPS / 2;              // chunk 1 = K-steps [0, C1STEPS)
-  static constexpr int C1 = C1STEPS * 16;                 // keys of chunk 1
+  // The keys are cut into NCHUNK chunks of whole K-steps; each chunk has its
+  // own row maximum and its own A.V accumulator, issued by its own warp.
+  static constexpr int NCHUNK = (D == 16) ? 3 : 2;
+  static constexpr int NSTREAM = NCHUNK;
+  // d = 16: a third B atom of ones makes the A.V MMA also produce the row
+  // sums of the bf16 P it consumed; d = 32 sums on the CUDA cores.
+  static constexpr bool SUM_BY_MMA = (D == 16);
   static constexpr int PCOLS = KP / 2;                    // packed bf16 P columns in TMEM
-  static constexpr int NSTREAM = (D == 16) ? 4 : 2;       // A.V issue streams (2 per chunk or 1)
-  static constexpr int O_N = 2 * D;                       // A.V N: [V_a | V_b]
+  static constexpr int O_N = SUM_BY_MMA ? 3 * D : 2 * D;  // A.V N: [V_a | V_b (| ones)]
   static constexpr int O_BASE = (PCOLS + 7) / 8 * 8;      // first O column
   static constexpr int Q_TILE = 64 * ROWB;
   static constexpr int K_TILE = kKRows * ROWB;
   static constexpr int V_TILE = KP * ROWB;
-  static constexpr int STAGE_RAW = 2 * (Q_TILE + K_TILE + V_TILE);
+  static constexpr int ONES_TILE = SUM_BY_MMA ? V_TILE : 0;  // right after V_b: third atom at 2*LBO
+  static constexpr int STAGE_RAW = 2 * (Q_TILE + K_TILE + V_TILE) + ONES_TILE;
   static constexpr int STAGE_BYTES = (STAGE_RAW + 1023) / 1024 * 1024;
   static constexpr int TX_BYTES = 2 * (64 + 2 * KS) * ROWB;
   static constexpr int SCRATCH = 256 * kScratchLine * 4;
@@ -113,22 +122,71 @@ struct Cfg {
   static_assert(NPOLY <= 8, "polynomial columns");
 };
 
+// First K-step of chunk i (i = 0..NCHUNK); chunk i covers keys
+// [16*chunk_step(i), 16*chunk_step(i+1)), the last one ending at the window.
+template <int KSTEPS, int NCHUNK>
+__host__ __device__ constexpr int chunk_step(int i) {
+  return (KSTEPS * i + NCHUNK / 2) / NCHUNK;
+}
+
 template <int D, int WIN>
 __host__ __device__ constexpr int smem_bytes(int stages) {
   using C = Cfg<D, WIN>;
   return 1024 + C::SCRATCH + stages * C::STAGE_BYTES;
 }
 
-// Which window columns take the polynomial exponential: a bit mask over kc,
-// spreading the picks over the block's own columns h+1, h+5, h+3, h+6, ...
+// Which window-column pairs (kc, kc+1), kc even, take the polynomial
+// exponential: about 30% of the columns, inside the block's own 8 columns
+// [h, h+8), which are never outside the image.  Bit kc/2 of the mask.
+#ifndef HALO_TC2_POLY_PAIRS
+#define HALO_TC2_POLY_PAIRS ((WIN * 3 + 10) / 20)  // 14 -> 2, 12 -> 2, 10 -> 2, 8 -> 1
+#endif
 template <int WIN>
-__host__ __device__ constexpr unsigned poly_mask() {
+__host__ __device__ constexpr unsigned poly_pair_mask() {
   constexpr int h = (WIN - kBlock) / 2;
-  constexpr int n = (WIN * 2 + 2) / 5;
-  const int order[8] = {1, 5, 3, 6, 2, 7, 4, 0};
+  constexpr int npairs = HALO_TC2_POLY_PAIRS;
   unsigned m = 0;
-  for (int i = 0; i < n; ++i) m |= 1u << (h + order[i]);
+  int picked = 0;
+  // even kc inside [h, h+8) with kc+1 < h+8, from the middle outwards
+  const int mid = (h + 3) & ~1;
+  for (int d = 0; d < 8 && picked < npairs; ++d) {
+    const int kc = mid + ((d & 1) ? -2 * ((d + 1) / 2) : 2 * (d / 2));
+    if (kc >= h && kc + 1 < h + 8 && !((m >> (kc / 2)) & 1u)) {
+      m |= 1u << (kc / 2);
+      ++picked;
+    }
+  }
   return m;
+}
+
+__device__ __forceinline__ float max3f(float a, float b, float c) {
+  float r;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
+}
+
+// 2^x for a pair of x <= 0 with packed f32x2 arithmetic on the FMA pipe:
+// x = j + f, j = floor(x) by a round-down add of 1.5*2^23, 2^f by the cubic
+// of exp2_poly, 2^j added into the exponent field.  Returns the values' bit
+// patterns (r) for the row sum.
+__device__ __forceinline__ void exp2_poly2(float2 x, uint32_t& rx, uint32_t& ry) {
+  x.x = fmaxf(x.x, -127.0f);
+  x.y = fmaxf(x.y, -127.0f);
+  const float2 t = __fadd2_rd(x, make_float2(12582912.0f, 12582912.0f));
+  const float2 j = __fadd2_rn(t, make_float2(-12582912.0f, -12582912.0f));
+  const float2 f = __ffma2_rn(j, make_float2(-1.0f, -1.0f), x);
+  float2 q = __ffma2_rn(f, make_float2(0.0770670548f, 0.0770670548f), make_float2(0.2276449651f, 0.2276449651f));
+  q = __ffma2_rn(q, f, make_float2(0.6951168180f, 0.6951168180f));
+  q = __ffma2_rn(q, f, make_float2(1.0f, 1.0f));
+  rx = __float_as_uint(q.x) + (__float_as_uint(t.x) << 23);
+  ry = __float_as_uint(q.y) + (__float_as_uint(t.y) << 23);
+}
+
+// bf16x2 of two floats given as bit patterns, round to nearest even: the
+// P operand of the A.V MMA.  (Truncating instead saves little and, even with
+// its mean bias compensated, doubles the worst-case error of a P value.)
+__device__ __forceinline__ uint32_t pack_p(uint32_t lo, uint32_t hi) {
+  return pack_bf16x2(__uint_as_float(lo), __uint_as_float(hi));
 }
 
 // tcgen05.ld / st, 32 lanes x 32 bit: thread t <-> lane t of the warp's quadrant
@@ -199,52 +257,79 @@ __device__ __forceinline__ ItemCoord item_coord(int item, int pairs, int nbx, in
 // chunk row sum, packed bf16 P stored over TMEM columns [J0/2, JP/2) where JP
 // pads the chunk to whole K-steps (keys >= J1 get P = 0).  Window rows have
 // an even number of keys, so a packed pair never straddles two rows.
-template <int WIN, int J0, int J1, int JP>
+template <int WIN, int J0, int J1, int JP, bool SUM>
 __device__ __forceinline__ void softmax_chunk(uint32_t ts, const float (&rw)[WIN], const float (&rh)[WIN], float c,
                                               float& m_out, float& l_out) {
   constexpr int NL = (J1 - J0 + 7) / 8 * 8;  // S columns loaded (multiple of 8)
   constexpr int NW = (JP - J0) / 2;          // packed P words
-  static_assert(J0 % 2 == 0 && NW % 8 == 0, "chunk alignment");
+  constexpr int NP = (J1 - J0) / 2;          // key pairs of the chunk
+  static_assert(J0 % 2 == 0 && J1 % 2 == 0 && WIN % 2 == 0 && NW % 8 == 0, "pairs never straddle rows");
   constexpr int R0 = J0 / WIN, NR = (J1 - 1) / WIN - R0 + 1;
-  constexpr unsigned kPoly = poly_mask<WIN>();
+  constexpr unsigned kPoly = poly_pair_mask<WIN>();
   float z[NL];
   tmem_ld_cols<NL>(ts + J0, z);
   tmem_wait_ld();
-  // z = S + rel_w; per window row the maximum, then the chunk maximum of z + rel_h
-  float mrow[NR];
+  // z = S + rel_w (pairs); per window row the maximum; chunk maximum of z + rel_h
+  float2 zz[NP];
 #pragma unroll
-  for (int r = 0; r < NR; ++r) mrow[r] = -INFINITY;
-#pragma unroll
-  for (int j = J0; j < J1; ++j) {
-    z[j - J0] += rw[j % WIN];
-    mrow[j / WIN - R0] = fmaxf(mrow[j / WIN - R0], z[j - J0]);
+  for (int i = 0; i < NP; ++i) {
+    const int kc = (J0 + 2 * i) % WIN;
+    zz[i] = __fadd2_rn(make_float2(z[2 * i], z[2 * i + 1]), make_float2(rw[kc], rw[kc + 1]));
   }
   float m = -INFINITY;
 #pragma unroll
-  for (int r = 0; r < NR; ++r) m = fmaxf(m, mrow[r] + rh[R0 + r]);
-  const float mc = m * c;
-  float bias[NR];
+  for (int r = 0; r < NR; ++r) {
+    constexpr int dummy = 0;
+    (void)dummy;
+    const int i0 = ((R0 + r) * WIN > J0 ? (R0 + r) * WIN - J0 : 0) / 2;
+    const int i1 = (((R0 + r) * WIN + WIN < J1 ? (R0 + r) * WIN + WIN : J1) - J0) / 2;
+    float mr = -INFINITY;
 #pragma unroll
-  for (int r = 0; r < NR; ++r) bias[r] = fmaf(rh[R0 + r], c, -mc);  // -inf for rows outside the image
-  // p = 2^(c*z - c*m): masked keys (-inf) give exactly 0 on both paths
-  float l = 0.f;
-#pragma unroll
-  for (int j = J0; j < J1; ++j) {
-    const float x = fmaf(z[j - J0], c, bias[j / WIN - R0]);
-    const float v = ((kPoly >> (j % WIN)) & 1u) ? exp2_poly(x) : exp2_mufu(x);
-    z[j - J0] = v;
-    l += v;
+    for (int i = i0; i < i1; ++i) mr = max3f(mr, zz[i].x, zz[i].y);
+    m = fmaxf(m, mr + rh[R0 + r]);
   }
+  // a chunk without in-image keys keeps m = -inf (weight 0 in the epilogue)
+  // and takes its exponentials against 0: all of them are exactly 0
+  const float mcr = (m == -INFINITY ? 0.f : m) * c;
+  float brow[NR];  // per window row: c*rel_h - c*m; -inf outside the image
+#pragma unroll
+  for (int r = 0; r < NR; ++r) brow[r] = fmaf(rh[R0 + r], c, -mcr);
+  // p = 2^(c*z - c*m); rows outside the image give exact 0
+  float2 lacc[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
   uint32_t pk[NW];
 #pragma unroll
-  for (int i = 0; i < NW; ++i) {
+  for (int i = 0; i < NP; ++i) {
     const int j = J0 + 2 * i;
-    pk[i] = (j < J1) ? pack_bf16x2(z[2 * i], (j + 1 < J1) ? z[2 * i + 1] : 0.f) : 0u;
+    const float bias = brow[j / WIN - R0];
+    const float2 x = __ffma2_rn(zz[i], make_float2(c, c), make_float2(bias, bias));
+    uint32_t rx, ry;
+    if ((kPoly >> ((j % WIN) / 2)) & 1u) {
+      exp2_poly2(x, rx, ry);
+    } else {
+      rx = __float_as_uint(exp2_mufu(x.x));
+      ry = __float_as_uint(exp2_mufu(x.y));
+    }
+    if constexpr (SUM) lacc[i & 3] = __fadd2_rn(lacc[i & 3], make_float2(__uint_as_float(rx), __uint_as_float(ry)));
+    pk[i] = pack_p(rx, ry);
   }
 #pragma unroll
+  for (int i = NP; i < NW; ++i) pk[i] = 0u;
+#pragma unroll
   for (int i = 0; i < NW; i += 8) tmem_st_x8(ts + J0 / 2 + i, pk + i);
+  const float2 la = __fadd2_rn(lacc[0], lacc[1]), lb = __fadd2_rn(lacc[2], lacc[3]);
   m_out = m;
-  l_out = l;
+  l_out = (la.x + lb.x) + (la.y + lb.y);
+}
+
+// All chunks of the row, in order (each with its own maximum).
+template <int WIN, class C, int... I>
+__device__ __forceinline__ void run_chunks(uint32_t ts, const float (&rw)[WIN], const float (&rh)[WIN], float c,
+                                           float (&mch)[C::NCHUNK], float (&lch)[C::NCHUNK],
+                                           std::integer_sequence<int, I...>) {
+  (softmax_chunk<WIN, 16 * chunk_step<C::KSTEPS, C::NCHUNK>(I),
+                 (I + 1 == C::NCHUNK) ? C::KS : 16 * chunk_step<C::KSTEPS, C::NCHUNK>(I + 1),
+                 16 * chunk_step<C::KSTEPS, C::NCHUNK>(I + 1), !C::SUM_BY_MMA>(ts, rw, rh, c, mch[I], lch[I]),
+   ...);
 }
 
 template <int D, int WIN>
@@ -256,10 +341,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   float* sScratch = reinterpret_cast<float*>(smem);             // 256 x 60 floats
   uint8_t* sStage = smem + (C::SCRATCH + 1023) / 1024 * 1024;   // stages x STAGE_BYTES
-  // stage layout: [Q_a][Q_b][K_a][K_b][V_a][V_b]
+  // stage layout: [Q_a][Q_b][K_a][K_b][V_a][V_b][ones]
   constexpr int OFF_QA = 0, OFF_QB = C::Q_TILE;
   constexpr int OFF_KA = 2 * C::Q_TILE, OFF_KB = OFF_KA + C::K_TILE;
   constexpr int OFF_VA = OFF_KB + C::K_TILE, OFF_VB = OFF_VA + C::V_TILE;
+  constexpr int OFF_ONES = OFF_VB + C::V_TILE;  // d = 16: ones atom of the A.V B operand
 
   __shared__ __align__(8) uint64_t bar_full[8];
   __shared__ __align__(8) uint64_t bar_empty[8];
@@ -317,6 +403,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       uint8_t* vt = st + (hb ? OFF_VB : OFF_VA);
       for (int idx = tid; idx < (C::KP - C::KS) * C::ROWB / 16; idx += kThreads)
         reinterpret_cast<uint4*>(vt + C::KS * C::ROWB)[idx] = make_uint4(0, 0, 0, 0);
+    }
+    if constexpr (C::SUM_BY_MMA) {
+      for (int idx = tid; idx < C::ONES_TILE / 16; idx += kThreads)
+        reinterpret_cast<uint4*>(st + OFF_ONES)[idx] = make_uint4(0x3f803f80u, 0x3f803f80u, 0x3f803f80u, 0x3f803f80u);
     }
   }
   fence_proxy_async_smem();
@@ -448,10 +538,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         rw[kc] = (X >= 0 && X < p.W) ? line[kRelW + kc - qx + WIN - 1] : -INFINITY;
       }
 
-      // ---- the two key chunks: softmax, P into TMEM over the consumed S columns
-      float m1, l1, m2, l2;
-      softmax_chunk<WIN, 0, C::C1, C::C1>(ts, rw, rh, c, m1, l1);
-      softmax_chunk<WIN, C::C1, C::KS, C::KP>(ts, rw, rh, c, m2, l2);
+      // ---- the key chunks: softmax, P into TMEM over the consumed S columns
+      float mch[C::NCHUNK], lch[C::NCHUNK];
+      run_chunks<WIN, C>(ts, rw, rh, c, mch, lch, std::make_integer_sequence<int, C::NCHUNK>{});
       tmem_wait_st();
       tc_fence_before();
       // the whole 128-row P is in TMEM before any A.V MMA reads it; a bounded
@@ -464,17 +553,13 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       tc_fence_after();
 
-      // ---- A.V: this warp's stream of K-steps (P from TMEM, V from shared memory)
+      // ---- A.V: warp w issues chunk w's K-steps (P from TMEM, V from shared memory)
       const int s = k % S;
       if (wq < C::NSTREAM && lane == 0) {
         const uint8_t* st = sStage + s * C::STAGE_BYTES;
         const uint32_t va = smem_addr(st + OFF_VA);
         const uint32_t slot = tmem + g * kSlotCols;
-        constexpr int per_chunk = C::NSTREAM / 2;
-        const int chunk = wq / per_chunk, part = wq % per_chunk;
-        const int c0 = chunk ? C::C1STEPS : 0, c1 = chunk ? C::KSTEPS : C::C1STEPS;
-        const int n = c1 - c0;
-        const int kb = c0 + (n * part) / per_chunk, ke = c0 + (n * (part + 1)) / per_chunk;
+        const int kb = chunk_step<C::KSTEPS, C::NCHUNK>(wq), ke = chunk_step<C::KSTEPS, C::NCHUNK>(wq + 1);
         const uint32_t dst = slot + C::O_BASE + wq * C::O_N;
 #pragma unroll 1
         for (int kk = kb; kk < ke; ++kk)
@@ -492,23 +577,29 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       tc_fence_after();
       {
-        const float mm = fmaxf(m1, m2);
-        const float f1 = exp2_mufu((m1 - mm) * c), f2 = exp2_mufu((m2 - mm) * c);
-        const float inv = 1.0f / (f1 * l1 + f2 * l2);
+        float mm = mch[0];
+#pragma unroll
+        for (int q = 1; q < C::NCHUNK; ++q) mm = fmaxf(mm, mch[q]);
         float o[D];
 #pragma unroll
         for (int e = 0; e < D; ++e) o[e] = 0.f;
+        float l = 0.f;
 #pragma unroll
-        for (int sIdx = 0; sIdx < C::NSTREAM; ++sIdx) {
-          // the whole warp loads both heads' columns (a warp-collective load
-          // must not diverge); this thread's head is [0, D) for a, [D, 2D) for b
-          float t[2 * D];
-          tmem_ld_cols<2 * D>(ts + C::O_BASE + sIdx * C::O_N, t);
+        for (int q = 0; q < C::NCHUNK; ++q) {
+          // the whole warp loads the accumulator's columns (a warp-collective
+          // load must not diverge); this thread's head is [0, D) for a, [D, 2D) for b
+          constexpr int kLd = C::SUM_BY_MMA ? 2 * D + 8 : 2 * D;  // one group of the ones columns
+          float t[kLd];
+          tmem_ld_cols<kLd>(ts + C::O_BASE + q * C::O_N, t);
           tmem_wait_ld();
-          const float f = (sIdx < C::NSTREAM / 2) ? f1 : f2;
+          const float f = exp2_mufu((mch[q] - mm) * c);
 #pragma unroll
           for (int e = 0; e < D; ++e) o[e] = fmaf(f, hb ? t[D + e] : t[e], o[e]);
+          // row sum of the bf16 P (ones columns) or of the fp32 exponentials
+          if constexpr (C::SUM_BY_MMA) l = fmaf(f, t[kLd - 8], l);
+          else l = fmaf(f, lch[q], l);
         }
+        const float inv = 1.0f / l;
         uint32_t pk[D / 2];
 #pragma unroll
         for (int t = 0; t < D / 2; ++t) pk[t] = pack_bf16x2(o[2 * t] * inv, o[2 * t + 1] * inv);

@@ -1,0 +1,551 @@
+// halo_tc3.cuh -- stride-1 bf16 kernel for blocked local self-attention with
+// haloing on sm_100a, for 16x16 query blocks (windows of 16..24 pixels).
+//
+// Operation (HaloNet, "Scaling Local Self-Attention for Parameter Efficient
+// Visual Backbones", sections 2.1-2.2 and appendix A; index conventions of the
+// blog page's RelPosEmb / HaloAttention modules):
+//   z[q, key] = s * q . (k[key] + rel_h[kr - qy + w - 1] + rel_w[kc - qx + w - 1])
+//   out[q]    = sum over in-image window keys of softmax(z) * v[key]
+//
+// A 16x16 block has 256 queries, so one head already fills two 128-row MMA
+// tiles; the window (up to 24 x 24 = 576 keys) is too wide for one TMEM pass.
+//
+// Work item = one 16x16 query block of one head.  Warpgroup g (g = 0, 1)
+// takes query rows [8g, 8g + 8) of the block (128 queries, TMEM lane = query):
+//   * TMA (warp 8): Q [256 x d], K and V [w*w keys x d] of the item into one
+//     pipeline stage; the relative table R = [rel_h; 0; rel_w; 0] (96 rows)
+//     is written to shared memory once at start-up.
+//   * G MMA (warp 9 + g): G = Q_g R^T, M=128, N=96: the query's dot products
+//     with every rel_h and rel_w row, into the S buffer the item's first chunk
+//     will use.  Each thread picks the w + w it needs: the warp-uniform part of
+//     the row shift through the TMEM load address, the per-lane part by
+//     selects (no scratch memory).  The warpgroup gathers item k+1's before
+//     item k's epilogue, so the G MMA hides behind the last A.V.
+//   * S MMA (warp 9 + g): the window in chunks of 4 window rows, S_c = Q_g K_c^T
+//     (N = 4w rounded to 16), alternating between two TMEM buffers across
+//     chunks and items.
+//   * softmax (one thread per query row): per chunk the exact chunk maximum of
+//     c*S + c*rel_w + c*rel_h; the running maximum moves only when the chunk's
+//     exceeds it by more than 8 (in log2 units), and only then is the fp32
+//     accumulator O rescaled (a rare path).  Exponentials part on MUFU, part as
+//     a cubic on the FMA pipe; bf16 P written back over the chunk's S columns.
+//   * A.V (warps 0 and 1 of the warpgroup, each half of the chunk's K-steps
+//     into its own accumulator): O_j += P_c V_c, M=128, N=d, P from TMEM.
+//   * epilogue: (O_0 + O_1) / (row sum), bf16, NHWC store.
+// Every wait is bounded and reports HALO_ERR_TIMEOUT.
+#pragma once
+
+#include <cstdint>
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <type_traits>
+#include <utility>
+
+#include "halo_tc.cuh"
+#include "halo_tc2.cuh"
+#include "sm100.cuh"
+
+namespace halo {
+namespace tc3 {
+
+using namespace sm100;
+using tc::exp2_mufu;
+using tc::pack_bf16x2;
+using tc::record_timeout;
+using tc::swz;
+using tc2::exp2_poly2;
+using tc2::max3f;
+using tc2::mma_f16_ts;
+using tc2::pack_p;
+using tc2::tmem_ld_cols;
+using tc2::tmem_ld_x32;
+using tc2::tmem_ld_x8;
+using tc2::tmem_st_x8;
+using tc2::tmem_wait_st;
+
+constexpr int kBlock = 16;
+constexpr int kThreads = 384;      // warpgroups 0-1 softmax, warp 8 TMA, warps 9-10 MMA
+constexpr int kTmaWarp = 8;
+constexpr int kMmaWarp = 9;        // warp 9 + g issues the G and S MMAs of warpgroup g
+constexpr int kSoftmaxRegs = tc::kSoftmaxRegs;
+constexpr int kProducerRegs = tc::kProducerRegs;
+constexpr uint32_t kTmemCols = 512;
+constexpr uint32_t kSlotCols = 256;  // warpgroup g owns columns [256g, 256g + 256)
+constexpr uint32_t kBufCols = 96;    // S buffers at slot columns [0, 96) and [96, 192)
+constexpr uint32_t kOCol = 192;      // O accumulators (two A.V streams) at [192, 192 + 2d)
+constexpr int kStreams = 2;          // A.V issue streams (warps 0 and 1 of the warpgroup)
+constexpr int kChunkRows = 4;        // window rows per key chunk
+constexpr int kRRows = 96;           // R tile: rel_h rows [0, 2w-1), rel_w rows [48, 48 + 2w-1)
+constexpr int kRelW = 48;
+constexpr float kRescale = 8.0f;     // move the running maximum when exceeded by this (log2 units)
+constexpr uint64_t kWaitNs = tc::kWaitNs;
+
+struct Params {
+  const __nv_bfloat16* rel_h;
+  const __nv_bfloat16* rel_w;
+  __nv_bfloat16* out;
+  int N, H, W, heads, halo;
+  int nbx, nby;
+  int num_items;   // N * nby * nbx * heads
+  int stages;
+  float c;         // log2(e) / sqrt(d)
+};
+
+template <int D, int WIN>
+struct Cfg {
+  static constexpr int ROWB = D * 2;
+  static constexpr int KS = WIN * WIN;
+  static constexpr int NCH = (WIN + kChunkRows - 1) / kChunkRows;
+  __host__ __device__ static constexpr int rows(int c) { return (c + 1 < NCH) ? kChunkRows : WIN - kChunkRows * (NCH - 1); }
+  __host__ __device__ static constexpr int start(int c) { return kChunkRows * WIN * c; }     // first key of chunk c
+  __host__ __device__ static constexpr int keys(int c) { return rows(c) * WIN; }
+  __host__ __device__ static constexpr int ns(int c) { return (keys(c) + 15) / 16 * 16; }    // S MMA N = P keys incl. padding
+  __host__ __device__ static constexpr int nbuf(int b) { return (NCH + 1 - b) / 2; }         // chunks using buffer b per item
+  static constexpr int KPAD = start(NCH - 1) + ns(NCH - 1);              // K / V rows incl. zero padding
+  static constexpr int Q_TILE = 256 * ROWB;
+  static constexpr int K_TILE = (KPAD * ROWB + 1023) / 1024 * 1024;
+  static constexpr int STAGE_BYTES = Q_TILE + 2 * K_TILE;
+  static constexpr int R_TILE = (kRRows * ROWB + 1023) / 1024 * 1024;
+  static constexpr int TX_BYTES = (256 + 2 * KS) * ROWB;
+  static constexpr SmemSwizzle SW = (ROWB == 32) ? SW_32B : (ROWB == 64 ? SW_64B : SW_128B);
+  static constexpr uint32_t SBO = 8 * ROWB;
+  static constexpr int HALO = (WIN - kBlock) / 2;
+  static_assert(D == 16 || D == 32, "dim_head 16 or 32");
+  static_assert(WIN % 2 == 0 && WIN >= kBlock && WIN <= 24, "window 16..24");
+  static_assert(ns(0) <= (int)kBufCols, "S chunk in one buffer");
+  static_assert(kOCol + kStreams * D <= kSlotCols, "O accumulators in the slot");
+  static_assert(ns(NCH - 1) / 16 >= kStreams, "every A.V stream has a K-step in every chunk");
+  static_assert(2 * WIN - 1 <= kRelW, "relative table rows");
+  static_assert((kChunkRows * WIN) % 8 == 0, "chunk starts on a swizzle atom");
+};
+
+template <int D, int WIN>
+__host__ __device__ constexpr int smem_bytes(int stages) {
+  using C = Cfg<D, WIN>;
+  return 1024 + C::R_TILE + stages * C::STAGE_BYTES;
+}
+
+// Window-column pairs (kc, kc+1), kc even, whose exponentials take the
+// polynomial: inside the block's own 16 columns [h, h+16), which are never
+// outside the image.  Bit kc/2 of the mask.
+#ifndef HALO_TC3_POLY_PAIRS
+#define HALO_TC3_POLY_PAIRS 4
+#endif
+template <int WIN>
+__host__ __device__ constexpr unsigned poly_pair_mask() {
+  constexpr int h = (WIN - kBlock) / 2;
+  unsigned m = 0;
+  int picked = 0;
+  const int mid = (h + 7) & ~1;
+  for (int d = 0; d < 16 && picked < HALO_TC3_POLY_PAIRS; ++d) {
+    const int kc = mid + ((d & 1) ? -2 * ((d + 1) / 2) : 2 * (d / 2));
+    if (kc >= h && kc + 1 < h + kBlock && !((m >> (kc / 2)) & 1u)) {
+      m |= 1u << (kc / 2);
+      ++picked;
+    }
+  }
+  return m;
+}
+
+// A wait's outcome, the same for every lane of the warp (a warp-collective
+// tcgen05 instruction must not be reached by part of a warp).
+__device__ __forceinline__ bool warp_ok(bool ok) { return __all_sync(0xffffffffu, ok); }
+
+struct ItemCoord {
+  int n, by, bx, head;
+};
+__device__ __forceinline__ ItemCoord item_coord(int item, int heads, int nbx, int nby) {
+  ItemCoord c;
+  c.head = item % heads;
+  const int blk = item / heads;
+  c.bx = blk % nbx;
+  c.by = (blk / nbx) % nby;
+  c.n = blk / (nbx * nby);
+  return c;
+}
+
+template <int D, int WIN>
+__global__ void __launch_bounds__(kThreads, 1)
+    halo_fwd_tc3(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__ CUtensorMap tmap_k,
+                 const __grid_constant__ CUtensorMap tmap_v, const Params p) {
+  using C = Cfg<D, WIN>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* sR = smem;
+  uint8_t* sStage = smem + C::R_TILE;
+  // stage layout: [Q 256 rows][K KPAD rows][V KPAD rows]
+  constexpr int OFF_Q = 0, OFF_K = C::Q_TILE, OFF_V = C::Q_TILE + C::K_TILE;
+
+  // Per warpgroup g, chunk t = k * NCH + c of its k-th item uses S buffer
+  // t & 1; sfull / bfree of a buffer complete once per chunk on it, so the
+  // phase of chunk t is t >> 1.
+  __shared__ __align__(8) uint64_t bar_full[4];
+  __shared__ __align__(8) uint64_t bar_empty[4];     // count 4: both streams of both warpgroups, last chunk
+  __shared__ __align__(8) uint64_t bar_gfull[2];     // G MMA done
+  __shared__ __align__(8) uint64_t bar_gfree[2];     // count 4: the warpgroup loaded G
+  __shared__ __align__(8) uint64_t bar_sfull[2][2];  // S of the chunk in buffer b done
+  __shared__ __align__(8) uint64_t bar_bfree[2][2];  // count 2: both streams' A.V of that chunk done
+  __shared__ __align__(8) uint64_t bar_pready[2];    // count 4: P of the chunk stored
+  __shared__ __align__(8) uint64_t bar_ofull[2];     // count 2: last chunk's A.V done
+  __shared__ __align__(8) uint64_t bar_done[2];
+  __shared__ __align__(8) uint64_t bar_pvdone[8];
+  __shared__ uint32_t tmem_base_sh;
+  __shared__ int abort_flag;
+
+  const int tid = threadIdx.x;
+  const int warp = tid >> 5;
+  const int lane = tid & 31;
+  const int S = p.stages;
+
+  // ---------------------------------------------------------------- set-up
+  if (tid == 0) {
+    for (int i = 0; i < S; ++i) {
+      mbar_init(&bar_full[i], 1);
+      mbar_init(&bar_empty[i], 2 * kStreams);
+    }
+    for (int g = 0; g < 2; ++g) {
+      mbar_init(&bar_gfull[g], 1);
+      mbar_init(&bar_gfree[g], 4);
+      mbar_init(&bar_sfull[g][0], 1);
+      mbar_init(&bar_sfull[g][1], 1);
+      mbar_init(&bar_bfree[g][0], kStreams);
+      mbar_init(&bar_bfree[g][1], kStreams);
+      mbar_init(&bar_pready[g], 4);
+      mbar_init(&bar_ofull[g], kStreams);
+      mbar_init(&bar_done[g], 1);
+    }
+    for (int w = 0; w < 8; ++w) mbar_init(&bar_pvdone[w], 1);
+    abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == kTmaWarp && lane == 0) {
+    prefetch_tensormap(&tmap_q);
+    prefetch_tensormap(&tmap_k);
+    prefetch_tensormap(&tmap_v);
+  }
+  // R tile (written once) and the K / V padding rows the TMA never writes
+  for (int idx = tid; idx < kRRows * (D / 8); idx += kThreads) {
+    const int r = idx / (D / 8), u = idx % (D / 8);
+    uint4 val = make_uint4(0, 0, 0, 0);
+    if (r < 2 * WIN - 1) val = *reinterpret_cast<const uint4*>(p.rel_h + r * D + u * 8);
+    else if (r >= kRelW && r < kRelW + 2 * WIN - 1)
+      val = *reinterpret_cast<const uint4*>(p.rel_w + (r - kRelW) * D + u * 8);
+    *reinterpret_cast<uint4*>(sR + swz<C::ROWB>(r, u)) = val;
+  }
+  for (int s = 0; s < S; ++s) {
+    uint8_t* st = sStage + s * C::STAGE_BYTES;
+    for (int idx = tid; idx < (C::KPAD - C::KS) * C::ROWB / 16; idx += kThreads) {
+      reinterpret_cast<uint4*>(st + OFF_K + C::KS * C::ROWB)[idx] = make_uint4(0, 0, 0, 0);
+      reinterpret_cast<uint4*>(st + OFF_V + C::KS * C::ROWB)[idx] = make_uint4(0, 0, 0, 0);
+    }
+  }
+  fence_proxy_async_smem();
+  if (warp == 0) {
+    tmem_alloc(&tmem_base_sh, kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = tmem_base_sh;
+  const int my_items = (p.num_items > (int)blockIdx.x)
+                           ? (p.num_items - 1 - (int)blockIdx.x) / (int)gridDim.x + 1 : 0;
+
+  if (warp >= 8) {
+  asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kProducerRegs));
+  if (warp == kTmaWarp) {
+    // ------------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      int issued = 0;
+      for (int k = 0; k < my_items; ++k) {
+        const int s = k % S;
+        if (k >= S && !mbar_wait(&bar_empty[s], ((k / S) - 1) & 1, kWaitNs, &abort_flag)) {
+          if (!abort_flag) record_timeout(&abort_flag);
+          break;
+        }
+        const ItemCoord ic = item_coord(blockIdx.x + k * gridDim.x, p.heads, p.nbx, p.nby);
+        uint8_t* st = sStage + s * C::STAGE_BYTES;
+        const int x0 = ic.bx * kBlock, y0 = ic.by * kBlock;
+        mbar_arrive_expect_tx(&bar_full[s], C::TX_BYTES);
+        tma_load_4d(st + OFF_Q, &tmap_q, &bar_full[s], ic.head * D, x0, y0, ic.n);
+        tma_load_4d(st + OFF_K, &tmap_k, &bar_full[s], ic.head * D, x0 - p.halo, y0 - p.halo, ic.n);
+        tma_load_4d(st + OFF_V, &tmap_v, &bar_full[s], ic.head * D, x0 - p.halo, y0 - p.halo, ic.n);
+        issued = k + 1;
+      }
+      if (abort_flag) {
+        for (int k = (issued > S ? issued - S : 0); k < issued; ++k)
+          mbar_wait(&bar_full[k % S], (k / S) & 1, kWaitNs);
+      }
+    }
+  } else if (warp == kMmaWarp || warp == kMmaWarp + 1) {
+    // ------------------------------------------------------------ G and S MMAs of warpgroup g
+    const int g = warp - kMmaWarp;
+    if (lane == 0) {
+      const uint32_t slot = tmem + g * kSlotCols;
+      const uint32_t idG = idesc_bf16_f32(128, kRRows, false);
+      const uint32_t ra = smem_addr(sR);
+      bool ok = true;
+      for (int k = 0; k < my_items && ok; ++k) {
+        const int s = k % S, t0 = k * C::NCH;
+        ok = mbar_wait(&bar_full[s], (k / S) & 1, kWaitNs, &abort_flag);
+        // G into the buffer of the item's first chunk, free once chunk t0 - 2's A.V is done
+        if (ok && t0 >= 2) ok = mbar_wait(&bar_bfree[g][t0 & 1], ((t0 - 2) >> 1) & 1, kWaitNs, &abort_flag);
+        if (!ok) break;
+        tc_fence_after();
+        const uint8_t* st = sStage + s * C::STAGE_BYTES;
+        const uint32_t qa = smem_addr(st + OFF_Q + g * 128 * C::ROWB);
+        const uint32_t ka = smem_addr(st + OFF_K);
+#pragma unroll
+        for (int ks = 0; ks < D / 16; ++ks)
+          mma_f16_ss(slot + (t0 & 1) * kBufCols, smem_desc(qa + 32 * ks, 16, C::SBO, C::SW),
+                     smem_desc(ra + 32 * ks, 16, C::SBO, C::SW), idG, ks != 0);
+        mma_commit(&bar_gfull[g]);
+#pragma unroll 1
+        for (int c = 0; c < C::NCH; ++c) {
+          const int t = t0 + c, b = t & 1;
+          if (c == 0) ok = mbar_wait(&bar_gfree[g], k & 1, kWaitNs, &abort_flag);
+          else if (t >= 2) ok = mbar_wait(&bar_bfree[g][b], ((t - 2) >> 1) & 1, kWaitNs, &abort_flag);
+          if (!ok) break;
+          tc_fence_after();
+          const int n = (c + 1 < C::NCH) ? C::ns(0) : C::ns(C::NCH - 1);
+          const uint32_t idS = idesc_bf16_f32(128, n, false);
+          const uint32_t kb = ka + C::start(c) * C::ROWB;
+#pragma unroll
+          for (int ks = 0; ks < D / 16; ++ks)
+            mma_f16_ss(slot + b * kBufCols, smem_desc(qa + 32 * ks, 16, C::SBO, C::SW),
+                       smem_desc(kb + 32 * ks, 16, C::SBO, C::SW), idS, ks != 0);
+          mma_commit(&bar_sfull[g][b]);
+        }
+      }
+      if (!ok && !abort_flag) record_timeout(&abort_flag);
+      mma_commit(&bar_done[g]);
+      mbar_wait(&bar_done[g], 0, kWaitNs);
+    }
+  }
+  __syncwarp();
+  tc_fence_before();
+  named_bar_sync(1, kThreads);
+  return;
+  }
+
+  asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kSoftmaxRegs));
+  {
+    // ------------------------------------------------------------ softmax warpgroups
+    const int g = warp >> 2;               // warpgroup = TMEM slot = query rows [8g, 8g + 8)
+    const int wq = warp & 3;               // lane quadrant
+    const int yl = 8 * g + 2 * wq + (lane >> 4);  // query row in the block
+    const int xl = lane & 15;                      // query column in the block
+    const uint32_t slot = tmem + g * kSlotCols;    // lane 0 of the slot (MMA operands)
+    const uint32_t ts = slot + (static_cast<uint32_t>(32 * wq) << 16);  // this warp's lanes
+    const float c = p.c;
+    const int C_all = p.heads * D;
+    const uint32_t idO = idesc_bf16_f32(128, D, true);
+    constexpr unsigned kPoly = poly_pair_mask<WIN>();
+
+    float rhc[WIN], rwc[WIN];
+    // ---- relative logits of item k: rhc[kr] = c * q.rel_h[kr - qy + w - 1], rwc[kc] likewise
+    auto gather = [&](int k) -> bool {
+      if (!warp_ok(mbar_wait(&bar_gfull[g], k & 1, kWaitNs, &abort_flag))) return false;
+      tc_fence_after();
+      const ItemCoord ic = item_coord(blockIdx.x + k * gridDim.x, p.heads, p.nbx, p.nby);
+      const int y0 = ic.by * kBlock - p.halo, x0 = ic.bx * kBlock - p.halo;
+      const uint32_t gcol = ((k * C::NCH) & 1) * kBufCols;
+      // rel_h: columns [base, base + 32) of G hold every row this warp needs;
+      // the two query rows of the warp differ by one column
+      const int base = WIN - 2 - 8 * g - 2 * wq;
+      float gh[32], gw[48];
+      tmem_ld_x32(ts + gcol + base, gh);
+      tmem_ld_x32(ts + gcol + kRelW, gw);
+      tmem_ld_x8(ts + gcol + kRelW + 32, gw + 32);
+      tmem_ld_x8(ts + gcol + kRelW + 40, gw + 40);
+      tmem_wait_ld();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bar_gfree[g]);
+      const bool odd = (lane >> 4) != 0;
+#pragma unroll
+      for (int kr = 0; kr < WIN; ++kr) {
+        const int Y = y0 + kr;
+        const float v = odd ? gh[kr] : gh[kr + 1];
+        rhc[kr] = (Y >= 0 && Y < p.H) ? v * c : -INFINITY;
+      }
+      // rel_w: the 16 query columns need 16 different shifts; a four-stage
+      // barrel shifter of selects over gw[w - 16 + i] by sh = 15 - qx
+      float a[WIN + 15];
+#pragma unroll
+      for (int i = 0; i < WIN + 15; ++i) a[i] = gw[WIN - 16 + i];
+      const int sh = 15 - xl;
+#pragma unroll
+      for (int i = 0; i < WIN + 7; ++i) a[i] = (sh & 8) ? a[i + 8] : a[i];
+#pragma unroll
+      for (int i = 0; i < WIN + 3; ++i) a[i] = (sh & 4) ? a[i + 4] : a[i];
+#pragma unroll
+      for (int i = 0; i < WIN + 1; ++i) a[i] = (sh & 2) ? a[i + 2] : a[i];
+#pragma unroll
+      for (int i = 0; i < WIN; ++i) a[i] = (sh & 1) ? a[i + 1] : a[i];
+#pragma unroll
+      for (int kc = 0; kc < WIN; ++kc) {
+        const int X = x0 + kc;
+        rwc[kc] = (X >= 0 && X < p.W) ? a[kc] * c : -INFINITY;
+      }
+      return true;
+    };
+
+    // ---- one key chunk (NR window rows; rhc[0..NR) are its rows' rel_h logits)
+    float m_run = -INFINITY, l = 0.f;
+    auto chunk = [&](auto nr, int k, int cidx) -> bool {
+      constexpr int NR = decltype(nr)::value;
+      constexpr int NK = NR * WIN, NL = (NK + 7) / 8 * 8, NP = NK / 2, NW = (NK + 15) / 16 * 8;
+      const int t = k * C::NCH + cidx, b = t & 1;
+      const uint32_t buf = ts + b * kBufCols;
+      if (!warp_ok(mbar_wait(&bar_sfull[g][b], (t >> 1) & 1, kWaitNs, &abort_flag))) return false;
+      tc_fence_after();
+      float z[NL];
+      tmem_ld_cols<NL>(buf, z);
+      tmem_wait_ld();
+      // y = c*S + c*rel_w (pairs); chunk maximum of y + c*rel_h
+      float2 y[NP];
+#pragma unroll
+      for (int i = 0; i < NP; ++i) {
+        const int kc = (2 * i) % WIN;
+        y[i] = __ffma2_rn(make_float2(z[2 * i], z[2 * i + 1]), make_float2(c, c), make_float2(rwc[kc], rwc[kc + 1]));
+      }
+      float mc = -INFINITY;
+#pragma unroll
+      for (int r = 0; r < NR; ++r) {
+        float mr = -INFINITY;
+#pragma unroll
+        for (int i = r * WIN / 2; i < (r + 1) * WIN / 2; ++i) mr = max3f(mr, y[i].x, y[i].y);
+        mc = fmaxf(mc, mr + rhc[r]);
+      }
+      const bool upd = mc > m_run + kRescale;
+      // O holds earlier chunks against m_run: rescale it when the maximum moves
+      // (a row whose earlier chunks had no in-image key has O = 0 and l = 0)
+      if (__any_sync(0xffffffffu, upd && m_run != -INFINITY && cidx > 0)) {
+        const int tp = t - 1;
+        if (!warp_ok(mbar_wait(&bar_bfree[g][tp & 1], (tp >> 1) & 1, kWaitNs, &abort_flag))) return false;
+        tc_fence_after();
+        const float alpha = (upd && m_run != -INFINITY) ? exp2_mufu(m_run - mc) : 1.0f;
+        // eight columns at a time: y[] is live, registers are short
+#pragma unroll 1
+        for (int e = 0; e < kStreams * D; e += 8) {
+          float o[8];
+          tmem_ld_x8(ts + kOCol + e, o);
+          tmem_wait_ld();
+          uint32_t ob[8];
+#pragma unroll
+          for (int i = 0; i < 8; ++i) ob[i] = __float_as_uint(o[i] * alpha);
+          tmem_st_x8(ts + kOCol + e, ob);
+        }
+        l *= alpha;
+      }
+      if (upd) m_run = mc;
+      const float mb = (m_run == -INFINITY ? 0.f : m_run);
+      // exponentials, row sum, packed bf16 P over the chunk's S columns
+      float2 lacc[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f),
+                        make_float2(0.f, 0.f)};
+      uint32_t pk[NW];
+#pragma unroll
+      for (int i = 0; i < NP; ++i) {
+        const int r = (2 * i) / WIN, kc = (2 * i) % WIN;
+        const float bias = rhc[r] - mb;
+        const float2 x = __fadd2_rn(y[i], make_float2(bias, bias));
+        uint32_t rx, ry;
+        if ((kPoly >> (kc / 2)) & 1u) {
+          exp2_poly2(x, rx, ry);
+        } else {
+          rx = __float_as_uint(exp2_mufu(x.x));
+          ry = __float_as_uint(exp2_mufu(x.y));
+        }
+        lacc[i & 3] = __fadd2_rn(lacc[i & 3], make_float2(__uint_as_float(rx), __uint_as_float(ry)));
+        pk[i] = pack_p(rx, ry);
+      }
+#pragma unroll
+      for (int i = NP; i < NW; ++i) pk[i] = 0u;
+#pragma unroll
+      for (int i = 0; i < NW; i += 8) tmem_st_x8(buf + i, pk + i);
+      const float2 la = __fadd2_rn(lacc[0], lacc[1]), lb = __fadd2_rn(lacc[2], lacc[3]);
+      l += (la.x + lb.x) + (la.y + lb.y);
+      tmem_wait_st();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bar_pready[g]);
+      // ---- A.V of the chunk: warps 0 and 1 each issue half of its K-steps
+      bool issued = true;
+      if (wq < kStreams && lane == 0) {
+        issued = mbar_wait(&bar_pready[g], t & 1, kWaitNs, &abort_flag);
+        if (issued) {
+          tc_fence_after();
+          constexpr int KSTEPS = NW / 8, HALF = (KSTEPS + 1) / 2;
+          const int kb = wq ? HALF : 0, ke = wq ? KSTEPS : HALF;
+          const uint32_t va = smem_addr(sStage + (k % S) * C::STAGE_BYTES + OFF_V + C::start(cidx) * C::ROWB);
+#pragma unroll 1
+          for (int kk = kb; kk < ke; ++kk)
+            mma_f16_ts(slot + kOCol + wq * D, slot + b * kBufCols + 8 * kk,
+                       smem_desc(va + kk * 16 * C::ROWB, C::K_TILE, C::SBO, C::SW), idO, (cidx > 0 || kk > kb));
+          mma_commit(&bar_bfree[g][b]);
+          if (cidx + 1 == C::NCH) {
+            mma_commit(&bar_ofull[g]);
+            mma_commit(&bar_empty[k % S]);
+          }
+        }
+      }
+      // next chunk's rows first
+#pragma unroll
+      for (int i = 0; i + NR < WIN; ++i) rhc[i] = rhc[i + NR];
+      return warp_ok(issued);
+    };
+
+    constexpr int kLastRows = C::rows(C::NCH - 1);
+    constexpr int kLoopChunks = (kLastRows == kChunkRows) ? C::NCH : C::NCH - 1;
+    bool ok = my_items > 0 ? gather(0) : true;
+    for (int k = 0; k < my_items && ok; ++k) {
+      const ItemCoord ic = item_coord(blockIdx.x + k * gridDim.x, p.heads, p.nbx, p.nby);
+      m_run = -INFINITY;
+      l = 0.f;
+#pragma unroll 1
+      for (int ci = 0; ci < kLoopChunks && ok; ++ci) ok = chunk(std::integral_constant<int, kChunkRows>{}, k, ci);
+      if constexpr (kLoopChunks < C::NCH) {
+        if (ok) ok = chunk(std::integral_constant<int, kLastRows>{}, k, C::NCH - 1);
+      }
+      // the next item's relative logits while this item's last A.V runs
+      if (ok && k + 1 < my_items) ok = gather(k + 1);
+      // ---- epilogue: (O_0 + O_1) / l, bf16, NHWC
+      if (ok) ok = warp_ok(mbar_wait(&bar_ofull[g], k & 1, kWaitNs, &abort_flag));
+      if (!ok) break;
+      tc_fence_after();
+      {
+        float o[kStreams * D];
+        tmem_ld_cols<kStreams * D>(ts + kOCol, o);
+        tmem_wait_ld();
+        const float inv = 1.0f / l;
+        uint32_t pk[D / 2];
+#pragma unroll
+        for (int t = 0; t < D / 2; ++t)
+          pk[t] = pack_bf16x2((o[2 * t] + o[D + 2 * t]) * inv, (o[2 * t + 1] + o[D + 2 * t + 1]) * inv);
+        const int y = ic.by * kBlock + yl, x = ic.bx * kBlock + xl;
+        __nv_bfloat16* dst = p.out + ((static_cast<size_t>(ic.n) * p.H + y) * p.W + x) * C_all + ic.head * D;
+#pragma unroll
+        for (int t = 0; t < D / 8; ++t)
+          reinterpret_cast<uint4*>(dst)[t] = make_uint4(pk[4 * t], pk[4 * t + 1], pk[4 * t + 2], pk[4 * t + 3]);
+      }
+      tc_fence_before();
+    }
+    if (!ok && !abort_flag) record_timeout(&abort_flag);
+    // A.V MMAs this warp issued are complete before TMEM is released
+    if (wq < kStreams && lane == 0) {
+      mma_commit(&bar_pvdone[warp]);
+      mbar_wait(&bar_pvdone[warp], 0, kWaitNs);
+    }
+    __syncwarp();
+  }
+
+  // ---------------------------------------------------------------- teardown
+  tc_fence_before();
+  named_bar_sync(1, kThreads);
+  tc_fence_after();
+  if (warp == 0) tmem_dealloc(tmem, kTmemCols);
+}
+
+}  // namespace tc3
+}  // namespace halo

@@ -108,6 +108,14 @@ int halo_attn_host(const void* q_h, const void* k_h, const void* v_h, const void
  * or HALO_KERNEL_NONE when the shape is rejected.  No device work. */
 int halo_kernel_for(int N, int H, int W, int heads, int dim_head, int block, int halo, int stride, int dtype);
 
+/* Name of the kernel instantiation halo_attn would launch for these arguments,
+ * e.g. "halo_fwd_tc2<16,14>" (template arguments: dim_head, window, and for
+ * halo_fwd_tc the stride), or "none" when the shape is rejected.  The string
+ * lives in thread-local storage of the library and stays valid until the next
+ * halo_kernel_name call on the same thread; never NULL.  No device work. */
+const char* halo_kernel_name(int N, int H, int W, int heads, int dim_head, int block, int halo, int stride,
+                             int dtype);
+
 /* Static description of a status code; never NULL. */
 const char* halo_strerror(int code);
 

@@ -24,7 +24,8 @@ def _lib():
 
 def test_header_declares_the_boundary():
     names = _declared_functions()
-    for expected in ("halo_attn", "halo_attn_host", "halo_kernel_for", "halo_strerror", "halo_get_last_error",
+    for expected in ("halo_attn", "halo_attn_host", "halo_kernel_for", "halo_kernel_name", "halo_strerror",
+                     "halo_get_last_error",
                      "halo_debug_wait_timeout", "halo_version"):
         assert expected in names
 
@@ -96,6 +97,20 @@ def test_kernel_selection_is_host_only():
     # float32 goes to the CUDA-core kernel, invalid shapes to none
     assert lib.halo_kernel_for(1, 16, 16, 2, 32, 4, 1, 1, 0) == 1
     assert lib.halo_kernel_for(1, 16, 16, 2, 32, 5, 1, 1, 0) == 0
+    # 16x16 blocks with a 4-pixel halo go to the block-16 tensor-core kernel
+    assert lib.halo_kernel_for(16, 128, 128, 8, 32, 16, 4, 1, 1) == 2
+
+
+def test_kernel_names():
+    lib = _lib()
+    name = lambda *a: lib.halo_kernel_name(*a).decode()
+    assert name(32, 64, 64, 8, 16, 8, 3, 1, 1) == "halo_fwd_tc2<16,14>"
+    assert name(64, 32, 32, 8, 64, 8, 3, 1, 1) == "halo_fwd_tc<64,14,1>"
+    assert name(64, 64, 64, 8, 32, 8, 3, 2, 1) == "halo_fwd_tc<32,14,2>"
+    assert name(16, 128, 128, 8, 32, 16, 4, 1, 1) == "halo_fwd_tc3<32,24>"
+    assert name(1, 16, 16, 2, 32, 4, 1, 1, 0) == "halo_fwd_simt<float,32>"
+    assert name(2, 32, 32, 4, 40, 16, 4, 1, 1) == "halo_fwd_simt<bf16,64>"
+    assert name(1, 16, 16, 2, 32, 5, 1, 1, 0) == "none"
 
 
 def test_host_entry_checks_before_any_copy():

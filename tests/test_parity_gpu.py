@@ -86,7 +86,8 @@ def test_full_size_sampled(name):
 
 
 @pytest.mark.parametrize("name,kernel", [("stage1_bf16", "tc_bf16"), ("deep_bf16", "tc_bf16"),
-                                         ("stride2_bf16", "tc_bf16"), ("tiny_f32", "simt_f32")])
+                                         ("stride2_bf16", "tc_bf16"), ("large_bf16", "tc_bf16"),
+                                         ("tiny_f32", "simt_f32")])
 def test_kernel_selection(name, kernel):
     h = _lib()
     wl = WORKLOADS[name]
@@ -104,7 +105,13 @@ for d in (16, 32, 64):
         for stride in (1, 2):
             CASES.append(dict(N=2, H=24, W=40, heads=8 if d < 64 else 4, dim_head=d, block=8, halo=halo,
                               stride=stride))
+# 16x16 query blocks (windows 16..24): every window of the block-16 kernel, both head sizes
+for d in (16, 32):
+    for halo in (0, 1, 2, 3, 4):
+        CASES.append(dict(N=2, H=32, W=48, heads=3, dim_head=d, block=16, halo=halo, stride=1))
 CASES += [
+    dict(N=1, H=16, W=16, heads=2, dim_head=32, block=16, halo=4, stride=1),  # block = map, halo all outside
+    dict(N=3, H=16, W=80, heads=1, dim_head=16, block=16, halo=4, stride=1),  # one block row, one head
     dict(N=1, H=8, W=8, heads=8, dim_head=16, block=8, halo=0, stride=1),    # global attention
     dict(N=1, H=8, W=8, heads=2, dim_head=32, block=8, halo=3, stride=1),    # block = map, halo all outside
     dict(N=3, H=16, W=8, heads=4, dim_head=64, block=8, halo=0, stride=2),   # isolated blocks, stride 2
@@ -130,7 +137,7 @@ SIMT_CASES = [
     dict(N=1, H=16, W=16, heads=2, dim_head=40, block=4, halo=1, stride=2, dtype="f32"),
     dict(N=1, H=9, W=9, heads=1, dim_head=16, block=3, halo=1, stride=1, dtype="f32"),
     dict(N=1, H=32, W=32, heads=2, dim_head=128, block=16, halo=2, stride=1, dtype="f32"),
-    dict(N=2, H=32, W=32, heads=4, dim_head=32, block=16, halo=4, stride=1, dtype="bf16"),
+    dict(N=2, H=32, W=32, heads=4, dim_head=40, block=16, halo=4, stride=1, dtype="bf16"),
     dict(N=1, H=16, W=16, heads=1, dim_head=16, block=8, halo=3, stride=2, dtype="bf16"),
     dict(N=2, H=24, W=16, heads=4, dim_head=16, block=8, halo=4, stride=1, dtype="bf16"),
 ]
@@ -161,6 +168,23 @@ def test_saturated_softmax_and_constant_values():
     vc = torch.full_like(v, 0.75)
     got = _run(wl, (q, k, vc, rh, rw))
     assert torch.all(got == 0.75)
+
+
+@pytest.mark.parametrize("scale", [2.0, 4.0, 8.0])
+def test_block16_running_maximum(scale):
+    """Scaled q and k make later key chunks exceed earlier maxima by a wide
+    margin, which exercises the block-16 kernel's rescaling of the
+    accumulator; the scale-2 case moves the maximum only sometimes."""
+    wl = custom("sat16", N=2, H=32, W=32, heads=2, dim_head=32, block=16, halo=4, stride=1, dtype="bf16")
+    q, k, v, rh, rw = make_inputs(wl, seed=13)
+    qs, ks = (q.float() * scale).to(torch.bfloat16), (k.float() * scale).to(torch.bfloat16)
+    # A peaked softmax passes single values of v through: v is halved so that
+    # |out| stays below ~2.5, where rounding the output to bf16 costs at most
+    # 0.0078 of the 2e-2 budget (above 4 it alone would cost 0.0156).
+    v = (v.float() * 0.5).to(torch.bfloat16)
+    got = _run(wl, (qs, ks, v, rh, rw))
+    want = oracle.halo_attention(qs, ks, v, rh, rw, block=16, halo=4)
+    _compare(got, want, TOL["bf16"], f"block16 scale {scale}")
 
 
 def test_deterministic():
