@@ -185,7 +185,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   __shared__ __align__(8) uint64_t bar_gfree[2];     // count 4: the warpgroup loaded G
   __shared__ __align__(8) uint64_t bar_sfull[2][2];  // S of the chunk in buffer b done
   __shared__ __align__(8) uint64_t bar_bfree[2][2];  // count 2: both streams' A.V of that chunk done
-  __shared__ __align__(8) uint64_t bar_pready[2];    // count 4: P of the chunk stored
+  // count 4: P of chunk t stored, alternating by t & 1: a warp can be one
+  // chunk ahead of another (its arrival for chunk t+1 must not complete the
+  // phase of chunk t), never two (chunk t+2's S needs chunk t's A.V)
+  __shared__ __align__(8) uint64_t bar_pready[2][2];
   __shared__ __align__(8) uint64_t bar_ofull[2];     // count 2: last chunk's A.V done
   __shared__ __align__(8) uint64_t bar_done[2];
   __shared__ __align__(8) uint64_t bar_pvdone[8];
@@ -210,7 +213,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&bar_sfull[g][1], 1);
       mbar_init(&bar_bfree[g][0], kStreams);
       mbar_init(&bar_bfree[g][1], kStreams);
-      mbar_init(&bar_pready[g], 4);
+      mbar_init(&bar_pready[g][0], 4);
+      mbar_init(&bar_pready[g][1], 4);
       mbar_init(&bar_ofull[g], kStreams);
       mbar_init(&bar_done[g], 1);
     }
@@ -469,11 +473,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       tmem_wait_st();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&bar_pready[g]);
+      if (lane == 0) mbar_arrive(&bar_pready[g][b]);
       // ---- A.V of the chunk: warps 0 and 1 each issue half of its K-steps
       bool issued = true;
       if (wq < kStreams && lane == 0) {
-        issued = mbar_wait(&bar_pready[g], t & 1, kWaitNs, &abort_flag);
+        issued = mbar_wait(&bar_pready[g][b], (t >> 1) & 1, kWaitNs, &abort_flag);
         if (issued) {
           tc_fence_after();
           constexpr int KSTEPS = NW / 8, HALF = (KSTEPS + 1) / 2;
