@@ -110,11 +110,17 @@ struct Cfg {
   static constexpr SmemSwizzle SW = (ROWB == 32) ? SW_32B : (ROWB == 64 ? SW_64B : SW_128B);
   static constexpr uint32_t SBO = 8 * ROWB;               // 8-row core-matrix group stride
   static constexpr int NROW = WIN / 2;                    // window rows per thread
+  // A.V issue streams: warp q < NST of the warpgroup issues a share of the
+  // PARTS x WIN K-steps (part q / SPP, window rows of slice q % SPP) into its
+  // own accumulator O_q at slot column q * O_COLS.
+  static constexpr int NST = (O_COLS * 4 <= (int)kTmemG) ? 4 : 3;
+  static constexpr int SPP = NST / PARTS;                 // streams per part
+  static_assert(NST % PARTS == 0 && SPP >= 1, "streams per part");
+  static_assert(NST * O_COLS <= (int)kTmemG, "O accumulators below the G columns");
   static_assert(WIN % 2 == 0 && WIN <= 14 && WIN >= 8, "window must be even, 8..14");
   static_assert(D == 16 || D == 32 || D == 64, "dim_head must be 16, 32 or 64");
   static_assert(NS <= (int)kTmemG, "S must fit below G in a TMEM slot");
   static_assert(2 * WIN - 1 <= kGRelW, "relative table rows");
-  static_assert(PARTS * O_COLS <= (int)kTmemG, "O region below the G columns");
 };
 
 // Bytes of dynamic shared memory for a given stage count (plus 1 KB alignment slack).
@@ -216,12 +222,12 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (tid == 0) {
     for (int i = 0; i < S; ++i) {
       mbar_init(&bar_full[i], 1);
-      mbar_init(&bar_empty[i], 1);
+      mbar_init(&bar_empty[i], C::NST);
     }
     for (int b = 0; b < 4; ++b) {
       mbar_init(&bar_sfull[b], 1);
       mbar_init(&bar_pfull[b], 4);
-      mbar_init(&bar_ofull[b], 1);
+      mbar_init(&bar_ofull[b], C::NST);
       mbar_init(&bar_tfree[b], 4);
     }
     mbar_init(&bar_done, 1);
@@ -323,7 +329,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (lane == 0) {
       const uint32_t idS = idesc_bf16_f32(64, C::NS, false);
       const uint32_t idG = idesc_bf16_f32(64, kGCols, false);
-      const uint32_t idO = idesc_bf16_f32(64, C::O_COLS, true);
       // S(k): QK^T and the relative dot products of item k into its TMEM slot.
       auto issue_s = [&](int k) {
         const int s = k % S, g = k & 1, sl = (k >> 1) & 1;
@@ -349,58 +354,17 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         mma_commit(&bar_sfull[2 * g + sl]);
       };
-      // O(k): P V of item k once its warpgroup has written P; frees stage k.
-      auto issue_o = [&](int k) {
-        const int s = k % S, g = k & 1, sl = (k >> 1) & 1;
-        const uint32_t dst = tmem + (static_cast<uint32_t>(g * 16) << 16) + sl * kSlotCols;
-        const uint8_t* st = sStage + s * C::STAGE_BYTES;
-        const uint32_t pa = smem_addr(sP + g * C::P_TILE);
-#pragma unroll 1
-        for (int part = 0; part < C::PARTS; ++part) {
-          const uint32_t va = smem_addr(st + C::Q_BYTES + C::PARTS * C::K_TILE + part * C::V_TILE);
-          // with the ones tile the B operand spans two swizzle atoms along N:
-          // V (D columns) then ones (D columns) at leading byte offset LBO
-          const uint32_t lbo = C::SUM_BY_MMA ? (smem_addr(sOnes) - va) : 16u;
-#pragma unroll 1
-          for (int kk = 0; kk < WIN; ++kk) {
-            mma_f16_ss(dst + part * C::O_COLS, smem_desc(pa + kk * 2048, 16, 256, SW_32B),
-                       smem_desc(va + kk * kRowKeys * C::ROWB, lbo, C::SBO, C::SW), idO, kk != 0);
-          }
+      // S(k) needs its stage loaded and the slot's previous item (k - 4)
+      // consumed (the A.V MMAs are issued by the softmax warpgroups)
+      for (int ns = 0; ns < my_items; ++ns) {
+        if (!mbar_wait(&bar_full[ns % S], (ns / S) & 1, kWaitNs, &abort_flag) ||
+            (ns >= 4 && !mbar_wait(&bar_tfree[2 * (ns & 1) + ((ns >> 1) & 1)], ((ns >> 2) - 1) & 1, kWaitNs,
+                                   &abort_flag))) {
+          if (!abort_flag) record_timeout(&abort_flag);
+          break;
         }
-        mma_commit(&bar_ofull[2 * g + sl]);
-        mma_commit(&bar_empty[s]);
-      };
-      // Issue whichever step is ready (O first: it releases a waiting
-      // warpgroup).  S(k) needs its stage loaded and the slot's previous
-      // item (k - 4) consumed; O(k) needs P(k).
-      int ns = 0, no = 0;
-      uint64_t idle_since = global_timer_ns();
-      uint32_t polls = 0;
-      while (no < my_items) {
-        bool did = false;
-        if (no < ns && mbar_test(&bar_pfull[2 * (no & 1) + ((no >> 1) & 1)], (no >> 2) & 1)) {
-          tc_fence_after();
-          issue_o(no);
-          ++no;
-          did = true;
-        } else if (ns < my_items && mbar_test(&bar_full[ns % S], (ns / S) & 1) &&
-                   (ns < 4 || mbar_test(&bar_tfree[2 * (ns & 1) + ((ns >> 1) & 1)], ((ns >> 2) - 1) & 1))) {
-          tc_fence_after();
-          issue_s(ns);
-          ++ns;
-          did = true;
-        }
-        if (did) {
-          polls = 0;
-          idle_since = global_timer_ns();
-        } else if ((++polls & 15u) == 0) {
-          __nanosleep(200);  // back off instead of spinning on the issue slots
-          if (*(volatile int*)&abort_flag) break;
-          if (global_timer_ns() - idle_since > kWaitNs) {
-            record_timeout(&abort_flag);
-            break;
-          }
-        }
+        tc_fence_after();
+        issue_s(ns);
       }
       // all issued MMAs complete before the CTA frees TMEM
       mma_commit(&bar_done);
@@ -430,6 +394,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int qx = (STRIDE == 1) ? (row & 7) : 2 * (r16 & 3);
     const float c = p.c;
     const int C_all = p.heads * D;
+    const uint32_t idO = idesc_bf16_f32(64, C::O_COLS, true);
 
     // Epilogue of a finished item: O (and row sums) from its TMEM slot,
     // normalise, bf16, store; then hand the slot back to the MMA warp.
@@ -442,29 +407,42 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_after();
       if (active) {
         const int head = ic.grp * C::PARTS + ((STRIDE == 1) ? 0 : wq);
-        const uint32_t oaddr = tq + (jj & 1) * kSlotCols + ((STRIDE == 1) ? 0 : wq * C::O_COLS);
+        // the streams of this warp's part: all of them at stride 1, part wq at stride 2
+        const int q0 = (STRIDE == 1) ? 0 : wq * C::SPP;
         float o[D / 2];
-        if constexpr (D == 16) {
-          uint32_t r[8];
-          tmem_ld_16x32bx2_x8<8>(oaddr, r);
-          uint32_t rs[8];
-          tmem_ld_16x32bx2_x8<8>(oaddr + D, rs);  // row sums (ones tile): every column holds the sum
-          tmem_wait_ld();
 #pragma unroll
-          for (int t = 0; t < 8; ++t) o[t] = __uint_as_float(r[t]);
-          l = __uint_as_float(rs[0]);
-        } else if constexpr (D == 32) {
-          uint32_t r[16];
-          tmem_ld_16x32bx2_x16<16>(oaddr, r);
-          tmem_wait_ld();
+        for (int t = 0; t < D / 2; ++t) o[t] = 0.f;
+        if constexpr (D == 16) l = 0.f;
+#pragma unroll 1
+        for (int q = q0; q < q0 + ((STRIDE == 1) ? C::NST : C::SPP); ++q) {
+          const uint32_t oaddr = tq + (jj & 1) * kSlotCols + q * C::O_COLS;
+          if constexpr (D == 16) {
+            uint32_t r[8];
+            tmem_ld_16x32bx2_x8<8>(oaddr, r);
+            uint32_t rs[8];
+            tmem_ld_16x32bx2_x8<8>(oaddr + D, rs);  // row sums (ones tile): every column holds the sum
+            tmem_wait_ld();
 #pragma unroll
-          for (int t = 0; t < 16; ++t) o[t] = __uint_as_float(r[t]);
-        } else {
-          uint32_t r[32];
-          tmem_ld_16x32bx2_x32<32>(oaddr, r);
-          tmem_wait_ld();
+            for (int t = 0; t < 8; ++t) o[t] += __uint_as_float(r[t]);
+            l += __uint_as_float(rs[0]);
+          } else if constexpr (D == 32) {
+            uint32_t r[16];
+            tmem_ld_16x32bx2_x16<16>(oaddr, r);
+            tmem_wait_ld();
 #pragma unroll
-          for (int t = 0; t < 32; ++t) o[t] = __uint_as_float(r[t]);
+            for (int t = 0; t < 16; ++t) o[t] += __uint_as_float(r[t]);
+          } else {
+            // two loads of 16 columns per half row: fewer registers live next
+            // to the S rows of the item in flight
+#pragma unroll
+            for (int hpart = 0; hpart < 2; ++hpart) {
+              uint32_t r[16];
+              tmem_ld_16x32bx2_x16<32>(oaddr + 16 * hpart, r);
+              tmem_wait_ld();
+#pragma unroll
+              for (int t = 0; t < 16; ++t) o[16 * hpart + t] += __uint_as_float(r[t]);
+            }
+          }
         }
         const float inv = 1.0f / l;
         uint32_t pk[D / 4];
@@ -597,6 +575,34 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       __syncwarp();
       if (lane == 0) mbar_arrive(&bar_pfull[b]);
+      // ---- A.V: warp wq < NST issues its share once the whole P tile is written
+      bool issued = true;
+      if (wq < C::NST && lane == 0) {
+        issued = mbar_wait(&bar_pfull[b], (j >> 1) & 1, kWaitNs, &abort_flag);
+        if (issued) {
+          tc_fence_after();
+          const int s = k % S, part = wq / C::SPP, sub = wq % C::SPP;
+          const int kb = WIN * sub / C::SPP, ke = WIN * (sub + 1) / C::SPP;
+          const uint32_t dst = tmem + (static_cast<uint32_t>(g * 16) << 16) + sl * kSlotCols + wq * C::O_COLS;
+          const uint32_t pa = smem_addr(pt);
+          const uint32_t va = smem_addr(sStage + s * C::STAGE_BYTES + C::Q_BYTES + C::PARTS * C::K_TILE +
+                                        part * C::V_TILE);
+          // with the ones tile the B operand spans two swizzle atoms along N:
+          // V (D columns) then ones (D columns) at leading byte offset LBO
+          const uint32_t lbo = C::SUM_BY_MMA ? (smem_addr(sOnes) - va) : 16u;
+#pragma unroll 1
+          for (int kk = kb; kk < ke; ++kk)
+            mma_f16_ss(dst, smem_desc(pa + kk * 2048, 16, 256, SW_32B),
+                       smem_desc(va + kk * kRowKeys * C::ROWB, lbo, C::SBO, C::SW), idO, kk != kb);
+          mma_commit(&bar_ofull[b]);
+          mma_commit(&bar_empty[s]);
+        }
+      }
+      if (!__all_sync(0xffffffffu, issued)) {
+        if (!abort_flag) record_timeout(&abort_flag);
+        ok = false;
+        break;
+      }
       prev_ic = ic;
       prev_l = l;
     }
