@@ -405,13 +405,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         return false;
       }
       tc_fence_after();
-      if (active) {
-        const int head = ic.grp * C::PARTS + ((STRIDE == 1) ? 0 : wq);
-        // the streams of this warp's part: all of them at stride 1, part wq at stride 2
-        const int q0 = (STRIDE == 1) ? 0 : wq * C::SPP;
-        float o[D / 2];
+      // the streams of this warp's part: all of them at stride 1, part wq at stride 2
+      float o[D / 2];
 #pragma unroll
-        for (int t = 0; t < D / 2; ++t) o[t] = 0.f;
+      for (int t = 0; t < D / 2; ++t) o[t] = 0.f;
+      if (active) {
+        const int q0 = (STRIDE == 1) ? 0 : wq * C::SPP;
         if constexpr (D == 16) l = 0.f;
 #pragma unroll 1
         for (int q = q0; q < q0 + ((STRIDE == 1) ? C::NST : C::SPP); ++q) {
@@ -444,6 +443,13 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
           }
         }
+      }
+      // the slot's TMEM has been read: hand it back before the arithmetic and stores
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bar_tfree[b]);
+      if (active) {
+        const int head = ic.grp * C::PARTS + ((STRIDE == 1) ? 0 : wq);
         const float inv = 1.0f / l;
         uint32_t pk[D / 4];
 #pragma unroll
@@ -456,9 +462,6 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int t = 0; t < D / 16; ++t)
           reinterpret_cast<uint4*>(dst)[t] = make_uint4(pk[4 * t], pk[4 * t + 1], pk[4 * t + 2], pk[4 * t + 3]);
       }
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&bar_tfree[b]);
       return true;
     };
 

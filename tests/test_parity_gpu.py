@@ -40,6 +40,7 @@ def _compare(got, want, tol, what=""):
     err = np.abs(got - want)
     assert np.all(np.isfinite(got)), f"{what}: non-finite outputs"
     assert err.max() <= tol, f"{what}: max abs err {err.max():.3e} > {tol} (mean {err.mean():.2e})"
+    print(f"[parity] {what}: max abs err {err.max():.3e} (mean {err.mean():.2e}, tol {tol})")
     return err.max()
 
 
