@@ -36,7 +36,8 @@ import workloads  # noqa: E402
 
 METRIC = "halo-attention output pixels/s and TFLOP/s, % of bf16 tensor/HBM roofline"
 KERNEL_SOURCES = ["blocked_local_self_b200/csrc/halo_tc.cuh", "blocked_local_self_b200/csrc/halo_tc2.cuh",
-                  "blocked_local_self_b200/csrc/halo_tc3.cuh", "blocked_local_self_b200/csrc/sm100.cuh"]
+                  "blocked_local_self_b200/csrc/halo_tc3.cuh", "blocked_local_self_b200/csrc/halo_tc4.cuh",
+                  "blocked_local_self_b200/csrc/sm100.cuh"]
 PROFILES = os.path.join(ROOT, "profiles")
 L2_BYTES = 126 * 1024 * 1024
 

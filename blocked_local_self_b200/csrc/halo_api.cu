@@ -16,6 +16,7 @@
 #include "halo_tc.cuh"
 #include "halo_tc2.cuh"
 #include "halo_tc3.cuh"
+#include "halo_tc4.cuh"
 
 namespace {
 
@@ -141,6 +142,29 @@ const Tc3Entry* find_tc3(const Shape& s) {
   return nullptr;
 }
 
+// Stride-1 kernel with two vertically adjacent blocks per item (dim_head 64).
+using Tc4Kernel = void (*)(const CUtensorMap, const CUtensorMap, const CUtensorMap, const halo::tc4::Params);
+struct Tc4Entry {
+  int d, win;
+  Tc4Kernel fn;
+  int (*smem)(int);
+};
+template <int D, int WIN>
+int tc4_smem(int stages) { return halo::tc4::smem_bytes<D, WIN>(stages); }
+#define HALO_TC4_ENTRY(D, WIN) \
+  Tc4Entry { D, WIN, halo::tc4::halo_fwd_tc4<D, WIN>, tc4_smem<D, WIN> }
+const Tc4Entry kTc4Table[] = {
+    HALO_TC4_ENTRY(64, 8), HALO_TC4_ENTRY(64, 10), HALO_TC4_ENTRY(64, 12), HALO_TC4_ENTRY(64, 14),
+};
+
+const Tc4Entry* find_tc4(const Shape& s) {
+  if (s.dtype != HALO_BF16 || s.block != halo::tc4::kBlock || s.stride != 1 || (s.H / s.block) % 2) return nullptr;
+  const int win = s.block + 2 * s.halo;
+  for (const Tc4Entry& e : kTc4Table)
+    if (e.d == s.d && e.win == win) return &e;
+  return nullptr;
+}
+
 const TcEntry* find_tc(const Shape& s) {
   if (s.dtype != HALO_BF16 || s.block != halo::tc::kBlock) return nullptr;
   const int win = s.block + 2 * s.halo;
@@ -151,7 +175,7 @@ const TcEntry* find_tc(const Shape& s) {
 
 int select_kernel(const Shape& s) {
   if (check_shape(s) != HALO_OK) return HALO_KERNEL_NONE;
-  if (find_tc2(s) || find_tc(s) || find_tc3(s)) return HALO_KERNEL_TC_BF16;
+  if (find_tc2(s) || find_tc4(s) || find_tc(s) || find_tc3(s)) return HALO_KERNEL_TC_BF16;
   if (s.d <= 128) return HALO_KERNEL_SIMT_F32;
   return HALO_KERNEL_NONE;
 }
@@ -395,6 +419,51 @@ int launch_tc3(const Tc3Entry& e, const void* q, const void* k, const void* v, c
   return cudaGetLastError() == cudaSuccess ? HALO_OK : HALO_ERR_CUDA;
 }
 
+int launch_tc4(const Tc4Entry& e, const void* q, const void* k, const void* v, const void* rh, const void* rw,
+               void* out, const Shape& s, int sm_count, cudaStream_t st) {
+  const int win = s.block + 2 * s.halo;
+  CUtensorMap mq, mk, mv;
+  if (!encode_nhwc(&mq, q, s, halo::tc4::kBlock, halo::tc4::kBlock, 1) ||
+      !encode_nhwc(&mk, k, s, win, win + halo::tc4::kBlock, 1) ||
+      !encode_nhwc(&mv, v, s, win, win + halo::tc4::kBlock, 1))
+    return HALO_ERR_CUDA;
+  cudaFuncAttributes attr;
+  if (cudaFuncGetAttributes(&attr, reinterpret_cast<const void*>(e.fn)) != cudaSuccess) return HALO_ERR_CUDA;
+  if (256 * halo::tc4::kSoftmaxRegs + 128 * halo::tc4::kProducerRegs > halo::tc4::kThreads * attr.numRegs)
+    return HALO_ERR_UNSUPPORTED;
+  int optin = 0, dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) != cudaSuccess)
+    return HALO_ERR_CUDA;
+  const int budget = (optin < kMaxDynSmem ? optin : kMaxDynSmem) - static_cast<int>(attr.sharedSizeBytes);
+  int stages = 4;  // the kernel has four stage barriers
+  while (stages > 1 && e.smem(stages) > budget) --stages;
+  const int smem = e.smem(stages);
+  if (smem > budget) return HALO_ERR_UNSUPPORTED;
+  if (cudaFuncSetAttribute(reinterpret_cast<const void*>(e.fn), cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           smem) != cudaSuccess)
+    return HALO_ERR_CUDA;
+  halo::tc4::Params p;
+  p.rel_h = static_cast<const __nv_bfloat16*>(rh);
+  p.rel_w = static_cast<const __nv_bfloat16*>(rw);
+  p.out = static_cast<__nv_bfloat16*>(out);
+  p.N = s.N;
+  p.H = s.H;
+  p.W = s.W;
+  p.heads = s.heads;
+  p.halo = s.halo;
+  p.nbx = s.W / halo::tc4::kBlock;
+  p.npy = s.H / (2 * halo::tc4::kBlock);
+  const long long items = static_cast<long long>(s.N) * p.nbx * p.npy * s.heads;
+  if (items > 0x7fffffffLL) return HALO_ERR_DIMS;
+  p.num_items = static_cast<int>(items);
+  p.stages = stages;
+  p.c = 1.4426950408889634f / std::sqrt(static_cast<float>(s.d));
+  const int grid = static_cast<int>(items < sm_count ? items : sm_count);
+  e.fn<<<grid, halo::tc4::kThreads, smem, st>>>(mq, mk, mv, p);
+  return cudaGetLastError() == cudaSuccess ? HALO_OK : HALO_ERR_CUDA;
+}
+
 int attn_device(const void* q, const void* k, const void* v, const void* rel_h, const void* rel_w, void* out,
                 const Shape& s, cudaStream_t st) {
   int rc = check_shape(s);
@@ -408,6 +477,7 @@ int attn_device(const void* q, const void* k, const void* v, const void* rel_h, 
   if (rc != HALO_OK) return rc;
   if (kind == HALO_KERNEL_TC_BF16) {
     if (const Tc2Entry* e2 = find_tc2(s)) return launch_tc2(*e2, q, k, v, rel_h, rel_w, out, s, sm_count, st);
+    if (const Tc4Entry* e4 = find_tc4(s)) return launch_tc4(*e4, q, k, v, rel_h, rel_w, out, s, sm_count, st);
     if (const Tc3Entry* e3 = find_tc3(s)) return launch_tc3(*e3, q, k, v, rel_h, rel_w, out, s, sm_count, st);
     return launch_tc(*find_tc(s), q, k, v, rel_h, rel_w, out, s, sm_count, st);
   }
@@ -478,6 +548,7 @@ const char* halo_kernel_name(int N, int H, int W, int heads, int dim_head, int b
     std::snprintf(name, sizeof(name), "none");
   } else if (kind == HALO_KERNEL_TC_BF16) {
     if (const Tc2Entry* e = find_tc2(s)) std::snprintf(name, sizeof(name), "halo_fwd_tc2<%d,%d>", e->d, e->win);
+    else if (const Tc4Entry* e = find_tc4(s)) std::snprintf(name, sizeof(name), "halo_fwd_tc4<%d,%d>", e->d, e->win);
     else if (const Tc3Entry* e = find_tc3(s)) std::snprintf(name, sizeof(name), "halo_fwd_tc3<%d,%d>", e->d, e->win);
     else {
       const TcEntry* t = find_tc(s);

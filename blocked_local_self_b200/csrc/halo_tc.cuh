@@ -209,7 +209,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   __shared__ __align__(8) uint64_t bar_pfull[4];
   __shared__ __align__(8) uint64_t bar_ofull[4];
   __shared__ __align__(8) uint64_t bar_tfree[4];
-  __shared__ __align__(8) uint64_t bar_done;
+  __shared__ __align__(8) uint64_t bar_done[2];
   __shared__ uint32_t tmem_base_sh;
   __shared__ int abort_flag;
 
@@ -225,12 +225,13 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&bar_empty[i], C::NST);
     }
     for (int b = 0; b < 4; ++b) {
-      mbar_init(&bar_sfull[b], 1);
+      mbar_init(&bar_sfull[b], 2);  // the S MMAs (warp 9) and the G MMAs (warp 10)
       mbar_init(&bar_pfull[b], 4);
       mbar_init(&bar_ofull[b], C::NST);
       mbar_init(&bar_tfree[b], 4);
     }
-    mbar_init(&bar_done, 1);
+    mbar_init(&bar_done[0], 1);
+    mbar_init(&bar_done[1], 1);
     abort_flag = 0;
     fence_mbar_init();
   }
@@ -324,7 +325,9 @@ __global__ void __launch_bounds__(kThreads, 1)
           mbar_wait(&bar_full[k % S], (k / S) & 1, kWaitNs);
       }
     }
-  } else if (warp == kMmaWarp) {
+  } else if (warp == kMmaWarp || warp == kMmaWarp + 1) {
+    // warp 9 issues S = Q K^T, warp 10 G = Q R^T, in parallel
+    const bool is_g = (warp == kMmaWarp + 1);
     // ------------------------------------------------------------ MMA issue
     if (lane == 0) {
       const uint32_t idS = idesc_bf16_f32(64, C::NS, false);
@@ -334,14 +337,18 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int s = k % S, g = k & 1, sl = (k >> 1) & 1;
         const uint32_t dst = tmem + (static_cast<uint32_t>(g * 16) << 16) + sl * kSlotCols;
         const uint8_t* st = sStage + s * C::STAGE_BYTES;
+        if (!is_g) {
 #pragma unroll 1
-        for (int part = 0; part < C::PARTS; ++part) {
-          const uint32_t qa = smem_addr(st + ((STRIDE == 1) ? 0 : (48 + 48 * part) * C::ROWB));
-          const uint32_t ka = smem_addr(st + C::Q_BYTES + part * C::K_TILE);
-          for (int ks = 0; ks < D / 16; ++ks) {
-            mma_f16_ss(dst, smem_desc(qa + 32 * ks, 16, C::SBO, C::SW), smem_desc(ka + 32 * ks, 16, C::SBO, C::SW),
-                       idS, (part | ks) != 0);
+          for (int part = 0; part < C::PARTS; ++part) {
+            const uint32_t qa = smem_addr(st + ((STRIDE == 1) ? 0 : (48 + 48 * part) * C::ROWB));
+            const uint32_t ka = smem_addr(st + C::Q_BYTES + part * C::K_TILE);
+            for (int ks = 0; ks < D / 16; ++ks) {
+              mma_f16_ss(dst, smem_desc(qa + 32 * ks, 16, C::SBO, C::SW),
+                         smem_desc(ka + 32 * ks, 16, C::SBO, C::SW), idS, (part | ks) != 0);
+            }
           }
+          mma_commit(&bar_sfull[2 * g + sl]);
+          return;
         }
         const uint32_t ra = smem_addr(sR);
 #pragma unroll 1
@@ -367,8 +374,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         issue_s(ns);
       }
       // all issued MMAs complete before the CTA frees TMEM
-      mma_commit(&bar_done);
-      mbar_wait(&bar_done, 0, kWaitNs);
+      mma_commit(&bar_done[is_g ? 1 : 0]);
+      mbar_wait(&bar_done[is_g ? 1 : 0], 0, kWaitNs);
     }
   }
   __syncwarp();  // reconverge lane 0 with its warp before the aligned barrier

@@ -1,0 +1,541 @@
+// halo_tc4.cuh -- stride-1 bf16 kernel for blocked local self-attention with
+// haloing on sm_100a, for wide heads (dim_head 64) and 8x8 query blocks.
+//
+// Operation (HaloNet, "Scaling Local Self-Attention for Parameter Efficient
+// Visual Backbones", sections 2.1-2.2 and appendix A; index conventions of the
+// blog page's RelPosEmb / HaloAttention modules):
+//   z[q, key] = s * q . (k[key] + rel_h[kr - qy + w - 1] + rel_w[kc - qx + w - 1])
+//   out[q]    = sum over in-image window keys of softmax(z) * v[key]
+//
+// Work item = two vertically adjacent 8x8 blocks of one head.  Their windows
+// (w x w each) overlap in w - 8 rows, so one TMA box of (w + 8) x w pixels
+// holds both: in the box's row-major order block A's window is keys
+// [0, w*w) and block B's is keys [8w, 8w + w*w), both contiguous.  With
+// d = 64 two heads' windows would not fit two pipeline stages in shared
+// memory; two blocks' union does (96 KB per stage).
+//   * TMA (warp 8): Q_A, Q_B [64 x d] and the union K, V tiles.
+//   * S MMA (warp 9): per block M=64, N=200 (its window) into its TMEM lane
+//     half (block A lanes 0-15 of each quadrant, block B 16-31).
+//   * G MMA (warp 10): per block G = Q R^T (N=56, R = [rel_h; 0; rel_w; 0]
+//     written once) into slot columns [200, 256); each thread takes the
+//     w + w relative logits of its query by a TMEM column shift and selects.
+//   * softmax (one thread per TMEM lane = one query row): pass 1 takes an
+//     upper bound of the row maximum, max over keys of c*S plus the maximum
+//     of c*rel_w and of c*rel_h (at most a few units above the exact one);
+//     pass 2 the exponentials (MUFU and the FMA-pipe cubic), the row sum and
+//     bf16 P written back over the S columns.
+//   * A.V (warp 0): O = P [V_A | V_B], M=128, N=2d: the B operand's second
+//     swizzle atom is block B's window, 8w rows below block A's in the same
+//     V tile.  Block A's rows use columns [0, d), block B's [d, 2d).
+//   * epilogue: O / l, bf16, NHWC.
+// Two softmax warpgroups take alternate items; every wait is bounded.
+#pragma once
+
+#include <cstdint>
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <utility>
+
+#include "halo_tc.cuh"
+#include "halo_tc2.cuh"
+#include "sm100.cuh"
+
+namespace halo {
+namespace tc4 {
+
+using namespace sm100;
+using tc::exp2_mufu;
+using tc::pack_bf16x2;
+using tc::record_timeout;
+using tc::swz;
+using tc2::exp2_poly2;
+using tc2::max3f;
+using tc2::mma_f16_ts;
+using tc2::pack_p;
+using tc2::poly_pair_mask;
+using tc2::tmem_ld_cols;
+using tc2::tmem_ld_x32;
+using tc2::tmem_ld_x8;
+using tc2::tmem_st_x8;
+using tc2::tmem_wait_st;
+
+constexpr int kBlock = 8;
+constexpr int kThreads = 384;   // warpgroups 0-1 softmax, warp 8 TMA, warp 9 S MMA, warp 10 G MMA
+constexpr int kTmaWarp = 8;
+constexpr int kMmaWarp = 9;
+constexpr int kGMmaWarp = 10;
+constexpr int kSoftmaxRegs = tc::kSoftmaxRegs;
+constexpr int kProducerRegs = tc::kProducerRegs;
+constexpr uint32_t kTmemCols = 512;
+constexpr uint32_t kSlotCols = 256;  // warpgroup g owns columns [256g, 256g + 256)
+constexpr uint32_t kGBase = 200;     // G at slot columns [200, 256): rel_h logits, then rel_w at +28
+constexpr int kRelW = 28;
+constexpr int kRRows = 56;
+constexpr uint64_t kWaitNs = tc::kWaitNs;
+
+struct Params {
+  const __nv_bfloat16* rel_h;
+  const __nv_bfloat16* rel_w;
+  __nv_bfloat16* out;
+  int N, H, W, heads, halo;
+  int nbx, npy;    // blocks along x, block pairs along y
+  int num_items;   // N * npy * nbx * heads
+  int stages;
+  float c;         // log2(e) / sqrt(d)
+};
+
+template <int D, int WIN>
+struct Cfg {
+  static constexpr int ROWB = D * 2;
+  static constexpr int KS = WIN * WIN;                    // window keys of one block
+  static constexpr int NS = (KS + 7) / 8 * 8;             // S MMA N
+  static constexpr int KSTEPS = (KS + 15) / 16;           // A.V K-steps
+  static constexpr int KP = KSTEPS * 16;                  // keys incl. zero padding
+  static constexpr int BOFF = kBlock * WIN;               // block B's first key in the union tile
+  static constexpr int UROWS = (WIN + kBlock) * WIN;      // union tile rows the TMA writes
+  static constexpr int KROWS = BOFF + (KP > NS ? KP : NS);  // rows read by the MMAs
+  static constexpr int Q_TILE = 64 * ROWB;
+  static constexpr int K_TILE = (KROWS * ROWB + 1023) / 1024 * 1024;
+  static constexpr int STAGE_BYTES = 2 * Q_TILE + 2 * K_TILE;
+  static constexpr int R_TILE = (kRRows * ROWB + 1023) / 1024 * 1024;
+  static constexpr int TX_BYTES = (2 * 64 + 2 * UROWS) * ROWB;
+  static constexpr int PCOLS = KP / 2;                    // packed bf16 P columns
+  static constexpr int O_BASE = (PCOLS + 7) / 8 * 8;      // first O column
+  static constexpr int O_N = 2 * D;                       // [V_A | V_B]
+  static constexpr SmemSwizzle SW = (ROWB == 32) ? SW_32B : (ROWB == 64 ? SW_64B : SW_128B);
+  static constexpr uint32_t SBO = 8 * ROWB;
+  static constexpr int HALO = (WIN - kBlock) / 2;
+  // softmax chunks (register working sets), boundaries at whole K-steps
+  static constexpr int NCHUNK = 3;
+  __host__ __device__ static constexpr int cstep(int i) { return (KSTEPS * i + NCHUNK / 2) / NCHUNK; }
+  static_assert(D == 32 || D == 64, "dim_head 32 or 64");
+  static_assert(WIN % 2 == 0 && WIN >= 8 && WIN <= 14, "window 8..14");
+  static_assert(NS <= (int)kGBase, "S columns below the relative logits");
+  static_assert(2 * WIN - 1 <= kRelW, "relative table rows");
+  static_assert(O_BASE + O_N <= (int)kSlotCols, "O accumulator in the slot");
+  static_assert((BOFF * ROWB) % 1024 == 0 || ROWB < 128, "block B's window on a swizzle atom");
+  static_assert(Q_TILE % 1024 == 0, "tiles on 1 KB boundaries");
+};
+
+template <int D, int WIN>
+__host__ __device__ constexpr int smem_bytes(int stages) {
+  using C = Cfg<D, WIN>;
+  return 1024 + C::R_TILE + stages * C::STAGE_BYTES;
+}
+
+// Load exactly N (< 32) consecutive TMEM columns (32x32b shape, thread t <->
+// lane t of the warp's quadrant) without reading past the last one.
+__device__ __forceinline__ void tmem_ld_x4(uint32_t taddr, float* r) {
+  uint32_t v[4];
+  asm volatile("tcgen05.ld.sync.aligned.32x32b.x4.b32 {%0,%1,%2,%3}, [%4];"
+               : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3])
+               : "r"(taddr));
+#pragma unroll
+  for (int i = 0; i < 4; ++i) r[i] = __uint_as_float(v[i]);
+}
+__device__ __forceinline__ void tmem_ld_x2(uint32_t taddr, float* r) {
+  uint32_t v[2];
+  asm volatile("tcgen05.ld.sync.aligned.32x32b.x2.b32 {%0,%1}, [%2];" : "=r"(v[0]), "=r"(v[1]) : "r"(taddr));
+  r[0] = __uint_as_float(v[0]);
+  r[1] = __uint_as_float(v[1]);
+}
+__device__ __forceinline__ void tmem_ld_x1(uint32_t taddr, float* r) {
+  uint32_t v;
+  asm volatile("tcgen05.ld.sync.aligned.32x32b.x1.b32 {%0}, [%1];" : "=r"(v) : "r"(taddr));
+  r[0] = __uint_as_float(v);
+}
+template <int N>
+__device__ __forceinline__ void tmem_ld_exact(uint32_t taddr, float* r) {
+  static_assert(N > 0 && N < 32, "at most 31 columns");
+  constexpr int a = N & 16, b = N & 8, c4 = N & 4, c2 = N & 2, c1 = N & 1;
+  if constexpr (a) {
+    float t[16];
+    tmem_ld_x8(taddr, t);
+    tmem_ld_x8(taddr + 8, t + 8);
+#pragma unroll
+    for (int i = 0; i < 16; ++i) r[i] = t[i];
+  }
+  if constexpr (b) tmem_ld_x8(taddr + a, r + a);
+  if constexpr (c4) tmem_ld_x4(taddr + a + b, r + a + b);
+  if constexpr (c2) tmem_ld_x2(taddr + a + b + c4, r + a + b + c4);
+  if constexpr (c1) tmem_ld_x1(taddr + a + b + c4 + c2, r + a + b + c4 + c2);
+}
+
+struct ItemCoord {
+  int n, py, bx, head;
+};
+__device__ __forceinline__ ItemCoord item_coord(int item, int heads, int nbx, int npy) {
+  ItemCoord c;
+  c.head = item % heads;
+  const int blk = item / heads;
+  c.bx = blk % nbx;
+  c.py = (blk / nbx) % npy;
+  c.n = blk / (nbx * npy);
+  return c;
+}
+
+// Pass 1 over keys [J0, J1) of this thread's S row: per window row the
+// maximum of the raw S values (rm[r], rows R0..).
+template <int WIN, int J0, int J1>
+__device__ __forceinline__ void row_max_chunk(uint32_t ts, float (&rm)[WIN]) {
+  constexpr int NL = (J1 - J0 + 7) / 8 * 8;
+  float z[NL];
+  tmem_ld_cols<NL>(ts + J0, z);
+  tmem_wait_ld();
+#pragma unroll
+  for (int i = 0; i < (J1 - J0) / 2; ++i) {
+    const int r = (J0 + 2 * i) / WIN;
+    rm[r] = max3f(rm[r], z[2 * i], z[2 * i + 1]);
+  }
+}
+
+// Pass 2 over keys [J0, J1) (padded to JP): p = 2^(c*(S + rel_w) + brow[row]),
+// row sum, packed bf16 P over TMEM columns [J0/2, JP/2).
+template <int WIN, int J0, int J1, int JP>
+__device__ __forceinline__ float exp_chunk(uint32_t ts, const float (&rw)[WIN], const float (&brow)[WIN], float c) {
+  constexpr int NL = (J1 - J0 + 7) / 8 * 8;
+  constexpr int NW = (JP - J0) / 2;
+  constexpr int NP = (J1 - J0) / 2;
+  static_assert(J0 % 2 == 0 && J1 % 2 == 0 && NW % 8 == 0, "pairs never straddle rows");
+  constexpr unsigned kPoly = poly_pair_mask<WIN>();
+  float z[NL];
+  tmem_ld_cols<NL>(ts + J0, z);
+  tmem_wait_ld();
+  float2 lacc[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
+  uint32_t pk[NW];
+#pragma unroll
+  for (int i = 0; i < NP; ++i) {
+    const int j = J0 + 2 * i, kc = j % WIN;
+    const float2 zz = __fadd2_rn(make_float2(z[2 * i], z[2 * i + 1]), make_float2(rw[kc], rw[kc + 1]));
+    const float bias = brow[j / WIN];
+    const float2 x = __ffma2_rn(zz, make_float2(c, c), make_float2(bias, bias));
+    uint32_t rx, ry;
+    if ((kPoly >> (kc / 2)) & 1u) {
+      exp2_poly2(x, rx, ry);
+    } else {
+      rx = __float_as_uint(exp2_mufu(x.x));
+      ry = __float_as_uint(exp2_mufu(x.y));
+    }
+    lacc[i & 3] = __fadd2_rn(lacc[i & 3], make_float2(__uint_as_float(rx), __uint_as_float(ry)));
+    pk[i] = pack_p(rx, ry);
+  }
+#pragma unroll
+  for (int i = NP; i < NW; ++i) pk[i] = 0u;
+#pragma unroll
+  for (int i = 0; i < NW; i += 8) tmem_st_x8(ts + J0 / 2 + i, pk + i);
+  const float2 la = __fadd2_rn(lacc[0], lacc[1]), lb = __fadd2_rn(lacc[2], lacc[3]);
+  return (la.x + lb.x) + (la.y + lb.y);
+}
+
+template <int WIN, class C, int... I>
+__device__ __forceinline__ void row_max_all(uint32_t ts, float (&rm)[WIN], std::integer_sequence<int, I...>) {
+  (row_max_chunk<WIN, 16 * C::cstep(I), (I + 1 == C::NCHUNK) ? C::KS : 16 * C::cstep(I + 1)>(ts, rm), ...);
+}
+template <int WIN, class C, int... I>
+__device__ __forceinline__ float exp_all(uint32_t ts, const float (&rw)[WIN], const float (&brow)[WIN], float c,
+                                         std::integer_sequence<int, I...>) {
+  return (exp_chunk<WIN, 16 * C::cstep(I), (I + 1 == C::NCHUNK) ? C::KS : 16 * C::cstep(I + 1),
+                    16 * C::cstep(I + 1)>(ts, rw, brow, c) + ...);
+}
+
+template <int D, int WIN>
+__global__ void __launch_bounds__(kThreads, 1)
+    halo_fwd_tc4(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__ CUtensorMap tmap_k,
+                 const __grid_constant__ CUtensorMap tmap_v, const Params p) {
+  using C = Cfg<D, WIN>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* sR = smem;
+  uint8_t* sStage = smem + C::R_TILE;
+  // stage layout: [Q_A][Q_B][K union][V union]
+  constexpr int OFF_QA = 0, OFF_QB = C::Q_TILE, OFF_K = 2 * C::Q_TILE, OFF_V = OFF_K + C::K_TILE;
+
+  __shared__ __align__(8) uint64_t bar_full[4];
+  __shared__ __align__(8) uint64_t bar_empty[4];
+  __shared__ __align__(8) uint64_t bar_sfull[2];   // count 2: the S and the G MMAs of the item
+  __shared__ __align__(8) uint64_t bar_ofull[2];
+  __shared__ __align__(8) uint64_t bar_tfree[2];   // count 4: the warpgroup read its slot's O
+  __shared__ __align__(8) uint64_t bar_pready[2];  // count 4, waited by every warp of the warpgroup
+  __shared__ __align__(8) uint64_t bar_done[2];
+  __shared__ __align__(8) uint64_t bar_pvdone[2];
+  __shared__ uint32_t tmem_base_sh;
+  __shared__ int abort_flag;
+
+  const int tid = threadIdx.x;
+  const int warp = tid >> 5;
+  const int lane = tid & 31;
+  const int S = p.stages;
+
+  // ---------------------------------------------------------------- set-up
+  if (tid == 0) {
+    for (int i = 0; i < S; ++i) {
+      mbar_init(&bar_full[i], 1);
+      mbar_init(&bar_empty[i], 1);
+    }
+    for (int g = 0; g < 2; ++g) {
+      mbar_init(&bar_sfull[g], 2);
+      mbar_init(&bar_ofull[g], 1);
+      mbar_init(&bar_tfree[g], 4);
+      mbar_init(&bar_pready[g], 4);
+      mbar_init(&bar_done[g], 1);
+      mbar_init(&bar_pvdone[g], 1);
+    }
+    abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == kTmaWarp && lane == 0) {
+    prefetch_tensormap(&tmap_q);
+    prefetch_tensormap(&tmap_k);
+    prefetch_tensormap(&tmap_v);
+  }
+  // R tile (once) and the union tiles' rows the TMA never writes (zero)
+  for (int idx = tid; idx < kRRows * (D / 8); idx += kThreads) {
+    const int r = idx / (D / 8), u = idx % (D / 8);
+    uint4 val = make_uint4(0, 0, 0, 0);
+    if (r < 2 * WIN - 1) val = *reinterpret_cast<const uint4*>(p.rel_h + r * D + u * 8);
+    else if (r >= kRelW && r < kRelW + 2 * WIN - 1)
+      val = *reinterpret_cast<const uint4*>(p.rel_w + (r - kRelW) * D + u * 8);
+    *reinterpret_cast<uint4*>(sR + swz<C::ROWB>(r, u)) = val;
+  }
+  for (int s = 0; s < S; ++s) {
+    uint8_t* st = sStage + s * C::STAGE_BYTES;
+    for (int idx = tid; idx < (C::KROWS - C::UROWS) * C::ROWB / 16; idx += kThreads) {
+      reinterpret_cast<uint4*>(st + OFF_K + C::UROWS * C::ROWB)[idx] = make_uint4(0, 0, 0, 0);
+      reinterpret_cast<uint4*>(st + OFF_V + C::UROWS * C::ROWB)[idx] = make_uint4(0, 0, 0, 0);
+    }
+  }
+  fence_proxy_async_smem();
+  if (warp == 0) {
+    tmem_alloc(&tmem_base_sh, kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = tmem_base_sh;
+  const int my_items = (p.num_items > (int)blockIdx.x)
+                           ? (p.num_items - 1 - (int)blockIdx.x) / (int)gridDim.x + 1 : 0;
+
+  if (warp >= 8) {
+  asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kProducerRegs));
+  if (warp == kTmaWarp) {
+    // ------------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      int issued = 0;
+      for (int k = 0; k < my_items; ++k) {
+        const int s = k % S;
+        if (k >= S && !mbar_wait(&bar_empty[s], ((k / S) - 1) & 1, kWaitNs, &abort_flag)) {
+          if (!abort_flag) record_timeout(&abort_flag);
+          break;
+        }
+        const ItemCoord ic = item_coord(blockIdx.x + k * gridDim.x, p.heads, p.nbx, p.npy);
+        uint8_t* st = sStage + s * C::STAGE_BYTES;
+        const int x0 = ic.bx * kBlock, y0 = ic.py * 2 * kBlock;
+        mbar_arrive_expect_tx(&bar_full[s], C::TX_BYTES);
+        tma_load_4d(st + OFF_QA, &tmap_q, &bar_full[s], ic.head * D, x0, y0, ic.n);
+        tma_load_4d(st + OFF_QB, &tmap_q, &bar_full[s], ic.head * D, x0, y0 + kBlock, ic.n);
+        tma_load_4d(st + OFF_K, &tmap_k, &bar_full[s], ic.head * D, x0 - p.halo, y0 - p.halo, ic.n);
+        tma_load_4d(st + OFF_V, &tmap_v, &bar_full[s], ic.head * D, x0 - p.halo, y0 - p.halo, ic.n);
+        issued = k + 1;
+      }
+      if (abort_flag) {
+        for (int k = (issued > S ? issued - S : 0); k < issued; ++k)
+          mbar_wait(&bar_full[k % S], (k / S) & 1, kWaitNs);
+      }
+    }
+  } else if (warp == kMmaWarp || warp == kGMmaWarp) {
+    // ------------------------------------------------------------ S (warp 9) and G (warp 10) MMAs
+    const bool is_g = (warp == kGMmaWarp);
+    if (lane == 0) {
+      const uint32_t idS = idesc_bf16_f32(64, C::NS, false);
+      const uint32_t idG = idesc_bf16_f32(64, kRRows, false);
+      const uint32_t ra = smem_addr(sR);
+      for (int k = 0; k < my_items; ++k) {
+        const int s = k % S, g = k & 1;
+        if (!mbar_wait(&bar_full[s], (k / S) & 1, kWaitNs, &abort_flag) ||
+            (k >= 2 && !mbar_wait(&bar_tfree[g], ((k >> 1) - 1) & 1, kWaitNs, &abort_flag))) {
+          if (!abort_flag) record_timeout(&abort_flag);
+          break;
+        }
+        tc_fence_after();
+        const uint8_t* st = sStage + s * C::STAGE_BYTES;
+        const uint32_t slot = tmem + g * kSlotCols;
+#pragma unroll 1
+        for (int blk = 0; blk < 2; ++blk) {
+          const uint32_t qa = smem_addr(st + (blk ? OFF_QB : OFF_QA));
+          const uint32_t dst = slot + (static_cast<uint32_t>(blk * 16) << 16);
+          if (is_g) {
+#pragma unroll
+            for (int ks = 0; ks < D / 16; ++ks)
+              mma_f16_ss(dst + kGBase, smem_desc(qa + 32 * ks, 16, C::SBO, C::SW),
+                         smem_desc(ra + 32 * ks, 16, C::SBO, C::SW), idG, ks != 0);
+          } else {
+            const uint32_t ka = smem_addr(st + OFF_K + blk * C::BOFF * C::ROWB);
+#pragma unroll
+            for (int ks = 0; ks < D / 16; ++ks)
+              mma_f16_ss(dst, smem_desc(qa + 32 * ks, 16, C::SBO, C::SW), smem_desc(ka + 32 * ks, 16, C::SBO, C::SW),
+                         idS, ks != 0);
+          }
+        }
+        mma_commit(&bar_sfull[g]);
+      }
+      const int w = is_g ? 1 : 0;
+      mma_commit(&bar_done[w]);
+      mbar_wait(&bar_done[w], 0, kWaitNs);
+    }
+  }
+  __syncwarp();
+  tc_fence_before();
+  named_bar_sync(1, kThreads);
+  return;
+  }
+
+  asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kSoftmaxRegs));
+  {
+    // ------------------------------------------------------------ softmax warpgroups
+    const int g = warp >> 2;             // warpgroup = TMEM slot
+    const int wq = warp & 3;             // lane quadrant
+    const int blk = lane >> 4;           // 0: block A (lanes 0-15), 1: block B (lanes 16-31)
+    const int row = 16 * wq + (lane & 15);  // query row in the 8x8 block
+    const int qy = row >> 3, qx = row & 7;
+    const uint32_t slot = tmem + g * kSlotCols;
+    const uint32_t ts = slot + (static_cast<uint32_t>(32 * wq) << 16);
+    const float c = p.c;
+    const int C_all = p.heads * D;
+    const uint32_t idO = idesc_bf16_f32(128, C::O_N, true);
+
+    int j = 0;
+    for (int k = g; k < my_items; k += 2, ++j) {
+      if (!mbar_wait(&bar_sfull[g], j & 1, kWaitNs, &abort_flag)) {
+        if (!abort_flag) record_timeout(&abort_flag);
+        break;
+      }
+      tc_fence_after();
+      const ItemCoord ic = item_coord(blockIdx.x + k * gridDim.x, p.heads, p.nbx, p.npy);
+      const int by = 2 * ic.py + blk;
+      const int y0 = by * kBlock - p.halo, x0 = ic.bx * kBlock - p.halo;
+
+      // ---- relative logits of this query, in log2 units:
+      //   rh[kr] = c * q.rel_h[kr - qy + w - 1], rw[kc] = c * q.rel_w[kc - qx + w - 1]
+      float rh[WIN], rw[WIN], rwz[WIN];  // rwz: rel_w logits unscaled (S units)
+      {
+        // rel_h: the warp's two query rows differ by one column; the shift by
+        // the warp's first row goes into the load address
+        float gh[WIN + 1];
+        tmem_ld_exact<WIN + 1>(ts + kGBase + (WIN - 2 - 2 * wq), gh);
+        // rel_w: a[i] = G[rel_w + w - 8 + i], shifted by sh = 7 - qx (3 bits)
+        float a[WIN + 7];
+        tmem_ld_exact<WIN + 7>(ts + kGBase + kRelW + WIN - 8, a);
+        tmem_wait_ld();
+        const bool odd = ((lane >> 3) & 1) != 0;
+#pragma unroll
+        for (int kr = 0; kr < WIN; ++kr) {
+          const int Y = y0 + kr;
+          const float v = odd ? gh[kr] : gh[kr + 1];
+          rh[kr] = (Y >= 0 && Y < p.H) ? v * c : -INFINITY;
+        }
+        const int sh = 7 - qx;
+#pragma unroll
+        for (int i = 0; i < WIN + 3; ++i) a[i] = (sh & 4) ? a[i + 4] : a[i];
+#pragma unroll
+        for (int i = 0; i < WIN + 1; ++i) a[i] = (sh & 2) ? a[i + 2] : a[i];
+#pragma unroll
+        for (int i = 0; i < WIN; ++i) a[i] = (sh & 1) ? a[i + 1] : a[i];
+#pragma unroll
+        for (int kc = 0; kc < WIN; ++kc) {
+          const int X = x0 + kc;
+          rwz[kc] = (X >= 0 && X < p.W) ? a[kc] : -INFINITY;
+          rw[kc] = rwz[kc] * c;
+        }
+      }
+
+      // ---- pass 1: upper bound of the row maximum (log2 units)
+      float rm[WIN];
+#pragma unroll
+      for (int r = 0; r < WIN; ++r) rm[r] = -INFINITY;
+      row_max_all<WIN, C>(ts, rm, std::make_integer_sequence<int, C::NCHUNK>{});
+      float mw = -INFINITY;
+#pragma unroll
+      for (int kc = 0; kc < WIN; ++kc) mw = fmaxf(mw, rw[kc]);
+      float m = -INFINITY;
+#pragma unroll
+      for (int r = 0; r < WIN; ++r) m = fmaxf(m, fmaf(rm[r], c, rh[r]));
+      m += mw;  // finite: the query's own block is in the image
+      // ---- pass 2: p = 2^(c*(S + rel_w) + c*rel_h - m)
+      float brow[WIN];
+#pragma unroll
+      for (int r = 0; r < WIN; ++r) brow[r] = rh[r] - m;
+      const float l = exp_all<WIN, C>(ts, rwz, brow, c, std::make_integer_sequence<int, C::NCHUNK>{});
+      tmem_wait_st();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bar_pready[g]);
+      if (!mbar_wait(&bar_pready[g], j & 1, kWaitNs, &abort_flag)) {
+        if (!abort_flag) record_timeout(&abort_flag);
+        break;
+      }
+      tc_fence_after();
+
+      // ---- A.V: O = P [V_A | V_B] (warp 0)
+      const int s = k % S;
+      if (wq == 0 && lane == 0) {
+        const uint32_t va = smem_addr(sStage + s * C::STAGE_BYTES + OFF_V);
+#pragma unroll 1
+        for (int kk = 0; kk < C::KSTEPS; ++kk)
+          mma_f16_ts(slot + C::O_BASE, slot + 8 * kk,
+                     smem_desc(va + kk * 16 * C::ROWB, C::BOFF * C::ROWB, C::SBO, C::SW), idO, kk != 0);
+        mma_commit(&bar_ofull[g]);
+        mma_commit(&bar_empty[s]);
+      }
+      __syncwarp();
+
+      // ---- epilogue: O / l, bf16, NHWC
+      if (!mbar_wait(&bar_ofull[g], j & 1, kWaitNs, &abort_flag)) {
+        if (!abort_flag) record_timeout(&abort_flag);
+        break;
+      }
+      tc_fence_after();
+      {
+        // the whole warp loads both blocks' columns; this thread keeps [0, D)
+        // for block A, [D, 2D) for block B
+        float o[D];
+#pragma unroll
+        for (int e = 0; e < D; e += 32) {
+          float ta[32], tb[32];
+          tmem_ld_x32(ts + C::O_BASE + e, ta);
+          tmem_ld_x32(ts + C::O_BASE + D + e, tb);
+          tmem_wait_ld();
+#pragma unroll
+          for (int i = 0; i < 32; ++i) o[e + i] = blk ? tb[i] : ta[i];
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bar_tfree[g]);
+        const float inv = 1.0f / l;
+        uint32_t pk[D / 2];
+#pragma unroll
+        for (int t = 0; t < D / 2; ++t) pk[t] = pack_bf16x2(o[2 * t] * inv, o[2 * t + 1] * inv);
+        const int y = by * kBlock + qy, x = ic.bx * kBlock + qx;
+        __nv_bfloat16* dst = p.out + ((static_cast<size_t>(ic.n) * p.H + y) * p.W + x) * C_all + ic.head * D;
+#pragma unroll
+        for (int t = 0; t < D / 8; ++t)
+          reinterpret_cast<uint4*>(dst)[t] = make_uint4(pk[4 * t], pk[4 * t + 1], pk[4 * t + 2], pk[4 * t + 3]);
+      }
+    }
+    // A.V MMAs warp 0 issued are complete before TMEM is released
+    if (wq == 0 && lane == 0) {
+      mma_commit(&bar_pvdone[g]);
+      mbar_wait(&bar_pvdone[g], 0, kWaitNs);
+    }
+    __syncwarp();
+  }
+
+  // ---------------------------------------------------------------- teardown
+  tc_fence_before();
+  named_bar_sync(1, kThreads);
+  tc_fence_after();
+  if (warp == 0) tmem_dealloc(tmem, kTmemCols);
+}
+
+}  // namespace tc4
+}  // namespace halo

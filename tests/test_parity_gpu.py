@@ -106,6 +106,11 @@ for d in (16, 32, 64):
         for stride in (1, 2):
             CASES.append(dict(N=2, H=24, W=40, heads=8 if d < 64 else 4, dim_head=d, block=8, halo=halo,
                               stride=stride))
+# dim_head 64 with an even number of block rows: the kernel that pairs two
+# vertically adjacent blocks (every window, one pair and several pairs)
+for halo in (0, 1, 2, 3):
+    CASES.append(dict(N=2, H=32, W=24, heads=3, dim_head=64, block=8, halo=halo, stride=1))
+CASES.append(dict(N=3, H=16, W=40, heads=2, dim_head=64, block=8, halo=3, stride=1))
 # 16x16 query blocks (windows 16..24): every window of the block-16 kernel, both head sizes
 for d in (16, 32):
     for halo in (0, 1, 2, 3, 4):
