@@ -506,6 +506,35 @@ int halo_attn(const void* q, const void* k, const void* v, const void* rel_h, co
   return attn_device(q, k, v, rel_h, rel_w, out, s, static_cast<cudaStream_t>(stream));
 }
 
+// Two library-owned streams and their events per device, created on first
+// use of halo_attn_host: chunk c of the images runs on stream c % 2, so the
+// copies of one chunk overlap the kernel and the copies of the previous one.
+struct HostPipe {
+  bool ready = false;
+  cudaStream_t st[2];
+  cudaEvent_t ev_in, ev_done[2];
+};
+HostPipe g_pipe[kMaxDevices];
+std::mutex g_pipe_mutex;  // one host thread at a time enqueues through the pipeline streams
+
+int host_pipe(HostPipe** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return HALO_ERR_CUDA;
+  std::lock_guard<std::mutex> lock(g_mutex);
+  HostPipe& hp = g_pipe[dev];
+  if (!hp.ready) {
+    if (cudaStreamCreateWithFlags(&hp.st[0], cudaStreamNonBlocking) != cudaSuccess ||
+        cudaStreamCreateWithFlags(&hp.st[1], cudaStreamNonBlocking) != cudaSuccess ||
+        cudaEventCreateWithFlags(&hp.ev_in, cudaEventDisableTiming) != cudaSuccess ||
+        cudaEventCreateWithFlags(&hp.ev_done[0], cudaEventDisableTiming) != cudaSuccess ||
+        cudaEventCreateWithFlags(&hp.ev_done[1], cudaEventDisableTiming) != cudaSuccess)
+      return HALO_ERR_CUDA;
+    hp.ready = true;
+  }
+  *out = &hp;
+  return HALO_OK;
+}
+
 int halo_attn_host(const void* q_h, const void* k_h, const void* v_h, const void* rel_h_h, const void* rel_w_h,
                    void* out_h, void* q_d, void* k_d, void* v_d, void* rel_h_d, void* rel_w_d, void* out_d, int N,
                    int H, int W, int heads, int dim_head, int block, int halo, int stride, int dtype,
@@ -520,17 +549,46 @@ int halo_attn_host(const void* q_h, const void* k_h, const void* v_h, const void
   int sm_count = 0;
   rc = device_info(&sm_count);
   if (rc != HALO_OK) return rc;
-  cudaStream_t st = static_cast<cudaStream_t>(stream);
-  const size_t ib = s.in_bytes(), rb = s.rel_bytes();
-  if (cudaMemcpyAsync(q_d, q_h, ib, cudaMemcpyHostToDevice, st) != cudaSuccess ||
-      cudaMemcpyAsync(k_d, k_h, ib, cudaMemcpyHostToDevice, st) != cudaSuccess ||
-      cudaMemcpyAsync(v_d, v_h, ib, cudaMemcpyHostToDevice, st) != cudaSuccess ||
-      cudaMemcpyAsync(rel_h_d, rel_h_h, rb, cudaMemcpyHostToDevice, st) != cudaSuccess ||
-      cudaMemcpyAsync(rel_w_d, rel_w_h, rb, cudaMemcpyHostToDevice, st) != cudaSuccess)
-    return HALO_ERR_CUDA;
-  rc = attn_device(q_d, k_d, v_d, rel_h_d, rel_w_d, out_d, s, st);
+  HostPipe* hp = nullptr;
+  rc = host_pipe(&hp);
   if (rc != HALO_OK) return rc;
-  if (cudaMemcpyAsync(out_h, out_d, s.out_bytes(), cudaMemcpyDeviceToHost, st) != cudaSuccess) return HALO_ERR_CUDA;
+  std::lock_guard<std::mutex> pipe_lock(g_pipe_mutex);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  // the tables first, on the caller's stream, then both pipeline streams wait
+  // for everything queued on it so far
+  const size_t rb = s.rel_bytes();
+  if (cudaMemcpyAsync(rel_h_d, rel_h_h, rb, cudaMemcpyHostToDevice, st) != cudaSuccess ||
+      cudaMemcpyAsync(rel_w_d, rel_w_h, rb, cudaMemcpyHostToDevice, st) != cudaSuccess ||
+      cudaEventRecord(hp->ev_in, st) != cudaSuccess || cudaStreamWaitEvent(hp->st[0], hp->ev_in, 0) != cudaSuccess ||
+      cudaStreamWaitEvent(hp->st[1], hp->ev_in, 0) != cudaSuccess)
+    return HALO_ERR_CUDA;
+  // chunks of whole images (NHWC: an image is a contiguous slice of every tensor)
+  const int chunks = N < 8 ? N : 8;
+  const size_t img_in = s.in_bytes() / N, img_out = s.out_bytes() / N;
+  for (int c = 0; c < chunks; ++c) {
+    const int n0 = static_cast<int>(static_cast<long long>(N) * c / chunks);
+    const int n1 = static_cast<int>(static_cast<long long>(N) * (c + 1) / chunks);
+    cudaStream_t cs = hp->st[c & 1];
+    const size_t oi = img_in * n0, bi = img_in * (n1 - n0), oo = img_out * n0, bo = img_out * (n1 - n0);
+    auto dev = [](void* p, size_t off) { return static_cast<void*>(static_cast<char*>(p) + off); };
+    auto host = [](const void* p, size_t off) { return static_cast<const void*>(static_cast<const char*>(p) + off); };
+    if (cudaMemcpyAsync(dev(q_d, oi), host(q_h, oi), bi, cudaMemcpyHostToDevice, cs) != cudaSuccess ||
+        cudaMemcpyAsync(dev(k_d, oi), host(k_h, oi), bi, cudaMemcpyHostToDevice, cs) != cudaSuccess ||
+        cudaMemcpyAsync(dev(v_d, oi), host(v_h, oi), bi, cudaMemcpyHostToDevice, cs) != cudaSuccess)
+      return HALO_ERR_CUDA;
+    Shape sc = s;
+    sc.N = n1 - n0;
+    rc = attn_device(dev(q_d, oi), dev(k_d, oi), dev(v_d, oi), rel_h_d, rel_w_d, dev(out_d, oo), sc, cs);
+    if (rc != HALO_OK) return rc;
+    if (cudaMemcpyAsync(dev(out_h, oo), dev(out_d, oo), bo, cudaMemcpyDeviceToHost, cs) != cudaSuccess)
+      return HALO_ERR_CUDA;
+  }
+  // work queued on the caller's stream after this call waits for both
+  if (cudaEventRecord(hp->ev_done[0], hp->st[0]) != cudaSuccess ||
+      cudaEventRecord(hp->ev_done[1], hp->st[1]) != cudaSuccess ||
+      cudaStreamWaitEvent(st, hp->ev_done[0], 0) != cudaSuccess ||
+      cudaStreamWaitEvent(st, hp->ev_done[1], 0) != cudaSuccess)
+    return HALO_ERR_CUDA;
   return HALO_OK;
 }
 

@@ -92,12 +92,18 @@ int halo_attn(const void* q, const void* k, const void* v, const void* rel_h, co
 /*
  * halo_attn_host -- the same operation on HOST buffers (end-to-end form).
  *
- * q_h .. rel_w_h: host input pointers (pinned memory is fastest), out_h: host
- * output pointer.  q_d .. out_d: caller-owned device buffers of the same sizes
- * that the call uses as staging; the library allocates nothing.  The call
- * queues host->device copies of the five inputs, the kernel and the
- * device->host copy of the output on `stream` and returns without waiting;
- * synchronise `stream` before reading out_h.
+ * q_h .. rel_w_h: host input pointers (pinned memory is needed for the copies
+ * to overlap), out_h: host output pointer.  q_d .. out_d: caller-owned device
+ * buffers of the same sizes that the call uses as staging; the library
+ * allocates no memory.  The call splits the batch into up to 8 chunks of
+ * whole images and queues, per chunk, the host->device copies of its q, k, v,
+ * the kernel on it and the device->host copy of its output, alternating
+ * between two library-owned streams (created once per device on first use),
+ * so that one chunk's copies overlap the previous chunk's kernel and copies.
+ * The work is ordered after everything queued on `stream` before the call,
+ * and work queued on `stream` after the call waits for all of it; the call
+ * returns without waiting: synchronise `stream` before reading out_h.  Calls
+ * from several host threads are serialised by a library lock.
  */
 int halo_attn_host(const void* q_h, const void* k_h, const void* v_h, const void* rel_h_h, const void* rel_w_h,
                    void* out_h, void* q_d, void* k_d, void* v_d, void* rel_h_d, void* rel_w_d, void* out_d,

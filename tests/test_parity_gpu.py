@@ -233,6 +233,28 @@ def test_host_entry_point_matches_device_entry_point():
     assert torch.equal(out_h, ref.cpu())
 
 
+@pytest.mark.parametrize("n", [5, 13])
+def test_host_entry_point_pipelined_chunks(n):
+    """The host entry point splits the batch into chunks on two library
+    streams: ragged chunk sizes give the same result as the device entry
+    point, and work queued on the caller's stream afterwards sees it all."""
+    wl = custom("e2e", N=n, H=16, W=24, heads=4, dim_head=32, block=8, halo=2, stride=1, dtype="bf16")
+    inputs = [t.pin_memory() for t in make_inputs(wl, seed=n)]
+    h = _lib()
+    staging = {nm: torch.empty_like(t, device="cuda") for nm, t in zip(("q", "k", "v", "rel_h", "rel_w"), inputs)}
+    staging["out"] = torch.empty((wl.N, wl.H, wl.W, wl.C), dtype=torch.bfloat16, device="cuda")
+    out_h = torch.empty((wl.N, wl.H, wl.W, wl.C), dtype=torch.bfloat16).pin_memory()
+    s = torch.cuda.Stream()
+    with torch.cuda.stream(s):
+        h.attn_host(*inputs, out_h, staging, block=8, halo=2)
+        after = staging["out"].float() * 1.0  # queued on the caller's stream after the call
+    s.synchronize()
+    ref = h.attn(*[t.cuda() for t in inputs], block=8, halo=2)
+    torch.cuda.synchronize()
+    assert torch.equal(out_h, ref.cpu())
+    assert torch.equal(after, ref.float())
+
+
 def test_side_stream():
     wl = custom("stream", N=2, H=16, W=24, heads=8, dim_head=32, block=8, halo=2, stride=1, dtype="bf16")
     inputs = make_inputs(wl, seed=11)
