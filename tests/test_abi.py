@@ -107,6 +107,8 @@ def test_kernel_names():
     assert name(32, 64, 64, 8, 16, 8, 3, 1, 1) == "halo_fwd_tc2<16,14>"
     assert name(64, 32, 32, 8, 64, 8, 3, 1, 1) == "halo_fwd_tc4<64,14>"
     assert name(64, 24, 32, 8, 64, 8, 3, 1, 1) == "halo_fwd_tc<64,14,1>"  # odd number of block rows
+    assert name(2, 16, 24, 3, 16, 8, 3, 1, 1) == "halo_fwd_tc<16,14,1>"   # odd head count
+    assert name(2, 32, 48, 3, 16, 16, 2, 1, 1) == "halo_fwd_tc3<16,20>"
     assert name(64, 64, 64, 8, 32, 8, 3, 2, 1) == "halo_fwd_tc<32,14,2>"
     assert name(16, 128, 128, 8, 32, 16, 4, 1, 1) == "halo_fwd_tc3<32,24>"
     assert name(1, 16, 16, 2, 32, 4, 1, 1, 0) == "halo_fwd_simt<float,32>"

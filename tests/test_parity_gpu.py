@@ -106,6 +106,11 @@ for d in (16, 32, 64):
         for stride in (1, 2):
             CASES.append(dict(N=2, H=24, W=40, heads=8 if d < 64 else 4, dim_head=d, block=8, halo=halo,
                               stride=stride))
+# odd head counts at stride 1 (d = 16, 32) go to the one-head-per-item kernel
+CASES += [
+    dict(N=2, H=16, W=24, heads=3, dim_head=16, block=8, halo=3, stride=1),
+    dict(N=2, H=16, W=24, heads=3, dim_head=32, block=8, halo=2, stride=1),
+]
 # dim_head 64 with an even number of block rows: the kernel that pairs two
 # vertically adjacent blocks (every window, one pair and several pairs)
 for halo in (0, 1, 2, 3):
