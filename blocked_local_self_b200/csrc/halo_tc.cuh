@@ -16,10 +16,12 @@
 //     the w x 16 window of K and of V (w = 8 + 2*halo rows; the window row is
 //     padded from w to 16 keys so every window row is one 32-byte swizzle
 //     chunk of the P operand).  Keys outside the image arrive as zeros.
-//   * warp 9 (one lane) issues tcgen05.mma: S = Q K^T (M=64, N=16w, bf16 in,
-//     f32 in TMEM), G = Q R^T with R = [rel_h; rel_w] (the 2(2w-1) relative
-//     dot products of every query), and after the softmax O = P V (and, for
-//     d = 16, the row sums through a ones tile appended to V).
+//   * warp 9 (one lane) issues S = Q K^T (tcgen05.mma, M=64, bf16 in, f32 in
+//     TMEM) and warp 10 G = Q R^T with R = [rel_h; rel_w] (the 2(2w-1)
+//     relative dot products of every query); after the softmax, warps
+//     q < NST of the owning warpgroup each issue a share of O = P V (window
+//     rows of one head) into their own accumulator, summed in the epilogue
+//     (for d = 16 the row sums come from a ones tile appended to V).
 //   * warps 0-3 and 4-7 are two softmax warpgroups that take alternate items;
 //     each owns one half of every TMEM lane quadrant (lanes 0-15 or 16-31), so
 //     the MMAs of one item overlap the softmax of the other.  A query row is
@@ -49,8 +51,8 @@ using namespace sm100;
 constexpr int kBlock = 8;         // query block side handled by this kernel
 constexpr int kRowKeys = 16;      // P / V window row pitch in keys (w padded to 16)
 constexpr int kThreads = 384;     // 2 softmax warpgroups + 1 producer warpgroup
-constexpr int kTmaWarp = 8;       // producer warpgroup: warp 8 TMA, warp 9 MMA,
-constexpr int kMmaWarp = 9;       // warps 10-11 idle
+constexpr int kTmaWarp = 8;       // producer warpgroup: warp 8 TMA, warps 9-10 MMA,
+constexpr int kMmaWarp = 9;       // warp 11 idle
 // Register split (setmaxnreg): the kernel launches with kLaunchRegs per thread
 // (3 warps per SM sub-partition cap it at 168); the producer warpgroup gives
 // registers back and the softmax warpgroups take more.  The sum stays within
