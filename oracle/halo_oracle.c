@@ -32,6 +32,11 @@
  *                     is inverted; the paper pads the border);
  *   stride 2        = queries at even in-block offsets 0,2,..,b-2; the
  *                     relative index uses the pixel's in-block offset.
+ *                     The tests pin stride 2 to stride 1 sampled at even
+ *                     pixels, but no page fixes the phase or the index
+ *                     convention: parity unpinned against the pages for
+ *                     this choice.  The absolute table offset is pinned only
+ *                     to the blog's rel_to_abs recipe.
  *
  * For each output pixel and head the oracle evaluates the defining formula
  * directly: every window key's logit, the maximum over in-image keys, the
