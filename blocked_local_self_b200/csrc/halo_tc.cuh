@@ -112,6 +112,10 @@ struct Cfg {
   static constexpr SmemSwizzle SW = (ROWB == 32) ? SW_32B : (ROWB == 64 ? SW_64B : SW_128B);
   static constexpr uint32_t SBO = 8 * ROWB;               // 8-row core-matrix group stride
   static constexpr int NROW = WIN / 2;                    // window rows per thread
+  // Stride 2 with fewer than 4 parts: warpgroup 1's parts go to the upper
+  // lane quadrants (its Q view starts QSHIFT rows earlier), so the two
+  // warpgroups' active warps sit on different schedulers.
+  static constexpr int QSHIFT = (STRIDE == 2 && PARTS <= 2) ? 32 : 0;
   // A.V issue streams: warp q < NST of the warpgroup issues a share of the
   // PARTS x WIN K-steps (part q / SPP, window rows of slice q % SPP) into its
   // own accumulator O_q at slot column q * O_COLS.
@@ -342,7 +346,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!is_g) {
 #pragma unroll 1
           for (int part = 0; part < C::PARTS; ++part) {
-            const uint32_t qa = smem_addr(st + ((STRIDE == 1) ? 0 : (48 + 48 * part) * C::ROWB));
+            const uint32_t qa =
+                smem_addr(st + ((STRIDE == 1) ? 0 : (48 + 48 * part - g * C::QSHIFT) * C::ROWB));
             const uint32_t ka = smem_addr(st + C::Q_BYTES + part * C::K_TILE);
             for (int ks = 0; ks < D / 16; ++ks) {
               mma_f16_ss(dst, smem_desc(qa + 32 * ks, 16, C::SBO, C::SW),
@@ -355,7 +360,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t ra = smem_addr(sR);
 #pragma unroll 1
         for (int part = 0; part < C::PARTS; ++part) {
-          const uint32_t qa = smem_addr(st + ((STRIDE == 1) ? 0 : (48 + 48 * part) * C::ROWB));
+          const uint32_t qa = smem_addr(st + ((STRIDE == 1) ? 0 : (48 + 48 * part - g * C::QSHIFT) * C::ROWB));
           for (int ks = 0; ks < D / 16; ++ks) {
             mma_f16_ss(dst + kTmemG, smem_desc(qa + 32 * ks, 16, C::SBO, C::SW),
                        smem_desc(ra + 32 * ks, 16, C::SBO, C::SW), idG, (part | ks) != 0);
@@ -393,7 +398,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int wq = warp & 3;          // TMEM lane quadrant
     const int half = lane >> 4;       // 0: even window rows, 1: odd window rows
     const int r16 = lane & 15;        // row within the quadrant
-    const bool active = (STRIDE == 1) || (wq < C::PARTS);
+    const int part_w = wq - g * (C::QSHIFT / 16);   // this warp's head part at stride 2
+    const bool active = (STRIDE == 1) || (part_w >= 0 && part_w < C::PARTS);
     const uint32_t tq = tmem + (static_cast<uint32_t>(32 * wq + 16 * g) << 16);
     uint8_t* pt = sP + g * C::P_TILE;
     float* scr = sScratch + (warp * 32) * C::SCRATCH_LINE;  // this warp's 32 lines
@@ -419,7 +425,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
       for (int t = 0; t < D / 2; ++t) o[t] = 0.f;
       if (active) {
-        const int q0 = (STRIDE == 1) ? 0 : wq * C::SPP;
+        const int q0 = (STRIDE == 1) ? 0 : part_w * C::SPP;
         if constexpr (D == 16) l = 0.f;
 #pragma unroll 1
         for (int q = q0; q < q0 + ((STRIDE == 1) ? C::NST : C::SPP); ++q) {
@@ -458,7 +464,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       __syncwarp();
       if (lane == 0) mbar_arrive(&bar_tfree[b]);
       if (active) {
-        const int head = ic.grp * C::PARTS + ((STRIDE == 1) ? 0 : wq);
+        const int head = ic.grp * C::PARTS + ((STRIDE == 1) ? 0 : part_w);
         const float inv = 1.0f / l;
         uint32_t pk[D / 4];
 #pragma unroll
