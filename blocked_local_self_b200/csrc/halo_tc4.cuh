@@ -13,21 +13,27 @@
 // [0, w*w) and block B's is keys [8w, 8w + w*w), both contiguous.  With
 // d = 64 two heads' windows would not fit two pipeline stages in shared
 // memory; two blocks' union does (96 KB per stage).
-//   * TMA (warp 8): Q_A, Q_B [64 x d] and the union K, V tiles.
-//   * S MMA (warp 9): per block M=64, N=200 (its window) into its TMEM lane
-//     half (block A lanes 0-15 of each quadrant, block B 16-31).
-//   * G MMA (warp 10): per block G = Q R^T (N=56, R = [rel_h; 0; rel_w; 0]
+//   * TMA (warp 8): Q_A, Q_B [64 x d] and the union K tile, and one item
+//     later the union V tile (separate barriers, so Q/K stages free early).
+//   * S MMAs (block A on warp 9, block B on warp 11): per block M=64, N=200
+//     (its window) into its TMEM lane half (block A lanes 0-15 of each
+//     quadrant, block B 16-31).
+//   * G MMAs (warp 10, own barrier): per block G = Q R^T (N=56, R = [rel_h; 0; rel_w; 0]
 //     written once) into slot columns [200, 256); each thread takes the
 //     w + w relative logits of its query by a TMEM column shift and selects.
-//   * softmax (one thread per TMEM lane = one query row): pass 1 takes an
-//     upper bound of the row maximum, max over keys of c*S plus the maximum
-//     of c*rel_w and of c*rel_h (at most a few units above the exact one);
+//   * softmax (one thread per TMEM lane = one query row): pass 1 takes the
+//     raw S maximum of every window row (before G is needed), then an upper
+//     bound of the row maximum, max over rows of c*S_max + c*rel_h plus the
+//     maximum of c*rel_w (at most a few units above the exact one);
 //     pass 2 the exponentials (MUFU and the FMA-pipe cubic), the row sum and
 //     bf16 P written back over the S columns.
-//   * A.V (warp 0): O = P [V_A | V_B], M=128, N=2d: the B operand's second
-//     swizzle atom is block B's window, 8w rows below block A's in the same
-//     V tile.  Block A's rows use columns [0, d), block B's [d, 2d).
-//   * epilogue: O / l, bf16, NHWC.
+//   * A.V: four independent MMA chains, one per softmax warp: warp q takes
+//     block q & 1 and key half q >> 1, O_h = P_blk[:, keys of half h]
+//     V_blk[keys of half h] with M=64, N=d, A (P) read from the block's TMEM
+//     lane half and the accumulator in the same lane half (block B's window
+//     8w rows below block A's in the V tile).  The two halves' accumulators
+//     share one maximum, so O = O_0 + O_1.
+//   * epilogue: (O_0 + O_1) / l, bf16, NHWC.
 // Two softmax warpgroups take alternate items; every wait is bounded.
 #pragma once
 
@@ -60,10 +66,11 @@ using tc2::tmem_st_x8;
 using tc2::tmem_wait_st;
 
 constexpr int kBlock = 8;
-constexpr int kThreads = 384;   // warpgroups 0-1 softmax, warp 8 TMA, warp 9 S MMA, warp 10 G MMA
+constexpr int kThreads = 384;   // warpgroups 0-1 softmax, warp 8 TMA, warps 9/11 S MMAs, warp 10 G MMAs
 constexpr int kTmaWarp = 8;
 constexpr int kMmaWarp = 9;
 constexpr int kGMmaWarp = 10;
+constexpr int kSBMmaWarp = 11;
 constexpr int kSoftmaxRegs = tc::kSoftmaxRegs;
 constexpr int kProducerRegs = tc::kProducerRegs;
 constexpr uint32_t kTmemCols = 512;
@@ -98,10 +105,12 @@ struct Cfg {
   static constexpr int K_TILE = (KROWS * ROWB + 1023) / 1024 * 1024;
   static constexpr int STAGE_BYTES = 2 * Q_TILE + 2 * K_TILE;
   static constexpr int R_TILE = (kRRows * ROWB + 1023) / 1024 * 1024;
-  static constexpr int TX_BYTES = (2 * 64 + 2 * UROWS) * ROWB;
+  static constexpr int TX_QK = (2 * 64 + UROWS) * ROWB;  // Q_A, Q_B and the K union tile
+  static constexpr int TX_V = UROWS * ROWB;               // the V union tile
   static constexpr int PCOLS = KP / 2;                    // packed bf16 P columns
   static constexpr int O_BASE = (PCOLS + 7) / 8 * 8;      // first O column
-  static constexpr int O_N = 2 * D;                       // [V_A | V_B]
+  static constexpr int KHALF = (KSTEPS + 1) / 2;          // A.V K-steps of key half 0
+  static constexpr int O_N = 2 * D;                       // O_0 | O_1, each in both lane halves
   static constexpr SmemSwizzle SW = (ROWB == 32) ? SW_32B : (ROWB == 64 ? SW_64B : SW_128B);
   static constexpr uint32_t SBO = 8 * ROWB;
   static constexpr int HALO = (WIN - kBlock) / 2;
@@ -250,13 +259,19 @@ __global__ void __launch_bounds__(kThreads, 1)
   // stage layout: [Q_A][Q_B][K union][V union]
   constexpr int OFF_QA = 0, OFF_QB = C::Q_TILE, OFF_K = 2 * C::Q_TILE, OFF_V = OFF_K + C::K_TILE;
 
-  __shared__ __align__(8) uint64_t bar_full[4];
-  __shared__ __align__(8) uint64_t bar_empty[4];
-  __shared__ __align__(8) uint64_t bar_sfull[2];   // count 2: the S and the G MMAs of the item
+  // Q/K and V of a stage have their own barriers: Q and K are released when
+  // the S and G MMAs finish, long before the A.V releases V, so the next
+  // items' Q/K loads are in flight during the softmax.
+  __shared__ __align__(8) uint64_t bar_fqk[4];
+  __shared__ __align__(8) uint64_t bar_fv[4];
+  __shared__ __align__(8) uint64_t bar_eqk[4];  // count 3: S_A, S_B, G
+  __shared__ __align__(8) uint64_t bar_ev[4];   // count 4: the A.V chains
+  __shared__ __align__(8) uint64_t bar_sfull[2];   // count 2: the two blocks' S MMAs
+  __shared__ __align__(8) uint64_t bar_gfull[2];
   __shared__ __align__(8) uint64_t bar_ofull[2];
   __shared__ __align__(8) uint64_t bar_tfree[2];   // count 4: the warpgroup read its slot's O
   __shared__ __align__(8) uint64_t bar_pready[2];  // count 4, waited by every warp of the warpgroup
-  __shared__ __align__(8) uint64_t bar_done[2];
+  __shared__ __align__(8) uint64_t bar_done[3];
   __shared__ __align__(8) uint64_t bar_pvdone[2];
   __shared__ uint32_t tmem_base_sh;
   __shared__ int abort_flag;
@@ -269,17 +284,21 @@ __global__ void __launch_bounds__(kThreads, 1)
   // ---------------------------------------------------------------- set-up
   if (tid == 0) {
     for (int i = 0; i < S; ++i) {
-      mbar_init(&bar_full[i], 1);
-      mbar_init(&bar_empty[i], 1);
+      mbar_init(&bar_fqk[i], 1);
+      mbar_init(&bar_fv[i], 1);
+      mbar_init(&bar_eqk[i], 3);
+      mbar_init(&bar_ev[i], 4);
     }
     for (int g = 0; g < 2; ++g) {
       mbar_init(&bar_sfull[g], 2);
-      mbar_init(&bar_ofull[g], 1);
+      mbar_init(&bar_ofull[g], 4);
       mbar_init(&bar_tfree[g], 4);
       mbar_init(&bar_pready[g], 4);
       mbar_init(&bar_done[g], 1);
-      mbar_init(&bar_pvdone[g], 1);
+      mbar_init(&bar_gfull[g], 1);
+      mbar_init(&bar_pvdone[g], 4);
     }
+    mbar_init(&bar_done[2], 1);
     abort_flag = 0;
     fence_mbar_init();
   }
@@ -320,31 +339,48 @@ __global__ void __launch_bounds__(kThreads, 1)
   asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kProducerRegs));
   if (warp == kTmaWarp) {
     // ------------------------------------------------------------ TMA producer
+    // issue order QK(0), QK(1), V(0), QK(2), V(1), ...: the Q/K of an item
+    // go out one item ahead of the V it does not need until its A.V
     if (lane == 0) {
-      int issued = 0;
-      for (int k = 0; k < my_items; ++k) {
-        const int s = k % S;
-        if (k >= S && !mbar_wait(&bar_empty[s], ((k / S) - 1) & 1, kWaitNs, &abort_flag)) {
-          if (!abort_flag) record_timeout(&abort_flag);
-          break;
+      int nqk = 0, nv = 0;
+      for (int t = 0; t <= my_items; ++t) {
+        if (t < my_items) {
+          const int s = t % S;
+          if (t >= S && !mbar_wait(&bar_eqk[s], ((t / S) - 1) & 1, kWaitNs, &abort_flag)) {
+            if (!abort_flag) record_timeout(&abort_flag);
+            break;
+          }
+          const ItemCoord ic = item_coord(blockIdx.x + t * gridDim.x, p.heads, p.nbx, p.npy);
+          uint8_t* st = sStage + s * C::STAGE_BYTES;
+          const int x0 = ic.bx * kBlock, y0 = ic.py * 2 * kBlock;
+          mbar_arrive_expect_tx(&bar_fqk[s], C::TX_QK);
+          tma_load_4d(st + OFF_QA, &tmap_q, &bar_fqk[s], ic.head * D, x0, y0, ic.n);
+          tma_load_4d(st + OFF_QB, &tmap_q, &bar_fqk[s], ic.head * D, x0, y0 + kBlock, ic.n);
+          tma_load_4d(st + OFF_K, &tmap_k, &bar_fqk[s], ic.head * D, x0 - p.halo, y0 - p.halo, ic.n);
+          nqk = t + 1;
         }
-        const ItemCoord ic = item_coord(blockIdx.x + k * gridDim.x, p.heads, p.nbx, p.npy);
-        uint8_t* st = sStage + s * C::STAGE_BYTES;
-        const int x0 = ic.bx * kBlock, y0 = ic.py * 2 * kBlock;
-        mbar_arrive_expect_tx(&bar_full[s], C::TX_BYTES);
-        tma_load_4d(st + OFF_QA, &tmap_q, &bar_full[s], ic.head * D, x0, y0, ic.n);
-        tma_load_4d(st + OFF_QB, &tmap_q, &bar_full[s], ic.head * D, x0, y0 + kBlock, ic.n);
-        tma_load_4d(st + OFF_K, &tmap_k, &bar_full[s], ic.head * D, x0 - p.halo, y0 - p.halo, ic.n);
-        tma_load_4d(st + OFF_V, &tmap_v, &bar_full[s], ic.head * D, x0 - p.halo, y0 - p.halo, ic.n);
-        issued = k + 1;
+        if (t >= 1) {
+          const int k = t - 1, s = k % S;
+          if (k >= S && !mbar_wait(&bar_ev[s], ((k / S) - 1) & 1, kWaitNs, &abort_flag)) {
+            if (!abort_flag) record_timeout(&abort_flag);
+            break;
+          }
+          const ItemCoord ic = item_coord(blockIdx.x + k * gridDim.x, p.heads, p.nbx, p.npy);
+          uint8_t* st = sStage + s * C::STAGE_BYTES;
+          const int x0 = ic.bx * kBlock, y0 = ic.py * 2 * kBlock;
+          mbar_arrive_expect_tx(&bar_fv[s], C::TX_V);
+          tma_load_4d(st + OFF_V, &tmap_v, &bar_fv[s], ic.head * D, x0 - p.halo, y0 - p.halo, ic.n);
+          nv = k + 1;
+        }
       }
       if (abort_flag) {
-        for (int k = (issued > S ? issued - S : 0); k < issued; ++k)
-          mbar_wait(&bar_full[k % S], (k / S) & 1, kWaitNs);
+        // loads still in flight land before the block exits
+        for (int k = (nqk > S ? nqk - S : 0); k < nqk; ++k) mbar_wait(&bar_fqk[k % S], (k / S) & 1, kWaitNs);
+        for (int k = (nv > S ? nv - S : 0); k < nv; ++k) mbar_wait(&bar_fv[k % S], (k / S) & 1, kWaitNs);
       }
     }
-  } else if (warp == kMmaWarp || warp == kGMmaWarp) {
-    // ------------------------------------------------------------ S (warp 9) and G (warp 10) MMAs
+  } else {
+    // ------------------------------------------------------------ S (warps 9, 11) and G (warp 10) MMAs
     const bool is_g = (warp == kGMmaWarp);
     if (lane == 0) {
       const uint32_t idS = idesc_bf16_f32(64, C::NS, false);
@@ -352,7 +388,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint32_t ra = smem_addr(sR);
       for (int k = 0; k < my_items; ++k) {
         const int s = k % S, g = k & 1;
-        if (!mbar_wait(&bar_full[s], (k / S) & 1, kWaitNs, &abort_flag) ||
+        if (!mbar_wait(&bar_fqk[s], (k / S) & 1, kWaitNs, &abort_flag) ||
             (k >= 2 && !mbar_wait(&bar_tfree[g], ((k >> 1) - 1) & 1, kWaitNs, &abort_flag))) {
           if (!abort_flag) record_timeout(&abort_flag);
           break;
@@ -361,7 +397,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint8_t* st = sStage + s * C::STAGE_BYTES;
         const uint32_t slot = tmem + g * kSlotCols;
 #pragma unroll 1
-        for (int blk = 0; blk < 2; ++blk) {
+        for (int blk = (warp == kSBMmaWarp); blk < (warp == kMmaWarp ? 1 : 2); ++blk) {
           const uint32_t qa = smem_addr(st + (blk ? OFF_QB : OFF_QA));
           const uint32_t dst = slot + (static_cast<uint32_t>(blk * 16) << 16);
           if (is_g) {
@@ -377,9 +413,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                          idS, ks != 0);
           }
         }
-        mma_commit(&bar_sfull[g]);
+        mma_commit(is_g ? &bar_gfull[g] : &bar_sfull[g]);
+        mma_commit(&bar_eqk[s]);
       }
-      const int w = is_g ? 1 : 0;
+      const int w = warp - kMmaWarp;
       mma_commit(&bar_done[w]);
       mbar_wait(&bar_done[w], 0, kWaitNs);
     }
@@ -402,7 +439,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t ts = slot + (static_cast<uint32_t>(32 * wq) << 16);
     const float c = p.c;
     const int C_all = p.heads * D;
-    const uint32_t idO = idesc_bf16_f32(128, C::O_N, true);
+    const uint32_t idO = idesc_bf16_f32(64, D, true);
 
     int j = 0;
     for (int k = g; k < my_items; k += 2, ++j) {
@@ -415,6 +452,16 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int by = 2 * ic.py + blk;
       const int y0 = by * kBlock - p.halo, x0 = ic.bx * kBlock - p.halo;
 
+      // ---- pass 1: per window row the maximum of the raw S values
+      float rm[WIN];
+#pragma unroll
+      for (int r = 0; r < WIN; ++r) rm[r] = -INFINITY;
+      row_max_all<WIN, C>(ts, rm, std::make_integer_sequence<int, C::NCHUNK>{});
+      if (!mbar_wait(&bar_gfull[g], j & 1, kWaitNs, &abort_flag)) {
+        if (!abort_flag) record_timeout(&abort_flag);
+        break;
+      }
+      tc_fence_after();
       // ---- relative logits of this query, in log2 units:
       //   rh[kr] = c * q.rel_h[kr - qy + w - 1], rw[kc] = c * q.rel_w[kc - qx + w - 1]
       float rh[WIN], rw[WIN], rwz[WIN];  // rwz: rel_w logits unscaled (S units)
@@ -449,11 +496,6 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
 
-      // ---- pass 1: upper bound of the row maximum (log2 units)
-      float rm[WIN];
-#pragma unroll
-      for (int r = 0; r < WIN; ++r) rm[r] = -INFINITY;
-      row_max_all<WIN, C>(ts, rm, std::make_integer_sequence<int, C::NCHUNK>{});
       float mw = -INFINITY;
 #pragma unroll
       for (int kc = 0; kc < WIN; ++kc) mw = fmaxf(mw, rw[kc]);
@@ -476,16 +518,21 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       tc_fence_after();
 
-      // ---- A.V: O = P [V_A | V_B] (warp 0)
+      // ---- A.V: warp wq issues block (wq & 1), key half (wq >> 1)
       const int s = k % S;
-      if (wq == 0 && lane == 0) {
-        const uint32_t va = smem_addr(sStage + s * C::STAGE_BYTES + OFF_V);
+      if (lane == 0 && !mbar_wait(&bar_fv[s], (k / S) & 1, kWaitNs, &abort_flag)) {
+        if (!abort_flag) record_timeout(&abort_flag);
+      } else if (lane == 0) {
+        const int ab = wq & 1, hf = wq >> 1;
+        const int kb = hf ? C::KHALF : 0, ke = hf ? C::KSTEPS : C::KHALF;
+        const uint32_t lanes = static_cast<uint32_t>(16 * ab) << 16;
+        const uint32_t va = smem_addr(sStage + s * C::STAGE_BYTES + OFF_V) + ab * C::BOFF * C::ROWB;
 #pragma unroll 1
-        for (int kk = 0; kk < C::KSTEPS; ++kk)
-          mma_f16_ts(slot + C::O_BASE, slot + 8 * kk,
-                     smem_desc(va + kk * 16 * C::ROWB, C::BOFF * C::ROWB, C::SBO, C::SW), idO, kk != 0);
+        for (int kk = kb; kk < ke; ++kk)
+          mma_f16_ts(slot + lanes + C::O_BASE + hf * D, slot + lanes + 8 * kk,
+                     smem_desc(va + kk * 16 * C::ROWB, 16, C::SBO, C::SW), idO, kk != kb);
         mma_commit(&bar_ofull[g]);
-        mma_commit(&bar_empty[s]);
+        mma_commit(&bar_ev[s]);
       }
       __syncwarp();
 
@@ -496,8 +543,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       tc_fence_after();
       {
-        // the whole warp loads both blocks' columns; this thread keeps [0, D)
-        // for block A, [D, 2D) for block B
+        // this thread's row of both key halves' accumulators
         float o[D];
 #pragma unroll
         for (int e = 0; e < D; e += 32) {
@@ -506,7 +552,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           tmem_ld_x32(ts + C::O_BASE + D + e, tb);
           tmem_wait_ld();
 #pragma unroll
-          for (int i = 0; i < 32; ++i) o[e + i] = blk ? tb[i] : ta[i];
+          for (int i = 0; i < 32; ++i) o[e + i] = ta[i] + tb[i];
         }
         tc_fence_before();
         __syncwarp();
@@ -522,8 +568,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           reinterpret_cast<uint4*>(dst)[t] = make_uint4(pk[4 * t], pk[4 * t + 1], pk[4 * t + 2], pk[4 * t + 3]);
       }
     }
-    // A.V MMAs warp 0 issued are complete before TMEM is released
-    if (wq == 0 && lane == 0) {
+    // A.V MMAs this warp issued are complete before TMEM is released
+    if (lane == 0) {
       mma_commit(&bar_pvdone[g]);
       mbar_wait(&bar_pvdone[g], 0, kWaitNs);
     }
