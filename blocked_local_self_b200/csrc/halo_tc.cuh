@@ -16,6 +16,8 @@
 //     the w x 16 window of K and of V (w = 8 + 2*halo rows; the window row is
 //     padded from w to 16 keys so every window row is one 32-byte swizzle
 //     chunk of the P operand).  Keys outside the image arrive as zeros.
+//     Q and K travel on their own stage barrier, one item ahead of V, and
+//     are released as soon as the S and G MMAs finish.
 //   * warp 9 (one lane) issues S = Q K^T (tcgen05.mma, M=64, bf16 in, f32 in
 //     TMEM) and warp 10 G = Q R^T with R = [rel_h; rel_w] (the 2(2w-1)
 //     relative dot products of every query); after the softmax, warps
@@ -101,7 +103,8 @@ struct Cfg {
   static constexpr int Q_BYTES = QBUF_ROWS * ROWB;
   static constexpr int STAGE_RAW = Q_BYTES + PARTS * (K_TILE + V_TILE);
   static constexpr int STAGE_BYTES = (STAGE_RAW + 1023) / 1024 * 1024;
-  static constexpr int TX_BYTES = PARTS * (QROWS_PER_HEAD * ROWB + (KS + KP) * ROWB);
+  static constexpr int TX_QK = PARTS * (QROWS_PER_HEAD + KS) * ROWB;  // Q and K of every part
+  static constexpr int TX_V = PARTS * KP * ROWB;                       // V of every part
   static constexpr int P_TILE = WIN * 2048;               // 64 rows x 16 keys x 2 B per window row
   static constexpr int R_TILE = kGCols * ROWB;            // [rel_h; 0; rel_w; 0] B operand
   static constexpr int SCRATCH_LINE = 36;                 // floats per (row, half) line of the gather scratch
@@ -209,8 +212,13 @@ __global__ void __launch_bounds__(kThreads, 1)
   // positive leading byte offset from any V tile
   uint8_t* sOnes = sStage + p.stages * C::STAGE_BYTES;
 
-  __shared__ __align__(8) uint64_t bar_full[8];
-  __shared__ __align__(8) uint64_t bar_empty[8];
+  // Q/K and V of a stage have their own barriers: Q and K are released when
+  // the S and G MMAs finish, long before the A.V releases V, so the next
+  // items' Q/K loads are in flight during the softmax.
+  __shared__ __align__(8) uint64_t bar_fqk[8];
+  __shared__ __align__(8) uint64_t bar_fv[8];
+  __shared__ __align__(8) uint64_t bar_eqk[8];  // count 2: the S and the G MMAs
+  __shared__ __align__(8) uint64_t bar_ev[8];   // count NST: the A.V streams
   __shared__ __align__(8) uint64_t bar_sfull[4];   // index 2*g + slot
   __shared__ __align__(8) uint64_t bar_pfull[4];
   __shared__ __align__(8) uint64_t bar_ofull[4];
@@ -227,8 +235,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   // ---------------------------------------------------------------- set-up
   if (tid == 0) {
     for (int i = 0; i < S; ++i) {
-      mbar_init(&bar_full[i], 1);
-      mbar_init(&bar_empty[i], C::NST);
+      mbar_init(&bar_fqk[i], 1);
+      mbar_init(&bar_fv[i], 1);
+      mbar_init(&bar_eqk[i], 2);
+      mbar_init(&bar_ev[i], C::NST);
     }
     for (int b = 0; b < 4; ++b) {
       mbar_init(&bar_sfull[b], 2);  // the S MMAs (warp 9) and the G MMAs (warp 10)
@@ -300,35 +310,54 @@ __global__ void __launch_bounds__(kThreads, 1)
   asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kProducerRegs));
   if (warp == kTmaWarp) {
     // ------------------------------------------------------------ TMA producer
+    // issue order QK(0), QK(1), V(0), QK(2), V(1), ...: the Q/K of an item
+    // go out one item ahead of the V it does not need until its A.V
     if (lane == 0) {
-      int issued = 0;
-      for (int k = 0; k < my_items; ++k) {
-        const int s = k % S;
-        if (k >= S && !mbar_wait(&bar_empty[s], ((k / S) - 1) & 1, kWaitNs, &abort_flag)) {
-          if (!abort_flag) record_timeout(&abort_flag);
-          break;
-        }
-        const ItemCoord ic = item_coord(blockIdx.x + k * gridDim.x, groups, p.nbx, p.nby);
-        uint8_t* st = sStage + s * C::STAGE_BYTES;
-        mbar_arrive_expect_tx(&bar_full[s], C::TX_BYTES);
+      int nqk = 0, nv = 0;
+      for (int t = 0; t <= my_items; ++t) {
+        if (t < my_items) {
+          const int s = t % S;
+          if (t >= S && !mbar_wait(&bar_eqk[s], ((t / S) - 1) & 1, kWaitNs, &abort_flag)) {
+            if (!abort_flag) record_timeout(&abort_flag);
+            break;
+          }
+          const ItemCoord ic = item_coord(blockIdx.x + t * gridDim.x, groups, p.nbx, p.nby);
+          uint8_t* st = sStage + s * C::STAGE_BYTES;
+          mbar_arrive_expect_tx(&bar_fqk[s], C::TX_QK);
 #pragma unroll 1
-        for (int part = 0; part < C::PARTS; ++part) {
-          const int head = ic.grp * C::PARTS + part;
-          uint8_t* qdst = st + ((STRIDE == 1) ? 0 : (48 + 64 * part) * C::ROWB);
-          tma_load_4d(qdst, &tmap_q, &bar_full[s], head * D, ic.bx * kBlock, ic.by * kBlock, ic.n);
-          uint8_t* kdst = st + C::Q_BYTES + part * C::K_TILE;
-          uint8_t* vdst = st + C::Q_BYTES + C::PARTS * C::K_TILE + part * C::V_TILE;
-          tma_load_4d(kdst, &tmap_k, &bar_full[s], head * D, ic.bx * kBlock - p.halo, ic.by * kBlock - p.halo,
-                      ic.n);
-          tma_load_4d(vdst, &tmap_v, &bar_full[s], head * D, ic.bx * kBlock - p.halo, ic.by * kBlock - p.halo,
-                      ic.n);
+          for (int part = 0; part < C::PARTS; ++part) {
+            const int head = ic.grp * C::PARTS + part;
+            uint8_t* qdst = st + ((STRIDE == 1) ? 0 : (48 + 64 * part) * C::ROWB);
+            tma_load_4d(qdst, &tmap_q, &bar_fqk[s], head * D, ic.bx * kBlock, ic.by * kBlock, ic.n);
+            uint8_t* kdst = st + C::Q_BYTES + part * C::K_TILE;
+            tma_load_4d(kdst, &tmap_k, &bar_fqk[s], head * D, ic.bx * kBlock - p.halo, ic.by * kBlock - p.halo,
+                        ic.n);
+          }
+          nqk = t + 1;
         }
-        issued = k + 1;
+        if (t >= 1) {
+          const int k = t - 1, s = k % S;
+          if (k >= S && !mbar_wait(&bar_ev[s], ((k / S) - 1) & 1, kWaitNs, &abort_flag)) {
+            if (!abort_flag) record_timeout(&abort_flag);
+            break;
+          }
+          const ItemCoord ic = item_coord(blockIdx.x + k * gridDim.x, groups, p.nbx, p.nby);
+          uint8_t* st = sStage + s * C::STAGE_BYTES;
+          mbar_arrive_expect_tx(&bar_fv[s], C::TX_V);
+#pragma unroll 1
+          for (int part = 0; part < C::PARTS; ++part) {
+            const int head = ic.grp * C::PARTS + part;
+            uint8_t* vdst = st + C::Q_BYTES + C::PARTS * C::K_TILE + part * C::V_TILE;
+            tma_load_4d(vdst, &tmap_v, &bar_fv[s], head * D, ic.bx * kBlock - p.halo, ic.by * kBlock - p.halo,
+                        ic.n);
+          }
+          nv = k + 1;
+        }
       }
       if (abort_flag) {
         // let loads that are still in flight land before the CTA exits
-        for (int k = (issued > S ? issued - S : 0); k < issued; ++k)
-          mbar_wait(&bar_full[k % S], (k / S) & 1, kWaitNs);
+        for (int k = (nqk > S ? nqk - S : 0); k < nqk; ++k) mbar_wait(&bar_fqk[k % S], (k / S) & 1, kWaitNs);
+        for (int k = (nv > S ? nv - S : 0); k < nv; ++k) mbar_wait(&bar_fv[k % S], (k / S) & 1, kWaitNs);
       }
     }
   } else if (warp == kMmaWarp || warp == kMmaWarp + 1) {
@@ -355,6 +384,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
           }
           mma_commit(&bar_sfull[2 * g + sl]);
+          mma_commit(&bar_eqk[s]);
           return;
         }
         const uint32_t ra = smem_addr(sR);
@@ -367,11 +397,12 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
         mma_commit(&bar_sfull[2 * g + sl]);
+        mma_commit(&bar_eqk[s]);
       };
       // S(k) needs its stage loaded and the slot's previous item (k - 4)
       // consumed (the A.V MMAs are issued by the softmax warpgroups)
       for (int ns = 0; ns < my_items; ++ns) {
-        if (!mbar_wait(&bar_full[ns % S], (ns / S) & 1, kWaitNs, &abort_flag) ||
+        if (!mbar_wait(&bar_fqk[ns % S], (ns / S) & 1, kWaitNs, &abort_flag) ||
             (ns >= 4 && !mbar_wait(&bar_tfree[2 * (ns & 1) + ((ns >> 1) & 1)], ((ns >> 2) - 1) & 1, kWaitNs,
                                    &abort_flag))) {
           if (!abort_flag) record_timeout(&abort_flag);
@@ -596,7 +627,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       // ---- A.V: warp wq < NST issues its share once the whole P tile is written
       bool issued = true;
       if (wq < C::NST && lane == 0) {
-        issued = mbar_wait(&bar_pfull[b], (j >> 1) & 1, kWaitNs, &abort_flag);
+        issued = mbar_wait(&bar_pfull[b], (j >> 1) & 1, kWaitNs, &abort_flag) &&
+                 mbar_wait(&bar_fv[k % S], (k / S) & 1, kWaitNs, &abort_flag);
         if (issued) {
           tc_fence_after();
           const int s = k % S, part = wq / C::SPP, sub = wq % C::SPP;
@@ -613,7 +645,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             mma_f16_ss(dst, smem_desc(pa + kk * 2048, 16, 256, SW_32B),
                        smem_desc(va + kk * kRowKeys * C::ROWB, lbo, C::SBO, C::SW), idO, kk != kb);
           mma_commit(&bar_ofull[b]);
-          mma_commit(&bar_empty[s]);
+          mma_commit(&bar_ev[s]);
         }
       }
       if (!__all_sync(0xffffffffu, issued)) {
