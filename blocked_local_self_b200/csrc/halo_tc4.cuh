@@ -25,15 +25,17 @@
 //     raw S maximum of every window row (before G is needed), then an upper
 //     bound of the row maximum, max over rows of c*S_max + c*rel_h plus the
 //     maximum of c*rel_w (at most a few units above the exact one);
-//     pass 2 the exponentials (MUFU and the FMA-pipe cubic), the row sum and
-//     bf16 P written back over the S columns.
+//     pass 2 the exponentials (MUFU and the FMA-pipe cubic) and bf16 P
+//     written back over the S columns.
 //   * A.V: four independent MMA chains, one per softmax warp: warp q takes
 //     block q & 1 and key half q >> 1, O_h = P_blk[:, keys of half h]
 //     V_blk[keys of half h] with M=64, N=d, A (P) read from the block's TMEM
 //     lane half and the accumulator in the same lane half (block B's window
-//     8w rows below block A's in the V tile).  The two halves' accumulators
-//     share one maximum, so O = O_0 + O_1.
-//   * epilogue: (O_0 + O_1) / l, bf16, NHWC.
+//     8w rows below block A's in the V tile).  The B operand's second
+//     swizzle atom is a ones tile: 8 more accumulator columns hold the row
+//     sum of the bf16 P.  The two halves share one maximum, so O = O_0 + O_1
+//     and l = l_0 + l_1.
+//   * epilogue: (O_0 + O_1) / (l_0 + l_1), bf16, NHWC.
 // Two softmax warpgroups take alternate items; every wait is bounded.
 #pragma once
 
@@ -110,7 +112,11 @@ struct Cfg {
   static constexpr int PCOLS = KP / 2;                    // packed bf16 P columns
   static constexpr int O_BASE = (PCOLS + 7) / 8 * 8;      // first O column
   static constexpr int KHALF = (KSTEPS + 1) / 2;          // A.V K-steps of key half 0
-  static constexpr int O_N = 2 * D;                       // O_0 | O_1, each in both lane halves
+  // A.V N: the block's V (d columns) and 8 columns of a ones tile, whose
+  // product with P is the row sum of the bf16 P the MMA consumed
+  static constexpr int ON = D + 8;
+  static constexpr int O_N = 2 * ON;                      // O_0 | O_1, each in both lane halves
+  static constexpr int ONES_BYTES = (KP * ROWB + 1023) / 1024 * 1024;  // ones rows, V's row pitch
   static constexpr SmemSwizzle SW = (ROWB == 32) ? SW_32B : (ROWB == 64 ? SW_64B : SW_128B);
   static constexpr uint32_t SBO = 8 * ROWB;
   static constexpr int HALO = (WIN - kBlock) / 2;
@@ -129,7 +135,7 @@ struct Cfg {
 template <int D, int WIN>
 __host__ __device__ constexpr int smem_bytes(int stages) {
   using C = Cfg<D, WIN>;
-  return 1024 + C::R_TILE + stages * C::STAGE_BYTES;
+  return 1024 + C::R_TILE + stages * C::STAGE_BYTES + C::ONES_BYTES;
 }
 
 // Load exactly N (< 32) consecutive TMEM columns (32x32b shape, thread t <->
@@ -199,9 +205,9 @@ __device__ __forceinline__ void row_max_chunk(uint32_t ts, float (&rm)[WIN]) {
 }
 
 // Pass 2 over keys [J0, J1) (padded to JP): p = 2^(c*(S + rel_w) + brow[row]),
-// row sum, packed bf16 P over TMEM columns [J0/2, JP/2).
+// packed bf16 P over TMEM columns [J0/2, JP/2).
 template <int WIN, int J0, int J1, int JP>
-__device__ __forceinline__ float exp_chunk(uint32_t ts, const float (&rw)[WIN], const float (&brow)[WIN], float c) {
+__device__ __forceinline__ void exp_chunk(uint32_t ts, const float (&rw)[WIN], const float (&brow)[WIN], float c) {
   constexpr int NL = (J1 - J0 + 7) / 8 * 8;
   constexpr int NW = (JP - J0) / 2;
   constexpr int NP = (J1 - J0) / 2;
@@ -210,7 +216,6 @@ __device__ __forceinline__ float exp_chunk(uint32_t ts, const float (&rw)[WIN], 
   float z[NL];
   tmem_ld_cols<NL>(ts + J0, z);
   tmem_wait_ld();
-  float2 lacc[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
   uint32_t pk[NW];
 #pragma unroll
   for (int i = 0; i < NP; ++i) {
@@ -225,15 +230,12 @@ __device__ __forceinline__ float exp_chunk(uint32_t ts, const float (&rw)[WIN], 
       rx = __float_as_uint(exp2_mufu(x.x));
       ry = __float_as_uint(exp2_mufu(x.y));
     }
-    lacc[i & 3] = __fadd2_rn(lacc[i & 3], make_float2(__uint_as_float(rx), __uint_as_float(ry)));
     pk[i] = pack_p(rx, ry);
   }
 #pragma unroll
   for (int i = NP; i < NW; ++i) pk[i] = 0u;
 #pragma unroll
   for (int i = 0; i < NW; i += 8) tmem_st_x8(ts + J0 / 2 + i, pk + i);
-  const float2 la = __fadd2_rn(lacc[0], lacc[1]), lb = __fadd2_rn(lacc[2], lacc[3]);
-  return (la.x + lb.x) + (la.y + lb.y);
 }
 
 template <int WIN, class C, int... I>
@@ -241,10 +243,11 @@ __device__ __forceinline__ void row_max_all(uint32_t ts, float (&rm)[WIN], std::
   (row_max_chunk<WIN, 16 * C::cstep(I), (I + 1 == C::NCHUNK) ? C::KS : 16 * C::cstep(I + 1)>(ts, rm), ...);
 }
 template <int WIN, class C, int... I>
-__device__ __forceinline__ float exp_all(uint32_t ts, const float (&rw)[WIN], const float (&brow)[WIN], float c,
-                                         std::integer_sequence<int, I...>) {
-  return (exp_chunk<WIN, 16 * C::cstep(I), (I + 1 == C::NCHUNK) ? C::KS : 16 * C::cstep(I + 1),
-                    16 * C::cstep(I + 1)>(ts, rw, brow, c) + ...);
+__device__ __forceinline__ void exp_all(uint32_t ts, const float (&rw)[WIN], const float (&brow)[WIN], float c,
+                                        std::integer_sequence<int, I...>) {
+  (exp_chunk<WIN, 16 * C::cstep(I), (I + 1 == C::NCHUNK) ? C::KS : 16 * C::cstep(I + 1), 16 * C::cstep(I + 1)>(
+       ts, rw, brow, c),
+   ...);
 }
 
 template <int D, int WIN>
@@ -256,6 +259,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sR = smem;
   uint8_t* sStage = smem + C::R_TILE;
+  uint8_t* sOnes = sStage + p.stages * C::STAGE_BYTES;  // after every stage: positive LBO from any V tile
   // stage layout: [Q_A][Q_B][K union][V union]
   constexpr int OFF_QA = 0, OFF_QB = C::Q_TILE, OFF_K = 2 * C::Q_TILE, OFF_V = OFF_K + C::K_TILE;
 
@@ -307,6 +311,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     prefetch_tensormap(&tmap_k);
     prefetch_tensormap(&tmap_v);
   }
+  // ones tile (bf16 1.0 in every element, so the swizzle does not matter)
+  for (int idx = tid; idx < C::ONES_BYTES / 16; idx += kThreads)
+    reinterpret_cast<uint4*>(sOnes)[idx] = make_uint4(0x3f803f80u, 0x3f803f80u, 0x3f803f80u, 0x3f803f80u);
   // R tile (once) and the union tiles' rows the TMA never writes (zero)
   for (int idx = tid; idx < kRRows * (D / 8); idx += kThreads) {
     const int r = idx / (D / 8), u = idx % (D / 8);
@@ -439,7 +446,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t ts = slot + (static_cast<uint32_t>(32 * wq) << 16);
     const float c = p.c;
     const int C_all = p.heads * D;
-    const uint32_t idO = idesc_bf16_f32(64, D, true);
+    const uint32_t idO = idesc_bf16_f32(64, C::ON, true);
 
     int j = 0;
     for (int k = g; k < my_items; k += 2, ++j) {
@@ -507,7 +514,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       float brow[WIN];
 #pragma unroll
       for (int r = 0; r < WIN; ++r) brow[r] = rh[r] - m;
-      const float l = exp_all<WIN, C>(ts, rwz, brow, c, std::make_integer_sequence<int, C::NCHUNK>{});
+      exp_all<WIN, C>(ts, rwz, brow, c, std::make_integer_sequence<int, C::NCHUNK>{});
       tmem_wait_st();
       tc_fence_before();
       __syncwarp();
@@ -527,10 +534,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int kb = hf ? C::KHALF : 0, ke = hf ? C::KSTEPS : C::KHALF;
         const uint32_t lanes = static_cast<uint32_t>(16 * ab) << 16;
         const uint32_t va = smem_addr(sStage + s * C::STAGE_BYTES + OFF_V) + ab * C::BOFF * C::ROWB;
+        // B = [V | ones]: the ones atom at leading byte offset lbo, same row pitch
+        const uint32_t lbo = smem_addr(sOnes) - va;
 #pragma unroll 1
         for (int kk = kb; kk < ke; ++kk)
-          mma_f16_ts(slot + lanes + C::O_BASE + hf * D, slot + lanes + 8 * kk,
-                     smem_desc(va + kk * 16 * C::ROWB, 16, C::SBO, C::SW), idO, kk != kb);
+          mma_f16_ts(slot + lanes + C::O_BASE + hf * C::ON, slot + lanes + 8 * kk,
+                     smem_desc(va + kk * 16 * C::ROWB, lbo, C::SBO, C::SW), idO, kk != kb);
         mma_commit(&bar_ofull[g]);
         mma_commit(&bar_ev[s]);
       }
@@ -544,16 +553,19 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_after();
       {
         // this thread's row of both key halves' accumulators
-        float o[D];
+        float o[D], la, lb;
+        tmem_ld_x1(ts + C::O_BASE + D, &la);
+        tmem_ld_x1(ts + C::O_BASE + C::ON + D, &lb);
 #pragma unroll
         for (int e = 0; e < D; e += 32) {
           float ta[32], tb[32];
           tmem_ld_x32(ts + C::O_BASE + e, ta);
-          tmem_ld_x32(ts + C::O_BASE + D + e, tb);
+          tmem_ld_x32(ts + C::O_BASE + C::ON + e, tb);
           tmem_wait_ld();
 #pragma unroll
           for (int i = 0; i < 32; ++i) o[e + i] = ta[i] + tb[i];
         }
+        const float l = la + lb;  // row sum of the bf16 P (ones columns)
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&bar_tfree[g]);
