@@ -35,9 +35,6 @@ import torch  # noqa: E402
 import workloads  # noqa: E402
 
 METRIC = "halo-attention output pixels/s and TFLOP/s, % of bf16 tensor/HBM roofline"
-KERNEL_SOURCES = ["blocked_local_self_b200/csrc/halo_tc.cuh", "blocked_local_self_b200/csrc/halo_tc2.cuh",
-                  "blocked_local_self_b200/csrc/halo_tc3.cuh", "blocked_local_self_b200/csrc/halo_tc4.cuh",
-                  "blocked_local_self_b200/csrc/sm100.cuh"]
 PROFILES = os.path.join(ROOT, "profiles")
 L2_BYTES = 126 * 1024 * 1024
 
@@ -175,13 +172,27 @@ def measured_peaks() -> dict:
     return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "source": "fallback"}
 
 
-def kernel_source_hash() -> str:
-    """Hash of the kernel sources with comments and blank space removed, so
-    that a profile summary stays attached to the code it measured."""
+def kernel_source_hash(kernel: str) -> str:
+    """Hash of the source of one kernel family (its header and the headers it
+    includes, comments and blank space removed), so that a profile summary
+    stays attached to the code it measured.  `kernel` is a name as
+    halo_kernel_name reports it, e.g. "halo_fwd_tc2<16,14>"."""
     import re
+    m = re.match(r"halo_fwd_(\w+?)<", kernel or "")
+    if not m:
+        return ""
+    csrc = os.path.join(ROOT, "blocked_local_self_b200", "csrc")
+    seen, todo = set(), ["halo_%s.cuh" % m.group(1)]
+    while todo:
+        name = todo.pop()
+        if name in seen or not os.path.exists(os.path.join(csrc, name)):
+            continue
+        seen.add(name)
+        with open(os.path.join(csrc, name)) as f:
+            todo += re.findall(r'^#include "([^"/]+)"', f.read(), flags=re.M)
     h = hashlib.sha256()
-    for rel in KERNEL_SOURCES:
-        with open(os.path.join(ROOT, rel)) as f:
+    for name in sorted(seen):
+        with open(os.path.join(csrc, name)) as f:
             text = f.read()
         text = re.sub(r"/\*.*?\*/", " ", text, flags=re.S)
         text = re.sub(r"//[^\n]*", " ", text)
@@ -189,10 +200,10 @@ def kernel_source_hash() -> str:
     return h.hexdigest()[:16]
 
 
-def ncu_traffic(workload: str):
+def ncu_traffic(workload: str, kernel: str):
     """DRAM bytes per launch (dram__bytes_read.sum + dram__bytes_write.sum)
     from a committed ncu summary under profiles/ that names this workload,
-    only while the kernel sources still hash to the value it records."""
+    only while the kernel's sources still hash to the value it records."""
     import glob
     import re
     for path in sorted(glob.glob(os.path.join(PROFILES, "*.md"))):
@@ -201,7 +212,7 @@ def ncu_traffic(workload: str):
         fields = dict(re.findall(r"^- (\w+): `?([^`\n]+?)`?\s*$", text, flags=re.M))
         if fields.get("workload") != workload or "dram_bytes_per_launch" not in fields:
             continue
-        if fields.get("kernel_source_sha") != kernel_source_hash():
+        if fields.get("kernel_source_sha") != kernel_source_hash(kernel):
             return None
         return float(fields["dram_bytes_per_launch"])
     return None
@@ -371,7 +382,7 @@ def main():
     peaks = measured_peaks()
     launch_s = ms_local * 1e-3 / args.steps  # one launch per step on this stream
     achieved_gbs = wl.bytes() / launch_s * 1e-9
-    traffic = ncu_traffic(wl.name)
+    traffic = ncu_traffic(wl.name, kernel)
     line = {
         "metric": METRIC,
         "value": value,
