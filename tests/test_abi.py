@@ -105,6 +105,8 @@ def test_kernel_names():
     lib = _lib()
     name = lambda *a: lib.halo_kernel_name(*a).decode()
     assert name(32, 64, 64, 8, 16, 8, 3, 1, 1) == "halo_fwd_tc2<16,14>"
+    assert name(2, 32, 32, 8, 16, 8, 1, 1, 1) == "halo_fwd_tc2<16,10>"
+    assert name(2, 32, 32, 8, 32, 8, 3, 1, 1) == "halo_fwd_tc2<32,14>"
     assert name(64, 32, 32, 8, 64, 8, 3, 1, 1) == "halo_fwd_tc4<64,14>"
     assert name(64, 24, 32, 8, 64, 8, 3, 1, 1) == "halo_fwd_tc<64,14,1>"  # odd number of block rows
     assert name(2, 16, 24, 3, 16, 8, 3, 1, 1) == "halo_fwd_tc<16,14,1>"   # odd head count

@@ -128,6 +128,9 @@ CASES += [
     dict(N=3, H=16, W=8, heads=4, dim_head=64, block=8, halo=0, stride=2),   # isolated blocks, stride 2
     dict(N=5, H=8, W=56, heads=8, dim_head=16, block=8, halo=3, stride=1),   # one block row, ragged items
     dict(N=1, H=64, W=8, heads=2, dim_head=32, block=8, halo=3, stride=2),   # one block column
+    # several items per CTA with both softmax warpgroups and every stage cycling
+    dict(N=8, H=32, W=48, heads=8, dim_head=16, block=8, halo=3, stride=1),
+    dict(N=8, H=32, W=48, heads=4, dim_head=16, block=8, halo=2, stride=1),
 ]
 
 
