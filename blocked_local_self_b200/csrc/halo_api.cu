@@ -94,7 +94,8 @@ const TcEntry kTcTable[] = {
     HALO_TC_WINS(16, 2), HALO_TC_WINS(32, 2), HALO_TC_WINS(64, 2),
 };
 
-// Stride-1 kernel with two heads per 128-row tile: (d, window) -> instantiation.
+// Stride-1 kernel with two heads per 128-row tile (maps with an odd number of
+// block rows): (d, window) -> instantiation.
 using Tc2Kernel = void (*)(const CUtensorMap, const CUtensorMap, const CUtensorMap, const halo::tc2::Params);
 struct Tc2Entry {
   int d, win;
@@ -142,7 +143,8 @@ const Tc3Entry* find_tc3(const Shape& s) {
   return nullptr;
 }
 
-// Stride-1 kernel with two vertically adjacent blocks per item (dim_head 64).
+// Stride-1 kernel with two vertically adjacent blocks of one head per item
+// (maps with an even number of block rows; taken before the head-pair kernel).
 using Tc4Kernel = void (*)(const CUtensorMap, const CUtensorMap, const CUtensorMap, const halo::tc4::Params);
 struct Tc4Entry {
   int d, win;
@@ -154,6 +156,8 @@ int tc4_smem(int stages) { return halo::tc4::smem_bytes<D, WIN>(stages); }
 #define HALO_TC4_ENTRY(D, WIN) \
   Tc4Entry { D, WIN, halo::tc4::halo_fwd_tc4<D, WIN>, tc4_smem<D, WIN> }
 const Tc4Entry kTc4Table[] = {
+    HALO_TC4_ENTRY(16, 8), HALO_TC4_ENTRY(16, 10), HALO_TC4_ENTRY(16, 12), HALO_TC4_ENTRY(16, 14),
+    HALO_TC4_ENTRY(32, 8), HALO_TC4_ENTRY(32, 10), HALO_TC4_ENTRY(32, 12), HALO_TC4_ENTRY(32, 14),
     HALO_TC4_ENTRY(64, 8), HALO_TC4_ENTRY(64, 10), HALO_TC4_ENTRY(64, 12), HALO_TC4_ENTRY(64, 14),
 };
 
@@ -175,7 +179,7 @@ const TcEntry* find_tc(const Shape& s) {
 
 int select_kernel(const Shape& s) {
   if (check_shape(s) != HALO_OK) return HALO_KERNEL_NONE;
-  if (find_tc2(s) || find_tc4(s) || find_tc(s) || find_tc3(s)) return HALO_KERNEL_TC_BF16;
+  if (find_tc4(s) || find_tc2(s) || find_tc(s) || find_tc3(s)) return HALO_KERNEL_TC_BF16;
   if (s.d <= 128) return HALO_KERNEL_SIMT_F32;
   return HALO_KERNEL_NONE;
 }
@@ -476,8 +480,8 @@ int attn_device(const void* q, const void* k, const void* v, const void* rel_h, 
   rc = device_info(&sm_count);
   if (rc != HALO_OK) return rc;
   if (kind == HALO_KERNEL_TC_BF16) {
-    if (const Tc2Entry* e2 = find_tc2(s)) return launch_tc2(*e2, q, k, v, rel_h, rel_w, out, s, sm_count, st);
     if (const Tc4Entry* e4 = find_tc4(s)) return launch_tc4(*e4, q, k, v, rel_h, rel_w, out, s, sm_count, st);
+    if (const Tc2Entry* e2 = find_tc2(s)) return launch_tc2(*e2, q, k, v, rel_h, rel_w, out, s, sm_count, st);
     if (const Tc3Entry* e3 = find_tc3(s)) return launch_tc3(*e3, q, k, v, rel_h, rel_w, out, s, sm_count, st);
     return launch_tc(*find_tc(s), q, k, v, rel_h, rel_w, out, s, sm_count, st);
   }
@@ -605,8 +609,8 @@ const char* halo_kernel_name(int N, int H, int W, int heads, int dim_head, int b
   if (kind == HALO_KERNEL_NONE) {
     std::snprintf(name, sizeof(name), "none");
   } else if (kind == HALO_KERNEL_TC_BF16) {
-    if (const Tc2Entry* e = find_tc2(s)) std::snprintf(name, sizeof(name), "halo_fwd_tc2<%d,%d>", e->d, e->win);
-    else if (const Tc4Entry* e = find_tc4(s)) std::snprintf(name, sizeof(name), "halo_fwd_tc4<%d,%d>", e->d, e->win);
+    if (const Tc4Entry* e = find_tc4(s)) std::snprintf(name, sizeof(name), "halo_fwd_tc4<%d,%d>", e->d, e->win);
+    else if (const Tc2Entry* e = find_tc2(s)) std::snprintf(name, sizeof(name), "halo_fwd_tc2<%d,%d>", e->d, e->win);
     else if (const Tc3Entry* e = find_tc3(s)) std::snprintf(name, sizeof(name), "halo_fwd_tc3<%d,%d>", e->d, e->win);
     else {
       const TcEntry* t = find_tc(s);

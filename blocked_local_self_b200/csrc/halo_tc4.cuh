@@ -1,5 +1,6 @@
 // halo_tc4.cuh -- stride-1 bf16 kernel for blocked local self-attention with
-// haloing on sm_100a, for wide heads (dim_head 64) and 8x8 query blocks.
+// haloing on sm_100a, 8x8 query blocks, dim_head 16, 32 or 64, maps with an
+// even number of block rows.
 //
 // Operation (HaloNet, "Scaling Local Self-Attention for Parameter Efficient
 // Visual Backbones", sections 2.1-2.2 and appendix A; index conventions of the
@@ -10,9 +11,10 @@
 // Work item = two vertically adjacent 8x8 blocks of one head.  Their windows
 // (w x w each) overlap in w - 8 rows, so one TMA box of (w + 8) x w pixels
 // holds both: in the box's row-major order block A's window is keys
-// [0, w*w) and block B's is keys [8w, 8w + w*w), both contiguous.  With
-// d = 64 two heads' windows would not fit two pipeline stages in shared
-// memory; two blocks' union does (96 KB per stage).
+// [0, w*w) and block B's is keys [8w, 8w + w*w), both contiguous: the item
+// loads (w + 8) w key and value pixels instead of the 2 w^2 of two separate
+// windows, and with d = 64 two pipeline stages fit in shared memory (96 KB
+// each).
 //   * TMA (warp 8): Q_A, Q_B [64 x d] and the union K tile, and one item
 //     later the union V tile (separate barriers, so Q/K stages free early).
 //   * S MMAs (block A on warp 9, block B on warp 11): per block M=64, N=200
@@ -123,7 +125,7 @@ struct Cfg {
   // softmax chunks (register working sets), boundaries at whole K-steps
   static constexpr int NCHUNK = 3;
   __host__ __device__ static constexpr int cstep(int i) { return (KSTEPS * i + NCHUNK / 2) / NCHUNK; }
-  static_assert(D == 32 || D == 64, "dim_head 32 or 64");
+  static_assert(D == 16 || D == 32 || D == 64, "dim_head 16, 32 or 64");
   static_assert(WIN % 2 == 0 && WIN >= 8 && WIN <= 14, "window 8..14");
   static_assert(NS <= (int)kGBase, "S columns below the relative logits");
   static_assert(2 * WIN - 1 <= kRelW, "relative table rows");
@@ -556,14 +558,22 @@ __global__ void __launch_bounds__(kThreads, 1)
         float o[D], la, lb;
         tmem_ld_x1(ts + C::O_BASE + D, &la);
         tmem_ld_x1(ts + C::O_BASE + C::ON + D, &lb);
+        constexpr int kSeg = (D % 32 == 0) ? 32 : 16;  // columns per load
 #pragma unroll
-        for (int e = 0; e < D; e += 32) {
-          float ta[32], tb[32];
-          tmem_ld_x32(ts + C::O_BASE + e, ta);
-          tmem_ld_x32(ts + C::O_BASE + C::ON + e, tb);
+        for (int e = 0; e < D; e += kSeg) {
+          float ta[kSeg], tb[kSeg];
+          if constexpr (kSeg == 32) {
+            tmem_ld_x32(ts + C::O_BASE + e, ta);
+            tmem_ld_x32(ts + C::O_BASE + C::ON + e, tb);
+          } else {
+            tmem_ld_x8(ts + C::O_BASE + e, ta);
+            tmem_ld_x8(ts + C::O_BASE + e + 8, ta + 8);
+            tmem_ld_x8(ts + C::O_BASE + C::ON + e, tb);
+            tmem_ld_x8(ts + C::O_BASE + C::ON + e + 8, tb + 8);
+          }
           tmem_wait_ld();
 #pragma unroll
-          for (int i = 0; i < 32; ++i) o[e + i] = ta[i] + tb[i];
+          for (int i = 0; i < kSeg; ++i) o[e + i] = ta[i] + tb[i];
         }
         const float l = la + lb;  // row sum of the bf16 P (ones columns)
         tc_fence_before();

@@ -106,15 +106,19 @@ for d in (16, 32, 64):
         for stride in (1, 2):
             CASES.append(dict(N=2, H=24, W=40, heads=8 if d < 64 else 4, dim_head=d, block=8, halo=halo,
                               stride=stride))
-# odd head counts at stride 1 (d = 16, 32) go to the one-head-per-item kernel
+# odd head counts at stride 1 (d = 16, 32): with an odd number of block rows
+# the one-head-per-item kernel, with an even number the two-block kernel
 CASES += [
+    dict(N=2, H=24, W=24, heads=3, dim_head=16, block=8, halo=3, stride=1),
+    dict(N=2, H=24, W=24, heads=3, dim_head=32, block=8, halo=2, stride=1),
     dict(N=2, H=16, W=24, heads=3, dim_head=16, block=8, halo=3, stride=1),
     dict(N=2, H=16, W=24, heads=3, dim_head=32, block=8, halo=2, stride=1),
 ]
-# dim_head 64 with an even number of block rows: the kernel that pairs two
-# vertically adjacent blocks (every window, one pair and several pairs)
-for halo in (0, 1, 2, 3):
-    CASES.append(dict(N=2, H=32, W=24, heads=3, dim_head=64, block=8, halo=halo, stride=1))
+# an even number of block rows: the kernel that pairs two vertically adjacent
+# blocks (every head size and window, one pair and several pairs)
+for d in (16, 32, 64):
+    for halo in (0, 1, 2, 3):
+        CASES.append(dict(N=2, H=32, W=24, heads=3, dim_head=d, block=8, halo=halo, stride=1))
 CASES.append(dict(N=3, H=16, W=40, heads=2, dim_head=64, block=8, halo=3, stride=1))
 # 16x16 query blocks (windows 16..24): every window of the block-16 kernel, both head sizes
 for d in (16, 32):
