@@ -142,9 +142,8 @@ __host__ __device__ constexpr int smem_bytes(int stages) {
 #define HALO_TC2_POLY_PAIRS ((WIN * 3 + 10) / 20)  // 14 -> 2, 12 -> 2, 10 -> 2, 8 -> 1
 #endif
 template <int WIN>
-__host__ __device__ constexpr unsigned poly_pair_mask() {
+__host__ __device__ constexpr unsigned poly_pair_mask(int npairs = HALO_TC2_POLY_PAIRS) {
   constexpr int h = (WIN - kBlock) / 2;
-  constexpr int npairs = HALO_TC2_POLY_PAIRS;
   unsigned m = 0;
   int picked = 0;
   // even kc inside [h, h+8) with kc+1 < h+8, from the middle outwards

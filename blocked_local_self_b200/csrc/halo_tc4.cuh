@@ -124,6 +124,11 @@ struct Cfg {
   static constexpr int HALO = (WIN - kBlock) / 2;
   // softmax chunks (register working sets), boundaries at whole K-steps
   static constexpr int NCHUNK = 3;
+  // window-column pairs whose exponentials take the FMA-pipe cubic: with
+  // d = 64 the larger MMAs leave the exponential unit less busy, and one
+  // pair measured faster than two (74.4 against 76.0 us on the deep-stage
+  // workload; at d = 16 two pairs, 111.3 against 114.9 us)
+  static constexpr int NPOLY = (D >= 64) ? 1 : HALO_TC2_POLY_PAIRS;
   __host__ __device__ static constexpr int cstep(int i) { return (KSTEPS * i + NCHUNK / 2) / NCHUNK; }
   static_assert(D == 16 || D == 32 || D == 64, "dim_head 16, 32 or 64");
   static_assert(WIN % 2 == 0 && WIN >= 8 && WIN <= 14, "window 8..14");
@@ -208,13 +213,13 @@ __device__ __forceinline__ void row_max_chunk(uint32_t ts, float (&rm)[WIN]) {
 
 // Pass 2 over keys [J0, J1) (padded to JP): p = 2^(c*(S + rel_w) + brow[row]),
 // packed bf16 P over TMEM columns [J0/2, JP/2).
-template <int WIN, int J0, int J1, int JP>
+template <int WIN, int NPOLY, int J0, int J1, int JP>
 __device__ __forceinline__ void exp_chunk(uint32_t ts, const float (&rw)[WIN], const float (&brow)[WIN], float c) {
   constexpr int NL = (J1 - J0 + 7) / 8 * 8;
   constexpr int NW = (JP - J0) / 2;
   constexpr int NP = (J1 - J0) / 2;
   static_assert(J0 % 2 == 0 && J1 % 2 == 0 && NW % 8 == 0, "pairs never straddle rows");
-  constexpr unsigned kPoly = poly_pair_mask<WIN>();
+  constexpr unsigned kPoly = poly_pair_mask<WIN>(NPOLY);
   float z[NL];
   tmem_ld_cols<NL>(ts + J0, z);
   tmem_wait_ld();
@@ -247,7 +252,8 @@ __device__ __forceinline__ void row_max_all(uint32_t ts, float (&rm)[WIN], std::
 template <int WIN, class C, int... I>
 __device__ __forceinline__ void exp_all(uint32_t ts, const float (&rw)[WIN], const float (&brow)[WIN], float c,
                                         std::integer_sequence<int, I...>) {
-  (exp_chunk<WIN, 16 * C::cstep(I), (I + 1 == C::NCHUNK) ? C::KS : 16 * C::cstep(I + 1), 16 * C::cstep(I + 1)>(
+  (exp_chunk<WIN, C::NPOLY, 16 * C::cstep(I), (I + 1 == C::NCHUNK) ? C::KS : 16 * C::cstep(I + 1),
+             16 * C::cstep(I + 1)>(
        ts, rw, brow, c),
    ...);
 }
