@@ -149,23 +149,6 @@ __device__ __forceinline__ uint32_t swz(int r, int u) {
   return r * 128 + ((u ^ (r & 7)) << 4);
 }
 
-// 2^x for x <= 0 on the FMA pipe: x = j + f with j = floor(x), f in [0, 1);
-// 2^f by a cubic fitted to the relative error on [0, 1) with p(0) = 1
-// (max relative error 8.6e-5), and 2^j added to the exponent field.
-// x is clamped at -127 so that masked (-inf) logits give a value < 2^-126.
-__device__ __forceinline__ float exp2_poly(float x) {
-  x = fmaxf(x, -127.0f);
-  const float magic = 12582912.0f;  // 1.5 * 2^23: adding it rounds to an integer
-  float t;
-  asm("add.rm.f32 %0, %1, %2;" : "=f"(t) : "f"(x), "f"(magic));
-  const float j = t - magic;
-  const float f = x - j;
-  float p = fmaf(f, 0.0770670548f, 0.2276449651f);
-  p = fmaf(p, f, 0.6951168180f);
-  p = fmaf(p, f, 1.0f);
-  return __int_as_float(__float_as_int(p) + (__float_as_int(t) << 23));
-}
-
 __device__ __forceinline__ float exp2_mufu(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
@@ -600,8 +583,11 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int kc = 0; kc < 16; ++kc) {
             if (kc < WIN) {
               const float x = fmaf(sv[i][kc], c, bias);
-              // about 40% of the exponentials run on the FMA pipe
-              e[kc] = (kc % 5 == 1 || kc % 5 == 3) ? exp2_poly(x) : exp2_mufu(x);
+              // every exponential on MUFU: here the unit runs at about 14% of
+              // its rate, and moving 40% of them to the FMA-pipe polynomial
+              // cost more issue slots than it saved (stride-2 workload 213.7
+              // against 176.4 us)
+              e[kc] = exp2_mufu(x);
             } else {
               e[kc] = 0.f;
             }

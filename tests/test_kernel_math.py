@@ -24,14 +24,19 @@ def _read(name):
 
 
 def _cubic_coefficients():
-    """(c3, c2, c1) of p(f) = ((c3 f + c2) f + c1) f + 1 from exp2_poly."""
-    src = _read("halo_tc.cuh")
-    body = src[src.index("float exp2_poly(float x)"):]
-    body = body[:body.index("}")]
-    c3, c2 = map(float, re.search(r"fmaf\(f, ([0-9.e+-]+)f, ([0-9.e+-]+)f\)", body).groups())
-    c1 = float(re.search(r"fmaf\(p, f, ([0-9.e+-]+)f\)", body).group(1))
-    assert re.search(r"fmaf\(p, f, 1\.0f\)", body)
-    return c3, c2, c1
+    """(c3, c2, c1) of p(f) = ((c3 f + c2) f + c1) f + 1 from exp2_poly2 (the
+    packed form: both lanes of every constant must agree)."""
+    src = _read("halo_tc2.cuh")
+    body = src[src.index("void exp2_poly2("):]
+    body = body[:body.index("\n}\n")]
+    pair = r"make_float2\(([0-9.e+-]+)f, ([0-9.e+-]+)f\)"
+    m = re.search(r"__ffma2_rn\(f, " + pair + ", " + pair + r"\)", body)
+    c3a, c3b, c2a, c2b = map(float, m.groups())
+    m1 = re.search(r"__ffma2_rn\(q, f, " + pair + r"\)", body)
+    c1a, c1b = map(float, m1.groups())
+    assert (c3a, c2a, c1a) == (c3b, c2b, c1b)
+    assert re.search(r"__ffma2_rn\(q, f, make_float2\(1\.0f, 1\.0f\)\)", body)
+    return c3a, c2a, c1a
 
 
 def _f32(x):
@@ -55,15 +60,6 @@ def _exp2_poly_emulated(x):
     p = _fma32(p, f, np.ones_like(f))
     bits = p.view(np.int32).astype(np.int64) + (j.astype(np.int64) << 23)
     return bits.astype(np.int32).view(np.float32)
-
-
-def test_both_exp2_forms_use_the_same_cubic():
-    c3, c2, c1 = _cubic_coefficients()
-    src2 = _read("halo_tc2.cuh")
-    body = src2[src2.index("void exp2_poly2("):]
-    body = body[:body.index("\n}\n")]
-    for c in (c3, c2, c1):
-        assert f"{c:.10f}".rstrip("0") in body or repr(c) in body, c
 
 
 def test_cubic_fixes_the_endpoints():
