@@ -125,10 +125,10 @@ struct Cfg {
   // softmax chunks (register working sets), boundaries at whole K-steps
   static constexpr int NCHUNK = 3;
   // window-column pairs whose exponentials take the FMA-pipe cubic: with
-  // d = 64 the larger MMAs leave the exponential unit less busy, and one
-  // pair measured faster than two (74.4 against 76.0 us on the deep-stage
-  // workload; at d = 16 two pairs, 111.3 against 114.9 us)
-  static constexpr int NPOLY = (D >= 64) ? 1 : HALO_TC2_POLY_PAIRS;
+  // d = 64 the larger MMAs leave the exponential unit less busy and every
+  // exponential goes to MUFU (deep-stage workload: 73.5 us, one pair 74.4,
+  // two 76.0); at d = 16 two pairs (111.3 us against 114.9 with one)
+  static constexpr int NPOLY = (D >= 64) ? 0 : HALO_TC2_POLY_PAIRS;
   __host__ __device__ static constexpr int cstep(int i) { return (KSTEPS * i + NCHUNK / 2) / NCHUNK; }
   static_assert(D == 16 || D == 32 || D == 64, "dim_head 16, 32 or 64");
   static_assert(WIN % 2 == 0 && WIN >= 8 && WIN <= 14, "window 8..14");
