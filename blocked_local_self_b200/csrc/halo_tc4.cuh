@@ -28,7 +28,8 @@
 //     bound of the row maximum, max over rows of c*S_max + c*rel_h plus the
 //     maximum of c*rel_w (at most a few units above the exact one);
 //     pass 2 the exponentials (MUFU and the FMA-pipe cubic) and bf16 P
-//     written back over the S columns.
+//     written back over the S columns.  Both passes walk the row in pieces
+//     of 32 keys with the next piece's TMEM load in flight.
 //   * A.V: four independent MMA chains, one per softmax warp: warp q takes
 //     block q & 1 and key half q >> 1, O_h = P_blk[:, keys of half h]
 //     V_blk[keys of half h] with M=64, N=d, A (P) read from the block's TMEM
@@ -122,14 +123,11 @@ struct Cfg {
   static constexpr SmemSwizzle SW = (ROWB == 32) ? SW_32B : (ROWB == 64 ? SW_64B : SW_128B);
   static constexpr uint32_t SBO = 8 * ROWB;
   static constexpr int HALO = (WIN - kBlock) / 2;
-  // softmax chunks (register working sets), boundaries at whole K-steps
-  static constexpr int NCHUNK = 3;
   // window-column pairs whose exponentials take the FMA-pipe cubic: with
   // d = 64 the larger MMAs leave the exponential unit less busy and every
   // exponential goes to MUFU (deep-stage workload: 73.5 us, one pair 74.4,
   // two 76.0); at d = 16 two pairs (111.3 us against 114.9 with one)
   static constexpr int NPOLY = (D >= 64) ? 0 : HALO_TC2_POLY_PAIRS;
-  __host__ __device__ static constexpr int cstep(int i) { return (KSTEPS * i + NCHUNK / 2) / NCHUNK; }
   static_assert(D == 16 || D == 32 || D == 64, "dim_head 16, 32 or 64");
   static_assert(WIN % 2 == 0 && WIN >= 8 && WIN <= 14, "window 8..14");
   static_assert(NS <= (int)kGBase, "S columns below the relative logits");
@@ -196,38 +194,56 @@ __device__ __forceinline__ ItemCoord item_coord(int item, int heads, int nbx, in
   return c;
 }
 
-// Pass 1 over keys [J0, J1) of this thread's S row: per window row the
-// maximum of the raw S values (rm[r], rows R0..).
-template <int WIN, int J0, int J1>
-__device__ __forceinline__ void row_max_chunk(uint32_t ts, float (&rm)[WIN]) {
-  constexpr int NL = (J1 - J0 + 7) / 8 * 8;
-  float z[NL];
-  tmem_ld_cols<NL>(ts + J0, z);
-  tmem_wait_ld();
+// Software-pipelined passes in pieces of 32 keys: the TMEM load of piece
+// i + 1 is issued before piece i is processed, so its latency overlaps the
+// arithmetic (a thread holds two 32-key buffers).
+template <class C>
+__host__ __device__ constexpr int pp_end(int i) { return (32 * (i + 1) < C::KS) ? 32 * (i + 1) : C::KS; }
+template <class C>
+__host__ __device__ constexpr int pp_pend(int i) { return (32 * (i + 1) < C::KP) ? 32 * (i + 1) : C::KP; }
+template <class C>
+__host__ __device__ constexpr int pp_count() { return (C::KP + 31) / 32; }
+
+template <int WIN, class C, int I>
+__device__ __forceinline__ void max_pipe(uint32_t ts, float (&rm)[WIN], float (&cur)[32], float (&nxt)[32]) {
+  constexpr int J0 = 32 * I, J1 = pp_end<C>(I);
+  if constexpr (I + 1 < pp_count<C>()) {
+    constexpr int K0 = 32 * (I + 1), K1 = pp_end<C>(I + 1);
+    tmem_ld_cols<(K1 - K0 + 7) / 8 * 8>(ts + K0, nxt);
+  }
 #pragma unroll
   for (int i = 0; i < (J1 - J0) / 2; ++i) {
     const int r = (J0 + 2 * i) / WIN;
-    rm[r] = max3f(rm[r], z[2 * i], z[2 * i + 1]);
+    rm[r] = max3f(rm[r], cur[2 * i], cur[2 * i + 1]);
+  }
+  if constexpr (I + 1 < pp_count<C>()) {
+    tmem_wait_ld();
+    max_pipe<WIN, C, I + 1>(ts, rm, nxt, cur);
   }
 }
-
-// Pass 2 over keys [J0, J1) (padded to JP): p = 2^(c*(S + rel_w) + brow[row]),
-// packed bf16 P over TMEM columns [J0/2, JP/2).
-template <int WIN, int NPOLY, int J0, int J1, int JP>
-__device__ __forceinline__ void exp_chunk(uint32_t ts, const float (&rw)[WIN], const float (&brow)[WIN], float c) {
-  constexpr int NL = (J1 - J0 + 7) / 8 * 8;
-  constexpr int NW = (JP - J0) / 2;
-  constexpr int NP = (J1 - J0) / 2;
-  static_assert(J0 % 2 == 0 && J1 % 2 == 0 && NW % 8 == 0, "pairs never straddle rows");
-  constexpr unsigned kPoly = poly_pair_mask<WIN>(NPOLY);
-  float z[NL];
-  tmem_ld_cols<NL>(ts + J0, z);
+template <int WIN, class C>
+__device__ __forceinline__ void row_max_pipelined(uint32_t ts, float (&rm)[WIN]) {
+  float za[32], zb[32];
+  tmem_ld_cols<(pp_end<C>(0) + 7) / 8 * 8>(ts, za);
   tmem_wait_ld();
+  max_pipe<WIN, C, 0>(ts, rm, za, zb);
+}
+
+template <int WIN, class C, int I>
+__device__ __forceinline__ void exp_pipe(uint32_t ts, const float (&rw)[WIN], const float (&brow)[WIN], float c,
+                                         float (&cur)[32], float (&nxt)[32]) {
+  constexpr int J0 = 32 * I, J1 = pp_end<C>(I), JP = pp_pend<C>(I);
+  constexpr int NW = (JP - J0) / 2, NP = (J1 > J0) ? (J1 - J0) / 2 : 0;
+  constexpr unsigned kPoly = poly_pair_mask<WIN>(C::NPOLY);
+  if constexpr (I + 1 < pp_count<C>()) {
+    constexpr int K0 = 32 * (I + 1), K1 = pp_end<C>(I + 1);
+    if constexpr (K1 > K0) tmem_ld_cols<(K1 - K0 + 7) / 8 * 8>(ts + K0, nxt);
+  }
   uint32_t pk[NW];
 #pragma unroll
   for (int i = 0; i < NP; ++i) {
     const int j = J0 + 2 * i, kc = j % WIN;
-    const float2 zz = __fadd2_rn(make_float2(z[2 * i], z[2 * i + 1]), make_float2(rw[kc], rw[kc + 1]));
+    const float2 zz = __fadd2_rn(make_float2(cur[2 * i], cur[2 * i + 1]), make_float2(rw[kc], rw[kc + 1]));
     const float bias = brow[j / WIN];
     const float2 x = __ffma2_rn(zz, make_float2(c, c), make_float2(bias, bias));
     uint32_t rx, ry;
@@ -243,19 +259,17 @@ __device__ __forceinline__ void exp_chunk(uint32_t ts, const float (&rw)[WIN], c
   for (int i = NP; i < NW; ++i) pk[i] = 0u;
 #pragma unroll
   for (int i = 0; i < NW; i += 8) tmem_st_x8(ts + J0 / 2 + i, pk + i);
+  if constexpr (I + 1 < pp_count<C>()) {
+    tmem_wait_ld();
+    exp_pipe<WIN, C, I + 1>(ts, rw, brow, c, nxt, cur);
+  }
 }
-
-template <int WIN, class C, int... I>
-__device__ __forceinline__ void row_max_all(uint32_t ts, float (&rm)[WIN], std::integer_sequence<int, I...>) {
-  (row_max_chunk<WIN, 16 * C::cstep(I), (I + 1 == C::NCHUNK) ? C::KS : 16 * C::cstep(I + 1)>(ts, rm), ...);
-}
-template <int WIN, class C, int... I>
-__device__ __forceinline__ void exp_all(uint32_t ts, const float (&rw)[WIN], const float (&brow)[WIN], float c,
-                                        std::integer_sequence<int, I...>) {
-  (exp_chunk<WIN, C::NPOLY, 16 * C::cstep(I), (I + 1 == C::NCHUNK) ? C::KS : 16 * C::cstep(I + 1),
-             16 * C::cstep(I + 1)>(
-       ts, rw, brow, c),
-   ...);
+template <int WIN, class C>
+__device__ __forceinline__ void exp_pipelined(uint32_t ts, const float (&rw)[WIN], const float (&brow)[WIN], float c) {
+  float za[32], zb[32];
+  tmem_ld_cols<(pp_end<C>(0) + 7) / 8 * 8>(ts, za);
+  tmem_wait_ld();
+  exp_pipe<WIN, C, 0>(ts, rw, brow, c, za, zb);
 }
 
 template <int D, int WIN>
@@ -471,7 +485,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       float rm[WIN];
 #pragma unroll
       for (int r = 0; r < WIN; ++r) rm[r] = -INFINITY;
-      row_max_all<WIN, C>(ts, rm, std::make_integer_sequence<int, C::NCHUNK>{});
+      row_max_pipelined<WIN, C>(ts, rm);
       if (!mbar_wait(&bar_gfull[g], j & 1, kWaitNs, &abort_flag)) {
         if (!abort_flag) record_timeout(&abort_flag);
         break;
@@ -522,7 +536,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       float brow[WIN];
 #pragma unroll
       for (int r = 0; r < WIN; ++r) brow[r] = rh[r] - m;
-      exp_all<WIN, C>(ts, rwz, brow, c, std::make_integer_sequence<int, C::NCHUNK>{});
+      exp_pipelined<WIN, C>(ts, rwz, brow, c);
       tmem_wait_st();
       tc_fence_before();
       __syncwarp();
