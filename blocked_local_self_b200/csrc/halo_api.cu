@@ -265,7 +265,7 @@ template <typename T, int DMAX>
 cudaError_t launch_simt_t(const void* q, const void* k, const void* v, const void* rh, const void* rw, void* out,
                           const Shape& s, cudaStream_t st) {
   const long long total = static_cast<long long>(s.N) * (s.H / s.stride) * (s.W / s.stride) * s.heads;
-  const long long blocks = (total + halo::simt::kThreads - 1) / halo::simt::kThreads;
+  const long long blocks = (32 * total + halo::simt::kThreads - 1) / halo::simt::kThreads;  // a warp each
   if (blocks > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
   halo::simt::halo_fwd_simt<T, DMAX><<<static_cast<unsigned>(blocks), halo::simt::kThreads, 0, st>>>(
       static_cast<const T*>(q), static_cast<const T*>(k), static_cast<const T*>(v), static_cast<const T*>(rh),
