@@ -47,6 +47,10 @@ def _load():
         lib.halo_oracle_f64.restype = ip
         lib.halo_oracle_samples_f64.argtypes = [vp] * 5 + [ctypes.POINTER(ctypes.c_int), ip, dp] + [ip] * 10
         lib.halo_oracle_samples_f64.restype = ip
+        lib.halo_oracle_masked_f64.argtypes = [vp] * 5 + [dp] + [ip] * 11
+        lib.halo_oracle_masked_f64.restype = ip
+        lib.halo_oracle_bwd_f64.argtypes = [vp] * 6 + [dp] * 5 + [ip] * 11
+        lib.halo_oracle_bwd_f64.restype = ip
         lib.halo_oracle_max_threads.argtypes = []
         lib.halo_oracle_max_threads.restype = ip
         _lib = lib
@@ -124,3 +128,55 @@ def halo_attention_samples(q, k, v, rel_h, rel_w, samples, block: int, halo: int
     if rc != 0:
         raise ValueError(f"oracle rejected the arguments (code {rc})")
     return out
+
+
+def halo_attention_masked(q, k, v, rel_h, rel_w, block: int, halo: int, kernel: int, stride: int = 1,
+                          heads: int | None = None, threads: int = 0) -> np.ndarray:
+    """SASA-masked variant: each query keeps only the ``kernel`` x ``kernel``
+    keys centred on it (``kernel`` odd, ``kernel // 2 <= halo``).  Float64
+    ``[N, H/stride, W/stride, C]``."""
+    lib = _load()
+    (qa, ka, va, rha, rwa), code = _prepare(q, k, v, rel_h, rel_w)
+    N, H, W, C = qa.shape
+    d = rha.shape[1]
+    if heads is None:
+        heads = C // d
+    out = np.empty((N, H // stride, W // stride, C), dtype=np.float64)
+    rc = lib.halo_oracle_masked_f64(qa.ctypes.data, ka.ctypes.data, va.ctypes.data, rha.ctypes.data,
+                                    rwa.ctypes.data, out.ctypes.data_as(ctypes.POINTER(ctypes.c_double)),
+                                    N, H, W, heads, d, block, halo, stride, kernel, code, threads)
+    if rc != 0:
+        raise ValueError(f"oracle rejected the arguments (code {rc})")
+    return out
+
+
+def halo_attention_bwd(q, k, v, rel_h, rel_w, dout, block: int, halo: int, stride: int = 1, kernel: int = 0,
+                       heads: int | None = None, threads: int = 0):
+    """Gradients of ``sum(out * dout)`` with respect to q, k, v, rel_h, rel_w
+    (float64 arrays ``dq, dk, dv`` of q's shape and ``drel_h, drel_w`` of the
+    tables' shape).  ``dout``: ``[N, H/stride, W/stride, C]`` in the inputs'
+    dtype.  ``kernel`` > 0 applies the SASA mask as in
+    ``halo_attention_masked``."""
+    lib = _load()
+    (qa, ka, va, rha, rwa, da), code = _prepare_n(q, k, v, rel_h, rel_w, dout)
+    N, H, W, C = qa.shape
+    d = rha.shape[1]
+    if heads is None:
+        heads = C // d
+    grads = [np.empty(qa.shape, dtype=np.float64) for _ in range(3)]
+    grads += [np.empty(rha.shape, dtype=np.float64) for _ in range(2)]
+    dptr = [g.ctypes.data_as(ctypes.POINTER(ctypes.c_double)) for g in grads]
+    rc = lib.halo_oracle_bwd_f64(qa.ctypes.data, ka.ctypes.data, va.ctypes.data, rha.ctypes.data, rwa.ctypes.data,
+                                 da.ctypes.data, *dptr, N, H, W, heads, d, block, halo, stride, kernel, code,
+                                 threads)
+    if rc != 0:
+        raise ValueError(f"oracle rejected the arguments (code {rc})")
+    return tuple(grads)
+
+
+def _prepare_n(*tensors):
+    arrs = [_as_host_array(t) for t in tensors]
+    codes = {c for _, c in arrs}
+    if len(codes) != 1:
+        raise TypeError("all tensors must share one dtype")
+    return [a for a, _ in arrs], codes.pop()

@@ -43,11 +43,33 @@
  * exponentials, their sum and the weighted sum of v, all in double precision,
  * from the stored input values (float32, or bf16 widened exactly).
  *
+ * SASA-masked variant (section 2.2, the paragraph after Figure 1): the same
+ * blocked neighbourhood with h = floor(k/2) and an attention mask that keeps,
+ * for each query pixel, only the k x k keys centred on it, so that the op
+ * emulates pixel-centred local attention.  Here `kmask` = k (odd, 1 <= k <=
+ * 2h + 1); a key is kept when |Y - y| <= k/2 and |X - x| <= k/2 (and it is
+ * inside the image).  kmask = 0 means no mask (HaloNet's own, unmasked form).
+ *
+ * Backward (the gradients of a scalar loss L = sum(out * dout) with respect to
+ * q, k, v, rel_h and rel_w; the pages train this layer, section 2.2 and
+ * Figure 3, but print no gradient): by the chain rule through the defining
+ * formula, per output pixel and head with p_j the softmax weights,
+ *     dp_j = dout . v_j,   D = sum_j p_j dp_j,   dz_j = p_j (dp_j - D),
+ *     dq  = s sum_j dz_j (k_j + rel_h[a_j] + rel_w[b_j]),
+ *     dk_j += s dz_j q,  dv_j += p_j dout,
+ *     drel_h[a_j] += s dz_j q,  drel_w[b_j] += s dz_j q,
+ * where a_j, b_j are the row and column table indices of key j.  The sums
+ * run over the kept keys only; dk, dv, drel_h, drel_w collect every query
+ * whose window holds the key or uses the table row (the tables are shared by
+ * all heads, section 2.1, footnote 1).  Pinned by central finite differences
+ * of the forward oracle and by closed-form identities of these sums.
+ *
  * Build: gcc -O2 -fopenmp -shared -fPIC halo_oracle.c -o liboracle.so -lm
  */
 #include <math.h>
 #include <stdint.h>
 #include <stddef.h>
+#include <stdlib.h>
 #include <string.h>
 #ifdef _OPENMP
 #include <omp.h>
@@ -72,7 +94,21 @@ static double read_elem(const void *base, size_t i, int dtype)
 typedef struct {
     const void *q, *k, *v, *rel_h, *rel_w;
     int N, H, W, heads, d, b, h, S, dtype;
+    int kmask;  /* 0: no mask; k: keep the k x k keys centred on the query */
 } oracle_args;
+
+/* Whether window key (kr, kc) of query pixel (y, x) takes part in the softmax:
+ * inside the image, and, with the SASA mask, inside the k x k square centred
+ * on the query. */
+static int key_kept(const oracle_args *a, int y, int x, int Y, int X)
+{
+    if (Y < 0 || Y >= a->H || X < 0 || X >= a->W) return 0;
+    if (a->kmask > 0) {
+        const int r = a->kmask / 2;
+        if (Y - y > r || y - Y > r || X - x > r || x - X > r) return 0;
+    }
+    return 1;
+}
 
 /*
  * One output pixel (n, oy, ox), one head: writes d doubles to out_vec.
@@ -100,7 +136,7 @@ static void one_pixel_head(const oracle_args *a, int n, int oy, int ox, int head
         for (int kc = 0; kc < w; ++kc) {
             const int Y = y0 + kr, X = x0 + kc;
             const int j = kr * w + kc;
-            if (Y < 0 || Y >= a->H || X < 0 || X >= a->W) {
+            if (!key_kept(a, y, x, Y, X)) {
                 valid[j] = 0;
                 z[j] = 0.0;
                 continue;
@@ -155,6 +191,7 @@ static int check_args(const oracle_args *a)
     if (a->b % a->S) return -3;
     if (a->dtype != ORACLE_F32 && a->dtype != ORACLE_BF16) return -9;
     if (a->b + 2 * a->h > 4096) return -2;
+    if (a->kmask < 0 || (a->kmask > 0 && (a->kmask % 2 == 0 || a->kmask / 2 > a->h))) return -2;
     return 0;
 }
 
@@ -162,16 +199,14 @@ static int check_args(const oracle_args *a)
  * Full output: out is [N, H/S, W/S, heads*d] doubles.  threads <= 0 uses the
  * OpenMP default.  Returns 0, or a negative code for invalid arguments.
  */
-int halo_oracle_f64(const void *q, const void *k, const void *v,
-                    const void *rel_h, const void *rel_w, double *out,
-                    int N, int H, int W, int heads, int dim_head,
-                    int block, int halo, int stride, int dtype, int threads)
+static int full_output(const oracle_args *ap, double *out, int threads)
 {
-    oracle_args a = {q, k, v, rel_h, rel_w, N, H, W, heads, dim_head, block, halo, stride, dtype};
+    const oracle_args a = *ap;
     int rc = check_args(&a);
     if (rc) return rc;
     if (!out) return -1;
-    const int OH = H / stride, OW = W / stride, C = heads * dim_head;
+    const int N = a.N, heads = a.heads, dim_head = a.d, stride = a.S, block = a.b, halo = a.h;
+    const int OH = a.H / stride, OW = a.W / stride, C = heads * dim_head;
     const int w = block + 2 * halo;
     const long total = (long)N * heads * OH * OW;
 #ifdef _OPENMP
@@ -200,6 +235,182 @@ int halo_oracle_f64(const void *q, const void *k, const void *v,
     return 0;
 }
 
+int halo_oracle_f64(const void *q, const void *k, const void *v,
+                    const void *rel_h, const void *rel_w, double *out,
+                    int N, int H, int W, int heads, int dim_head,
+                    int block, int halo, int stride, int dtype, int threads)
+{
+    oracle_args a = {q, k, v, rel_h, rel_w, N, H, W, heads, dim_head, block, halo, stride, dtype, 0};
+    return full_output(&a, out, threads);
+}
+
+/*
+ * SASA-masked variant: as halo_oracle_f64, each query keeping only the
+ * kmask x kmask keys centred on it (kmask odd, kmask/2 <= halo).
+ */
+int halo_oracle_masked_f64(const void *q, const void *k, const void *v,
+                           const void *rel_h, const void *rel_w, double *out,
+                           int N, int H, int W, int heads, int dim_head,
+                           int block, int halo, int stride, int kmask, int dtype, int threads)
+{
+    oracle_args a = {q, k, v, rel_h, rel_w, N, H, W, heads, dim_head, block, halo, stride, dtype, kmask};
+    if (kmask <= 0) return -2;
+    return full_output(&a, out, threads);
+}
+
+/*
+ * Backward of one output pixel and head: recomputes the softmax weights of
+ * the kept keys (as one_pixel_head does), then adds this query's terms to
+ * dq (written), dk, dv (accumulated, [N, H, W, C] doubles) and to the
+ * caller's table accumulators drh, drw ([2w-1, d] doubles each).
+ * Scratch: z, p hold w*w doubles, valid w*w chars, dov d doubles.
+ */
+static void one_pixel_head_bwd(const oracle_args *a, const void *dout, int n, int oy, int ox, int head,
+                               double *z, char *valid, double *dov,
+                               double *dq, double *dk, double *dv, double *drh, double *drw)
+{
+    const int w = a->b + 2 * a->h;
+    const int C = a->heads * a->d;
+    const int OH = a->H / a->S, OW = a->W / a->S;
+    const double s = 1.0 / sqrt((double)a->d);
+    const int y = a->S * oy, x = a->S * ox;
+    const int by = y / a->b, bx = x / a->b;
+    const int qy = y - by * a->b, qx = x - bx * a->b;
+    const int y0 = by * a->b - a->h, x0 = bx * a->b - a->h;
+    const size_t qoff = (((size_t)n * a->H + y) * a->W + x) * C + (size_t)head * a->d;
+    const size_t ooff = (((size_t)n * OH + oy) * OW + ox) * C + (size_t)head * a->d;
+
+    /* forward: logits of the kept keys, maximum, softmax weights p_j */
+    double m = -INFINITY;
+    for (int kr = 0; kr < w; ++kr) {
+        for (int kc = 0; kc < w; ++kc) {
+            const int Y = y0 + kr, X = x0 + kc, j = kr * w + kc;
+            valid[j] = (char)key_kept(a, y, x, Y, X);
+            z[j] = 0.0;
+            if (!valid[j]) continue;
+            const size_t koff = (((size_t)n * a->H + Y) * a->W + X) * C + (size_t)head * a->d;
+            const size_t rh = (size_t)(kr - qy + w - 1) * a->d, rw = (size_t)(kc - qx + w - 1) * a->d;
+            double acc = 0.0;
+            for (int e = 0; e < a->d; ++e)
+                acc += read_elem(a->q, qoff + e, a->dtype) *
+                       (read_elem(a->k, koff + e, a->dtype) + read_elem(a->rel_h, rh + e, a->dtype) +
+                        read_elem(a->rel_w, rw + e, a->dtype));
+            z[j] = s * acc;
+            if (z[j] > m) m = z[j];
+        }
+    }
+    double Z = 0.0;
+    for (int j = 0; j < w * w; ++j)
+        if (valid[j]) { z[j] = exp(z[j] - m); Z += z[j]; }
+    for (int j = 0; j < w * w; ++j) z[j] = valid[j] ? z[j] / Z : 0.0;  /* z now holds p_j */
+
+    /* dp_j = dout . v_j and D = sum_j p_j dp_j */
+    for (int e = 0; e < a->d; ++e) dov[e] = read_elem(dout, ooff + e, a->dtype);
+    double D = 0.0;
+    for (int kr = 0; kr < w; ++kr) {
+        for (int kc = 0; kc < w; ++kc) {
+            const int j = kr * w + kc;
+            if (!valid[j]) continue;
+            const size_t voff = (((size_t)n * a->H + (y0 + kr)) * a->W + (x0 + kc)) * C + (size_t)head * a->d;
+            double dp = 0.0;
+            for (int e = 0; e < a->d; ++e) dp += dov[e] * read_elem(a->v, voff + e, a->dtype);
+            D += z[j] * dp;
+        }
+    }
+    /* second sweep: dz_j and every gradient term */
+    double *dqv = dq + qoff;
+    for (int e = 0; e < a->d; ++e) dqv[e] = 0.0;
+    for (int kr = 0; kr < w; ++kr) {
+        for (int kc = 0; kc < w; ++kc) {
+            const int j = kr * w + kc;
+            if (!valid[j]) continue;
+            const size_t koff = (((size_t)n * a->H + (y0 + kr)) * a->W + (x0 + kc)) * C + (size_t)head * a->d;
+            const size_t rh = (size_t)(kr - qy + w - 1) * a->d, rw = (size_t)(kc - qx + w - 1) * a->d;
+            double dp = 0.0;
+            for (int e = 0; e < a->d; ++e) dp += dov[e] * read_elem(a->v, koff + e, a->dtype);
+            const double dz = z[j] * (dp - D);
+            for (int e = 0; e < a->d; ++e) {
+                const double qe = read_elem(a->q, qoff + e, a->dtype);
+                dqv[e] += s * dz * (read_elem(a->k, koff + e, a->dtype) + read_elem(a->rel_h, rh + e, a->dtype) +
+                                    read_elem(a->rel_w, rw + e, a->dtype));
+                dk[koff + e] += s * dz * qe;
+                dv[koff + e] += z[j] * dov[e];
+                drh[rh + e] += s * dz * qe;
+                drw[rw + e] += s * dz * qe;
+            }
+        }
+    }
+}
+
+/*
+ * Gradients of L = sum(out * dout): dout is [N, H/S, W/S, C] in the inputs'
+ * dtype; dq, dk, dv are [N, H, W, C] doubles (dq is zero at the pixels that
+ * are not queries at stride 2), drel_h, drel_w [2w-1, d] doubles.  kmask as
+ * in halo_oracle_masked_f64 (0: no mask).  Parallel over (image, head): those
+ * write disjoint parts of dq, dk, dv; the tables' sums are kept per thread
+ * and added in thread order at the end.
+ */
+int halo_oracle_bwd_f64(const void *q, const void *k, const void *v,
+                        const void *rel_h, const void *rel_w, const void *dout,
+                        double *dq, double *dk, double *dv, double *drel_h, double *drel_w,
+                        int N, int H, int W, int heads, int dim_head,
+                        int block, int halo, int stride, int kmask, int dtype, int threads)
+{
+    oracle_args a = {q, k, v, rel_h, rel_w, N, H, W, heads, dim_head, block, halo, stride, dtype, kmask};
+    int rc = check_args(&a);
+    if (rc) return rc;
+    if (!dout || !dq || !dk || !dv || !drel_h || !drel_w) return -1;
+    const int OH = H / stride, OW = W / stride, C = heads * dim_head;
+    const int w = block + 2 * halo, R = 2 * w - 1;
+    const size_t nin = (size_t)N * H * W * C, ntab = (size_t)R * dim_head;
+    memset(dq, 0, nin * sizeof(double));
+    memset(dk, 0, nin * sizeof(double));
+    memset(dv, 0, nin * sizeof(double));
+#ifdef _OPENMP
+    if (threads > 0) omp_set_num_threads(threads);
+    const int nt = omp_get_max_threads();
+#else
+    (void)threads;
+    const int nt = 1;
+#endif
+    double *part = (double *)calloc((size_t)nt * 2 * ntab, sizeof(double));
+    if (!part) return -2;
+    const long units = (long)N * heads;
+#pragma omp parallel
+    {
+#ifdef _OPENMP
+        const int tid = omp_get_thread_num();
+#else
+        const int tid = 0;
+#endif
+        double *z = (double *)malloc(sizeof(double) * (size_t)w * w);
+        char *valid = (char *)malloc((size_t)w * w);
+        double *dov = (double *)malloc(sizeof(double) * (size_t)dim_head);
+        double *drh = part + (size_t)tid * 2 * ntab, *drw = drh + ntab;
+#pragma omp for schedule(static)
+        for (long u = 0; u < units; ++u) {
+            const int n = (int)(u / heads), head = (int)(u % heads);
+            for (int oy = 0; oy < OH; ++oy)
+                for (int ox = 0; ox < OW; ++ox)
+                    one_pixel_head_bwd(&a, dout, n, oy, ox, head, z, valid, dov, dq, dk, dv, drh, drw);
+        }
+        free(z);
+        free(valid);
+        free(dov);
+    }
+    for (size_t i = 0; i < ntab; ++i) {
+        double sh = 0.0, sw = 0.0;
+        for (int t = 0; t < nt; ++t) {
+            sh += part[(size_t)t * 2 * ntab + i];
+            sw += part[(size_t)t * 2 * ntab + ntab + i];
+        }
+        drel_h[i] = sh;
+        drel_w[i] = sw;
+    }
+    free(part);
+    return 0;
+}
+
 /*
  * Sampled output pixels: samples holds nsamples (n, oy, ox) triples; out is
  * [nsamples, heads*d] doubles.  Used for parity at full sizes, where the whole
@@ -211,7 +422,7 @@ int halo_oracle_samples_f64(const void *q, const void *k, const void *v,
                             int N, int H, int W, int heads, int dim_head,
                             int block, int halo, int stride, int dtype, int threads)
 {
-    oracle_args a = {q, k, v, rel_h, rel_w, N, H, W, heads, dim_head, block, halo, stride, dtype};
+    oracle_args a = {q, k, v, rel_h, rel_w, N, H, W, heads, dim_head, block, halo, stride, dtype, 0};
     int rc = check_args(&a);
     if (rc) return rc;
     if (!samples || !out) return -1;
