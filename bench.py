@@ -20,6 +20,7 @@ from __future__ import annotations
 import argparse
 import hashlib
 import json
+import math
 import os
 import statistics
 import subprocess
@@ -50,6 +51,10 @@ def parse_args():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-graph", action="store_true",
                     help="launch every step from Python instead of replaying captured CUDA graphs")
+    ap.add_argument("--min-timed-s", type=float, default=0.5,
+                    help="repeat the K-step timed region until about this much time is covered (median reported)")
+    ap.add_argument("--no-per-config", action="store_true",
+                    help="skip timing every workload for the per_config object")
     return ap.parse_args()
 
 
@@ -131,7 +136,14 @@ class ClockSampler:
             except subprocess.TimeoutExpired:
                 self.proc.kill()
 
-    def summary(self, t0: float, t1: float) -> dict:
+    def cleanup(self):
+        try:
+            if self.path:
+                os.unlink(self.path)
+        except OSError:
+            pass
+
+    def summary(self, t0: float, t1: float, keep: bool = False) -> dict:
         rows = []
         try:
             with open(self.path) as f:
@@ -145,7 +157,8 @@ class ClockSampler:
                     except (ValueError, IndexError):
                         continue
                     rows.append((ts, parts))
-            os.unlink(self.path)
+            if not keep:
+                os.unlink(self.path)
         except OSError:
             pass
         inside = [p for ts, p in rows if t0 - 0.15 <= ts <= t1 + 0.15]
@@ -286,6 +299,167 @@ def run_reference(args):
 # main (CUDA path)
 # ---------------------------------------------------------------------------
 
+def make_device_sets(wl, inputs_cpu):
+    """Input sets on the device, enough of them that the step's inputs are not
+    L2-resident when it runs (each set holds q, k, v of the whole batch)."""
+    in_bytes = sum(t.numel() * t.element_size() for t in inputs_cpu[:3])
+    n_sets = max(2, -(-3 * L2_BYTES // in_bytes))
+    sets = []
+    for i in range(n_sets):
+        if i == 0:
+            sets.append([t.cuda() for t in inputs_cpu])
+        else:
+            sets.append([(t.cuda() * 1.0).roll(i, dims=0) if t.dim() == 4 else t.cuda() for t in inputs_cpu])
+    return sets, in_bytes
+
+
+class DeviceBench:
+    """Times `halo_attn` on one workload: CUDA graphs of the per-step launches
+    (inputs rotating over sets larger than L2) replayed on one stream, CUDA
+    events on that stream."""
+
+    def __init__(self, halo, wl, inputs_cpu, stream, use_graph=True):
+        self.halo, self.wl, self.stream, self.use_graph = halo, wl, stream, use_graph
+        self.sets, self.in_bytes = make_device_sets(wl, inputs_cpu)
+        self.n_sets = len(self.sets)
+        OH, OW = wl.out_hw
+        self.outs = [torch.empty((wl.N, OH, OW, wl.C), dtype=wl.torch_dtype, device="cuda")
+                     for _ in range(self.n_sets)]
+        self.kernel = halo.kernel_name(wl.N, wl.H, wl.W, wl.heads, wl.dim_head, wl.block, wl.halo, wl.stride,
+                                       wl.torch_dtype)
+        self.graphs = []
+
+    def step(self, i):
+        wl, s = self.wl, self.sets[i % self.n_sets]
+        self.halo.attn(*s, block=wl.block, halo=wl.halo, stride=wl.stride, out=self.outs[i % self.n_sets],
+                       stream=self.stream)
+
+    def warmup(self, n):
+        with torch.cuda.stream(self.stream):
+            for i in range(n):
+                self.step(i)
+        torch.cuda.synchronize()
+
+    def prepare(self, steps):
+        """Capture the timed steps: a graph of `per` steps replayed steps // per
+        times, then one graph of the remaining steps."""
+        self.steps = steps
+        self.graphs = []
+        if not self.use_graph:
+            return
+        per = self.n_sets * max(1, -(-64 // self.n_sets))
+        plan = [(per, steps // per), (steps % per, 1)]
+        start = 0
+        for n, reps in plan:
+            if n == 0 or reps == 0:
+                continue
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, stream=self.stream):
+                for i in range(n):
+                    self.step(start + i)
+            self.graphs.append((g, reps))
+            start += n
+        with torch.cuda.stream(self.stream):
+            for g, _ in self.graphs:
+                g.replay()
+        torch.cuda.synchronize()
+
+    def region(self):
+        """One timed region of exactly `steps` steps; returns milliseconds."""
+        ev0 = torch.cuda.Event(enable_timing=True)
+        ev1 = torch.cuda.Event(enable_timing=True)
+        ev0.record(self.stream)
+        with torch.cuda.stream(self.stream):
+            if self.graphs:
+                for g, reps in self.graphs:
+                    for _ in range(reps):
+                        g.replay()
+            else:
+                for i in range(self.steps):
+                    self.step(i)
+        ev1.record(self.stream)
+        ev1.synchronize()
+        return ev0.elapsed_time(ev1)
+
+    def release(self):
+        self.graphs = []
+        self.sets = []
+        self.outs = []
+
+
+def time_flushed_launches(halo, wl, inputs_cpu, stream, launches=200):
+    """For a workload whose inputs fit in L2 many times over (the tiny float32
+    case): each launch timed on its own with CUDA events, a 256 MiB buffer
+    written between launches (outside the events) so that none starts with its
+    inputs in L2 (the buffer is twice the L2 size).  Returns the median launch
+    time in ms."""
+    dev = [t.cuda() for t in inputs_cpu]
+    OH, OW = wl.out_hw
+    out = torch.empty((wl.N, OH, OW, wl.C), dtype=wl.torch_dtype, device="cuda")
+    flush = torch.empty(2 * L2_BYTES, dtype=torch.uint8, device="cuda")
+    times = []
+    with torch.cuda.stream(stream):
+        for i in range(launches + 5):
+            flush.fill_(i & 0xff)
+            e0 = torch.cuda.Event(enable_timing=True)
+            e1 = torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            halo.attn(*dev, block=wl.block, halo=wl.halo, stride=wl.stride, out=out, stream=stream)
+            e1.record(stream)
+            e1.synchronize()
+            if i >= 5:
+                times.append(e0.elapsed_time(e1))
+    return statistics.median(times)
+
+
+def roofline_entry(wl, launch_s, peaks, traffic):
+    """HBM and tensor fractions of one launch of `wl` taking `launch_s` seconds."""
+    gbs = wl.bytes() / launch_s * 1e-9
+    tflops = wl.flops() / launch_s * 1e-12
+    return {"achieved_gbs": gbs, "hbm_frac": gbs / peaks["hbm_gbs"], "tflops": tflops,
+            "tensor_frac": (tflops / peaks["bf16_tflops"]) if wl.dtype == "bf16" else None,
+            "traffic": traffic, "algorithmic_bytes": wl.bytes(), "flops": wl.flops()}
+
+
+def per_config(halo, stream, sampler, peaks, seconds=0.5):
+    """Every workload, timed in this run: ms per launch, pixels/s, HBM and
+    tensor fractions of the measured peaks, the kernel, ncu traffic when the
+    committed summary matches the kernel's sources, and the clocks seen."""
+    res = {}
+    for name, wl in workloads.WORKLOADS.items():
+        inputs_cpu = workloads.make_inputs(wl)
+        kernel = halo.kernel_name(wl.N, wl.H, wl.W, wl.heads, wl.dim_head, wl.block, wl.halo, wl.stride,
+                                  wl.torch_dtype)
+        t0 = time.time()
+        if wl.N * wl.H * wl.W * wl.C * wl.elem_bytes * 3 < L2_BYTES // 4:
+            ms = time_flushed_launches(halo, wl, inputs_cpu, stream)
+            how, steps, reps = "each launch alone after a 252 MiB (2x L2) flush; median of 200", 1, 200
+        else:
+            b = DeviceBench(halo, wl, inputs_cpu, stream)
+            b.warmup(10)
+            b.prepare(20)
+            est = b.region() / 20
+            steps = max(20, int(seconds * 1e3 / max(est, 1e-3)))
+            b.prepare(steps)
+            regions = [b.region() / steps for _ in range(3)]
+            ms = statistics.median(regions)
+            reps = 3
+            how = (f"median of 3 regions of {steps} graph-replayed launches, inputs rotating over "
+                   f"{b.n_sets} sets ({b.n_sets * b.in_bytes / 2**20:.0f} MiB) > L2")
+            b.release()
+        t1 = time.time()
+        torch.cuda.synchronize()
+        err = halo.get_last_error()
+        if err != 0:
+            raise RuntimeError(f"device error flag {err} after timing {name}")
+        entry = {"kernel": kernel, "ms": ms, "value": wl.out_pixels / (ms * 1e-3), "unit": "pixels/s",
+                 "timing": how, "clocks": (t0, t1)}  # summarised once the sampler has stopped
+        entry.update(roofline_entry(wl, ms * 1e-3, peaks, ncu_traffic(wl.name, kernel)))
+        res[name] = entry
+        torch.cuda.empty_cache()
+    return res
+
+
 def main():
     args = parse_args()
     if args.impl == "reference":
@@ -298,90 +472,59 @@ def main():
 
     wl = workloads.WORKLOADS[args.workload]
     inputs_cpu = workloads.make_inputs(wl, seed=rank_seed(wl, rank))
-    in_bytes = sum(t.numel() * t.element_size() for t in inputs_cpu[:3])
-    # rotate among enough input sets that the step's inputs are not L2-resident
-    n_sets = max(2, -(-3 * L2_BYTES // in_bytes))
-    sets = []
-    for i in range(n_sets):
-        if i == 0:
-            sets.append([t.cuda() for t in inputs_cpu])
-        else:
-            sets.append([(t.cuda() * 1.0).roll(i, dims=0) if t.dim() == 4 else t.cuda() for t in inputs_cpu])
-    OH, OW = wl.out_hw
-    outs = [torch.empty((wl.N, OH, OW, wl.C), dtype=wl.torch_dtype, device="cuda") for _ in range(n_sets)]
     stream = torch.cuda.Stream() if not args.no_graph else torch.cuda.current_stream()
-
-    def step(i):
-        s = sets[i % n_sets]
-        halo.attn(*s, block=wl.block, halo=wl.halo, stride=wl.stride, out=outs[i % n_sets], stream=stream)
-
-    kernel = halo.kernel_name(wl.N, wl.H, wl.W, wl.heads, wl.dim_head, wl.block, wl.halo, wl.stride,
-                              wl.torch_dtype)
-    with torch.cuda.stream(stream):
-        for i in range(args.warmup):
-            step(i)
-    torch.cuda.synchronize()
+    bench = DeviceBench(halo, wl, inputs_cpu, stream, use_graph=not args.no_graph)
+    kernel = bench.kernel
+    bench.warmup(args.warmup)
     # The timed steps replay CUDA graphs of the same launches (one kernel per
     # step, inputs rotating as above), so that the host's per-call cost
-    # (tensor-map encoding, argument checks) does not pace the GPU: a graph of
-    # `per` steps replayed steps // per times, then one of the remaining steps.
-    graphs = []
-    if not args.no_graph:
-        per = n_sets * max(1, -(-64 // n_sets))
-        plan = [(per, args.steps // per), (args.steps % per, 1)]
-        start = 0
-        for n, reps in plan:
-            if n == 0 or reps == 0:
-                continue
-            g = torch.cuda.CUDAGraph()
-            with torch.cuda.graph(g, stream=stream):
-                for i in range(n):
-                    step(start + i)
-            graphs.append((g, reps))
-            start += n
-        with torch.cuda.stream(stream):
-            for g, _ in graphs:
-                g.replay()
-        torch.cuda.synchronize()
-    barrier(world)
+    # (tensor-map encoding, argument checks) does not pace the GPU.
+    bench.prepare(args.steps)
+    # A short run (few steps) is timed as several regions of exactly K steps
+    # each, bracketed like the first, and the median region is reported.
+    est = bench.region()
+    repeats = max(1, min(100, int(math.ceil(args.min_timed_s * 1e3 / max(est, 1e-3)))))
     sampler = ClockSampler(local)
     sampler.start()
-    torch.cuda.synchronize()
-    barrier(world)
-    ev0 = torch.cuda.Event(enable_timing=True)
-    ev1 = torch.cuda.Event(enable_timing=True)
+    regions = []
     t_host0 = time.time()
-    ev0.record(stream)
-    with torch.cuda.stream(stream):
-        if graphs:
-            for g, reps in graphs:
-                for _ in range(reps):
-                    g.replay()
-        else:
-            for i in range(args.steps):
-                step(i)
-    ev1.record(stream)
-    ev1.synchronize()
-    torch.cuda.synchronize()
+    for _ in range(repeats):
+        barrier(world)
+        torch.cuda.synchronize()
+        r = bench.region()
+        torch.cuda.synchronize()
+        barrier(world)
+        regions.append(r)
     t_host1 = time.time()
-    barrier(world)
-    sampler.stop()
-    ms_local = ev0.elapsed_time(ev1)
+    ms_local = statistics.median(regions)
     ms = max_over_ranks(ms_local, world)
     err = halo.get_last_error()
     if err != 0:
         raise RuntimeError(f"device error flag {err} after the timed region")
-    clocks = sampler.summary(t_host0, t_host1)
+    peaks = measured_peaks()
+    configs = None
+    if rank == 0 and world == 1 and not args.no_per_config:
+        bench.release()
+        torch.cuda.empty_cache()
+        configs = per_config(halo, stream, sampler, peaks)
+    # nvidia-smi buffers its file output: read the samples once it has stopped
+    sampler.stop()
+    clocks = sampler.summary(t_host0, t_host1, keep=True)
+    for entry in (configs or {}).values():
+        entry["clocks"] = sampler.summary(*entry["clocks"], keep=True)
+    sampler.cleanup()
 
     # end to end through the host entry point: H2D inputs, kernel, D2H output
+    OH, OW = wl.out_hw
     h2d = sum(t.numel() * t.element_size() for t in inputs_cpu)
     d2h = wl.out_pixels * wl.C * wl.elem_bytes
     e2e = None
     if args.e2e_steps > 0:
         pinned = [t.pin_memory() for t in inputs_cpu]
         out_h = torch.empty((wl.N, OH, OW, wl.C), dtype=wl.torch_dtype).pin_memory()
-        staging = dict(zip(("q", "k", "v", "rel_h", "rel_w"), sets[0]))
-        staging["out"] = outs[0]
+        staging = dict(zip(("q", "k", "v", "rel_h", "rel_w"), [torch.empty_like(t, device="cuda")
+                                                              for t in inputs_cpu]))
+        staging["out"] = torch.empty((wl.N, OH, OW, wl.C), dtype=wl.torch_dtype, device="cuda")
         for _ in range(2):
             halo.attn_host(*pinned, out_h, staging, block=wl.block, halo=wl.halo, stride=wl.stride, stream=stream)
         torch.cuda.synchronize()
@@ -410,7 +553,6 @@ def main():
     pixels = wl.out_pixels * world
     value = pixels / per_step_s
     tflops = wl.flops() * world / per_step_s * 1e-12
-    peaks = measured_peaks()
     launch_s = ms_local * 1e-3 / args.steps  # one launch per step on this stream
     achieved_gbs = wl.bytes() / launch_s * 1e-9
     traffic = ncu_traffic(wl.name, kernel)
@@ -421,6 +563,7 @@ def main():
         "n_gpus": world,
         "steps": args.steps,
         "warmup": args.warmup,
+        "repeats": repeats,
         "ms_per_step": ms / args.steps,
         "higher_is_better": True,
         "scaling": "weak",
@@ -430,9 +573,11 @@ def main():
         "config": {"workload": f"{wl.name}: N={wl.N} per GPU, {wl.H}x{wl.W}, heads={wl.heads}, "
                                f"dim_head={wl.dim_head}, block={wl.block}, halo={wl.halo}, stride={wl.stride}",
                    "global_batch": wl.N * world, "parallelism": f"replicas x{world} (batch sharding)",
-                   "l2": f"inputs rotate over {n_sets} sets ({n_sets * in_bytes / 2**20:.0f} MiB) > L2",
+                   "l2": f"inputs rotate over {bench.n_sets} sets ({bench.n_sets * bench.in_bytes / 2**20:.0f} MiB) > L2",
                    "launch": ("one launch per step from Python" if args.no_graph else
                               "CUDA graphs of the per-step launches, replayed"),
+                   "timing": f"median of {repeats} timed regions of exactly {args.steps} steps each, "
+                             "each bracketed by a barrier and a device synchronisation",
                    "kernel": kernel},
         "tflops": tflops,
         "roofline": {"bound": "hbm", "achieved": achieved_gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
@@ -442,9 +587,10 @@ def main():
                      "algorithmic_bytes_per_launch": wl.bytes(),
                      "tensor_frac": tflops / world / peaks["bf16_tflops"]},
         "e2e": e2e,
-        "gpu_launches": args.steps,
+        "gpu_launches": args.steps * repeats,
         "clocks": clocks,
         "cpu_baseline": base,
+        "per_config": configs,
     }
     print(json.dumps(line), flush=True)
     return 0

@@ -12,6 +12,7 @@
 #include <mutex>
 
 #include "../../include/halo.h"
+#include "halo_bwd.cuh"
 #include "halo_simt.cuh"
 #include "halo_tc.cuh"
 #include "halo_tc2.cuh"
@@ -37,12 +38,15 @@ const char* status_text(int code) {
     case HALO_ERR_DTYPE: return "dtype must be HALO_F32 or HALO_BF16";
     case HALO_ERR_ALIAS: return "out overlaps an input";
     case HALO_ERR_DEVICE: return "the current device is not an sm_100 GPU";
+    case HALO_ERR_KERNEL: return "the SASA mask size must be odd, and at most 2*halo+1";
+    case HALO_ERR_WORKSPACE: return "the workspace is missing, misaligned or too small";
     default: return "unknown status code";
   }
 }
 
 struct Shape {
   int N, H, W, heads, d, block, halo, stride, dtype;
+  int kmask = 0;  // SASA mask size: 0 = none, else odd k with k / 2 <= halo
   size_t elem() const { return dtype == HALO_F32 ? 4 : 2; }
   size_t in_bytes() const { return static_cast<size_t>(N) * H * W * heads * d * elem(); }
   size_t out_bytes() const { return static_cast<size_t>(N) * (H / stride) * (W / stride) * heads * d * elem(); }
@@ -62,6 +66,7 @@ int check_shape(const Shape& s) {
   if (s.stride != 1 && s.stride != 2) return HALO_ERR_STRIDE;
   if (s.H % s.block || s.W % s.block || s.block % s.stride) return HALO_ERR_DIVISIBILITY;
   if ((C * static_cast<long long>(s.elem())) % 16 != 0) return HALO_ERR_ALIGN;
+  if (s.kmask < 0 || (s.kmask > 0 && (s.kmask % 2 == 0 || s.kmask / 2 > s.halo))) return HALO_ERR_KERNEL;
   return HALO_OK;
 }
 
@@ -148,13 +153,16 @@ const Tc3Entry* find_tc3(const Shape& s) {
 using Tc4Kernel = void (*)(const CUtensorMap, const CUtensorMap, const CUtensorMap, const halo::tc4::Params);
 struct Tc4Entry {
   int d, win;
-  Tc4Kernel fn;
+  Tc4Kernel fn, fn_masked;  // fn_masked: the SASA-masked instantiation
   int (*smem)(int);
 };
 template <int D, int WIN>
 int tc4_smem(int stages) { return halo::tc4::smem_bytes<D, WIN>(stages); }
-#define HALO_TC4_ENTRY(D, WIN) \
-  Tc4Entry { D, WIN, halo::tc4::halo_fwd_tc4<D, WIN>, tc4_smem<D, WIN> }
+#define HALO_TC4_ENTRY(D, WIN)                                                                     \
+  Tc4Entry {                                                                                       \
+    D, WIN, halo::tc4::halo_fwd_tc4<D, WIN, false>, halo::tc4::halo_fwd_tc4<D, WIN, true>,         \
+        tc4_smem<D, WIN>                                                                           \
+  }
 const Tc4Entry kTc4Table[] = {
     HALO_TC4_ENTRY(16, 8), HALO_TC4_ENTRY(16, 10), HALO_TC4_ENTRY(16, 12), HALO_TC4_ENTRY(16, 14),
     HALO_TC4_ENTRY(32, 8), HALO_TC4_ENTRY(32, 10), HALO_TC4_ENTRY(32, 12), HALO_TC4_ENTRY(32, 14),
@@ -179,7 +187,8 @@ const TcEntry* find_tc(const Shape& s) {
 
 int select_kernel(const Shape& s) {
   if (check_shape(s) != HALO_OK) return HALO_KERNEL_NONE;
-  if (find_tc4(s) || find_tc2(s) || find_tc(s) || find_tc3(s)) return HALO_KERNEL_TC_BF16;
+  if (s.kmask == 0 && (find_tc4(s) || find_tc2(s) || find_tc(s) || find_tc3(s))) return HALO_KERNEL_TC_BF16;
+  if (s.kmask > 0 && find_tc4(s)) return HALO_KERNEL_TC_BF16;
   if (s.d <= 128) return HALO_KERNEL_SIMT_F32;
   return HALO_KERNEL_NONE;
 }
@@ -270,7 +279,7 @@ cudaError_t launch_simt_t(const void* q, const void* k, const void* v, const voi
   halo::simt::halo_fwd_simt<T, DMAX><<<static_cast<unsigned>(blocks), halo::simt::kThreads, 0, st>>>(
       static_cast<const T*>(q), static_cast<const T*>(k), static_cast<const T*>(v), static_cast<const T*>(rh),
       static_cast<const T*>(rw), static_cast<T*>(out), s.N, s.H, s.W, s.heads, s.d, s.block, s.halo, s.stride,
-      1.0f / std::sqrt(static_cast<float>(s.d)));
+      s.kmask, 1.0f / std::sqrt(static_cast<float>(s.d)));
   return cudaGetLastError();
 }
 
@@ -431,8 +440,9 @@ int launch_tc4(const Tc4Entry& e, const void* q, const void* k, const void* v, c
       !encode_nhwc(&mk, k, s, win, win + halo::tc4::kBlock, 1) ||
       !encode_nhwc(&mv, v, s, win, win + halo::tc4::kBlock, 1))
     return HALO_ERR_CUDA;
+  const Tc4Kernel fn = s.kmask > 0 ? e.fn_masked : e.fn;
   cudaFuncAttributes attr;
-  if (cudaFuncGetAttributes(&attr, reinterpret_cast<const void*>(e.fn)) != cudaSuccess) return HALO_ERR_CUDA;
+  if (cudaFuncGetAttributes(&attr, reinterpret_cast<const void*>(fn)) != cudaSuccess) return HALO_ERR_CUDA;
   if (256 * halo::tc4::kSoftmaxRegs + 128 * halo::tc4::kProducerRegs > halo::tc4::kThreads * attr.numRegs)
     return HALO_ERR_UNSUPPORTED;
   int optin = 0, dev = 0;
@@ -444,7 +454,7 @@ int launch_tc4(const Tc4Entry& e, const void* q, const void* k, const void* v, c
   while (stages > 1 && e.smem(stages) > budget) --stages;
   const int smem = e.smem(stages);
   if (smem > budget) return HALO_ERR_UNSUPPORTED;
-  if (cudaFuncSetAttribute(reinterpret_cast<const void*>(e.fn), cudaFuncAttributeMaxDynamicSharedMemorySize,
+  if (cudaFuncSetAttribute(reinterpret_cast<const void*>(fn), cudaFuncAttributeMaxDynamicSharedMemorySize,
                            smem) != cudaSuccess)
     return HALO_ERR_CUDA;
   halo::tc4::Params p;
@@ -463,8 +473,9 @@ int launch_tc4(const Tc4Entry& e, const void* q, const void* k, const void* v, c
   p.num_items = static_cast<int>(items);
   p.stages = stages;
   p.c = 1.4426950408889634f / std::sqrt(static_cast<float>(s.d));
+  p.kmask = s.kmask;
   const int grid = static_cast<int>(items < sm_count ? items : sm_count);
-  e.fn<<<grid, halo::tc4::kThreads, smem, st>>>(mq, mk, mv, p);
+  fn<<<grid, halo::tc4::kThreads, smem, st>>>(mq, mk, mv, p);
   return cudaGetLastError() == cudaSuccess ? HALO_OK : HALO_ERR_CUDA;
 }
 
@@ -481,6 +492,7 @@ int attn_device(const void* q, const void* k, const void* v, const void* rel_h, 
   if (rc != HALO_OK) return rc;
   if (kind == HALO_KERNEL_TC_BF16) {
     if (const Tc4Entry* e4 = find_tc4(s)) return launch_tc4(*e4, q, k, v, rel_h, rel_w, out, s, sm_count, st);
+    if (s.kmask > 0) return HALO_ERR_UNSUPPORTED;  // not reached: select_kernel routes masked shapes to tc4 or simt
     if (const Tc2Entry* e2 = find_tc2(s)) return launch_tc2(*e2, q, k, v, rel_h, rel_w, out, s, sm_count, st);
     if (const Tc3Entry* e3 = find_tc3(s)) return launch_tc3(*e3, q, k, v, rel_h, rel_w, out, s, sm_count, st);
     return launch_tc(*find_tc(s), q, k, v, rel_h, rel_w, out, s, sm_count, st);
@@ -490,14 +502,186 @@ int attn_device(const void* q, const void* k, const void* v, const void* rel_h, 
   return err == cudaSuccess ? HALO_OK : HALO_ERR_CUDA;
 }
 
+// ----------------------------------------------------------------------------
+// Backward
+// ----------------------------------------------------------------------------
+struct BwdPlan {
+  halo::bwd::Params p;
+  int smem;
+  size_t off_dk, off_dv, off_drh, off_drw, ws_bytes;  // workspace layout (bytes)
+};
+
+size_t align256(size_t x) { return (x + 255) / 256 * 256; }
+
+int bwd_plan(const Shape& s, BwdPlan* plan) {
+  int rc = check_shape(s);
+  if (rc != HALO_OK) return rc;
+  if (s.d != 8 && s.d != 16 && s.d != 32 && s.d != 64 && s.d != 128) return HALO_ERR_UNSUPPORTED;
+  halo::bwd::Params& p = plan->p;
+  p.N = s.N;
+  p.H = s.H;
+  p.W = s.W;
+  p.heads = s.heads;
+  p.block = s.block;
+  p.halo = s.halo;
+  p.stride = s.stride;
+  p.kmask = s.kmask;
+  p.w = s.block + 2 * s.halo;
+  p.R = 2 * p.w - 1;
+  p.nqx = s.block / s.stride;
+  p.nq = p.nqx * p.nqx;
+  p.nbx = s.W / s.block;
+  p.nby = s.H / s.block;
+  p.c = 1.4426950408889634f / std::sqrt(static_cast<float>(s.d));
+  p.s = 1.0f / std::sqrt(static_cast<float>(s.d));
+  // largest power-of-two query tile (at most 256) whose item fits in shared memory
+  const long long KS = static_cast<long long>(p.w) * p.w;
+  if (KS > (1 << 20)) return HALO_ERR_UNSUPPORTED;
+  int qt = 256;
+  while (qt > p.nq * 2) qt /= 2;
+  for (; qt >= 1; qt /= 2) {
+    const halo::bwd::Layout L(s.d, static_cast<int>(KS), qt, p.w, p.R);
+    if (L.bytes() <= kMaxDynSmem) break;
+  }
+  if (qt < 1) return HALO_ERR_UNSUPPORTED;
+  p.QT = qt < p.nq ? qt : p.nq;
+  p.ntiles = (p.nq + p.QT - 1) / p.QT;
+  plan->smem = halo::bwd::Layout(s.d, static_cast<int>(KS), p.QT, p.w, p.R).bytes();
+  p.num_items = static_cast<long long>(s.N) * p.nby * p.nbx * s.heads * p.ntiles;
+  const size_t nin = static_cast<size_t>(s.N) * s.H * s.W * s.heads * s.d;
+  const size_t ntab = static_cast<size_t>(p.R) * s.d;
+  plan->off_dk = 0;
+  plan->off_dv = align256(nin * 4);
+  plan->off_drh = plan->off_dv + align256(nin * 4);
+  plan->off_drw = plan->off_drh + align256(ntab * 4);
+  plan->ws_bytes = plan->off_drw + align256(ntab * 4);
+  return HALO_OK;
+}
+
+template <typename T, int D>
+int launch_bwd_t(const BwdPlan& plan, const void* const* in, void* const* grads, void* ws, int sm_count,
+                 cudaStream_t st) {
+  auto fn = halo::bwd::halo_bwd_simt<T, D>;
+  if (cudaFuncSetAttribute(reinterpret_cast<const void*>(fn), cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           plan.smem) != cudaSuccess)
+    return HALO_ERR_CUDA;
+  int per_sm = 0;
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, fn, halo::bwd::kThreads, plan.smem) != cudaSuccess ||
+      per_sm < 1)
+    return HALO_ERR_UNSUPPORTED;
+  halo::bwd::Ptrs<T> g;
+  g.q = static_cast<const T*>(in[0]);
+  g.k = static_cast<const T*>(in[1]);
+  g.v = static_cast<const T*>(in[2]);
+  g.rel_h = static_cast<const T*>(in[3]);
+  g.rel_w = static_cast<const T*>(in[4]);
+  g.out = static_cast<const T*>(in[5]);
+  g.dout = static_cast<const T*>(in[6]);
+  g.dq = static_cast<T*>(grads[0]);
+  char* w = static_cast<char*>(ws);
+  g.dk32 = reinterpret_cast<float*>(w + plan.off_dk);
+  g.dv32 = reinterpret_cast<float*>(w + plan.off_dv);
+  g.drh32 = reinterpret_cast<float*>(w + plan.off_drh);
+  g.drw32 = reinterpret_cast<float*>(w + plan.off_drw);
+  const long long cap = static_cast<long long>(per_sm) * sm_count;
+  const int grid = static_cast<int>(plan.p.num_items < cap ? plan.p.num_items : cap);
+  fn<<<grid, halo::bwd::kThreads, plan.smem, st>>>(g, plan.p);
+  if (cudaGetLastError() != cudaSuccess) return HALO_ERR_CUDA;
+  const long long nin = static_cast<long long>(plan.p.N) * plan.p.H * plan.p.W * plan.p.heads * D;
+  const int ntab = plan.p.R * D;
+  const long long nmax = nin > ntab ? nin : ntab;
+  long long fb = (nmax + 255) / 256;
+  if (fb > 8LL * sm_count) fb = 8LL * sm_count;
+  halo::bwd::halo_bwd_finalize<T><<<static_cast<int>(fb), 256, 0, st>>>(
+      g.dk32, g.dv32, g.drh32, g.drw32, static_cast<T*>(grads[1]), static_cast<T*>(grads[2]),
+      static_cast<T*>(grads[3]), static_cast<T*>(grads[4]), nin, ntab);
+  return cudaGetLastError() == cudaSuccess ? HALO_OK : HALO_ERR_CUDA;
+}
+
+template <typename T>
+int launch_bwd(const BwdPlan& plan, int d, const void* const* in, void* const* grads, void* ws, int sm_count,
+               cudaStream_t st) {
+  switch (d) {
+    case 8: return launch_bwd_t<T, 8>(plan, in, grads, ws, sm_count, st);
+    case 16: return launch_bwd_t<T, 16>(plan, in, grads, ws, sm_count, st);
+    case 32: return launch_bwd_t<T, 32>(plan, in, grads, ws, sm_count, st);
+    case 64: return launch_bwd_t<T, 64>(plan, in, grads, ws, sm_count, st);
+    case 128: return launch_bwd_t<T, 128>(plan, in, grads, ws, sm_count, st);
+    default: return HALO_ERR_UNSUPPORTED;
+  }
+}
+
+// Shared by the workspace-taking backward entry point (and any variant that
+// brings its own scratch): checks, zeroing, the two launches.
+int attn_bwd(const void* const* in, void* const* grads, void* ws, size_t ws_bytes, const Shape& s,
+             cudaStream_t st) {
+  BwdPlan plan;
+  int rc = bwd_plan(s, &plan);
+  if (rc != HALO_OK) return rc;
+  for (int i = 0; i < 7; ++i)
+    if (!in[i]) return HALO_ERR_NULL;
+  for (int i = 0; i < 5; ++i)
+    if (!grads[i]) return HALO_ERR_NULL;
+  for (int i = 0; i < 7; ++i)
+    if (reinterpret_cast<uintptr_t>(in[i]) % 16) return HALO_ERR_ALIGN;
+  for (int i = 0; i < 5; ++i)
+    if (reinterpret_cast<uintptr_t>(grads[i]) % 16) return HALO_ERR_ALIGN;
+  if (!ws || reinterpret_cast<uintptr_t>(ws) % 256 || ws_bytes < plan.ws_bytes) return HALO_ERR_WORKSPACE;
+  // no gradient (or the workspace) may overlap an input or another gradient
+  const size_t ib = s.in_bytes(), ob = s.out_bytes(), rb = s.rel_bytes();
+  const size_t in_sz[7] = {ib, ib, ib, rb, rb, ob, ob};
+  const size_t g_sz[6] = {ib, ib, ib, rb, rb, plan.ws_bytes};
+  const void* gp[6] = {grads[0], grads[1], grads[2], grads[3], grads[4], ws};
+  for (int a = 0; a < 6; ++a) {
+    for (int i = 0; i < 7; ++i)
+      if (overlaps(gp[a], g_sz[a], in[i], in_sz[i])) return HALO_ERR_ALIAS;
+    for (int b = a + 1; b < 6; ++b)
+      if (overlaps(gp[a], g_sz[a], gp[b], g_sz[b])) return HALO_ERR_ALIAS;
+  }
+  int sm_count = 0;
+  rc = device_info(&sm_count);
+  if (rc != HALO_OK) return rc;
+  if (cudaMemsetAsync(ws, 0, plan.ws_bytes, st) != cudaSuccess) return HALO_ERR_CUDA;
+  // at stride 2 only the strided pixels are queries: dq is zero elsewhere
+  if (s.stride == 2 && cudaMemsetAsync(grads[0], 0, ib, st) != cudaSuccess) return HALO_ERR_CUDA;
+  return s.dtype == HALO_F32 ? launch_bwd<float>(plan, s.d, in, grads, ws, sm_count, st)
+                             : launch_bwd<__nv_bfloat16>(plan, s.d, in, grads, ws, sm_count, st);
+}
+
+// The self test's own result flag: a timeout that a real halo_attn recorded
+// in g_halo_error stays there for halo_get_last_error.
+__device__ int g_selftest_flag;
+
 __global__ void wait_timeout_kernel(unsigned long long limit_ns) {
   __shared__ __align__(8) uint64_t bar;
   if (threadIdx.x == 0) {
     halo::sm100::mbar_init(&bar, 1);
     halo::sm100::fence_mbar_init();
     // nothing ever arrives on `bar`: the wait must end by its time limit
-    if (!halo::sm100::mbar_wait(&bar, 0, limit_ns)) atomicExch(&halo::g_halo_error, HALO_ERR_TIMEOUT);
+    g_selftest_flag = halo::sm100::mbar_wait(&bar, 0, limit_ns) ? HALO_OK : HALO_ERR_TIMEOUT;
   }
+}
+
+const char* kernel_name_of(const Shape& s) {
+  thread_local char name[64];
+  const int kind = select_kernel(s);
+  if (kind == HALO_KERNEL_NONE) {
+    std::snprintf(name, sizeof(name), "none");
+  } else if (kind == HALO_KERNEL_TC_BF16) {
+    if (const Tc4Entry* e = find_tc4(s))
+      std::snprintf(name, sizeof(name), s.kmask > 0 ? "halo_fwd_tc4<%d,%d,masked>" : "halo_fwd_tc4<%d,%d>", e->d,
+                    e->win);
+    else if (const Tc2Entry* e = find_tc2(s)) std::snprintf(name, sizeof(name), "halo_fwd_tc2<%d,%d>", e->d, e->win);
+    else if (const Tc3Entry* e = find_tc3(s)) std::snprintf(name, sizeof(name), "halo_fwd_tc3<%d,%d>", e->d, e->win);
+    else {
+      const TcEntry* t = find_tc(s);
+      std::snprintf(name, sizeof(name), "halo_fwd_tc<%d,%d,%d>", t->d, t->win, t->stride);
+    }
+  } else {
+    const int dmax = s.d <= 16 ? 16 : s.d <= 32 ? 32 : s.d <= 64 ? 64 : 128;
+    std::snprintf(name, sizeof(name), "halo_fwd_simt<%s,%d>", s.dtype == HALO_F32 ? "float" : "bf16", dmax);
+  }
+  return name;
 }
 
 }  // namespace
@@ -558,6 +742,14 @@ int halo_attn_host(const void* q_h, const void* k_h, const void* v_h, const void
   if (rc != HALO_OK) return rc;
   std::lock_guard<std::mutex> pipe_lock(g_pipe_mutex);
   cudaStream_t st = static_cast<cudaStream_t>(stream);
+  // On an error after the first copy was queued, the caller's stream is still
+  // made to wait for everything already queued on the pipeline streams, so
+  // that synchronising it before freeing the buffers stays safe.
+  auto fail = [&](int code) {
+    for (int i = 0; i < 2; ++i)
+      if (cudaEventRecord(hp->ev_done[i], hp->st[i]) == cudaSuccess) cudaStreamWaitEvent(st, hp->ev_done[i], 0);
+    return code;
+  };
   // the tables first, on the caller's stream, then both pipeline streams wait
   // for everything queued on it so far
   const size_t rb = s.rel_bytes();
@@ -565,7 +757,7 @@ int halo_attn_host(const void* q_h, const void* k_h, const void* v_h, const void
       cudaMemcpyAsync(rel_w_d, rel_w_h, rb, cudaMemcpyHostToDevice, st) != cudaSuccess ||
       cudaEventRecord(hp->ev_in, st) != cudaSuccess || cudaStreamWaitEvent(hp->st[0], hp->ev_in, 0) != cudaSuccess ||
       cudaStreamWaitEvent(hp->st[1], hp->ev_in, 0) != cudaSuccess)
-    return HALO_ERR_CUDA;
+    return fail(HALO_ERR_CUDA);
   // chunks of whole images (NHWC: an image is a contiguous slice of every tensor)
   const int chunks = N < 8 ? N : 8;
   const size_t img_in = s.in_bytes() / N, img_out = s.out_bytes() / N;
@@ -579,21 +771,53 @@ int halo_attn_host(const void* q_h, const void* k_h, const void* v_h, const void
     if (cudaMemcpyAsync(dev(q_d, oi), host(q_h, oi), bi, cudaMemcpyHostToDevice, cs) != cudaSuccess ||
         cudaMemcpyAsync(dev(k_d, oi), host(k_h, oi), bi, cudaMemcpyHostToDevice, cs) != cudaSuccess ||
         cudaMemcpyAsync(dev(v_d, oi), host(v_h, oi), bi, cudaMemcpyHostToDevice, cs) != cudaSuccess)
-      return HALO_ERR_CUDA;
+      return fail(HALO_ERR_CUDA);
     Shape sc = s;
     sc.N = n1 - n0;
     rc = attn_device(dev(q_d, oi), dev(k_d, oi), dev(v_d, oi), rel_h_d, rel_w_d, dev(out_d, oo), sc, cs);
-    if (rc != HALO_OK) return rc;
+    if (rc != HALO_OK) return fail(rc);
     if (cudaMemcpyAsync(dev(out_h, oo), dev(out_d, oo), bo, cudaMemcpyDeviceToHost, cs) != cudaSuccess)
-      return HALO_ERR_CUDA;
+      return fail(HALO_ERR_CUDA);
   }
   // work queued on the caller's stream after this call waits for both
   if (cudaEventRecord(hp->ev_done[0], hp->st[0]) != cudaSuccess ||
       cudaEventRecord(hp->ev_done[1], hp->st[1]) != cudaSuccess ||
       cudaStreamWaitEvent(st, hp->ev_done[0], 0) != cudaSuccess ||
       cudaStreamWaitEvent(st, hp->ev_done[1], 0) != cudaSuccess)
-    return HALO_ERR_CUDA;
+    return fail(HALO_ERR_CUDA);
   return HALO_OK;
+}
+
+int halo_attn_masked(const void* q, const void* k, const void* v, const void* rel_h, const void* rel_w, void* out,
+                     int N, int H, int W, int heads, int dim_head, int block, int halo, int stride, int kernel,
+                     int dtype, void* stream) {
+  Shape s{N, H, W, heads, dim_head, block, halo, stride, dtype};
+  s.kmask = kernel;
+  if (kernel <= 0) return HALO_ERR_KERNEL;
+  return attn_device(q, k, v, rel_h, rel_w, out, s, static_cast<cudaStream_t>(stream));
+}
+
+int halo_attn_bwd_workspace_size(int N, int H, int W, int heads, int dim_head, int block, int halo, int stride,
+                                 int kernel, int dtype, size_t* bytes) {
+  if (!bytes) return HALO_ERR_NULL;
+  Shape s{N, H, W, heads, dim_head, block, halo, stride, dtype};
+  s.kmask = kernel;
+  BwdPlan plan;
+  const int rc = bwd_plan(s, &plan);
+  if (rc != HALO_OK) return rc;
+  *bytes = plan.ws_bytes;
+  return HALO_OK;
+}
+
+int halo_attn_bwd(const void* q, const void* k, const void* v, const void* rel_h, const void* rel_w,
+                  const void* out, const void* dout, void* dq, void* dk, void* dv, void* drel_h, void* drel_w,
+                  void* workspace, size_t workspace_bytes, int N, int H, int W, int heads, int dim_head, int block,
+                  int halo, int stride, int kernel, int dtype, void* stream) {
+  Shape s{N, H, W, heads, dim_head, block, halo, stride, dtype};
+  s.kmask = kernel;
+  const void* in[7] = {q, k, v, rel_h, rel_w, out, dout};
+  void* grads[5] = {dq, dk, dv, drel_h, drel_w};
+  return attn_bwd(in, grads, workspace, workspace_bytes, s, static_cast<cudaStream_t>(stream));
 }
 
 int halo_kernel_for(int N, int H, int W, int heads, int dim_head, int block, int halo, int stride, int dtype) {
@@ -603,24 +827,16 @@ int halo_kernel_for(int N, int H, int W, int heads, int dim_head, int block, int
 
 const char* halo_kernel_name(int N, int H, int W, int heads, int dim_head, int block, int halo, int stride,
                              int dtype) {
-  thread_local char name[64];
   const Shape s{N, H, W, heads, dim_head, block, halo, stride, dtype};
-  const int kind = select_kernel(s);
-  if (kind == HALO_KERNEL_NONE) {
-    std::snprintf(name, sizeof(name), "none");
-  } else if (kind == HALO_KERNEL_TC_BF16) {
-    if (const Tc4Entry* e = find_tc4(s)) std::snprintf(name, sizeof(name), "halo_fwd_tc4<%d,%d>", e->d, e->win);
-    else if (const Tc2Entry* e = find_tc2(s)) std::snprintf(name, sizeof(name), "halo_fwd_tc2<%d,%d>", e->d, e->win);
-    else if (const Tc3Entry* e = find_tc3(s)) std::snprintf(name, sizeof(name), "halo_fwd_tc3<%d,%d>", e->d, e->win);
-    else {
-      const TcEntry* t = find_tc(s);
-      std::snprintf(name, sizeof(name), "halo_fwd_tc<%d,%d,%d>", t->d, t->win, t->stride);
-    }
-  } else {
-    const int dmax = s.d <= 16 ? 16 : s.d <= 32 ? 32 : s.d <= 64 ? 64 : 128;
-    std::snprintf(name, sizeof(name), "halo_fwd_simt<%s,%d>", s.dtype == HALO_F32 ? "float" : "bf16", dmax);
-  }
-  return name;
+  return kernel_name_of(s);
+}
+
+const char* halo_masked_kernel_name(int N, int H, int W, int heads, int dim_head, int block, int halo, int stride,
+                                    int kernel, int dtype) {
+  Shape s{N, H, W, heads, dim_head, block, halo, stride, dtype};
+  s.kmask = kernel;
+  if (kernel <= 0) return "none";
+  return kernel_name_of(s);
 }
 
 const char* halo_strerror(int code) { return status_text(code); }
@@ -643,10 +859,7 @@ int halo_debug_wait_timeout(int limit_us, void* stream) {
   wait_timeout_kernel<<<1, 32, 0, st>>>(static_cast<unsigned long long>(limit_us) * 1000ull);
   if (cudaGetLastError() != cudaSuccess || cudaStreamSynchronize(st) != cudaSuccess) return HALO_ERR_CUDA;
   int flag = 0;
-  const int zero = 0;
-  if (cudaMemcpyFromSymbol(&flag, halo::g_halo_error, sizeof(int)) != cudaSuccess ||
-      cudaMemcpyToSymbol(halo::g_halo_error, &zero, sizeof(int)) != cudaSuccess)
-    return HALO_ERR_CUDA;
+  if (cudaMemcpyFromSymbol(&flag, g_selftest_flag, sizeof(int)) != cudaSuccess) return HALO_ERR_CUDA;
   return flag;
 }
 

@@ -26,7 +26,9 @@
 //   * softmax (one thread per TMEM lane = one query row): pass 1 takes the
 //     raw S maximum of every window row (before G is needed), then an upper
 //     bound of the row maximum, max over rows of c*S_max + c*rel_h plus the
-//     maximum of c*rel_w (at most a few units above the exact one);
+//     maximum of c*rel_w (a few units above the exact one with HaloNet's
+//     tables; when a lower bound from the block's own keys says it may be
+//     more than 100 log2 units above, the exact maximum is taken instead);
 //     pass 2 the exponentials (MUFU and the FMA-pipe cubic) and bf16 P
 //     written back over the S columns.  Both passes walk the row in pieces
 //     of 32 keys with the next piece's TMEM load in flight.
@@ -94,6 +96,7 @@ struct Params {
   int num_items;   // N * npy * nbx * heads
   int stages;
   float c;         // log2(e) / sqrt(d)
+  int kmask;       // SASA mask size (MASK instantiations only): keys within kmask/2 of the query
 };
 
 template <int D, int WIN>
@@ -204,8 +207,19 @@ __host__ __device__ constexpr int pp_pend(int i) { return (32 * (i + 1) < C::KP)
 template <class C>
 __host__ __device__ constexpr int pp_count() { return (C::KP + 31) / 32; }
 
+// Window-column pairs (kc, kc + 1), kc even, that lie inside the block's own
+// eight columns [h, h + 8): those keys are never outside the image.
+template <int WIN>
+__host__ __device__ constexpr bool own_pair(int kc) {
+  return kc >= (WIN - kBlock) / 2 && kc + 1 < (WIN - kBlock) / 2 + kBlock;
+}
+
+// Pass 1 keeps two maxima per window row: rmo over the own-column pairs
+// (in-image keys only) and rm over the other pairs; the caller merges them.
+// rmo also yields a lower bound of the exact row maximum (see the caller).
 template <int WIN, class C, int I>
-__device__ __forceinline__ void max_pipe(uint32_t ts, float (&rm)[WIN], float (&cur)[32], float (&nxt)[32]) {
+__device__ __forceinline__ void max_pipe(uint32_t ts, float (&rm)[WIN], float (&rmo)[WIN], float (&cur)[32],
+                                         float (&nxt)[32]) {
   constexpr int J0 = 32 * I, J1 = pp_end<C>(I);
   if constexpr (I + 1 < pp_count<C>()) {
     constexpr int K0 = 32 * (I + 1), K1 = pp_end<C>(I + 1);
@@ -214,19 +228,43 @@ __device__ __forceinline__ void max_pipe(uint32_t ts, float (&rm)[WIN], float (&
 #pragma unroll
   for (int i = 0; i < (J1 - J0) / 2; ++i) {
     const int r = (J0 + 2 * i) / WIN;
-    rm[r] = max3f(rm[r], cur[2 * i], cur[2 * i + 1]);
+    if (own_pair<WIN>((J0 + 2 * i) % WIN)) rmo[r] = max3f(rmo[r], cur[2 * i], cur[2 * i + 1]);
+    else rm[r] = max3f(rm[r], cur[2 * i], cur[2 * i + 1]);
   }
   if constexpr (I + 1 < pp_count<C>()) {
     tmem_wait_ld();
-    max_pipe<WIN, C, I + 1>(ts, rm, nxt, cur);
+    max_pipe<WIN, C, I + 1>(ts, rm, rmo, nxt, cur);
   }
 }
 template <int WIN, class C>
-__device__ __forceinline__ void row_max_pipelined(uint32_t ts, float (&rm)[WIN]) {
+__device__ __forceinline__ void row_max_pipelined(uint32_t ts, float (&rm)[WIN], float (&rmo)[WIN]) {
   float za[32], zb[32];
   tmem_ld_cols<(pp_end<C>(0) + 7) / 8 * 8>(ts, za);
   tmem_wait_ld();
-  max_pipe<WIN, C, 0>(ts, rm, za, zb);
+  max_pipe<WIN, C, 0>(ts, rm, rmo, za, zb);
+}
+
+// Exact row maximum of c * S + rh[row] + rw[col] over the window (masked rows
+// and columns carry -inf in rh / rw).  Taken only when the cheap bound of the
+// caller may lie too far above the exact maximum; not pipelined.  Whole-warp
+// (tcgen05.ld): the caller takes it for every thread of the warp.
+template <int WIN, class C>
+__device__ __forceinline__ float exact_row_max(uint32_t ts, const float (&rh)[WIN], const float (&rw)[WIN], float c) {
+  float m = -INFINITY;
+#pragma unroll
+  for (int i = 0; i < pp_count<C>(); ++i) {
+    const int j0 = 32 * i, j1 = (32 * (i + 1) < C::KS) ? 32 * (i + 1) : C::KS;
+    float z[32];
+    tmem_ld_x8(ts + j0, z);
+    tmem_ld_x8(ts + j0 + 8, z + 8);
+    tmem_ld_x8(ts + j0 + 16, z + 16);
+    tmem_ld_x8(ts + j0 + 24, z + 24);
+    tmem_wait_ld();
+#pragma unroll
+    for (int t = 0; t < 32; ++t)
+      if (j0 + t < j1) m = fmaxf(m, fmaf(z[t], c, rh[(j0 + t) / WIN] + rw[(j0 + t) % WIN]));
+  }
+  return m;
 }
 
 template <int WIN, class C, int I>
@@ -272,7 +310,13 @@ __device__ __forceinline__ void exp_pipelined(uint32_t ts, const float (&rw)[WIN
   exp_pipe<WIN, C, 0>(ts, rw, brow, c, za, zb);
 }
 
-template <int D, int WIN>
+// MASK: the SASA-masked variant (section 2.2: halo floor(k/2) and a mask
+// keeping the k x k keys centred on each query).  That mask is a band of
+// window rows times a band of window columns per query, so it is applied
+// through the query's rel_h / rel_w logits (-inf outside the bands), and the
+// row maximum is always the exact one (the own-column lower bound of the
+// unmasked kernel does not hold once own columns can be masked).
+template <int D, int WIN, bool MASK>
 __global__ void __launch_bounds__(kThreads, 1)
     halo_fwd_tc4(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__ CUtensorMap tmap_k,
                  const __grid_constant__ CUtensorMap tmap_v, const Params p) {
@@ -482,10 +526,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int y0 = by * kBlock - p.halo, x0 = ic.bx * kBlock - p.halo;
 
       // ---- pass 1: per window row the maximum of the raw S values
-      float rm[WIN];
+      float rm[WIN], rmo[WIN];
 #pragma unroll
-      for (int r = 0; r < WIN; ++r) rm[r] = -INFINITY;
-      row_max_pipelined<WIN, C>(ts, rm);
+      for (int r = 0; r < WIN; ++r) rm[r] = rmo[r] = -INFINITY;
+      row_max_pipelined<WIN, C>(ts, rm, rmo);
       if (!mbar_wait(&bar_gfull[g], j & 1, kWaitNs, &abort_flag)) {
         if (!abort_flag) record_timeout(&abort_flag);
         break;
@@ -508,7 +552,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int kr = 0; kr < WIN; ++kr) {
           const int Y = y0 + kr;
           const float v = odd ? gh[kr] : gh[kr + 1];
-          rh[kr] = (Y >= 0 && Y < p.H) ? v * c : -INFINITY;
+          bool keep = Y >= 0 && Y < p.H;
+          if constexpr (MASK) keep = keep && kr - qy - p.halo <= (p.kmask >> 1) && qy + p.halo - kr <= (p.kmask >> 1);
+          rh[kr] = keep ? v * c : -INFINITY;
         }
         const int sh = 7 - qx;
 #pragma unroll
@@ -520,18 +566,38 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
         for (int kc = 0; kc < WIN; ++kc) {
           const int X = x0 + kc;
-          rwz[kc] = (X >= 0 && X < p.W) ? a[kc] : -INFINITY;
+          bool keep = X >= 0 && X < p.W;
+          if constexpr (MASK) keep = keep && kc - qx - p.halo <= (p.kmask >> 1) && qx + p.halo - kc <= (p.kmask >> 1);
+          rwz[kc] = keep ? a[kc] : -INFINITY;
           rw[kc] = rwz[kc] * c;
         }
       }
 
-      float mw = -INFINITY;
+      // Upper bound of the row maximum: max over rows of (c * raw row max +
+      // rel_h) plus the largest rel_w.  It lies above the exact maximum by at
+      // most the spread of the rel_w logits, plus, at the image border, the
+      // gap between the valid keys' logits and the zero-filled masked keys'
+      // S = 0.  A lower bound comes from the own-column pairs of the block's
+      // own rows (in-image keys only): max over those rows of (c * own row
+      // max + rel_h) plus the smallest rel_w of those columns.  While the two
+      // are within 100 log2 units the largest p is at least 2^-100 (no
+      // underflow of the row sum); beyond that (huge relative tables, or
+      // strongly negative logits at a border) the exact maximum is taken.
+      float mw = -INFINITY, mwo = INFINITY;
 #pragma unroll
-      for (int kc = 0; kc < WIN; ++kc) mw = fmaxf(mw, rw[kc]);
-      float m = -INFINITY;
+      for (int kc = 0; kc < WIN; ++kc) {
+        mw = fmaxf(mw, rw[kc]);
+        if (own_pair<WIN>(kc & ~1)) mwo = fminf(mwo, rw[kc]);
+      }
+      float m = -INFINITY, mlo = -INFINITY;
 #pragma unroll
-      for (int r = 0; r < WIN; ++r) m = fmaxf(m, fmaf(rm[r], c, rh[r]));
+      for (int r = 0; r < WIN; ++r) {
+        if (r >= C::HALO && r < C::HALO + kBlock) mlo = fmaxf(mlo, fmaf(rmo[r], c, rh[r]));
+        m = fmaxf(m, fmaf(fmaxf(rm[r], rmo[r]), c, rh[r]));
+      }
       m += mw;  // finite: the query's own block is in the image
+      mlo += mwo;
+      if (MASK || __any_sync(0xffffffffu, m - mlo > 100.0f)) m = exact_row_max<WIN, C>(ts, rh, rw, c);
       // ---- pass 2: p = 2^(c*(S + rel_w) + c*rel_h - m)
       float brow[WIN];
 #pragma unroll

@@ -62,7 +62,9 @@ typedef enum {
   HALO_ERR_TIMEOUT = -8,       /* a bounded device-side wait ran out (reported by halo_get_last_error) */
   HALO_ERR_DTYPE = -9,         /* dtype is not a halo_dtype_t value */
   HALO_ERR_ALIAS = -10,        /* out overlaps an input */
-  HALO_ERR_DEVICE = -11        /* the current device is not an sm_100 GPU */
+  HALO_ERR_DEVICE = -11,       /* the current device is not an sm_100 GPU */
+  HALO_ERR_KERNEL = -12,       /* SASA mask size not odd, or larger than 2*halo+1 */
+  HALO_ERR_WORKSPACE = -13     /* the backward's workspace is NULL, not 256-byte aligned or too small */
 } halo_status;
 
 /* Which kernel halo_attn would launch for a shape (halo_kernel_for). */
@@ -103,12 +105,67 @@ int halo_attn(const void* q, const void* k, const void* v, const void* rel_h, co
  * The work is ordered after everything queued on `stream` before the call,
  * and work queued on `stream` after the call waits for all of it; the call
  * returns without waiting: synchronise `stream` before reading out_h.  Calls
- * from several host threads are serialised by a library lock.
+ * from several host threads are serialised by a library lock.  When the call
+ * fails after some copies or kernels were queued, `stream` is still made to
+ * wait for them before the error is returned: synchronise it before freeing
+ * or reusing any buffer passed to the failed call.
  */
 int halo_attn_host(const void* q_h, const void* k_h, const void* v_h, const void* rel_h_h, const void* rel_w_h,
                    void* out_h, void* q_d, void* k_d, void* v_d, void* rel_h_d, void* rel_w_d, void* out_d,
                    int N, int H, int W, int heads, int dim_head, int block, int halo, int stride, int dtype,
                    void* stream);
+
+/*
+ * halo_attn_masked -- the SASA-masked variant (section 2.2, the paragraph
+ * after Figure 1: SASA uses the same blocking with halo = floor(k/2) and an
+ * attention mask that emulates a k x k pixel-centred window).  Same
+ * arguments and layouts as halo_attn plus `kernel` = k: each query keeps only
+ * the window keys (Y, X) with |Y - y| <= k/2 and |X - x| <= k/2 (and inside
+ * the image).  k must be odd with k/2 <= halo (HALO_ERR_KERNEL otherwise);
+ * k = 2*halo + 1 is SASA's setting.  The relative tables are indexed as in
+ * halo_attn.  Asynchronous on `stream`; allocates nothing.
+ */
+int halo_attn_masked(const void* q, const void* k, const void* v, const void* rel_h, const void* rel_w, void* out,
+                     int N, int H, int W, int heads, int dim_head, int block, int halo, int stride, int kernel,
+                     int dtype, void* stream);
+
+/*
+ * halo_attn_bwd -- gradients of a loss L with respect to q, k, v, rel_h and
+ * rel_w, given dout = dL/dout (the pages train this layer, section 2.2 and
+ * Figure 3; the gradient is the chain rule through the operation above):
+ *   with p the softmax weights of query i over its kept keys j,
+ *   dz_ij = p_ij (dout_i . v_j - dout_i . out_i)
+ *   dq_i  = s sum_j dz_ij (k_j + rel_h[a_ij] + rel_w[b_ij])
+ *   dk_j  = s sum_i dz_ij q_i,   dv_j = sum_i p_ij dout_i  (over every window holding j)
+ *   drel_h[a] = s sum over (image, head, query, key) with row index a of dz q, likewise drel_w
+ *
+ * Inputs (device, dtype `dtype`, 16-byte aligned): q, k, v, rel_h, rel_w as
+ * for halo_attn; out = the forward's output for these inputs (same layout as
+ * halo_attn's out; used for dout . out); dout = dL/dout, same layout.
+ * Outputs (device, same dtype, 16-byte aligned, overlapping no input and no
+ * other output): dq, dk, dv [N, H, W, heads*dim_head] (at stride 2 dq is zero
+ * at pixels that are not queries), drel_h, drel_w [2w-1, dim_head].
+ * `kernel`: 0 for halo_attn's operation, or the SASA mask size of
+ * halo_attn_masked.
+ * workspace: caller-owned device scratch of at least the size that
+ * halo_attn_bwd_workspace_size reports, 256-byte aligned (HALO_ERR_WORKSPACE
+ * otherwise); float32 accumulators, overwritten by the call.  The library
+ * allocates nothing.  dim_head must be 8, 16, 32, 64 or 128, and one block's
+ * window must fit the kernel's shared memory (HALO_ERR_UNSUPPORTED
+ * otherwise).  Asynchronous on `stream`; the workspace must stay untouched
+ * until the stream work is done.  Gradients are computed in float32 and
+ * rounded to the dtype once.
+ */
+int halo_attn_bwd(const void* q, const void* k, const void* v, const void* rel_h, const void* rel_w,
+                  const void* out, const void* dout, void* dq, void* dk, void* dv, void* drel_h, void* drel_w,
+                  void* workspace, size_t workspace_bytes, int N, int H, int W, int heads, int dim_head, int block,
+                  int halo, int stride, int kernel, int dtype, void* stream);
+
+/* Workspace bytes halo_attn_bwd needs for these arguments, in *bytes
+ * (2 N H W heads dim_head + 2 (2w - 1) dim_head floats, each part rounded up
+ * to 256 bytes).  Returns a halo_status; no device work. */
+int halo_attn_bwd_workspace_size(int N, int H, int W, int heads, int dim_head, int block, int halo, int stride,
+                                 int kernel, int dtype, size_t* bytes);
 
 /* Which kernel halo_attn would launch for these arguments (halo_kernel_t),
  * or HALO_KERNEL_NONE when the shape is rejected.  No device work. */
@@ -122,6 +179,11 @@ int halo_kernel_for(int N, int H, int W, int heads, int dim_head, int block, int
 const char* halo_kernel_name(int N, int H, int W, int heads, int dim_head, int block, int halo, int stride,
                              int dtype);
 
+/* As halo_kernel_name, for halo_attn_masked with mask size `kernel`
+ * (e.g. "halo_fwd_tc4<16,14,masked>"); "none" when the shape is rejected. */
+const char* halo_masked_kernel_name(int N, int H, int W, int heads, int dim_head, int block, int halo, int stride,
+                                    int kernel, int dtype);
+
 /* Static description of a status code; never NULL. */
 const char* halo_strerror(int code);
 
@@ -133,9 +195,11 @@ int halo_get_last_error(void);
  * halo_debug_wait_timeout -- failure-detection self test.  Launches one tiny
  * kernel that waits on an mbarrier nobody arrives at, with a limit of
  * `limit_us` microseconds (1 .. 1000000); when the limit runs out the kernel
- * records HALO_ERR_TIMEOUT in the device flag and returns normally.  Returns
- * the flag's value (it synchronises `stream`), so a working timeout path
- * returns HALO_ERR_TIMEOUT.  Touches no caller memory.
+ * records HALO_ERR_TIMEOUT in a flag of its own and returns normally.
+ * Returns that flag's value (it synchronises `stream`), so a working timeout
+ * path returns HALO_ERR_TIMEOUT.  It neither reads nor clears the flag that
+ * halo_get_last_error reports, so a timeout recorded by an earlier halo_attn
+ * stays there.  Touches no caller memory.
  */
 int halo_debug_wait_timeout(int limit_us, void* stream);
 

@@ -2,10 +2,11 @@
 element on the same seeded inputs.
 
 Tolerances (max-abs): 1e-4 for float32 inputs, 2e-2 for bf16 inputs with
-float32 accumulation.  Full-size workloads are compared on sampled output
-pixels (borders, corners and random interior pixels) that the oracle computes
-one by one; smaller cases that span many blocks, heads and a ragged number of
-work items are compared in full.
+float32 accumulation.  The five full-size workloads are compared on every
+output pixel (the multi-threaded oracle takes a few seconds each); smaller
+cases that span many blocks, heads and a ragged number of work items are
+compared in full too, and so are the numerics stress cases (large relative
+tables, strongly negative logits at the image border).
 """
 import numpy as np
 import pytest
@@ -76,14 +77,27 @@ def test_tiny_f32_full():
 
 
 @pytest.mark.parametrize("name", ["stage1_bf16", "deep_bf16", "stride2_bf16", "large_bf16"])
-def test_full_size_sampled(name):
+def test_full_size_every_pixel(name):
+    """The full-size workload in the launch configuration the benchmark times
+    (one launch over the whole batch), every output pixel against the oracle."""
+    wl = WORKLOADS[name]
+    inputs = make_inputs(wl)
+    got = _run(wl, inputs)
+    want = oracle.halo_attention(*inputs, block=wl.block, halo=wl.halo, stride=wl.stride)
+    _compare(got, want, TOL[wl.dtype], name)
+
+
+@pytest.mark.parametrize("name", ["stage1_bf16", "large_bf16"])
+def test_full_size_sampled_pixels_match_full_oracle(name):
+    """The oracle's sampled form (used by smaller checks) agrees with its full
+    form on the GPU output's pixels: borders, corners and random pixels."""
     wl = WORKLOADS[name]
     inputs = make_inputs(wl)
     got = _run(wl, inputs)
     smp = _samples(wl, 384)
     want = oracle.halo_attention_samples(*inputs, smp, block=wl.block, halo=wl.halo, stride=wl.stride)
     g = got[smp[:, 0], smp[:, 1], smp[:, 2]]
-    _compare(g, want, TOL[wl.dtype], name)
+    _compare(g, want, TOL[wl.dtype], name + " sampled")
 
 
 @pytest.mark.parametrize("name,kernel", [("stage1_bf16", "tc_bf16"), ("deep_bf16", "tc_bf16"),
@@ -205,6 +219,71 @@ def test_block16_running_maximum(scale):
     _compare(got, want, TOL["bf16"], f"block16 scale {scale}")
 
 
+# One case per tensor-core kernel family (the kernel name prefix it must
+# select), used by the large-relative-table stress test.
+FAMILY_CASES = {
+    "halo_fwd_tc4<16,": dict(N=2, H=32, W=24, heads=3, dim_head=16, block=8, halo=3, stride=1),
+    "halo_fwd_tc4<32,": dict(N=2, H=32, W=24, heads=3, dim_head=32, block=8, halo=3, stride=1),
+    "halo_fwd_tc4<64,": dict(N=2, H=32, W=24, heads=2, dim_head=64, block=8, halo=3, stride=1),
+    "halo_fwd_tc2<16,": dict(N=2, H=24, W=24, heads=4, dim_head=16, block=8, halo=3, stride=1),
+    "halo_fwd_tc2<32,": dict(N=2, H=24, W=24, heads=2, dim_head=32, block=8, halo=2, stride=1),
+    "halo_fwd_tc<64,14,1>": dict(N=2, H=24, W=24, heads=2, dim_head=64, block=8, halo=3, stride=1),
+    "halo_fwd_tc<16,14,2>": dict(N=2, H=32, W=32, heads=8, dim_head=16, block=8, halo=3, stride=2),
+    "halo_fwd_tc<32,14,2>": dict(N=2, H=32, W=32, heads=4, dim_head=32, block=8, halo=3, stride=2),
+    "halo_fwd_tc3<16,": dict(N=1, H=32, W=32, heads=2, dim_head=16, block=16, halo=3, stride=1),
+    "halo_fwd_tc3<32,": dict(N=1, H=32, W=48, heads=2, dim_head=32, block=16, halo=4, stride=1),
+}
+
+
+def _scaled(t, f):
+    """Multiply a bf16 tensor by a power of two (exact)."""
+    return (t.float() * f).to(t.dtype)
+
+
+@pytest.mark.parametrize("rel_scale", [8.0, 32.0, 64.0])
+@pytest.mark.parametrize("family", sorted(FAMILY_CASES))
+def test_large_relative_tables(family, rel_scale):
+    """Relative tables scaled by 8..64 and q by 4: the relative logits span
+    tens to hundreds of log2 units, so the two-block kernel's bound of the row
+    maximum overshoots by more than the exponential's range (its exact
+    maximum must take over), the block-16 kernel moves its running maximum
+    and rescales, and the per-chunk maxima of the other kernels see chunks
+    far below the row's maximum.  v is halved so that the near one-hot
+    outputs stay where rounding the output to bf16 fits the bar."""
+    case = FAMILY_CASES[family]
+    wl = custom("bigrel", dtype="bf16", **case)
+    h = _lib()
+    assert h.kernel_name(wl.N, wl.H, wl.W, wl.heads, wl.dim_head, wl.block, wl.halo, wl.stride,
+                         wl.torch_dtype).startswith(family)
+    q, k, v, rh, rw = make_inputs(wl, seed=21)
+    q, rh, rw, v = _scaled(q, 4.0), _scaled(rh, rel_scale), _scaled(rw, rel_scale), _scaled(v, 0.5)
+    got = _run(wl, (q, k, v, rh, rw))
+    want = oracle.halo_attention(q, k, v, rh, rw, block=wl.block, halo=wl.halo, stride=wl.stride)
+    _compare(got, want, TOL["bf16"], f"{family} rel x{rel_scale:g}")
+
+
+@pytest.mark.parametrize("family", sorted(FAMILY_CASES))
+def test_strongly_negative_logits_at_border(family):
+    """q and k anti-aligned (q = a u + noise, k = -a u + noise per head): every
+    in-image logit is strongly negative (about -150 log2 units and below),
+    while the zero-filled out-of-image keys of a border window give S = 0.
+    The two-block kernel's cheap bound of the row maximum then lies far above
+    the exact one; the output must still match."""
+    case = FAMILY_CASES[family]
+    wl = custom("antialign", dtype="bf16", **case)
+    q, k, v, rh, rw = make_inputs(wl, seed=22)
+    g = torch.Generator().manual_seed(23)
+    u = torch.randn((wl.heads, wl.dim_head), generator=g)
+    a = 6.0
+    base = (a * u).reshape(1, 1, 1, wl.C)
+    qa = (base + q.float()).to(torch.bfloat16)
+    ka = (-base + k.float()).to(torch.bfloat16)
+    v = _scaled(v, 0.5)
+    got = _run(wl, (qa, ka, v, rh, rw))
+    want = oracle.halo_attention(qa, ka, v, rh, rw, block=wl.block, halo=wl.halo, stride=wl.stride)
+    _compare(got, want, TOL["bf16"], f"{family} anti-aligned")
+
+
 def test_deterministic():
     wl = WORKLOADS["stage1_bf16"]
     inputs = [t.cuda() for t in make_inputs(wl)]
@@ -299,8 +378,10 @@ def test_timeout_path_reports_and_device_stays_usable():
     and the context keeps working."""
     h = _lib()
     from blocked_local_self_b200 import _native as n
+    assert h.get_last_error() == 0
     assert h.debug_wait_timeout(2000) == n.HALO_ERR_TIMEOUT
-    assert h.get_last_error() == 0  # the flag was cleared by the self test
+    assert h.debug_wait_timeout(2000) == n.HALO_ERR_TIMEOUT  # its own flag starts clear each call
+    assert h.get_last_error() == 0  # the self test does not set the operation's flag
     wl = WORKLOADS["tiny_f32"]
     inputs = make_inputs(wl)
     got = _run(wl, inputs)
