@@ -55,6 +55,8 @@ def parse_args():
                     help="repeat the K-step timed region until about this much time is covered (median reported)")
     ap.add_argument("--no-per-config", action="store_true",
                     help="skip timing every workload for the per_config object")
+    ap.add_argument("--no-extra", action="store_true",
+                    help="skip timing the backward and the SASA-masked forward (next_rows object)")
     return ap.parse_args()
 
 
@@ -427,36 +429,159 @@ def per_config(halo, stream, sampler, peaks, seconds=0.5):
     committed summary matches the kernel's sources, and the clocks seen."""
     res = {}
     for name, wl in workloads.WORKLOADS.items():
+        res[name] = time_forward(halo, wl, stream, peaks, seconds)
+    return res
+
+
+def time_forward(halo, wl, stream, peaks, seconds=0.5):
+    """One workload's forward: ms per launch, pixels/s, roofline fractions,
+    kernel, ncu traffic (when the committed summary matches the kernel's
+    sources) and the host-time window for the clock summary."""
+    inputs_cpu = workloads.make_inputs(wl)
+    kernel = halo.kernel_name(wl.N, wl.H, wl.W, wl.heads, wl.dim_head, wl.block, wl.halo, wl.stride,
+                              wl.torch_dtype)
+    t0 = time.time()
+    if wl.N * wl.H * wl.W * wl.C * wl.elem_bytes * 3 < L2_BYTES // 4:
+        ms = time_flushed_launches(halo, wl, inputs_cpu, stream)
+        how, steps, reps = "each launch alone after a 252 MiB (2x L2) flush; median of 200", 1, 200
+    else:
+        b = DeviceBench(halo, wl, inputs_cpu, stream)
+        b.warmup(10)
+        b.prepare(20)
+        est = b.region() / 20
+        steps = max(20, int(seconds * 1e3 / max(est, 1e-3)))
+        b.prepare(steps)
+        regions = [b.region() / steps for _ in range(3)]
+        ms = statistics.median(regions)
+        reps = 3
+        how = (f"median of 3 regions of {steps} graph-replayed launches, inputs rotating over "
+               f"{b.n_sets} sets ({b.n_sets * b.in_bytes / 2**20:.0f} MiB) > L2")
+        b.release()
+    t1 = time.time()
+    torch.cuda.synchronize()
+    err = halo.get_last_error()
+    if err != 0:
+        raise RuntimeError(f"device error flag {err} after timing {wl.name}")
+    entry = {"kernel": kernel, "ms": ms, "value": wl.out_pixels / (ms * 1e-3), "unit": "pixels/s",
+             "timing": how, "clocks": (t0, t1)}  # summarised once the sampler has stopped
+    entry.update(roofline_entry(wl, ms * 1e-3, peaks, ncu_traffic(wl.name, kernel)))
+    torch.cuda.empty_cache()
+    return entry
+
+
+# float32 FMA peak of the CUDA cores (148 SMs x 128 lanes x 2 FLOP x 1.965 GHz),
+# for kernels that run on them (the backward).
+FP32_CUDA_CORE_TFLOPS = 148 * 128 * 2 * 1.965e9 * 1e-12
+
+
+def bwd_bytes(wl) -> float:
+    """Unavoidable HBM traffic of the backward: q, k, v, out, dout read once,
+    dq, dk, dv written once (the tables are negligible)."""
+    e = wl.elem_bytes
+    inp = wl.N * wl.H * wl.W * wl.C * e
+    outp = wl.out_pixels * wl.C * e
+    return float(3 * inp + 2 * outp + 3 * inp)
+
+
+def bwd_flops(wl) -> float:
+    """Algorithmic FLOPs of the backward: the five window products per output
+    pixel and head (q.k again, dout.v, p dout, dz q, dz k), 2 d w^2 each."""
+    w = wl.window
+    return 10.0 * wl.dim_head * w * w * wl.heads * wl.out_pixels
+
+
+def time_extra(halo, stream, sampler, peaks, seconds=0.5):
+    """The NEXT rows measured in the same run: the backward on the stage-1 and
+    stride-2 workloads, and the SASA-masked forward (7 x 7 centred window,
+    the paper's comparison) on the stage-1 workload.  Inputs rotate over sets
+    larger than L2 as for the forward."""
+    res = {}
+    for name in ("stage1_bf16", "stride2_bf16"):
+        wl = workloads.WORKLOADS[name]
         inputs_cpu = workloads.make_inputs(wl)
-        kernel = halo.kernel_name(wl.N, wl.H, wl.W, wl.heads, wl.dim_head, wl.block, wl.halo, wl.stride,
-                                  wl.torch_dtype)
-        t0 = time.time()
-        if wl.N * wl.H * wl.W * wl.C * wl.elem_bytes * 3 < L2_BYTES // 4:
-            ms = time_flushed_launches(halo, wl, inputs_cpu, stream)
-            how, steps, reps = "each launch alone after a 252 MiB (2x L2) flush; median of 200", 1, 200
-        else:
-            b = DeviceBench(halo, wl, inputs_cpu, stream)
-            b.warmup(10)
-            b.prepare(20)
-            est = b.region() / 20
-            steps = max(20, int(seconds * 1e3 / max(est, 1e-3)))
-            b.prepare(steps)
-            regions = [b.region() / steps for _ in range(3)]
-            ms = statistics.median(regions)
-            reps = 3
-            how = (f"median of 3 regions of {steps} graph-replayed launches, inputs rotating over "
-                   f"{b.n_sets} sets ({b.n_sets * b.in_bytes / 2**20:.0f} MiB) > L2")
-            b.release()
-        t1 = time.time()
+        sets, in_bytes = make_device_sets(wl, inputs_cpu)
+        OH, OW = wl.out_hw
+        outs = [halo.attn(*st, block=wl.block, halo=wl.halo, stride=wl.stride) for st in sets]
+        g = torch.Generator().manual_seed(7)
+        douts = [torch.randn((wl.N, OH, OW, wl.C), generator=g).to(wl.torch_dtype).cuda() for _ in sets]
+        grads = [tuple(torch.empty_like(t) for t in st) for st in sets]
+        nbytes = halo.bwd_workspace_size(wl.N, wl.H, wl.W, wl.heads, wl.dim_head, wl.block, wl.halo, wl.stride, 0,
+                                         wl.torch_dtype)
+        ws = torch.empty(nbytes, dtype=torch.uint8, device="cuda")
+
+        def step(i):
+            j = i % len(sets)
+            halo.attn_bwd(*sets[j], outs[j], douts[j], block=wl.block, halo=wl.halo, stride=wl.stride,
+                          grads=grads[j], workspace=ws, stream=stream)
+
+        with torch.cuda.stream(stream):
+            for i in range(3):
+                step(i)
         torch.cuda.synchronize()
-        err = halo.get_last_error()
-        if err != 0:
-            raise RuntimeError(f"device error flag {err} after timing {name}")
-        entry = {"kernel": kernel, "ms": ms, "value": wl.out_pixels / (ms * 1e-3), "unit": "pixels/s",
-                 "timing": how, "clocks": (t0, t1)}  # summarised once the sampler has stopped
-        entry.update(roofline_entry(wl, ms * 1e-3, peaks, ncu_traffic(wl.name, kernel)))
-        res[name] = entry
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        with torch.cuda.stream(stream):
+            step(0)
+        e1.record(stream)
+        e1.synchronize()
+        est = e0.elapsed_time(e1)
+        steps = max(3, int(seconds * 1e3 / max(est, 1e-3)))
+        t0 = time.time()
+        e0.record(stream)
+        with torch.cuda.stream(stream):
+            for i in range(steps):
+                step(i)
+        e1.record(stream)
+        e1.synchronize()
+        t1 = time.time()
+        ms = e0.elapsed_time(e1) / steps
+        launch_s = ms * 1e-3
+        gbs = bwd_bytes(wl) / launch_s * 1e-9
+        tf = bwd_flops(wl) / launch_s * 1e-12
+        res["bwd_" + name] = {
+            "what": "halo_attn_bwd: dq, dk, dv, drel_h, drel_w (workspace zeroing, CUDA-core kernel, finalize)",
+            "kernel": "halo_bwd_simt", "ms": ms, "value": wl.out_pixels / launch_s, "unit": "pixels/s",
+            "timing": f"{steps} back-to-back calls, inputs rotating over {len(sets)} sets > L2",
+            "achieved_gbs": gbs, "hbm_frac": gbs / peaks["hbm_gbs"], "algorithmic_bytes": bwd_bytes(wl),
+            "tflops": tf, "flops": bwd_flops(wl), "fp32_alu_frac": tf / FP32_CUDA_CORE_TFLOPS,
+            "clocks": (t0, t1)}
+        del sets, outs, douts, grads, ws
         torch.cuda.empty_cache()
+        halo_err = halo.get_last_error()
+        if halo_err != 0:
+            raise RuntimeError(f"device error flag {halo_err} after the backward of {name}")
+    # SASA-masked forward, 7 x 7 centred window on the stage-1 layer
+    wl = workloads.WORKLOADS["stage1_bf16"]
+    inputs_cpu = workloads.make_inputs(wl)
+    b = DeviceBench(halo, wl, inputs_cpu, stream)
+    kern = 7
+
+    def sstep(i):
+        st = b.sets[i % b.n_sets]
+        halo.attn_masked(*st, block=wl.block, halo=wl.halo, kernel=kern, stride=wl.stride,
+                         out=b.outs[i % b.n_sets], stream=stream)
+
+    b.step = sstep
+    b.warmup(10)
+    b.prepare(20)
+    est = b.region() / 20
+    steps = max(20, int(seconds * 1e3 / max(est, 1e-3)))
+    b.prepare(steps)
+    t0 = time.time()
+    ms = statistics.median([b.region() / steps for _ in range(3)])
+    t1 = time.time()
+    kname = halo.masked_kernel_name(wl.N, wl.H, wl.W, wl.heads, wl.dim_head, wl.block, wl.halo, wl.stride, kern,
+                                    wl.torch_dtype)
+    entry = {"what": "halo_attn_masked, kernel 7 (SASA's 7 x 7 centred window) on the stage-1 layer",
+             "kernel": kname, "ms": ms, "value": wl.out_pixels / (ms * 1e-3), "unit": "pixels/s",
+             "timing": f"median of 3 regions of {steps} graph-replayed launches", "clocks": (t0, t1)}
+    entry.update(roofline_entry(wl, ms * 1e-3, peaks, None))
+    res["sasa_k7_stage1_bf16"] = entry
+    b.release()
+    torch.cuda.empty_cache()
+    # block 32: global attention on a 32x32 map, and block 32 with halo 3
+    for name, wl in workloads.NEXT_WORKLOADS.items():
+        res[name] = time_forward(halo, wl, stream, peaks, seconds)
     return res
 
 
@@ -507,10 +632,13 @@ def main():
         bench.release()
         torch.cuda.empty_cache()
         configs = per_config(halo, stream, sampler, peaks)
+    extra = None
+    if rank == 0 and world == 1 and not args.no_extra:
+        extra = time_extra(halo, stream, sampler, peaks)
     # nvidia-smi buffers its file output: read the samples once it has stopped
     sampler.stop()
     clocks = sampler.summary(t_host0, t_host1, keep=True)
-    for entry in (configs or {}).values():
+    for entry in list((configs or {}).values()) + list((extra or {}).values()):
         entry["clocks"] = sampler.summary(*entry["clocks"], keep=True)
     sampler.cleanup()
 
@@ -591,6 +719,7 @@ def main():
         "clocks": clocks,
         "cpu_baseline": base,
         "per_config": configs,
+        "next_rows": extra,
     }
     print(json.dumps(line), flush=True)
     return 0

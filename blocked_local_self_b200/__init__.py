@@ -18,8 +18,8 @@ import torch
 from . import _native
 from ._native import HaloError, HALO_BF16, HALO_F32
 
-__all__ = ["attn", "attn_host", "kernel_for", "kernel_name", "get_last_error", "debug_wait_timeout", "version", "HaloError",
-           "load"]
+__all__ = ["attn", "attn_masked", "attn_bwd", "bwd_workspace_size", "attn_host", "kernel_for", "kernel_name",
+           "masked_kernel_name", "get_last_error", "debug_wait_timeout", "version", "HaloError", "load"]
 
 
 def load():
@@ -77,6 +77,65 @@ def attn(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, rel_h: torch.Tensor,
     return out
 
 
+def attn_masked(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, rel_h: torch.Tensor, rel_w: torch.Tensor,
+                block: int, halo: int, kernel: int, stride: int = 1, heads: int | None = None,
+                out: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """SASA-masked variant: each query keeps only the ``kernel`` x ``kernel``
+    keys centred on it (``halo_attn_masked``)."""
+    for t in (q, k, v, rel_h, rel_w):
+        if not t.is_cuda or not t.is_contiguous():
+            raise ValueError("attn_masked expects contiguous CUDA tensors")
+    N, H, W, heads, d = _sizes(q, rel_h, heads)
+    if out is None:
+        out = torch.empty((N, H // stride, W // stride, heads * d), dtype=q.dtype, device=q.device)
+    rc = _native.lib().halo_attn_masked(q.data_ptr(), k.data_ptr(), v.data_ptr(), rel_h.data_ptr(),
+                                        rel_w.data_ptr(), out.data_ptr(), N, H, W, heads, d, block, halo, stride,
+                                        kernel, _dtype_code(q), _stream_ptr(stream))
+    if rc != 0:
+        raise HaloError(rc, "halo_attn_masked")
+    return out
+
+
+def bwd_workspace_size(N: int, H: int, W: int, heads: int, dim_head: int, block: int, halo: int, stride: int,
+                       kernel: int, dtype: torch.dtype) -> int:
+    """Bytes of device workspace ``attn_bwd`` needs (``halo_attn_bwd_workspace_size``)."""
+    import ctypes
+    nb = ctypes.c_size_t(0)
+    code = HALO_BF16 if dtype == torch.bfloat16 else HALO_F32
+    rc = _native.lib().halo_attn_bwd_workspace_size(N, H, W, heads, dim_head, block, halo, stride, kernel, code,
+                                                    ctypes.byref(nb))
+    if rc != 0:
+        raise HaloError(rc, "halo_attn_bwd_workspace_size")
+    return int(nb.value)
+
+
+def attn_bwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, rel_h: torch.Tensor, rel_w: torch.Tensor,
+             out: torch.Tensor, dout: torch.Tensor, block: int, halo: int, stride: int = 1, kernel: int = 0,
+             heads: int | None = None, grads: tuple | None = None, workspace: torch.Tensor | None = None,
+             stream=None):
+    """Gradients (dq, dk, dv, drel_h, drel_w) of ``sum(out * dout)``
+    (``halo_attn_bwd``).  ``out`` is the forward's output for these inputs.
+    ``grads`` may pass preallocated outputs and ``workspace`` a uint8 CUDA
+    tensor of at least ``bwd_workspace_size`` bytes."""
+    for t in (q, k, v, rel_h, rel_w, out, dout):
+        if not t.is_cuda or not t.is_contiguous():
+            raise ValueError("attn_bwd expects contiguous CUDA tensors")
+    N, H, W, heads, d = _sizes(q, rel_h, heads)
+    if grads is None:
+        grads = (torch.empty_like(q), torch.empty_like(k), torch.empty_like(v), torch.empty_like(rel_h),
+                 torch.empty_like(rel_w))
+    nbytes = bwd_workspace_size(N, H, W, heads, d, block, halo, stride, kernel, q.dtype)
+    if workspace is None:
+        workspace = torch.empty(nbytes, dtype=torch.uint8, device=q.device)
+    rc = _native.lib().halo_attn_bwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), rel_h.data_ptr(), rel_w.data_ptr(),
+                                     out.data_ptr(), dout.data_ptr(), *[g_.data_ptr() for g_ in grads],
+                                     workspace.data_ptr(), workspace.numel() * workspace.element_size(), N, H, W,
+                                     heads, d, block, halo, stride, kernel, _dtype_code(q), _stream_ptr(stream))
+    if rc != 0:
+        raise HaloError(rc, "halo_attn_bwd")
+    return grads
+
+
 def attn_host(q_h: torch.Tensor, k_h: torch.Tensor, v_h: torch.Tensor, rel_h_h: torch.Tensor,
               rel_w_h: torch.Tensor, out_h: torch.Tensor, staging: dict, block: int, halo: int, stride: int = 1,
               heads: int | None = None, stream=None) -> torch.Tensor:
@@ -109,6 +168,14 @@ def kernel_name(N: int, H: int, W: int, heads: int, dim_head: int, block: int, h
     """Instantiation ``attn`` launches for a shape, e.g. "halo_fwd_tc2<16,14>", or "none"."""
     code = HALO_BF16 if dtype == torch.bfloat16 else HALO_F32
     return _native.lib().halo_kernel_name(N, H, W, heads, dim_head, block, halo, stride, code).decode()
+
+
+def masked_kernel_name(N: int, H: int, W: int, heads: int, dim_head: int, block: int, halo: int, stride: int,
+                       kernel: int, dtype: torch.dtype) -> str:
+    """Instantiation ``attn_masked`` launches for a shape, or "none"."""
+    code = HALO_BF16 if dtype == torch.bfloat16 else HALO_F32
+    return _native.lib().halo_masked_kernel_name(N, H, W, heads, dim_head, block, halo, stride, kernel,
+                                                 code).decode()
 
 
 def get_last_error() -> int:

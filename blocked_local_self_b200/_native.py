@@ -27,6 +27,8 @@ HALO_ERR_TIMEOUT = -8
 HALO_ERR_DTYPE = -9
 HALO_ERR_ALIAS = -10
 HALO_ERR_DEVICE = -11
+HALO_ERR_KERNEL = -12
+HALO_ERR_WORKSPACE = -13
 
 HALO_KERNEL_NONE = 0
 HALO_KERNEL_SIMT_F32 = 1
@@ -39,8 +41,12 @@ _i = ctypes.c_int
 SIGNATURES = {
     "halo_attn": (_i, [_vp] * 6 + [_i] * 9 + [_vp]),
     "halo_attn_host": (_i, [_vp] * 12 + [_i] * 9 + [_vp]),
+    "halo_attn_masked": (_i, [_vp] * 6 + [_i] * 10 + [_vp]),
+    "halo_attn_bwd": (_i, [_vp] * 13 + [ctypes.c_size_t] + [_i] * 10 + [_vp]),
+    "halo_attn_bwd_workspace_size": (_i, [_i] * 10 + [ctypes.POINTER(ctypes.c_size_t)]),
     "halo_kernel_for": (_i, [_i] * 9),
     "halo_kernel_name": (ctypes.c_char_p, [_i] * 9),
+    "halo_masked_kernel_name": (ctypes.c_char_p, [_i] * 10),
     "halo_strerror": (ctypes.c_char_p, [_i]),
     "halo_get_last_error": (_i, []),
     "halo_debug_wait_timeout": (_i, [_i, _vp]),

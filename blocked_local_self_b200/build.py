@@ -14,7 +14,7 @@ ROOT = os.path.dirname(HERE)
 CSRC = os.path.join(HERE, "csrc")
 LIB = os.path.join(HERE, "libhalo.so")
 SOURCES = [os.path.join(CSRC, "halo_api.cu")]
-DEPS = SOURCES + [os.path.join(CSRC, f) for f in ("halo_tc.cuh", "halo_tc2.cuh", "halo_tc3.cuh", "halo_tc4.cuh", "halo_simt.cuh", "sm100.cuh")] + [
+DEPS = SOURCES + [os.path.join(CSRC, f) for f in ("halo_tc.cuh", "halo_tc2.cuh", "halo_tc3.cuh", "halo_tc4.cuh", "halo_simt.cuh", "halo_bwd.cuh", "sm100.cuh")] + [
     os.path.join(ROOT, "include", "halo.h")]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 FLAGS = ["-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC", "-shared", "-cudart", "static",

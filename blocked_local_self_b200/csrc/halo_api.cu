@@ -127,24 +127,27 @@ const Tc2Entry* find_tc2(const Shape& s) {
 // Stride-1 kernel for 16x16 query blocks: (d, window) -> instantiation.
 using Tc3Kernel = void (*)(const CUtensorMap, const CUtensorMap, const CUtensorMap, const halo::tc3::Params);
 struct Tc3Entry {
-  int d, win;
+  int d, win, block;
   Tc3Kernel fn;
   int (*smem)(int);
 };
-template <int D, int WIN>
-int tc3_smem(int stages) { return halo::tc3::smem_bytes<D, WIN>(stages); }
-#define HALO_TC3_ENTRY(D, WIN) \
-  Tc3Entry { D, WIN, halo::tc3::halo_fwd_tc3<D, WIN>, tc3_smem<D, WIN> }
-#define HALO_TC3_WINS(D)                                                                   \
-  HALO_TC3_ENTRY(D, 16), HALO_TC3_ENTRY(D, 18), HALO_TC3_ENTRY(D, 20), HALO_TC3_ENTRY(D, 22), \
-      HALO_TC3_ENTRY(D, 24)
+template <int D, int WIN, int BLOCK>
+int tc3_smem(int stages) { return halo::tc3::smem_bytes<D, WIN, BLOCK>(stages); }
+#define HALO_TC3_ENTRY(D, WIN, B) \
+  Tc3Entry { D, WIN, B, halo::tc3::halo_fwd_tc3<D, WIN, B>, tc3_smem<D, WIN, B> }
+#define HALO_TC3_WINS(D)                                                                                   \
+  HALO_TC3_ENTRY(D, 16, 16), HALO_TC3_ENTRY(D, 18, 16), HALO_TC3_ENTRY(D, 20, 16), HALO_TC3_ENTRY(D, 22, 16), \
+      HALO_TC3_ENTRY(D, 24, 16), HALO_TC3_ENTRY(D, 32, 32), HALO_TC3_ENTRY(D, 34, 32),                      \
+      HALO_TC3_ENTRY(D, 36, 32), HALO_TC3_ENTRY(D, 38, 32)
 const Tc3Entry kTc3Table[] = {HALO_TC3_WINS(16), HALO_TC3_WINS(32)};
 
+// 16x16 blocks (halo <= 4) and 32x32 blocks (halo <= 3: global attention on
+// a 32x32 map, and the block-32 detection setting)
 const Tc3Entry* find_tc3(const Shape& s) {
-  if (s.dtype != HALO_BF16 || s.block != halo::tc3::kBlock || s.stride != 1) return nullptr;
+  if (s.dtype != HALO_BF16 || (s.block != 16 && s.block != 32) || s.stride != 1) return nullptr;
   const int win = s.block + 2 * s.halo;
   for (const Tc3Entry& e : kTc3Table)
-    if (e.d == s.d && e.win == win) return &e;
+    if (e.d == s.d && e.win == win && e.block == s.block) return &e;
   return nullptr;
 }
 
@@ -392,8 +395,11 @@ int launch_tc3(const Tc3Entry& e, const void* q, const void* k, const void* v, c
                void* out, const Shape& s, int sm_count, cudaStream_t st) {
   const int win = s.block + 2 * s.halo;
   CUtensorMap mq, mk, mv;
-  if (!encode_nhwc(&mq, q, s, halo::tc3::kBlock, halo::tc3::kBlock, 1) || !encode_nhwc(&mk, k, s, win, win, 1) ||
-      !encode_nhwc(&mv, v, s, win, win, 1))
+  // Q box: the item's 256 queries (a whole 16x16 block, or 8 rows of a 32x32 block)
+  // K / V box: window rows padded to the kernel's row pitch (block 32: a multiple of 8)
+  const int pitch = e.block == 16 ? win : (win + 7) / 8 * 8;
+  if (!encode_nhwc(&mq, q, s, e.block, 256 / e.block, 1) || !encode_nhwc(&mk, k, s, pitch, win, 1) ||
+      !encode_nhwc(&mv, v, s, pitch, win, 1))
     return HALO_ERR_CUDA;
   cudaFuncAttributes attr;
   if (cudaFuncGetAttributes(&attr, reinterpret_cast<const void*>(e.fn)) != cudaSuccess) return HALO_ERR_CUDA;
@@ -420,9 +426,10 @@ int launch_tc3(const Tc3Entry& e, const void* q, const void* k, const void* v, c
   p.W = s.W;
   p.heads = s.heads;
   p.halo = s.halo;
-  p.nbx = s.W / halo::tc3::kBlock;
-  p.nby = s.H / halo::tc3::kBlock;
-  const long long items = static_cast<long long>(s.N) * p.nbx * p.nby * s.heads;
+  p.nbx = s.W / e.block;
+  p.nby = s.H / e.block;
+  const int quarters = e.block * e.block / 256;
+  const long long items = static_cast<long long>(s.N) * p.nbx * p.nby * s.heads * quarters;
   if (items > 0x7fffffffLL) return HALO_ERR_DIMS;
   p.num_items = static_cast<int>(items);
   p.stages = stages;
@@ -672,7 +679,8 @@ const char* kernel_name_of(const Shape& s) {
       std::snprintf(name, sizeof(name), s.kmask > 0 ? "halo_fwd_tc4<%d,%d,masked>" : "halo_fwd_tc4<%d,%d>", e->d,
                     e->win);
     else if (const Tc2Entry* e = find_tc2(s)) std::snprintf(name, sizeof(name), "halo_fwd_tc2<%d,%d>", e->d, e->win);
-    else if (const Tc3Entry* e = find_tc3(s)) std::snprintf(name, sizeof(name), "halo_fwd_tc3<%d,%d>", e->d, e->win);
+    else if (const Tc3Entry* e = find_tc3(s))
+      std::snprintf(name, sizeof(name), "halo_fwd_tc3<%d,%d,%d>", e->d, e->win, e->block);
     else {
       const TcEntry* t = find_tc(s);
       std::snprintf(name, sizeof(name), "halo_fwd_tc<%d,%d,%d>", t->d, t->win, t->stride);

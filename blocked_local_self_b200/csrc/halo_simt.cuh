@@ -11,7 +11,7 @@
 // keys' k, rel_h, rel_w and v channels together (coalesced across the warp,
 // four keys' loads in flight), each key's logit is a warp sum, and an online
 // softmax (running max, rescaled sum and accumulator) skips keys outside the
-// image.
+// image (and, with the SASA mask on, keys outside the query's k x k square).
 #pragma once
 
 #include <cstdint>
@@ -23,6 +23,18 @@ namespace simt {
 constexpr int kThreads = 128;   // four warps, four (pixel, head) pairs
 constexpr int kKeysAtOnce = 4;
 
+// Whether window key (kr, kc) is kept for the query at in-block offset
+// (qy, qx) under the SASA mask (section 2.2: halo floor(k/2) and a mask that
+// keeps the k x k keys centred on the query): |kr - (qy + halo)| <= kmask/2
+// and the same for columns.  kmask 0 keeps every key (HaloNet's own form).
+// Image bounds are checked separately.
+__device__ __forceinline__ bool sasa_kept(int kr, int kc, int qy, int qx, int halo, int kmask) {
+  if (kmask <= 0) return true;
+  const int r = kmask >> 1;
+  const int dy = kr - qy - halo, dx = kc - qx - halo;
+  return dy <= r && dy >= -r && dx <= r && dx >= -r;
+}
+
 __device__ __forceinline__ float load_f(const float* p) { return __ldg(p); }
 __device__ __forceinline__ float load_f(const __nv_bfloat16* p) { return __bfloat162float(__ldg(p)); }
 __device__ __forceinline__ void store_f(float* p, float v) { *p = v; }
@@ -32,7 +44,7 @@ template <typename T, int DMAX>
 __global__ void __launch_bounds__(kThreads)
     halo_fwd_simt(const T* __restrict__ q, const T* __restrict__ k, const T* __restrict__ v,
                   const T* __restrict__ rel_h, const T* __restrict__ rel_w, T* __restrict__ out, int N, int H,
-                  int W, int heads, int d, int block, int halo, int stride, float scale) {
+                  int W, int heads, int d, int block, int halo, int stride, int kmask, float scale) {
   constexpr int NC = (DMAX + 31) / 32;  // channels per lane
   const int OH = H / stride, OW = W / stride;
   const long long total = static_cast<long long>(N) * OH * OW * heads;
@@ -71,7 +83,7 @@ __global__ void __launch_bounds__(kThreads)
     for (int g = 0; g < kKeysAtOnce; ++g) {
       const int key = kb + g, kr = key / w, kc = key - (key / w) * w;
       const int Y = y0 + kr, X = x0 + kc;
-      valid[g] = key < nkeys && Y >= 0 && Y < H && X >= 0 && X < W;
+      valid[g] = key < nkeys && Y >= 0 && Y < H && X >= 0 && X < W && sasa_kept(kr, kc, qy, qx, halo, kmask);
       const size_t off = valid[g] ? ((static_cast<size_t>(n) * H + Y) * W + X) * C + static_cast<size_t>(head) * d : 0;
       const T* rh = rel_h + static_cast<size_t>(valid[g] ? kr - qy + w - 1 : 0) * d;
       const T* rw = rel_w + static_cast<size_t>(valid[g] ? kc - qx + w - 1 : 0) * d;

@@ -1,5 +1,7 @@
 // halo_tc3.cuh -- stride-1 bf16 kernel for blocked local self-attention with
-// haloing on sm_100a, for 16x16 query blocks (windows of 16..24 pixels).
+// haloing on sm_100a, for 16x16 query blocks (windows of 16..24 pixels) and
+// 32x32 query blocks (windows of 32..38 pixels: global attention on a 32x32
+// map, section 2.2, and the block-32 detection setting, section 4.5).
 //
 // Operation (HaloNet, "Scaling Local Self-Attention for Parameter Efficient
 // Visual Backbones", sections 2.1-2.2 and appendix A; index conventions of the
@@ -10,20 +12,23 @@
 // A 16x16 block has 256 queries, so one head already fills two 128-row MMA
 // tiles; the window (up to 24 x 24 = 576 keys) is too wide for one TMEM pass.
 //
-// Work item = one 16x16 query block of one head.  Warpgroup g (g = 0, 1)
-// takes query rows [8g, 8g + 8) of the block (128 queries, TMEM lane = query):
+// Work item = 256 queries of one head: a whole 16x16 block, or a quarter
+// (8 query rows) of a 32x32 block.  Warpgroup g (g = 0, 1) takes half of the
+// item's query rows (128 queries, TMEM lane = query):
 //   * TMA (warp 8): Q [256 x d], K and V [w*w keys x d] of the item into one
 //     pipeline stage; the relative table R = [rel_h; 0; rel_w; 0] (96 rows)
 //     is written to shared memory once at start-up.
-//   * G MMA (warp 9 + g): G = Q_g R^T, M=128, N=96: the query's dot products
-//     with every rel_h and rel_w row, into the S buffer the item's first chunk
-//     will use.  Each thread picks the w + w it needs: the warp-uniform part of
-//     the row shift through the TMEM load address, the per-lane part by
-//     selects (no scratch memory).  The warpgroup gathers item k+1's before
-//     item k's epilogue, so the G MMA hides behind the last A.V.
-//   * S MMA (warp 9 + g): the window in chunks of 4 window rows, S_c = Q_g K_c^T
-//     (N = 4w rounded to 16), alternating between two TMEM buffers across
-//     chunks and items.
+//   * G MMA (warp 9 + g): G = Q_g R^T, M=128, N=96 (block 16) or 160
+//     (block 32): the query's dot products with every rel_h and rel_w row,
+//     into the S buffer the item's first chunk will use (block 16), or
+//     across both S buffers (block 32).  Each thread picks the w + w it
+//     needs: the warp-uniform part of the row shift through the TMEM load
+//     address, the per-lane part by selects (no scratch memory).  At block 16
+//     the warpgroup gathers item k+1's before item k's epilogue, so the G MMA
+//     hides behind the last A.V; at block 32 it follows the epilogue.
+//   * S MMA (warp 9 + g): the window in chunks of 4 (block 16) or 2 (block
+//     32) window rows, S_c = Q_g K_c^T (N = rows * w rounded to 16),
+//     alternating between two TMEM buffers across chunks and items.
 //   * softmax (one thread per query row): per chunk the exact chunk maximum of
 //     c*S + c*rel_w + c*rel_h; the running maximum moves only when the chunk's
 //     exceeds it by more than 8 (in log2 units), and only then is the fp32
@@ -63,7 +68,6 @@ using tc2::tmem_ld_x8;
 using tc2::tmem_st_x8;
 using tc2::tmem_wait_st;
 
-constexpr int kBlock = 16;
 constexpr int kThreads = 384;      // warpgroups 0-1 softmax, warp 8 TMA, warps 9-10 MMA
 constexpr int kTmaWarp = 8;
 constexpr int kMmaWarp = 9;        // warp 9 + g issues the G and S MMAs of warpgroup g
@@ -71,12 +75,8 @@ constexpr int kSoftmaxRegs = tc::kSoftmaxRegs;
 constexpr int kProducerRegs = tc::kProducerRegs;
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kSlotCols = 256;  // warpgroup g owns columns [256g, 256g + 256)
-constexpr uint32_t kBufCols = 96;    // S buffers at slot columns [0, 96) and [96, 192)
 constexpr uint32_t kOCol = 192;      // O accumulators (two A.V streams) at [192, 192 + 2d)
 constexpr int kStreams = 2;          // A.V issue streams (warps 0 and 1 of the warpgroup)
-constexpr int kChunkRows = 4;        // window rows per key chunk
-constexpr int kRRows = 96;           // R tile: rel_h rows [0, 2w-1), rel_w rows [48, 48 + 2w-1)
-constexpr int kRelW = 48;
 constexpr float kRescale = 8.0f;     // move the running maximum when exceeded by this (log2 units)
 constexpr uint64_t kWaitNs = tc::kWaitNs;
 
@@ -91,14 +91,28 @@ struct Params {
   float c;         // log2(e) / sqrt(d)
 };
 
-template <int D, int WIN>
+template <int D, int WIN, int BLOCK>
 struct Cfg {
+  static constexpr int kBlock = BLOCK;
+  static constexpr int QROWS = 256 / BLOCK;               // query rows of the block per item
+  static constexpr int NQUART = BLOCK / QROWS;            // items per block and head (1 or 4)
+  // S buffers at slot columns [0, kBufCols) and [kBufCols, 2 kBufCols)
+  static constexpr uint32_t kBufCols = (BLOCK == 16) ? 96 : 80;
+  static constexpr int kChunkRows = (BLOCK == 16) ? 4 : 2;   // window rows per key chunk
+  // R tile: rel_h rows [0, 2w-1), rel_w rows [kRelW, kRelW + 2w-1)
+  static constexpr int kRRows = (BLOCK == 16) ? 96 : 160;
+  static constexpr int kRelW = (BLOCK == 16) ? 48 : 80;
+  static constexpr bool kGBothBufs = (BLOCK == 32);      // G spans both S buffers
   static constexpr int ROWB = D * 2;
-  static constexpr int KS = WIN * WIN;
+  // Keys per window row in shared memory: the window width, or at block 32
+  // the width rounded up to 8 so that every 2-row chunk starts on a swizzle
+  // atom (the TMA box loads the extra columns; they are masked out).
+  static constexpr int WP = (BLOCK == 16) ? WIN : (WIN + 7) / 8 * 8;
+  static constexpr int KS = WP * WIN;                      // keys the TMA writes per tile
   static constexpr int NCH = (WIN + kChunkRows - 1) / kChunkRows;
   __host__ __device__ static constexpr int rows(int c) { return (c + 1 < NCH) ? kChunkRows : WIN - kChunkRows * (NCH - 1); }
-  __host__ __device__ static constexpr int start(int c) { return kChunkRows * WIN * c; }     // first key of chunk c
-  __host__ __device__ static constexpr int keys(int c) { return rows(c) * WIN; }
+  __host__ __device__ static constexpr int start(int c) { return kChunkRows * WP * c; }      // first key of chunk c
+  __host__ __device__ static constexpr int keys(int c) { return rows(c) * WP; }
   __host__ __device__ static constexpr int ns(int c) { return (keys(c) + 15) / 16 * 16; }    // S MMA N = P keys incl. padding
   __host__ __device__ static constexpr int nbuf(int b) { return (NCH + 1 - b) / 2; }         // chunks using buffer b per item
   static constexpr int KPAD = start(NCH - 1) + ns(NCH - 1);              // K / V rows incl. zero padding
@@ -110,36 +124,42 @@ struct Cfg {
   static constexpr SmemSwizzle SW = (ROWB == 32) ? SW_32B : (ROWB == 64 ? SW_64B : SW_128B);
   static constexpr uint32_t SBO = 8 * ROWB;
   static constexpr int HALO = (WIN - kBlock) / 2;
+  static_assert(BLOCK == 16 || BLOCK == 32, "block 16 or 32");
   static_assert(D == 16 || D == 32, "dim_head 16 or 32");
-  static_assert(WIN % 2 == 0 && WIN >= kBlock && WIN <= 24, "window 16..24");
+  static_assert(WIN % 2 == 0 && WIN >= kBlock && WIN <= kBlock + 8 && WIN <= 38, "window b..b+6 (b=32), b..b+8 (b=16)");
   static_assert(ns(0) <= (int)kBufCols, "S chunk in one buffer");
+  static_assert(2 * kBufCols <= kOCol, "S buffers below the O accumulators");
+  static_assert(!kGBothBufs || kRRows <= 2 * (int)kBufCols, "G inside the two S buffers");
+  static_assert(kGBothBufs || kRRows <= (int)kBufCols, "G inside one S buffer");
   static_assert(kOCol + kStreams * D <= kSlotCols, "O accumulators in the slot");
   static_assert(ns(NCH - 1) / 16 >= kStreams, "every A.V stream has a K-step in every chunk");
-  static_assert(2 * WIN - 1 <= kRelW, "relative table rows");
-  static_assert((kChunkRows * WIN) % 8 == 0, "chunk starts on a swizzle atom");
+  static_assert(2 * WIN - 1 <= kRelW && kRelW + 2 * WIN - 1 <= kRRows, "relative table rows");
+  static_assert((kChunkRows * WP) % 8 == 0, "chunk starts on a swizzle atom");
+  static_assert(WP % 2 == 0 && WP <= 40, "row pitch");
 };
 
-template <int D, int WIN>
+template <int D, int WIN, int BLOCK>
 __host__ __device__ constexpr int smem_bytes(int stages) {
-  using C = Cfg<D, WIN>;
+  using C = Cfg<D, WIN, BLOCK>;
   return 1024 + C::R_TILE + stages * C::STAGE_BYTES;
 }
 
 // Window-column pairs (kc, kc+1), kc even, whose exponentials take the
-// polynomial: inside the block's own 16 columns [h, h+16), which are never
+// polynomial: inside the block's own columns [h, h+b), which are never
 // outside the image.  Bit kc/2 of the mask.
 #ifndef HALO_TC3_POLY_PAIRS
 #define HALO_TC3_POLY_PAIRS 4
 #endif
-template <int WIN>
+template <int WIN, int BLOCK>
 __host__ __device__ constexpr unsigned poly_pair_mask() {
-  constexpr int h = (WIN - kBlock) / 2;
+  constexpr int h = (WIN - BLOCK) / 2;
+  const int npairs = HALO_TC3_POLY_PAIRS * BLOCK / 16;
   unsigned m = 0;
   int picked = 0;
-  const int mid = (h + 7) & ~1;
-  for (int d = 0; d < 16 && picked < HALO_TC3_POLY_PAIRS; ++d) {
+  const int mid = (h + BLOCK / 2 - 1) & ~1;
+  for (int d = 0; d < BLOCK && picked < npairs; ++d) {
     const int kc = mid + ((d & 1) ? -2 * ((d + 1) / 2) : 2 * (d / 2));
-    if (kc >= h && kc + 1 < h + kBlock && !((m >> (kc / 2)) & 1u)) {
+    if (kc >= h && kc + 1 < h + BLOCK && !((m >> (kc / 2)) & 1u)) {
       m |= 1u << (kc / 2);
       ++picked;
     }
@@ -152,23 +172,31 @@ __host__ __device__ constexpr unsigned poly_pair_mask() {
 __device__ __forceinline__ bool warp_ok(bool ok) { return __all_sync(0xffffffffu, ok); }
 
 struct ItemCoord {
-  int n, by, bx, head;
+  int n, by, bx, head, quart;  // quart: which QROWS query rows of the block
 };
+template <int NQUART>
 __device__ __forceinline__ ItemCoord item_coord(int item, int heads, int nbx, int nby) {
   ItemCoord c;
-  c.head = item % heads;
-  const int blk = item / heads;
+  c.quart = item % NQUART;
+  const int hb = item / NQUART;
+  c.head = hb % heads;
+  const int blk = hb / heads;
   c.bx = blk % nbx;
   c.by = (blk / nbx) % nby;
   c.n = blk / (nbx * nby);
   return c;
 }
 
-template <int D, int WIN>
+template <int D, int WIN, int BLOCK>
 __global__ void __launch_bounds__(kThreads, 1)
     halo_fwd_tc3(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__ CUtensorMap tmap_k,
                  const __grid_constant__ CUtensorMap tmap_v, const Params p) {
-  using C = Cfg<D, WIN>;
+  using C = Cfg<D, WIN, BLOCK>;
+  constexpr int kBlock = C::kBlock;
+  constexpr uint32_t kBufCols = C::kBufCols;
+  constexpr int kChunkRows = C::kChunkRows;
+  constexpr int kRRows = C::kRRows;
+  constexpr int kRelW = C::kRelW;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sR = smem;
@@ -267,11 +295,11 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (!abort_flag) record_timeout(&abort_flag);
           break;
         }
-        const ItemCoord ic = item_coord(blockIdx.x + k * gridDim.x, p.heads, p.nbx, p.nby);
+        const ItemCoord ic = item_coord<C::NQUART>(blockIdx.x + k * gridDim.x, p.heads, p.nbx, p.nby);
         uint8_t* st = sStage + s * C::STAGE_BYTES;
         const int x0 = ic.bx * kBlock, y0 = ic.by * kBlock;
         mbar_arrive_expect_tx(&bar_full[s], C::TX_BYTES);
-        tma_load_4d(st + OFF_Q, &tmap_q, &bar_full[s], ic.head * D, x0, y0, ic.n);
+        tma_load_4d(st + OFF_Q, &tmap_q, &bar_full[s], ic.head * D, x0, y0 + ic.quart * C::QROWS, ic.n);
         tma_load_4d(st + OFF_K, &tmap_k, &bar_full[s], ic.head * D, x0 - p.halo, y0 - p.halo, ic.n);
         tma_load_4d(st + OFF_V, &tmap_v, &bar_full[s], ic.head * D, x0 - p.halo, y0 - p.halo, ic.n);
         issued = k + 1;
@@ -294,14 +322,18 @@ __global__ void __launch_bounds__(kThreads, 1)
         ok = mbar_wait(&bar_full[s], (k / S) & 1, kWaitNs, &abort_flag);
         // G into the buffer of the item's first chunk, free once chunk t0 - 2's A.V is done
         if (ok && t0 >= 2) ok = mbar_wait(&bar_bfree[g][t0 & 1], ((t0 - 2) >> 1) & 1, kWaitNs, &abort_flag);
+        // block 32: G spans both buffers; the other one frees with chunk t0 - 1's A.V
+        if (C::kGBothBufs && ok && t0 >= 1)
+          ok = mbar_wait(&bar_bfree[g][(t0 - 1) & 1], ((t0 - 1) >> 1) & 1, kWaitNs, &abort_flag);
         if (!ok) break;
         tc_fence_after();
         const uint8_t* st = sStage + s * C::STAGE_BYTES;
         const uint32_t qa = smem_addr(st + OFF_Q + g * 128 * C::ROWB);
         const uint32_t ka = smem_addr(st + OFF_K);
+        const uint32_t gdst = slot + (C::kGBothBufs ? 0u : (t0 & 1) * kBufCols);
 #pragma unroll
         for (int ks = 0; ks < D / 16; ++ks)
-          mma_f16_ss(slot + (t0 & 1) * kBufCols, smem_desc(qa + 32 * ks, 16, C::SBO, C::SW),
+          mma_f16_ss(gdst, smem_desc(qa + 32 * ks, 16, C::SBO, C::SW),
                      smem_desc(ra + 32 * ks, 16, C::SBO, C::SW), idG, ks != 0);
         mma_commit(&bar_gfull[g]);
 #pragma unroll 1
@@ -335,50 +367,78 @@ __global__ void __launch_bounds__(kThreads, 1)
   asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kSoftmaxRegs));
   {
     // ------------------------------------------------------------ softmax warpgroups
-    const int g = warp >> 2;               // warpgroup = TMEM slot = query rows [8g, 8g + 8)
+    const int g = warp >> 2;               // warpgroup = TMEM slot = half of the item's query rows
     const int wq = warp & 3;               // lane quadrant
-    const int yl = 8 * g + 2 * wq + (lane >> 4);  // query row in the block
-    const int xl = lane & 15;                      // query column in the block
+    // query row among the item's QROWS rows, and column in the block: block
+    // 16 puts two query rows in a warp (16 lanes each), block 32 one
+    const int yq = (kBlock == 16) ? 8 * g + 2 * wq + (lane >> 4) : 4 * g + wq;
+    const int xl = (kBlock == 16) ? (lane & 15) : lane;
     const uint32_t slot = tmem + g * kSlotCols;    // lane 0 of the slot (MMA operands)
     const uint32_t ts = slot + (static_cast<uint32_t>(32 * wq) << 16);  // this warp's lanes
     const float c = p.c;
     const int C_all = p.heads * D;
     const uint32_t idO = idesc_bf16_f32(128, D, true);
-    constexpr unsigned kPoly = poly_pair_mask<WIN>();
+    constexpr unsigned kPoly = poly_pair_mask<WIN, kBlock>();
 
-    float rhc[WIN], rwc[WIN];
+    float rhc[WIN], rwc[C::WP];
     // ---- relative logits of item k: rhc[kr] = c * q.rel_h[kr - qy + w - 1], rwc[kc] likewise
     auto gather = [&](int k) -> bool {
       if (!warp_ok(mbar_wait(&bar_gfull[g], k & 1, kWaitNs, &abort_flag))) return false;
       tc_fence_after();
-      const ItemCoord ic = item_coord(blockIdx.x + k * gridDim.x, p.heads, p.nbx, p.nby);
+      const ItemCoord ic = item_coord<C::NQUART>(blockIdx.x + k * gridDim.x, p.heads, p.nbx, p.nby);
       const int y0 = ic.by * kBlock - p.halo, x0 = ic.bx * kBlock - p.halo;
-      const uint32_t gcol = ((k * C::NCH) & 1) * kBufCols;
-      // rel_h: columns [base, base + 32) of G hold every row this warp needs;
-      // the two query rows of the warp differ by one column
-      const int base = WIN - 2 - 8 * g - 2 * wq;
-      float gh[32], gw[48];
-      tmem_ld_x32(ts + gcol + base, gh);
-      tmem_ld_x32(ts + gcol + kRelW, gw);
-      tmem_ld_x8(ts + gcol + kRelW + 32, gw + 32);
-      tmem_ld_x8(ts + gcol + kRelW + 40, gw + 40);
-      tmem_wait_ld();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&bar_gfree[g]);
-      const bool odd = (lane >> 4) != 0;
+      const uint32_t gcol = C::kGBothBufs ? 0u : ((k * C::NCH) & 1) * kBufCols;
+      float a[WIN + kBlock - 1];
+      if constexpr (kBlock == 16) {
+        // rel_h: columns [base, base + 32) of G hold every row this warp needs;
+        // the two query rows of the warp differ by one column
+        const int base = WIN - 2 - 8 * g - 2 * wq;
+        float gh[32], gw[48];
+        tmem_ld_x32(ts + gcol + base, gh);
+        tmem_ld_x32(ts + gcol + kRelW, gw);
+        tmem_ld_x8(ts + gcol + kRelW + 32, gw + 32);
+        tmem_ld_x8(ts + gcol + kRelW + 40, gw + 40);
+        tmem_wait_ld();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bar_gfree[g]);
+        const bool odd = (lane >> 4) != 0;
 #pragma unroll
-      for (int kr = 0; kr < WIN; ++kr) {
-        const int Y = y0 + kr;
-        const float v = odd ? gh[kr] : gh[kr + 1];
-        rhc[kr] = (Y >= 0 && Y < p.H) ? v * c : -INFINITY;
+        for (int kr = 0; kr < WIN; ++kr) {
+          const int Y = y0 + kr;
+          const float v = odd ? gh[kr] : gh[kr + 1];
+          rhc[kr] = (Y >= 0 && Y < p.H) ? v * c : -INFINITY;
+        }
+#pragma unroll
+        for (int i = 0; i < WIN + 15; ++i) a[i] = gw[WIN - 16 + i];
+      } else {
+        // rel_h: one query row per warp, the whole shift in the load address
+        const int qy = ic.quart * C::QROWS + yq;
+        float gh[40], gw[72];
+        tmem_ld_x32(ts + gcol + (WIN - 1 - qy), gh);
+        tmem_ld_x8(ts + gcol + (WIN - 1 - qy) + 32, gh + 32);
+        tmem_ld_x32(ts + gcol + kRelW + WIN - 32, gw);
+        tmem_ld_x32(ts + gcol + kRelW + WIN, gw + 32);
+        tmem_ld_x8(ts + gcol + kRelW + WIN + 32, gw + 64);
+        tmem_wait_ld();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bar_gfree[g]);
+#pragma unroll
+        for (int kr = 0; kr < WIN; ++kr) {
+          const int Y = y0 + kr;
+          rhc[kr] = (Y >= 0 && Y < p.H) ? gh[kr] * c : -INFINITY;
+        }
+#pragma unroll
+        for (int i = 0; i < WIN + 31; ++i) a[i] = gw[i];
       }
-      // rel_w: the 16 query columns need 16 different shifts; a four-stage
-      // barrel shifter of selects over gw[w - 16 + i] by sh = 15 - qx
-      float a[WIN + 15];
+      // rel_w: the b query columns need b different shifts; a barrel shifter
+      // of selects over G[rel_w + w - b + i] by sh = b - 1 - qx
+      const int sh = kBlock - 1 - xl;
+      if constexpr (kBlock == 32) {
 #pragma unroll
-      for (int i = 0; i < WIN + 15; ++i) a[i] = gw[WIN - 16 + i];
-      const int sh = 15 - xl;
+        for (int i = 0; i < WIN + 15; ++i) a[i] = (sh & 16) ? a[i + 16] : a[i];
+      }
 #pragma unroll
       for (int i = 0; i < WIN + 7; ++i) a[i] = (sh & 8) ? a[i + 8] : a[i];
 #pragma unroll
@@ -388,9 +448,9 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
       for (int i = 0; i < WIN; ++i) a[i] = (sh & 1) ? a[i + 1] : a[i];
 #pragma unroll
-      for (int kc = 0; kc < WIN; ++kc) {
+      for (int kc = 0; kc < C::WP; ++kc) {
         const int X = x0 + kc;
-        rwc[kc] = (X >= 0 && X < p.W) ? a[kc] * c : -INFINITY;
+        rwc[kc] = (kc < WIN && X >= 0 && X < p.W) ? a[kc] * c : -INFINITY;  // row padding masked
       }
       return true;
     };
@@ -399,7 +459,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     float m_run = -INFINITY, l = 0.f;
     auto chunk = [&](auto nr, int k, int cidx) -> bool {
       constexpr int NR = decltype(nr)::value;
-      constexpr int NK = NR * WIN, NL = (NK + 7) / 8 * 8, NP = NK / 2, NW = (NK + 15) / 16 * 8;
+      constexpr int WP = C::WP;
+      constexpr int NK = NR * WP, NL = (NK + 7) / 8 * 8, NP = NK / 2, NW = (NK + 15) / 16 * 8;
       const int t = k * C::NCH + cidx, b = t & 1;
       const uint32_t buf = ts + b * kBufCols;
       if (!warp_ok(mbar_wait(&bar_sfull[g][b], (t >> 1) & 1, kWaitNs, &abort_flag))) return false;
@@ -411,7 +472,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       float2 y[NP];
 #pragma unroll
       for (int i = 0; i < NP; ++i) {
-        const int kc = (2 * i) % WIN;
+        const int kc = (2 * i) % WP;
         y[i] = __ffma2_rn(make_float2(z[2 * i], z[2 * i + 1]), make_float2(c, c), make_float2(rwc[kc], rwc[kc + 1]));
       }
       float mc = -INFINITY;
@@ -419,7 +480,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int r = 0; r < NR; ++r) {
         float mr = -INFINITY;
 #pragma unroll
-        for (int i = r * WIN / 2; i < (r + 1) * WIN / 2; ++i) mr = max3f(mr, y[i].x, y[i].y);
+        for (int i = r * WP / 2; i < (r + 1) * WP / 2; ++i) mr = max3f(mr, y[i].x, y[i].y);
         mc = fmaxf(mc, mr + rhc[r]);
       }
       const bool upd = mc > m_run + kRescale;
@@ -451,7 +512,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       uint32_t pk[NW];
 #pragma unroll
       for (int i = 0; i < NP; ++i) {
-        const int r = (2 * i) / WIN, kc = (2 * i) % WIN;
+        const int r = (2 * i) / WP, kc = (2 * i) % WP;
         const float bias = rhc[r] - mb;
         const float2 x = __fadd2_rn(y[i], make_float2(bias, bias));
         uint32_t rx, ry;
@@ -504,7 +565,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     constexpr int kLoopChunks = (kLastRows == kChunkRows) ? C::NCH : C::NCH - 1;
     bool ok = my_items > 0 ? gather(0) : true;
     for (int k = 0; k < my_items && ok; ++k) {
-      const ItemCoord ic = item_coord(blockIdx.x + k * gridDim.x, p.heads, p.nbx, p.nby);
+      const ItemCoord ic = item_coord<C::NQUART>(blockIdx.x + k * gridDim.x, p.heads, p.nbx, p.nby);
       m_run = -INFINITY;
       l = 0.f;
 #pragma unroll 1
@@ -513,7 +574,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (ok) ok = chunk(std::integral_constant<int, kLastRows>{}, k, C::NCH - 1);
       }
       // the next item's relative logits while this item's last A.V runs
-      if (ok && k + 1 < my_items) ok = gather(k + 1);
+      // (block 32: G needs both S buffers, so it follows the epilogue)
+      if (!C::kGBothBufs && ok && k + 1 < my_items) ok = gather(k + 1);
       // ---- epilogue: (O_0 + O_1) / l, bf16, NHWC
       if (ok) ok = warp_ok(mbar_wait(&bar_ofull[g], k & 1, kWaitNs, &abort_flag));
       if (!ok) break;
@@ -527,13 +589,14 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
         for (int t = 0; t < D / 2; ++t)
           pk[t] = pack_bf16x2((o[2 * t] + o[D + 2 * t]) * inv, (o[2 * t + 1] + o[D + 2 * t + 1]) * inv);
-        const int y = ic.by * kBlock + yl, x = ic.bx * kBlock + xl;
+        const int y = ic.by * kBlock + ic.quart * C::QROWS + yq, x = ic.bx * kBlock + xl;
         __nv_bfloat16* dst = p.out + ((static_cast<size_t>(ic.n) * p.H + y) * p.W + x) * C_all + ic.head * D;
 #pragma unroll
         for (int t = 0; t < D / 8; ++t)
           reinterpret_cast<uint4*>(dst)[t] = make_uint4(pk[4 * t], pk[4 * t + 1], pk[4 * t + 2], pk[4 * t + 3]);
       }
       tc_fence_before();
+      if (C::kGBothBufs && k + 1 < my_items) ok = gather(k + 1);
     }
     if (!ok && !abort_flag) record_timeout(&abort_flag);
     // A.V MMAs this warp issued are complete before TMEM is released

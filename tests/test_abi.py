@@ -50,7 +50,7 @@ def test_status_codes_match_header():
 
 def test_strerror_covers_codes():
     lib = _lib()
-    for code in range(0, -12, -1):
+    for code in range(0, -14, -1):
         text = lib.halo_strerror(code).decode()
         assert text and text != "unknown status code"
     assert lib.halo_strerror(-99).decode() == "unknown status code"
@@ -113,9 +113,9 @@ def test_kernel_names():
     assert name(64, 24, 32, 8, 64, 8, 3, 1, 1) == "halo_fwd_tc<64,14,1>"  # odd number of block rows
     assert name(2, 16, 24, 3, 16, 8, 3, 1, 1) == "halo_fwd_tc4<16,14>"   # odd head count, even block rows
     assert name(2, 24, 24, 3, 16, 8, 3, 1, 1) == "halo_fwd_tc<16,14,1>"   # odd head count, odd block rows
-    assert name(2, 32, 48, 3, 16, 16, 2, 1, 1) == "halo_fwd_tc3<16,20>"
+    assert name(2, 32, 48, 3, 16, 16, 2, 1, 1) == "halo_fwd_tc3<16,20,16>"
     assert name(64, 64, 64, 8, 32, 8, 3, 2, 1) == "halo_fwd_tc<32,14,2>"
-    assert name(16, 128, 128, 8, 32, 16, 4, 1, 1) == "halo_fwd_tc3<32,24>"
+    assert name(16, 128, 128, 8, 32, 16, 4, 1, 1) == "halo_fwd_tc3<32,24,16>"
     assert name(1, 16, 16, 2, 32, 4, 1, 1, 0) == "halo_fwd_simt<float,32>"
     assert name(2, 32, 32, 4, 40, 16, 4, 1, 1) == "halo_fwd_simt<bf16,64>"
     assert name(1, 16, 16, 2, 32, 5, 1, 1, 0) == "none"

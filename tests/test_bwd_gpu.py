@@ -1,0 +1,172 @@
+"""GPU parity of the backward (``halo_attn_bwd`` through the C ABI) against
+the CPU oracle's float64 gradients, on the same seeded inputs.
+
+Tolerance: each gradient's max-abs error must be at most
+tol * max(1, max |oracle gradient|), with tol = 1e-4 for float32 and 2e-2 for
+bf16 (the forward's bars).  The scale factor matters only for the table
+gradients, which sum over every query of the batch and reach tens to
+hundreds; rounding them to the dtype costs a relative, not an absolute, error.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from workloads import WORKLOADS, custom, make_inputs
+
+pytestmark = pytest.mark.gpu
+
+TOL = {"f32": 1e-4, "bf16": 2e-2}
+NAMES = ("dq", "dk", "dv", "drel_h", "drel_w")
+
+
+def _lib():
+    import blocked_local_self_b200 as h
+    h.load()
+    return h
+
+
+def _dout(wl, seed):
+    g = torch.Generator().manual_seed(seed)
+    OH, OW = wl.out_hw
+    return torch.randn((wl.N, OH, OW, wl.C), generator=g).to(wl.torch_dtype)
+
+
+def _forward(h, wl, dev, kernel):
+    if kernel:
+        return h.attn_masked(*dev, block=wl.block, halo=wl.halo, kernel=kernel, stride=wl.stride)
+    return h.attn(*dev, block=wl.block, halo=wl.halo, stride=wl.stride)
+
+
+def _compare(got, want, tol, what):
+    worst = 0.0
+    for g, w_, name in zip(got, want, NAMES):
+        g = g.detach().cpu().to(torch.float64).numpy()
+        assert np.all(np.isfinite(g)), f"{what} {name}: non-finite"
+        scale = max(1.0, float(np.abs(w_).max()))
+        err = float(np.abs(g - w_).max())
+        assert err <= tol * scale, f"{what} {name}: max abs err {err:.3e} > {tol} x {scale:.3g}"
+        worst = max(worst, err / scale)
+        print(f"[bwd parity] {what} {name}: max abs err {err:.3e} (scale {scale:.3g}, tol {tol})")
+    return worst
+
+
+def _run_case(case, seed=3):
+    kernel = case.pop("kernel", 0)
+    wl = custom("bwd", **case)
+    h = _lib()
+    inputs = make_inputs(wl, seed=seed)
+    dout = _dout(wl, seed + 100)
+    dev = [t.cuda() for t in inputs]
+    out = _forward(h, wl, dev, kernel)
+    grads = h.attn_bwd(*dev, out, dout.cuda(), block=wl.block, halo=wl.halo, stride=wl.stride, kernel=kernel)
+    torch.cuda.synchronize()
+    assert h.get_last_error() == 0
+    want = oracle.halo_attention_bwd(*inputs, dout, block=wl.block, halo=wl.halo, stride=wl.stride,
+                                     kernel=kernel)
+    return _compare(grads, want, TOL[wl.dtype], str(case) + f" kernel={kernel}")
+
+
+BWD_CASES = [
+    dict(N=2, H=16, W=24, heads=3, dim_head=16, block=8, halo=3, stride=1, dtype="bf16"),
+    dict(N=2, H=16, W=16, heads=2, dim_head=32, block=8, halo=2, stride=1, dtype="bf16"),
+    dict(N=1, H=16, W=24, heads=2, dim_head=64, block=8, halo=3, stride=1, dtype="bf16"),
+    dict(N=2, H=16, W=16, heads=4, dim_head=32, block=8, halo=3, stride=2, dtype="bf16"),
+    dict(N=1, H=32, W=32, heads=2, dim_head=32, block=16, halo=4, stride=1, dtype="bf16"),
+    dict(N=1, H=16, W=16, heads=2, dim_head=16, block=8, halo=0, stride=1, dtype="bf16"),
+    dict(N=1, H=16, W=16, heads=2, dim_head=32, block=4, halo=1, stride=1, dtype="f32"),
+    dict(N=2, H=12, W=8, heads=3, dim_head=8, block=4, halo=2, stride=2, dtype="f32"),
+    dict(N=1, H=8, W=8, heads=1, dim_head=128, block=8, halo=0, stride=1, dtype="f32"),
+    dict(N=1, H=16, W=16, heads=2, dim_head=16, block=16, halo=0, stride=1, dtype="f32"),   # global attention
+    # SASA-masked backward (k x k keys centred on each query)
+    dict(N=1, H=16, W=16, heads=2, dim_head=16, block=8, halo=3, stride=1, dtype="bf16", kernel=7),
+    dict(N=1, H=16, W=16, heads=2, dim_head=32, block=4, halo=2, stride=1, dtype="f32", kernel=3),
+]
+
+
+@pytest.mark.parametrize("case", BWD_CASES, ids=lambda c: "{dtype}_d{dim_head}_b{block}_h{halo}_s{stride}".format(**c)
+                         + ("_k%d" % c["kernel"] if "kernel" in c else ""))
+def test_bwd_small_full(case):
+    _run_case(dict(case))
+
+
+@pytest.mark.parametrize("name", ["stage1_bf16", "stride2_bf16"])
+def test_bwd_full_size(name):
+    """The full batch in one call (the benchmark's launch).  Images are
+    independent, so the gradients of q, k, v for the first and last image are
+    compared with the oracle run on those two images; the table gradients sum
+    over the whole batch, so they are checked by a property that holds at any
+    size (each table's gradient sums to zero over its rows, up to the float32
+    accumulation) and, for the two-image slice, against the oracle."""
+    wl = WORKLOADS[name]
+    h = _lib()
+    inputs = make_inputs(wl)
+    dout = _dout(wl, 7)
+    dev = [t.cuda() for t in inputs]
+    out = _forward(h, wl, dev, 0)
+    grads = h.attn_bwd(*dev, out, dout.cuda(), block=wl.block, halo=wl.halo, stride=wl.stride)
+    torch.cuda.synchronize()
+    assert h.get_last_error() == 0
+    sel = [0, wl.N - 1]
+    sub = [t[sel].contiguous() if t.dim() == 4 else t for t in inputs]
+    want = oracle.halo_attention_bwd(*sub, dout[sel].contiguous(), block=wl.block, halo=wl.halo, stride=wl.stride)
+    got = [g[sel] for g in grads[:3]]
+    tol = TOL[wl.dtype]
+    for g, w_, nm in zip(got, want[:3], NAMES[:3]):
+        g = g.cpu().to(torch.float64).numpy()
+        err = float(np.abs(g - w_).max())
+        scale = max(1.0, float(np.abs(w_).max()))
+        assert err <= tol * scale, f"{name} {nm}: {err:.3e}"
+        print(f"[bwd parity] {name} {nm} (images 0, N-1): max abs err {err:.3e}")
+    for t, nm in zip(grads[3:], NAMES[3:]):
+        s = t.float().sum(dim=0).abs().max().item()
+        mag = t.float().abs().max().item()
+        assert s <= 2e-2 * max(1.0, mag) * t.shape[0] ** 0.5, f"{name} {nm} rows sum to {s} (magnitude {mag})"
+    # the two-image slice through the library: all five gradients
+    sdev = [t.cuda() for t in sub]
+    sout = _forward(h, wl, sdev, 0)
+    sg = h.attn_bwd(*sdev, sout, dout[sel].contiguous().cuda(), block=wl.block, halo=wl.halo, stride=wl.stride)
+    torch.cuda.synchronize()
+    _compare(sg, want, tol, name + " two-image slice")
+
+
+def test_bwd_workspace_checks():
+    h = _lib()
+    from blocked_local_self_b200 import _native as n
+    wl = custom("ws", N=1, H=16, W=16, heads=2, dim_head=16, block=8, halo=3, dtype="bf16")
+    dev = [t.cuda() for t in make_inputs(wl)]
+    out = h.attn(*dev, block=8, halo=3)
+    dout = torch.randn_like(out)
+    need = h.bwd_workspace_size(1, 16, 16, 2, 16, 8, 3, 1, 0, torch.bfloat16)
+    assert need >= 2 * 16 * 16 * 32 * 4
+    small = torch.empty(need - 256, dtype=torch.uint8, device="cuda")
+    with pytest.raises(h.HaloError) as e:
+        h.attn_bwd(*dev, out, dout, block=8, halo=3, workspace=small)
+    assert e.value.code == n.HALO_ERR_WORKSPACE
+    with pytest.raises(h.HaloError) as e:
+        h.attn_bwd(*dev, out, dout, block=8, halo=3, kernel=9)
+    assert e.value.code == n.HALO_ERR_KERNEL
+    # a gradient that overlaps an input is refused
+    g = (dev[0], torch.empty_like(dev[1]), torch.empty_like(dev[2]), torch.empty_like(dev[3]),
+         torch.empty_like(dev[4]))
+    with pytest.raises(h.HaloError) as e:
+        h.attn_bwd(*dev, out, dout, block=8, halo=3, grads=g)
+    assert e.value.code == n.HALO_ERR_ALIAS
+
+
+def test_bwd_repeatable_and_workspace_reused():
+    """Two calls with one workspace give the same gradients (the workspace is
+    cleared by each call) up to the order of float32 atomic additions."""
+    h = _lib()
+    wl = custom("rep", N=2, H=16, W=16, heads=2, dim_head=16, block=8, halo=3, dtype="bf16")
+    dev = [t.cuda() for t in make_inputs(wl, seed=9)]
+    out = h.attn(*dev, block=8, halo=3)
+    dout = torch.randn_like(out)
+    ws = torch.empty(h.bwd_workspace_size(2, 16, 16, 2, 16, 8, 3, 1, 0, torch.bfloat16), dtype=torch.uint8,
+                     device="cuda")
+    a = h.attn_bwd(*dev, out, dout, block=8, halo=3, workspace=ws)
+    a = [t.clone() for t in a]
+    b = h.attn_bwd(*dev, out, dout, block=8, halo=3, workspace=ws)
+    torch.cuda.synchronize()
+    for x, y in zip(a, b):
+        assert torch.allclose(x.float(), y.float(), rtol=1e-2, atol=1e-2)

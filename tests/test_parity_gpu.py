@@ -138,6 +138,15 @@ CASES.append(dict(N=3, H=16, W=40, heads=2, dim_head=64, block=8, halo=3, stride
 for d in (16, 32):
     for halo in (0, 1, 2, 3, 4):
         CASES.append(dict(N=2, H=32, W=48, heads=3, dim_head=d, block=16, halo=halo, stride=1))
+# 32x32 query blocks (windows 32..38): global attention on a 32x32 map and
+# haloed 32x32 blocks, both head sizes, every window
+for d in (16, 32):
+    for halo in (0, 1, 2, 3):
+        CASES.append(dict(N=1, H=64, W=32 if halo else 64, heads=2, dim_head=d, block=32, halo=halo, stride=1))
+CASES += [
+    dict(N=3, H=32, W=32, heads=3, dim_head=32, block=32, halo=0, stride=1),  # global attention, several items per CTA
+    dict(N=1, H=32, W=96, heads=1, dim_head=16, block=32, halo=3, stride=1),  # one block row
+]
 CASES += [
     dict(N=1, H=16, W=16, heads=2, dim_head=32, block=16, halo=4, stride=1),  # block = map, halo all outside
     dict(N=3, H=16, W=80, heads=1, dim_head=16, block=16, halo=4, stride=1),  # one block row, one head
@@ -232,6 +241,8 @@ FAMILY_CASES = {
     "halo_fwd_tc<32,14,2>": dict(N=2, H=32, W=32, heads=4, dim_head=32, block=8, halo=3, stride=2),
     "halo_fwd_tc3<16,": dict(N=1, H=32, W=32, heads=2, dim_head=16, block=16, halo=3, stride=1),
     "halo_fwd_tc3<32,": dict(N=1, H=32, W=48, heads=2, dim_head=32, block=16, halo=4, stride=1),
+    "halo_fwd_tc3<16,38,32>": dict(N=1, H=64, W=32, heads=2, dim_head=16, block=32, halo=3, stride=1),
+    "halo_fwd_tc3<32,32,32>": dict(N=2, H=32, W=32, heads=2, dim_head=32, block=32, halo=0, stride=1),
 }
 
 

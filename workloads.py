@@ -126,6 +126,19 @@ WORKLOADS: dict[str, Workload] = {
 # The workload the throughput benchmark times (the stage-1 layer).
 BENCH_WORKLOAD = "stage1_bf16"
 
+# Shapes of the paper's further settings, measured beside the five above:
+# global attention at the smallest resolution (block = the whole 32x32 map,
+# halo 0; section 2.2 and the deep stages of section 4) and the block-32,
+# halo-3 setting of the detection backbones (section 4.5, Table 5).
+NEXT_WORKLOADS: dict[str, Workload] = {
+    w.name: w
+    for w in [
+        Workload("global32_bf16", N=64, H=32, W=32, heads=8, dim_head=32, block=32, halo=0, stride=1, dtype="bf16"),
+        Workload("block32_h3_bf16", N=4, H=128, W=128, heads=8, dim_head=32, block=32, halo=3, stride=1,
+                 dtype="bf16"),
+    ]
+}
+
 
 def make_inputs(wl: Workload, seed: int | None = None):
     """Draw (q, k, v, rel_h, rel_w) on the CPU for workload ``wl``.
