@@ -46,7 +46,8 @@ def parse_args():
     ap.add_argument("--steps", type=int, default=20000)
     ap.add_argument("--warmup", type=int, default=200)
     ap.add_argument("--impl", choices=["halo", "reference"], default="halo")
-    ap.add_argument("--workload", default=workloads.BENCH_WORKLOAD, choices=sorted(workloads.WORKLOADS))
+    ap.add_argument("--workload", default=workloads.BENCH_WORKLOAD,
+                    choices=sorted(workloads.WORKLOADS) + sorted(workloads.NEXT_WORKLOADS))
     ap.add_argument("--e2e-steps", type=int, default=10)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-graph", action="store_true",
@@ -55,6 +56,9 @@ def parse_args():
                     help="repeat the K-step timed region until about this much time is covered (median reported)")
     ap.add_argument("--no-per-config", action="store_true",
                     help="skip timing every workload for the per_config object")
+    ap.add_argument("--pass", dest="which", choices=["fwd", "bwd", "masked"], default="fwd",
+                    help="what one step runs: the forward (default), the backward (halo_attn_bwd, one launch per "
+                         "step from Python), or the SASA-masked forward with a 2*halo+1 window")
     ap.add_argument("--no-extra", action="store_true",
                     help="skip timing the backward and the SASA-masked forward (next_rows object)")
     return ap.parse_args()
@@ -270,7 +274,7 @@ def run_reference(args):
     if rank != 0:
         return 0
     import oracle
-    wl = workloads.WORKLOADS[args.workload]
+    wl = {**workloads.WORKLOADS, **workloads.NEXT_WORKLOADS}[args.workload]
     inputs = workloads.make_inputs(wl)
     # each step: one image of the workload (a bounded sample of the batch)
     n_img = 1
@@ -538,12 +542,16 @@ def time_extra(halo, stream, sampler, peaks, seconds=0.5):
         launch_s = ms * 1e-3
         gbs = bwd_bytes(wl) / launch_s * 1e-9
         tf = bwd_flops(wl) / launch_s * 1e-12
+        kname = halo.bwd_kernel_name(wl.N, wl.H, wl.W, wl.heads, wl.dim_head, wl.block, wl.halo, wl.stride, 0,
+                                     wl.torch_dtype)
         res["bwd_" + name] = {
-            "what": "halo_attn_bwd: dq, dk, dv, drel_h, drel_w (workspace zeroing, CUDA-core kernel, finalize)",
-            "kernel": "halo_bwd_simt", "ms": ms, "value": wl.out_pixels / launch_s, "unit": "pixels/s",
+            "what": "halo_attn_bwd: dq, dk, dv, drel_h, drel_w (workspace zeroing, the kernel, finalize)",
+            "kernel": kname, "ms": ms, "value": wl.out_pixels / launch_s, "unit": "pixels/s",
             "timing": f"{steps} back-to-back calls, inputs rotating over {len(sets)} sets > L2",
             "achieved_gbs": gbs, "hbm_frac": gbs / peaks["hbm_gbs"], "algorithmic_bytes": bwd_bytes(wl),
-            "tflops": tf, "flops": bwd_flops(wl), "fp32_alu_frac": tf / FP32_CUDA_CORE_TFLOPS,
+            "tflops": tf, "flops": bwd_flops(wl),
+            "compute_frac": tf / (peaks["bf16_tflops"] if "_tc<" in kname else FP32_CUDA_CORE_TFLOPS),
+            "compute_peak": "bf16 tensor (measured)" if "_tc<" in kname else "float32 CUDA cores (nominal)",
             "clocks": (t0, t1)}
         del sets, outs, douts, grads, ws
         torch.cuda.empty_cache()
@@ -595,11 +603,40 @@ def main():
     import blocked_local_self_b200 as halo
     halo.load()
 
-    wl = workloads.WORKLOADS[args.workload]
+    wl = {**workloads.WORKLOADS, **workloads.NEXT_WORKLOADS}[args.workload]
     inputs_cpu = workloads.make_inputs(wl, seed=rank_seed(wl, rank))
-    stream = torch.cuda.Stream() if not args.no_graph else torch.cuda.current_stream()
-    bench = DeviceBench(halo, wl, inputs_cpu, stream, use_graph=not args.no_graph)
+    use_graph = not args.no_graph and args.which != "bwd"
+    stream = torch.cuda.Stream() if use_graph else torch.cuda.current_stream()
+    bench = DeviceBench(halo, wl, inputs_cpu, stream, use_graph=use_graph)
     kernel = bench.kernel
+    if args.which == "masked":
+        kmask = 2 * wl.halo + 1
+
+        def masked_step(i, b=bench):
+            st = b.sets[i % b.n_sets]
+            halo.attn_masked(*st, block=wl.block, halo=wl.halo, kernel=kmask, stride=wl.stride,
+                             out=b.outs[i % b.n_sets], stream=stream)
+
+        bench.step = masked_step
+        kernel = halo.masked_kernel_name(wl.N, wl.H, wl.W, wl.heads, wl.dim_head, wl.block, wl.halo, wl.stride,
+                                         kmask, wl.torch_dtype)
+    elif args.which == "bwd":
+        with torch.cuda.stream(stream):
+            fwd_outs = [halo.attn(*st, block=wl.block, halo=wl.halo, stride=wl.stride) for st in bench.sets]
+        g = torch.Generator().manual_seed(7)
+        douts = [torch.randn(o.shape, generator=g).to(o.dtype).cuda() for o in fwd_outs]
+        grads = [tuple(torch.empty_like(t) for t in st) for st in bench.sets]
+        ws = torch.empty(halo.bwd_workspace_size(wl.N, wl.H, wl.W, wl.heads, wl.dim_head, wl.block, wl.halo,
+                                                 wl.stride, 0, wl.torch_dtype), dtype=torch.uint8, device="cuda")
+
+        def bwd_step(i, b=bench):
+            j = i % b.n_sets
+            halo.attn_bwd(*b.sets[j], fwd_outs[j], douts[j], block=wl.block, halo=wl.halo, stride=wl.stride,
+                          grads=grads[j], workspace=ws, stream=stream)
+
+        bench.step = bwd_step
+        kernel = halo.bwd_kernel_name(wl.N, wl.H, wl.W, wl.heads, wl.dim_head, wl.block, wl.halo, wl.stride, 0,
+                                      wl.torch_dtype)
     bench.warmup(args.warmup)
     # The timed steps replay CUDA graphs of the same launches (one kernel per
     # step, inputs rotating as above), so that the host's per-call cost
@@ -647,7 +684,7 @@ def main():
     h2d = sum(t.numel() * t.element_size() for t in inputs_cpu)
     d2h = wl.out_pixels * wl.C * wl.elem_bytes
     e2e = None
-    if args.e2e_steps > 0:
+    if args.e2e_steps > 0 and args.which == "fwd":
         pinned = [t.pin_memory() for t in inputs_cpu]
         out_h = torch.empty((wl.N, OH, OW, wl.C), dtype=wl.torch_dtype).pin_memory()
         staging = dict(zip(("q", "k", "v", "rel_h", "rel_w"), [torch.empty_like(t, device="cuda")
@@ -680,9 +717,11 @@ def main():
     per_step_s = ms * 1e-3 / args.steps
     pixels = wl.out_pixels * world
     value = pixels / per_step_s
-    tflops = wl.flops() * world / per_step_s * 1e-12
-    launch_s = ms_local * 1e-3 / args.steps  # one launch per step on this stream
-    achieved_gbs = wl.bytes() / launch_s * 1e-9
+    step_flops = bwd_flops(wl) if args.which == "bwd" else wl.flops()
+    step_bytes = bwd_bytes(wl) if args.which == "bwd" else wl.bytes()
+    tflops = step_flops * world / per_step_s * 1e-12
+    launch_s = ms_local * 1e-3 / args.steps  # one step per launch sequence on this stream
+    achieved_gbs = step_bytes / launch_s * 1e-9
     traffic = ncu_traffic(wl.name, kernel)
     line = {
         "metric": METRIC,
@@ -702,20 +741,22 @@ def main():
                                f"dim_head={wl.dim_head}, block={wl.block}, halo={wl.halo}, stride={wl.stride}",
                    "global_batch": wl.N * world, "parallelism": f"replicas x{world} (batch sharding)",
                    "l2": f"inputs rotate over {bench.n_sets} sets ({bench.n_sets * bench.in_bytes / 2**20:.0f} MiB) > L2",
-                   "launch": ("one launch per step from Python" if args.no_graph else
+                   "launch": ("one call per step from Python" if not use_graph else
                               "CUDA graphs of the per-step launches, replayed"),
                    "timing": f"median of {repeats} timed regions of exactly {args.steps} steps each, "
                              "each bracketed by a barrier and a device synchronisation",
+                   "pass": args.which,
                    "kernel": kernel},
         "tflops": tflops,
         "roofline": {"bound": "hbm", "achieved": achieved_gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
                      "frac": achieved_gbs / peaks["hbm_gbs"], "traffic": traffic,
                      "peak_source": f"{peaks['source']} (MEASURED_PEAKS.json hbm_gbs)" if peaks["source"] ==
                      "measured" else "fallback 6.65 TB/s",
-                     "algorithmic_bytes_per_launch": wl.bytes(),
+                     "algorithmic_bytes_per_launch": step_bytes,
                      "tensor_frac": tflops / world / peaks["bf16_tflops"]},
         "e2e": e2e,
-        "gpu_launches": args.steps * repeats,
+        # one kernel per forward step; the backward launches its kernel and the finalize kernel
+        "gpu_launches": args.steps * repeats * (2 if args.which == "bwd" else 1),
         "clocks": clocks,
         "cpu_baseline": base,
         "per_config": configs,

@@ -19,7 +19,7 @@ from . import _native
 from ._native import HaloError, HALO_BF16, HALO_F32
 
 __all__ = ["attn", "attn_masked", "attn_bwd", "bwd_workspace_size", "attn_host", "kernel_for", "kernel_name",
-           "masked_kernel_name", "get_last_error", "debug_wait_timeout", "version", "HaloError", "load"]
+           "masked_kernel_name", "bwd_kernel_name", "get_last_error", "debug_wait_timeout", "version", "HaloError", "load"]
 
 
 def load():
@@ -176,6 +176,14 @@ def masked_kernel_name(N: int, H: int, W: int, heads: int, dim_head: int, block:
     code = HALO_BF16 if dtype == torch.bfloat16 else HALO_F32
     return _native.lib().halo_masked_kernel_name(N, H, W, heads, dim_head, block, halo, stride, kernel,
                                                  code).decode()
+
+
+def bwd_kernel_name(N: int, H: int, W: int, heads: int, dim_head: int, block: int, halo: int, stride: int,
+                    kernel: int, dtype: torch.dtype) -> str:
+    """Kernel ``attn_bwd`` launches for a shape, or "none"."""
+    code = HALO_BF16 if dtype == torch.bfloat16 else HALO_F32
+    return _native.lib().halo_bwd_kernel_name(N, H, W, heads, dim_head, block, halo, stride, kernel,
+                                              code).decode()
 
 
 def get_last_error() -> int:

@@ -47,6 +47,7 @@ SIGNATURES = {
     "halo_kernel_for": (_i, [_i] * 9),
     "halo_kernel_name": (ctypes.c_char_p, [_i] * 9),
     "halo_masked_kernel_name": (ctypes.c_char_p, [_i] * 10),
+    "halo_bwd_kernel_name": (ctypes.c_char_p, [_i] * 10),
     "halo_strerror": (ctypes.c_char_p, [_i]),
     "halo_get_last_error": (_i, []),
     "halo_debug_wait_timeout": (_i, [_i, _vp]),

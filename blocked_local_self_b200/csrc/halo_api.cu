@@ -13,11 +13,13 @@
 
 #include "../../include/halo.h"
 #include "halo_bwd.cuh"
+#include "halo_bwd_tc.cuh"
 #include "halo_simt.cuh"
 #include "halo_tc.cuh"
 #include "halo_tc2.cuh"
 #include "halo_tc3.cuh"
 #include "halo_tc4.cuh"
+#include "halo_win.cuh"
 
 namespace {
 
@@ -83,20 +85,24 @@ struct TcEntry {
   int parts;
 };
 
-template <int D, int WIN, int STRIDE>
-int tc_smem(int stages) { return halo::tc::smem_bytes<D, WIN, STRIDE>(stages); }
+template <int D, int WIN, int STRIDE, int PP>
+int tc_smem(int stages) { return halo::tc::smem_bytes<D, WIN, STRIDE, PP>(stages); }
 
-#define HALO_TC_ENTRY(D, WIN, S)                                                                 \
+#define HALO_TC_ENTRY(D, WIN, S, PP)                                                             \
   TcEntry {                                                                                      \
-    D, WIN, S, halo::tc::halo_fwd_tc<D, WIN, S>, tc_smem<D, WIN, S>,                             \
-        halo::tc::Cfg<D, WIN, S>::STAGE_BYTES, halo::tc::Cfg<D, WIN, S>::PARTS                   \
+    D, WIN, S, halo::tc::halo_fwd_tc<D, WIN, S, PP>, tc_smem<D, WIN, S, PP>,                     \
+        halo::tc::Cfg<D, WIN, S, PP>::STAGE_BYTES, PP                                            \
   }
-#define HALO_TC_WINS(D, S) \
-  HALO_TC_ENTRY(D, 8, S), HALO_TC_ENTRY(D, 10, S), HALO_TC_ENTRY(D, 12, S), HALO_TC_ENTRY(D, 14, S)
+#define HALO_TC_WINS(D, S, PP)                                                                  \
+  HALO_TC_ENTRY(D, 8, S, PP), HALO_TC_ENTRY(D, 10, S, PP), HALO_TC_ENTRY(D, 12, S, PP),         \
+      HALO_TC_ENTRY(D, 14, S, PP)
 
+// Stride 2 packs several heads into the 64-row tile (16 queries each): four
+// where the head count allows (every softmax thread then has a query row),
+// else two at d = 32; the first matching entry is taken.
 const TcEntry kTcTable[] = {
-    HALO_TC_WINS(16, 1), HALO_TC_WINS(32, 1), HALO_TC_WINS(64, 1),
-    HALO_TC_WINS(16, 2), HALO_TC_WINS(32, 2), HALO_TC_WINS(64, 2),
+    HALO_TC_WINS(16, 1, 1), HALO_TC_WINS(32, 1, 1), HALO_TC_WINS(64, 1, 1), HALO_TC_WINS(16, 2, 4),
+    HALO_TC_WINS(32, 2, 4), HALO_TC_WINS(32, 2, 2), HALO_TC_WINS(64, 2, 1),
 };
 
 // Stride-1 kernel with two heads per 128-row tile (maps with an odd number of
@@ -295,35 +301,98 @@ cudaError_t launch_simt(const void* q, const void* k, const void* v, const void*
   return launch_simt_t<T, 128>(q, k, v, rh, rw, out, s, st);
 }
 
-int launch_tc(const TcEntry& e, const void* q, const void* k, const void* v, const void* rh, const void* rw,
-              void* out, const Shape& s, int sm_count, cudaStream_t st) {
-  const int win = s.block + 2 * s.halo;
-  CUtensorMap mq, mk, mv;
-  if (!encode_nhwc(&mq, q, s, halo::tc::kBlock, halo::tc::kBlock, s.stride) ||
-      !encode_nhwc(&mk, k, s, win, win, 1) || !encode_nhwc(&mv, v, s, halo::tc::kRowKeys, win, 1))
+// Window-staged CUDA-core kernel: dim_head 8, 16, 32, 64 or 128 and one
+// block's window (k, v and the tables as float32) within shared memory.
+bool win_plan(const Shape& s, halo::win::Params* p, int* threads, int* smem) {
+  if (s.d != 8 && s.d != 16 && s.d != 32 && s.d != 64 && s.d != 128) return false;
+  const int w = s.block + 2 * s.halo;
+  if (w > 64) return false;
+  const int tt = s.d >= 16 ? s.d / 16 : 1;
+  p->N = s.N;
+  p->H = s.H;
+  p->W = s.W;
+  p->heads = s.heads;
+  p->block = s.block;
+  p->halo = s.halo;
+  p->stride = s.stride;
+  p->kmask = s.kmask;
+  p->w = w;
+  p->nqx = s.block / s.stride;
+  p->nq = p->nqx * p->nqx;
+  p->nbx = s.W / s.block;
+  p->nby = s.H / s.block;
+  p->qpass = p->nq < halo::win::kMaxThreads / tt ? p->nq : halo::win::kMaxThreads / tt;
+  p->c = 1.4426950408889634f / std::sqrt(static_cast<float>(s.d));
+  *threads = (p->qpass * tt + 31) / 32 * 32;
+  *smem = halo::win::smem_floats(s.d, w, p->qpass) * 4;
+  return *smem <= kMaxDynSmem;
+}
+
+template <typename T, int D>
+int launch_win_t(const void* q, const void* k, const void* v, const void* rh, const void* rw, void* out,
+                 const Shape& s, const halo::win::Params& p, int threads, int smem, cudaStream_t st) {
+  auto fn = halo::win::halo_fwd_win<T, D>;
+  if (cudaFuncSetAttribute(reinterpret_cast<const void*>(fn), cudaFuncAttributeMaxDynamicSharedMemorySize, smem) !=
+      cudaSuccess)
     return HALO_ERR_CUDA;
-  // The kernel moves registers between its warpgroups with setmaxnreg; that is
-  // only safe if the launch allocation covers the split (otherwise the
-  // increase would wait forever).  Refuse to launch when it does not.
+  const long long items = static_cast<long long>(s.N) * p.nby * p.nbx * s.heads;
+  if (items > 0x7fffffffLL) return HALO_ERR_DIMS;
+  fn<<<static_cast<unsigned>(items), threads, smem, st>>>(
+      static_cast<const T*>(q), static_cast<const T*>(k), static_cast<const T*>(v), static_cast<const T*>(rh),
+      static_cast<const T*>(rw), static_cast<T*>(out), p);
+  return cudaGetLastError() == cudaSuccess ? HALO_OK : HALO_ERR_CUDA;
+}
+
+template <typename T>
+int launch_win(const void* q, const void* k, const void* v, const void* rh, const void* rw, void* out,
+               const Shape& s, const halo::win::Params& p, int threads, int smem, cudaStream_t st) {
+  switch (s.d) {
+    case 8: return launch_win_t<T, 8>(q, k, v, rh, rw, out, s, p, threads, smem, st);
+    case 16: return launch_win_t<T, 16>(q, k, v, rh, rw, out, s, p, threads, smem, st);
+    case 32: return launch_win_t<T, 32>(q, k, v, rh, rw, out, s, p, threads, smem, st);
+    case 64: return launch_win_t<T, 64>(q, k, v, rh, rw, out, s, p, threads, smem, st);
+    case 128: return launch_win_t<T, 128>(q, k, v, rh, rw, out, s, p, threads, smem, st);
+    default: return HALO_ERR_UNSUPPORTED;
+  }
+}
+
+// What every tensor-core kernel's launch shares: the register split check
+// (the kernels move registers between warpgroups with setmaxnreg, which is
+// only safe when the launch's allocation covers the split; otherwise the
+// increase would wait forever, so the launch is refused), the number of
+// pipeline stages that fit the opt-in shared memory next to the kernel's
+// static shared memory, and a persistent grid of one CTA per SM.
+template <class Params>
+int launch_persistent(void (*fn)(const CUtensorMap, const CUtensorMap, const CUtensorMap, const Params),
+                      int threads, int softmax_regs, int producer_regs, int (*smem_fn)(int), int max_stages,
+                      const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv, Params& p,
+                      long long items, int sm_count, cudaStream_t st) {
   cudaFuncAttributes attr;
-  if (cudaFuncGetAttributes(&attr, reinterpret_cast<const void*>(e.fn)) != cudaSuccess) return HALO_ERR_CUDA;
-  if (256 * halo::tc::kSoftmaxRegs + 128 * halo::tc::kProducerRegs > halo::tc::kThreads * attr.numRegs)
-    return HALO_ERR_UNSUPPORTED;
-  // dynamic shared memory budget: the per-block opt-in limit minus the
-  // kernel's static shared memory (mbarriers and flags)
+  if (cudaFuncGetAttributes(&attr, reinterpret_cast<const void*>(fn)) != cudaSuccess) return HALO_ERR_CUDA;
+  if (256 * softmax_regs + 128 * producer_regs > threads * attr.numRegs) return HALO_ERR_UNSUPPORTED;
   int optin = 0, dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess ||
       cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) != cudaSuccess)
     return HALO_ERR_CUDA;
   const int budget = (optin < kMaxDynSmem ? optin : kMaxDynSmem) - static_cast<int>(attr.sharedSizeBytes);
-  int stages = 8;
-  while (stages > 1 && e.smem(stages) > budget) --stages;
-  const int smem = e.smem(stages);
+  int stages = max_stages;
+  while (stages > 1 && smem_fn(stages) > budget) --stages;
+  const int smem = smem_fn(stages);
   if (smem > budget) return HALO_ERR_UNSUPPORTED;
-  if (cudaFuncSetAttribute(reinterpret_cast<const void*>(e.fn), cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           smem) != cudaSuccess)
+  if (cudaFuncSetAttribute(reinterpret_cast<const void*>(fn), cudaFuncAttributeMaxDynamicSharedMemorySize, smem) !=
+      cudaSuccess)
     return HALO_ERR_CUDA;
-  halo::tc::Params p;
+  if (items > 0x7fffffffLL) return HALO_ERR_DIMS;
+  p.num_items = static_cast<int>(items);
+  p.stages = stages;
+  const int grid = static_cast<int>(items < sm_count ? items : sm_count);
+  fn<<<grid, threads, smem, st>>>(mq, mk, mv, p);
+  return cudaGetLastError() == cudaSuccess ? HALO_OK : HALO_ERR_CUDA;
+}
+
+// Fields every tensor-core kernel's Params has.
+template <class Params>
+void fill_common(Params& p, const void* rh, const void* rw, void* out, const Shape& s) {
   p.rel_h = static_cast<const __nv_bfloat16*>(rh);
   p.rel_w = static_cast<const __nv_bfloat16*>(rw);
   p.out = static_cast<__nv_bfloat16*>(out);
@@ -332,19 +401,26 @@ int launch_tc(const TcEntry& e, const void* q, const void* k, const void* v, con
   p.W = s.W;
   p.heads = s.heads;
   p.halo = s.halo;
+  p.c = 1.4426950408889634f / std::sqrt(static_cast<float>(s.d));
+}
+
+int launch_tc(const TcEntry& e, const void* q, const void* k, const void* v, const void* rh, const void* rw,
+              void* out, const Shape& s, int sm_count, cudaStream_t st) {
+  const int win = s.block + 2 * s.halo;
+  CUtensorMap mq, mk, mv;
+  if (!encode_nhwc(&mq, q, s, halo::tc::kBlock, halo::tc::kBlock, s.stride) ||
+      !encode_nhwc(&mk, k, s, win, win, 1) || !encode_nhwc(&mv, v, s, halo::tc::kRowKeys, win, 1))
+    return HALO_ERR_CUDA;
+  halo::tc::Params p;
+  fill_common(p, rh, rw, out, s);
   p.nbx = s.W / halo::tc::kBlock;
   p.nby = s.H / halo::tc::kBlock;
   p.heads_per_item = e.parts;
-  const long long items = static_cast<long long>(s.N) * p.nbx * p.nby * (s.heads / e.parts);
-  if (items > 0x7fffffffLL) return HALO_ERR_DIMS;
-  p.num_items = static_cast<int>(items);
-  p.stages = stages;
   p.OH = s.H / s.stride;
   p.OW = s.W / s.stride;
-  p.c = 1.4426950408889634f / std::sqrt(static_cast<float>(s.d));
-  const int grid = static_cast<int>(items < sm_count ? items : sm_count);
-  e.fn<<<grid, halo::tc::kThreads, smem, st>>>(mq, mk, mv, p);
-  return cudaGetLastError() == cudaSuccess ? HALO_OK : HALO_ERR_CUDA;
+  const long long items = static_cast<long long>(s.N) * p.nbx * p.nby * (s.heads / e.parts);
+  return launch_persistent(e.fn, halo::tc::kThreads, halo::tc::kSoftmaxRegs, halo::tc::kProducerRegs, e.smem, 8,
+                           mq, mk, mv, p, items, sm_count, st);
 }
 
 int launch_tc2(const Tc2Entry& e, const void* q, const void* k, const void* v, const void* rh, const void* rw,
@@ -354,89 +430,35 @@ int launch_tc2(const Tc2Entry& e, const void* q, const void* k, const void* v, c
   if (!encode_nhwc(&mq, q, s, halo::tc2::kBlock, halo::tc2::kBlock, 1) || !encode_nhwc(&mk, k, s, win, win, 1) ||
       !encode_nhwc(&mv, v, s, win, win, 1))
     return HALO_ERR_CUDA;
-  cudaFuncAttributes attr;
-  if (cudaFuncGetAttributes(&attr, reinterpret_cast<const void*>(e.fn)) != cudaSuccess) return HALO_ERR_CUDA;
-  if (256 * halo::tc2::kSoftmaxRegs + 128 * halo::tc2::kProducerRegs > halo::tc2::kThreads * attr.numRegs)
-    return HALO_ERR_UNSUPPORTED;
-  int optin = 0, dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess ||
-      cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) != cudaSuccess)
-    return HALO_ERR_CUDA;
-  const int budget = (optin < kMaxDynSmem ? optin : kMaxDynSmem) - static_cast<int>(attr.sharedSizeBytes);
-  int stages = 8;
-  while (stages > 1 && e.smem(stages) > budget) --stages;
-  const int smem = e.smem(stages);
-  if (smem > budget) return HALO_ERR_UNSUPPORTED;
-  if (cudaFuncSetAttribute(reinterpret_cast<const void*>(e.fn), cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           smem) != cudaSuccess)
-    return HALO_ERR_CUDA;
   halo::tc2::Params p;
-  p.rel_h = static_cast<const __nv_bfloat16*>(rh);
-  p.rel_w = static_cast<const __nv_bfloat16*>(rw);
-  p.out = static_cast<__nv_bfloat16*>(out);
-  p.N = s.N;
-  p.H = s.H;
-  p.W = s.W;
-  p.heads = s.heads;
-  p.halo = s.halo;
+  fill_common(p, rh, rw, out, s);
   p.nbx = s.W / halo::tc2::kBlock;
   p.nby = s.H / halo::tc2::kBlock;
   const long long items = static_cast<long long>(s.N) * p.nbx * p.nby * (s.heads / 2);
-  if (items > 0x7fffffffLL) return HALO_ERR_DIMS;
-  p.num_items = static_cast<int>(items);
-  p.stages = stages;
-  p.c = 1.4426950408889634f / std::sqrt(static_cast<float>(s.d));
-  const int grid = static_cast<int>(items < sm_count ? items : sm_count);
-  e.fn<<<grid, halo::tc2::kThreads, smem, st>>>(mq, mk, mv, p);
-  return cudaGetLastError() == cudaSuccess ? HALO_OK : HALO_ERR_CUDA;
+  return launch_persistent(e.fn, halo::tc2::kThreads, halo::tc2::kSoftmaxRegs, halo::tc2::kProducerRegs, e.smem, 8,
+                           mq, mk, mv, p, items, sm_count, st);
 }
 
 int launch_tc3(const Tc3Entry& e, const void* q, const void* k, const void* v, const void* rh, const void* rw,
                void* out, const Shape& s, int sm_count, cudaStream_t st) {
   const int win = s.block + 2 * s.halo;
   CUtensorMap mq, mk, mv;
-  // Q box: the item's 256 queries (a whole 16x16 block, or 8 rows of a 32x32 block)
-  // K / V box: window rows padded to the kernel's row pitch (block 32: a multiple of 8)
+  // Q box: the item's 256 queries (a whole 16x16 block, or 8 rows of a 32x32
+  // block); K / V box: window rows padded to the kernel's row pitch (block
+  // 32: a multiple of 8)
   const int pitch = e.block == 16 ? win : (win + 7) / 8 * 8;
   if (!encode_nhwc(&mq, q, s, e.block, 256 / e.block, 1) || !encode_nhwc(&mk, k, s, pitch, win, 1) ||
       !encode_nhwc(&mv, v, s, pitch, win, 1))
     return HALO_ERR_CUDA;
-  cudaFuncAttributes attr;
-  if (cudaFuncGetAttributes(&attr, reinterpret_cast<const void*>(e.fn)) != cudaSuccess) return HALO_ERR_CUDA;
-  if (256 * halo::tc3::kSoftmaxRegs + 128 * halo::tc3::kProducerRegs > halo::tc3::kThreads * attr.numRegs)
-    return HALO_ERR_UNSUPPORTED;
-  int optin = 0, dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess ||
-      cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) != cudaSuccess)
-    return HALO_ERR_CUDA;
-  const int budget = (optin < kMaxDynSmem ? optin : kMaxDynSmem) - static_cast<int>(attr.sharedSizeBytes);
-  int stages = 4;  // the kernel has four stage barriers
-  while (stages > 1 && e.smem(stages) > budget) --stages;
-  const int smem = e.smem(stages);
-  if (smem > budget) return HALO_ERR_UNSUPPORTED;
-  if (cudaFuncSetAttribute(reinterpret_cast<const void*>(e.fn), cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           smem) != cudaSuccess)
-    return HALO_ERR_CUDA;
   halo::tc3::Params p;
-  p.rel_h = static_cast<const __nv_bfloat16*>(rh);
-  p.rel_w = static_cast<const __nv_bfloat16*>(rw);
-  p.out = static_cast<__nv_bfloat16*>(out);
-  p.N = s.N;
-  p.H = s.H;
-  p.W = s.W;
-  p.heads = s.heads;
-  p.halo = s.halo;
+  fill_common(p, rh, rw, out, s);
   p.nbx = s.W / e.block;
   p.nby = s.H / e.block;
   const int quarters = e.block * e.block / 256;
   const long long items = static_cast<long long>(s.N) * p.nbx * p.nby * s.heads * quarters;
-  if (items > 0x7fffffffLL) return HALO_ERR_DIMS;
-  p.num_items = static_cast<int>(items);
-  p.stages = stages;
-  p.c = 1.4426950408889634f / std::sqrt(static_cast<float>(s.d));
-  const int grid = static_cast<int>(items < sm_count ? items : sm_count);
-  e.fn<<<grid, halo::tc3::kThreads, smem, st>>>(mq, mk, mv, p);
-  return cudaGetLastError() == cudaSuccess ? HALO_OK : HALO_ERR_CUDA;
+  // the kernel has four stage barriers
+  return launch_persistent(e.fn, halo::tc3::kThreads, halo::tc3::kSoftmaxRegs, halo::tc3::kProducerRegs, e.smem, 4,
+                           mq, mk, mv, p, items, sm_count, st);
 }
 
 int launch_tc4(const Tc4Entry& e, const void* q, const void* k, const void* v, const void* rh, const void* rw,
@@ -447,43 +469,15 @@ int launch_tc4(const Tc4Entry& e, const void* q, const void* k, const void* v, c
       !encode_nhwc(&mk, k, s, win, win + halo::tc4::kBlock, 1) ||
       !encode_nhwc(&mv, v, s, win, win + halo::tc4::kBlock, 1))
     return HALO_ERR_CUDA;
-  const Tc4Kernel fn = s.kmask > 0 ? e.fn_masked : e.fn;
-  cudaFuncAttributes attr;
-  if (cudaFuncGetAttributes(&attr, reinterpret_cast<const void*>(fn)) != cudaSuccess) return HALO_ERR_CUDA;
-  if (256 * halo::tc4::kSoftmaxRegs + 128 * halo::tc4::kProducerRegs > halo::tc4::kThreads * attr.numRegs)
-    return HALO_ERR_UNSUPPORTED;
-  int optin = 0, dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess ||
-      cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) != cudaSuccess)
-    return HALO_ERR_CUDA;
-  const int budget = (optin < kMaxDynSmem ? optin : kMaxDynSmem) - static_cast<int>(attr.sharedSizeBytes);
-  int stages = 4;  // the kernel has four stage barriers
-  while (stages > 1 && e.smem(stages) > budget) --stages;
-  const int smem = e.smem(stages);
-  if (smem > budget) return HALO_ERR_UNSUPPORTED;
-  if (cudaFuncSetAttribute(reinterpret_cast<const void*>(fn), cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           smem) != cudaSuccess)
-    return HALO_ERR_CUDA;
   halo::tc4::Params p;
-  p.rel_h = static_cast<const __nv_bfloat16*>(rh);
-  p.rel_w = static_cast<const __nv_bfloat16*>(rw);
-  p.out = static_cast<__nv_bfloat16*>(out);
-  p.N = s.N;
-  p.H = s.H;
-  p.W = s.W;
-  p.heads = s.heads;
-  p.halo = s.halo;
+  fill_common(p, rh, rw, out, s);
   p.nbx = s.W / halo::tc4::kBlock;
   p.npy = s.H / (2 * halo::tc4::kBlock);
-  const long long items = static_cast<long long>(s.N) * p.nbx * p.npy * s.heads;
-  if (items > 0x7fffffffLL) return HALO_ERR_DIMS;
-  p.num_items = static_cast<int>(items);
-  p.stages = stages;
-  p.c = 1.4426950408889634f / std::sqrt(static_cast<float>(s.d));
   p.kmask = s.kmask;
-  const int grid = static_cast<int>(items < sm_count ? items : sm_count);
-  fn<<<grid, halo::tc4::kThreads, smem, st>>>(mq, mk, mv, p);
-  return cudaGetLastError() == cudaSuccess ? HALO_OK : HALO_ERR_CUDA;
+  const long long items = static_cast<long long>(s.N) * p.nbx * p.npy * s.heads;
+  // the kernel has four stage barriers
+  return launch_persistent(s.kmask > 0 ? e.fn_masked : e.fn, halo::tc4::kThreads, halo::tc4::kSoftmaxRegs,
+                           halo::tc4::kProducerRegs, e.smem, 4, mq, mk, mv, p, items, sm_count, st);
 }
 
 int attn_device(const void* q, const void* k, const void* v, const void* rel_h, const void* rel_w, void* out,
@@ -504,6 +498,11 @@ int attn_device(const void* q, const void* k, const void* v, const void* rel_h, 
     if (const Tc3Entry* e3 = find_tc3(s)) return launch_tc3(*e3, q, k, v, rel_h, rel_w, out, s, sm_count, st);
     return launch_tc(*find_tc(s), q, k, v, rel_h, rel_w, out, s, sm_count, st);
   }
+  halo::win::Params wp;
+  int wthreads = 0, wsmem = 0;
+  if (win_plan(s, &wp, &wthreads, &wsmem))
+    return (s.dtype == HALO_F32) ? launch_win<float>(q, k, v, rel_h, rel_w, out, s, wp, wthreads, wsmem, st)
+                                 : launch_win<__nv_bfloat16>(q, k, v, rel_h, rel_w, out, s, wp, wthreads, wsmem, st);
   cudaError_t err = (s.dtype == HALO_F32) ? launch_simt<float>(q, k, v, rel_h, rel_w, out, s, st)
                                           : launch_simt<__nv_bfloat16>(q, k, v, rel_h, rel_w, out, s, st);
   return err == cudaSuccess ? HALO_OK : HALO_ERR_CUDA;
@@ -618,6 +617,93 @@ int launch_bwd(const BwdPlan& plan, int d, const void* const* in, void* const* g
   }
 }
 
+// Tensor-core backward: bf16, block 8, stride 1, dim_head 16 or 32, window
+// 8..14: (d, window) -> instantiation.
+using BwdTcKernel = void (*)(const CUtensorMap, const CUtensorMap, const CUtensorMap, const CUtensorMap,
+                             const halo::bwdtc::Params);
+struct BwdTcEntry {
+  int d, win;
+  BwdTcKernel fn;
+  int (*smem)(int);
+};
+template <int D, int WIN>
+int bwdtc_smem(int stages) { return halo::bwdtc::smem_bytes<D, WIN>(stages); }
+#define HALO_BWDTC_ENTRY(D, WIN) \
+  BwdTcEntry { D, WIN, halo::bwdtc::halo_bwd_tc<D, WIN>, bwdtc_smem<D, WIN> }
+const BwdTcEntry kBwdTcTable[] = {
+    HALO_BWDTC_ENTRY(16, 8), HALO_BWDTC_ENTRY(16, 10), HALO_BWDTC_ENTRY(16, 12), HALO_BWDTC_ENTRY(16, 14),
+    HALO_BWDTC_ENTRY(32, 8), HALO_BWDTC_ENTRY(32, 10), HALO_BWDTC_ENTRY(32, 12), HALO_BWDTC_ENTRY(32, 14),
+};
+
+const BwdTcEntry* find_bwdtc(const Shape& s) {
+  if (s.dtype != HALO_BF16 || s.block != halo::bwdtc::kBlock || s.stride != 1) return nullptr;
+  const int win = s.block + 2 * s.halo;
+  for (const BwdTcEntry& e : kBwdTcTable)
+    if (e.d == s.d && e.win == win) return &e;
+  return nullptr;
+}
+
+int launch_bwdtc(const BwdTcEntry& e, const BwdPlan& plan, const void* const* in, void* const* grads, void* ws,
+                 const Shape& s, int sm_count, cudaStream_t st) {
+  const int win = s.block + 2 * s.halo;
+  CUtensorMap mq, mk, mv, mdo;
+  if (!encode_nhwc(&mq, in[0], s, halo::bwdtc::kBlock, halo::bwdtc::kBlock, 1) ||
+      !encode_nhwc(&mk, in[1], s, win, win, 1) || !encode_nhwc(&mv, in[2], s, win, win, 1) ||
+      !encode_nhwc(&mdo, in[6], s, halo::bwdtc::kBlock, halo::bwdtc::kBlock, 1))
+    return HALO_ERR_CUDA;
+  cudaFuncAttributes attr;
+  if (cudaFuncGetAttributes(&attr, reinterpret_cast<const void*>(e.fn)) != cudaSuccess) return HALO_ERR_CUDA;
+  int optin = 0, dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) != cudaSuccess)
+    return HALO_ERR_CUDA;
+  const int budget = (optin < kMaxDynSmem ? optin : kMaxDynSmem) - static_cast<int>(attr.sharedSizeBytes);
+  int stages = 4;  // the kernel has four stage barriers
+  while (stages > 1 && e.smem(stages) > budget) --stages;
+  const int smem = e.smem(stages);
+  if (smem > budget) return HALO_ERR_UNSUPPORTED;
+  if (cudaFuncSetAttribute(reinterpret_cast<const void*>(e.fn), cudaFuncAttributeMaxDynamicSharedMemorySize, smem) !=
+      cudaSuccess)
+    return HALO_ERR_CUDA;
+  halo::bwdtc::Params p;
+  p.rel_h = static_cast<const __nv_bfloat16*>(in[3]);
+  p.rel_w = static_cast<const __nv_bfloat16*>(in[4]);
+  p.out = static_cast<const __nv_bfloat16*>(in[5]);
+  p.dout = static_cast<const __nv_bfloat16*>(in[6]);
+  p.dq = static_cast<__nv_bfloat16*>(grads[0]);
+  char* w = static_cast<char*>(ws);
+  p.dk32 = reinterpret_cast<float*>(w + plan.off_dk);
+  p.dv32 = reinterpret_cast<float*>(w + plan.off_dv);
+  p.drh32 = reinterpret_cast<float*>(w + plan.off_drh);
+  p.drw32 = reinterpret_cast<float*>(w + plan.off_drw);
+  p.N = s.N;
+  p.H = s.H;
+  p.W = s.W;
+  p.heads = s.heads;
+  p.halo = s.halo;
+  p.nbx = s.W / halo::bwdtc::kBlock;
+  p.nby = s.H / halo::bwdtc::kBlock;
+  const long long items = static_cast<long long>(s.N) * p.nbx * p.nby * s.heads;
+  if (items > 0x7fffffffLL) return HALO_ERR_DIMS;
+  p.num_items = static_cast<int>(items);
+  p.stages = stages;
+  p.kmask = s.kmask;
+  p.c = plan.p.c;
+  p.s = plan.p.s;
+  const int grid = static_cast<int>(items < sm_count ? items : sm_count);
+  e.fn<<<grid, halo::bwdtc::kThreads, smem, st>>>(mq, mk, mv, mdo, p);
+  if (cudaGetLastError() != cudaSuccess) return HALO_ERR_CUDA;
+  const long long nin = static_cast<long long>(s.N) * s.H * s.W * s.heads * s.d;
+  const int ntab = plan.p.R * s.d;
+  const long long nmax = nin > ntab ? nin : ntab;
+  long long fb = (nmax + 255) / 256;
+  if (fb > 8LL * sm_count) fb = 8LL * sm_count;
+  halo::bwd::halo_bwd_finalize<__nv_bfloat16><<<static_cast<int>(fb), 256, 0, st>>>(
+      p.dk32, p.dv32, p.drh32, p.drw32, static_cast<__nv_bfloat16*>(grads[1]), static_cast<__nv_bfloat16*>(grads[2]),
+      static_cast<__nv_bfloat16*>(grads[3]), static_cast<__nv_bfloat16*>(grads[4]), nin, ntab);
+  return cudaGetLastError() == cudaSuccess ? HALO_OK : HALO_ERR_CUDA;
+}
+
 // Shared by the workspace-taking backward entry point (and any variant that
 // brings its own scratch): checks, zeroing, the two launches.
 int attn_bwd(const void* const* in, void* const* grads, void* ws, size_t ws_bytes, const Shape& s,
@@ -651,6 +737,7 @@ int attn_bwd(const void* const* in, void* const* grads, void* ws, size_t ws_byte
   if (cudaMemsetAsync(ws, 0, plan.ws_bytes, st) != cudaSuccess) return HALO_ERR_CUDA;
   // at stride 2 only the strided pixels are queries: dq is zero elsewhere
   if (s.stride == 2 && cudaMemsetAsync(grads[0], 0, ib, st) != cudaSuccess) return HALO_ERR_CUDA;
+  if (const BwdTcEntry* e = find_bwdtc(s)) return launch_bwdtc(*e, plan, in, grads, ws, s, sm_count, st);
   return s.dtype == HALO_F32 ? launch_bwd<float>(plan, s.d, in, grads, ws, sm_count, st)
                              : launch_bwd<__nv_bfloat16>(plan, s.d, in, grads, ws, sm_count, st);
 }
@@ -683,11 +770,17 @@ const char* kernel_name_of(const Shape& s) {
       std::snprintf(name, sizeof(name), "halo_fwd_tc3<%d,%d,%d>", e->d, e->win, e->block);
     else {
       const TcEntry* t = find_tc(s);
-      std::snprintf(name, sizeof(name), "halo_fwd_tc<%d,%d,%d>", t->d, t->win, t->stride);
+      std::snprintf(name, sizeof(name), "halo_fwd_tc<%d,%d,%d,%d>", t->d, t->win, t->stride, t->parts);
     }
   } else {
-    const int dmax = s.d <= 16 ? 16 : s.d <= 32 ? 32 : s.d <= 64 ? 64 : 128;
-    std::snprintf(name, sizeof(name), "halo_fwd_simt<%s,%d>", s.dtype == HALO_F32 ? "float" : "bf16", dmax);
+    halo::win::Params wp;
+    int wthreads = 0, wsmem = 0;
+    if (win_plan(s, &wp, &wthreads, &wsmem)) {
+      std::snprintf(name, sizeof(name), "halo_fwd_win<%s,%d>", s.dtype == HALO_F32 ? "float" : "bf16", s.d);
+    } else {
+      const int dmax = s.d <= 16 ? 16 : s.d <= 32 ? 32 : s.d <= 64 ? 64 : 128;
+      std::snprintf(name, sizeof(name), "halo_fwd_simt<%s,%d>", s.dtype == HALO_F32 ? "float" : "bf16", dmax);
+    }
   }
   return name;
 }
@@ -837,6 +930,22 @@ const char* halo_kernel_name(int N, int H, int W, int heads, int dim_head, int b
                              int dtype) {
   const Shape s{N, H, W, heads, dim_head, block, halo, stride, dtype};
   return kernel_name_of(s);
+}
+
+const char* halo_bwd_kernel_name(int N, int H, int W, int heads, int dim_head, int block, int halo, int stride,
+                                 int kernel, int dtype) {
+  thread_local char name[64];
+  Shape s{N, H, W, heads, dim_head, block, halo, stride, dtype};
+  s.kmask = kernel;
+  BwdPlan plan;
+  if (bwd_plan(s, &plan) != HALO_OK) {
+    std::snprintf(name, sizeof(name), "none");
+  } else if (const BwdTcEntry* e = find_bwdtc(s)) {
+    std::snprintf(name, sizeof(name), "halo_bwd_tc<%d,%d>", e->d, e->win);
+  } else {
+    std::snprintf(name, sizeof(name), "halo_bwd_simt<%s,%d>", s.dtype == HALO_F32 ? "float" : "bf16", s.d);
+  }
+  return name;
 }
 
 const char* halo_masked_kernel_name(int N, int H, int W, int heads, int dim_head, int block, int halo, int stride,

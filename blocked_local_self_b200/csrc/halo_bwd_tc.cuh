@@ -1,0 +1,575 @@
+// halo_bwd_tc.cuh -- tensor-core backward of blocked local self-attention with
+// haloing on sm_100a: bf16, 8x8 query blocks, stride 1, dim_head 16 or 32,
+// windows 8..14 (HaloNet, "Scaling Local Self-Attention for Parameter
+// Efficient Visual Backbones", sections 2.1-2.2 and appendix A; the blog
+// page's RelPosEmb / HaloAttention index conventions).
+//
+// Gradients of a loss L given dout = dL/dout.  Per query i and window key j,
+// with p the softmax weights over the kept keys and s = d^-1/2:
+//   dS_ij = p_ij (dout_i . v_j - dout_i . out_i)
+//   dq = s (dS K + T R),  dk = s dS^T Q,  dv = P^T dout,  d[rel_h; rel_w] += s T^T Q
+// where T (per query, one row of 64) holds the query's sums of dS over each
+// window row at that row's rel_h table index and over each window column at
+// that column's rel_w index, and R = [rel_h; 0; rel_w; 0] (64 rows).  All six
+// products are tcgen05 MMAs.
+//
+// Work item = one 8x8 block of one head.  Two warpgroups take alternate items,
+// each with a 256-column TMEM slot and its own P / dS / T buffers in shared
+// memory; the elected thread of a warpgroup issues its MMAs:
+//   R1  S = Q K^T (M=64, N=w^2 rounded to 8) at slot column 0 and
+//       G = Q R^T (N=56) at column 200: the relative logits, gathered per
+//       query as in the forward two-block kernel (out-of-image rows and
+//       columns, and with the SASA mask of section 2.2 the rows and columns
+//       outside the query's k x k square, get -inf).
+//   softmax pass A: exact row maximum of c (S + rel); pass B: p' =
+//       2^(c (S + rel) - m) as bf16 into the P buffer and the row sum l.
+//   R2  dP = dout V^T (N as S) over the S columns, once every thread is done
+//       with S.
+//   pass C: p = p' / l, dS = p (dP - D) with D = dout . out (the forward's
+//       output); bf16 p and dS into the P and dS buffers, the row and column
+//       sums of dS into the query's T row.
+//   R3  dV_t = P^T[keys of tile t] dout, dK_t = dS^T[tile t] Q (M=128, keys
+//       in 128-row tiles), dQ = dS K + T R (M=64), dR = T^T Q (M=64).  One
+//       shared-memory layout serves as the K-major A operand of dQ (rows =
+//       queries, K = keys) and as the MN-major A operand of dK and dV
+//       (M = keys, K = queries): rows of 64 keys (128 B, 128-byte swizzle),
+//       atoms of 64 rows 8 KB apart.
+//   epilogue: dk (x s) and dv of every in-image window key added to float32
+//       accumulators in global memory (up to four windows hold a key); dq
+//       (x s) stored as bf16; dR (x s) added to the warpgroup's table
+//       accumulator in shared memory, flushed to global memory at exit.
+// A TMA warp streams Q, dout, K and V (two stages when they fit).  Every wait
+// is bounded and reports HALO_ERR_TIMEOUT.
+#pragma once
+
+#include <cstdint>
+#include <cuda.h>
+#include <cuda_bf16.h>
+
+#include "halo_tc.cuh"
+#include "halo_tc2.cuh"
+#include "halo_tc4.cuh"
+#include "sm100.cuh"
+
+namespace halo {
+namespace bwdtc {
+
+using namespace sm100;
+using tc::exp2_mufu;
+using tc::pack_bf16x2;
+using tc::record_timeout;
+using tc::swz;
+using tc2::tmem_ld_x8;
+using tc4::tmem_ld_exact;
+
+constexpr int kBlock = 8;
+constexpr int kThreads = 288;        // warpgroups 0-1 (softmax, MMA issue), warp 8 TMA
+constexpr int kTmaWarp = 8;
+constexpr uint32_t kTmemCols = 512;
+constexpr uint32_t kSlotCols = 256;  // warpgroup g owns columns [256g, 256g + 256)
+constexpr uint32_t kGBase = 200;     // G at slot columns [200, 256): rel_h logits, then rel_w at +28
+constexpr int kRelW = 28;
+constexpr int kRRows = 64;           // R tile rows: [rel_h; 0; rel_w; 0] padded to one 64-row K extent
+constexpr uint64_t kWaitNs = tc::kWaitNs;
+
+struct Params {
+  const __nv_bfloat16* rel_h;
+  const __nv_bfloat16* rel_w;
+  const __nv_bfloat16* out;
+  const __nv_bfloat16* dout;
+  __nv_bfloat16* dq;
+  float *dk32, *dv32, *drh32, *drw32;  // float32 accumulators (zeroed by the host)
+  int N, H, W, heads, halo;
+  int nbx, nby;
+  int num_items;   // N * nby * nbx * heads
+  int stages;
+  int kmask;       // SASA mask size (0: none): keys within kmask/2 of the query
+  float c;         // log2(e) / sqrt(d)
+  float s;         // 1 / sqrt(d)
+};
+
+template <int D, int WIN>
+struct Cfg {
+  static constexpr int ROWB = D * 2;
+  static constexpr int KS = WIN * WIN;                 // window keys
+  static constexpr int NS = (KS + 7) / 8 * 8;          // S / dP MMA N
+  static constexpr int KP = (KS + 15) / 16 * 16;       // keys incl. padding: dQ K extent
+  static constexpr int KSTEPS = KP / 16;
+  static constexpr int MT = (KS + 127) / 128;          // 128-key tiles of dK / dV
+  static constexpr int Q_TILE = 64 * ROWB;
+  static constexpr int K_TILE = (KP * ROWB + 1023) / 1024 * 1024;
+  static constexpr int OFF_Q = 0, OFF_DO = Q_TILE, OFF_K = 2 * Q_TILE, OFF_V = 2 * Q_TILE + K_TILE;
+  static constexpr int STAGE_BYTES = 2 * Q_TILE + 2 * K_TILE;
+  static constexpr int TX = (2 * 64 + 2 * KS) * ROWB;
+  static constexpr int R_TILE = (kRRows * ROWB + 1023) / 1024 * 1024;
+  static constexpr int PBUF = MT * 2 * 8192;           // 64 queries x MT*128 keys, bf16, 8 KB atoms of 64 keys
+  static constexpr int TBUF = 8192;                    // 64 queries x 64 table entries
+  static constexpr int WG_BYTES = 2 * PBUF + TBUF;     // P, dS, T of one warpgroup
+  static constexpr int DREL_BYTES = 2 * 64 * D * 4;    // two warpgroups' table accumulators (float32)
+  // TMEM columns of R3's accumulators: dV tiles, dK tiles, dQ, dR
+  static constexpr uint32_t COL_DV = 0, COL_DK = MT * D, COL_DQ = 2 * MT * D, COL_DR = 2 * MT * D + D;
+  static constexpr SmemSwizzle SW = (ROWB == 32) ? SW_32B : SW_64B;
+  static constexpr uint32_t SBO = 8 * ROWB;
+  static constexpr int HALO = (WIN - kBlock) / 2;
+  static_assert(D == 16 || D == 32, "dim_head 16 or 32");
+  static_assert(WIN % 2 == 0 && WIN >= 8 && WIN <= 14, "window 8..14");
+  static_assert(NS <= (int)kGBase, "S columns below the relative logits");
+  static_assert(COL_DR + D <= kGBase, "R3 accumulators below G");
+  static_assert(2 * WIN - 1 <= kRelW && kRelW + 2 * WIN - 1 <= 56, "relative table rows");
+};
+
+template <int D, int WIN>
+__host__ __device__ constexpr int smem_bytes(int stages) {
+  using C = Cfg<D, WIN>;
+  return 1024 + C::R_TILE + 2 * C::WG_BYTES + C::DREL_BYTES + stages * C::STAGE_BYTES;
+}
+
+// tcgen05 instruction descriptor, kind::f16, bf16 A and B, f32 D, with the
+// A major bit (15) as well as the B major bit (16).
+__host__ __device__ constexpr uint32_t idesc_ab(int M, int N, bool a_mn, bool b_mn) {
+  return idesc_bf16_f32(M, N, b_mn) | ((a_mn ? 1u : 0u) << 15);
+}
+
+// Byte offset of the 16-byte chunk holding keys [8u, 8u + 8) of query row r
+// in a P / dS buffer: atoms of 64 keys (8 KB), 128-byte rows, 128-byte swizzle.
+__device__ __forceinline__ uint32_t pofs(int r, int u) { return (u >> 3) * 8192 + swz<128>(r, u & 7); }
+
+// A wait's outcome, the same for every lane of the warp (warp-collective
+// tcgen05 instructions follow).
+__device__ __forceinline__ bool warp_ok(bool ok) { return __all_sync(0xffffffffu, ok); }
+
+// D consecutive TMEM columns of this thread's lane (32x32b shape).
+template <int D>
+__device__ __forceinline__ void tmem_ld_d(uint32_t taddr, float* r) {
+  if constexpr (D == 32) tc2::tmem_ld_x32(taddr, r);
+  else tmem_ld_exact<D>(taddr, r);
+}
+
+// Barrier of one warpgroup's four warps on an mbarrier of count 4, so that
+// the wait is bounded (a named barrier would hang if a warp gave up early).
+// `ph` counts this warpgroup's uses of the barrier.
+__device__ __forceinline__ bool wg_sync(uint64_t* bar, int& ph, int lane, int* abort_flag) {
+  __syncwarp();
+  if (lane == 0) mbar_arrive(bar);
+  const bool ok = warp_ok(mbar_wait(bar, ph & 1, kWaitNs, abort_flag));
+  ++ph;
+  return ok;
+}
+
+template <int D, int WIN>
+__global__ void __launch_bounds__(kThreads, 1)
+    halo_bwd_tc(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__ CUtensorMap tmap_k,
+                const __grid_constant__ CUtensorMap tmap_v, const __grid_constant__ CUtensorMap tmap_do,
+                const Params p) {
+  using C = Cfg<D, WIN>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* sR = smem;
+  uint8_t* sWG = sR + C::R_TILE;                          // [g][P | dS | T]
+  float* sDrel = reinterpret_cast<float*>(sWG + 2 * C::WG_BYTES);  // [g][64][D]
+  uint8_t* sStage = sWG + 2 * C::WG_BYTES + C::DREL_BYTES;
+
+  __shared__ __align__(8) uint64_t bar_full[4];
+  __shared__ __align__(8) uint64_t bar_empty[4];
+  __shared__ __align__(8) uint64_t bar_r1[2];
+  __shared__ __align__(8) uint64_t bar_r2[2];
+  __shared__ __align__(8) uint64_t bar_r3[2];
+  __shared__ __align__(8) uint64_t bar_wg[2];    // count 4: the warps of warpgroup g
+  __shared__ __align__(8) uint64_t bar_drain[2];
+  __shared__ uint32_t tmem_base_sh;
+  __shared__ int abort_flag;
+
+  const int tid = threadIdx.x;
+  const int warp = tid >> 5;
+  const int lane = tid & 31;
+  const int S = p.stages;
+
+  // ---------------------------------------------------------------- set-up
+  if (tid == 0) {
+    for (int i = 0; i < S; ++i) {
+      mbar_init(&bar_full[i], 1);
+      mbar_init(&bar_empty[i], 1);
+    }
+    for (int g = 0; g < 2; ++g) {
+      mbar_init(&bar_r1[g], 1);
+      mbar_init(&bar_r2[g], 1);
+      mbar_init(&bar_r3[g], 1);
+      mbar_init(&bar_wg[g], 4);
+      mbar_init(&bar_drain[g], 1);
+    }
+    abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == kTmaWarp && lane == 0) {
+    prefetch_tensormap(&tmap_q);
+    prefetch_tensormap(&tmap_k);
+    prefetch_tensormap(&tmap_v);
+    prefetch_tensormap(&tmap_do);
+  }
+  // R tile, zeroed P / dS / T buffers and table accumulators, and the K / V
+  // rows the TMA never writes
+  for (int idx = tid; idx < kRRows * (D / 8); idx += kThreads) {
+    const int r = idx / (D / 8), u = idx % (D / 8);
+    uint4 val = make_uint4(0, 0, 0, 0);
+    if (r < 2 * WIN - 1) val = *reinterpret_cast<const uint4*>(p.rel_h + r * D + u * 8);
+    else if (r >= kRelW && r < kRelW + 2 * WIN - 1)
+      val = *reinterpret_cast<const uint4*>(p.rel_w + (r - kRelW) * D + u * 8);
+    *reinterpret_cast<uint4*>(sR + swz<C::ROWB>(r, u)) = val;
+  }
+  for (int idx = tid; idx < (2 * C::WG_BYTES + C::DREL_BYTES) / 16; idx += kThreads)
+    reinterpret_cast<uint4*>(sWG)[idx] = make_uint4(0, 0, 0, 0);
+  for (int s = 0; s < S; ++s) {
+    uint8_t* st = sStage + s * C::STAGE_BYTES;
+    for (int idx = tid; idx < (C::KP - C::KS) * C::ROWB / 16; idx += kThreads) {
+      reinterpret_cast<uint4*>(st + C::OFF_K + C::KS * C::ROWB)[idx] = make_uint4(0, 0, 0, 0);
+      reinterpret_cast<uint4*>(st + C::OFF_V + C::KS * C::ROWB)[idx] = make_uint4(0, 0, 0, 0);
+    }
+  }
+  fence_proxy_async_smem();
+  if (warp == 0) {
+    tmem_alloc(&tmem_base_sh, kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = tmem_base_sh;
+  const int my_items = (p.num_items > (int)blockIdx.x)
+                           ? (p.num_items - 1 - (int)blockIdx.x) / (int)gridDim.x + 1 : 0;
+  const int C_all = p.heads * D;
+
+  if (warp == kTmaWarp) {
+    // ------------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      int issued = 0;
+      for (int k = 0; k < my_items; ++k) {
+        const int s = k % S;
+        if (k >= S && !mbar_wait(&bar_empty[s], ((k / S) - 1) & 1, kWaitNs, &abort_flag)) {
+          if (!abort_flag) record_timeout(&abort_flag);
+          break;
+        }
+        const int item = blockIdx.x + k * gridDim.x;
+        const int head = item % p.heads, blk = item / p.heads;
+        const int bx = blk % p.nbx, by = (blk / p.nbx) % p.nby, n = blk / (p.nbx * p.nby);
+        uint8_t* st = sStage + s * C::STAGE_BYTES;
+        const int x0 = bx * kBlock, y0 = by * kBlock;
+        mbar_arrive_expect_tx(&bar_full[s], C::TX);
+        tma_load_4d(st + C::OFF_Q, &tmap_q, &bar_full[s], head * D, x0, y0, n);
+        tma_load_4d(st + C::OFF_DO, &tmap_do, &bar_full[s], head * D, x0, y0, n);
+        tma_load_4d(st + C::OFF_K, &tmap_k, &bar_full[s], head * D, x0 - p.halo, y0 - p.halo, n);
+        tma_load_4d(st + C::OFF_V, &tmap_v, &bar_full[s], head * D, x0 - p.halo, y0 - p.halo, n);
+        issued = k + 1;
+      }
+      if (abort_flag) {
+        for (int k = (issued > S ? issued - S : 0); k < issued; ++k) mbar_wait(&bar_full[k % S], (k / S) & 1, kWaitNs);
+      }
+    }
+    __syncwarp();
+  } else {
+    // ------------------------------------------------------------ softmax warpgroups
+    const int g = warp >> 2;                 // warpgroup = TMEM slot
+    const int wq = warp & 3;                 // lane quadrant
+    const bool act = lane < 16;              // M=64 tiles: rows in lanes 0-15 of each quadrant
+    const int row = 16 * wq + (lane & 15);   // query row in the 8x8 block
+    const int qy = row >> 3, qx = row & 7;
+    const uint32_t slot = tmem + g * kSlotCols;
+    const uint32_t ts = slot + (static_cast<uint32_t>(32 * wq) << 16);
+    uint8_t* sP = sWG + g * C::WG_BYTES;
+    uint8_t* sDS = sP + C::PBUF;
+    uint8_t* sT = sDS + C::PBUF;
+    float* drel = sDrel + g * 64 * D;
+    const bool elected = (wq == 0 && lane == 0);
+    const float c = p.c;
+    const uint32_t idS = idesc_ab(64, C::NS, false, false);
+    const uint32_t idG = idesc_ab(64, 56, false, false);
+    const uint32_t idKV = idesc_ab(128, D, true, true);   // dV, dK: A = P^T / dS^T (MN-major), B MN-major
+    const uint32_t idQ = idesc_ab(64, D, false, true);    // dQ: A = dS / T (K-major), B MN-major
+    const uint32_t idR = idesc_ab(64, D, true, true);     // dR: A = T^T (MN-major), B = Q (MN-major)
+    const uint32_t pa = smem_addr(sP), dsa = smem_addr(sDS), tA = smem_addr(sT), ra = smem_addr(sR);
+    int ph = 0;  // uses of bar_wg[g]
+
+    bool ok = true;
+    int j = 0;
+    for (int k = g; k < my_items && ok; k += 2, ++j) {
+      const int s = k % S;
+      const uint8_t* st = sStage + s * C::STAGE_BYTES;
+      const uint32_t qa = smem_addr(st + C::OFF_Q), doa = smem_addr(st + C::OFF_DO);
+      const uint32_t ka = smem_addr(st + C::OFF_K), va = smem_addr(st + C::OFF_V);
+      // ---- R1: S and G
+      if (elected) {
+        if (mbar_wait(&bar_full[s], (k / S) & 1, kWaitNs, &abort_flag)) {
+          tc_fence_after();
+#pragma unroll
+          for (int ks = 0; ks < D / 16; ++ks) {
+            mma_f16_ss(slot, smem_desc(qa + 32 * ks, 16, C::SBO, C::SW), smem_desc(ka + 32 * ks, 16, C::SBO, C::SW),
+                       idS, ks != 0);
+            mma_f16_ss(slot + kGBase, smem_desc(qa + 32 * ks, 16, C::SBO, C::SW),
+                       smem_desc(ra + 32 * ks, 16, C::SBO, C::SW), idG, ks != 0);
+          }
+          mma_commit(&bar_r1[g]);
+        } else if (!abort_flag) {
+          record_timeout(&abort_flag);
+        }
+      }
+      ok = warp_ok(mbar_wait(&bar_r1[g], j & 1, kWaitNs, &abort_flag));
+      if (!ok) break;
+      tc_fence_after();
+
+      const int item = blockIdx.x + k * gridDim.x;
+      const int head = item % p.heads, blk = item / p.heads;
+      const int bx = blk % p.nbx, by = (blk / p.nbx) % p.nby, n = blk / (p.nbx * p.nby);
+      const int y0 = by * kBlock - p.halo, x0 = bx * kBlock - p.halo;
+      // ---- relative logits of this query (log2 units), -inf for masked rows / columns
+      float rh[WIN], rw[WIN];
+      {
+        float gh[WIN + 1];
+        tmem_ld_exact<WIN + 1>(ts + kGBase + (WIN - 2 - 2 * wq), gh);
+        float a[WIN + 7];
+        tmem_ld_exact<WIN + 7>(ts + kGBase + kRelW + WIN - 8, a);
+        tmem_wait_ld();
+        const bool odd = ((lane >> 3) & 1) != 0;
+#pragma unroll
+        for (int kr = 0; kr < WIN; ++kr) {
+          const int Y = y0 + kr;
+          const bool keep = Y >= 0 && Y < p.H &&
+                            (p.kmask == 0 || (kr - qy - p.halo <= (p.kmask >> 1) && qy + p.halo - kr <= (p.kmask >> 1)));
+          rh[kr] = keep ? (odd ? gh[kr] : gh[kr + 1]) * c : -INFINITY;
+        }
+        const int sh = 7 - qx;
+#pragma unroll
+        for (int i = 0; i < WIN + 3; ++i) a[i] = (sh & 4) ? a[i + 4] : a[i];
+#pragma unroll
+        for (int i = 0; i < WIN + 1; ++i) a[i] = (sh & 2) ? a[i + 2] : a[i];
+#pragma unroll
+        for (int i = 0; i < WIN; ++i) a[i] = (sh & 1) ? a[i + 1] : a[i];
+#pragma unroll
+        for (int kc = 0; kc < WIN; ++kc) {
+          const int X = x0 + kc;
+          const bool keep = X >= 0 && X < p.W &&
+                            (p.kmask == 0 || (kc - qx - p.halo <= (p.kmask >> 1) && qx + p.halo - kc <= (p.kmask >> 1)));
+          rw[kc] = keep ? a[kc] * c : -INFINITY;
+        }
+      }
+      // ---- D = dout . out of this query
+      const int y = by * kBlock + qy, x = bx * kBlock + qx;
+      const size_t pix = ((static_cast<size_t>(n) * p.H + y) * p.W + x) * C_all + static_cast<size_t>(head) * D;
+      float Dq = 0.f;
+      if (act) {
+#pragma unroll
+        for (int e = 0; e < D; e += 8) {
+          const uint4 o = *reinterpret_cast<const uint4*>(p.out + pix + e);
+          const uint4 d = *reinterpret_cast<const uint4*>(p.dout + pix + e);
+          const __nv_bfloat162* o2 = reinterpret_cast<const __nv_bfloat162*>(&o);
+          const __nv_bfloat162* d2 = reinterpret_cast<const __nv_bfloat162*>(&d);
+#pragma unroll
+          for (int t = 0; t < 4; ++t) {
+            const float2 of = __bfloat1622float2(o2[t]), df = __bfloat1622float2(d2[t]);
+            Dq = fmaf(of.x, df.x, fmaf(of.y, df.y, Dq));
+          }
+        }
+      }
+      // ---- pass A: exact row maximum, per window row max of c S + c rel_w,
+      // then over rows with c rel_h added
+      float m = -INFINITY;
+      {
+        float rmax[WIN];
+#pragma unroll
+        for (int r = 0; r < WIN; ++r) rmax[r] = -INFINITY;
+#pragma unroll
+        for (int j0 = 0; j0 < C::NS; j0 += 8) {
+          float z[8];
+          tmem_ld_x8(ts + j0, z);
+          tmem_wait_ld();
+#pragma unroll
+          for (int t = 0; t < 8; ++t)
+            if (j0 + t < C::KS) rmax[(j0 + t) / WIN] = fmaxf(rmax[(j0 + t) / WIN], fmaf(z[t], c, rw[(j0 + t) % WIN]));
+        }
+#pragma unroll
+        for (int r = 0; r < WIN; ++r) m = fmaxf(m, rmax[r] + rh[r]);
+      }
+      // ---- pass B: p' = 2^(c S + c rel_w + (c rel_h - m)) into the P buffer, row sum
+      float brow[WIN];
+#pragma unroll
+      for (int r = 0; r < WIN; ++r) brow[r] = rh[r] - m;
+      float l = 0.f;
+#pragma unroll
+      for (int j0 = 0; j0 < C::NS; j0 += 8) {
+        float z[8];
+        tmem_ld_x8(ts + j0, z);
+        tmem_wait_ld();
+        uint32_t pk[4];
+#pragma unroll
+        for (int t = 0; t < 8; t += 2) {
+          float e0 = 0.f, e1 = 0.f;
+          if (j0 + t < C::KS) e0 = exp2_mufu(fmaf(z[t], c, rw[(j0 + t) % WIN]) + brow[(j0 + t) / WIN]);
+          if (j0 + t + 1 < C::KS)
+            e1 = exp2_mufu(fmaf(z[t + 1], c, rw[(j0 + t + 1) % WIN]) + brow[(j0 + t + 1) / WIN]);
+          l += e0 + e1;
+          pk[t / 2] = pack_bf16x2(e0, e1);
+        }
+        if (act) *reinterpret_cast<uint4*>(sP + pofs(row, j0 / 8)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+      }
+      const float inv_l = 1.0f / l;
+      // ---- R2: dP = dout V^T over the S columns
+      tc_fence_before();
+      ok = wg_sync(&bar_wg[g], ph, lane, &abort_flag);
+      if (!ok) break;
+      if (elected) {
+        tc_fence_after();
+#pragma unroll
+        for (int ks = 0; ks < D / 16; ++ks)
+          mma_f16_ss(slot, smem_desc(doa + 32 * ks, 16, C::SBO, C::SW), smem_desc(va + 32 * ks, 16, C::SBO, C::SW),
+                     idS, ks != 0);
+        mma_commit(&bar_r2[g]);
+      }
+      ok = warp_ok(mbar_wait(&bar_r2[g], j & 1, kWaitNs, &abort_flag));
+      if (!ok) break;
+      tc_fence_after();
+      // ---- pass C: p = p' / l, dS = p (dP - D); bf16 P and dS; row / column sums of dS
+      float rs[WIN], cs[WIN];
+#pragma unroll
+      for (int i = 0; i < WIN; ++i) rs[i] = cs[i] = 0.f;
+#pragma unroll
+      for (int j0 = 0; j0 < C::NS; j0 += 8) {
+        float dp[8];
+        tmem_ld_x8(ts + j0, dp);
+        const uint4 pv = *reinterpret_cast<const uint4*>(sP + pofs(row, j0 / 8));
+        tmem_wait_ld();
+        const __nv_bfloat162* p2 = reinterpret_cast<const __nv_bfloat162*>(&pv);
+        uint32_t pk[4], dk[4];
+#pragma unroll
+        for (int t = 0; t < 8; t += 2) {
+          const float2 pp = __bfloat1622float2(p2[t / 2]);
+          const float p0 = pp.x * inv_l, p1 = pp.y * inv_l;
+          float d0 = 0.f, d1 = 0.f;
+          if (j0 + t < C::KS) {
+            d0 = p0 * (dp[t] - Dq);
+            rs[(j0 + t) / WIN] += d0;
+            cs[(j0 + t) % WIN] += d0;
+          }
+          if (j0 + t + 1 < C::KS) {
+            d1 = p1 * (dp[t + 1] - Dq);
+            rs[(j0 + t + 1) / WIN] += d1;
+            cs[(j0 + t + 1) % WIN] += d1;
+          }
+          pk[t / 2] = pack_bf16x2(p0, p1);
+          dk[t / 2] = pack_bf16x2(d0, d1);
+        }
+        if (act) {
+          *reinterpret_cast<uint4*>(sP + pofs(row, j0 / 8)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+          *reinterpret_cast<uint4*>(sDS + pofs(row, j0 / 8)) = make_uint4(dk[0], dk[1], dk[2], dk[3]);
+        }
+      }
+      // T row: rel_h entries kr - qy + w - 1, rel_w entries 28 + kc - qx + w - 1
+      if (act) {
+#pragma unroll
+        for (int u = 0; u < 8; ++u) *reinterpret_cast<uint4*>(sT + swz<128>(row, u)) = make_uint4(0, 0, 0, 0);
+#pragma unroll
+        for (int i = 0; i < WIN; ++i) {
+          const int ah = i - qy + WIN - 1, aw = kRelW + i - qx + WIN - 1;
+          *reinterpret_cast<__nv_bfloat16*>(sT + swz<128>(row, ah >> 3) + (ah & 7) * 2) = __float2bfloat16_rn(rs[i]);
+          *reinterpret_cast<__nv_bfloat16*>(sT + swz<128>(row, aw >> 3) + (aw & 7) * 2) = __float2bfloat16_rn(cs[i]);
+        }
+      }
+      fence_proxy_async_smem();
+      tc_fence_before();
+      ok = wg_sync(&bar_wg[g], ph, lane, &abort_flag);
+      if (!ok) break;
+      // ---- R3: dV, dK (per 128-key tile), dQ, dR
+      if (elected) {
+        tc_fence_after();
+#pragma unroll 1
+        for (int t = 0; t < C::MT; ++t) {
+#pragma unroll 1
+          for (int ks = 0; ks < 4; ++ks) {
+            mma_f16_ss(slot + C::COL_DV + t * D, smem_desc(pa + t * 16384 + ks * 2048, 8192, 1024, SW_128B),
+                       smem_desc(doa + ks * 16 * C::ROWB, 16, C::SBO, C::SW), idKV, ks != 0);
+            mma_f16_ss(slot + C::COL_DK + t * D, smem_desc(dsa + t * 16384 + ks * 2048, 8192, 1024, SW_128B),
+                       smem_desc(qa + ks * 16 * C::ROWB, 16, C::SBO, C::SW), idKV, ks != 0);
+          }
+        }
+#pragma unroll 1
+        for (int ks = 0; ks < C::KSTEPS; ++ks)
+          mma_f16_ss(slot + C::COL_DQ, smem_desc(dsa + (ks >> 2) * 8192 + (ks & 3) * 32, 16, 1024, SW_128B),
+                     smem_desc(ka + ks * 16 * C::ROWB, 16, C::SBO, C::SW), idQ, ks != 0);
+#pragma unroll 1
+        for (int ks = 0; ks < 4; ++ks) {
+          mma_f16_ss(slot + C::COL_DQ, smem_desc(tA + ks * 32, 16, 1024, SW_128B),
+                     smem_desc(ra + ks * 16 * C::ROWB, 16, C::SBO, C::SW), idQ, 1);
+          mma_f16_ss(slot + C::COL_DR, smem_desc(tA + ks * 2048, 8192, 1024, SW_128B),
+                     smem_desc(qa + ks * 16 * C::ROWB, 16, C::SBO, C::SW), idR, ks != 0);
+        }
+        mma_commit(&bar_r3[g]);
+        mma_commit(&bar_empty[s]);
+      }
+      ok = warp_ok(mbar_wait(&bar_r3[g], j & 1, kWaitNs, &abort_flag));
+      if (!ok) break;
+      tc_fence_after();
+      // ---- epilogue
+#pragma unroll
+      for (int t = 0; t < C::MT; ++t) {
+        float dv[D], dk[D];
+        tmem_ld_d<D>(ts + C::COL_DV + t * D, dv);
+        tmem_ld_d<D>(ts + C::COL_DK + t * D, dk);
+        tmem_wait_ld();
+        const int key = t * 128 + 32 * wq + lane;
+        const int kr = key / WIN, kc = key - (key / WIN) * WIN;
+        const int Y = y0 + kr, X = x0 + kc;
+        if (key < C::KS && Y >= 0 && Y < p.H && X >= 0 && X < p.W) {
+          const size_t off = ((static_cast<size_t>(n) * p.H + Y) * p.W + X) * C_all + static_cast<size_t>(head) * D;
+#pragma unroll
+          for (int e = 0; e < D; e += 4) {
+            atomicAdd(reinterpret_cast<float4*>(p.dv32 + off + e), make_float4(dv[e], dv[e + 1], dv[e + 2], dv[e + 3]));
+            atomicAdd(reinterpret_cast<float4*>(p.dk32 + off + e),
+                      make_float4(p.s * dk[e], p.s * dk[e + 1], p.s * dk[e + 2], p.s * dk[e + 3]));
+          }
+        }
+      }
+      {
+        float dqv[D], drv[D];
+        tmem_ld_d<D>(ts + C::COL_DQ, dqv);
+        tmem_ld_d<D>(ts + C::COL_DR, drv);
+        tmem_wait_ld();
+        if (act) {
+          uint32_t pk[D / 2];
+#pragma unroll
+          for (int e = 0; e < D / 2; ++e) pk[e] = pack_bf16x2(p.s * dqv[2 * e], p.s * dqv[2 * e + 1]);
+#pragma unroll
+          for (int e = 0; e < D / 8; ++e)
+            reinterpret_cast<uint4*>(p.dq + pix)[e] = make_uint4(pk[4 * e], pk[4 * e + 1], pk[4 * e + 2], pk[4 * e + 3]);
+          // dR row = table entry `row` (rows 56..63 stay zero)
+#pragma unroll
+          for (int e = 0; e < D; ++e) drel[row * D + e] += p.s * drv[e];
+        }
+      }
+      tc_fence_before();
+      ok = wg_sync(&bar_wg[g], ph, lane, &abort_flag);
+    }
+    if (!ok && !abort_flag) record_timeout(&abort_flag);
+    // MMAs this warpgroup issued are complete before TMEM is released
+    if (elected) {
+      mma_commit(&bar_drain[g]);
+      mbar_wait(&bar_drain[g], 0, kWaitNs);
+    }
+    __syncwarp();
+  }
+
+  // ---------------------------------------------------------------- teardown
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  // both warpgroups' table sums into the float32 accumulators
+  for (int idx = tid; idx < (4 * WIN - 2) * D; idx += kThreads) {
+    const int r = idx / D, e = idx % D;      // r < 2w - 1: rel_h row; 2w - 1 <= r: rel_w row r - (2w - 1)
+    if (r < 2 * WIN - 1) {
+      atomicAdd(p.drh32 + r * D + e, sDrel[r * D + e] + sDrel[64 * D + r * D + e]);
+    } else if (r < 4 * WIN - 2) {
+      const int rr = r - (2 * WIN - 1);
+      atomicAdd(p.drw32 + rr * D + e, sDrel[(kRelW + rr) * D + e] + sDrel[64 * D + (kRelW + rr) * D + e]);
+    }
+  }
+  if (warp == 0) tmem_dealloc(tmem, kTmemCols);
+}
+
+}  // namespace bwdtc
+}  // namespace halo

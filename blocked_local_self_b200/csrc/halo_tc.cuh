@@ -87,10 +87,13 @@ struct Params {
   float c;                 // log2(e) / sqrt(d)
 };
 
-template <int D, int WIN, int STRIDE>
+// PP = PARTS: heads per item at stride 2 (4 x 16 queries fill the 64-row
+// tile; 2 at d = 32 when the head count is not a multiple of 4, 1 at d = 64).
+template <int D, int WIN, int STRIDE, int PP>
 struct Cfg {
   static constexpr int ROWB = D * 2;                      // bytes of one pixel's head slice
-  static constexpr int PARTS = (STRIDE == 1) ? 1 : (D == 16 ? 4 : (D == 32 ? 2 : 1));
+  static constexpr int PARTS = PP;
+  static_assert(STRIDE == 2 || PP == 1, "one head per item at stride 1");
   static constexpr int QROWS_PER_HEAD = (STRIDE == 1) ? 64 : 16;
   // stride 1: 64-row Q tile.  stride 2: zero-gap buffer so that the 64-row view
   // of head p holds its 16 queries in rows 16p..16p+15 and zeros elsewhere.
@@ -133,9 +136,9 @@ struct Cfg {
 };
 
 // Bytes of dynamic shared memory for a given stage count (plus 1 KB alignment slack).
-template <int D, int WIN, int STRIDE>
+template <int D, int WIN, int STRIDE, int PP>
 __host__ __device__ constexpr int smem_bytes(int stages) {
-  using C = Cfg<D, WIN, STRIDE>;
+  using C = Cfg<D, WIN, STRIDE, PP>;
   return 1024 + 2 * C::P_TILE + C::SCRATCH + ((C::R_TILE + 1023) / 1024) * 1024 + stages * C::STAGE_BYTES +
          C::ONES_TILE;
 }
@@ -180,11 +183,11 @@ __device__ __forceinline__ ItemCoord item_coord(int item, int groups, int nbx, i
   return c;
 }
 
-template <int D, int WIN, int STRIDE>
+template <int D, int WIN, int STRIDE, int PP>
 __global__ void __launch_bounds__(kThreads, 1)
     halo_fwd_tc(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__ CUtensorMap tmap_k,
                 const __grid_constant__ CUtensorMap tmap_v, const Params p) {
-  using C = Cfg<D, WIN, STRIDE>;
+  using C = Cfg<D, WIN, STRIDE, PP>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sP = smem;                                          // 2 x P_TILE (one per warpgroup)

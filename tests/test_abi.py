@@ -110,13 +110,15 @@ def test_kernel_names():
     assert name(2, 24, 32, 8, 16, 8, 3, 1, 1) == "halo_fwd_tc2<16,14>"  # odd: head pairs
     assert name(2, 40, 32, 8, 32, 8, 2, 1, 1) == "halo_fwd_tc2<32,12>"
     assert name(64, 32, 32, 8, 64, 8, 3, 1, 1) == "halo_fwd_tc4<64,14>"
-    assert name(64, 24, 32, 8, 64, 8, 3, 1, 1) == "halo_fwd_tc<64,14,1>"  # odd number of block rows
+    assert name(64, 24, 32, 8, 64, 8, 3, 1, 1) == "halo_fwd_tc<64,14,1,1>"  # odd number of block rows
     assert name(2, 16, 24, 3, 16, 8, 3, 1, 1) == "halo_fwd_tc4<16,14>"   # odd head count, even block rows
-    assert name(2, 24, 24, 3, 16, 8, 3, 1, 1) == "halo_fwd_tc<16,14,1>"   # odd head count, odd block rows
+    assert name(2, 24, 24, 3, 16, 8, 3, 1, 1) == "halo_fwd_tc<16,14,1,1>"   # odd head count, odd block rows
     assert name(2, 32, 48, 3, 16, 16, 2, 1, 1) == "halo_fwd_tc3<16,20,16>"
-    assert name(64, 64, 64, 8, 32, 8, 3, 2, 1) == "halo_fwd_tc<32,14,2>"
+    assert name(64, 64, 64, 8, 32, 8, 3, 2, 1) == "halo_fwd_tc<32,14,2,4>"  # four heads per 64-row tile
+    assert name(64, 64, 64, 6, 32, 8, 3, 2, 1) == "halo_fwd_tc<32,14,2,2>"  # six heads: pairs
     assert name(16, 128, 128, 8, 32, 16, 4, 1, 1) == "halo_fwd_tc3<32,24,16>"
-    assert name(1, 16, 16, 2, 32, 4, 1, 1, 0) == "halo_fwd_simt<float,32>"
+    assert name(1, 16, 16, 2, 32, 4, 1, 1, 0) == "halo_fwd_win<float,32>"   # window staged in shared memory
+    assert name(1, 16, 16, 2, 40, 4, 1, 1, 0) == "halo_fwd_simt<float,64>"  # dim_head the staged kernel lacks
     assert name(2, 32, 32, 4, 40, 16, 4, 1, 1) == "halo_fwd_simt<bf16,64>"
     assert name(1, 16, 16, 2, 32, 5, 1, 1, 0) == "none"
 

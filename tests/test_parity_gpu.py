@@ -173,6 +173,19 @@ def test_small_full_bf16(case):
     _compare(got, want, TOL["bf16"], str(case))
 
 
+def test_stage1_shape_in_float32_every_pixel():
+    """The float32 path (window staged in shared memory) at the stage-1
+    layer's full size, every output pixel against the oracle at 1e-4."""
+    wl = workloads.NEXT_WORKLOADS["stage1_f32"]
+    h = _lib()
+    assert h.kernel_name(wl.N, wl.H, wl.W, wl.heads, wl.dim_head, wl.block, wl.halo, wl.stride,
+                         wl.torch_dtype) == "halo_fwd_win<float,16>"
+    inputs = make_inputs(wl)
+    got = _run(wl, inputs)
+    want = oracle.halo_attention(*inputs, block=wl.block, halo=wl.halo, stride=wl.stride)
+    _compare(got, want, TOL["f32"], wl.name)
+
+
 SIMT_CASES = [
     dict(N=2, H=12, W=20, heads=3, dim_head=8, block=4, halo=2, stride=1, dtype="f32"),
     dict(N=1, H=16, W=16, heads=2, dim_head=40, block=4, halo=1, stride=2, dtype="f32"),
@@ -181,6 +194,12 @@ SIMT_CASES = [
     dict(N=2, H=32, W=32, heads=4, dim_head=40, block=16, halo=4, stride=1, dtype="bf16"),
     dict(N=1, H=16, W=16, heads=1, dim_head=16, block=8, halo=3, stride=2, dtype="bf16"),
     dict(N=2, H=24, W=16, heads=4, dim_head=16, block=8, halo=4, stride=1, dtype="bf16"),
+    # window staged in shared memory: every dim_head it takes, both strides, ragged passes
+    dict(N=2, H=16, W=24, heads=3, dim_head=64, block=8, halo=3, stride=1, dtype="f32"),
+    dict(N=1, H=32, W=32, heads=2, dim_head=128, block=8, halo=2, stride=2, dtype="f32"),
+    dict(N=1, H=32, W=32, heads=2, dim_head=16, block=32, halo=0, stride=1, dtype="f32"),  # 1024 queries, 4 passes
+    dict(N=2, H=16, W=16, heads=2, dim_head=8, block=16, halo=3, stride=2, dtype="f32"),
+    dict(N=1, H=24, W=24, heads=2, dim_head=32, block=12, halo=5, stride=1, dtype="bf16"),
 ]
 
 
@@ -236,9 +255,10 @@ FAMILY_CASES = {
     "halo_fwd_tc4<64,": dict(N=2, H=32, W=24, heads=2, dim_head=64, block=8, halo=3, stride=1),
     "halo_fwd_tc2<16,": dict(N=2, H=24, W=24, heads=4, dim_head=16, block=8, halo=3, stride=1),
     "halo_fwd_tc2<32,": dict(N=2, H=24, W=24, heads=2, dim_head=32, block=8, halo=2, stride=1),
-    "halo_fwd_tc<64,14,1>": dict(N=2, H=24, W=24, heads=2, dim_head=64, block=8, halo=3, stride=1),
-    "halo_fwd_tc<16,14,2>": dict(N=2, H=32, W=32, heads=8, dim_head=16, block=8, halo=3, stride=2),
-    "halo_fwd_tc<32,14,2>": dict(N=2, H=32, W=32, heads=4, dim_head=32, block=8, halo=3, stride=2),
+    "halo_fwd_tc<64,14,1,1>": dict(N=2, H=24, W=24, heads=2, dim_head=64, block=8, halo=3, stride=1),
+    "halo_fwd_tc<16,14,2,4>": dict(N=2, H=32, W=32, heads=8, dim_head=16, block=8, halo=3, stride=2),
+    "halo_fwd_tc<32,14,2,4>": dict(N=2, H=32, W=32, heads=4, dim_head=32, block=8, halo=3, stride=2),
+    "halo_fwd_tc<32,14,2,2>": dict(N=2, H=32, W=32, heads=2, dim_head=32, block=8, halo=3, stride=2),
     "halo_fwd_tc3<16,": dict(N=1, H=32, W=32, heads=2, dim_head=16, block=16, halo=3, stride=1),
     "halo_fwd_tc3<32,": dict(N=1, H=32, W=48, heads=2, dim_head=32, block=16, halo=4, stride=1),
     "halo_fwd_tc3<16,38,32>": dict(N=1, H=64, W=32, heads=2, dim_head=16, block=32, halo=3, stride=1),

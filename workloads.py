@@ -126,16 +126,18 @@ WORKLOADS: dict[str, Workload] = {
 # The workload the throughput benchmark times (the stage-1 layer).
 BENCH_WORKLOAD = "stage1_bf16"
 
-# Shapes of the paper's further settings, measured beside the five above:
-# global attention at the smallest resolution (block = the whole 32x32 map,
-# halo 0; section 2.2 and the deep stages of section 4) and the block-32,
-# halo-3 setting of the detection backbones (section 4.5, Table 5).
+# Shapes measured beside the five above: global attention at the smallest
+# resolution (block = the whole 32x32 map, halo 0; section 2.2 and the deep
+# stages of section 4), the block-32, halo-3 setting of the detection
+# backbones (section 4.5, Table 5), and the stage-1 layer in float32.
 NEXT_WORKLOADS: dict[str, Workload] = {
     w.name: w
     for w in [
         Workload("global32_bf16", N=64, H=32, W=32, heads=8, dim_head=32, block=32, halo=0, stride=1, dtype="bf16"),
         Workload("block32_h3_bf16", N=4, H=128, W=128, heads=8, dim_head=32, block=32, halo=3, stride=1,
                  dtype="bf16"),
+        # the stage-1 layer in float32 (the float32 path at a full-size shape)
+        Workload("stage1_f32", N=32, H=64, W=64, heads=8, dim_head=16, block=8, halo=3, stride=1, dtype="f32"),
     ]
 }
 
