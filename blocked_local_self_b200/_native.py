@@ -29,6 +29,7 @@ HALO_ERR_ALIAS = -10
 HALO_ERR_DEVICE = -11
 HALO_ERR_KERNEL = -12
 HALO_ERR_WORKSPACE = -13
+HALO_ERR_SCRATCH_LIMIT = -14
 
 HALO_KERNEL_NONE = 0
 HALO_KERNEL_SIMT_F32 = 1
@@ -44,6 +45,7 @@ SIGNATURES = {
     "halo_attn_masked": (_i, [_vp] * 6 + [_i] * 10 + [_vp]),
     "halo_attn_bwd": (_i, [_vp] * 13 + [ctypes.c_size_t] + [_i] * 10 + [_vp]),
     "halo_attn_bwd_workspace_size": (_i, [_i] * 10 + [ctypes.POINTER(ctypes.c_size_t)]),
+    "halo_attn_bwd_noalloc": (_i, [_vp] * 12 + [_i] * 10 + [_vp]),
     "halo_kernel_for": (_i, [_i] * 9),
     "halo_kernel_name": (ctypes.c_char_p, [_i] * 9),
     "halo_masked_kernel_name": (ctypes.c_char_p, [_i] * 10),

@@ -42,6 +42,8 @@ const char* status_text(int code) {
     case HALO_ERR_DEVICE: return "the current device is not an sm_100 GPU";
     case HALO_ERR_KERNEL: return "the SASA mask size must be odd, and at most 2*halo+1";
     case HALO_ERR_WORKSPACE: return "the workspace is missing, misaligned or too small";
+    case HALO_ERR_SCRATCH_LIMIT:
+      return "the shape needs more scratch than halo_attn_bwd_noalloc's built-in 16 MiB (use halo_attn_bwd)";
     default: return "unknown status code";
   }
 }
@@ -742,6 +744,31 @@ int attn_bwd(const void* const* in, void* const* grads, void* ws, size_t ws_byte
                              : launch_bwd<__nv_bfloat16>(plan, s.d, in, grads, ws, sm_count, st);
 }
 
+// ----------------------------------------------------------------------------
+// Backward with built-in scratch (halo_attn_bwd_noalloc)
+// ----------------------------------------------------------------------------
+// The backward's float32 accumulators live in this file-scope array instead
+// of a caller-provided workspace.  Every device that loads the library holds
+// it until the process exits.  Host code may not pass `g_bwd_scratch` itself
+// to a kernel (on the host the name is only a stand-in for the device
+// object): its device address is fetched once per device with
+// cudaGetSymbolAddress, with that device current, and cached here.
+static __device__ __align__(256) unsigned char g_bwd_scratch[HALO_BWD_NOALLOC_MAX_WORKSPACE];
+void* g_bwd_scratch_addr[kMaxDevices];
+
+int bwd_scratch(void** addr) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return HALO_ERR_CUDA;
+  std::lock_guard<std::mutex> lock(g_mutex);
+  if (!g_bwd_scratch_addr[dev]) {
+    void* ptr = nullptr;
+    if (cudaGetSymbolAddress(&ptr, g_bwd_scratch) != cudaSuccess || !ptr) return HALO_ERR_CUDA;
+    g_bwd_scratch_addr[dev] = ptr;
+  }
+  *addr = g_bwd_scratch_addr[dev];
+  return HALO_OK;
+}
+
 // The self test's own result flag: a timeout that a real halo_attn recorded
 // in g_halo_error stays there for halo_get_last_error.
 __device__ int g_selftest_flag;
@@ -896,6 +923,24 @@ int halo_attn_masked(const void* q, const void* k, const void* v, const void* re
   s.kmask = kernel;
   if (kernel <= 0) return HALO_ERR_KERNEL;
   return attn_device(q, k, v, rel_h, rel_w, out, s, static_cast<cudaStream_t>(stream));
+}
+
+int halo_attn_bwd_noalloc(const void* q, const void* k, const void* v, const void* rel_h, const void* rel_w,
+                          const void* out, const void* dout, void* dq, void* dk, void* dv, void* drel_h,
+                          void* drel_w, int N, int H, int W, int heads, int dim_head, int block, int halo,
+                          int stride, int kernel, int dtype, void* stream) {
+  Shape s{N, H, W, heads, dim_head, block, halo, stride, dtype};
+  s.kmask = kernel;
+  BwdPlan plan;
+  int rc = bwd_plan(s, &plan);
+  if (rc != HALO_OK) return rc;
+  if (plan.ws_bytes > HALO_BWD_NOALLOC_MAX_WORKSPACE) return HALO_ERR_SCRATCH_LIMIT;
+  void* ws = nullptr;
+  rc = bwd_scratch(&ws);
+  if (rc != HALO_OK) return rc;
+  const void* in[7] = {q, k, v, rel_h, rel_w, out, dout};
+  void* grads[5] = {dq, dk, dv, drel_h, drel_w};
+  return attn_bwd(in, grads, ws, HALO_BWD_NOALLOC_MAX_WORKSPACE, s, static_cast<cudaStream_t>(stream));
 }
 
 int halo_attn_bwd_workspace_size(int N, int H, int W, int heads, int dim_head, int block, int halo, int stride,

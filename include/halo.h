@@ -64,7 +64,8 @@ typedef enum {
   HALO_ERR_ALIAS = -10,        /* out overlaps an input */
   HALO_ERR_DEVICE = -11,       /* the current device is not an sm_100 GPU */
   HALO_ERR_KERNEL = -12,       /* SASA mask size not odd, or larger than 2*halo+1 */
-  HALO_ERR_WORKSPACE = -13     /* the backward's workspace is NULL, not 256-byte aligned or too small */
+  HALO_ERR_WORKSPACE = -13,    /* the backward's workspace is NULL, not 256-byte aligned or too small */
+  HALO_ERR_SCRATCH_LIMIT = -14 /* halo_attn_bwd_noalloc: the shape needs more than its built-in scratch */
 } halo_status;
 
 /* Which kernel halo_attn would launch for a shape (halo_kernel_for). */
@@ -168,6 +169,37 @@ int halo_attn_bwd(const void* q, const void* k, const void* v, const void* rel_h
  * rejected.  Thread-local storage as for halo_kernel_name; no device work. */
 const char* halo_bwd_kernel_name(int N, int H, int W, int heads, int dim_head, int block, int halo, int stride,
                                  int kernel, int dtype);
+
+/*
+ * halo_attn_bwd_noalloc -- halo_attn_bwd for callers that cannot allocate
+ * device memory when they run the backward.  The pages have no counterpart;
+ * this is a convenience of this library.  Such callers are, for instance,
+ * code whose device memory all belongs to a caching allocator (a cudaMalloc
+ * of its own would fail once the allocator has reserved the free memory, or
+ * would fragment it), and latency-critical paths where the device-wide
+ * synchronisation that cudaMalloc and cudaFree can cause is not acceptable.
+ *
+ * Same arguments and results as halo_attn_bwd without workspace and
+ * workspace_bytes: the float32 accumulators live in a static device array
+ * of HALO_BWD_NOALLOC_MAX_WORKSPACE bytes (16 MiB) inside the library, which
+ * every GPU that loads the library holds until the process exits.  Shapes
+ * whose halo_attn_bwd_workspace_size exceeds that return
+ * HALO_ERR_SCRATCH_LIMIT before any device work.  The call allocates
+ * nothing (no cudaMalloc, cudaFree or allocating library routine); it
+ * clears the part of the array it uses at the start of every call.
+ *
+ * The first call on a device looks up the array's device address on that
+ * device (cudaGetSymbolAddress, with that device current) and keeps it; make
+ * that first call before any stream capture.  Every call shares the one
+ * array: calls whose work overlaps on the GPU (other streams, other host
+ * threads, without ordering between them) race on it and give wrong
+ * gradients.  Order such calls, or use halo_attn_bwd with a workspace each.
+ */
+#define HALO_BWD_NOALLOC_MAX_WORKSPACE (16u << 20)
+int halo_attn_bwd_noalloc(const void* q, const void* k, const void* v, const void* rel_h, const void* rel_w,
+                          const void* out, const void* dout, void* dq, void* dk, void* dv, void* drel_h,
+                          void* drel_w, int N, int H, int W, int heads, int dim_head, int block, int halo,
+                          int stride, int kernel, int dtype, void* stream);
 
 /* Workspace bytes halo_attn_bwd needs for these arguments, in *bytes
  * (2 N H W heads dim_head + 2 (2w - 1) dim_head floats, each part rounded up

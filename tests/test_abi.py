@@ -50,7 +50,7 @@ def test_status_codes_match_header():
 
 def test_strerror_covers_codes():
     lib = _lib()
-    for code in range(0, -14, -1):
+    for code in range(0, -15, -1):
         text = lib.halo_strerror(code).decode()
         assert text and text != "unknown status code"
     assert lib.halo_strerror(-99).decode() == "unknown status code"
