@@ -233,6 +233,9 @@ def ncu_traffic(workload: str, kernel: str):
         fields = dict(re.findall(r"^- (\w+): `?([^`\n]+?)`?\s*$", text, flags=re.M))
         if fields.get("workload") != workload or "dram_bytes_per_launch" not in fields:
             continue
+        family = (kernel or "").split("<")[0]
+        if "kernel" in fields and family and family + "<" not in fields["kernel"]:
+            continue  # a summary of another kernel on the same workload (e.g. the backward)
         if fields.get("kernel_source_sha") != kernel_source_hash(kernel):
             return None
         return float(fields["dram_bytes_per_launch"])
