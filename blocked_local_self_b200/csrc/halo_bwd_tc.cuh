@@ -15,7 +15,7 @@
 //
 // Work item = one 8x8 block of one head.  Two warpgroups take alternate items,
 // each with a 256-column TMEM slot and its own P / dS / T buffers in shared
-// memory; the elected thread of a warpgroup issues its MMAs:
+// memory; lane 0 of its warps issue its MMAs (independent chains in parallel):
 //   R1  S = Q K^T (M=64, N=w^2 rounded to 8) at slot column 0 and
 //       G = Q R^T (N=56) at column 200: the relative logits, gathered per
 //       query as in the forward two-block kernel (out-of-image rows and
@@ -29,7 +29,8 @@
 //       output); bf16 p and dS into the P and dS buffers, the row and column
 //       sums of dS into the query's T row.
 //   R3  dV_t = P^T[keys of tile t] dout, dK_t = dS^T[tile t] Q (M=128, keys
-//       in 128-row tiles), dQ = dS K + T R (M=64), dR = T^T Q (M=64).  One
+//       in 128-row tiles), dQ = dS K + T R (M=64, two accumulators),
+//       dR = T^T Q (M=64): four chains issued by the four warps.  One
 //       shared-memory layout serves as the K-major A operand of dQ (rows =
 //       queries, K = keys) and as the MN-major A operand of dK and dV
 //       (M = keys, K = queries): rows of 64 keys (128 B, 128-byte swizzle),
@@ -45,6 +46,7 @@
 #include <cstdint>
 #include <cuda.h>
 #include <cuda_bf16.h>
+#include <type_traits>
 
 #include "halo_tc.cuh"
 #include "halo_tc2.cuh"
@@ -107,14 +109,16 @@ struct Cfg {
   static constexpr int WG_BYTES = 2 * PBUF + TBUF;     // P, dS, T of one warpgroup
   static constexpr int DREL_BYTES = 2 * 64 * D * 4;    // two warpgroups' table accumulators (float32)
   // TMEM columns of R3's accumulators: dV tiles, dK tiles, dQ, dR
-  static constexpr uint32_t COL_DV = 0, COL_DK = MT * D, COL_DQ = 2 * MT * D, COL_DR = 2 * MT * D + D;
+  // (after pass A the G columns are free too, so R3 may use the whole slot)
+  static constexpr uint32_t COL_DV = 0, COL_DK = MT * D, COL_DQ = 2 * MT * D, COL_DQ2 = 2 * MT * D + D,
+                            COL_DR = 2 * MT * D + 2 * D;
   static constexpr SmemSwizzle SW = (ROWB == 32) ? SW_32B : SW_64B;
   static constexpr uint32_t SBO = 8 * ROWB;
   static constexpr int HALO = (WIN - kBlock) / 2;
   static_assert(D == 16 || D == 32, "dim_head 16 or 32");
   static_assert(WIN % 2 == 0 && WIN >= 8 && WIN <= 14, "window 8..14");
   static_assert(NS <= (int)kGBase, "S columns below the relative logits");
-  static_assert(COL_DR + D <= kGBase, "R3 accumulators below G");
+  static_assert(COL_DR + D <= kSlotCols, "R3 accumulators in the slot");
   static_assert(2 * WIN - 1 <= kRelW && kRelW + 2 * WIN - 1 <= 56, "relative table rows");
 };
 
@@ -143,6 +147,29 @@ template <int D>
 __device__ __forceinline__ void tmem_ld_d(uint32_t taddr, float* r) {
   if constexpr (D == 32) tc2::tmem_ld_x32(taddr, r);
   else tmem_ld_exact<D>(taddr, r);
+}
+
+// A sweep over TMEM columns [0, NS) of this thread's lane in pieces of 16,
+// the next piece's load in flight while the current one is processed:
+// f(z, std::integral_constant<int, J0>) gets columns [J0, J0 + 16).
+template <int J0, int NS, class F>
+__device__ __forceinline__ void sweep16_at(uint32_t ts, uint32_t (&cur)[16], uint32_t (&nxt)[16], F& f) {
+  if constexpr (J0 + 16 < NS) tmem_ld_32x32b_x16(ts + J0 + 16, nxt);
+  float z[16];
+#pragma unroll
+  for (int i = 0; i < 16; ++i) z[i] = __uint_as_float(cur[i]);
+  f(z, std::integral_constant<int, J0>{});
+  if constexpr (J0 + 16 < NS) {
+    tmem_wait_ld();
+    sweep16_at<J0 + 16, NS>(ts, nxt, cur, f);
+  }
+}
+template <int NS, class F>
+__device__ __forceinline__ void sweep16(uint32_t ts, F&& f) {
+  uint32_t a[16], b[16];
+  tmem_ld_32x32b_x16(ts, a);
+  tmem_wait_ld();
+  sweep16_at<0, NS>(ts, a, b, f);
 }
 
 // Barrier of one warpgroup's four warps on an mbarrier of count 4, so that
@@ -175,7 +202,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   __shared__ __align__(8) uint64_t bar_r2[2];
   __shared__ __align__(8) uint64_t bar_r3[2];
   __shared__ __align__(8) uint64_t bar_wg[2];    // count 4: the warps of warpgroup g
-  __shared__ __align__(8) uint64_t bar_drain[2];
+  __shared__ __align__(8) uint64_t bar_drain[8];  // per softmax warp (its lane 0 issues MMAs)
   __shared__ uint32_t tmem_base_sh;
   __shared__ int abort_flag;
 
@@ -188,15 +215,15 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (tid == 0) {
     for (int i = 0; i < S; ++i) {
       mbar_init(&bar_full[i], 1);
-      mbar_init(&bar_empty[i], 1);
+      mbar_init(&bar_empty[i], 4);   // the four R3 issuers
     }
     for (int g = 0; g < 2; ++g) {
-      mbar_init(&bar_r1[g], 1);
+      mbar_init(&bar_r1[g], 2);      // S (warp 0) and G (warp 1)
       mbar_init(&bar_r2[g], 1);
-      mbar_init(&bar_r3[g], 1);
+      mbar_init(&bar_r3[g], 4);      // one commit per issuing warp
       mbar_init(&bar_wg[g], 4);
-      mbar_init(&bar_drain[g], 1);
     }
+    for (int w = 0; w < 8; ++w) mbar_init(&bar_drain[w], 1);
     abort_flag = 0;
     fence_mbar_init();
   }
@@ -295,17 +322,29 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint8_t* st = sStage + s * C::STAGE_BYTES;
       const uint32_t qa = smem_addr(st + C::OFF_Q), doa = smem_addr(st + C::OFF_DO);
       const uint32_t ka = smem_addr(st + C::OFF_K), va = smem_addr(st + C::OFF_V);
-      // ---- R1: S and G
-      if (elected) {
+      const int item = blockIdx.x + k * gridDim.x;
+      const int head = item % p.heads, blk = item / p.heads;
+      const int bx = blk % p.nbx, by = (blk / p.nbx) % p.nby, n = blk / (p.nbx * p.nby);
+      const int y0 = by * kBlock - p.halo, x0 = bx * kBlock - p.halo;
+      const int y = by * kBlock + qy, x = bx * kBlock + qx;
+      const size_t pix = ((static_cast<size_t>(n) * p.H + y) * p.W + x) * C_all + static_cast<size_t>(head) * D;
+      // this query's out and dout rows (for D = dout . out), in flight during the MMAs and pass A
+      uint4 orow[D / 8], drow[D / 8];
+#pragma unroll
+      for (int e = 0; e < D / 8; ++e) {
+        orow[e] = act ? *reinterpret_cast<const uint4*>(p.out + pix + 8 * e) : make_uint4(0, 0, 0, 0);
+        drow[e] = act ? *reinterpret_cast<const uint4*>(p.dout + pix + 8 * e) : make_uint4(0, 0, 0, 0);
+      }
+      // ---- R1: S (warp 0) and G (warp 1), issued in parallel
+      if (wq < 2 && lane == 0) {
         if (mbar_wait(&bar_full[s], (k / S) & 1, kWaitNs, &abort_flag)) {
           tc_fence_after();
+          const uint32_t dst = slot + (wq ? kGBase : 0u), ba = wq ? ra : ka;
+          const uint32_t id = wq ? idG : idS;
 #pragma unroll
-          for (int ks = 0; ks < D / 16; ++ks) {
-            mma_f16_ss(slot, smem_desc(qa + 32 * ks, 16, C::SBO, C::SW), smem_desc(ka + 32 * ks, 16, C::SBO, C::SW),
-                       idS, ks != 0);
-            mma_f16_ss(slot + kGBase, smem_desc(qa + 32 * ks, 16, C::SBO, C::SW),
-                       smem_desc(ra + 32 * ks, 16, C::SBO, C::SW), idG, ks != 0);
-          }
+          for (int ks = 0; ks < D / 16; ++ks)
+            mma_f16_ss(dst, smem_desc(qa + 32 * ks, 16, C::SBO, C::SW), smem_desc(ba + 32 * ks, 16, C::SBO, C::SW),
+                       id, ks != 0);
           mma_commit(&bar_r1[g]);
         } else if (!abort_flag) {
           record_timeout(&abort_flag);
@@ -315,10 +354,6 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (!ok) break;
       tc_fence_after();
 
-      const int item = blockIdx.x + k * gridDim.x;
-      const int head = item % p.heads, blk = item / p.heads;
-      const int bx = blk % p.nbx, by = (blk / p.nbx) % p.nby, n = blk / (p.nbx * p.nby);
-      const int y0 = by * kBlock - p.halo, x0 = bx * kBlock - p.halo;
       // ---- relative logits of this query (log2 units), -inf for masked rows / columns
       float rh[WIN], rw[WIN];
       {
@@ -350,24 +385,6 @@ __global__ void __launch_bounds__(kThreads, 1)
           rw[kc] = keep ? a[kc] * c : -INFINITY;
         }
       }
-      // ---- D = dout . out of this query
-      const int y = by * kBlock + qy, x = bx * kBlock + qx;
-      const size_t pix = ((static_cast<size_t>(n) * p.H + y) * p.W + x) * C_all + static_cast<size_t>(head) * D;
-      float Dq = 0.f;
-      if (act) {
-#pragma unroll
-        for (int e = 0; e < D; e += 8) {
-          const uint4 o = *reinterpret_cast<const uint4*>(p.out + pix + e);
-          const uint4 d = *reinterpret_cast<const uint4*>(p.dout + pix + e);
-          const __nv_bfloat162* o2 = reinterpret_cast<const __nv_bfloat162*>(&o);
-          const __nv_bfloat162* d2 = reinterpret_cast<const __nv_bfloat162*>(&d);
-#pragma unroll
-          for (int t = 0; t < 4; ++t) {
-            const float2 of = __bfloat1622float2(o2[t]), df = __bfloat1622float2(d2[t]);
-            Dq = fmaf(of.x, df.x, fmaf(of.y, df.y, Dq));
-          }
-        }
-      }
       // ---- pass A: exact row maximum, per window row max of c S + c rel_w,
       // then over rows with c rel_h added
       float m = -INFINITY;
@@ -375,40 +392,49 @@ __global__ void __launch_bounds__(kThreads, 1)
         float rmax[WIN];
 #pragma unroll
         for (int r = 0; r < WIN; ++r) rmax[r] = -INFINITY;
+        sweep16<C::NS>(ts, [&](const float (&z)[16], auto jc) {
+          constexpr int J0 = decltype(jc)::value;
 #pragma unroll
-        for (int j0 = 0; j0 < C::NS; j0 += 8) {
-          float z[8];
-          tmem_ld_x8(ts + j0, z);
-          tmem_wait_ld();
-#pragma unroll
-          for (int t = 0; t < 8; ++t)
-            if (j0 + t < C::KS) rmax[(j0 + t) / WIN] = fmaxf(rmax[(j0 + t) / WIN], fmaf(z[t], c, rw[(j0 + t) % WIN]));
-        }
+          for (int t = 0; t < 16; ++t)
+            if (J0 + t < C::KS) rmax[(J0 + t) / WIN] = fmaxf(rmax[(J0 + t) / WIN], fmaf(z[t], c, rw[(J0 + t) % WIN]));
+        });
 #pragma unroll
         for (int r = 0; r < WIN; ++r) m = fmaxf(m, rmax[r] + rh[r]);
+      }
+      // ---- D = dout . out of this query
+      float Dq = 0.f;
+#pragma unroll
+      for (int e = 0; e < D / 8; ++e) {
+        const __nv_bfloat162* o2 = reinterpret_cast<const __nv_bfloat162*>(&orow[e]);
+        const __nv_bfloat162* d2 = reinterpret_cast<const __nv_bfloat162*>(&drow[e]);
+#pragma unroll
+        for (int t = 0; t < 4; ++t) {
+          const float2 of = __bfloat1622float2(o2[t]), df = __bfloat1622float2(d2[t]);
+          Dq = fmaf(of.x, df.x, fmaf(of.y, df.y, Dq));
+        }
       }
       // ---- pass B: p' = 2^(c S + c rel_w + (c rel_h - m)) into the P buffer, row sum
       float brow[WIN];
 #pragma unroll
       for (int r = 0; r < WIN; ++r) brow[r] = rh[r] - m;
       float l = 0.f;
+      sweep16<C::NS>(ts, [&](const float (&z)[16], auto jc) {
+        constexpr int J0 = decltype(jc)::value;
+        uint32_t pk[8];
 #pragma unroll
-      for (int j0 = 0; j0 < C::NS; j0 += 8) {
-        float z[8];
-        tmem_ld_x8(ts + j0, z);
-        tmem_wait_ld();
-        uint32_t pk[4];
-#pragma unroll
-        for (int t = 0; t < 8; t += 2) {
+        for (int t = 0; t < 16; t += 2) {
           float e0 = 0.f, e1 = 0.f;
-          if (j0 + t < C::KS) e0 = exp2_mufu(fmaf(z[t], c, rw[(j0 + t) % WIN]) + brow[(j0 + t) / WIN]);
-          if (j0 + t + 1 < C::KS)
-            e1 = exp2_mufu(fmaf(z[t + 1], c, rw[(j0 + t + 1) % WIN]) + brow[(j0 + t + 1) / WIN]);
+          if (J0 + t < C::KS) e0 = exp2_mufu(fmaf(z[t], c, rw[(J0 + t) % WIN]) + brow[(J0 + t) / WIN]);
+          if (J0 + t + 1 < C::KS)
+            e1 = exp2_mufu(fmaf(z[t + 1], c, rw[(J0 + t + 1) % WIN]) + brow[(J0 + t + 1) / WIN]);
           l += e0 + e1;
           pk[t / 2] = pack_bf16x2(e0, e1);
         }
-        if (act) *reinterpret_cast<uint4*>(sP + pofs(row, j0 / 8)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
-      }
+        if (act) {
+          *reinterpret_cast<uint4*>(sP + pofs(row, J0 / 8)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+          *reinterpret_cast<uint4*>(sP + pofs(row, J0 / 8 + 1)) = make_uint4(pk[4], pk[5], pk[6], pk[7]);
+        }
+      });
       const float inv_l = 1.0f / l;
       // ---- R2: dP = dout V^T over the S columns
       tc_fence_before();
@@ -429,37 +455,38 @@ __global__ void __launch_bounds__(kThreads, 1)
       float rs[WIN], cs[WIN];
 #pragma unroll
       for (int i = 0; i < WIN; ++i) rs[i] = cs[i] = 0.f;
+      sweep16<C::NS>(ts, [&](const float (&dp)[16], auto jc) {
+        constexpr int J0 = decltype(jc)::value;
+        uint4 pv[2];
+        pv[0] = *reinterpret_cast<const uint4*>(sP + pofs(row, J0 / 8));
+        pv[1] = *reinterpret_cast<const uint4*>(sP + pofs(row, J0 / 8 + 1));
+        const __nv_bfloat162* p2 = reinterpret_cast<const __nv_bfloat162*>(pv);
+        uint32_t pk[8], dk[8];
 #pragma unroll
-      for (int j0 = 0; j0 < C::NS; j0 += 8) {
-        float dp[8];
-        tmem_ld_x8(ts + j0, dp);
-        const uint4 pv = *reinterpret_cast<const uint4*>(sP + pofs(row, j0 / 8));
-        tmem_wait_ld();
-        const __nv_bfloat162* p2 = reinterpret_cast<const __nv_bfloat162*>(&pv);
-        uint32_t pk[4], dk[4];
-#pragma unroll
-        for (int t = 0; t < 8; t += 2) {
+        for (int t = 0; t < 16; t += 2) {
           const float2 pp = __bfloat1622float2(p2[t / 2]);
           const float p0 = pp.x * inv_l, p1 = pp.y * inv_l;
           float d0 = 0.f, d1 = 0.f;
-          if (j0 + t < C::KS) {
+          if (J0 + t < C::KS) {
             d0 = p0 * (dp[t] - Dq);
-            rs[(j0 + t) / WIN] += d0;
-            cs[(j0 + t) % WIN] += d0;
+            rs[(J0 + t) / WIN] += d0;
+            cs[(J0 + t) % WIN] += d0;
           }
-          if (j0 + t + 1 < C::KS) {
+          if (J0 + t + 1 < C::KS) {
             d1 = p1 * (dp[t + 1] - Dq);
-            rs[(j0 + t + 1) / WIN] += d1;
-            cs[(j0 + t + 1) % WIN] += d1;
+            rs[(J0 + t + 1) / WIN] += d1;
+            cs[(J0 + t + 1) % WIN] += d1;
           }
           pk[t / 2] = pack_bf16x2(p0, p1);
           dk[t / 2] = pack_bf16x2(d0, d1);
         }
         if (act) {
-          *reinterpret_cast<uint4*>(sP + pofs(row, j0 / 8)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
-          *reinterpret_cast<uint4*>(sDS + pofs(row, j0 / 8)) = make_uint4(dk[0], dk[1], dk[2], dk[3]);
+          *reinterpret_cast<uint4*>(sP + pofs(row, J0 / 8)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+          *reinterpret_cast<uint4*>(sP + pofs(row, J0 / 8 + 1)) = make_uint4(pk[4], pk[5], pk[6], pk[7]);
+          *reinterpret_cast<uint4*>(sDS + pofs(row, J0 / 8)) = make_uint4(dk[0], dk[1], dk[2], dk[3]);
+          *reinterpret_cast<uint4*>(sDS + pofs(row, J0 / 8 + 1)) = make_uint4(dk[4], dk[5], dk[6], dk[7]);
         }
-      }
+      });
       // T row: rel_h entries kr - qy + w - 1, rel_w entries 28 + kc - qx + w - 1
       if (act) {
 #pragma unroll
@@ -475,29 +502,33 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_before();
       ok = wg_sync(&bar_wg[g], ph, lane, &abort_flag);
       if (!ok) break;
-      // ---- R3: dV, dK (per 128-key tile), dQ, dR
-      if (elected) {
+      // ---- R3, four independent MMA chains on the four warps' lane 0:
+      // warp 0 dV tiles, warp 1 dK tiles, warp 2 dQ = dS K, warp 3 T R (a
+      // second dQ accumulator) and dR = T^T Q
+      if (lane == 0) {
         tc_fence_after();
+        if (wq < 2) {
+          const uint32_t col = wq ? C::COL_DK : C::COL_DV;
+          const uint32_t aa = wq ? dsa : pa, bb = wq ? qa : doa;
 #pragma unroll 1
-        for (int t = 0; t < C::MT; ++t) {
+          for (int t = 0; t < C::MT; ++t)
+#pragma unroll 1
+            for (int ks = 0; ks < 4; ++ks)
+              mma_f16_ss(slot + col + t * D, smem_desc(aa + t * 16384 + ks * 2048, 8192, 1024, SW_128B),
+                         smem_desc(bb + ks * 16 * C::ROWB, 16, C::SBO, C::SW), idKV, ks != 0);
+        } else if (wq == 2) {
+#pragma unroll 1
+          for (int ks = 0; ks < C::KSTEPS; ++ks)
+            mma_f16_ss(slot + C::COL_DQ, smem_desc(dsa + (ks >> 2) * 8192 + (ks & 3) * 32, 16, 1024, SW_128B),
+                       smem_desc(ka + ks * 16 * C::ROWB, 16, C::SBO, C::SW), idQ, ks != 0);
+        } else {
 #pragma unroll 1
           for (int ks = 0; ks < 4; ++ks) {
-            mma_f16_ss(slot + C::COL_DV + t * D, smem_desc(pa + t * 16384 + ks * 2048, 8192, 1024, SW_128B),
-                       smem_desc(doa + ks * 16 * C::ROWB, 16, C::SBO, C::SW), idKV, ks != 0);
-            mma_f16_ss(slot + C::COL_DK + t * D, smem_desc(dsa + t * 16384 + ks * 2048, 8192, 1024, SW_128B),
-                       smem_desc(qa + ks * 16 * C::ROWB, 16, C::SBO, C::SW), idKV, ks != 0);
+            mma_f16_ss(slot + C::COL_DQ2, smem_desc(tA + ks * 32, 16, 1024, SW_128B),
+                       smem_desc(ra + ks * 16 * C::ROWB, 16, C::SBO, C::SW), idQ, ks != 0);
+            mma_f16_ss(slot + C::COL_DR, smem_desc(tA + ks * 2048, 8192, 1024, SW_128B),
+                       smem_desc(qa + ks * 16 * C::ROWB, 16, C::SBO, C::SW), idR, ks != 0);
           }
-        }
-#pragma unroll 1
-        for (int ks = 0; ks < C::KSTEPS; ++ks)
-          mma_f16_ss(slot + C::COL_DQ, smem_desc(dsa + (ks >> 2) * 8192 + (ks & 3) * 32, 16, 1024, SW_128B),
-                     smem_desc(ka + ks * 16 * C::ROWB, 16, C::SBO, C::SW), idQ, ks != 0);
-#pragma unroll 1
-        for (int ks = 0; ks < 4; ++ks) {
-          mma_f16_ss(slot + C::COL_DQ, smem_desc(tA + ks * 32, 16, 1024, SW_128B),
-                     smem_desc(ra + ks * 16 * C::ROWB, 16, C::SBO, C::SW), idQ, 1);
-          mma_f16_ss(slot + C::COL_DR, smem_desc(tA + ks * 2048, 8192, 1024, SW_128B),
-                     smem_desc(qa + ks * 16 * C::ROWB, 16, C::SBO, C::SW), idR, ks != 0);
         }
         mma_commit(&bar_r3[g]);
         mma_commit(&bar_empty[s]);
@@ -530,6 +561,13 @@ __global__ void __launch_bounds__(kThreads, 1)
         tmem_ld_d<D>(ts + C::COL_DQ, dqv);
         tmem_ld_d<D>(ts + C::COL_DR, drv);
         tmem_wait_ld();
+        {
+          float dq2[D];
+          tmem_ld_d<D>(ts + C::COL_DQ2, dq2);
+          tmem_wait_ld();
+#pragma unroll
+          for (int e = 0; e < D; ++e) dqv[e] += dq2[e];
+        }
         if (act) {
           uint32_t pk[D / 2];
 #pragma unroll
@@ -546,10 +584,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       ok = wg_sync(&bar_wg[g], ph, lane, &abort_flag);
     }
     if (!ok && !abort_flag) record_timeout(&abort_flag);
-    // MMAs this warpgroup issued are complete before TMEM is released
-    if (elected) {
-      mma_commit(&bar_drain[g]);
-      mbar_wait(&bar_drain[g], 0, kWaitNs);
+    // MMAs this warp issued are complete before TMEM is released
+    if (lane == 0) {
+      mma_commit(&bar_drain[warp]);
+      mbar_wait(&bar_drain[warp], 0, kWaitNs);
     }
     __syncwarp();
   }

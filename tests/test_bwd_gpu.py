@@ -130,6 +130,42 @@ def test_bwd_full_size(name):
     _compare(sg, want, tol, name + " two-image slice")
 
 
+def _scaled(t, f):
+    return (t.float() * f).to(t.dtype)
+
+
+@pytest.mark.parametrize("d", [16, 32])
+@pytest.mark.parametrize("stress", ["large_tables", "anti_aligned"])
+def test_bwd_tensor_core_stress(d, stress):
+    """The tensor-core backward under the forward's numerics stress cases:
+    relative tables x32 with q x4 (relative logits of hundreds of log2 units,
+    near one-hot softmax rows), and q, k anti-aligned so that every in-image
+    logit is strongly negative next to zero-filled border keys.  v and dout
+    are halved so that the gradients stay where bf16 rounding fits the bar."""
+    wl = custom("bwdstress", N=1, H=16, W=24, heads=2, dim_head=d, block=8, halo=3, stride=1, dtype="bf16")
+    h = _lib()
+    assert h.bwd_kernel_name(wl.N, wl.H, wl.W, wl.heads, wl.dim_head, wl.block, wl.halo, wl.stride, 0,
+                             wl.torch_dtype) == f"halo_bwd_tc<{d},14>"
+    q, k, v, rh, rw = make_inputs(wl, seed=41)
+    if stress == "large_tables":
+        q, rh, rw = _scaled(q, 4.0), _scaled(rh, 32.0), _scaled(rw, 32.0)
+    else:
+        g = torch.Generator().manual_seed(42)
+        u = torch.randn((wl.heads, wl.dim_head), generator=g)
+        base = (6.0 * u).reshape(1, 1, 1, wl.C)
+        q, k = (base + q.float()).to(torch.bfloat16), (-base + k.float()).to(torch.bfloat16)
+    v = _scaled(v, 0.5)
+    dout = _scaled(_dout(wl, 43), 0.5)
+    inputs = (q, k, v, rh, rw)
+    dev = [t.cuda() for t in inputs]
+    out = h.attn(*dev, block=wl.block, halo=wl.halo)
+    grads = h.attn_bwd(*dev, out, dout.cuda(), block=wl.block, halo=wl.halo)
+    torch.cuda.synchronize()
+    assert h.get_last_error() == 0
+    want = oracle.halo_attention_bwd(*inputs, dout, block=wl.block, halo=wl.halo)
+    _compare(grads, want, TOL["bf16"], f"tensor-core backward d{d} {stress}")
+
+
 def test_bwd_workspace_checks():
     h = _lib()
     from blocked_local_self_b200 import _native as n
