@@ -51,6 +51,8 @@ def _load():
         lib.halo_oracle_masked_f64.restype = ip
         lib.halo_oracle_bwd_f64.argtypes = [vp] * 6 + [dp] * 5 + [ip] * 11
         lib.halo_oracle_bwd_f64.restype = ip
+        lib.halo_oracle_fused_f64.argtypes = [vp] * 5 + [dp] + [ip] * 11
+        lib.halo_oracle_fused_f64.restype = ip
         lib.halo_oracle_max_threads.argtypes = []
         lib.halo_oracle_max_threads.restype = ip
         _lib = lib
@@ -180,3 +182,23 @@ def _prepare_n(*tensors):
     if len(codes) != 1:
         raise TypeError("all tensors must share one dtype")
     return [a for a, _ in arrs], codes.pop()
+
+
+def halo_attention_fused(x, wq, wkv, rel_h, rel_w, block: int, halo: int, heads: int, stride: int = 1,
+                         threads: int = 0) -> np.ndarray:
+    """Fused projections: q = x wq^T, [k | v] = x wkv^T per pixel (exact, each
+    rounded to the inputs' dtype), then the operation.  x: ``[N, H, W, c_in]``;
+    wq: ``[heads*d, c_in]``; wkv: ``[2*heads*d, c_in]``.  Float64
+    ``[N, H/stride, W/stride, heads*d]``."""
+    lib = _load()
+    (xa, qa, ka, rha, rwa), code = _prepare_n(x, wq, wkv, rel_h, rel_w)
+    N, H, W, c_in = xa.shape
+    d = rha.shape[1]
+    C = qa.shape[0]
+    out = np.empty((N, H // stride, W // stride, C), dtype=np.float64)
+    rc = lib.halo_oracle_fused_f64(xa.ctypes.data, qa.ctypes.data, ka.ctypes.data, rha.ctypes.data,
+                                   rwa.ctypes.data, out.ctypes.data_as(ctypes.POINTER(ctypes.c_double)),
+                                   N, H, W, c_in, heads, d, block, halo, stride, code, threads)
+    if rc != 0:
+        raise ValueError(f"oracle rejected the arguments (code {rc})")
+    return out

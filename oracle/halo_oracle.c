@@ -50,6 +50,13 @@
  * 2h + 1); a key is kept when |Y - y| <= k/2 and |X - x| <= k/2 (and it is
  * inside the image).  kmask = 0 means no mask (HaloNet's own, unmasked form).
  *
+ * Fused projections (the blog page's HaloAttention: to_q and to_kv are
+ * bias-free linear maps of the input feature map x, k and v being the two
+ * halves of to_kv's output): q = x Wq^T, [k | v] = x Wkv^T per pixel, exactly
+ * (double precision), each rounded to the inputs' dtype as an unfused
+ * pipeline would store them, then the operation above.  Pixels outside the
+ * image project to zero (no bias), the same as zero-filled keys.
+ *
  * Backward (the gradients of a scalar loss L = sum(out * dout) with respect to
  * q, k, v, rel_h and rel_w; the pages train this layer, section 2.2 and
  * Figure 3, but print no gradient): by the chain rule through the defining
@@ -79,11 +86,16 @@
 #define ORACLE_F32 0
 #define ORACLE_BF16 1
 
+#define ORACLE_F64 2  /* internal: projected values held in double */
+
 /* Read element i of a float32 or bf16 array as a double (exact widening). */
 static double read_elem(const void *base, size_t i, int dtype)
 {
     if (dtype == ORACLE_F32) {
         return (double)((const float *)base)[i];
+    }
+    if (dtype == ORACLE_F64) {
+        return ((const double *)base)[i];
     }
     uint32_t bits = ((uint32_t)((const uint16_t *)base)[i]) << 16;
     float f;
@@ -189,7 +201,7 @@ static int check_args(const oracle_args *a)
     if (a->H % a->b || a->W % a->b) return -3;
     if (a->S != 1 && a->S != 2) return -4;
     if (a->b % a->S) return -3;
-    if (a->dtype != ORACLE_F32 && a->dtype != ORACLE_BF16) return -9;
+    if (a->dtype != ORACLE_F32 && a->dtype != ORACLE_BF16 && a->dtype != ORACLE_F64) return -9;
     if (a->b + 2 * a->h > 4096) return -2;
     if (a->kmask < 0 || (a->kmask > 0 && (a->kmask % 2 == 0 || a->kmask / 2 > a->h))) return -2;
     return 0;
@@ -409,6 +421,73 @@ int halo_oracle_bwd_f64(const void *q, const void *k, const void *v,
     }
     free(part);
     return 0;
+}
+
+/* A double rounded to the stored dtype (float32, or bf16 by round to nearest
+ * even of the float32 value), returned as a double. */
+static double round_to_dtype(double x, int dtype)
+{
+    float f = (float)x;
+    if (dtype == ORACLE_F32) return (double)f;
+    uint32_t bits;
+    memcpy(&bits, &f, sizeof bits);
+    bits = (bits + 0x7FFFu + ((bits >> 16) & 1u)) & 0xFFFF0000u;
+    memcpy(&f, &bits, sizeof f);
+    return (double)f;
+}
+
+/*
+ * Fused projections: x [N, H, W, c_in] and the weights wq [heads*d, c_in],
+ * wkv [2*heads*d, c_in] (the linear layers' [out, in] layout) in `dtype`;
+ * out [N, H/S, W/S, heads*d] doubles.  q, k, v are formed exactly, rounded
+ * to `dtype`, then the operation.
+ */
+int halo_oracle_fused_f64(const void *x, const void *wq, const void *wkv,
+                          const void *rel_h, const void *rel_w, double *out,
+                          int N, int H, int W, int c_in, int heads, int dim_head,
+                          int block, int halo, int stride, int dtype, int threads)
+{
+    if (!x || !wq || !wkv || !rel_h || !rel_w || !out) return -1;
+    if (c_in <= 0) return -2;
+    if (dtype != ORACLE_F32 && dtype != ORACLE_BF16) return -9;
+    const int C = heads * dim_head;
+    const size_t npix = (size_t)N * H * W;
+    double *q = (double *)malloc(npix * C * sizeof(double));
+    double *k = (double *)malloc(npix * C * sizeof(double));
+    double *v = (double *)malloc(npix * C * sizeof(double));
+    double *rh = (double *)malloc((size_t)(2 * (block + 2 * halo) - 1) * dim_head * sizeof(double));
+    double *rw = (double *)malloc((size_t)(2 * (block + 2 * halo) - 1) * dim_head * sizeof(double));
+    if (!q || !k || !v || !rh || !rw) {
+        free(q); free(k); free(v); free(rh); free(rw);
+        return -2;
+    }
+#ifdef _OPENMP
+    if (threads > 0) omp_set_num_threads(threads);
+#endif
+#pragma omp parallel for schedule(static)
+    for (long pix = 0; pix < (long)npix; ++pix) {
+        for (int o = 0; o < C; ++o) {
+            double aq = 0.0, ak = 0.0, av = 0.0;
+            for (int ci = 0; ci < c_in; ++ci) {
+                const double xe = read_elem(x, (size_t)pix * c_in + ci, dtype);
+                aq += xe * read_elem(wq, (size_t)o * c_in + ci, dtype);
+                ak += xe * read_elem(wkv, (size_t)o * c_in + ci, dtype);
+                av += xe * read_elem(wkv, (size_t)(C + o) * c_in + ci, dtype);
+            }
+            q[(size_t)pix * C + o] = round_to_dtype(aq, dtype);
+            k[(size_t)pix * C + o] = round_to_dtype(ak, dtype);
+            v[(size_t)pix * C + o] = round_to_dtype(av, dtype);
+        }
+    }
+    const size_t ntab = (size_t)(2 * (block + 2 * halo) - 1) * dim_head;
+    for (size_t i = 0; i < ntab; ++i) {
+        rh[i] = read_elem(rel_h, i, dtype);
+        rw[i] = read_elem(rel_w, i, dtype);
+    }
+    oracle_args a = {q, k, v, rh, rw, N, H, W, heads, dim_head, block, halo, stride, ORACLE_F64, 0};
+    const int rc = full_output(&a, out, threads);
+    free(q); free(k); free(v); free(rh); free(rw);
+    return rc;
 }
 
 /*
