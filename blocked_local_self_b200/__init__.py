@@ -96,6 +96,32 @@ def attn_masked(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, rel_h: torch.
     return out
 
 
+def attn_fused(x: torch.Tensor, wq: torch.Tensor, wkv: torch.Tensor, rel_h: torch.Tensor, rel_w: torch.Tensor,
+               heads: int, block: int, halo: int, stride: int = 1, out: torch.Tensor | None = None,
+               stream=None) -> torch.Tensor:
+    """The operation with the q, k, v projections inside the kernel
+    (``halo_attn_fused``): ``x`` is the NHWC input map [N, H, W, c_in], ``wq``
+    [heads*d, c_in] and ``wkv`` [2*heads*d, c_in] are bias-free linear layers'
+    weights ([out, in]; key rows, then value rows)."""
+    for t in (x, wq, wkv, rel_h, rel_w):
+        if not t.is_cuda or not t.is_contiguous():
+            raise ValueError("attn_fused expects contiguous CUDA tensors")
+    if x.dim() != 4 or wq.dim() != 2 or wkv.dim() != 2:
+        raise ValueError("x must be [N, H, W, c_in], wq [heads*d, c_in], wkv [2*heads*d, c_in]")
+    N, H, W, c_in = x.shape
+    d = rel_h.shape[-1]
+    if wq.shape != (heads * d, c_in) or wkv.shape != (2 * heads * d, c_in):
+        raise ValueError("weight shapes do not match heads, dim_head and c_in")
+    if out is None:
+        out = torch.empty((N, H // stride, W // stride, heads * d), dtype=x.dtype, device=x.device)
+    rc = _native.lib().halo_attn_fused(x.data_ptr(), wq.data_ptr(), wkv.data_ptr(), rel_h.data_ptr(),
+                                       rel_w.data_ptr(), out.data_ptr(), N, H, W, c_in, heads, d, block, halo,
+                                       stride, _dtype_code(x), _stream_ptr(stream))
+    if rc != 0:
+        raise HaloError(rc, "halo_attn_fused")
+    return out
+
+
 def bwd_workspace_size(N: int, H: int, W: int, heads: int, dim_head: int, block: int, halo: int, stride: int,
                        kernel: int, dtype: torch.dtype) -> int:
     """Bytes of device workspace ``attn_bwd`` needs (``halo_attn_bwd_workspace_size``)."""
@@ -176,6 +202,14 @@ def masked_kernel_name(N: int, H: int, W: int, heads: int, dim_head: int, block:
     code = HALO_BF16 if dtype == torch.bfloat16 else HALO_F32
     return _native.lib().halo_masked_kernel_name(N, H, W, heads, dim_head, block, halo, stride, kernel,
                                                  code).decode()
+
+
+def fused_kernel_name(N: int, H: int, W: int, c_in: int, heads: int, dim_head: int, block: int, halo: int,
+                      stride: int, dtype: torch.dtype) -> str:
+    """Kernel ``attn_fused`` launches for a shape, or "none"."""
+    code = HALO_BF16 if dtype == torch.bfloat16 else HALO_F32
+    return _native.lib().halo_fused_kernel_name(N, H, W, c_in, heads, dim_head, block, halo, stride,
+                                                code).decode()
 
 
 def bwd_kernel_name(N: int, H: int, W: int, heads: int, dim_head: int, block: int, halo: int, stride: int,

@@ -43,12 +43,14 @@ SIGNATURES = {
     "halo_attn": (_i, [_vp] * 6 + [_i] * 9 + [_vp]),
     "halo_attn_host": (_i, [_vp] * 12 + [_i] * 9 + [_vp]),
     "halo_attn_masked": (_i, [_vp] * 6 + [_i] * 10 + [_vp]),
+    "halo_attn_fused": (_i, [_vp] * 6 + [_i] * 10 + [_vp]),
     "halo_attn_bwd": (_i, [_vp] * 13 + [ctypes.c_size_t] + [_i] * 10 + [_vp]),
     "halo_attn_bwd_workspace_size": (_i, [_i] * 10 + [ctypes.POINTER(ctypes.c_size_t)]),
     "halo_attn_bwd_noalloc": (_i, [_vp] * 12 + [_i] * 10 + [_vp]),
     "halo_kernel_for": (_i, [_i] * 9),
     "halo_kernel_name": (ctypes.c_char_p, [_i] * 9),
     "halo_masked_kernel_name": (ctypes.c_char_p, [_i] * 10),
+    "halo_fused_kernel_name": (ctypes.c_char_p, [_i] * 10),
     "halo_bwd_kernel_name": (ctypes.c_char_p, [_i] * 10),
     "halo_strerror": (ctypes.c_char_p, [_i]),
     "halo_get_last_error": (_i, []),

@@ -14,7 +14,7 @@ ROOT = os.path.dirname(HERE)
 CSRC = os.path.join(HERE, "csrc")
 LIB = os.path.join(HERE, "libhalo.so")
 SOURCES = [os.path.join(CSRC, "halo_api.cu")]
-DEPS = SOURCES + [os.path.join(CSRC, f) for f in ("halo_tc.cuh", "halo_tc2.cuh", "halo_tc3.cuh", "halo_tc4.cuh", "halo_simt.cuh", "halo_bwd.cuh", "halo_bwd_tc.cuh", "halo_win.cuh", "sm100.cuh")] + [
+DEPS = SOURCES + [os.path.join(CSRC, f) for f in ("halo_tc.cuh", "halo_tc2.cuh", "halo_tc3.cuh", "halo_tc4.cuh", "halo_simt.cuh", "halo_bwd.cuh", "halo_bwd_tc.cuh", "halo_win.cuh", "halo_fused.cuh", "sm100.cuh")] + [
     os.path.join(ROOT, "include", "halo.h")]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 FLAGS = ["-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC", "-shared", "-cudart", "static",
@@ -50,7 +50,7 @@ def build(force: bool = False, verbose: bool = False) -> str:
     checked = 0
     for m in re.finditer(r"Compiling entry function '(\w+)'(.*?)Used (\d+) registers", log, re.S):
         name, spill, regs = m.group(1), m.group(2), int(m.group(3))
-        if "halo_fwd_tc" in name:  # the forward tensor-core kernels (setmaxnreg split)
+        if "halo_fwd_tc" in name or "halo_fused_tc" in name:  # the forward tensor-core kernels (setmaxnreg split)
             sp = re.search(r"(\d+) bytes spill stores", spill)
             if sp and int(sp.group(1)) > 32:
                 raise RuntimeError(f"{name} spills registers: {spill.strip()}")

@@ -14,6 +14,7 @@
 #include "../../include/halo.h"
 #include "halo_bwd.cuh"
 #include "halo_bwd_tc.cuh"
+#include "halo_fused.cuh"
 #include "halo_simt.cuh"
 #include "halo_tc.cuh"
 #include "halo_tc2.cuh"
@@ -511,6 +512,129 @@ int attn_device(const void* q, const void* k, const void* v, const void* rel_h, 
 }
 
 // ----------------------------------------------------------------------------
+// Forward with the q, k, v projections inside the kernel (halo_attn_fused)
+// ----------------------------------------------------------------------------
+using FusedKernel = void (*)(const CUtensorMap, const CUtensorMap, const CUtensorMap, const CUtensorMap,
+                             const halo::fused::Params);
+struct FusedEntry {
+  int d, win, cin;
+  FusedKernel fn;
+  int (*smem)(int);
+};
+template <int D, int WIN, int CIN>
+int fused_smem(int xstages) { return halo::fused::smem_bytes<D, WIN, CIN>(xstages); }
+#define HALO_FUSED_ENTRY(D, WIN, CIN) \
+  FusedEntry { D, WIN, CIN, halo::fused::halo_fused_tc<D, WIN, CIN>, fused_smem<D, WIN, CIN> }
+#define HALO_FUSED_WINS(D, CIN)                                                                       \
+  HALO_FUSED_ENTRY(D, 8, CIN), HALO_FUSED_ENTRY(D, 10, CIN), HALO_FUSED_ENTRY(D, 12, CIN),            \
+      HALO_FUSED_ENTRY(D, 14, CIN)
+// (d = 32, c_in = 128 needs more shared memory than a CTA has: the x tiles
+// alone are 128 KB next to 144 KB of per-warpgroup tiles and weights)
+const FusedEntry kFusedTable[] = {HALO_FUSED_WINS(16, 64), HALO_FUSED_WINS(16, 128), HALO_FUSED_WINS(32, 64)};
+
+const FusedEntry* find_fused(const Shape& s, int c_in) {
+  if (s.dtype != HALO_BF16 || s.block != halo::fused::kBlock || s.stride != 1 || (s.H / s.block) % 2)
+    return nullptr;
+  const int win = s.block + 2 * s.halo;
+  for (const FusedEntry& e : kFusedTable)
+    if (e.d == s.d && e.win == win && e.cin == c_in) return &e;
+  return nullptr;
+}
+
+// 4-D map over the NHWC bf16 input map {c_in, W, H, N}; box {64, bw, bh, 1}
+// (64 channels = one 128-byte swizzle atom per row).
+bool encode_x(CUtensorMap* m, const void* base, const Shape& s, int c_in, int bw, int bh) {
+  EncodeTiledFn enc = encoder();
+  if (!enc) return false;
+  const cuuint64_t C = static_cast<cuuint64_t>(c_in);
+  cuuint64_t dims[4] = {C, static_cast<cuuint64_t>(s.W), static_cast<cuuint64_t>(s.H),
+                        static_cast<cuuint64_t>(s.N)};
+  cuuint64_t strides[3] = {C * 2, C * 2 * s.W, C * 2 * s.W * s.H};
+  cuuint32_t box[4] = {64, static_cast<cuuint32_t>(bw), static_cast<cuuint32_t>(bh), 1};
+  cuuint32_t es[4] = {1, 1, 1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, strides, box, es,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// 2-D map over a [rows, c_in] bf16 weight matrix; box {64, d}.
+bool encode_w(CUtensorMap* m, const void* base, int rows, int c_in, int d) {
+  EncodeTiledFn enc = encoder();
+  if (!enc) return false;
+  cuuint64_t dims[2] = {static_cast<cuuint64_t>(c_in), static_cast<cuuint64_t>(rows)};
+  cuuint64_t strides[1] = {static_cast<cuuint64_t>(c_in) * 2};
+  cuuint32_t box[2] = {64, static_cast<cuuint32_t>(d)};
+  cuuint32_t es[2] = {1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, es,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+int attn_fused_device(const void* x, const void* wq, const void* wkv, const void* rel_h, const void* rel_w, void* out,
+                      const Shape& s, int c_in, cudaStream_t st) {
+  int rc = check_shape(s);
+  if (rc != HALO_OK) return rc;
+  if (c_in <= 0 || c_in > (1 << 16)) return HALO_ERR_DIMS;
+  if (!x || !wq || !wkv || !rel_h || !rel_w || !out) return HALO_ERR_NULL;
+  const void* ptrs[6] = {x, wq, wkv, rel_h, rel_w, out};
+  for (const void* ptr : ptrs)
+    if (reinterpret_cast<uintptr_t>(ptr) % 16) return HALO_ERR_ALIGN;
+  if ((static_cast<long long>(c_in) * s.elem()) % 16) return HALO_ERR_ALIGN;
+  const size_t xb = static_cast<size_t>(s.N) * s.H * s.W * c_in * s.elem();
+  const size_t wb = static_cast<size_t>(s.heads) * s.d * c_in * s.elem();
+  const size_t ob = s.out_bytes(), rb = s.rel_bytes();
+  if (overlaps(out, ob, x, xb) || overlaps(out, ob, wq, wb) || overlaps(out, ob, wkv, 2 * wb) ||
+      overlaps(out, ob, rel_h, rb) || overlaps(out, ob, rel_w, rb))
+    return HALO_ERR_ALIAS;
+  const FusedEntry* e = find_fused(s, c_in);
+  if (!e) return HALO_ERR_UNSUPPORTED;
+  int sm_count = 0;
+  rc = device_info(&sm_count);
+  if (rc != HALO_OK) return rc;
+  const int win = s.block + 2 * s.halo;
+  CUtensorMap mxq, mxkv, mwq, mwkv;
+  if (!encode_x(&mxq, x, s, c_in, halo::fused::kBlock, 2 * halo::fused::kBlock) ||
+      !encode_x(&mxkv, x, s, c_in, win, win + halo::fused::kBlock) ||
+      !encode_w(&mwq, wq, s.heads * s.d, c_in, s.d) || !encode_w(&mwkv, wkv, 2 * s.heads * s.d, c_in, s.d))
+    return HALO_ERR_CUDA;
+  cudaFuncAttributes attr;
+  if (cudaFuncGetAttributes(&attr, reinterpret_cast<const void*>(e->fn)) != cudaSuccess) return HALO_ERR_CUDA;
+  // the setmaxnreg split must fit the launch's registers (see launch_persistent)
+  if (256 * halo::fused::kSoftmaxRegs + 128 * halo::fused::kProducerRegs > halo::fused::kThreads * attr.numRegs)
+    return HALO_ERR_UNSUPPORTED;
+  int optin = 0, dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) != cudaSuccess)
+    return HALO_ERR_CUDA;
+  const int budget = (optin < kMaxDynSmem ? optin : kMaxDynSmem) - static_cast<int>(attr.sharedSizeBytes);
+  const int xstages = e->smem(2) <= budget ? 2 : 1;
+  const int smem = e->smem(xstages);
+  if (smem > budget) return HALO_ERR_UNSUPPORTED;
+  if (cudaFuncSetAttribute(reinterpret_cast<const void*>(e->fn), cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           smem) != cudaSuccess)
+    return HALO_ERR_CUDA;
+  halo::fused::Params p;
+  p.rel_h = static_cast<const __nv_bfloat16*>(rel_h);
+  p.rel_w = static_cast<const __nv_bfloat16*>(rel_w);
+  p.out = static_cast<__nv_bfloat16*>(out);
+  p.N = s.N;
+  p.H = s.H;
+  p.W = s.W;
+  p.heads = s.heads;
+  p.halo = s.halo;
+  p.nbx = s.W / halo::fused::kBlock;
+  p.npy = s.H / (2 * halo::fused::kBlock);
+  const long long pairs = static_cast<long long>(s.N) * p.nbx * p.npy;
+  if (pairs * s.heads > 0x7fffffffLL) return HALO_ERR_DIMS;
+  p.num_pairs = static_cast<int>(pairs);
+  p.xstages = xstages;
+  p.c = 1.4426950408889634f / std::sqrt(static_cast<float>(s.d));
+  const int grid = static_cast<int>(pairs < sm_count ? pairs : sm_count);
+  e->fn<<<grid, halo::fused::kThreads, smem, st>>>(mxq, mxkv, mwq, mwkv, p);
+  return cudaGetLastError() == cudaSuccess ? HALO_OK : HALO_ERR_CUDA;
+}
+
+// ----------------------------------------------------------------------------
 // Backward
 // ----------------------------------------------------------------------------
 struct BwdPlan {
@@ -914,6 +1038,23 @@ int halo_attn_host(const void* q_h, const void* k_h, const void* v_h, const void
       cudaStreamWaitEvent(st, hp->ev_done[1], 0) != cudaSuccess)
     return fail(HALO_ERR_CUDA);
   return HALO_OK;
+}
+
+int halo_attn_fused(const void* x, const void* wq, const void* wkv, const void* rel_h, const void* rel_w, void* out,
+                    int N, int H, int W, int c_in, int heads, int dim_head, int block, int halo, int stride, int dtype,
+                    void* stream) {
+  const Shape s{N, H, W, heads, dim_head, block, halo, stride, dtype};
+  return attn_fused_device(x, wq, wkv, rel_h, rel_w, out, s, c_in, static_cast<cudaStream_t>(stream));
+}
+
+const char* halo_fused_kernel_name(int N, int H, int W, int c_in, int heads, int dim_head, int block, int halo,
+                                   int stride, int dtype) {
+  thread_local char name[64];
+  const Shape s{N, H, W, heads, dim_head, block, halo, stride, dtype};
+  const FusedEntry* e = (check_shape(s) == HALO_OK) ? find_fused(s, c_in) : nullptr;
+  if (e) std::snprintf(name, sizeof(name), "halo_fused_tc<%d,%d,%d>", e->d, e->win, e->cin);
+  else std::snprintf(name, sizeof(name), "none");
+  return name;
 }
 
 int halo_attn_masked(const void* q, const void* k, const void* v, const void* rel_h, const void* rel_w, void* out,

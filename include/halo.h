@@ -131,6 +131,34 @@ int halo_attn_masked(const void* q, const void* k, const void* v, const void* re
                      int dtype, void* stream);
 
 /*
+ * halo_attn_fused -- the same operation with the q, k, v projections done
+ * inside the kernel (the blog page's HaloAttention module: q = x Wq^T and
+ * [k | v] = x Wkv^T, bias-free linear maps of the input map x; HaloNet
+ * appendix D: its speed-ups came from fusing around the attention op and
+ * avoiding format changes).  x is read from HBM instead of stored q, k, v.
+ *   x     : [N, H, W, c_in]        NHWC input map
+ *   wq    : [heads*dim_head, c_in] query weights (a linear layer's [out, in])
+ *   wkv   : [2*heads*dim_head, c_in] key rows first, then value rows
+ *   rel_h, rel_w, out : as in halo_attn (out [N, H, W, heads*dim_head])
+ * Every projection is accumulated in float32 and rounded to bf16 before the
+ * attention, as a pipeline that stored q, k and v in bf16 would.  Supported:
+ * bf16, block 8, stride 1, H/8 even, window 8..14 (halo 0..3), and
+ * (dim_head, c_in) = (16, 64), (16, 128) or (32, 64); other shapes return
+ * HALO_ERR_UNSUPPORTED (project with a GEMM and call halo_attn instead).
+ * Pointers 16-byte aligned (HALO_ERR_ALIGN); out may not overlap an input
+ * (HALO_ERR_ALIAS).  Asynchronous on `stream`; allocates nothing.
+ */
+int halo_attn_fused(const void* x, const void* wq, const void* wkv, const void* rel_h, const void* rel_w, void* out,
+                    int N, int H, int W, int c_in, int heads, int dim_head, int block, int halo, int stride, int dtype,
+                    void* stream);
+
+/* Name of the kernel halo_attn_fused launches for this shape (e.g.
+ * "halo_fused_tc<16,14,128>"), or "none" when it returns HALO_ERR_UNSUPPORTED
+ * or rejects the shape.  Thread-local storage; never NULL. */
+const char* halo_fused_kernel_name(int N, int H, int W, int c_in, int heads, int dim_head, int block, int halo,
+                                   int stride, int dtype);
+
+/*
  * halo_attn_bwd -- gradients of a loss L with respect to q, k, v, rel_h and
  * rel_w, given dout = dL/dout (the pages train this layer, section 2.2 and
  * Figure 3; the gradient is the chain rule through the operation above):

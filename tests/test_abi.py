@@ -123,6 +123,41 @@ def test_kernel_names():
     assert name(1, 16, 16, 2, 32, 5, 1, 1, 0) == "none"
 
 
+def test_fused_kernel_selection():
+    lib = _lib()
+    name = lambda *a: lib.halo_fused_kernel_name(*a).decode()
+    # (N, H, W, c_in, heads, d, block, halo, stride, dtype)
+    assert name(32, 64, 64, 128, 8, 16, 8, 3, 1, 1) == "halo_fused_tc<16,14,128>"
+    assert name(2, 16, 16, 64, 2, 16, 8, 2, 1, 1) == "halo_fused_tc<16,12,64>"
+    assert name(2, 32, 32, 64, 4, 32, 8, 0, 1, 1) == "halo_fused_tc<32,8,64>"
+    assert name(2, 32, 32, 128, 4, 32, 8, 3, 1, 1) == "none"   # d 32 with c_in 128: no room in shared memory
+    assert name(2, 24, 32, 128, 8, 16, 8, 3, 1, 1) == "none"   # odd number of block rows
+    assert name(2, 32, 32, 96, 8, 16, 8, 3, 1, 1) == "none"    # c_in 96
+    assert name(2, 32, 32, 128, 8, 16, 8, 3, 2, 1) == "none"   # stride 2
+    assert name(2, 32, 32, 128, 8, 16, 8, 3, 1, 0) == "none"   # float32
+    assert name(2, 32, 32, 128, 8, 16, 16, 3, 1, 1) == "none"  # block 16
+
+
+def _fused(ptrs=(16,) * 6, **over):
+    a = dict(dict(ARGS, c_in=128), **over)
+    return _lib().halo_attn_fused(*ptrs, a["N"], a["H"], a["W"], a["c_in"], a["heads"], a["d"], a["block"],
+                                  a["halo"], a["stride"], a["dtype"], None)
+
+
+def test_fused_entry_checks_on_the_host():
+    assert _fused(N=0) == -2
+    assert _fused(c_in=0) == -2
+    assert _fused(H=12) == -3
+    assert _fused(ptrs=(16, 0, 16, 16, 16, 16)) == -1
+    assert _fused(ptrs=(16, 24, 16, 16, 16, 4096)) == -5
+    assert _fused(c_in=4) == -5                     # x rows of 8 bytes
+    # out overlapping the weights
+    assert _fused(ptrs=(1 << 20, 1 << 22, 1 << 23, 1 << 24, 1 << 25, (1 << 22) + 256)) == -10
+    # valid arguments, shape without a fused kernel: refused before any device call
+    assert _fused(ptrs=(1 << 20, 1 << 22, 1 << 23, 1 << 24, 1 << 25, 1 << 26), c_in=96) == -6
+    assert _fused(ptrs=(1 << 20, 1 << 22, 1 << 23, 1 << 24, 1 << 25, 1 << 26), stride=2) == -6
+
+
 def test_host_entry_checks_before_any_copy():
     lib = _lib()
     a = ARGS

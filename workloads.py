@@ -162,6 +162,34 @@ def make_inputs(wl: Workload, seed: int | None = None):
     return tuple(t.to(dt).contiguous() for t in (q, k, v, rel_h, rel_w))
 
 
+# The fused-projection form (the blog page's HaloAttention: to_q and to_kv are
+# bias-free linear layers of the layer's input map x) on the stage-1 layer,
+# with c_in = heads * dim_head = 128 input channels.
+FUSED_WORKLOADS: dict[str, tuple[Workload, int]] = {
+    "stage1_fused_bf16": (WORKLOADS["stage1_bf16"], 128),
+}
+
+
+def make_fused_inputs(wl: Workload, c_in: int, seed: int | None = None):
+    """Draw (x, wq, wkv, rel_h, rel_w) on the CPU for the fused form.
+
+    One CPU generator seeded with ``seed`` (default the workload's); ``randn``
+    in float32 in the order x [N, H, W, c_in], wq [heads*d, c_in],
+    wkv [2*heads*d, c_in] (key rows, then value rows), rel_h, rel_w; the
+    weights are scaled by ``c_in ** -0.5`` (so q, k, v have unit variance),
+    the tables by ``dim_head ** -0.5``; then everything is cast to the
+    workload dtype."""
+    g = torch.Generator(device="cpu")
+    g.manual_seed(wl.seed if seed is None else seed)
+    x = torch.randn((wl.N, wl.H, wl.W, c_in), generator=g, dtype=torch.float32)
+    wq = torch.randn((wl.C, c_in), generator=g, dtype=torch.float32) * c_in ** -0.5
+    wkv = torch.randn((2 * wl.C, c_in), generator=g, dtype=torch.float32) * c_in ** -0.5
+    rel_h = torch.randn((wl.rel_rows, wl.dim_head), generator=g, dtype=torch.float32) * wl.dim_head ** -0.5
+    rel_w = torch.randn((wl.rel_rows, wl.dim_head), generator=g, dtype=torch.float32) * wl.dim_head ** -0.5
+    dt = wl.torch_dtype
+    return tuple(t.to(dt).contiguous() for t in (x, wq, wkv, rel_h, rel_w))
+
+
 def custom(name: str = "custom", **kw) -> Workload:
     """A workload with explicit sizes (used by the parity and edge-case tests)."""
     base = dict(N=1, H=16, W=16, heads=2, dim_head=16, block=4, halo=1, stride=1, dtype="bf16")
