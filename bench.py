@@ -500,8 +500,9 @@ def bwd_flops(wl) -> float:
 def time_extra(halo, stream, sampler, peaks, seconds=0.5):
     """The NEXT rows measured in the same run: the backward on the stage-1 and
     stride-2 workloads, and the SASA-masked forward (7 x 7 centred window,
-    the paper's comparison) on the stage-1 workload.  Inputs rotate over sets
-    larger than L2 as for the forward."""
+    the paper's comparison) and the fused-projection form on the stage-1
+    workload, and the block-32 workloads.  Inputs rotate over sets larger than
+    L2 as for the forward."""
     res = {}
     for name in ("stage1_bf16", "stride2_bf16"):
         wl = workloads.WORKLOADS[name]
@@ -590,9 +591,88 @@ def time_extra(halo, stream, sampler, peaks, seconds=0.5):
     res["sasa_k7_stage1_bf16"] = entry
     b.release()
     torch.cuda.empty_cache()
+    res.update(time_fused(halo, stream, peaks, seconds))
     # block 32: global attention on a 32x32 map, and block 32 with halo 3
     for name, wl in workloads.NEXT_WORKLOADS.items():
         res[name] = time_forward(halo, wl, stream, peaks, seconds)
+    return res
+
+
+def fused_bytes(wl, c_in) -> float:
+    """Unavoidable HBM traffic of the fused form: x read once, out written
+    once (the weights and tables are a few KB)."""
+    return float(wl.N * wl.H * wl.W * c_in * wl.elem_bytes + wl.out_pixels * wl.C * wl.elem_bytes)
+
+
+def fused_flops(wl, c_in) -> float:
+    """Algorithmic FLOPs of the fused form: the three projections (2 c_in
+    FLOPs per output channel of q, k and v at every pixel) plus the
+    operation's q.k and p.v."""
+    return 2.0 * c_in * 3 * wl.C * wl.N * wl.H * wl.W + wl.flops()
+
+
+def time_fused(halo, stream, peaks, seconds=0.5):
+    """The fused-projection form on the stage-1 layer (c_in = 128), and, for
+    context, the same result computed unfused: three cuBLAS projections into
+    bf16 q, k, v, then ``halo_attn``.  Graph-replayed, inputs rotating over
+    sets larger than L2."""
+    res = {}
+    for name, (wl, c_in) in workloads.FUSED_WORKLOADS.items():
+        inputs_cpu = workloads.make_fused_inputs(wl, c_in)
+        b = DeviceBench(halo, wl, inputs_cpu, stream)
+
+        def fstep(i, b=b, wl=wl):
+            x, wq, wkv, rh, rw = b.sets[i % b.n_sets]
+            halo.attn_fused(x, wq, wkv, rh, rw, heads=wl.heads, block=wl.block, halo=wl.halo,
+                            out=b.outs[i % b.n_sets], stream=stream)
+
+        b.step = fstep
+        b.warmup(10)
+        b.prepare(20)
+        est = b.region() / 20
+        steps = max(20, int(seconds * 1e3 / max(est, 1e-3)))
+        b.prepare(steps)
+        t0 = time.time()
+        ms = statistics.median([b.region() / steps for _ in range(3)])
+        t1 = time.time()
+        # unfused, for context: q, k, v projected by cuBLAS, then halo_attn
+        shape = (wl.N, wl.H, wl.W, wl.C)
+        q, k, v = (torch.empty(shape, dtype=wl.torch_dtype, device="cuda") for _ in range(3))
+
+        def ustep(i, b=b, wl=wl):
+            x, wq, wkv, rh, rw = b.sets[i % b.n_sets]
+            torch.matmul(x, wq.t(), out=q)
+            torch.matmul(x, wkv[:wl.C].t(), out=k)
+            torch.matmul(x, wkv[wl.C:].t(), out=v)
+            halo.attn(q, k, v, rh, rw, block=wl.block, halo=wl.halo, out=b.outs[i % b.n_sets], stream=stream)
+
+        b.step = ustep
+        b.warmup(5)
+        b.prepare(steps)
+        ums = statistics.median([b.region() / steps for _ in range(3)])
+        torch.cuda.synchronize()
+        err = halo.get_last_error()
+        if err != 0:
+            raise RuntimeError(f"device error flag {err} after timing {name}")
+        launch_s = ms * 1e-3
+        gbs = fused_bytes(wl, c_in) / launch_s * 1e-9
+        tf = fused_flops(wl, c_in) / launch_s * 1e-12
+        kname = halo.fused_kernel_name(wl.N, wl.H, wl.W, c_in, wl.heads, wl.dim_head, wl.block, wl.halo,
+                                       wl.stride, wl.torch_dtype)
+        res["fused_" + wl.name] = {
+            "what": f"halo_attn_fused: q, k, v projected from x (c_in {c_in}) inside the kernel, then the "
+                    "operation, on the stage-1 layer",
+            "kernel": kname, "ms": ms, "value": wl.out_pixels / launch_s, "unit": "pixels/s",
+            "timing": f"median of 3 regions of {steps} graph-replayed launches, inputs rotating over "
+                      f"{b.n_sets} sets > L2",
+            "achieved_gbs": gbs, "hbm_frac": gbs / peaks["hbm_gbs"], "algorithmic_bytes": fused_bytes(wl, c_in),
+            "tflops": tf, "tensor_frac": tf / peaks["bf16_tflops"], "flops": fused_flops(wl, c_in),
+            "unfused_ms": ums,
+            "unfused": "three cuBLAS projections (torch.matmul into bf16 q, k, v) + halo_attn, graph-replayed",
+            "clocks": (t0, t1)}
+        b.release()
+        del q, k, v
+        torch.cuda.empty_cache()
     return res
 
 

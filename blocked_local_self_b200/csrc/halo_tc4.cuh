@@ -122,6 +122,12 @@ struct Cfg {
   // product with P is the row sum of the bf16 P the MMA consumed
   static constexpr int ON = D + 8;
   static constexpr int O_N = 2 * ON;                      // O_0 | O_1, each in both lane halves
+  // Where the columns allow (d = 16), O goes to the relative-logit columns,
+  // which the softmax has consumed before the A.V: the S MMA of the slot's
+  // next item then waits only for this item's A.V to finish reading P, not
+  // for the epilogue to read O (only the next G waits for that).
+  static constexpr bool O_IN_G = (int)kGBase + O_N <= (int)kSlotCols;
+  static constexpr int O_COL = O_IN_G ? (int)kGBase : O_BASE;
   static constexpr int ONES_BYTES = (KP * ROWB + 1023) / 1024 * 1024;  // ones rows, V's row pitch
   static constexpr SmemSwizzle SW = (ROWB == 32) ? SW_32B : (ROWB == 64 ? SW_64B : SW_128B);
   static constexpr uint32_t SBO = 8 * ROWB;
@@ -419,7 +425,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int t = 0; t <= my_items; ++t) {
         if (t < my_items) {
           const int s = t % S;
-          if (t >= S && !mbar_wait(&bar_eqk[s], ((t / S) - 1) & 1, kWaitNs, &abort_flag)) {
+          if (t >= S && !mbar_wait_idle(&bar_eqk[s], ((t / S) - 1) & 1, kWaitNs, &abort_flag)) {
             if (!abort_flag) record_timeout(&abort_flag);
             break;
           }
@@ -434,7 +440,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         if (t >= 1) {
           const int k = t - 1, s = k % S;
-          if (k >= S && !mbar_wait(&bar_ev[s], ((k / S) - 1) & 1, kWaitNs, &abort_flag)) {
+          if (k >= S && !mbar_wait_idle(&bar_ev[s], ((k / S) - 1) & 1, kWaitNs, &abort_flag)) {
             if (!abort_flag) record_timeout(&abort_flag);
             break;
           }
@@ -461,8 +467,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint32_t ra = smem_addr(sR);
       for (int k = 0; k < my_items; ++k) {
         const int s = k % S, g = k & 1;
-        if (!mbar_wait(&bar_fqk[s], (k / S) & 1, kWaitNs, &abort_flag) ||
-            (k >= 2 && !mbar_wait(&bar_tfree[g], ((k >> 1) - 1) & 1, kWaitNs, &abort_flag))) {
+        // the slot is free for S once the A.V of item k - 2 has read its P
+        // (O elsewhere) or once its epilogue has read O; for G, always the latter
+        uint64_t* slot_free = (C::O_IN_G && !is_g) ? &bar_ofull[g] : &bar_tfree[g];
+        if (!mbar_wait_idle(&bar_fqk[s], (k / S) & 1, kWaitNs, &abort_flag) ||
+            (k >= 2 && !mbar_wait_idle(slot_free, ((k >> 1) - 1) & 1, kWaitNs, &abort_flag))) {
           if (!abort_flag) record_timeout(&abort_flag);
           break;
         }
@@ -626,7 +635,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t lbo = smem_addr(sOnes) - va;
 #pragma unroll 1
         for (int kk = kb; kk < ke; ++kk)
-          mma_f16_ts(slot + lanes + C::O_BASE + hf * C::ON, slot + lanes + 8 * kk,
+          mma_f16_ts(slot + lanes + C::O_COL + hf * C::ON, slot + lanes + 8 * kk,
                      smem_desc(va + kk * 16 * C::ROWB, lbo, C::SBO, C::SW), idO, kk != kb);
         mma_commit(&bar_ofull[g]);
         mma_commit(&bar_ev[s]);
@@ -642,20 +651,20 @@ __global__ void __launch_bounds__(kThreads, 1)
       {
         // this thread's row of both key halves' accumulators
         float o[D], la, lb;
-        tmem_ld_x1(ts + C::O_BASE + D, &la);
-        tmem_ld_x1(ts + C::O_BASE + C::ON + D, &lb);
+        tmem_ld_x1(ts + C::O_COL + D, &la);
+        tmem_ld_x1(ts + C::O_COL + C::ON + D, &lb);
         constexpr int kSeg = (D % 32 == 0) ? 32 : 16;  // columns per load
 #pragma unroll
         for (int e = 0; e < D; e += kSeg) {
           float ta[kSeg], tb[kSeg];
           if constexpr (kSeg == 32) {
-            tmem_ld_x32(ts + C::O_BASE + e, ta);
-            tmem_ld_x32(ts + C::O_BASE + C::ON + e, tb);
+            tmem_ld_x32(ts + C::O_COL + e, ta);
+            tmem_ld_x32(ts + C::O_COL + C::ON + e, tb);
           } else {
-            tmem_ld_x8(ts + C::O_BASE + e, ta);
-            tmem_ld_x8(ts + C::O_BASE + e + 8, ta + 8);
-            tmem_ld_x8(ts + C::O_BASE + C::ON + e, tb);
-            tmem_ld_x8(ts + C::O_BASE + C::ON + e + 8, tb + 8);
+            tmem_ld_x8(ts + C::O_COL + e, ta);
+            tmem_ld_x8(ts + C::O_COL + e + 8, ta + 8);
+            tmem_ld_x8(ts + C::O_COL + C::ON + e, tb);
+            tmem_ld_x8(ts + C::O_COL + C::ON + e + 8, tb + 8);
           }
           tmem_wait_ld();
 #pragma unroll
