@@ -182,23 +182,13 @@ __device__ __forceinline__ void exp2_poly2(float2 x, uint32_t& rx, uint32_t& ry)
   ry = __float_as_uint(q.y) + (__float_as_uint(t.y) << 23);
 }
 
-// bf16x2 of two non-negative floats given as bit patterns (the P operand of
-// the A.V MMA), rounded to nearest.  With HALO_PACK_P_ALU the rounding is
-// integer arithmetic: half a bf16 ulp (0x8000) is added to each pattern and
-// a byte permute keeps the two upper halves (ties round away from zero
-// instead of to even; p <= 1, so the add cannot carry into an infinity).
-// That keeps the conversion off the XU pipe, which the exponentials
-// already saturate; the add folds into the exponent add of the polynomial
-// path.  Otherwise cvt.rn.bf16x2.f32 (round to nearest even).
-#ifndef HALO_PACK_P_ALU
-#define HALO_PACK_P_ALU 0
-#endif
+// bf16x2 of two floats given as bit patterns, round to nearest even: the
+// P operand of the A.V MMA.  (Measured: truncating saves little and doubles
+// the worst-case error of a P value; rounding with integer adds and a byte
+// permute instead of the conversion instruction is slower, 117 against
+// 111 us on the stage-1 workload.)
 __device__ __forceinline__ uint32_t pack_p(uint32_t lo, uint32_t hi) {
-#if HALO_PACK_P_ALU
-  return __byte_perm(lo + 0x8000u, hi + 0x8000u, 0x7632);
-#else
   return pack_bf16x2(__uint_as_float(lo), __uint_as_float(hi));
-#endif
 }
 
 // tcgen05.ld / st, 32 lanes x 32 bit: thread t <-> lane t of the warp's quadrant

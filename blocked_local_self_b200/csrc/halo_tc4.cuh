@@ -425,7 +425,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int t = 0; t <= my_items; ++t) {
         if (t < my_items) {
           const int s = t % S;
-          if (t >= S && !mbar_wait_idle(&bar_eqk[s], ((t / S) - 1) & 1, kWaitNs, &abort_flag)) {
+          if (t >= S && !mbar_wait(&bar_eqk[s], ((t / S) - 1) & 1, kWaitNs, &abort_flag)) {
             if (!abort_flag) record_timeout(&abort_flag);
             break;
           }
@@ -440,7 +440,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         if (t >= 1) {
           const int k = t - 1, s = k % S;
-          if (k >= S && !mbar_wait_idle(&bar_ev[s], ((k / S) - 1) & 1, kWaitNs, &abort_flag)) {
+          if (k >= S && !mbar_wait(&bar_ev[s], ((k / S) - 1) & 1, kWaitNs, &abort_flag)) {
             if (!abort_flag) record_timeout(&abort_flag);
             break;
           }
@@ -470,8 +470,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         // the slot is free for S once the A.V of item k - 2 has read its P
         // (O elsewhere) or once its epilogue has read O; for G, always the latter
         uint64_t* slot_free = (C::O_IN_G && !is_g) ? &bar_ofull[g] : &bar_tfree[g];
-        if (!mbar_wait_idle(&bar_fqk[s], (k / S) & 1, kWaitNs, &abort_flag) ||
-            (k >= 2 && !mbar_wait_idle(slot_free, ((k >> 1) - 1) & 1, kWaitNs, &abort_flag))) {
+        if (!mbar_wait(&bar_fqk[s], (k / S) & 1, kWaitNs, &abort_flag) ||
+            (k >= 2 && !mbar_wait(slot_free, ((k >> 1) - 1) & 1, kWaitNs, &abort_flag))) {
           if (!abort_flag) record_timeout(&abort_flag);
           break;
         }

@@ -87,27 +87,6 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, uint64
   }
 }
 
-// As mbar_wait, for threads whose wait is off the critical path (the TMA and
-// MMA-issuing lanes of the producer warps): between tests the thread sleeps
-// for `backoff_ns`, so that its retries do not take issue slots from the
-// softmax warps of the same scheduler.
-#ifndef HALO_IDLE_BACKOFF_NS
-#define HALO_IDLE_BACKOFF_NS 0
-#endif
-__device__ __forceinline__ bool mbar_wait_idle(uint64_t* bar, uint32_t parity, uint64_t limit_ns,
-                                               const volatile int* abort_flag = nullptr) {
-  if (mbar_try_wait(bar, parity)) return true;
-  const uint64_t t0 = global_timer_ns();
-  for (;;) {
-#if HALO_IDLE_BACKOFF_NS > 0
-    __nanosleep(HALO_IDLE_BACKOFF_NS);
-#endif
-    if (mbar_try_wait(bar, parity)) return true;
-    if (abort_flag && *abort_flag) return false;
-    if (global_timer_ns() - t0 > limit_ns) return false;
-  }
-}
-
 // Named barrier `id` over `count` threads (a multiple of 32).
 __device__ __forceinline__ void named_bar_sync(int id, int count) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
