@@ -669,16 +669,25 @@ int bwd_plan(const Shape& s, BwdPlan* plan) {
   // largest power-of-two query tile (at most 256) whose item fits in shared memory
   const long long KS = static_cast<long long>(p.w) * p.w;
   if (KS > (1 << 20)) return HALO_ERR_UNSUPPORTED;
+  // Row groups per query in the query phase: enough that the tile's queries
+  // occupy the CTA's threads (at most one window row per group).
+  const int tt = s.d >= 16 ? s.d / 16 : 1;  // threads per (query, row group)
+  auto ksplit_for = [&](int qt) {
+    const int k = halo::bwd::kThreads / (qt * tt);
+    return k < 1 ? 1 : (k > p.w ? p.w : k);
+  };
   int qt = 256;
   while (qt > p.nq * 2) qt /= 2;
   for (; qt >= 1; qt /= 2) {
-    const halo::bwd::Layout L(s.d, static_cast<int>(KS), qt, p.w, p.R);
+    const int q = qt < p.nq ? qt : p.nq;
+    const halo::bwd::Layout L(s.d, static_cast<int>(KS), q, p.w, p.R, ksplit_for(q));
     if (L.bytes() <= kMaxDynSmem) break;
   }
   if (qt < 1) return HALO_ERR_UNSUPPORTED;
   p.QT = qt < p.nq ? qt : p.nq;
   p.ntiles = (p.nq + p.QT - 1) / p.QT;
-  plan->smem = halo::bwd::Layout(s.d, static_cast<int>(KS), p.QT, p.w, p.R).bytes();
+  p.ksplit = ksplit_for(p.QT);
+  plan->smem = halo::bwd::Layout(s.d, static_cast<int>(KS), p.QT, p.w, p.R, p.ksplit).bytes();
   p.num_items = static_cast<long long>(s.N) * p.nby * p.nbx * s.heads * p.ntiles;
   const size_t nin = static_cast<size_t>(s.N) * s.H * s.W * s.heads * s.d;
   const size_t ntab = static_cast<size_t>(p.R) * s.d;

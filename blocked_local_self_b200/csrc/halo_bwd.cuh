@@ -18,13 +18,17 @@
 // persistent CTA (256 threads) takes items in turn:
 //   * load: the item's K and V window (zero outside the image), its queries'
 //     q and dout, as float32 in shared memory; the tables once per CTA.
-//   * query phase: D/16 threads per query (16 channels each, dot products
-//     summed with shuffles).  The query's relative logits go to shared
-//     memory; pass 1 takes the row maximum and sum (online, rescaled only
-//     when the maximum moves); pass 2 recomputes p, takes dp and dz and
-//     accumulates dq in registers, the row sums of dz (per window row, added
-//     at once to dq's rel_h term and to the CTA's drel_h accumulator) and the
-//     column sums (shared memory, for the rel_w terms at the end).
+//   * query phase: D/16 threads per (query, row group) (16 channels each,
+//     dot products summed with shuffles); a query's window rows are dealt
+//     to ksplit groups (rows g, g + ksplit, ...) so that a tile of few
+//     queries (16 in a stride-2 block) still occupies the CTA.  The
+//     query's relative logits go to shared memory; pass 1 takes each
+//     group's row maximum and sum (online, rescaled only when the maximum
+//     moves), merged over the groups in shared memory; pass 2 recomputes
+//     p, takes dp and dz and accumulates dq, the row sums of dz (per window
+//     row, added at once to dq's rel_h term and to the CTA's drel_h
+//     accumulator) and the column sums (shared memory, for the rel_w terms
+//     at the end); the groups' dq parts are summed in shared memory.
 //   * key phase: D/16 threads per window key, dk and dv of the key in
 //     registers, looping over the tile's queries with the saved maximum,
 //     1/sum and D; the key's sums are added to float32 accumulators in
@@ -48,6 +52,7 @@ struct Params {
   int w, R;           // window side, table rows 2w - 1
   int nqx, nq;        // queries per block row, per block
   int QT, ntiles;     // queries per item, items per (block, head)
+  int ksplit;         // thread groups sharing one query's window rows in the query phase
   int nbx, nby;
   long long num_items;
   float c;            // log2(e) / sqrt(d): logits in log2 units
@@ -63,8 +68,8 @@ struct Ptrs {
 
 // Shared-memory layout (floats), the same on host and device.
 struct Layout {
-  int ks, kv, qs, dos, rh, rw, rlh, rlw, cs, st, drh, drw, total;
-  __host__ __device__ Layout(int D, int KS, int QT, int w, int R) {
+  int ks, kv, qs, dos, rh, rw, rlh, rlw, cs, st, drh, drw, ms, dqs, total;
+  __host__ __device__ Layout(int D, int KS, int QT, int w, int R, int ksplit) {
     int o = 0;
     ks = o; o += KS * D;
     kv = o; o += KS * D;
@@ -78,6 +83,8 @@ struct Layout {
     st = o; o += QT * 4;   // m (log2 units), 1/l, D, packed (qy, qx)
     drh = o; o += R * D;
     drw = o; o += R * D;
+    ms = o; o += ksplit > 1 ? 2 * kThreads : 0;   // per (query, row group): maximum, sum
+    dqs = o; o += ksplit > 1 ? QT * D : 0;        // dq summed over the row groups
     total = o;
   }
   __host__ __device__ int bytes() const { return total * 4; }
@@ -105,7 +112,8 @@ __global__ void __launch_bounds__(kThreads)
   static_assert(D % SL == 0 && (TT & (TT - 1)) == 0 && TT <= 32, "dim_head 8, 16, 32, 64 or 128");
   extern __shared__ float sm[];
   const int w = p.w, R = p.R, KS = w * w, QT = p.QT;
-  const Layout L(D, KS, QT, w, R);
+  const int KSPLIT = p.ksplit;
+  const Layout L(D, KS, QT, w, R, KSPLIT);
   float* Ks = sm + L.ks;
   float* Vs = sm + L.kv;
   float* Qs = sm + L.qs;
@@ -118,6 +126,8 @@ __global__ void __launch_bounds__(kThreads)
   float* ST = sm + L.st;
   float* DRH = sm + L.drh;
   float* DRW = sm + L.drw;
+  float* MS = sm + L.ms;
+  float* DQS = sm + L.dqs;
   const int tid = threadIdx.x;
   const int C = p.heads * D;
   const float c = p.c, sc = p.s;
@@ -171,12 +181,18 @@ __global__ void __launch_bounds__(kThreads)
       DOs[idx] = dd;
     }
     for (int idx = tid; idx < QT * w; idx += kThreads) CS[idx] = 0.f;
+    if (KSPLIT > 1)
+      for (int idx = tid; idx < QT * D; idx += kThreads) DQS[idx] = 0.f;
     __syncthreads();
 
-    // ---- query phase
-    for (int base = 0; base < QT; base += RPP) {
-      const int r = base + tid / TT, sl = tid % TT;
-      const bool act = r < qn;
+    // ---- query phase: TT threads per (query, row group), KSPLIT row groups
+    // per query (window rows kg, kg + KSPLIT, ...), so that few queries (a
+    // stride-2 block has 16) still occupy the whole CTA
+    const int QPP = kThreads / (TT * KSPLIT);  // queries per pass
+    for (int base = 0; base < QT; base += QPP) {
+      const int grp = tid / TT;                  // (query, row group) of this thread
+      const int r = base + grp / KSPLIT, kg = grp % KSPLIT, sl = tid % TT;
+      const bool act = r < qn && grp < QPP * KSPLIT;
       const int rr = act ? r : 0;
       const int iq = q0 + rr;
       const int qy = p.stride * (iq / p.nqx), qx = p.stride * (iq % p.nqx);
@@ -187,8 +203,15 @@ __global__ void __launch_bounds__(kThreads)
         qv[e] = Qs[rr * D + sl * SL + e];
         dov[e] = DOs[rr * D + sl * SL + e];
       }
-      // relative logits of this query (log2 units)
-      for (int kr = 0; kr < w; ++kr) {
+      // Every lane of a warp runs the same number of row iterations (the
+      // shuffles of group_sum need the whole warp); a group's iteration past
+      // the last window row is computed on row 0 and discarded.
+      const int NIT = (w + KSPLIT - 1) / KSPLIT;
+      // relative logits of this query (log2 units): rel_h of window row kr
+      // and rel_w of window column kr, for this group's indices kr
+      for (int it = 0; it < NIT; ++it) {
+        const bool rv = kg + it * KSPLIT < w;
+        const int kr = rv ? kg + it * KSPLIT : 0;
         const float* th = RH + (kr - qy + w - 1) * D + sl * SL;
         const float* tw = RW + (kr - qx + w - 1) * D + sl * SL;
         float ah = 0.f, aw = 0.f;
@@ -199,7 +222,7 @@ __global__ void __launch_bounds__(kThreads)
         }
         ah = group_sum<TT>(ah);
         aw = group_sum<TT>(aw);
-        if (sl == 0 && act) {
+        if (sl == 0 && act && rv) {
           RLH[r * w + kr] = c * ah;
           RLW[r * w + kr] = c * aw;
         }
@@ -212,12 +235,14 @@ __global__ void __launch_bounds__(kThreads)
         for (int e = 0; e < SL; ++e) dd = fmaf(dov[e], act ? ld(op + e) : 0.f, dd);
         dd = group_sum<TT>(dd);
       }
-      __syncwarp();
-      // pass 1: maximum and sum over the kept keys
+      __syncthreads();  // every group's relative logits are in shared memory
+      // pass 1: maximum and sum over this group's kept keys
       float m = -INFINITY, l = 0.f;
-      for (int kr = 0; kr < w; ++kr) {
+      for (int it = 0; it < NIT; ++it) {
+        const bool rv = kg + it * KSPLIT < w;
+        const int kr = rv ? kg + it * KSPLIT : 0;
         const int Y = y0 + kr;
-        const bool rin = act && Y >= 0 && Y < p.H;
+        const bool rin = act && rv && Y >= 0 && Y < p.H;
         const float rlh = RLH[rr * w + kr];
         for (int kc = 0; kc < w; ++kc) {
           const int X = x0 + kc, j = kr * w + kc;
@@ -237,14 +262,34 @@ __global__ void __launch_bounds__(kThreads)
           }
         }
       }
+      if (KSPLIT > 1) {
+        // merge the groups' (maximum, sum) pairs of each query
+        if (sl == 0) {
+          MS[2 * grp] = m;
+          MS[2 * grp + 1] = l;
+        }
+        __syncthreads();
+        const int g0 = (grp / KSPLIT) * KSPLIT;
+        float mm = -INFINITY;
+        for (int u = 0; u < KSPLIT; ++u) mm = fmaxf(mm, MS[2 * (g0 + u)]);
+        float ll = 0.f;
+        for (int u = 0; u < KSPLIT; ++u) {
+          const float mu = MS[2 * (g0 + u)];
+          if (mu != -INFINITY) ll += MS[2 * (g0 + u) + 1] * exp2f(mu - mm);
+        }
+        m = mm;
+        l = ll;
+      }
       const float inv_l = act ? 1.0f / l : 0.f;
       // pass 2: p, dz; dq and the row / column sums of dz
       float dq[SL];
 #pragma unroll
       for (int e = 0; e < SL; ++e) dq[e] = 0.f;
-      for (int kr = 0; kr < w; ++kr) {
+      for (int it = 0; it < NIT; ++it) {
+        const bool rv = kg + it * KSPLIT < w;
+        const int kr = rv ? kg + it * KSPLIT : 0;
         const int Y = y0 + kr;
-        const bool rin = act && Y >= 0 && Y < p.H;
+        const bool rin = act && rv && Y >= 0 && Y < p.H;
         const float rlh = RLH[rr * w + kr];
         float rowsum = 0.f;
         for (int kc = 0; kc < w; ++kc) {
@@ -265,7 +310,10 @@ __global__ void __launch_bounds__(kThreads)
 #pragma unroll
           for (int e = 0; e < SL; ++e) dq[e] = fmaf(dz, kp[e], dq[e]);
           rowsum += dz;
-          if (sl == 0 && act) CS[r * w + kc] += dz;
+          if (sl == 0 && act && rv) {
+            if (KSPLIT > 1) atomicAdd(&CS[r * w + kc], dz);
+            else CS[r * w + kc] += dz;
+          }
         }
         if (rin) {
           const int a = kr - qy + w - 1;
@@ -277,18 +325,46 @@ __global__ void __launch_bounds__(kThreads)
           }
         }
       }
-      __syncwarp();
+      if (KSPLIT > 1) {
+        if (act) {
+#pragma unroll
+          for (int e = 0; e < SL; ++e) atomicAdd(&DQS[r * D + sl * SL + e], dq[e]);
+        }
+        __syncthreads();  // column sums and dq partials complete
+      } else {
+        __syncwarp();
+      }
+      // rel_w terms of dq and drel_w: window columns kg, kg + KSPLIT, ...
       if (act) {
-        for (int kc = 0; kc < w; ++kc) {
+        float dw[SL];
+#pragma unroll
+        for (int e = 0; e < SL; ++e) dw[e] = 0.f;
+        for (int kc = kg; kc < w; kc += KSPLIT) {
           const float cs = CS[r * w + kc];
           const int b = kc - qx + w - 1;
           const float* tw = RW + b * D + sl * SL;
 #pragma unroll
           for (int e = 0; e < SL; ++e) {
-            dq[e] = fmaf(cs, tw[e], dq[e]);
+            dw[e] = fmaf(cs, tw[e], dw[e]);
             atomicAdd(DRW + b * D + sl * SL + e, sc * cs * qv[e]);
           }
         }
+        if (KSPLIT > 1) {
+#pragma unroll
+          for (int e = 0; e < SL; ++e) atomicAdd(&DQS[r * D + sl * SL + e], dw[e]);
+        } else {
+#pragma unroll
+          for (int e = 0; e < SL; ++e) dq[e] += dw[e];
+        }
+      }
+      if (KSPLIT > 1) {
+        __syncthreads();  // every group's rel_w terms are in
+        if (act && kg == 0) {
+#pragma unroll
+          for (int e = 0; e < SL; ++e) dq[e] = DQS[r * D + sl * SL + e];
+        }
+      }
+      if (act && kg == 0) {
         const int y = oy * p.stride, x = ox * p.stride;
         T* dst = g.dq + ((static_cast<size_t>(n) * p.H + y) * p.W + x) * C + static_cast<size_t>(head) * D + sl * SL;
 #pragma unroll
@@ -300,6 +376,7 @@ __global__ void __launch_bounds__(kThreads)
           ST[4 * r + 3] = __int_as_float((qy << 16) | qx);
         }
       }
+      __syncthreads();  // the next pass reuses the merge buffer
     }
     __syncthreads();
 
