@@ -18,9 +18,9 @@
 //     each, the linear layers' [out, in] layout, i.e. K-major B operands) per
 //     item.
 //   * projection round (lane 0 of three warps of the item's warpgroup):
-//     Q = x_q Wq_h^T (M=128: both blocks' queries), K_t = x_kv[tile t] Wk_h^T
-//     and V_t likewise (three 128-row tiles of the union window), fp32 into
-//     the warpgroup's TMEM slot.
+//     Q = x_q Wq_h^T (M=128: both blocks' queries) and [K_t | V_t] =
+//     x_kv[tile t] [Wk_h; Wv_h]^T (one N = 2d MMA chain per 128-row tile of
+//     the union window), fp32 into the warpgroup's TMEM slot.
 //   * the warpgroup reads them back (one TMEM lane = one row), rounds to
 //     bf16 (as an unfused pipeline would store q, k, v) and writes the Q_A,
 //     Q_B, K and V tiles of the two-block kernel (halo_tc4.cuh) into shared
@@ -93,18 +93,33 @@ struct Cfg {
   static constexpr int XKV_ATOM = KVT * 128 * 128;       // window pixels (padded to KVT tiles) x 64 channels
   static constexpr int XSTAGE = KA * (XQ_ATOM + XKV_ATOM);
   static constexpr int TX_X = KA * (128 + UROWS) * 128;
+  // The head's weights per 64-channel atom: Wq_h (d rows), and Wk_h over
+  // Wv_h (2d rows), so that one N = 2d MMA projects k and v of a tile.
   static constexpr int W_ATOM = D * 128;                 // d rows x 64 channels
-  static constexpr int W_BYTES = 3 * KA * W_ATOM;        // Wq_h, Wk_h, Wv_h
+  static constexpr int WKV_ATOM = 2 * W_ATOM;
+  static constexpr int OFF_WKV = KA * W_ATOM;            // the [Wk_h; Wv_h] atoms after the Wq_h atoms
+  static constexpr int W_BYTES = 3 * KA * W_ATOM;
   // converted attention tiles of one warpgroup: Q_A, Q_B, K union, V union
   static constexpr int OFF_QA = 0, OFF_QB = A::Q_TILE, OFF_K = 2 * A::Q_TILE, OFF_V = 2 * A::Q_TILE + A::K_TILE;
   static constexpr int TILES = 2 * A::Q_TILE + 2 * A::K_TILE;
   static constexpr int WG_BYTES = (TILES + W_BYTES + 1023) / 1024 * 1024;
   static constexpr int R_TILE = A::R_TILE;
-  // projection accumulators in the slot: Q at 0, K tiles, V tiles
-  static constexpr uint32_t COL_Q = 0, COL_K = D, COL_V = D + KVT * D;
+  // EARLY (d = 16): O goes to the relative-logit columns, so that after an
+  // item's exponent pass the S columns past P are dead until the next S: the
+  // next item's K and V projections are issued there as soon as this item's
+  // A.V is issued, and its Q projection into P's first columns once the A.V
+  // is done; the projections then overlap this item's A.V and epilogue.
+  // Otherwise all three are issued at the start of the item: Q at 0, K and V
+  // after it.
+  static constexpr bool EARLY = (int)kGBase + 2 * A::ON <= (int)kSlotCols &&
+                                A::O_BASE + 2 * KVT * D <= (int)kGBase;
+  static constexpr uint32_t COL_Q = 0;
+  static constexpr uint32_t COL_K = EARLY ? A::O_BASE : D;
+  static constexpr uint32_t COL_V = COL_K + KVT * 2 * D;  // end of the [k | v] tile columns
+  static constexpr uint32_t O_COL = EARLY ? kGBase : A::O_BASE;
   static_assert(CIN == 64 || CIN == 128, "c_in 64 or 128");
   static_assert(D == 16 || D == 32, "dim_head 16 or 32");
-  static_assert(COL_V + KVT * D <= kSlotCols, "projections in the slot");
+  static_assert(COL_V <= kSlotCols, "projections in the slot");
   static_assert(A::KROWS <= KVT * 128, "window tiles cover the rows the MMAs read");
 };
 
@@ -264,8 +279,9 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll 1
       for (int a = 0; a < C::KA; ++a) {
         tma_load_2d(wb + a * C::W_ATOM, &tmap_wq, &bar_wfull[g], 64 * a, head * D);
-        tma_load_2d(wb + (C::KA + a) * C::W_ATOM, &tmap_wkv, &bar_wfull[g], 64 * a, head * D);
-        tma_load_2d(wb + (2 * C::KA + a) * C::W_ATOM, &tmap_wkv, &bar_wfull[g], 64 * a, heads * D + head * D);
+        tma_load_2d(wb + C::OFF_WKV + a * C::WKV_ATOM, &tmap_wkv, &bar_wfull[g], 64 * a, head * D);
+        tma_load_2d(wb + C::OFF_WKV + a * C::WKV_ATOM + C::W_ATOM, &tmap_wkv, &bar_wfull[g], 64 * a,
+                    heads * D + head * D);
       }
       wi = j + 1;
     }
@@ -298,25 +314,22 @@ __global__ void __launch_bounds__(kThreads, 1)
     const float c = p.c;
     const int C_all = heads * D;
     const uint32_t idP = idesc_bf16_f32(128, D, false);       // projections: A = x (K-major), B = W (K-major)
+    const uint32_t idKV = idesc_bf16_f32(128, 2 * D, false);  // k and v of a window tile in one MMA
     const uint32_t idS = idesc_bf16_f32(64, A::NS, false);
     const uint32_t idG = idesc_bf16_f32(64, kRRows, false);
     const uint32_t idO = idesc_bf16_f32(64, A::ON, true);
     int ph = 0;
 
-    bool ok = true;
-    int jj = 0;
-    for (int j = g; j < my_items && ok; j += 2, ++jj) {
-      const int pi = j / heads, head = j % heads;
-      const int pair = blockIdx.x + pi * gridDim.x;
-      const int bx = pair % p.nbx, py = (pair / p.nbx) % p.npy, n = pair / (p.nbx * p.npy);
-      const int s = pi % XS;
-      const uint8_t* xs = sX + s * C::XSTAGE;
-      const uint32_t xqa = smem_addr(xs), xkva = smem_addr(xs + C::KA * C::XQ_ATOM);
-      // ---- projection round: Q (warp 0), K tiles (warp 1), V tiles (warp 2)
-      if (wq < 3 && lane == 0) {
-        const bool got = mbar_wait(&bar_xfull[s], (pi / XS) & 1, kWaitNs, &abort_flag) &&
-                         mbar_wait(&bar_wfull[g], jj & 1, kWaitNs, &abort_flag);
-        if (got) {
+    // Projections of item jn (the warpgroup's jjn-th): q_part issues Q (lane 0
+    // of warp 0), otherwise K (warp 1) and V (warp 2); each commits to bar_pr.
+    auto issue_proj = [&](int jn, int jjn, bool q_part) {
+      if (lane != 0 || (q_part ? wq != 0 : (wq != 1 && wq != 2))) return;
+      const int pin = jn / heads, sn = pin % XS;
+      const uint8_t* xsn = sX + sn * C::XSTAGE;
+      const uint32_t xqa = smem_addr(xsn), xkva = smem_addr(xsn + C::KA * C::XQ_ATOM);
+      const bool got = mbar_wait(&bar_xfull[sn], (pin / XS) & 1, kWaitNs, &abort_flag) &&
+                       mbar_wait(&bar_wfull[g], jjn & 1, kWaitNs, &abort_flag);
+      if (got) {
           tc_fence_after();
           constexpr int KSTEPS = CIN / 16;
           if (wq == 0) {
@@ -325,20 +338,40 @@ __global__ void __launch_bounds__(kThreads, 1)
               mma_f16_ss(slot + C::COL_Q, smem_desc(xqa + (ks >> 2) * C::XQ_ATOM + (ks & 3) * 32, 16, 1024, SW_128B),
                          smem_desc(wba + (ks >> 2) * C::W_ATOM + (ks & 3) * 32, 16, 1024, SW_128B), idP, ks != 0);
           } else {
-            const uint32_t col = wq == 1 ? C::COL_K : C::COL_V;
-            const uint32_t wm = wba + (wq == 1 ? 1 : 2) * C::KA * C::W_ATOM;
+            // [k | v] of the window tiles, N = 2d: warp 1 the first tiles, warp 2 the rest
+            const int t0 = wq == 1 ? 0 : (C::KVT + 1) / 2, t1 = wq == 1 ? (C::KVT + 1) / 2 : C::KVT;
+            const uint32_t wm = wba + C::OFF_WKV;
 #pragma unroll 1
-            for (int t = 0; t < C::KVT; ++t)
+            for (int t = t0; t < t1; ++t)
 #pragma unroll 1
               for (int ks = 0; ks < KSTEPS; ++ks)
-                mma_f16_ss(slot + col + t * D,
+                mma_f16_ss(slot + C::COL_K + t * 2 * D,
                            smem_desc(xkva + (ks >> 2) * C::XKV_ATOM + t * 128 * 128 + (ks & 3) * 32, 16, 1024, SW_128B),
-                           smem_desc(wm + (ks >> 2) * C::W_ATOM + (ks & 3) * 32, 16, 1024, SW_128B), idP, ks != 0);
+                           smem_desc(wm + (ks >> 2) * C::WKV_ATOM + (ks & 3) * 32, 16, 1024, SW_128B), idKV, ks != 0);
           }
           mma_commit(&bar_pr[g]);
-        } else if (!abort_flag) {
-          record_timeout(&abort_flag);
-        }
+      } else if (!abort_flag) {
+        record_timeout(&abort_flag);
+      }
+    };
+
+    bool ok = true;
+    int jj = 0;
+    if constexpr (C::EARLY) {
+      if (g < my_items) {
+        issue_proj(g, 0, false);
+        issue_proj(g, 0, true);
+      }
+    }
+    for (int j = g; j < my_items && ok; j += 2, ++jj) {
+      const int pi = j / heads, head = j % heads;
+      const int pair = blockIdx.x + pi * gridDim.x;
+      const int bx = pair % p.nbx, py = (pair / p.nbx) % p.npy, n = pair / (p.nbx * p.npy);
+      const int s = pi % XS;
+      // ---- projection round: Q (warp 0), K tiles (warp 1), V tiles (warp 2)
+      if constexpr (!C::EARLY) {
+        issue_proj(j, jj, false);
+        issue_proj(j, jj, true);
       }
       ok = warp_ok(mbar_wait(&bar_pr[g], jj & 1, kWaitNs, &abort_flag));
       if (!ok) break;
@@ -359,8 +392,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll 1
         for (int t = 0; t < C::KVT; ++t) {
           float kv[D], vv[D];
-          tmem_ld_d<D>(ts + C::COL_K + t * D, kv);
-          tmem_ld_d<D>(ts + C::COL_V + t * D, vv);
+          tmem_ld_d<D>(ts + C::COL_K + t * 2 * D, kv);
+          tmem_ld_d<D>(ts + C::COL_K + t * 2 * D + D, vv);
           tmem_wait_ld();
           const int kr = 128 * t + 32 * wq + lane;
           if (kr < C::UROWS) {
@@ -468,30 +501,38 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t lbo = smem_addr(sOnes) - va;
 #pragma unroll 1
         for (int kk = kb; kk < ke; ++kk)
-          mma_f16_ts(slot + lanes + A::O_BASE + hf * A::ON, slot + lanes + 8 * kk,
+          mma_f16_ts(slot + lanes + C::O_COL + hf * A::ON, slot + lanes + 8 * kk,
                      smem_desc(va + kk * 16 * A::ROWB, lbo, A::SBO, A::SW), idO, kk != kb);
         mma_commit(&bar_o[g]);
+      }
+      // the next item's K and V projections into the dead S columns
+      if constexpr (C::EARLY) {
+        if (j + 2 < my_items) issue_proj(j + 2, jj + 1, false);
       }
       ok = warp_ok(mbar_wait(&bar_o[g], jj & 1, kWaitNs, &abort_flag));
       if (!ok) break;
       tc_fence_after();
+      // and its Q projection into P's first columns, which the A.V has read
+      if constexpr (C::EARLY) {
+        if (j + 2 < my_items) issue_proj(j + 2, jj + 1, true);
+      }
       // ---- epilogue: (O_0 + O_1) / (l_0 + l_1), bf16, NHWC
       {
         float o[D], la, lb;
-        tmem_ld_x1(ts + A::O_BASE + D, &la);
-        tmem_ld_x1(ts + A::O_BASE + A::ON + D, &lb);
+        tmem_ld_x1(ts + C::O_COL + D, &la);
+        tmem_ld_x1(ts + C::O_COL + A::ON + D, &lb);
         constexpr int kSeg = (D % 32 == 0) ? 32 : 16;
 #pragma unroll
         for (int e = 0; e < D; e += kSeg) {
           float ta[kSeg], tb[kSeg];
           if constexpr (kSeg == 32) {
-            tmem_ld_x32(ts + A::O_BASE + e, ta);
-            tmem_ld_x32(ts + A::O_BASE + A::ON + e, tb);
+            tmem_ld_x32(ts + C::O_COL + e, ta);
+            tmem_ld_x32(ts + C::O_COL + A::ON + e, tb);
           } else {
-            tmem_ld_x8(ts + A::O_BASE + e, ta);
-            tmem_ld_x8(ts + A::O_BASE + e + 8, ta + 8);
-            tmem_ld_x8(ts + A::O_BASE + A::ON + e, tb);
-            tmem_ld_x8(ts + A::O_BASE + A::ON + e + 8, tb + 8);
+            tmem_ld_x8(ts + C::O_COL + e, ta);
+            tmem_ld_x8(ts + C::O_COL + e + 8, ta + 8);
+            tmem_ld_x8(ts + C::O_COL + A::ON + e, tb);
+            tmem_ld_x8(ts + C::O_COL + A::ON + e + 8, tb + 8);
           }
           tmem_wait_ld();
 #pragma unroll
