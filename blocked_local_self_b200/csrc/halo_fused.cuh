@@ -61,10 +61,11 @@ using tc4::tmem_ld_exact;
 using tc4::tmem_ld_x1;
 
 constexpr int kBlock = 8;
-constexpr int kThreads = 384;        // warpgroups 0-1 compute, warp 8 TMA, warps 9-11 idle
+constexpr int kThreads = 384;        // warpgroups 0-1 compute, warpgroup 2 conversion (warp 8 also TMA)
 constexpr int kTmaWarp = 8;
-constexpr int kSoftmaxRegs = tc::kSoftmaxRegs;
-constexpr int kProducerRegs = tc::kProducerRegs;
+constexpr int kSoftmaxRegs = 200;
+constexpr int kProducerRegs = 96;    // the conversion warps hold a tile row's q, k and v
+static_assert(256 * kSoftmaxRegs + 128 * kProducerRegs <= kThreads * 168, "register split");
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kSlotCols = 256;
 constexpr uint32_t kGBase = tc4::kGBase;  // 200
@@ -174,14 +175,14 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint8_t* sOnes = sX + p.xstages * C::XSTAGE;             // after the V tiles: positive LBO from any of them
 
   __shared__ __align__(8) uint64_t bar_xfull[2];
-  __shared__ __align__(8) uint64_t bar_xempty[2];  // count heads: every item of the pair has projected
   __shared__ __align__(8) uint64_t bar_wfull[2];
-  __shared__ __align__(8) uint64_t bar_wempty[2];
   __shared__ __align__(8) uint64_t bar_pr[2];      // count 3: Q, K, V projections
-  __shared__ __align__(8) uint64_t bar_s[2];       // count 3: S_A, S_B, G
+  __shared__ __align__(8) uint64_t bar_s[2];       // count 1: S_A, S_B, G
   __shared__ __align__(8) uint64_t bar_o[2];       // count 4: the A.V chains
+  __shared__ __align__(8) uint64_t bar_tfree[2];   // count 4: the warpgroup has read its O
   __shared__ __align__(8) uint64_t bar_wg[2];      // count 4: the warps of warpgroup g
-  __shared__ __align__(8) uint64_t bar_drain[8];
+  __shared__ __align__(8) uint64_t bar_cv;         // count 4: the conversion warps
+  __shared__ __align__(8) uint64_t bar_drain[9];
   __shared__ uint32_t tmem_base_sh;
   __shared__ int abort_flag;
 
@@ -193,19 +194,17 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   // ---------------------------------------------------------------- set-up
   if (tid == 0) {
-    for (int i = 0; i < XS; ++i) {
-      mbar_init(&bar_xfull[i], 1);
-      mbar_init(&bar_xempty[i], heads);
-    }
+    for (int i = 0; i < XS; ++i) mbar_init(&bar_xfull[i], 1);
     for (int g = 0; g < 2; ++g) {
       mbar_init(&bar_wfull[g], 1);
-      mbar_init(&bar_wempty[g], 1);
       mbar_init(&bar_pr[g], 3);
-      mbar_init(&bar_s[g], 3);
+      mbar_init(&bar_s[g], 1);
       mbar_init(&bar_o[g], 4);
+      mbar_init(&bar_tfree[g], 4);
       mbar_init(&bar_wg[g], 4);
     }
-    for (int w = 0; w < 8; ++w) mbar_init(&bar_drain[w], 1);
+    mbar_init(&bar_cv, 4);
+    for (int w = 0; w < 9; ++w) mbar_init(&bar_drain[w], 1);
     abort_flag = 0;
     fence_mbar_init();
   }
@@ -245,49 +244,147 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (warp >= 8) {
   asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kProducerRegs));
-  if (warp == kTmaWarp && lane == 0) {
-    // ------------------------------------------------------------ TMA producer
-    int xi = 0, wi = 0;
-    for (int j = 0; j < my_items; ++j) {
-      const int pi = j / heads, head = j % heads;
-      const int pair = blockIdx.x + pi * gridDim.x;
+  {
+    // ------------------------------------------------------------ conversion warpgroup (warps 8-11)
+    // Item by item (the two slots in turn): wait for the item's projections,
+    // refill the weight buffer and the x stage they have released (TMA, lane
+    // 0 of warp 8), wait until the slot's previous item has finished with the
+    // attention tiles, round q, k, v to bf16 into them, then issue the item's
+    // S and G MMAs (lane 0 of warp 9).  The softmax warpgroups meanwhile work
+    // on the previous items.
+    const int cw = warp - 8;  // TMEM lane quadrant
+    auto load_x = [&](int pin) {
+      const int pair = blockIdx.x + pin * gridDim.x;
       const int bx = pair % p.nbx, py = (pair / p.nbx) % p.npy, n = pair / (p.nbx * p.npy);
-      if (head == 0) {
-        const int s = pi % XS;
-        if (pi >= XS && !mbar_wait(&bar_xempty[s], ((pi / XS) - 1) & 1, kWaitNs, &abort_flag)) {
-          if (!abort_flag) record_timeout(&abort_flag);
-          break;
-        }
-        uint8_t* xs = sX + s * C::XSTAGE;
-        mbar_arrive_expect_tx(&bar_xfull[s], C::TX_X);
-        const int x0 = bx * kBlock, y0 = py * 2 * kBlock;
-#pragma unroll 1
-        for (int a = 0; a < C::KA; ++a) {
-          tma_load_4d(xs + a * C::XQ_ATOM, &tmap_xq, &bar_xfull[s], 64 * a, x0, y0, n);
-          tma_load_4d(xs + C::KA * C::XQ_ATOM + a * C::XKV_ATOM, &tmap_xkv, &bar_xfull[s], 64 * a, x0 - p.halo,
-                      y0 - p.halo, n);
-        }
-        xi = pi + 1;
-      }
-      const int g = j & 1;
-      if (j >= 2 && !mbar_wait(&bar_wempty[g], ((j >> 1) - 1) & 1, kWaitNs, &abort_flag)) {
-        if (!abort_flag) record_timeout(&abort_flag);
-        break;
-      }
-      uint8_t* wb = sWG + g * C::WG_BYTES + C::TILES;
-      mbar_arrive_expect_tx(&bar_wfull[g], C::W_BYTES);
+      const int sn = pin % XS;
+      uint8_t* xs = sX + sn * C::XSTAGE;
+      mbar_arrive_expect_tx(&bar_xfull[sn], C::TX_X);
+      const int x0 = bx * kBlock, y0 = py * 2 * kBlock;
 #pragma unroll 1
       for (int a = 0; a < C::KA; ++a) {
-        tma_load_2d(wb + a * C::W_ATOM, &tmap_wq, &bar_wfull[g], 64 * a, head * D);
-        tma_load_2d(wb + C::OFF_WKV + a * C::WKV_ATOM, &tmap_wkv, &bar_wfull[g], 64 * a, head * D);
-        tma_load_2d(wb + C::OFF_WKV + a * C::WKV_ATOM + C::W_ATOM, &tmap_wkv, &bar_wfull[g], 64 * a,
+        tma_load_4d(xs + a * C::XQ_ATOM, &tmap_xq, &bar_xfull[sn], 64 * a, x0, y0, n);
+        tma_load_4d(xs + C::KA * C::XQ_ATOM + a * C::XKV_ATOM, &tmap_xkv, &bar_xfull[sn], 64 * a, x0 - p.halo,
+                    y0 - p.halo, n);
+      }
+    };
+    auto load_w = [&](int jn) {
+      const int head = jn % heads, gn = jn & 1;
+      uint8_t* wb = sWG + gn * C::WG_BYTES + C::TILES;
+      mbar_arrive_expect_tx(&bar_wfull[gn], C::W_BYTES);
+#pragma unroll 1
+      for (int a = 0; a < C::KA; ++a) {
+        tma_load_2d(wb + a * C::W_ATOM, &tmap_wq, &bar_wfull[gn], 64 * a, head * D);
+        tma_load_2d(wb + C::OFF_WKV + a * C::WKV_ATOM, &tmap_wkv, &bar_wfull[gn], 64 * a, head * D);
+        tma_load_2d(wb + C::OFF_WKV + a * C::WKV_ATOM + C::W_ATOM, &tmap_wkv, &bar_wfull[gn], 64 * a,
                     heads * D + head * D);
       }
-      wi = j + 1;
+    };
+    const bool tma_lane = (warp == kTmaWarp && lane == 0);
+    const bool mma_lane = (warp == kTmaWarp + 1 && lane == 0);
+    int nx = 0, nw = 0;  // loads issued (drained on an abort)
+    if (tma_lane) {
+      for (int pin = 0; pin < XS && pin < my_pairs; ++pin) {
+        load_x(pin);
+        nx = pin + 1;
+      }
+      for (int jn = 0; jn < 2 && jn < my_items; ++jn) {
+        load_w(jn);
+        nw = jn + 1;
+      }
     }
-    if (abort_flag) {
-      for (int k = (xi > XS ? xi - XS : 0); k < xi; ++k) mbar_wait(&bar_xfull[k % XS], (k / XS) & 1, kWaitNs);
-      for (int k = (wi > 2 ? wi - 2 : 0); k < wi; ++k) mbar_wait(&bar_wfull[k & 1], (k >> 1) & 1, kWaitNs);
+    const uint32_t idS = idesc_bf16_f32(64, A::NS, false);
+    const uint32_t idG = idesc_bf16_f32(64, kRRows, false);
+    const uint32_t ra = smem_addr(sR);
+    int cph = 0;
+    bool ok = true;
+    for (int j = 0; j < my_items && ok; ++j) {
+      const int g = j & 1, jj = j >> 1;
+      const int pi = j / heads, head = j % heads;
+      ok = warp_ok(mbar_wait(&bar_pr[g], jj & 1, kWaitNs, &abort_flag));
+      if (!ok) break;
+      tc_fence_after();
+      // the projections of item j have read its weights, and, for the pair's
+      // last head, the pair's x: refill both
+      if (tma_lane) {
+        if (j + 2 < my_items) {
+          load_w(j + 2);
+          nw = j + 3;
+        }
+        if (head == heads - 1 && pi + XS < my_pairs) {
+          load_x(pi + XS);
+          nx = pi + XS + 1;
+        }
+      }
+      // the slot's previous item (j - 2) has finished its MMAs on the tiles
+      if (j >= 2) {
+        ok = warp_ok(mbar_wait(&bar_o[g], (jj - 1) & 1, kWaitNs, &abort_flag));
+        if (!ok) break;
+        tc_fence_after();
+      }
+      // ---- back to bf16 tiles: Q_A, Q_B (query rows), K and V (window rows)
+      uint8_t* wgb = sWG + g * C::WG_BYTES;
+      const uint32_t tsc = tmem + g * kSlotCols + (static_cast<uint32_t>(32 * cw) << 16);
+      {
+        float v[D];
+        tmem_ld_d<D>(tsc + C::COL_Q, v);
+        tmem_wait_ld();
+        const int r = 32 * cw + lane;  // query pixel: rows 0-63 block A, 64-127 block B
+        store_row<D>(wgb + (r < 64 ? C::OFF_QA : C::OFF_QB), r & 63, v);
+#pragma unroll 1
+        for (int t = 0; t < C::KVT; ++t) {
+          float kv[D], vv[D];
+          tmem_ld_d<D>(tsc + C::COL_K + t * 2 * D, kv);
+          tmem_ld_d<D>(tsc + C::COL_K + t * 2 * D + D, vv);
+          tmem_wait_ld();
+          const int kr = 128 * t + 32 * cw + lane;
+          if (kr < C::UROWS) {
+            store_row<D>(wgb + C::OFF_K, kr, kv);
+            store_row<D>(wgb + C::OFF_V, kr, vv);
+          }
+        }
+      }
+      fence_proxy_async_smem();
+      tc_fence_before();
+      ok = wg_sync(&bar_cv, cph, lane, &abort_flag);
+      if (!ok) break;
+      // ---- S (both blocks) and G: G's columns (and, without EARLY, S's)
+      // hold item j - 2's O until its epilogue has read it
+      if (mma_lane) {
+        tc_fence_after();
+        if (j >= 2 && !mbar_wait(&bar_tfree[g], (jj - 1) & 1, kWaitNs, &abort_flag)) {
+          if (!abort_flag) record_timeout(&abort_flag);
+        } else {
+          tc_fence_after();
+          const uint32_t slot = tmem + g * kSlotCols;
+          const uint32_t qaa = smem_addr(wgb + C::OFF_QA), qab = smem_addr(wgb + C::OFF_QB);
+          const uint32_t kta = smem_addr(wgb + C::OFF_K);
+#pragma unroll
+          for (int b = 0; b < 2; ++b) {
+            const uint32_t dst = slot + (static_cast<uint32_t>(b * 16) << 16);
+            const uint32_t qa = b ? qab : qaa, ka = kta + b * A::BOFF * A::ROWB;
+#pragma unroll
+            for (int ks = 0; ks < D / 16; ++ks)
+              mma_f16_ss(dst, smem_desc(qa + 32 * ks, 16, A::SBO, A::SW), smem_desc(ka + 32 * ks, 16, A::SBO, A::SW),
+                         idS, ks != 0);
+#pragma unroll
+            for (int ks = 0; ks < D / 16; ++ks)
+              mma_f16_ss(dst + kGBase, smem_desc(qa + 32 * ks, 16, A::SBO, A::SW),
+                         smem_desc(ra + 32 * ks, 16, A::SBO, A::SW), idG, ks != 0);
+          }
+          mma_commit(&bar_s[g]);
+        }
+      }
+    }
+    if (!ok && !abort_flag) record_timeout(&abort_flag);
+    if (tma_lane && abort_flag) {
+      // loads still in flight land before the block exits
+      for (int k = (nx > XS ? nx - XS : 0); k < nx; ++k) mbar_wait(&bar_xfull[k % XS], (k / XS) & 1, kWaitNs);
+      for (int k = (nw > 2 ? nw - 2 : 0); k < nw; ++k) mbar_wait(&bar_wfull[k & 1], (k >> 1) & 1, kWaitNs);
+    }
+    // the S and G MMAs are complete before TMEM is released
+    if (mma_lane) {
+      mma_commit(&bar_drain[8]);
+      mbar_wait(&bar_drain[8], 0, kWaitNs);
     }
   }
   __syncwarp();
@@ -307,126 +404,65 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t slot = tmem + g * kSlotCols;
     const uint32_t ts = slot + (static_cast<uint32_t>(32 * wq) << 16);
     uint8_t* wgb = sWG + g * C::WG_BYTES;
-    const uint32_t qaa = smem_addr(wgb + C::OFF_QA), qab = smem_addr(wgb + C::OFF_QB);
-    const uint32_t kta = smem_addr(wgb + C::OFF_K), vta = smem_addr(wgb + C::OFF_V);
+    const uint32_t vta = smem_addr(wgb + C::OFF_V);
     const uint32_t wba = smem_addr(wgb + C::TILES);
-    const uint32_t ra = smem_addr(sR);
     const float c = p.c;
     const int C_all = heads * D;
     const uint32_t idP = idesc_bf16_f32(128, D, false);       // projections: A = x (K-major), B = W (K-major)
     const uint32_t idKV = idesc_bf16_f32(128, 2 * D, false);  // k and v of a window tile in one MMA
-    const uint32_t idS = idesc_bf16_f32(64, A::NS, false);
-    const uint32_t idG = idesc_bf16_f32(64, kRRows, false);
     const uint32_t idO = idesc_bf16_f32(64, A::ON, true);
     int ph = 0;
 
     // Projections of item jn (the warpgroup's jjn-th): q_part issues Q (lane 0
-    // of warp 0), otherwise K (warp 1) and V (warp 2); each commits to bar_pr.
-    auto issue_proj = [&](int jn, int jjn, bool q_part) {
-      if (lane != 0 || (q_part ? wq != 0 : (wq != 1 && wq != 2))) return;
+    // of warp 0), otherwise K and V (warps 1 and 2); each commits to bar_pr.
+    // Without `wait` the call returns false, issuing nothing, when x or the
+    // weights have not landed yet (the caller issues them later).
+    auto issue_proj = [&](int jn, int jjn, bool q_part, bool wait) {
+      if (lane != 0 || (q_part ? wq != 0 : (wq != 1 && wq != 2))) return true;
       const int pin = jn / heads, sn = pin % XS;
       const uint8_t* xsn = sX + sn * C::XSTAGE;
       const uint32_t xqa = smem_addr(xsn), xkva = smem_addr(xsn + C::KA * C::XQ_ATOM);
+      if (!wait && !(mbar_test(&bar_xfull[sn], (pin / XS) & 1) && mbar_test(&bar_wfull[g], jjn & 1))) return false;
       const bool got = mbar_wait(&bar_xfull[sn], (pin / XS) & 1, kWaitNs, &abort_flag) &&
                        mbar_wait(&bar_wfull[g], jjn & 1, kWaitNs, &abort_flag);
       if (got) {
-          tc_fence_after();
-          constexpr int KSTEPS = CIN / 16;
-          if (wq == 0) {
+        tc_fence_after();
+        constexpr int KSTEPS = CIN / 16;
+        if (wq == 0) {
+#pragma unroll 1
+          for (int ks = 0; ks < KSTEPS; ++ks)
+            mma_f16_ss(slot + C::COL_Q, smem_desc(xqa + (ks >> 2) * C::XQ_ATOM + (ks & 3) * 32, 16, 1024, SW_128B),
+                       smem_desc(wba + (ks >> 2) * C::W_ATOM + (ks & 3) * 32, 16, 1024, SW_128B), idP, ks != 0);
+        } else {
+          // [k | v] of the window tiles, N = 2d: warp 1 the first tiles, warp 2 the rest
+          const int t0 = wq == 1 ? 0 : (C::KVT + 1) / 2, t1 = wq == 1 ? (C::KVT + 1) / 2 : C::KVT;
+          const uint32_t wm = wba + C::OFF_WKV;
+#pragma unroll 1
+          for (int t = t0; t < t1; ++t)
 #pragma unroll 1
             for (int ks = 0; ks < KSTEPS; ++ks)
-              mma_f16_ss(slot + C::COL_Q, smem_desc(xqa + (ks >> 2) * C::XQ_ATOM + (ks & 3) * 32, 16, 1024, SW_128B),
-                         smem_desc(wba + (ks >> 2) * C::W_ATOM + (ks & 3) * 32, 16, 1024, SW_128B), idP, ks != 0);
-          } else {
-            // [k | v] of the window tiles, N = 2d: warp 1 the first tiles, warp 2 the rest
-            const int t0 = wq == 1 ? 0 : (C::KVT + 1) / 2, t1 = wq == 1 ? (C::KVT + 1) / 2 : C::KVT;
-            const uint32_t wm = wba + C::OFF_WKV;
-#pragma unroll 1
-            for (int t = t0; t < t1; ++t)
-#pragma unroll 1
-              for (int ks = 0; ks < KSTEPS; ++ks)
-                mma_f16_ss(slot + C::COL_K + t * 2 * D,
-                           smem_desc(xkva + (ks >> 2) * C::XKV_ATOM + t * 128 * 128 + (ks & 3) * 32, 16, 1024, SW_128B),
-                           smem_desc(wm + (ks >> 2) * C::WKV_ATOM + (ks & 3) * 32, 16, 1024, SW_128B), idKV, ks != 0);
-          }
-          mma_commit(&bar_pr[g]);
+              mma_f16_ss(slot + C::COL_K + t * 2 * D,
+                         smem_desc(xkva + (ks >> 2) * C::XKV_ATOM + t * 128 * 128 + (ks & 3) * 32, 16, 1024, SW_128B),
+                         smem_desc(wm + (ks >> 2) * C::WKV_ATOM + (ks & 3) * 32, 16, 1024, SW_128B), idKV, ks != 0);
+        }
+        mma_commit(&bar_pr[g]);
       } else if (!abort_flag) {
         record_timeout(&abort_flag);
       }
+      return true;
     };
 
     bool ok = true;
     int jj = 0;
-    if constexpr (C::EARLY) {
-      if (g < my_items) {
-        issue_proj(g, 0, false);
-        issue_proj(g, 0, true);
-      }
-    }
+    bool kv_due = C::EARLY, q_due = C::EARLY;  // projections of the next item still to issue
     for (int j = g; j < my_items && ok; j += 2, ++jj) {
       const int pi = j / heads, head = j % heads;
       const int pair = blockIdx.x + pi * gridDim.x;
       const int bx = pair % p.nbx, py = (pair / p.nbx) % p.npy, n = pair / (p.nbx * p.npy);
-      const int s = pi % XS;
-      // ---- projection round: Q (warp 0), K tiles (warp 1), V tiles (warp 2)
-      if constexpr (!C::EARLY) {
-        issue_proj(j, jj, false);
-        issue_proj(j, jj, true);
-      }
-      ok = warp_ok(mbar_wait(&bar_pr[g], jj & 1, kWaitNs, &abort_flag));
-      if (!ok) break;
-      tc_fence_after();
-      // the three projections have read x and the weights: release both (x
-      // after every head of the pair, hence the barrier's count of heads)
-      if (wq == 0 && lane == 0) {
-        mbar_arrive(&bar_xempty[s]);
-        mbar_arrive(&bar_wempty[g]);
-      }
-      // ---- back to bf16 tiles: Q_A, Q_B (query rows), K and V (window rows)
-      {
-        float v[D];
-        tmem_ld_d<D>(ts + C::COL_Q, v);
-        tmem_wait_ld();
-        const int r = 32 * wq + lane;  // query pixel: rows 0-63 block A, 64-127 block B
-        store_row<D>(wgb + (r < 64 ? C::OFF_QA : C::OFF_QB), r & 63, v);
-#pragma unroll 1
-        for (int t = 0; t < C::KVT; ++t) {
-          float kv[D], vv[D];
-          tmem_ld_d<D>(ts + C::COL_K + t * 2 * D, kv);
-          tmem_ld_d<D>(ts + C::COL_K + t * 2 * D + D, vv);
-          tmem_wait_ld();
-          const int kr = 128 * t + 32 * wq + lane;
-          if (kr < C::UROWS) {
-            store_row<D>(wgb + C::OFF_K, kr, kv);
-            store_row<D>(wgb + C::OFF_V, kr, vv);
-          }
-        }
-      }
-      fence_proxy_async_smem();
-      tc_fence_before();
-      ok = wg_sync(&bar_wg[g], ph, lane, &abort_flag);
-      if (!ok) break;
-      // ---- S (block A on warp 0, block B on warp 1) and G (warp 2)
-      if (wq < 3 && lane == 0) {
-        tc_fence_after();
-        if (wq < 2) {
-          const uint32_t dst = slot + (static_cast<uint32_t>(wq * 16) << 16);
-          const uint32_t qa = wq ? qab : qaa, ka = kta + wq * A::BOFF * A::ROWB;
-#pragma unroll
-          for (int ks = 0; ks < D / 16; ++ks)
-            mma_f16_ss(dst, smem_desc(qa + 32 * ks, 16, A::SBO, A::SW), smem_desc(ka + 32 * ks, 16, A::SBO, A::SW),
-                       idS, ks != 0);
-        } else {
-#pragma unroll
-          for (int b = 0; b < 2; ++b)
-#pragma unroll
-            for (int ks = 0; ks < D / 16; ++ks)
-              mma_f16_ss(slot + (static_cast<uint32_t>(b * 16) << 16) + kGBase,
-                         smem_desc((b ? qab : qaa) + 32 * ks, 16, A::SBO, A::SW),
-                         smem_desc(ra + 32 * ks, 16, A::SBO, A::SW), idG, ks != 0);
-        }
-        mma_commit(&bar_s[g]);
-      }
+      // ---- this item's projections, unless issued during the previous item
+      if (!C::EARLY || kv_due) issue_proj(j, jj, false, true);
+      if (!C::EARLY || q_due) issue_proj(j, jj, true, true);
+      kv_due = q_due = true;
       ok = warp_ok(mbar_wait(&bar_s[g], jj & 1, kWaitNs, &abort_flag));
       if (!ok) break;
       tc_fence_after();
@@ -505,16 +541,17 @@ __global__ void __launch_bounds__(kThreads, 1)
                      smem_desc(va + kk * 16 * A::ROWB, lbo, A::SBO, A::SW), idO, kk != kb);
         mma_commit(&bar_o[g]);
       }
-      // the next item's K and V projections into the dead S columns
+      // the next item's K and V projections into the dead S columns (if its
+      // x and weights have landed; else at the start of that item)
       if constexpr (C::EARLY) {
-        if (j + 2 < my_items) issue_proj(j + 2, jj + 1, false);
+        if (j + 2 < my_items && issue_proj(j + 2, jj + 1, false, false)) kv_due = false;
       }
       ok = warp_ok(mbar_wait(&bar_o[g], jj & 1, kWaitNs, &abort_flag));
       if (!ok) break;
       tc_fence_after();
       // and its Q projection into P's first columns, which the A.V has read
       if constexpr (C::EARLY) {
-        if (j + 2 < my_items) issue_proj(j + 2, jj + 1, true);
+        if (j + 2 < my_items && issue_proj(j + 2, jj + 1, true, false)) q_due = false;
       }
       // ---- epilogue: (O_0 + O_1) / (l_0 + l_1), bf16, NHWC
       {
@@ -538,6 +575,10 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
           for (int i = 0; i < kSeg; ++i) o[e + i] = ta[i] + tb[i];
         }
+        // O is read: the next G (and, without EARLY, S) may take its columns
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bar_tfree[g]);
         const float inv = 1.0f / (la + lb);
         uint32_t pk[D / 2];
 #pragma unroll
@@ -548,8 +589,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int t = 0; t < D / 8; ++t)
           reinterpret_cast<uint4*>(dst)[t] = make_uint4(pk[4 * t], pk[4 * t + 1], pk[4 * t + 2], pk[4 * t + 3]);
       }
-      tc_fence_before();
-      ok = wg_sync(&bar_wg[g], ph, lane, &abort_flag);
+      // without EARLY the next item's projections overwrite this item's
+      // columns: every warp of the warpgroup is done with them first
+      if constexpr (!C::EARLY) {
+        tc_fence_before();
+        ok = wg_sync(&bar_wg[g], ph, lane, &abort_flag);
+      }
     }
     if (!ok && !abort_flag) record_timeout(&abort_flag);
     // MMAs this warp issued are complete before TMEM is released
