@@ -56,9 +56,10 @@ def parse_args():
                     help="repeat the K-step timed region until about this much time is covered (median reported)")
     ap.add_argument("--no-per-config", action="store_true",
                     help="skip timing every workload for the per_config object")
-    ap.add_argument("--pass", dest="which", choices=["fwd", "bwd", "masked"], default="fwd",
+    ap.add_argument("--pass", dest="which", choices=["fwd", "bwd", "masked", "fused"], default="fwd",
                     help="what one step runs: the forward (default), the backward (halo_attn_bwd, one launch per "
-                         "step from Python), or the SASA-masked forward with a 2*halo+1 window")
+                         "step from Python), the SASA-masked forward with a 2*halo+1 window, or the forward with "
+                         "the q, k, v projections fused in (halo_attn_fused; workloads with a fused form)")
     ap.add_argument("--no-extra", action="store_true",
                     help="skip timing the backward and the SASA-masked forward (next_rows object)")
     return ap.parse_args()
@@ -196,14 +197,22 @@ def measured_peaks() -> dict:
 def kernel_source_hash(kernel: str) -> str:
     """Hash of the source of one kernel family (its header and the headers it
     includes, comments and blank space removed), so that a profile summary
-    stays attached to the code it measured.  `kernel` is a name as
-    halo_kernel_name reports it, e.g. "halo_fwd_tc2<16,14>"."""
+    stays attached to the code it measured.  `kernel` is a name as the
+    kernel-name queries report it, e.g. "halo_fwd_tc2<16,14>",
+    "halo_bwd_tc<16,14>" or "halo_fused_tc<16,14,128>"."""
     import re
-    m = re.match(r"halo_fwd_(\w+?)<", kernel or "")
+    m = re.match(r"halo_(fwd_|bwd_|)(\w+?)<", kernel or "")
     if not m:
         return ""
+    kind, fam = m.groups()
+    if kind == "fwd_":
+        first = "halo_%s.cuh" % fam                                   # halo_fwd_tc4 -> halo_tc4.cuh
+    elif kind == "bwd_":
+        first = "halo_bwd_tc.cuh" if fam == "tc" else "halo_bwd.cuh"  # tensor-core / CUDA-core backward
+    else:
+        first = "halo_%s.cuh" % fam.split("_")[0]                     # halo_fused_tc -> halo_fused.cuh
     csrc = os.path.join(ROOT, "blocked_local_self_b200", "csrc")
-    seen, todo = set(), ["halo_%s.cuh" % m.group(1)]
+    seen, todo = set(), [first]
     while todo:
         name = todo.pop()
         if name in seen or not os.path.exists(os.path.join(csrc, name)):
@@ -687,7 +696,15 @@ def main():
     halo.load()
 
     wl = {**workloads.WORKLOADS, **workloads.NEXT_WORKLOADS}[args.workload]
-    inputs_cpu = workloads.make_inputs(wl, seed=rank_seed(wl, rank))
+    c_in = 0
+    if args.which == "fused":
+        forms = [ci for (fw, ci) in workloads.FUSED_WORKLOADS.values() if fw.name == wl.name]
+        if not forms:
+            raise SystemExit(f"--pass fused: {wl.name} has no fused form (see workloads.FUSED_WORKLOADS)")
+        c_in = forms[0]
+        inputs_cpu = workloads.make_fused_inputs(wl, c_in, seed=rank_seed(wl, rank))
+    else:
+        inputs_cpu = workloads.make_inputs(wl, seed=rank_seed(wl, rank))
     use_graph = not args.no_graph and args.which != "bwd"
     stream = torch.cuda.Stream() if use_graph else torch.cuda.current_stream()
     bench = DeviceBench(halo, wl, inputs_cpu, stream, use_graph=use_graph)
@@ -703,6 +720,15 @@ def main():
         bench.step = masked_step
         kernel = halo.masked_kernel_name(wl.N, wl.H, wl.W, wl.heads, wl.dim_head, wl.block, wl.halo, wl.stride,
                                          kmask, wl.torch_dtype)
+    elif args.which == "fused":
+        def fused_step(i, b=bench):
+            x, wq, wkv, rh, rw = b.sets[i % b.n_sets]
+            halo.attn_fused(x, wq, wkv, rh, rw, heads=wl.heads, block=wl.block, halo=wl.halo,
+                            out=b.outs[i % b.n_sets], stream=stream)
+
+        bench.step = fused_step
+        kernel = halo.fused_kernel_name(wl.N, wl.H, wl.W, c_in, wl.heads, wl.dim_head, wl.block, wl.halo,
+                                        wl.stride, wl.torch_dtype)
     elif args.which == "bwd":
         with torch.cuda.stream(stream):
             fwd_outs = [halo.attn(*st, block=wl.block, halo=wl.halo, stride=wl.stride) for st in bench.sets]
@@ -790,7 +816,7 @@ def main():
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": args.e2e_steps}
 
     base = None
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+    if rank == 0 and world == 1 and not args.no_cpu_baseline and args.which != "fused":
         base = cpu_baseline(wl, inputs_cpu)
     barrier(world)
     dist_done(world)
@@ -800,8 +826,8 @@ def main():
     per_step_s = ms * 1e-3 / args.steps
     pixels = wl.out_pixels * world
     value = pixels / per_step_s
-    step_flops = bwd_flops(wl) if args.which == "bwd" else wl.flops()
-    step_bytes = bwd_bytes(wl) if args.which == "bwd" else wl.bytes()
+    step_flops = {"bwd": bwd_flops(wl), "fused": fused_flops(wl, c_in)}.get(args.which, wl.flops())
+    step_bytes = {"bwd": bwd_bytes(wl), "fused": fused_bytes(wl, c_in)}.get(args.which, wl.bytes())
     tflops = step_flops * world / per_step_s * 1e-12
     launch_s = ms_local * 1e-3 / args.steps  # one step per launch sequence on this stream
     achieved_gbs = step_bytes / launch_s * 1e-9
