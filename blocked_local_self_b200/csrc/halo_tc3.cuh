@@ -34,8 +34,11 @@
 //     exceeds it by more than 8 (in log2 units), and only then is the fp32
 //     accumulator O rescaled (a rare path).  Exponentials part on MUFU, part as
 //     a cubic on the FMA pipe; bf16 P written back over the chunk's S columns.
-//   * A.V (warps 0 and 1 of the warpgroup, each half of the chunk's K-steps
-//     into its own accumulator): O_j += P_c V_c, M=128, N=d, P from TMEM.
+//   * A.V (issued by the warpgroup's MMA warp once all four softmax warps
+//     have stored the chunk's P, right after it issued the next chunk's S;
+//     each half of the chunk's K-steps into its own accumulator, the two
+//     interleaved): O_j += P_c V_c, M=128, N=d, P from TMEM.  The softmax
+//     warps never wait for one another within an item.
 //   * epilogue: (O_0 + O_1) / (row sum), bf16, NHWC store.
 // Every wait is bounded and reports HALO_ERR_TIMEOUT.
 #pragma once
@@ -76,7 +79,7 @@ constexpr int kProducerRegs = tc::kProducerRegs;
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kSlotCols = 256;  // warpgroup g owns columns [256g, 256g + 256)
 constexpr uint32_t kOCol = 192;      // O accumulators (two A.V streams) at [192, 192 + 2d)
-constexpr int kStreams = 2;          // A.V issue streams (warps 0 and 1 of the warpgroup)
+constexpr int kStreams = 2;          // A.V accumulators (halves of a chunk's K-steps), issued interleaved
 constexpr float kRescale = 8.0f;     // move the running maximum when exceeded by this (log2 units)
 constexpr uint64_t kWaitNs = tc::kWaitNs;
 
@@ -219,7 +222,6 @@ __global__ void __launch_bounds__(kThreads, 1)
   __shared__ __align__(8) uint64_t bar_pready[2][2];
   __shared__ __align__(8) uint64_t bar_ofull[2];     // count 2: last chunk's A.V done
   __shared__ __align__(8) uint64_t bar_done[2];
-  __shared__ __align__(8) uint64_t bar_pvdone[8];
   __shared__ uint32_t tmem_base_sh;
   __shared__ int abort_flag;
 
@@ -246,7 +248,6 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&bar_ofull[g], kStreams);
       mbar_init(&bar_done[g], 1);
     }
-    for (int w = 0; w < 8; ++w) mbar_init(&bar_pvdone[w], 1);
     abort_flag = 0;
     fence_mbar_init();
   }
@@ -310,12 +311,44 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
     }
   } else if (warp == kMmaWarp || warp == kMmaWarp + 1) {
-    // ------------------------------------------------------------ G and S MMAs of warpgroup g
+    // ------------------------------------------------------------ G, S and A.V MMAs of warpgroup g
+    // Chunk by chunk: S of chunk t, then, once the warpgroup has stored P of
+    // chunk t - 1, that chunk's A.V (the softmax warps only arrive on
+    // pready and go on to chunk t).
     const int g = warp - kMmaWarp;
     if (lane == 0) {
       const uint32_t slot = tmem + g * kSlotCols;
       const uint32_t idG = idesc_bf16_f32(128, kRRows, false);
+      const uint32_t idO = idesc_bf16_f32(128, D, true);
       const uint32_t ra = smem_addr(sR);
+      // A.V of chunk c of item k: two accumulators, each over half of the
+      // chunk's K-steps, issued alternately so that neither waits on the other
+      auto issue_av = [&](int k, int c) -> bool {
+        const int t = k * C::NCH + c, b = t & 1;
+        if (!mbar_wait(&bar_pready[g][b], (t >> 1) & 1, kWaitNs, &abort_flag)) return false;
+        tc_fence_after();
+        const int ksteps = (C::rows(c) * C::WP + 15) / 16, half = (ksteps + 1) / 2;
+        const uint32_t va = smem_addr(sStage + (k % S) * C::STAGE_BYTES + OFF_V + C::start(c) * C::ROWB);
+#pragma unroll 1
+        for (int i = 0; i < half; ++i) {
+#pragma unroll
+          for (int st = 0; st < kStreams; ++st) {
+            const int kk = st * half + i;
+            if (kk < (st ? ksteps : half))
+              mma_f16_ts(slot + kOCol + st * D, slot + b * kBufCols + 8 * kk,
+                         smem_desc(va + kk * 16 * C::ROWB, C::K_TILE, C::SBO, C::SW), idO, (c > 0 || i > 0));
+          }
+        }
+#pragma unroll
+        for (int st = 0; st < kStreams; ++st) {
+          mma_commit(&bar_bfree[g][b]);
+          if (c + 1 == C::NCH) {
+            mma_commit(&bar_ofull[g]);
+            mma_commit(&bar_empty[k % S]);
+          }
+        }
+        return true;
+      };
       bool ok = true;
       for (int k = 0; k < my_items && ok; ++k) {
         const int s = k % S, t0 = k * C::NCH;
@@ -351,7 +384,10 @@ __global__ void __launch_bounds__(kThreads, 1)
             mma_f16_ss(slot + b * kBufCols, smem_desc(qa + 32 * ks, 16, C::SBO, C::SW),
                        smem_desc(kb + 32 * ks, 16, C::SBO, C::SW), idS, ks != 0);
           mma_commit(&bar_sfull[g][b]);
+          if (c > 0 && !(ok = issue_av(k, c - 1))) break;
         }
+        // the item's last chunk
+        if (ok) ok = issue_av(k, C::NCH - 1);
       }
       if (!ok && !abort_flag) record_timeout(&abort_flag);
       mma_commit(&bar_done[g]);
@@ -377,7 +413,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t ts = slot + (static_cast<uint32_t>(32 * wq) << 16);  // this warp's lanes
     const float c = p.c;
     const int C_all = p.heads * D;
-    const uint32_t idO = idesc_bf16_f32(128, D, true);
     constexpr unsigned kPoly = poly_pair_mask<WIN, kBlock>();
 
     float rhc[WIN], rwc[C::WP];
@@ -535,30 +570,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&bar_pready[g][b]);
-      // ---- A.V of the chunk: warps 0 and 1 each issue half of its K-steps
-      bool issued = true;
-      if (wq < kStreams && lane == 0) {
-        issued = mbar_wait(&bar_pready[g][b], (t >> 1) & 1, kWaitNs, &abort_flag);
-        if (issued) {
-          tc_fence_after();
-          constexpr int KSTEPS = NW / 8, HALF = (KSTEPS + 1) / 2;
-          const int kb = wq ? HALF : 0, ke = wq ? KSTEPS : HALF;
-          const uint32_t va = smem_addr(sStage + (k % S) * C::STAGE_BYTES + OFF_V + C::start(cidx) * C::ROWB);
-#pragma unroll 1
-          for (int kk = kb; kk < ke; ++kk)
-            mma_f16_ts(slot + kOCol + wq * D, slot + b * kBufCols + 8 * kk,
-                       smem_desc(va + kk * 16 * C::ROWB, C::K_TILE, C::SBO, C::SW), idO, (cidx > 0 || kk > kb));
-          mma_commit(&bar_bfree[g][b]);
-          if (cidx + 1 == C::NCH) {
-            mma_commit(&bar_ofull[g]);
-            mma_commit(&bar_empty[k % S]);
-          }
-        }
-      }
+      // (the chunk's A.V is issued by the warpgroup's MMA warp)
       // next chunk's rows first
 #pragma unroll
       for (int i = 0; i + NR < WIN; ++i) rhc[i] = rhc[i + NR];
-      return warp_ok(issued);
+      return true;
     };
 
     constexpr int kLastRows = C::rows(C::NCH - 1);
@@ -599,11 +615,6 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (C::kGBothBufs && k + 1 < my_items) ok = gather(k + 1);
     }
     if (!ok && !abort_flag) record_timeout(&abort_flag);
-    // A.V MMAs this warp issued are complete before TMEM is released
-    if (wq < kStreams && lane == 0) {
-      mma_commit(&bar_pvdone[warp]);
-      mbar_wait(&bar_pvdone[warp], 0, kWaitNs);
-    }
     __syncwarp();
   }
 
