@@ -349,26 +349,32 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         return true;
       };
-      bool ok = true;
-      for (int k = 0; k < my_items && ok; ++k) {
+      // G of item k into the buffer of its first chunk (free once chunk
+      // t0 - 2's A.V is done; block 32: G spans both buffers, the other one
+      // frees with chunk t0 - 1's A.V)
+      auto issue_g = [&](int k) -> bool {
         const int s = k % S, t0 = k * C::NCH;
-        ok = mbar_wait(&bar_full[s], (k / S) & 1, kWaitNs, &abort_flag);
-        // G into the buffer of the item's first chunk, free once chunk t0 - 2's A.V is done
-        if (ok && t0 >= 2) ok = mbar_wait(&bar_bfree[g][t0 & 1], ((t0 - 2) >> 1) & 1, kWaitNs, &abort_flag);
-        // block 32: G spans both buffers; the other one frees with chunk t0 - 1's A.V
-        if (C::kGBothBufs && ok && t0 >= 1)
-          ok = mbar_wait(&bar_bfree[g][(t0 - 1) & 1], ((t0 - 1) >> 1) & 1, kWaitNs, &abort_flag);
-        if (!ok) break;
+        bool got = mbar_wait(&bar_full[s], (k / S) & 1, kWaitNs, &abort_flag);
+        if (got && t0 >= 2) got = mbar_wait(&bar_bfree[g][t0 & 1], ((t0 - 2) >> 1) & 1, kWaitNs, &abort_flag);
+        if (C::kGBothBufs && got && t0 >= 1)
+          got = mbar_wait(&bar_bfree[g][(t0 - 1) & 1], ((t0 - 1) >> 1) & 1, kWaitNs, &abort_flag);
+        if (!got) return false;
         tc_fence_after();
-        const uint8_t* st = sStage + s * C::STAGE_BYTES;
-        const uint32_t qa = smem_addr(st + OFF_Q + g * 128 * C::ROWB);
-        const uint32_t ka = smem_addr(st + OFF_K);
+        const uint32_t qa = smem_addr(sStage + s * C::STAGE_BYTES + OFF_Q + g * 128 * C::ROWB);
         const uint32_t gdst = slot + (C::kGBothBufs ? 0u : (t0 & 1) * kBufCols);
 #pragma unroll
         for (int ks = 0; ks < D / 16; ++ks)
           mma_f16_ss(gdst, smem_desc(qa + 32 * ks, 16, C::SBO, C::SW),
                      smem_desc(ra + 32 * ks, 16, C::SBO, C::SW), idG, ks != 0);
         mma_commit(&bar_gfull[g]);
+        return true;
+      };
+      bool ok = my_items > 0 ? issue_g(0) : true;
+      for (int k = 0; k < my_items && ok; ++k) {
+        const int s = k % S, t0 = k * C::NCH;
+        const uint8_t* st = sStage + s * C::STAGE_BYTES;
+        const uint32_t qa = smem_addr(st + OFF_Q + g * 128 * C::ROWB);
+        const uint32_t ka = smem_addr(st + OFF_K);
 #pragma unroll 1
         for (int c = 0; c < C::NCH; ++c) {
           const int t = t0 + c, b = t & 1;
@@ -386,8 +392,17 @@ __global__ void __launch_bounds__(kThreads, 1)
           mma_commit(&bar_sfull[g][b]);
           if (c > 0 && !(ok = issue_av(k, c - 1))) break;
         }
-        // the item's last chunk
-        if (ok) ok = issue_av(k, C::NCH - 1);
+        if (!ok) break;
+        // the next item's G, then this item's last A.V: the softmax gathers
+        // the next item's relative logits while the last chunk finishes
+        // (block 32: G needs the last chunk's buffer too, so it comes after)
+        if constexpr (!C::kGBothBufs) {
+          if (k + 1 < my_items) ok = issue_g(k + 1);
+          if (ok) ok = issue_av(k, C::NCH - 1);
+        } else {
+          ok = issue_av(k, C::NCH - 1);
+          if (ok && k + 1 < my_items) ok = issue_g(k + 1);
+        }
       }
       if (!ok && !abort_flag) record_timeout(&abort_flag);
       mma_commit(&bar_done[g]);
