@@ -26,9 +26,12 @@
 //     group's row maximum and sum (online, rescaled only when the maximum
 //     moves), merged over the groups in shared memory; pass 2 recomputes
 //     p, takes dp and dz and accumulates dq, the row sums of dz (per window
-//     row, added at once to dq's rel_h term and to the CTA's drel_h
-//     accumulator) and the column sums (shared memory, for the rel_w terms
-//     at the end); the groups' dq parts are summed in shared memory.
+//     row, added at once to dq's rel_h term) and the column sums (for the
+//     rel_w terms at the end), both kept in shared memory; the groups' dq
+//     parts are summed in shared memory.
+//   * table phase: drel_h[a] += s sum over the tile's queries of the row sum
+//     at table row a times q, drel_w likewise from the column sums; one
+//     thread per table element (no atomics), into the CTA's accumulators.
 //   * key phase: D/16 threads per window key, dk and dv of the key in
 //     registers, looping over the tile's queries with the saved maximum,
 //     1/sum and D; the key's sums are added to float32 accumulators in
@@ -68,7 +71,7 @@ struct Ptrs {
 
 // Shared-memory layout (floats), the same on host and device.
 struct Layout {
-  int ks, kv, qs, dos, rh, rw, rlh, rlw, cs, st, drh, drw, ms, dqs, total;
+  int ks, kv, qs, dos, rh, rw, rlh, rlw, cs, rs, st, drh, drw, ms, dqs, total;
   __host__ __device__ Layout(int D, int KS, int QT, int w, int R, int ksplit) {
     int o = 0;
     ks = o; o += KS * D;
@@ -80,6 +83,7 @@ struct Layout {
     rlh = o; o += QT * w;
     rlw = o; o += QT * w;
     cs = o; o += QT * w;
+    rs = o; o += QT * w;   // per (query, window row) sum of dz
     st = o; o += QT * 4;   // m (log2 units), 1/l, D, packed (qy, qx)
     drh = o; o += R * D;
     drw = o; o += R * D;
@@ -103,6 +107,7 @@ __device__ __forceinline__ float group_sum(float x) {
 
 using simt::sasa_kept;
 
+
 template <typename T, int D>
 __global__ void __launch_bounds__(kThreads)
     halo_bwd_simt(const Ptrs<T> g, const Params p) {
@@ -123,6 +128,7 @@ __global__ void __launch_bounds__(kThreads)
   float* RLH = sm + L.rlh;
   float* RLW = sm + L.rlw;
   float* CS = sm + L.cs;
+  float* RS = sm + L.rs;
   float* ST = sm + L.st;
   float* DRH = sm + L.drh;
   float* DRW = sm + L.drw;
@@ -319,11 +325,10 @@ __global__ void __launch_bounds__(kThreads)
           const int a = kr - qy + w - 1;
           const float* th = RH + a * D + sl * SL;
 #pragma unroll
-          for (int e = 0; e < SL; ++e) {
-            dq[e] = fmaf(rowsum, th[e], dq[e]);
-            atomicAdd(DRH + a * D + sl * SL + e, sc * rowsum * qv[e]);
-          }
+          for (int e = 0; e < SL; ++e) dq[e] = fmaf(rowsum, th[e], dq[e]);
         }
+        // the row's dz sum for the drel_h phase (zero for rows outside the image)
+        if (sl == 0 && act && rv) RS[r * w + kr] = rin ? rowsum : 0.f;
       }
       if (KSPLIT > 1) {
         if (act) {
@@ -344,10 +349,7 @@ __global__ void __launch_bounds__(kThreads)
           const int b = kc - qx + w - 1;
           const float* tw = RW + b * D + sl * SL;
 #pragma unroll
-          for (int e = 0; e < SL; ++e) {
-            dw[e] = fmaf(cs, tw[e], dw[e]);
-            atomicAdd(DRW + b * D + sl * SL + e, sc * cs * qv[e]);
-          }
+          for (int e = 0; e < SL; ++e) dw[e] = fmaf(cs, tw[e], dw[e]);
         }
         if (KSPLIT > 1) {
 #pragma unroll
@@ -379,6 +381,23 @@ __global__ void __launch_bounds__(kThreads)
       __syncthreads();  // the next pass reuses the merge buffer
     }
     __syncthreads();
+
+    // ---- table phase: drel_h[a] += s sum over the tile's queries of the dz
+    // sum of the window row at index a, times q; drel_w likewise with the
+    // column sums.  One thread per table element: no atomics.
+    for (int idx = tid; idx < 2 * R * D; idx += kThreads) {
+      const bool wcol = idx >= R * D;
+      const int ae = wcol ? idx - R * D : idx, a = ae / D, e = ae - a * D;
+      const float* sums = wcol ? CS : RS;
+      float acc = 0.f;
+      for (int i = 0; i < qn; ++i) {
+        const int qyx = __float_as_int(ST[4 * i + 3]);
+        // table row a = kr - qy + w - 1 (rel_h), a = kc - qx + w - 1 (rel_w)
+        const int kr = a + (wcol ? (qyx & 0xffff) : (qyx >> 16)) - (w - 1);
+        if (kr >= 0 && kr < w) acc = fmaf(sums[i * w + kr], Qs[i * D + e], acc);
+      }
+      (wcol ? DRW : DRH)[ae] += sc * acc;
+    }
 
     // ---- key phase
     for (int base = 0; base < KS; base += RPP) {
