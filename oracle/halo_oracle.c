@@ -222,11 +222,12 @@ static int full_output(const oracle_args *ap, double *out, int threads)
     const int w = block + 2 * halo;
     const long total = (long)N * heads * OH * OW;
 #ifdef _OPENMP
-    if (threads > 0) omp_set_num_threads(threads);
+    const int nt_call = threads > 0 ? threads : omp_get_max_threads();
 #else
     (void)threads;
+    const int nt_call = 1;
 #endif
-#pragma omp parallel
+#pragma omp parallel num_threads(nt_call)
     {
         double *z = (double *)__builtin_alloca(sizeof(double) * (size_t)w * w);
         char *valid = (char *)__builtin_alloca((size_t)w * w);
@@ -379,16 +380,17 @@ int halo_oracle_bwd_f64(const void *q, const void *k, const void *v,
     memset(dk, 0, nin * sizeof(double));
     memset(dv, 0, nin * sizeof(double));
 #ifdef _OPENMP
-    if (threads > 0) omp_set_num_threads(threads);
-    const int nt = omp_get_max_threads();
+    const int nt_call = threads > 0 ? threads : omp_get_max_threads();
+    const int nt = nt_call;
 #else
     (void)threads;
+    const int nt_call = 1;
     const int nt = 1;
 #endif
     double *part = (double *)calloc((size_t)nt * 2 * ntab, sizeof(double));
     if (!part) return -2;
     const long units = (long)N * heads;
-#pragma omp parallel
+#pragma omp parallel num_threads(nt_call)
     {
 #ifdef _OPENMP
         const int tid = omp_get_thread_num();
@@ -462,9 +464,9 @@ int halo_oracle_fused_f64(const void *x, const void *wq, const void *wkv,
         return -2;
     }
 #ifdef _OPENMP
-    if (threads > 0) omp_set_num_threads(threads);
+    const int nt_call = threads > 0 ? threads : omp_get_max_threads();
 #endif
-#pragma omp parallel for schedule(static)
+#pragma omp parallel for num_threads(nt_call) schedule(static)
     for (long pix = 0; pix < (long)npix; ++pix) {
         for (int o = 0; o < C; ++o) {
             double aq = 0.0, ak = 0.0, av = 0.0;
@@ -513,11 +515,12 @@ int halo_oracle_samples_f64(const void *q, const void *k, const void *v,
     }
     const long total = (long)nsamples * heads;
 #ifdef _OPENMP
-    if (threads > 0) omp_set_num_threads(threads);
+    const int nt_call = threads > 0 ? threads : omp_get_max_threads();
 #else
     (void)threads;
+    const int nt_call = 1;
 #endif
-#pragma omp parallel
+#pragma omp parallel num_threads(nt_call)
     {
         double *z = (double *)__builtin_alloca(sizeof(double) * (size_t)w * w);
         char *valid = (char *)__builtin_alloca((size_t)w * w);
