@@ -35,11 +35,11 @@
 //     accumulator O rescaled (a rare path).  Exponentials part on MUFU, part as
 //     a cubic on the FMA pipe; bf16 P written back over the chunk's S columns.
 //   * A.V (issued by the warpgroup's MMA warp once all four softmax warps
-//     have stored the chunk's P, right after it issued the next chunk's S;
-//     each half of the chunk's K-steps into its own accumulator, the two
-//     interleaved): O_j += P_c V_c, M=128, N=d, P from TMEM.  The softmax
-//     warps never wait for one another within an item.
-//   * epilogue: (O_0 + O_1) / (row sum), bf16, NHWC store.
+//     have stored the chunk's P, right after it issued the next chunk's S):
+//     [O | l] += P_c [V_c | ones], M=128, N=d+8, P from TMEM; the ones
+//     columns give the row sum of the bf16 P.  The softmax warps never wait
+//     for one another within an item.
+//   * epilogue: O / (row sum from the ones columns), bf16, NHWC store.
 // Every wait is bounded and reports HALO_ERR_TIMEOUT.
 #pragma once
 
@@ -79,7 +79,9 @@ constexpr int kProducerRegs = tc::kProducerRegs;
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kSlotCols = 256;  // warpgroup g owns columns [256g, 256g + 256)
 constexpr uint32_t kOCol = 192;      // O accumulators (two A.V streams) at [192, 192 + 2d)
-constexpr int kStreams = 2;          // A.V accumulators (halves of a chunk's K-steps), issued interleaved
+// A.V: one accumulator [O | row sums] of d + 8 columns: the B operand is
+// [V | ones], the ones tile's 8 columns returning the row sum of the very
+// bf16 P the MMA consumed (no per-logit additions in the softmax).
 constexpr float kRescale = 8.0f;     // move the running maximum when exceeded by this (log2 units)
 constexpr uint64_t kWaitNs = tc::kWaitNs;
 
@@ -134,8 +136,9 @@ struct Cfg {
   static_assert(2 * kBufCols <= kOCol, "S buffers below the O accumulators");
   static_assert(!kGBothBufs || kRRows <= 2 * (int)kBufCols, "G inside the two S buffers");
   static_assert(kGBothBufs || kRRows <= (int)kBufCols, "G inside one S buffer");
-  static_assert(kOCol + kStreams * D <= kSlotCols, "O accumulators in the slot");
-  static_assert(ns(NCH - 1) / 16 >= kStreams, "every A.V stream has a K-step in every chunk");
+  static constexpr int ON = D + 8;                                       // A.V N: V and the ones columns
+  static constexpr int ONES_BYTES = ((kChunkRows * WP + 15) / 16 * 16 * ROWB + 1023) / 1024 * 1024;
+  static_assert(kOCol + ON <= kSlotCols, "O accumulator in the slot");
   static_assert(2 * WIN - 1 <= kRelW && kRelW + 2 * WIN - 1 <= kRRows, "relative table rows");
   static_assert((kChunkRows * WP) % 8 == 0, "chunk starts on a swizzle atom");
   static_assert(WP % 2 == 0 && WP <= 40, "row pitch");
@@ -144,7 +147,7 @@ struct Cfg {
 template <int D, int WIN, int BLOCK>
 __host__ __device__ constexpr int smem_bytes(int stages) {
   using C = Cfg<D, WIN, BLOCK>;
-  return 1024 + C::R_TILE + stages * C::STAGE_BYTES;
+  return 1024 + C::R_TILE + stages * C::STAGE_BYTES + C::ONES_BYTES;
 }
 
 // Window-column pairs (kc, kc+1), kc even, whose exponentials take the
@@ -211,16 +214,16 @@ __global__ void __launch_bounds__(kThreads, 1)
   // t & 1; sfull / bfree of a buffer complete once per chunk on it, so the
   // phase of chunk t is t >> 1.
   __shared__ __align__(8) uint64_t bar_full[4];
-  __shared__ __align__(8) uint64_t bar_empty[4];     // count 4: both streams of both warpgroups, last chunk
+  __shared__ __align__(8) uint64_t bar_empty[4];     // count 2: both warpgroups' last chunk
   __shared__ __align__(8) uint64_t bar_gfull[2];     // G MMA done
   __shared__ __align__(8) uint64_t bar_gfree[2];     // count 4: the warpgroup loaded G
   __shared__ __align__(8) uint64_t bar_sfull[2][2];  // S of the chunk in buffer b done
-  __shared__ __align__(8) uint64_t bar_bfree[2][2];  // count 2: both streams' A.V of that chunk done
+  __shared__ __align__(8) uint64_t bar_bfree[2][2];  // the A.V of that chunk done
   // count 4: P of chunk t stored, alternating by t & 1: a warp can be one
   // chunk ahead of another (its arrival for chunk t+1 must not complete the
   // phase of chunk t), never two (chunk t+2's S needs chunk t's A.V)
   __shared__ __align__(8) uint64_t bar_pready[2][2];
-  __shared__ __align__(8) uint64_t bar_ofull[2];     // count 2: last chunk's A.V done
+  __shared__ __align__(8) uint64_t bar_ofull[2];     // the item's last A.V done
   __shared__ __align__(8) uint64_t bar_done[2];
   __shared__ uint32_t tmem_base_sh;
   __shared__ int abort_flag;
@@ -229,23 +232,24 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int warp = tid >> 5;
   const int lane = tid & 31;
   const int S = p.stages;
+  uint8_t* sOnes = sStage + S * C::STAGE_BYTES;  // after every stage: positive LBO from any V chunk
 
   // ---------------------------------------------------------------- set-up
   if (tid == 0) {
     for (int i = 0; i < S; ++i) {
       mbar_init(&bar_full[i], 1);
-      mbar_init(&bar_empty[i], 2 * kStreams);
+      mbar_init(&bar_empty[i], 2);
     }
     for (int g = 0; g < 2; ++g) {
       mbar_init(&bar_gfull[g], 1);
       mbar_init(&bar_gfree[g], 4);
       mbar_init(&bar_sfull[g][0], 1);
       mbar_init(&bar_sfull[g][1], 1);
-      mbar_init(&bar_bfree[g][0], kStreams);
-      mbar_init(&bar_bfree[g][1], kStreams);
+      mbar_init(&bar_bfree[g][0], 1);
+      mbar_init(&bar_bfree[g][1], 1);
       mbar_init(&bar_pready[g][0], 4);
       mbar_init(&bar_pready[g][1], 4);
-      mbar_init(&bar_ofull[g], kStreams);
+      mbar_init(&bar_ofull[g], 1);
       mbar_init(&bar_done[g], 1);
     }
     abort_flag = 0;
@@ -265,6 +269,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       val = *reinterpret_cast<const uint4*>(p.rel_w + (r - kRelW) * D + u * 8);
     *reinterpret_cast<uint4*>(sR + swz<C::ROWB>(r, u)) = val;
   }
+  // ones tile (bf16 1.0 in every element, so the swizzle does not matter)
+  for (int idx = tid; idx < C::ONES_BYTES / 16; idx += kThreads)
+    reinterpret_cast<uint4*>(sOnes)[idx] = make_uint4(0x3f803f80u, 0x3f803f80u, 0x3f803f80u, 0x3f803f80u);
   for (int s = 0; s < S; ++s) {
     uint8_t* st = sStage + s * C::STAGE_BYTES;
     for (int idx = tid; idx < (C::KPAD - C::KS) * C::ROWB / 16; idx += kThreads) {
@@ -319,33 +326,25 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (lane == 0) {
       const uint32_t slot = tmem + g * kSlotCols;
       const uint32_t idG = idesc_bf16_f32(128, kRRows, false);
-      const uint32_t idO = idesc_bf16_f32(128, D, true);
+      const uint32_t idO = idesc_bf16_f32(128, C::ON, true);
       const uint32_t ra = smem_addr(sR);
-      // A.V of chunk c of item k: two accumulators, each over half of the
-      // chunk's K-steps, issued alternately so that neither waits on the other
+      // A.V of chunk c of item k into [O | row sums]
       auto issue_av = [&](int k, int c) -> bool {
         const int t = k * C::NCH + c, b = t & 1;
         if (!mbar_wait(&bar_pready[g][b], (t >> 1) & 1, kWaitNs, &abort_flag)) return false;
         tc_fence_after();
-        const int ksteps = (C::rows(c) * C::WP + 15) / 16, half = (ksteps + 1) / 2;
+        const int ksteps = (C::rows(c) * C::WP + 15) / 16;
         const uint32_t va = smem_addr(sStage + (k % S) * C::STAGE_BYTES + OFF_V + C::start(c) * C::ROWB);
+        // B = [V | ones]: the ones atom at leading byte offset lbo, same row pitch
+        const uint32_t lbo = smem_addr(sOnes) - va;
 #pragma unroll 1
-        for (int i = 0; i < half; ++i) {
-#pragma unroll
-          for (int st = 0; st < kStreams; ++st) {
-            const int kk = st * half + i;
-            if (kk < (st ? ksteps : half))
-              mma_f16_ts(slot + kOCol + st * D, slot + b * kBufCols + 8 * kk,
-                         smem_desc(va + kk * 16 * C::ROWB, C::K_TILE, C::SBO, C::SW), idO, (c > 0 || i > 0));
-          }
-        }
-#pragma unroll
-        for (int st = 0; st < kStreams; ++st) {
-          mma_commit(&bar_bfree[g][b]);
-          if (c + 1 == C::NCH) {
-            mma_commit(&bar_ofull[g]);
-            mma_commit(&bar_empty[k % S]);
-          }
+        for (int kk = 0; kk < ksteps; ++kk)
+          mma_f16_ts(slot + kOCol, slot + b * kBufCols + 8 * kk, smem_desc(va + kk * 16 * C::ROWB, lbo, C::SBO, C::SW),
+                     idO, (c > 0 || kk > 0));
+        mma_commit(&bar_bfree[g][b]);
+        if (c + 1 == C::NCH) {
+          mma_commit(&bar_ofull[g]);
+          mma_commit(&bar_empty[k % S]);
         }
         return true;
       };
@@ -506,7 +505,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     };
 
     // ---- one key chunk (NR window rows; rhc[0..NR) are its rows' rel_h logits)
-    float m_run = -INFINITY, l = 0.f;
+    float m_run = -INFINITY;
     auto chunk = [&](auto nr, int k, int cidx) -> bool {
       constexpr int NR = decltype(nr)::value;
       constexpr int WP = C::WP;
@@ -534,8 +533,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         mc = fmaxf(mc, mr + rhc[r]);
       }
       const bool upd = mc > m_run + kRescale;
-      // O holds earlier chunks against m_run: rescale it when the maximum moves
-      // (a row whose earlier chunks had no in-image key has O = 0 and l = 0)
+      // O and its row sums hold earlier chunks against m_run: rescale them
+      // when the maximum moves (a row whose earlier chunks had no in-image key
+      // has O = 0, sums included)
       if (__any_sync(0xffffffffu, upd && m_run != -INFINITY && cidx > 0)) {
         const int tp = t - 1;
         if (!warp_ok(mbar_wait(&bar_bfree[g][tp & 1], (tp >> 1) & 1, kWaitNs, &abort_flag))) return false;
@@ -543,7 +543,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const float alpha = (upd && m_run != -INFINITY) ? exp2_mufu(m_run - mc) : 1.0f;
         // eight columns at a time: y[] is live, registers are short
 #pragma unroll 1
-        for (int e = 0; e < kStreams * D; e += 8) {
+        for (int e = 0; e < C::ON; e += 8) {
           float o[8];
           tmem_ld_x8(ts + kOCol + e, o);
           tmem_wait_ld();
@@ -552,13 +552,11 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int i = 0; i < 8; ++i) ob[i] = __float_as_uint(o[i] * alpha);
           tmem_st_x8(ts + kOCol + e, ob);
         }
-        l *= alpha;
       }
       if (upd) m_run = mc;
       const float mb = (m_run == -INFINITY ? 0.f : m_run);
-      // exponentials, row sum, packed bf16 P over the chunk's S columns
-      float2 lacc[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f),
-                        make_float2(0.f, 0.f)};
+      // exponentials, packed bf16 P over the chunk's S columns (the row sum
+      // comes from the A.V's ones columns)
       uint32_t pk[NW];
 #pragma unroll
       for (int i = 0; i < NP; ++i) {
@@ -572,15 +570,12 @@ __global__ void __launch_bounds__(kThreads, 1)
           rx = __float_as_uint(exp2_mufu(x.x));
           ry = __float_as_uint(exp2_mufu(x.y));
         }
-        lacc[i & 3] = __fadd2_rn(lacc[i & 3], make_float2(__uint_as_float(rx), __uint_as_float(ry)));
         pk[i] = pack_p(rx, ry);
       }
 #pragma unroll
       for (int i = NP; i < NW; ++i) pk[i] = 0u;
 #pragma unroll
       for (int i = 0; i < NW; i += 8) tmem_st_x8(buf + i, pk + i);
-      const float2 la = __fadd2_rn(lacc[0], lacc[1]), lb = __fadd2_rn(lacc[2], lacc[3]);
-      l += (la.x + lb.x) + (la.y + lb.y);
       tmem_wait_st();
       tc_fence_before();
       __syncwarp();
@@ -598,7 +593,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int k = 0; k < my_items && ok; ++k) {
       const ItemCoord ic = item_coord<C::NQUART>(blockIdx.x + k * gridDim.x, p.heads, p.nbx, p.nby);
       m_run = -INFINITY;
-      l = 0.f;
 #pragma unroll 1
       for (int ci = 0; ci < kLoopChunks && ok; ++ci) ok = chunk(std::integral_constant<int, kChunkRows>{}, k, ci);
       if constexpr (kLoopChunks < C::NCH) {
@@ -607,19 +601,19 @@ __global__ void __launch_bounds__(kThreads, 1)
       // the next item's relative logits while this item's last A.V runs
       // (block 32: G needs both S buffers, so it follows the epilogue)
       if (!C::kGBothBufs && ok && k + 1 < my_items) ok = gather(k + 1);
-      // ---- epilogue: (O_0 + O_1) / l, bf16, NHWC
+      // ---- epilogue: O / l, bf16, NHWC
       if (ok) ok = warp_ok(mbar_wait(&bar_ofull[g], k & 1, kWaitNs, &abort_flag));
       if (!ok) break;
       tc_fence_after();
       {
-        float o[kStreams * D];
-        tmem_ld_cols<kStreams * D>(ts + kOCol, o);
+        float o[C::ON];
+        tmem_ld_cols<C::ON>(ts + kOCol, o);
         tmem_wait_ld();
-        const float inv = 1.0f / l;
+        const float inv = 1.0f / o[D];  // row sum of the bf16 P (ones columns)
         uint32_t pk[D / 2];
 #pragma unroll
         for (int t = 0; t < D / 2; ++t)
-          pk[t] = pack_bf16x2((o[2 * t] + o[D + 2 * t]) * inv, (o[2 * t + 1] + o[D + 2 * t + 1]) * inv);
+          pk[t] = pack_bf16x2(o[2 * t] * inv, o[2 * t + 1] * inv);
         const int y = ic.by * kBlock + ic.quart * C::QROWS + yq, x = ic.bx * kBlock + xl;
         __nv_bfloat16* dst = p.out + ((static_cast<size_t>(ic.n) * p.H + y) * p.W + x) * C_all + ic.head * D;
 #pragma unroll
