@@ -152,14 +152,20 @@ __host__ __device__ constexpr int smem_bytes(int stages) {
 
 // Window-column pairs (kc, kc+1), kc even, whose exponentials take the
 // polynomial: inside the block's own columns [h, h+b), which are never
-// outside the image.  Bit kc/2 of the mask.
+// outside the image.  Bit kc/2 of the mask.  Measured balance of MUFU and
+// FMA-pipe issue (row sums from the MMA): block 16, 4 of 12 pairs (large
+// workload 549 / 542 / 539 / 563 / 582 us with 2 / 3 / 4 / 5 / 6); block 32,
+// 6 of 20 (block 32 halo 3: 398 / 395 / 411 with 4 / 6 / 8).
 #ifndef HALO_TC3_POLY_PAIRS
 #define HALO_TC3_POLY_PAIRS 4
+#endif
+#ifndef HALO_TC3_POLY_PAIRS_B32
+#define HALO_TC3_POLY_PAIRS_B32 6
 #endif
 template <int WIN, int BLOCK>
 __host__ __device__ constexpr unsigned poly_pair_mask() {
   constexpr int h = (WIN - BLOCK) / 2;
-  const int npairs = HALO_TC3_POLY_PAIRS * BLOCK / 16;
+  const int npairs = (BLOCK == 32) ? HALO_TC3_POLY_PAIRS_B32 : HALO_TC3_POLY_PAIRS;
   unsigned m = 0;
   int picked = 0;
   const int mid = (h + BLOCK / 2 - 1) & ~1;
