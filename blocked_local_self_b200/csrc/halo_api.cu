@@ -365,11 +365,15 @@ int launch_win(const void* q, const void* k, const void* v, const void* rh, cons
 // increase would wait forever, so the launch is refused), the number of
 // pipeline stages that fit the opt-in shared memory next to the kernel's
 // static shared memory, and a persistent grid of one CTA per SM.
+// opt_bytes / opt_flag: shared memory a kernel can use for an optional
+// feature; the flag is set (and the bytes added) only when they fit next to
+// the stages chosen without them.
 template <class Params>
 int launch_persistent(void (*fn)(const CUtensorMap, const CUtensorMap, const CUtensorMap, const Params),
                       int threads, int softmax_regs, int producer_regs, int (*smem_fn)(int), int max_stages,
                       const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv, Params& p,
-                      long long items, int sm_count, cudaStream_t st) {
+                      long long items, int sm_count, cudaStream_t st, int opt_bytes = 0,
+                      int Params::*opt_flag = nullptr) {
   cudaFuncAttributes attr;
   if (cudaFuncGetAttributes(&attr, reinterpret_cast<const void*>(fn)) != cudaSuccess) return HALO_ERR_CUDA;
   if (256 * softmax_regs + 128 * producer_regs > threads * attr.numRegs) return HALO_ERR_UNSUPPORTED;
@@ -380,8 +384,12 @@ int launch_persistent(void (*fn)(const CUtensorMap, const CUtensorMap, const CUt
   const int budget = (optin < kMaxDynSmem ? optin : kMaxDynSmem) - static_cast<int>(attr.sharedSizeBytes);
   int stages = max_stages;
   while (stages > 1 && smem_fn(stages) > budget) --stages;
-  const int smem = smem_fn(stages);
+  int smem = smem_fn(stages);
   if (smem > budget) return HALO_ERR_UNSUPPORTED;
+  if (opt_flag) {
+    p.*opt_flag = (opt_bytes > 0 && smem + opt_bytes <= budget) ? 1 : 0;
+    if (p.*opt_flag) smem += opt_bytes;
+  }
   if (cudaFuncSetAttribute(reinterpret_cast<const void*>(fn), cudaFuncAttributeMaxDynamicSharedMemorySize, smem) !=
       cudaSuccess)
     return HALO_ERR_CUDA;
@@ -457,11 +465,14 @@ int launch_tc3(const Tc3Entry& e, const void* q, const void* k, const void* v, c
   fill_common(p, rh, rw, out, s);
   p.nbx = s.W / e.block;
   p.nby = s.H / e.block;
+  // output map: box = one softmax warp's 32 query rows (block x 32/block)
+  if (!encode_nhwc(&p.tmap_o, out, s, e.block, 32 / e.block, 1)) return HALO_ERR_CUDA;
   const int quarters = e.block * e.block / 256;
   const long long items = static_cast<long long>(s.N) * p.nbx * p.nby * s.heads * quarters;
-  // the kernel has four stage barriers
+  // the kernel has four stage barriers; the output staging (8 warps x 32
+  // rows) is used where it fits next to the stages
   return launch_persistent(e.fn, halo::tc3::kThreads, halo::tc3::kSoftmaxRegs, halo::tc3::kProducerRegs, e.smem, 4,
-                           mq, mk, mv, p, items, sm_count, st);
+                           mq, mk, mv, p, items, sm_count, st, 8 * 32 * s.d * 2, &halo::tc3::Params::tma_out);
 }
 
 int launch_tc4(const Tc4Entry& e, const void* q, const void* k, const void* v, const void* rh, const void* rw,

@@ -86,6 +86,9 @@ constexpr float kRescale = 8.0f;     // move the running maximum when exceeded b
 constexpr uint64_t kWaitNs = tc::kWaitNs;
 
 struct Params {
+  // output tensor map: box {d, block, 32 / block, 1} = one warp's 32 query
+  // rows (used when tma_out is set)
+  CUtensorMap tmap_o;
   const __nv_bfloat16* rel_h;
   const __nv_bfloat16* rel_w;
   __nv_bfloat16* out;
@@ -93,6 +96,7 @@ struct Params {
   int nbx, nby;
   int num_items;   // N * nby * nbx * heads
   int stages;
+  int tma_out;     // 1: the epilogue stages each warp's rows in shared memory and stores them by TMA
   float c;         // log2(e) / sqrt(d)
 };
 
@@ -138,6 +142,8 @@ struct Cfg {
   static_assert(kGBothBufs || kRRows <= (int)kBufCols, "G inside one S buffer");
   static constexpr int ON = D + 8;                                       // A.V N: V and the ones columns
   static constexpr int ONES_BYTES = ((kChunkRows * WP + 15) / 16 * 16 * ROWB + 1023) / 1024 * 1024;
+  static constexpr int OUT_WARP = 32 * ROWB;        // one softmax warp's output rows (TMA store staging)
+  static constexpr int OUT_BYTES = 8 * OUT_WARP;
   static_assert(kOCol + ON <= kSlotCols, "O accumulator in the slot");
   static_assert(2 * WIN - 1 <= kRelW && kRelW + 2 * WIN - 1 <= kRRows, "relative table rows");
   static_assert((kChunkRows * WP) % 8 == 0, "chunk starts on a swizzle atom");
@@ -202,7 +208,7 @@ __device__ __forceinline__ ItemCoord item_coord(int item, int heads, int nbx, in
 template <int D, int WIN, int BLOCK>
 __global__ void __launch_bounds__(kThreads, 1)
     halo_fwd_tc3(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__ CUtensorMap tmap_k,
-                 const __grid_constant__ CUtensorMap tmap_v, const Params p) {
+                 const __grid_constant__ CUtensorMap tmap_v, const __grid_constant__ Params p) {
   using C = Cfg<D, WIN, BLOCK>;
   constexpr int kBlock = C::kBlock;
   constexpr uint32_t kBufCols = C::kBufCols;
@@ -239,6 +245,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int lane = tid & 31;
   const int S = p.stages;
   uint8_t* sOnes = sStage + S * C::STAGE_BYTES;  // after every stage: positive LBO from any V chunk
+  uint8_t* sOut = sOnes + C::ONES_BYTES;         // output staging (when p.tma_out)
 
   // ---------------------------------------------------------------- set-up
   if (tid == 0) {
@@ -620,16 +627,36 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
         for (int t = 0; t < D / 2; ++t)
           pk[t] = pack_bf16x2(o[2 * t] * inv, o[2 * t + 1] * inv);
-        const int y = ic.by * kBlock + ic.quart * C::QROWS + yq, x = ic.bx * kBlock + xl;
-        __nv_bfloat16* dst = p.out + ((static_cast<size_t>(ic.n) * p.H + y) * p.W + x) * C_all + ic.head * D;
+        if (p.tma_out) {
+          // the warp's 32 rows (lane = row of its box) through shared memory,
+          // one TMA store per warp: coalesced, and the warp does not wait
+          uint8_t* stg = sOut + warp * C::OUT_WARP;
+          if (lane == 0) bulk_wait_read_all();  // the previous store has read the buffer
+          __syncwarp();
 #pragma unroll
-        for (int t = 0; t < D / 8; ++t)
-          reinterpret_cast<uint4*>(dst)[t] = make_uint4(pk[4 * t], pk[4 * t + 1], pk[4 * t + 2], pk[4 * t + 3]);
+          for (int t = 0; t < D / 8; ++t)
+            *reinterpret_cast<uint4*>(stg + swz<C::ROWB>(lane, t)) =
+                make_uint4(pk[4 * t], pk[4 * t + 1], pk[4 * t + 2], pk[4 * t + 3]);
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) {
+            const int y0w = ic.by * kBlock + ic.quart * C::QROWS + (kBlock == 16 ? 8 * g + 2 * wq : 4 * g + wq);
+            tma_store_4d(&p.tmap_o, stg, ic.head * D, ic.bx * kBlock, y0w, ic.n);
+            bulk_commit_group();
+          }
+        } else {
+          const int y = ic.by * kBlock + ic.quart * C::QROWS + yq, x = ic.bx * kBlock + xl;
+          __nv_bfloat16* dst = p.out + ((static_cast<size_t>(ic.n) * p.H + y) * p.W + x) * C_all + ic.head * D;
+#pragma unroll
+          for (int t = 0; t < D / 8; ++t)
+            reinterpret_cast<uint4*>(dst)[t] = make_uint4(pk[4 * t], pk[4 * t + 1], pk[4 * t + 2], pk[4 * t + 3]);
+        }
       }
       tc_fence_before();
       if (C::kGBothBufs && k + 1 < my_items) ok = gather(k + 1);
     }
     if (!ok && !abort_flag) record_timeout(&abort_flag);
+    if (p.tma_out && lane == 0) bulk_wait_all();  // this warp's output stores are complete
     __syncwarp();
   }
 
