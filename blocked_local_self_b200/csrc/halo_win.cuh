@@ -14,8 +14,11 @@
 // key costs 2 SL fused multiply-adds per thread and one exponential per query.
 // Each query's relative logits q.rel_h[kr - qy + w - 1] and
 // q.rel_w[kc - qx + w - 1] are taken once (2w dot products) and kept in
-// shared memory.  Optional SASA mask (section 2.2): keys outside the query's
-// k x k square are skipped.
+// shared memory.  The softmax offset is a per-query upper bound of the largest
+// logit (|q| max|k| plus the largest relative logits), so a row takes one pass
+// without rescaling; the online softmax remains for rows where the bound could
+// lie too far above the maximum.  Optional SASA mask (section 2.2): keys
+// outside the query's k x k square are skipped.
 #pragma once
 
 #include <cstdint>
@@ -35,10 +38,10 @@ struct Params {
   float c;       // log2(e) / sqrt(d): logits in log2 units
 };
 
-// Shared-memory floats for one item.
+// Shared-memory floats for one item (the last 8: per-warp maxima of |k|).
 __host__ __device__ inline int smem_floats(int D, int w, int qpass) {
   const int KS = w * w, R = 2 * w - 1;
-  return 2 * KS * D + 2 * R * D + 2 * qpass * w;
+  return 2 * KS * D + 2 * R * D + 2 * qpass * w + 8;
 }
 
 __device__ __forceinline__ float ldf(const float* p) { return __ldg(p); }
@@ -65,6 +68,7 @@ __global__ void __launch_bounds__(kMaxThreads)
   float* RH = Vs + KS * D;
   float* RW = RH + R * D;
   float* RL = RW + R * D;  // per query of the pass: w rel_h logits, then w rel_w logits
+  float* KM = RL + 2 * p.qpass * w;  // per-warp maxima of |k| over the window
   const int C = p.heads * D;
   const int tid = threadIdx.x, nthr = blockDim.x;
 
@@ -96,6 +100,23 @@ __global__ void __launch_bounds__(kMaxThreads)
     RW[idx] = ldf(rel_w + idx);
   }
   __syncthreads();
+  // the largest key norm of the window (zero keys outside the image)
+  {
+    float km = 0.f;
+    for (int j = tid; j < KS; j += nthr) {
+      float s2 = 0.f;
+#pragma unroll
+      for (int e = 0; e < D; ++e) s2 = fmaf(Ks[j * D + e], Ks[j * D + e], s2);
+      km = fmaxf(km, s2);
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) km = fmaxf(km, __shfl_xor_sync(0xffffffffu, km, o));
+    if ((tid & 31) == 0) KM[tid >> 5] = km;
+    __syncthreads();
+  }
+  float kmax = 0.f;
+  for (int i = 0; i < (nthr + 31) / 32; ++i) kmax = fmaxf(kmax, KM[i]);
+  kmax = sqrtf(kmax);
 
   const float c = p.c;
   const int r_kept = p.kmask > 0 ? (p.kmask >> 1) : (1 << 20);
@@ -134,7 +155,34 @@ __global__ void __launch_bounds__(kMaxThreads)
       }
     }
     __syncwarp();
-    float m = -INFINITY, l = 0.f;
+    // The softmax offset.  An upper bound of the row's largest logit:
+    // |q c| max|k| (Cauchy-Schwarz) plus the largest relative logits; the
+    // query's own pixel (always a kept key) gives a lower bound.  While the
+    // two are within 100 (log2 units) every p = 2^(z - m) stays a normal
+    // float and the largest is at least 2^-100, so one pass with this fixed m
+    // loses nothing; otherwise the online softmax (running maximum, rescaled
+    // sums) takes the row.
+    float qn2 = 0.f;
+#pragma unroll
+    for (int e = 0; e < SL; ++e) qn2 = fmaf(qv[e], qv[e], qn2);
+    qn2 = group_sum<TT>(qn2);
+    float mh = -INFINITY, mw = -INFINITY;
+    for (int i = 0; i < w; ++i) {
+      mh = fmaxf(mh, rlq[i]);
+      mw = fmaxf(mw, rlq[w + i]);
+    }
+    const float m_ub = sqrtf(qn2) * kmax + mh + mw;
+    float z_self;
+    {
+      const int js = (qy + p.halo) * w + qx + p.halo;
+      const float* kp = Ks + js * D + sl * SL;
+      float z = 0.f;
+#pragma unroll
+      for (int e = 0; e < SL; ++e) z = fmaf(qv[e], kp[e], z);
+      z_self = group_sum<TT>(z) + rlq[qy + p.halo] + rlq[w + qx + p.halo];
+    }
+    const bool bounded = m_ub - z_self <= 100.0f;
+    float m = bounded ? m_ub : -INFINITY, l = 0.f;
     for (int kr = 0; kr < w; ++kr) {
       const int Y = y0 + kr;
       const bool rin = Y >= 0 && Y < p.H && kr - qy - p.halo <= r_kept && qy + p.halo - kr <= r_kept;
@@ -142,13 +190,16 @@ __global__ void __launch_bounds__(kMaxThreads)
       for (int kc = 0; kc < w; ++kc) {
         const int X = x0 + kc, j = kr * w + kc;
         const float* kp = Ks + j * D + sl * SL;
-        float z = 0.f;
+        float z0 = 0.f, z1 = 0.f;
 #pragma unroll
-        for (int e = 0; e < SL; ++e) z = fmaf(qv[e], kp[e], z);
-        z = group_sum<TT>(z) + zr + rlq[w + kc];
+        for (int e = 0; e < SL; e += 2) {
+          z0 = fmaf(qv[e], kp[e], z0);
+          z1 = fmaf(qv[e + 1], kp[e + 1], z1);
+        }
+        const float z = group_sum<TT>(z0 + z1) + zr + rlq[w + kc];
         const bool kept = rin && X >= 0 && X < p.W && kc - qx - p.halo <= r_kept && qx + p.halo - kc <= r_kept;
         if (kept) {  // the same for every thread of a query's group
-          if (z > m) {
+          if (!bounded && z > m) {
             const float corr = exp2f(m - z);  // 0 on the first kept key
             l *= corr;
 #pragma unroll
