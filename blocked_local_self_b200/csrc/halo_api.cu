@@ -86,6 +86,7 @@ struct TcEntry {
   int (*smem)(int);
   int stage_bytes;
   int parts;
+  int hpb;  // heads per TMA box
 };
 
 template <int D, int WIN, int STRIDE, int PP>
@@ -94,7 +95,7 @@ int tc_smem(int stages) { return halo::tc::smem_bytes<D, WIN, STRIDE, PP>(stages
 #define HALO_TC_ENTRY(D, WIN, S, PP)                                                             \
   TcEntry {                                                                                      \
     D, WIN, S, halo::tc::halo_fwd_tc<D, WIN, S, PP>, tc_smem<D, WIN, S, PP>,                     \
-        halo::tc::Cfg<D, WIN, S, PP>::STAGE_BYTES, PP                                            \
+        halo::tc::Cfg<D, WIN, S, PP>::STAGE_BYTES, PP, halo::tc::Cfg<D, WIN, S, PP>::HPB         \
   }
 #define HALO_TC_WINS(D, S, PP)                                                                  \
   HALO_TC_ENTRY(D, 8, S, PP), HALO_TC_ENTRY(D, 10, S, PP), HALO_TC_ENTRY(D, 12, S, PP),         \
@@ -247,18 +248,20 @@ EncodeTiledFn encoder() {
   return g_encode;
 }
 
-// 4-D map over an NHWC bf16 tensor {C, W, H, N}; box {d, bw, bh, 1}.
-bool encode_nhwc(CUtensorMap* m, const void* base, const Shape& s, int bw, int bh, int estride) {
+// 4-D map over an NHWC bf16 tensor {C, W, H, N}; box {hpb * d, bw, bh, 1}
+// (hpb heads' channels per box row), swizzled by the box row's width.
+bool encode_nhwc(CUtensorMap* m, const void* base, const Shape& s, int bw, int bh, int estride, int hpb = 1) {
   EncodeTiledFn enc = encoder();
   if (!enc) return false;
   const cuuint64_t C = static_cast<cuuint64_t>(s.heads) * s.d;
   cuuint64_t dims[4] = {C, static_cast<cuuint64_t>(s.W), static_cast<cuuint64_t>(s.H),
                         static_cast<cuuint64_t>(s.N)};
   cuuint64_t strides[3] = {C * 2, C * 2 * s.W, C * 2 * s.W * s.H};
-  cuuint32_t box[4] = {static_cast<cuuint32_t>(s.d), static_cast<cuuint32_t>(bw), static_cast<cuuint32_t>(bh), 1};
+  const int inner = s.d * hpb;
+  cuuint32_t box[4] = {static_cast<cuuint32_t>(inner), static_cast<cuuint32_t>(bw), static_cast<cuuint32_t>(bh), 1};
   cuuint32_t es[4] = {1, static_cast<cuuint32_t>(estride), static_cast<cuuint32_t>(estride), 1};
-  const CUtensorMapSwizzle sw = s.d == 16 ? CU_TENSOR_MAP_SWIZZLE_32B
-                                          : (s.d == 32 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_128B);
+  const CUtensorMapSwizzle sw = inner == 16 ? CU_TENSOR_MAP_SWIZZLE_32B
+                                            : (inner == 32 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_128B);
   return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, strides, box, es,
              CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
@@ -419,8 +422,8 @@ int launch_tc(const TcEntry& e, const void* q, const void* k, const void* v, con
               void* out, const Shape& s, int sm_count, cudaStream_t st) {
   const int win = s.block + 2 * s.halo;
   CUtensorMap mq, mk, mv;
-  if (!encode_nhwc(&mq, q, s, halo::tc::kBlock, halo::tc::kBlock, s.stride) ||
-      !encode_nhwc(&mk, k, s, win, win, 1) || !encode_nhwc(&mv, v, s, halo::tc::kRowKeys, win, 1))
+  if (!encode_nhwc(&mq, q, s, halo::tc::kBlock, halo::tc::kBlock, s.stride, e.hpb) ||
+      !encode_nhwc(&mk, k, s, win, win, 1, e.hpb) || !encode_nhwc(&mv, v, s, halo::tc::kRowKeys, win, 1, e.hpb))
     return HALO_ERR_CUDA;
   halo::tc::Params p;
   fill_common(p, rh, rw, out, s);

@@ -196,7 +196,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   float* sDrel = reinterpret_cast<float*>(sWG + 2 * C::WG_BYTES);  // [g][64][D]
   uint8_t* sStage = sWG + 2 * C::WG_BYTES + C::DREL_BYTES;
 
-  __shared__ __align__(8) uint64_t bar_full[4];
+  // The stage of item k lands on bar_full[k % (2S)]: a barrier per stage and
+  // per warpgroup, so that a warpgroup never waits on a barrier whose previous
+  // phase (the other warpgroup's item k - S, at an odd stage count) is still
+  // open, where a parity wait would pass one phase early.
+  __shared__ __align__(8) uint64_t bar_full[8];
   __shared__ __align__(8) uint64_t bar_empty[4];
   __shared__ __align__(8) uint64_t bar_r1[2];
   __shared__ __align__(8) uint64_t bar_r2[2];
@@ -215,6 +219,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (tid == 0) {
     for (int i = 0; i < S; ++i) {
       mbar_init(&bar_full[i], 1);
+      mbar_init(&bar_full[S + i], 1);
       mbar_init(&bar_empty[i], 4);   // the four R3 issuers
     }
     for (int g = 0; g < 2; ++g) {
@@ -280,15 +285,17 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int bx = blk % p.nbx, by = (blk / p.nbx) % p.nby, n = blk / (p.nbx * p.nby);
         uint8_t* st = sStage + s * C::STAGE_BYTES;
         const int x0 = bx * kBlock, y0 = by * kBlock;
-        mbar_arrive_expect_tx(&bar_full[s], C::TX);
-        tma_load_4d(st + C::OFF_Q, &tmap_q, &bar_full[s], head * D, x0, y0, n);
-        tma_load_4d(st + C::OFF_DO, &tmap_do, &bar_full[s], head * D, x0, y0, n);
-        tma_load_4d(st + C::OFF_K, &tmap_k, &bar_full[s], head * D, x0 - p.halo, y0 - p.halo, n);
-        tma_load_4d(st + C::OFF_V, &tmap_v, &bar_full[s], head * D, x0 - p.halo, y0 - p.halo, n);
+        uint64_t* full = &bar_full[k % (2 * S)];
+        mbar_arrive_expect_tx(full, C::TX);
+        tma_load_4d(st + C::OFF_Q, &tmap_q, full, head * D, x0, y0, n);
+        tma_load_4d(st + C::OFF_DO, &tmap_do, full, head * D, x0, y0, n);
+        tma_load_4d(st + C::OFF_K, &tmap_k, full, head * D, x0 - p.halo, y0 - p.halo, n);
+        tma_load_4d(st + C::OFF_V, &tmap_v, full, head * D, x0 - p.halo, y0 - p.halo, n);
         issued = k + 1;
       }
       if (abort_flag) {
-        for (int k = (issued > S ? issued - S : 0); k < issued; ++k) mbar_wait(&bar_full[k % S], (k / S) & 1, kWaitNs);
+        for (int k = (issued > S ? issued - S : 0); k < issued; ++k)
+          mbar_wait(&bar_full[k % (2 * S)], (k / (2 * S)) & 1, kWaitNs);
       }
     }
     __syncwarp();
@@ -337,7 +344,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       // ---- R1: S (warp 0) and G (warp 1), issued in parallel
       if (wq < 2 && lane == 0) {
-        if (mbar_wait(&bar_full[s], (k / S) & 1, kWaitNs, &abort_flag)) {
+        if (mbar_wait(&bar_full[k % (2 * S)], (k / (2 * S)) & 1, kWaitNs, &abort_flag)) {
           tc_fence_after();
           const uint32_t dst = slot + (wq ? kGBase : 0u), ba = wq ? ra : ka;
           const uint32_t id = wq ? idG : idS;

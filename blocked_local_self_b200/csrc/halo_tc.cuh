@@ -23,7 +23,8 @@
 //     relative dot products of every query); after the softmax, warps
 //     q < NST of the owning warpgroup each issue a share of O = P V (window
 //     rows of one head) into their own accumulator, summed in the epilogue
-//     (for d = 16 the row sums come from a ones tile appended to V).
+//     (for d = 16 the row sums come from a ones tile appended to V); with
+//     four heads of d = 32 per tile, one chain over all four V tiles.
 //   * warps 0-3 and 4-7 are two softmax warpgroups that take alternate items;
 //     each owns one half of every TMEM lane quadrant (lanes 0-15 or 16-31), so
 //     the MMAs of one item overlap the softmax of the other.  A query row is
@@ -95,16 +96,31 @@ struct Cfg {
   static constexpr int PARTS = PP;
   static_assert(STRIDE == 2 || PP == 1, "one head per item at stride 1");
   static constexpr int QROWS_PER_HEAD = (STRIDE == 1) ? 64 : 16;
+  // Four heads of d = 32 travel in pairs: one TMA box of 2d channels (128-byte
+  // rows, 128B swizzle) per pair for q, k and v, half the box rows of one box
+  // per head (the TMA unit's cost goes by rows).  A head's K-major operands
+  // then start d*2 bytes into the row for the second head of a pair.
+  static constexpr bool PAIRED = (STRIDE == 2 && PARTS == 4 && D == 32);
+  static constexpr int HPB = PAIRED ? 2 : 1;              // heads per TMA box
+  static constexpr int BOXES = PARTS / HPB;
+  static constexpr int BROWB = ROWB * HPB;                // bytes of one pixel's row in a q/k/v tile
   // stride 1: 64-row Q tile.  stride 2: zero-gap buffer so that the 64-row view
-  // of head p holds its 16 queries in rows 16p..16p+15 and zeros elsewhere.
-  static constexpr int QBUF_ROWS = (STRIDE == 1) ? 64 : (112 + 48 * (PARTS - 1));
+  // of head p holds its 16 queries in rows 16p..16p+15 and zeros elsewhere
+  // (paired: rows [16 zero][pair 0][48 zero][pair 1][16 zero], the views of
+  // the two heads of a pair 16 rows apart).
+  static constexpr int QBUF_ROWS = (STRIDE == 1) ? 64 : (PAIRED ? 112 : (112 + 48 * (PARTS - 1)));
+  // buffer row of box b's first query, first buffer row of head p's view and
+  // the byte offset of head p's channels in a row
+  __host__ __device__ static constexpr int q_row(int b) { return PAIRED ? 16 + 64 * b : 48 + 64 * b; }
+  __host__ __device__ static constexpr int view_row(int p) { return PAIRED ? q_row(p / 2) - 16 * p : 48 + 48 * p; }
+  __host__ __device__ static constexpr int koff(int p) { return ROWB * (p % HPB); }
   static constexpr int KS = WIN * WIN;                    // keys of the window (K tile rows written)
   static constexpr int NS = (KS + 7) / 8 * 8;             // S columns (QK^T N); rows KS..NS-1 zero
   static constexpr int KP = WIN * kRowKeys;               // PV K extent (V tile rows, P columns)
-  static constexpr int K_TILE = NS * ROWB;
-  static constexpr int V_TILE = KP * ROWB;
-  static constexpr int Q_BYTES = QBUF_ROWS * ROWB;
-  static constexpr int STAGE_RAW = Q_BYTES + PARTS * (K_TILE + V_TILE);
+  static constexpr int K_TILE = NS * BROWB;               // one box's K tile
+  static constexpr int V_TILE = KP * BROWB;
+  static constexpr int Q_BYTES = QBUF_ROWS * BROWB;
+  static constexpr int STAGE_RAW = Q_BYTES + BOXES * (K_TILE + V_TILE);
   static constexpr int STAGE_BYTES = (STAGE_RAW + 1023) / 1024 * 1024;
   static constexpr int TX_QK = PARTS * (QROWS_PER_HEAD + KS) * ROWB;  // Q and K of every part
   static constexpr int TX_V = PARTS * KP * ROWB;                       // V of every part
@@ -117,6 +133,8 @@ struct Cfg {
   static constexpr int O_COLS = SUM_BY_MMA ? 2 * D : D;   // PV N
   static constexpr SmemSwizzle SW = (ROWB == 32) ? SW_32B : (ROWB == 64 ? SW_64B : SW_128B);
   static constexpr uint32_t SBO = 8 * ROWB;               // 8-row core-matrix group stride
+  static constexpr SmemSwizzle BSW = (BROWB == 32) ? SW_32B : (BROWB == 64 ? SW_64B : SW_128B);
+  static constexpr uint32_t BSBO = 8 * BROWB;             // the same for the q/k/v tiles
   static constexpr int NROW = WIN / 2;                    // window rows per thread
   // Stride 2 with fewer than 4 parts: warpgroup 1's parts go to the upper
   // lane quadrants (its Q view starts QSHIFT rows earlier), so the two
@@ -128,6 +146,14 @@ struct Cfg {
   static constexpr int NST = (O_COLS * 4 <= (int)kTmemG) ? 4 : 3;
   static constexpr int SPP = NST / PARTS;                 // streams per part
   static_assert(NST % PARTS == 0 && SPP >= 1, "streams per part");
+  // Paired heads: the two pair tiles of V sit V_TILE apart, so one chain with
+  // B = [V_0 V_1 | V_2 V_3] (N = 4d, each pair tile one 64-column N atom, at
+  // leading byte offset V_TILE) replaces the four per-head chains; rows of
+  // head p keep only columns p*d..p*d+d-1, which is where stream p's
+  // accumulator was.  One issuer, a quarter of the MMAs.
+  static constexpr bool AV_ONE_CHAIN = PAIRED;
+  static_assert(!PAIRED || (SPP == 1 && !SUM_BY_MMA), "paired heads: one stream per head");
+  static constexpr int NIS = AV_ONE_CHAIN ? 1 : NST;      // A.V issuers (commits per item)
   static_assert(NST * O_COLS <= (int)kTmemG, "O accumulators below the G columns");
   static_assert(WIN % 2 == 0 && WIN <= 14 && WIN >= 8, "window must be even, 8..14");
   static_assert(D == 16 || D == 32 || D == 64, "dim_head must be 16, 32 or 64");
@@ -202,9 +228,13 @@ __global__ void __launch_bounds__(kThreads, 1)
   // the S and G MMAs finish, long before the A.V releases V, so the next
   // items' Q/K loads are in flight during the softmax.
   __shared__ __align__(8) uint64_t bar_fqk[8];
-  __shared__ __align__(8) uint64_t bar_fv[8];
+  // V of item k lands on bar_fv[k % (2S)]: a barrier per stage and per
+  // warpgroup, so that the A.V issuer of item k never waits on a barrier
+  // whose previous phase (the other warpgroup's item k - 1, at one stage) is
+  // still open, where a parity wait would pass one phase early.
+  __shared__ __align__(8) uint64_t bar_fv[16];
   __shared__ __align__(8) uint64_t bar_eqk[8];  // count 2: the S and the G MMAs
-  __shared__ __align__(8) uint64_t bar_ev[8];   // count NST: the A.V streams
+  __shared__ __align__(8) uint64_t bar_ev[8];   // count NIS: the A.V issuers
   __shared__ __align__(8) uint64_t bar_sfull[4];   // index 2*g + slot
   __shared__ __align__(8) uint64_t bar_pfull[4];
   __shared__ __align__(8) uint64_t bar_ofull[4];
@@ -223,13 +253,14 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int i = 0; i < S; ++i) {
       mbar_init(&bar_fqk[i], 1);
       mbar_init(&bar_fv[i], 1);
+      mbar_init(&bar_fv[S + i], 1);
       mbar_init(&bar_eqk[i], 2);
-      mbar_init(&bar_ev[i], C::NST);
+      mbar_init(&bar_ev[i], C::NIS);
     }
     for (int b = 0; b < 4; ++b) {
       mbar_init(&bar_sfull[b], 2);  // the S MMAs (warp 9) and the G MMAs (warp 10)
       mbar_init(&bar_pfull[b], 4);
-      mbar_init(&bar_ofull[b], C::NST);
+      mbar_init(&bar_ofull[b], C::NIS);
       mbar_init(&bar_tfree[b], 4);
     }
     mbar_init(&bar_done[0], 1);
@@ -265,9 +296,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         reinterpret_cast<uint4*>(st)[idx] = make_uint4(0, 0, 0, 0);
     }
     if constexpr (C::NS > C::KS) {
-      constexpr int tail = (C::NS - C::KS) * C::ROWB / 16;
-      for (int idx = tid; idx < C::PARTS * tail; idx += kThreads) {
-        uint8_t* kt = st + C::Q_BYTES + (idx / tail) * C::K_TILE + C::KS * C::ROWB;
+      constexpr int tail = (C::NS - C::KS) * C::BROWB / 16;
+      for (int idx = tid; idx < C::BOXES * tail; idx += kThreads) {
+        uint8_t* kt = st + C::Q_BYTES + (idx / tail) * C::K_TILE + C::KS * C::BROWB;
         reinterpret_cast<uint4*>(kt)[idx % tail] = make_uint4(0, 0, 0, 0);
       }
     }
@@ -311,11 +342,11 @@ __global__ void __launch_bounds__(kThreads, 1)
           uint8_t* st = sStage + s * C::STAGE_BYTES;
           mbar_arrive_expect_tx(&bar_fqk[s], C::TX_QK);
 #pragma unroll 1
-          for (int part = 0; part < C::PARTS; ++part) {
-            const int head = ic.grp * C::PARTS + part;
-            uint8_t* qdst = st + ((STRIDE == 1) ? 0 : (48 + 64 * part) * C::ROWB);
+          for (int box = 0; box < C::BOXES; ++box) {
+            const int head = ic.grp * C::PARTS + box * C::HPB;
+            uint8_t* qdst = st + ((STRIDE == 1) ? 0 : C::q_row(box) * C::BROWB);
             tma_load_4d(qdst, &tmap_q, &bar_fqk[s], head * D, ic.bx * kBlock, ic.by * kBlock, ic.n);
-            uint8_t* kdst = st + C::Q_BYTES + part * C::K_TILE;
+            uint8_t* kdst = st + C::Q_BYTES + box * C::K_TILE;
             tma_load_4d(kdst, &tmap_k, &bar_fqk[s], head * D, ic.bx * kBlock - p.halo, ic.by * kBlock - p.halo,
                         ic.n);
           }
@@ -329,12 +360,13 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           const ItemCoord ic = item_coord(blockIdx.x + k * gridDim.x, groups, p.nbx, p.nby);
           uint8_t* st = sStage + s * C::STAGE_BYTES;
-          mbar_arrive_expect_tx(&bar_fv[s], C::TX_V);
+          uint64_t* fv = &bar_fv[k % (2 * S)];
+          mbar_arrive_expect_tx(fv, C::TX_V);
 #pragma unroll 1
-          for (int part = 0; part < C::PARTS; ++part) {
-            const int head = ic.grp * C::PARTS + part;
-            uint8_t* vdst = st + C::Q_BYTES + C::PARTS * C::K_TILE + part * C::V_TILE;
-            tma_load_4d(vdst, &tmap_v, &bar_fv[s], head * D, ic.bx * kBlock - p.halo, ic.by * kBlock - p.halo,
+          for (int box = 0; box < C::BOXES; ++box) {
+            const int head = ic.grp * C::PARTS + box * C::HPB;
+            uint8_t* vdst = st + C::Q_BYTES + C::BOXES * C::K_TILE + box * C::V_TILE;
+            tma_load_4d(vdst, &tmap_v, fv, head * D, ic.bx * kBlock - p.halo, ic.by * kBlock - p.halo,
                         ic.n);
           }
           nv = k + 1;
@@ -343,7 +375,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (abort_flag) {
         // let loads that are still in flight land before the CTA exits
         for (int k = (nqk > S ? nqk - S : 0); k < nqk; ++k) mbar_wait(&bar_fqk[k % S], (k / S) & 1, kWaitNs);
-        for (int k = (nv > S ? nv - S : 0); k < nv; ++k) mbar_wait(&bar_fv[k % S], (k / S) & 1, kWaitNs);
+        for (int k = (nv > S ? nv - S : 0); k < nv; ++k) mbar_wait(&bar_fv[k % (2 * S)], (k / (2 * S)) & 1, kWaitNs);
       }
     }
   } else if (warp == kMmaWarp || warp == kMmaWarp + 1) {
@@ -362,11 +394,11 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll 1
           for (int part = 0; part < C::PARTS; ++part) {
             const uint32_t qa =
-                smem_addr(st + ((STRIDE == 1) ? 0 : (48 + 48 * part - g * C::QSHIFT) * C::ROWB));
-            const uint32_t ka = smem_addr(st + C::Q_BYTES + part * C::K_TILE);
+                smem_addr(st + ((STRIDE == 1) ? 0 : (C::view_row(part) - g * C::QSHIFT) * C::BROWB) + C::koff(part));
+            const uint32_t ka = smem_addr(st + C::Q_BYTES + (part / C::HPB) * C::K_TILE + C::koff(part));
             for (int ks = 0; ks < D / 16; ++ks) {
-              mma_f16_ss(dst, smem_desc(qa + 32 * ks, 16, C::SBO, C::SW),
-                         smem_desc(ka + 32 * ks, 16, C::SBO, C::SW), idS, (part | ks) != 0);
+              mma_f16_ss(dst, smem_desc(qa + 32 * ks, 16, C::BSBO, C::BSW),
+                         smem_desc(ka + 32 * ks, 16, C::BSBO, C::BSW), idS, (part | ks) != 0);
             }
           }
           mma_commit(&bar_sfull[2 * g + sl]);
@@ -376,9 +408,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t ra = smem_addr(sR);
 #pragma unroll 1
         for (int part = 0; part < C::PARTS; ++part) {
-          const uint32_t qa = smem_addr(st + ((STRIDE == 1) ? 0 : (48 + 48 * part - g * C::QSHIFT) * C::ROWB));
+          const uint32_t qa =
+              smem_addr(st + ((STRIDE == 1) ? 0 : (C::view_row(part) - g * C::QSHIFT) * C::BROWB) + C::koff(part));
           for (int ks = 0; ks < D / 16; ++ks) {
-            mma_f16_ss(dst + kTmemG, smem_desc(qa + 32 * ks, 16, C::SBO, C::SW),
+            mma_f16_ss(dst + kTmemG, smem_desc(qa + 32 * ks, 16, C::BSBO, C::BSW),
                        smem_desc(ra + 32 * ks, 16, C::SBO, C::SW), idG, (part | ks) != 0);
           }
         }
@@ -426,7 +459,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int qx = (STRIDE == 1) ? (row & 7) : 2 * (r16 & 3);
     const float c = p.c;
     const int C_all = p.heads * D;
-    const uint32_t idO = idesc_bf16_f32(64, C::O_COLS, true);
+    const uint32_t idO = idesc_bf16_f32(64, C::AV_ONE_CHAIN ? C::PARTS * D : C::O_COLS, true);
 
     // Epilogue of a finished item: O (and row sums) from its TMEM slot,
     // normalise, bf16, store; then hand the slot back to the MMA warp.
@@ -613,26 +646,26 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       __syncwarp();
       if (lane == 0) mbar_arrive(&bar_pfull[b]);
-      // ---- A.V: warp wq < NST issues its share once the whole P tile is written
+      // ---- A.V: warp wq < NIS issues its share once the whole P tile is written
       bool issued = true;
-      if (wq < C::NST && lane == 0) {
+      if (wq < C::NIS && lane == 0) {
         issued = mbar_wait(&bar_pfull[b], (j >> 1) & 1, kWaitNs, &abort_flag) &&
-                 mbar_wait(&bar_fv[k % S], (k / S) & 1, kWaitNs, &abort_flag);
+                 mbar_wait(&bar_fv[k % (2 * S)], (k / (2 * S)) & 1, kWaitNs, &abort_flag);
         if (issued) {
           tc_fence_after();
           const int s = k % S, part = wq / C::SPP, sub = wq % C::SPP;
           const int kb = WIN * sub / C::SPP, ke = WIN * (sub + 1) / C::SPP;
           const uint32_t dst = tmem + (static_cast<uint32_t>(g * 16) << 16) + sl * kSlotCols + wq * C::O_COLS;
           const uint32_t pa = smem_addr(pt);
-          const uint32_t va = smem_addr(sStage + s * C::STAGE_BYTES + C::Q_BYTES + C::PARTS * C::K_TILE +
+          const uint32_t va = smem_addr(sStage + s * C::STAGE_BYTES + C::Q_BYTES + C::BOXES * C::K_TILE +
                                         part * C::V_TILE);
           // with the ones tile the B operand spans two swizzle atoms along N:
           // V (D columns) then ones (D columns) at leading byte offset LBO
-          const uint32_t lbo = C::SUM_BY_MMA ? (smem_addr(sOnes) - va) : 16u;
+          const uint32_t lbo = C::SUM_BY_MMA ? (smem_addr(sOnes) - va) : (C::AV_ONE_CHAIN ? C::V_TILE : 16u);
 #pragma unroll 1
           for (int kk = kb; kk < ke; ++kk)
             mma_f16_ss(dst, smem_desc(pa + kk * 2048, 16, 256, SW_32B),
-                       smem_desc(va + kk * kRowKeys * C::ROWB, lbo, C::SBO, C::SW), idO, kk != kb);
+                       smem_desc(va + kk * kRowKeys * C::BROWB, lbo, C::BSBO, C::BSW), idO, kk != kb);
           mma_commit(&bar_ofull[b]);
           mma_commit(&bar_ev[s]);
         }

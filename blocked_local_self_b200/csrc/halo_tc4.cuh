@@ -339,7 +339,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   // the S and G MMAs finish, long before the A.V releases V, so the next
   // items' Q/K loads are in flight during the softmax.
   __shared__ __align__(8) uint64_t bar_fqk[4];
-  __shared__ __align__(8) uint64_t bar_fv[4];
+  // V of item k lands on bar_fv[k % (2S)]: a barrier per stage and per
+  // warpgroup, so that the A.V issuers of item k never wait on a barrier whose
+  // previous phase (the other warpgroup's item k - S, at an odd stage count)
+  // is still open, where a parity wait would pass one phase early.
+  __shared__ __align__(8) uint64_t bar_fv[8];
   __shared__ __align__(8) uint64_t bar_eqk[4];  // count 3: S_A, S_B, G
   __shared__ __align__(8) uint64_t bar_ev[4];   // count 4: the A.V chains
   __shared__ __align__(8) uint64_t bar_sfull[2];   // count 2: the two blocks' S MMAs
@@ -362,6 +366,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int i = 0; i < S; ++i) {
       mbar_init(&bar_fqk[i], 1);
       mbar_init(&bar_fv[i], 1);
+      mbar_init(&bar_fv[S + i], 1);
       mbar_init(&bar_eqk[i], 3);
       mbar_init(&bar_ev[i], 4);
     }
@@ -447,15 +452,16 @@ __global__ void __launch_bounds__(kThreads, 1)
           const ItemCoord ic = item_coord(blockIdx.x + k * gridDim.x, p.heads, p.nbx, p.npy);
           uint8_t* st = sStage + s * C::STAGE_BYTES;
           const int x0 = ic.bx * kBlock, y0 = ic.py * 2 * kBlock;
-          mbar_arrive_expect_tx(&bar_fv[s], C::TX_V);
-          tma_load_4d(st + OFF_V, &tmap_v, &bar_fv[s], ic.head * D, x0 - p.halo, y0 - p.halo, ic.n);
+          uint64_t* fv = &bar_fv[k % (2 * S)];
+          mbar_arrive_expect_tx(fv, C::TX_V);
+          tma_load_4d(st + OFF_V, &tmap_v, fv, ic.head * D, x0 - p.halo, y0 - p.halo, ic.n);
           nv = k + 1;
         }
       }
       if (abort_flag) {
         // loads still in flight land before the block exits
         for (int k = (nqk > S ? nqk - S : 0); k < nqk; ++k) mbar_wait(&bar_fqk[k % S], (k / S) & 1, kWaitNs);
-        for (int k = (nv > S ? nv - S : 0); k < nv; ++k) mbar_wait(&bar_fv[k % S], (k / S) & 1, kWaitNs);
+        for (int k = (nv > S ? nv - S : 0); k < nv; ++k) mbar_wait(&bar_fv[k % (2 * S)], (k / (2 * S)) & 1, kWaitNs);
       }
     }
   } else {
@@ -624,7 +630,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
       // ---- A.V: warp wq issues block (wq & 1), key half (wq >> 1)
       const int s = k % S;
-      if (lane == 0 && !mbar_wait(&bar_fv[s], (k / S) & 1, kWaitNs, &abort_flag)) {
+      if (lane == 0 && !mbar_wait(&bar_fv[k % (2 * S)], (k / (2 * S)) & 1, kWaitNs, &abort_flag)) {
         if (!abort_flag) record_timeout(&abort_flag);
       } else if (lane == 0) {
         const int ab = wq & 1, hf = wq >> 1;
