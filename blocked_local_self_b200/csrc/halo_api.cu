@@ -433,8 +433,9 @@ int launch_tc(const TcEntry& e, const void* q, const void* k, const void* v, con
   p.OH = s.H / s.stride;
   p.OW = s.W / s.stride;
   const long long items = static_cast<long long>(s.N) * p.nbx * p.nby * (s.heads / e.parts);
-  return launch_persistent(e.fn, halo::tc::kThreads, halo::tc::kSoftmaxRegs, halo::tc::kProducerRegs, e.smem, 8,
-                           mq, mk, mv, p, items, sm_count, st);
+  // eight V-buffer barriers: paired heads have two V buffers per stage
+  return launch_persistent(e.fn, halo::tc::kThreads, halo::tc::kSoftmaxRegs, halo::tc::kProducerRegs, e.smem,
+                           e.hpb == 2 ? 4 : 8, mq, mk, mv, p, items, sm_count, st);
 }
 
 int launch_tc2(const Tc2Entry& e, const void* q, const void* k, const void* v, const void* rh, const void* rw,

@@ -120,11 +120,20 @@ struct Cfg {
   static constexpr int K_TILE = NS * BROWB;               // one box's K tile
   static constexpr int V_TILE = KP * BROWB;
   static constexpr int Q_BYTES = QBUF_ROWS * BROWB;
-  static constexpr int STAGE_RAW = Q_BYTES + BOXES * (K_TILE + V_TILE);
+  // Paired heads keep P in TMEM (bf16 over the first S columns, the A operand
+  // of a TMEM-A MMA), and the shared memory the P tiles took holds a second V
+  // buffer: a stage is [Q | K of every box] then VPS V buffers, so the V of
+  // item k + 1 loads while the A.V of item k runs.
+  static constexpr int VPS = PAIRED ? 2 : 1;              // V buffers per stage
+  static constexpr int QK_BYTES = Q_BYTES + BOXES * K_TILE;
+  static constexpr int VB_BYTES = BOXES * V_TILE;
+  static constexpr int STAGE_RAW = QK_BYTES + VPS * VB_BYTES;
   static constexpr int STAGE_BYTES = (STAGE_RAW + 1023) / 1024 * 1024;
+  static_assert(!PAIRED || (QK_BYTES % 1024 == 0 && VB_BYTES % 1024 == 0), "1 KB aligned tiles");
   static constexpr int TX_QK = PARTS * (QROWS_PER_HEAD + KS) * ROWB;  // Q and K of every part
   static constexpr int TX_V = PARTS * KP * ROWB;                       // V of every part
   static constexpr int P_TILE = WIN * 2048;               // 64 rows x 16 keys x 2 B per window row
+  static constexpr int P_SMEM = PAIRED ? 0 : 2 * P_TILE;  // P tiles in shared memory (one per warpgroup)
   static constexpr int R_TILE = kGCols * ROWB;            // [rel_h; 0; rel_w; 0] B operand
   static constexpr int SCRATCH_LINE = 36;                 // floats per (row, half) line of the gather scratch
   static constexpr int SCRATCH = 8 * 32 * SCRATCH_LINE * 4;
@@ -154,6 +163,10 @@ struct Cfg {
   static constexpr bool AV_ONE_CHAIN = PAIRED;
   static_assert(!PAIRED || (SPP == 1 && !SUM_BY_MMA), "paired heads: one stream per head");
   static constexpr int NIS = AV_ONE_CHAIN ? 1 : NST;      // A.V issuers (commits per item)
+  // first O column of a slot: paired, P (8 columns per window row) sits at
+  // [0, 8w) and O at [128, 256), over S's tail and G, both read by then
+  static constexpr int O_BASE = PAIRED ? 128 : 0;
+  static_assert(!PAIRED || (8 * WIN <= O_BASE && O_BASE + PARTS * D <= (int)kSlotCols), "paired TMEM slot");
   static_assert(NST * O_COLS <= (int)kTmemG, "O accumulators below the G columns");
   static_assert(WIN % 2 == 0 && WIN <= 14 && WIN >= 8, "window must be even, 8..14");
   static_assert(D == 16 || D == 32 || D == 64, "dim_head must be 16, 32 or 64");
@@ -165,7 +178,7 @@ struct Cfg {
 template <int D, int WIN, int STRIDE, int PP>
 __host__ __device__ constexpr int smem_bytes(int stages) {
   using C = Cfg<D, WIN, STRIDE, PP>;
-  return 1024 + 2 * C::P_TILE + C::SCRATCH + ((C::R_TILE + 1023) / 1024) * 1024 + stages * C::STAGE_BYTES +
+  return 1024 + C::P_SMEM + C::SCRATCH + ((C::R_TILE + 1023) / 1024) * 1024 + stages * C::STAGE_BYTES +
          C::ONES_TILE;
 }
 
@@ -216,9 +229,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   using C = Cfg<D, WIN, STRIDE, PP>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint8_t* sP = smem;                                          // 2 x P_TILE (one per warpgroup)
-  float* sScratch = reinterpret_cast<float*>(sP + 2 * C::P_TILE);  // relative-logit gather scratch
-  uint8_t* sR = sP + 2 * C::P_TILE + C::SCRATCH;               // R tile (1 KB aligned)
+  uint8_t* sP = smem;                                          // P tiles (one per warpgroup) unless in TMEM
+  float* sScratch = reinterpret_cast<float*>(sP + C::P_SMEM);  // relative-logit gather scratch
+  uint8_t* sR = sP + C::P_SMEM + C::SCRATCH;                   // R tile (1 KB aligned)
   uint8_t* sStage = sR + ((C::R_TILE + 1023) / 1024) * 1024;   // stages x STAGE_BYTES
   // ones tile (d = 16) after the stages: the PV B descriptor reaches it with a
   // positive leading byte offset from any V tile
@@ -228,13 +241,13 @@ __global__ void __launch_bounds__(kThreads, 1)
   // the S and G MMAs finish, long before the A.V releases V, so the next
   // items' Q/K loads are in flight during the softmax.
   __shared__ __align__(8) uint64_t bar_fqk[8];
-  // V of item k lands on bar_fv[k % (2S)]: a barrier per stage and per
+  // V of item k lands on bar_fv[k % (2 SVB)]: a barrier per V buffer and per
   // warpgroup, so that the A.V issuer of item k never waits on a barrier
-  // whose previous phase (the other warpgroup's item k - 1, at one stage) is
-  // still open, where a parity wait would pass one phase early.
+  // whose previous phase (the other warpgroup's item k - 1, with one buffer)
+  // is still open, where a parity wait would pass one phase early.
   __shared__ __align__(8) uint64_t bar_fv[16];
   __shared__ __align__(8) uint64_t bar_eqk[8];  // count 2: the S and the G MMAs
-  __shared__ __align__(8) uint64_t bar_ev[8];   // count NIS: the A.V issuers
+  __shared__ __align__(8) uint64_t bar_ev[8];   // V buffer free; count NIS: the A.V issuers
   __shared__ __align__(8) uint64_t bar_sfull[4];   // index 2*g + slot
   __shared__ __align__(8) uint64_t bar_pfull[4];
   __shared__ __align__(8) uint64_t bar_ofull[4];
@@ -247,14 +260,21 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int warp = tid >> 5;
   const int lane = tid & 31;
   const int S = p.stages;
+  const int SVB = C::VPS * S;  // V buffers: item k's V in buffer k % SVB
+  auto vbuf = [&](int k) -> uint8_t* {
+    const int vb = k % SVB;
+    return sStage + (vb / C::VPS) * C::STAGE_BYTES + C::QK_BYTES + (vb % C::VPS) * C::VB_BYTES;
+  };
 
   // ---------------------------------------------------------------- set-up
   if (tid == 0) {
     for (int i = 0; i < S; ++i) {
       mbar_init(&bar_fqk[i], 1);
-      mbar_init(&bar_fv[i], 1);
-      mbar_init(&bar_fv[S + i], 1);
       mbar_init(&bar_eqk[i], 2);
+    }
+    for (int i = 0; i < SVB; ++i) {
+      mbar_init(&bar_fv[i], 1);
+      mbar_init(&bar_fv[SVB + i], 1);
       mbar_init(&bar_ev[i], C::NIS);
     }
     for (int b = 0; b < 4; ++b) {
@@ -353,19 +373,19 @@ __global__ void __launch_bounds__(kThreads, 1)
           nqk = t + 1;
         }
         if (t >= 1) {
-          const int k = t - 1, s = k % S;
-          if (k >= S && !mbar_wait(&bar_ev[s], ((k / S) - 1) & 1, kWaitNs, &abort_flag)) {
+          const int k = t - 1, vb = k % SVB;
+          if (k >= SVB && !mbar_wait(&bar_ev[vb], ((k / SVB) - 1) & 1, kWaitNs, &abort_flag)) {
             if (!abort_flag) record_timeout(&abort_flag);
             break;
           }
           const ItemCoord ic = item_coord(blockIdx.x + k * gridDim.x, groups, p.nbx, p.nby);
-          uint8_t* st = sStage + s * C::STAGE_BYTES;
-          uint64_t* fv = &bar_fv[k % (2 * S)];
+          uint8_t* vt = vbuf(k);
+          uint64_t* fv = &bar_fv[k % (2 * SVB)];
           mbar_arrive_expect_tx(fv, C::TX_V);
 #pragma unroll 1
           for (int box = 0; box < C::BOXES; ++box) {
             const int head = ic.grp * C::PARTS + box * C::HPB;
-            uint8_t* vdst = st + C::Q_BYTES + C::BOXES * C::K_TILE + box * C::V_TILE;
+            uint8_t* vdst = vt + box * C::V_TILE;
             tma_load_4d(vdst, &tmap_v, fv, head * D, ic.bx * kBlock - p.halo, ic.by * kBlock - p.halo,
                         ic.n);
           }
@@ -375,7 +395,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (abort_flag) {
         // let loads that are still in flight land before the CTA exits
         for (int k = (nqk > S ? nqk - S : 0); k < nqk; ++k) mbar_wait(&bar_fqk[k % S], (k / S) & 1, kWaitNs);
-        for (int k = (nv > S ? nv - S : 0); k < nv; ++k) mbar_wait(&bar_fv[k % (2 * S)], (k / (2 * S)) & 1, kWaitNs);
+        for (int k = (nv > SVB ? nv - SVB : 0); k < nv; ++k)
+          mbar_wait(&bar_fv[k % (2 * SVB)], (k / (2 * SVB)) & 1, kWaitNs);
       }
     }
   } else if (warp == kMmaWarp || warp == kMmaWarp + 1) {
@@ -479,7 +500,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         if constexpr (D == 16) l = 0.f;
 #pragma unroll 1
         for (int q = q0; q < q0 + ((STRIDE == 1) ? C::NST : C::SPP); ++q) {
-          const uint32_t oaddr = tq + (jj & 1) * kSlotCols + q * C::O_COLS;
+          const uint32_t oaddr = tq + (jj & 1) * kSlotCols + C::O_BASE + q * C::O_COLS;
           if constexpr (D == 16) {
             uint32_t r[8];
             tmem_ld_16x32bx2_x8<8>(oaddr, r);
@@ -635,14 +656,25 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
             for (int kc = 0; kc < WIN; ++kc) l += e[kc];
           }
-          const int kr = 2 * i + half;
-          uint8_t* dst = pt + kr * 2048 + row * 32;
-          const int sw = (row >> 2) & 1;
-          *reinterpret_cast<uint4*>(dst + (sw << 4)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
-          *reinterpret_cast<uint4*>(dst + ((sw ^ 1) << 4)) = make_uint4(pk[4], pk[5], pk[6], pk[7]);
+          if constexpr (C::PAIRED) {
+            // window rows 2i (this lane < 16) and 2i + 1 (its partner) at
+            // columns 16i and 16i + 8: 8 columns of bf16 pairs per K-step
+            tmem_st_16x32bx2_x8<8>(ts + 16 * i, pk);
+          } else {
+            const int kr = 2 * i + half;
+            uint8_t* dst = pt + kr * 2048 + row * 32;
+            const int sw = (row >> 2) & 1;
+            *reinterpret_cast<uint4*>(dst + (sw << 4)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+            *reinterpret_cast<uint4*>(dst + ((sw ^ 1) << 4)) = make_uint4(pk[4], pk[5], pk[6], pk[7]);
+          }
         }
         if constexpr (!C::SUM_BY_MMA) l += __shfl_xor_sync(0xffffffffu, l, 16);
-        fence_proxy_async_smem();
+        if constexpr (C::PAIRED) {
+          tmem_wait_st();
+          tc_fence_before();
+        } else {
+          fence_proxy_async_smem();
+        }
       }
       __syncwarp();
       if (lane == 0) mbar_arrive(&bar_pfull[b]);
@@ -650,24 +682,31 @@ __global__ void __launch_bounds__(kThreads, 1)
       bool issued = true;
       if (wq < C::NIS && lane == 0) {
         issued = mbar_wait(&bar_pfull[b], (j >> 1) & 1, kWaitNs, &abort_flag) &&
-                 mbar_wait(&bar_fv[k % (2 * S)], (k / (2 * S)) & 1, kWaitNs, &abort_flag);
+                 mbar_wait(&bar_fv[k % (2 * SVB)], (k / (2 * SVB)) & 1, kWaitNs, &abort_flag);
         if (issued) {
           tc_fence_after();
-          const int s = k % S, part = wq / C::SPP, sub = wq % C::SPP;
+          const int part = wq / C::SPP, sub = wq % C::SPP;
           const int kb = WIN * sub / C::SPP, ke = WIN * (sub + 1) / C::SPP;
-          const uint32_t dst = tmem + (static_cast<uint32_t>(g * 16) << 16) + sl * kSlotCols + wq * C::O_COLS;
-          const uint32_t pa = smem_addr(pt);
-          const uint32_t va = smem_addr(sStage + s * C::STAGE_BYTES + C::Q_BYTES + C::BOXES * C::K_TILE +
-                                        part * C::V_TILE);
+          const uint32_t slot = tmem + (static_cast<uint32_t>(g * 16) << 16) + sl * kSlotCols;
+          const uint32_t dst = slot + C::O_BASE + wq * C::O_COLS;
+          const uint32_t va = smem_addr(vbuf(k) + part * C::V_TILE);
           // with the ones tile the B operand spans two swizzle atoms along N:
           // V (D columns) then ones (D columns) at leading byte offset LBO
           const uint32_t lbo = C::SUM_BY_MMA ? (smem_addr(sOnes) - va) : (C::AV_ONE_CHAIN ? C::V_TILE : 16u);
+          if constexpr (C::PAIRED) {
 #pragma unroll 1
-          for (int kk = kb; kk < ke; ++kk)
-            mma_f16_ss(dst, smem_desc(pa + kk * 2048, 16, 256, SW_32B),
-                       smem_desc(va + kk * kRowKeys * C::BROWB, lbo, C::BSBO, C::BSW), idO, kk != kb);
+            for (int kk = kb; kk < ke; ++kk)
+              mma_f16_ts(dst, slot + 8 * kk, smem_desc(va + kk * kRowKeys * C::BROWB, lbo, C::BSBO, C::BSW), idO,
+                         kk != kb);
+          } else {
+            const uint32_t pa = smem_addr(pt);
+#pragma unroll 1
+            for (int kk = kb; kk < ke; ++kk)
+              mma_f16_ss(dst, smem_desc(pa + kk * 2048, 16, 256, SW_32B),
+                         smem_desc(va + kk * kRowKeys * C::BROWB, lbo, C::BSBO, C::BSW), idO, kk != kb);
+          }
           mma_commit(&bar_ofull[b]);
-          mma_commit(&bar_ev[s]);
+          mma_commit(&bar_ev[k % SVB]);
         }
       }
       if (!__all_sync(0xffffffffu, issued)) {
