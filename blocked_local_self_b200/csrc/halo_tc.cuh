@@ -131,6 +131,13 @@ struct Cfg {
   static constexpr int STAGE_BYTES = (STAGE_RAW + 1023) / 1024 * 1024;
   static_assert(!PAIRED || (QK_BYTES % 1024 == 0 && VB_BYTES % 1024 == 0), "1 KB aligned tiles");
   static constexpr int TX_QK = PARTS * (QROWS_PER_HEAD + KS) * ROWB;  // Q and K of every part
+  // Q/K barrier groups per stage: paired, one per pair, so that the S and G
+  // MMAs of heads 0-1 start once their pair has landed and the pair's next
+  // load starts once those MMAs are done (the two pairs' loads and MMAs
+  // pipeline at half-item granularity)
+  static constexpr int QKG = PAIRED ? BOXES : 1;
+  static constexpr int TX_QKG = TX_QK / QKG;
+  static constexpr int BPG = BOXES / QKG;                 // boxes per group
   static constexpr int TX_V = PARTS * KP * ROWB;                       // V of every part
   static constexpr int P_TILE = WIN * 2048;               // 64 rows x 16 keys x 2 B per window row
   static constexpr int P_SMEM = PAIRED ? 0 : 2 * P_TILE;  // P tiles in shared memory (one per warpgroup)
@@ -240,13 +247,13 @@ __global__ void __launch_bounds__(kThreads, 1)
   // Q/K and V of a stage have their own barriers: Q and K are released when
   // the S and G MMAs finish, long before the A.V releases V, so the next
   // items' Q/K loads are in flight during the softmax.
-  __shared__ __align__(8) uint64_t bar_fqk[8];
+  __shared__ __align__(8) uint64_t bar_fqk[16];  // index QKG * stage + group
   // V of item k lands on bar_fv[k % (2 SVB)]: a barrier per V buffer and per
   // warpgroup, so that the A.V issuer of item k never waits on a barrier
   // whose previous phase (the other warpgroup's item k - 1, with one buffer)
   // is still open, where a parity wait would pass one phase early.
   __shared__ __align__(8) uint64_t bar_fv[16];
-  __shared__ __align__(8) uint64_t bar_eqk[8];  // count 2: the S and the G MMAs
+  __shared__ __align__(8) uint64_t bar_eqk[16];  // count 2: the S and the G MMAs of the group
   __shared__ __align__(8) uint64_t bar_ev[8];   // V buffer free; count NIS: the A.V issuers
   __shared__ __align__(8) uint64_t bar_sfull[4];   // index 2*g + slot
   __shared__ __align__(8) uint64_t bar_pfull[4];
@@ -269,8 +276,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   // ---------------------------------------------------------------- set-up
   if (tid == 0) {
     for (int i = 0; i < S; ++i) {
-      mbar_init(&bar_fqk[i], 1);
-      mbar_init(&bar_eqk[i], 2);
+      for (int q = 0; q < C::QKG; ++q) {
+        mbar_init(&bar_fqk[C::QKG * i + q], 1);
+        mbar_init(&bar_eqk[C::QKG * i + q], 2);
+      }
     }
     for (int i = 0; i < SVB; ++i) {
       mbar_init(&bar_fv[i], 1);
@@ -350,27 +359,33 @@ __global__ void __launch_bounds__(kThreads, 1)
     // issue order QK(0), QK(1), V(0), QK(2), V(1), ...: the Q/K of an item
     // go out one item ahead of the V it does not need until its A.V
     if (lane == 0) {
-      int nqk = 0, nv = 0;
+      int nv = 0, nqkg = 0;  // items with V loads, groups with Q/K loads issued
       for (int t = 0; t <= my_items; ++t) {
         if (t < my_items) {
           const int s = t % S;
-          if (t >= S && !mbar_wait(&bar_eqk[s], ((t / S) - 1) & 1, kWaitNs, &abort_flag)) {
+          const ItemCoord ic = item_coord(blockIdx.x + t * gridDim.x, groups, p.nbx, p.nby);
+          uint8_t* st = sStage + s * C::STAGE_BYTES;
+          bool waited = true;
+#pragma unroll 1
+          for (int q = 0; q < C::QKG && waited; ++q) {
+            uint64_t* fqk = &bar_fqk[C::QKG * s + q];
+            waited = t < S || mbar_wait(&bar_eqk[C::QKG * s + q], ((t / S) - 1) & 1, kWaitNs, &abort_flag);
+            if (!waited) break;
+            mbar_arrive_expect_tx(fqk, C::TX_QKG);
+#pragma unroll 1
+            for (int box = q * C::BPG; box < (q + 1) * C::BPG; ++box) {
+              const int head = ic.grp * C::PARTS + box * C::HPB;
+              uint8_t* qdst = st + ((STRIDE == 1) ? 0 : C::q_row(box) * C::BROWB);
+              tma_load_4d(qdst, &tmap_q, fqk, head * D, ic.bx * kBlock, ic.by * kBlock, ic.n);
+              uint8_t* kdst = st + C::Q_BYTES + box * C::K_TILE;
+              tma_load_4d(kdst, &tmap_k, fqk, head * D, ic.bx * kBlock - p.halo, ic.by * kBlock - p.halo, ic.n);
+            }
+            nqkg = C::QKG * t + q + 1;
+          }
+          if (!waited) {
             if (!abort_flag) record_timeout(&abort_flag);
             break;
           }
-          const ItemCoord ic = item_coord(blockIdx.x + t * gridDim.x, groups, p.nbx, p.nby);
-          uint8_t* st = sStage + s * C::STAGE_BYTES;
-          mbar_arrive_expect_tx(&bar_fqk[s], C::TX_QK);
-#pragma unroll 1
-          for (int box = 0; box < C::BOXES; ++box) {
-            const int head = ic.grp * C::PARTS + box * C::HPB;
-            uint8_t* qdst = st + ((STRIDE == 1) ? 0 : C::q_row(box) * C::BROWB);
-            tma_load_4d(qdst, &tmap_q, &bar_fqk[s], head * D, ic.bx * kBlock, ic.by * kBlock, ic.n);
-            uint8_t* kdst = st + C::Q_BYTES + box * C::K_TILE;
-            tma_load_4d(kdst, &tmap_k, &bar_fqk[s], head * D, ic.bx * kBlock - p.halo, ic.by * kBlock - p.halo,
-                        ic.n);
-          }
-          nqk = t + 1;
         }
         if (t >= 1) {
           const int k = t - 1, vb = k % SVB;
@@ -394,7 +409,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       if (abort_flag) {
         // let loads that are still in flight land before the CTA exits
-        for (int k = (nqk > S ? nqk - S : 0); k < nqk; ++k) mbar_wait(&bar_fqk[k % S], (k / S) & 1, kWaitNs);
+        for (int u = (nqkg > C::QKG * S ? nqkg - C::QKG * S : 0); u < nqkg; ++u) {
+          const int k = u / C::QKG, q = u % C::QKG;
+          mbar_wait(&bar_fqk[C::QKG * (k % S) + q], (k / S) & 1, kWaitNs);
+        }
         for (int k = (nv > SVB ? nv - SVB : 0); k < nv; ++k)
           mbar_wait(&bar_fv[k % (2 * SVB)], (k / (2 * SVB)) & 1, kWaitNs);
       }
@@ -407,13 +425,15 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint32_t idS = idesc_bf16_f32(64, C::NS, false);
       const uint32_t idG = idesc_bf16_f32(64, kGCols, false);
       // S(k): QK^T and the relative dot products of item k into its TMEM slot.
-      auto issue_s = [&](int k) {
+      // Group q: the heads of its boxes; the last group commits sfull.
+      auto issue_s = [&](int k, int q) {
         const int s = k % S, g = k & 1, sl = (k >> 1) & 1;
         const uint32_t dst = tmem + (static_cast<uint32_t>(g * 16) << 16) + sl * kSlotCols;
         const uint8_t* st = sStage + s * C::STAGE_BYTES;
+        constexpr int PPG = C::PARTS / C::QKG;  // heads per group
         if (!is_g) {
 #pragma unroll 1
-          for (int part = 0; part < C::PARTS; ++part) {
+          for (int part = q * PPG; part < (q + 1) * PPG; ++part) {
             const uint32_t qa =
                 smem_addr(st + ((STRIDE == 1) ? 0 : (C::view_row(part) - g * C::QSHIFT) * C::BROWB) + C::koff(part));
             const uint32_t ka = smem_addr(st + C::Q_BYTES + (part / C::HPB) * C::K_TILE + C::koff(part));
@@ -422,13 +442,13 @@ __global__ void __launch_bounds__(kThreads, 1)
                          smem_desc(ka + 32 * ks, 16, C::BSBO, C::BSW), idS, (part | ks) != 0);
             }
           }
-          mma_commit(&bar_sfull[2 * g + sl]);
-          mma_commit(&bar_eqk[s]);
+          if (q == C::QKG - 1) mma_commit(&bar_sfull[2 * g + sl]);
+          mma_commit(&bar_eqk[C::QKG * s + q]);
           return;
         }
         const uint32_t ra = smem_addr(sR);
 #pragma unroll 1
-        for (int part = 0; part < C::PARTS; ++part) {
+        for (int part = q * PPG; part < (q + 1) * PPG; ++part) {
           const uint32_t qa =
               smem_addr(st + ((STRIDE == 1) ? 0 : (C::view_row(part) - g * C::QSHIFT) * C::BROWB) + C::koff(part));
           for (int ks = 0; ks < D / 16; ++ks) {
@@ -436,21 +456,25 @@ __global__ void __launch_bounds__(kThreads, 1)
                        smem_desc(ra + 32 * ks, 16, C::SBO, C::SW), idG, (part | ks) != 0);
           }
         }
-        mma_commit(&bar_sfull[2 * g + sl]);
-        mma_commit(&bar_eqk[s]);
+        if (q == C::QKG - 1) mma_commit(&bar_sfull[2 * g + sl]);
+        mma_commit(&bar_eqk[C::QKG * s + q]);
       };
       // S(k) needs its stage loaded and the slot's previous item (k - 4)
       // consumed (the A.V MMAs are issued by the softmax warpgroups)
-      for (int ns = 0; ns < my_items; ++ns) {
-        if (!mbar_wait(&bar_fqk[ns % S], (ns / S) & 1, kWaitNs, &abort_flag) ||
-            (ns >= 4 && !mbar_wait(&bar_tfree[2 * (ns & 1) + ((ns >> 1) & 1)], ((ns >> 2) - 1) & 1, kWaitNs,
-                                   &abort_flag))) {
-          if (!abort_flag) record_timeout(&abort_flag);
-          break;
+      bool fine = true;
+      for (int ns = 0; ns < my_items && fine; ++ns) {
+        fine = ns < 4 || mbar_wait(&bar_tfree[2 * (ns & 1) + ((ns >> 1) & 1)], ((ns >> 2) - 1) & 1, kWaitNs,
+                                   &abort_flag);
+#pragma unroll 1
+        for (int q = 0; q < C::QKG && fine; ++q) {
+          fine = mbar_wait(&bar_fqk[C::QKG * (ns % S) + q], (ns / S) & 1, kWaitNs, &abort_flag);
+          if (fine) {
+            tc_fence_after();
+            issue_s(ns, q);
+          }
         }
-        tc_fence_after();
-        issue_s(ns);
       }
+      if (!fine && !abort_flag) record_timeout(&abort_flag);
       // all issued MMAs complete before the CTA frees TMEM
       mma_commit(&bar_done[is_g ? 1 : 0]);
       mbar_wait(&bar_done[is_g ? 1 : 0], 0, kWaitNs);
