@@ -767,29 +767,30 @@ int launch_bwd(const BwdPlan& plan, int d, const void* const* in, void* const* g
   }
 }
 
-// Tensor-core backward: bf16, block 8, stride 1, dim_head 16 or 32, window
-// 8..14: (d, window) -> instantiation.
+// Tensor-core backward: bf16, block 8, stride 1 or 2, dim_head 16 or 32,
+// window 8..14: (d, window, stride) -> instantiation.
 using BwdTcKernel = void (*)(const CUtensorMap, const CUtensorMap, const CUtensorMap, const CUtensorMap,
                              const halo::bwdtc::Params);
 struct BwdTcEntry {
-  int d, win;
+  int d, win, stride;
   BwdTcKernel fn;
   int (*smem)(int);
 };
-template <int D, int WIN>
-int bwdtc_smem(int stages) { return halo::bwdtc::smem_bytes<D, WIN>(stages); }
-#define HALO_BWDTC_ENTRY(D, WIN) \
-  BwdTcEntry { D, WIN, halo::bwdtc::halo_bwd_tc<D, WIN>, bwdtc_smem<D, WIN> }
+template <int D, int WIN, int STRIDE>
+int bwdtc_smem(int stages) { return halo::bwdtc::smem_bytes<D, WIN, STRIDE>(stages); }
+#define HALO_BWDTC_ENTRY(D, WIN, S) \
+  BwdTcEntry { D, WIN, S, halo::bwdtc::halo_bwd_tc<D, WIN, S>, bwdtc_smem<D, WIN, S> }
+#define HALO_BWDTC_WINS(D, S) \
+  HALO_BWDTC_ENTRY(D, 8, S), HALO_BWDTC_ENTRY(D, 10, S), HALO_BWDTC_ENTRY(D, 12, S), HALO_BWDTC_ENTRY(D, 14, S)
 const BwdTcEntry kBwdTcTable[] = {
-    HALO_BWDTC_ENTRY(16, 8), HALO_BWDTC_ENTRY(16, 10), HALO_BWDTC_ENTRY(16, 12), HALO_BWDTC_ENTRY(16, 14),
-    HALO_BWDTC_ENTRY(32, 8), HALO_BWDTC_ENTRY(32, 10), HALO_BWDTC_ENTRY(32, 12), HALO_BWDTC_ENTRY(32, 14),
+    HALO_BWDTC_WINS(16, 1), HALO_BWDTC_WINS(32, 1), HALO_BWDTC_WINS(16, 2), HALO_BWDTC_WINS(32, 2),
 };
 
 const BwdTcEntry* find_bwdtc(const Shape& s) {
-  if (s.dtype != HALO_BF16 || s.block != halo::bwdtc::kBlock || s.stride != 1) return nullptr;
+  if (s.dtype != HALO_BF16 || s.block != halo::bwdtc::kBlock) return nullptr;
   const int win = s.block + 2 * s.halo;
   for (const BwdTcEntry& e : kBwdTcTable)
-    if (e.d == s.d && e.win == win) return &e;
+    if (e.d == s.d && e.win == win && e.stride == s.stride) return &e;
   return nullptr;
 }
 
@@ -797,9 +798,15 @@ int launch_bwdtc(const BwdTcEntry& e, const BwdPlan& plan, const void* const* in
                  const Shape& s, int sm_count, cudaStream_t st) {
   const int win = s.block + 2 * s.halo;
   CUtensorMap mq, mk, mv, mdo;
-  if (!encode_nhwc(&mq, in[0], s, halo::bwdtc::kBlock, halo::bwdtc::kBlock, 1) ||
+  // dout is at the output resolution: its map covers (H, W) / stride, and a
+  // block's box is (8 / stride)^2 output pixels
+  Shape so = s;
+  so.H = s.H / s.stride;
+  so.W = s.W / s.stride;
+  const int ob = halo::bwdtc::kBlock / s.stride;
+  if (!encode_nhwc(&mq, in[0], s, halo::bwdtc::kBlock, halo::bwdtc::kBlock, s.stride) ||
       !encode_nhwc(&mk, in[1], s, win, win, 1) || !encode_nhwc(&mv, in[2], s, win, win, 1) ||
-      !encode_nhwc(&mdo, in[6], s, halo::bwdtc::kBlock, halo::bwdtc::kBlock, 1))
+      !encode_nhwc(&mdo, in[6], so, ob, ob, 1))
     return HALO_ERR_CUDA;
   cudaFuncAttributes attr;
   if (cudaFuncGetAttributes(&attr, reinterpret_cast<const void*>(e.fn)) != cudaSuccess) return HALO_ERR_CUDA;
@@ -1151,7 +1158,10 @@ const char* halo_bwd_kernel_name(int N, int H, int W, int heads, int dim_head, i
   if (bwd_plan(s, &plan) != HALO_OK) {
     std::snprintf(name, sizeof(name), "none");
   } else if (const BwdTcEntry* e = find_bwdtc(s)) {
-    std::snprintf(name, sizeof(name), "halo_bwd_tc<%d,%d>", e->d, e->win);
+    if (e->stride == 1)
+      std::snprintf(name, sizeof(name), "halo_bwd_tc<%d,%d>", e->d, e->win);
+    else
+      std::snprintf(name, sizeof(name), "halo_bwd_tc<%d,%d,%d>", e->d, e->win, e->stride);
   } else {
     std::snprintf(name, sizeof(name), "halo_bwd_simt<%s,%d>", s.dtype == HALO_F32 ? "float" : "bf16", s.d);
   }

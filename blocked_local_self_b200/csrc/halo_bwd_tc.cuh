@@ -1,5 +1,5 @@
 // halo_bwd_tc.cuh -- tensor-core backward of blocked local self-attention with
-// haloing on sm_100a: bf16, 8x8 query blocks, stride 1, dim_head 16 or 32,
+// haloing on sm_100a: bf16, 8x8 query blocks, stride 1 or 2, dim_head 16 or 32,
 // windows 8..14 (HaloNet, "Scaling Local Self-Attention for Parameter
 // Efficient Visual Backbones", sections 2.1-2.2 and appendix A; the blog
 // page's RelPosEmb / HaloAttention index conventions).
@@ -13,7 +13,10 @@
 // that column's rel_w index, and R = [rel_h; 0; rel_w; 0] (64 rows).  All six
 // products are tcgen05 MMAs.
 //
-// Work item = one 8x8 block of one head.  Two warpgroups take alternate items,
+// Work item = one 8x8 block of one head (stride 2: its 16 strided queries in
+// rows 0-15 of the 64-row tiles, rows 16-63 of Q and dout zero and their P,
+// dS and T rows never written, so they add nothing to dK, dV and dR; the
+// window is the stride-1 one).  Two warpgroups take alternate items,
 // each with a 256-column TMEM slot and its own P / dS / T buffers in shared
 // memory; lane 0 of its warps issue its MMAs (independent chains in parallel):
 //   R1  S = Q K^T (M=64, N=w^2 rounded to 8) at slot column 0 and
@@ -90,9 +93,10 @@ struct Params {
   float s;         // 1 / sqrt(d)
 };
 
-template <int D, int WIN>
+template <int D, int WIN, int STRIDE>
 struct Cfg {
   static constexpr int ROWB = D * 2;
+  static constexpr int QR = 64 / (STRIDE * STRIDE);    // query rows a block loads (Q and dout)
   static constexpr int KS = WIN * WIN;                 // window keys
   static constexpr int NS = (KS + 7) / 8 * 8;          // S / dP MMA N
   static constexpr int KP = (KS + 15) / 16 * 16;       // keys incl. padding: dQ K extent
@@ -102,7 +106,7 @@ struct Cfg {
   static constexpr int K_TILE = (KP * ROWB + 1023) / 1024 * 1024;
   static constexpr int OFF_Q = 0, OFF_DO = Q_TILE, OFF_K = 2 * Q_TILE, OFF_V = 2 * Q_TILE + K_TILE;
   static constexpr int STAGE_BYTES = 2 * Q_TILE + 2 * K_TILE;
-  static constexpr int TX = (2 * 64 + 2 * KS) * ROWB;
+  static constexpr int TX = (2 * QR + 2 * KS) * ROWB;
   static constexpr int R_TILE = (kRRows * ROWB + 1023) / 1024 * 1024;
   static constexpr int PBUF = MT * 2 * 8192;           // 64 queries x MT*128 keys, bf16, 8 KB atoms of 64 keys
   static constexpr int TBUF = 8192;                    // 64 queries x 64 table entries
@@ -116,15 +120,16 @@ struct Cfg {
   static constexpr uint32_t SBO = 8 * ROWB;
   static constexpr int HALO = (WIN - kBlock) / 2;
   static_assert(D == 16 || D == 32, "dim_head 16 or 32");
+  static_assert(STRIDE == 1 || STRIDE == 2, "stride 1 or 2");
   static_assert(WIN % 2 == 0 && WIN >= 8 && WIN <= 14, "window 8..14");
   static_assert(NS <= (int)kGBase, "S columns below the relative logits");
   static_assert(COL_DR + D <= kSlotCols, "R3 accumulators in the slot");
   static_assert(2 * WIN - 1 <= kRelW && kRelW + 2 * WIN - 1 <= 56, "relative table rows");
 };
 
-template <int D, int WIN>
+template <int D, int WIN, int STRIDE>
 __host__ __device__ constexpr int smem_bytes(int stages) {
-  using C = Cfg<D, WIN>;
+  using C = Cfg<D, WIN, STRIDE>;
   return 1024 + C::R_TILE + 2 * C::WG_BYTES + C::DREL_BYTES + stages * C::STAGE_BYTES;
 }
 
@@ -183,12 +188,12 @@ __device__ __forceinline__ bool wg_sync(uint64_t* bar, int& ph, int lane, int* a
   return ok;
 }
 
-template <int D, int WIN>
+template <int D, int WIN, int STRIDE>
 __global__ void __launch_bounds__(kThreads, 1)
     halo_bwd_tc(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__ CUtensorMap tmap_k,
                 const __grid_constant__ CUtensorMap tmap_v, const __grid_constant__ CUtensorMap tmap_do,
                 const Params p) {
-  using C = Cfg<D, WIN>;
+  using C = Cfg<D, WIN, STRIDE>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sR = smem;
@@ -256,6 +261,12 @@ __global__ void __launch_bounds__(kThreads, 1)
       reinterpret_cast<uint4*>(st + C::OFF_K + C::KS * C::ROWB)[idx] = make_uint4(0, 0, 0, 0);
       reinterpret_cast<uint4*>(st + C::OFF_V + C::KS * C::ROWB)[idx] = make_uint4(0, 0, 0, 0);
     }
+    // stride 2: Q and dout rows QR..63 (finite, so that the zero P rows
+    // times them stay zero)
+    for (int idx = tid; idx < (64 - C::QR) * C::ROWB / 16; idx += kThreads) {
+      reinterpret_cast<uint4*>(st + C::OFF_Q + C::QR * C::ROWB)[idx] = make_uint4(0, 0, 0, 0);
+      reinterpret_cast<uint4*>(st + C::OFF_DO + C::QR * C::ROWB)[idx] = make_uint4(0, 0, 0, 0);
+    }
   }
   fence_proxy_async_smem();
   if (warp == 0) {
@@ -288,7 +299,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         uint64_t* full = &bar_full[k % (2 * S)];
         mbar_arrive_expect_tx(full, C::TX);
         tma_load_4d(st + C::OFF_Q, &tmap_q, full, head * D, x0, y0, n);
-        tma_load_4d(st + C::OFF_DO, &tmap_do, full, head * D, x0, y0, n);
+        tma_load_4d(st + C::OFF_DO, &tmap_do, full, head * D, x0 / STRIDE, y0 / STRIDE, n);
         tma_load_4d(st + C::OFF_K, &tmap_k, full, head * D, x0 - p.halo, y0 - p.halo, n);
         tma_load_4d(st + C::OFF_V, &tmap_v, full, head * D, x0 - p.halo, y0 - p.halo, n);
         issued = k + 1;
@@ -304,8 +315,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int g = warp >> 2;                 // warpgroup = TMEM slot
     const int wq = warp & 3;                 // lane quadrant
     const bool act = lane < 16;              // M=64 tiles: rows in lanes 0-15 of each quadrant
-    const int row = 16 * wq + (lane & 15);   // query row in the 8x8 block
-    const int qy = row >> 3, qx = row & 7;
+    const int row = 16 * wq + (lane & 15);   // query row in the 8x8 block (stride 2: rows 0-15)
+    // this thread's query (stride 2: rows 0-15, warp 0); at stride 2 the
+    // other rows' P, dS and T are written as zeros every item
+    const bool live = act && (STRIDE == 1 || wq == 0);
+    const int qy = STRIDE == 1 ? (row >> 3) : 2 * ((row & 15) >> 2);
+    const int qx = STRIDE == 1 ? (row & 7) : 2 * (row & 3);
     const uint32_t slot = tmem + g * kSlotCols;
     const uint32_t ts = slot + (static_cast<uint32_t>(32 * wq) << 16);
     uint8_t* sP = sWG + g * C::WG_BYTES;
@@ -335,12 +350,15 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int y0 = by * kBlock - p.halo, x0 = bx * kBlock - p.halo;
       const int y = by * kBlock + qy, x = bx * kBlock + qx;
       const size_t pix = ((static_cast<size_t>(n) * p.H + y) * p.W + x) * C_all + static_cast<size_t>(head) * D;
+      const int OH = p.H / STRIDE, OW = p.W / STRIDE;
+      const size_t opix = ((static_cast<size_t>(n) * OH + y / STRIDE) * OW + x / STRIDE) * C_all +
+                          static_cast<size_t>(head) * D;
       // this query's out and dout rows (for D = dout . out), in flight during the MMAs and pass A
       uint4 orow[D / 8], drow[D / 8];
 #pragma unroll
       for (int e = 0; e < D / 8; ++e) {
-        orow[e] = act ? *reinterpret_cast<const uint4*>(p.out + pix + 8 * e) : make_uint4(0, 0, 0, 0);
-        drow[e] = act ? *reinterpret_cast<const uint4*>(p.dout + pix + 8 * e) : make_uint4(0, 0, 0, 0);
+        orow[e] = live ? *reinterpret_cast<const uint4*>(p.out + opix + 8 * e) : make_uint4(0, 0, 0, 0);
+        drow[e] = live ? *reinterpret_cast<const uint4*>(p.dout + opix + 8 * e) : make_uint4(0, 0, 0, 0);
       }
       // ---- R1: S (warp 0) and G (warp 1), issued in parallel
       if (wq < 2 && lane == 0) {
@@ -364,18 +382,33 @@ __global__ void __launch_bounds__(kThreads, 1)
       // ---- relative logits of this query (log2 units), -inf for masked rows / columns
       float rh[WIN], rw[WIN];
       {
-        float gh[WIN + 1];
-        tmem_ld_exact<WIN + 1>(ts + kGBase + (WIN - 2 - 2 * wq), gh);
+        float gh[WIN + 7];
+        if constexpr (STRIDE == 1) {
+          tmem_ld_exact<WIN + 1>(ts + kGBase + (WIN - 2 - 2 * wq), gh);
+        } else {
+          tmem_ld_exact<WIN + 7>(ts + kGBase + WIN - 8, gh);
+        }
         float a[WIN + 7];
         tmem_ld_exact<WIN + 7>(ts + kGBase + kRelW + WIN - 8, a);
         tmem_wait_ld();
+        if constexpr (STRIDE == 2) {
+          // columns WIN - 8 + i: the query's entry kr - qy + WIN - 1 is i = kr + 7 - qy
+          const int shh = 7 - qy;
+#pragma unroll
+          for (int i = 0; i < WIN + 3; ++i) gh[i] = (shh & 4) ? gh[i + 4] : gh[i];
+#pragma unroll
+          for (int i = 0; i < WIN + 1; ++i) gh[i] = (shh & 2) ? gh[i + 2] : gh[i];
+#pragma unroll
+          for (int i = 0; i < WIN; ++i) gh[i] = (shh & 1) ? gh[i + 1] : gh[i];
+        }
         const bool odd = ((lane >> 3) & 1) != 0;
 #pragma unroll
         for (int kr = 0; kr < WIN; ++kr) {
           const int Y = y0 + kr;
           const bool keep = Y >= 0 && Y < p.H &&
                             (p.kmask == 0 || (kr - qy - p.halo <= (p.kmask >> 1) && qy + p.halo - kr <= (p.kmask >> 1)));
-          rh[kr] = keep ? (odd ? gh[kr] : gh[kr + 1]) * c : -INFINITY;
+          const float gv = STRIDE == 1 ? (odd ? gh[kr] : gh[kr + 1]) : gh[kr];
+          rh[kr] = keep ? gv * c : -INFINITY;
         }
         const int sh = 7 - qx;
 #pragma unroll
@@ -438,6 +471,10 @@ __global__ void __launch_bounds__(kThreads, 1)
           pk[t / 2] = pack_bf16x2(e0, e1);
         }
         if (act) {
+          if (!live) {
+#pragma unroll
+            for (int t = 0; t < 8; ++t) pk[t] = 0u;
+          }
           *reinterpret_cast<uint4*>(sP + pofs(row, J0 / 8)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
           *reinterpret_cast<uint4*>(sP + pofs(row, J0 / 8 + 1)) = make_uint4(pk[4], pk[5], pk[6], pk[7]);
         }
@@ -488,6 +525,10 @@ __global__ void __launch_bounds__(kThreads, 1)
           dk[t / 2] = pack_bf16x2(d0, d1);
         }
         if (act) {
+          if (!live) {
+#pragma unroll
+            for (int t = 0; t < 8; ++t) pk[t] = dk[t] = 0u;
+          }
           *reinterpret_cast<uint4*>(sP + pofs(row, J0 / 8)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
           *reinterpret_cast<uint4*>(sP + pofs(row, J0 / 8 + 1)) = make_uint4(pk[4], pk[5], pk[6], pk[7]);
           *reinterpret_cast<uint4*>(sDS + pofs(row, J0 / 8)) = make_uint4(dk[0], dk[1], dk[2], dk[3]);
@@ -498,6 +539,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (act) {
 #pragma unroll
         for (int u = 0; u < 8; ++u) *reinterpret_cast<uint4*>(sT + swz<128>(row, u)) = make_uint4(0, 0, 0, 0);
+      }
+      if (live) {
 #pragma unroll
         for (int i = 0; i < WIN; ++i) {
           const int ah = i - qy + WIN - 1, aw = kRelW + i - qx + WIN - 1;
@@ -575,13 +618,15 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
           for (int e = 0; e < D; ++e) dqv[e] += dq2[e];
         }
-        if (act) {
+        if (live) {
           uint32_t pk[D / 2];
 #pragma unroll
           for (int e = 0; e < D / 2; ++e) pk[e] = pack_bf16x2(p.s * dqv[2 * e], p.s * dqv[2 * e + 1]);
 #pragma unroll
           for (int e = 0; e < D / 8; ++e)
             reinterpret_cast<uint4*>(p.dq + pix)[e] = make_uint4(pk[4 * e], pk[4 * e + 1], pk[4 * e + 2], pk[4 * e + 3]);
+        }
+        if (act) {
           // dR row = table entry `row` (rows 56..63 stay zero)
 #pragma unroll
           for (int e = 0; e < D; ++e) drel[row * D + e] += p.s * drv[e];
