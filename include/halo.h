@@ -192,7 +192,8 @@ int halo_attn_bwd(const void* q, const void* k, const void* v, const void* rel_h
 
 /* Name of the kernel halo_attn_bwd launches for these arguments (besides
  * zeroing the workspace and the finalize kernel), e.g. "halo_bwd_tc<16,14>"
- * (tensor cores: bf16, block 8, stride 1, dim_head 16 or 32, halo <= 3) or
+ * or, at stride 2, "halo_bwd_tc<32,14,2>" (tensor cores: bf16, block 8,
+ * dim_head 16 or 32, halo <= 3) or
  * "halo_bwd_simt<bf16,64>" (CUDA cores), or "none" when the shape is
  * rejected.  Thread-local storage as for halo_kernel_name; no device work. */
 const char* halo_bwd_kernel_name(int N, int H, int W, int heads, int dim_head, int block, int halo, int stride,
