@@ -123,6 +123,23 @@ def test_kernel_names():
     assert name(1, 16, 16, 2, 32, 5, 1, 1, 0) == "none"
 
 
+def test_bwd_kernel_names():
+    """The backward's kernel choice (host-only): the tensor-core kernel for
+    bf16 8x8 blocks with d 16 or 32 at stride 1 and 2 (the stride-2 form named
+    with its stride), the CUDA-core kernel for every other shape."""
+    lib = _lib()
+    name = lambda *a: lib.halo_bwd_kernel_name(*a).decode()
+    assert name(32, 64, 64, 8, 16, 8, 3, 1, 0, 1) == "halo_bwd_tc<16,14>"
+    assert name(2, 32, 32, 4, 32, 8, 2, 1, 0, 1) == "halo_bwd_tc<32,12>"
+    assert name(64, 64, 64, 8, 32, 8, 3, 2, 0, 1) == "halo_bwd_tc<32,14,2>"
+    assert name(2, 32, 32, 4, 16, 8, 0, 2, 0, 1) == "halo_bwd_tc<16,8,2>"
+    assert name(1, 16, 16, 2, 16, 8, 3, 2, 5, 1) == "halo_bwd_tc<16,14,2>"   # SASA mask
+    assert name(64, 32, 32, 8, 64, 8, 3, 1, 0, 1) == "halo_bwd_simt<bf16,64>"
+    assert name(1, 16, 16, 2, 32, 8, 3, 2, 0, 0) == "halo_bwd_simt<float,32>"
+    assert name(1, 32, 32, 2, 32, 16, 4, 1, 0, 1) == "halo_bwd_simt<bf16,32>"  # block 16
+    assert name(1, 16, 16, 2, 32, 5, 1, 1, 0, 1) == "none"
+
+
 def test_fused_kernel_selection():
     lib = _lib()
     name = lambda *a: lib.halo_fused_kernel_name(*a).decode()
