@@ -14,9 +14,9 @@
 // products are tcgen05 MMAs.
 //
 // Work item = one 8x8 block of one head (stride 2: its 16 strided queries in
-// rows 0-15 of the 64-row tiles, rows 16-63 of Q and dout zero and their P,
-// dS and T rows never written, so they add nothing to dK, dV and dR; the
-// window is the stride-1 one).  Two warpgroups take alternate items,
+// rows 0-15 of the 64-row tiles; the sums over queries take those rows only,
+// and the results of rows 16-63 are not used; the window is the stride-1
+// one).  Two warpgroups take alternate items,
 // each with a 256-column TMEM slot and its own P / dS / T buffers in shared
 // memory; lane 0 of its warps issue its MMAs (independent chains in parallel):
 //   R1  S = Q K^T (M=64, N=w^2 rounded to 8) at slot column 0 and
@@ -102,7 +102,14 @@ struct Cfg {
   static constexpr int KP = (KS + 15) / 16 * 16;       // keys incl. padding: dQ K extent
   static constexpr int KSTEPS = KP / 16;
   static constexpr int MT = (KS + 127) / 128;          // 128-key tiles of dK / dV
-  static constexpr int Q_TILE = 64 * ROWB;
+  // Q and dout tiles: 64 rows at stride 1.  At stride 2 the QR = 16 loaded
+  // rows only (1 KB): the M = 64 MMAs that take Q or dout as their A operand
+  // (S, G, dP) read on into the next tile for rows 16-63, whose results are
+  // never used, and the products summed over queries (dK, dV, dR) take one
+  // K-step of 16 queries.  That halves the stage and fits two.
+  static constexpr int Q_TILE = STRIDE == 1 ? 64 * ROWB : 1024;
+  static constexpr int QKS = QR / 16;                  // K-steps over queries (dK, dV, dR)
+  static_assert(QR * ROWB <= Q_TILE, "query rows in the tile");
   static constexpr int K_TILE = (KP * ROWB + 1023) / 1024 * 1024;
   static constexpr int OFF_Q = 0, OFF_DO = Q_TILE, OFF_K = 2 * Q_TILE, OFF_V = 2 * Q_TILE + K_TILE;
   static constexpr int STAGE_BYTES = 2 * Q_TILE + 2 * K_TILE;
@@ -260,12 +267,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int idx = tid; idx < (C::KP - C::KS) * C::ROWB / 16; idx += kThreads) {
       reinterpret_cast<uint4*>(st + C::OFF_K + C::KS * C::ROWB)[idx] = make_uint4(0, 0, 0, 0);
       reinterpret_cast<uint4*>(st + C::OFF_V + C::KS * C::ROWB)[idx] = make_uint4(0, 0, 0, 0);
-    }
-    // stride 2: Q and dout rows QR..63 (finite, so that the zero P rows
-    // times them stay zero)
-    for (int idx = tid; idx < (64 - C::QR) * C::ROWB / 16; idx += kThreads) {
-      reinterpret_cast<uint4*>(st + C::OFF_Q + C::QR * C::ROWB)[idx] = make_uint4(0, 0, 0, 0);
-      reinterpret_cast<uint4*>(st + C::OFF_DO + C::QR * C::ROWB)[idx] = make_uint4(0, 0, 0, 0);
     }
   }
   fence_proxy_async_smem();
@@ -563,7 +564,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll 1
           for (int t = 0; t < C::MT; ++t)
 #pragma unroll 1
-            for (int ks = 0; ks < 4; ++ks)
+            for (int ks = 0; ks < C::QKS; ++ks)
               mma_f16_ss(slot + col + t * D, smem_desc(aa + t * 16384 + ks * 2048, 8192, 1024, SW_128B),
                          smem_desc(bb + ks * 16 * C::ROWB, 16, C::SBO, C::SW), idKV, ks != 0);
         } else if (wq == 2) {
@@ -576,8 +577,9 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int ks = 0; ks < 4; ++ks) {
             mma_f16_ss(slot + C::COL_DQ2, smem_desc(tA + ks * 32, 16, 1024, SW_128B),
                        smem_desc(ra + ks * 16 * C::ROWB, 16, C::SBO, C::SW), idQ, ks != 0);
-            mma_f16_ss(slot + C::COL_DR, smem_desc(tA + ks * 2048, 8192, 1024, SW_128B),
-                       smem_desc(qa + ks * 16 * C::ROWB, 16, C::SBO, C::SW), idR, ks != 0);
+            if (ks < C::QKS)
+              mma_f16_ss(slot + C::COL_DR, smem_desc(tA + ks * 2048, 8192, 1024, SW_128B),
+                         smem_desc(qa + ks * 16 * C::ROWB, 16, C::SBO, C::SW), idR, ks != 0);
           }
         }
         mma_commit(&bar_r3[g]);
