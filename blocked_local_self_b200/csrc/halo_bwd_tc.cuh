@@ -109,6 +109,14 @@ struct Cfg {
   // K-step of 16 queries.  That halves the stage and fits two.
   static constexpr int Q_TILE = STRIDE == 1 ? 64 * ROWB : 1024;
   static constexpr int QKS = QR / 16;                  // K-steps over queries (dK, dV, dR)
+  // A query row's keys are split between the two threads of its TMEM lane
+  // (tcgen05.ld 16x32bx2): lanes 0-15 take window rows [0, R0), lanes 16-31
+  // rows [R0, WIN), with K0 = R0 * WIN a multiple of 16 so that both halves
+  // run NP pieces of 16 keys whose row / column indices are compile-time.
+  static constexpr int R0 = (WIN == 8) ? 4 : 8;
+  static constexpr int K0 = R0 * WIN;
+  static constexpr int NP = K0 / 16;
+  static_assert(K0 % 16 == 0 && KS - K0 <= K0 && R0 <= WIN, "key split");
   static_assert(QR * ROWB <= Q_TILE, "query rows in the tile");
   static constexpr int K_TILE = (KP * ROWB + 1023) / 1024 * 1024;
   static constexpr int OFF_Q = 0, OFF_DO = Q_TILE, OFF_K = 2 * Q_TILE, OFF_V = 2 * Q_TILE + K_TILE;
@@ -182,6 +190,29 @@ __device__ __forceinline__ void sweep16(uint32_t ts, F&& f) {
   tmem_ld_32x32b_x16(ts, a);
   tmem_wait_ld();
   sweep16_at<0, NS>(ts, a, b, f);
+}
+
+// The same sweep over this thread's half of a row's keys: pieces [J0, J0 + 16)
+// of keys K0 * half + J0 (lanes 16-31 read their partner's TMEM lane at
+// column offset K0), for J0 < 16 * NP.
+template <int J0, int NP, int K0, class F>
+__device__ __forceinline__ void sweep_half_at(uint32_t ts, uint32_t (&cur)[16], uint32_t (&nxt)[16], F& f) {
+  if constexpr (J0 + 16 < 16 * NP) tmem_ld_16x32bx2_x16<K0>(ts + J0 + 16, nxt);
+  float z[16];
+#pragma unroll
+  for (int i = 0; i < 16; ++i) z[i] = __uint_as_float(cur[i]);
+  f(z, std::integral_constant<int, J0>{});
+  if constexpr (J0 + 16 < 16 * NP) {
+    tmem_wait_ld();
+    sweep_half_at<J0 + 16, NP, K0>(ts, nxt, cur, f);
+  }
+}
+template <int NP, int K0, class F>
+__device__ __forceinline__ void sweep_half(uint32_t ts, F&& f) {
+  uint32_t a[16], b[16];
+  tmem_ld_16x32bx2_x16<K0>(ts, a);
+  tmem_wait_ld();
+  sweep_half_at<0, NP, K0>(ts, a, b, f);
 }
 
 // Barrier of one warpgroup's four warps on an mbarrier of count 4, so that
@@ -317,9 +348,13 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int wq = warp & 3;                 // lane quadrant
     const bool act = lane < 16;              // M=64 tiles: rows in lanes 0-15 of each quadrant
     const int row = 16 * wq + (lane & 15);   // query row in the 8x8 block (stride 2: rows 0-15)
-    // this thread's query (stride 2: rows 0-15, warp 0); at stride 2 the
-    // other rows' P, dS and T are written as zeros every item
-    const bool live = act && (STRIDE == 1 || wq == 0);
+    // rows with a query (stride 2: rows 0-15, warp 0); at stride 2 the other
+    // rows' P, dS and T are written as zeros every item.  Both threads of a
+    // TMEM lane work on its row (half = which part of its keys); `live`
+    // marks the one that stores the row's dq.
+    const bool rowlive = STRIDE == 1 || wq == 0;
+    const bool live = act && rowlive;
+    const int half = lane >> 4;
     const int qy = STRIDE == 1 ? (row >> 3) : 2 * ((row & 15) >> 2);
     const int qx = STRIDE == 1 ? (row & 7) : 2 * (row & 3);
     const uint32_t slot = tmem + g * kSlotCols;
@@ -358,8 +393,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       uint4 orow[D / 8], drow[D / 8];
 #pragma unroll
       for (int e = 0; e < D / 8; ++e) {
-        orow[e] = live ? *reinterpret_cast<const uint4*>(p.out + opix + 8 * e) : make_uint4(0, 0, 0, 0);
-        drow[e] = live ? *reinterpret_cast<const uint4*>(p.dout + opix + 8 * e) : make_uint4(0, 0, 0, 0);
+        orow[e] = rowlive ? *reinterpret_cast<const uint4*>(p.out + opix + 8 * e) : make_uint4(0, 0, 0, 0);
+        drow[e] = rowlive ? *reinterpret_cast<const uint4*>(p.dout + opix + 8 * e) : make_uint4(0, 0, 0, 0);
       }
       // ---- R1: S (warp 0) and G (warp 1), issued in parallel
       if (wq < 2 && lane == 0) {
@@ -426,21 +461,35 @@ __global__ void __launch_bounds__(kThreads, 1)
           rw[kc] = keep ? a[kc] * c : -INFINITY;
         }
       }
+      // lanes 16-31 take their partner's (lanes 0-15 hold the row's TMEM lane)
+#pragma unroll
+      for (int i = 0; i < WIN; ++i) {
+        rh[i] = __shfl_sync(0xffffffffu, rh[i], lane & 15);
+        rw[i] = __shfl_sync(0xffffffffu, rw[i], lane & 15);
+      }
+      // this half's window rows: local row r is row r + R0 * half, -inf past the window
+      float rhl[C::R0];
+#pragma unroll
+      for (int r = 0; r < C::R0; ++r) rhl[r] = half ? (r + C::R0 < WIN ? rh[(r + C::R0) % WIN] : -INFINITY) : rh[r];
       // ---- pass A: exact row maximum, per window row max of c S + c rel_w,
-      // then over rows with c rel_h added
+      // then over rows with c rel_h added (keys past the window: rhl = -inf)
       float m = -INFINITY;
       {
-        float rmax[WIN];
+        float rmax[C::R0];
 #pragma unroll
-        for (int r = 0; r < WIN; ++r) rmax[r] = -INFINITY;
-        sweep16<C::NS>(ts, [&](const float (&z)[16], auto jc) {
+        for (int r = 0; r < C::R0; ++r) rmax[r] = -INFINITY;
+        sweep_half<C::NP, C::K0>(ts, [&](const float (&z)[16], auto jc) {
           constexpr int J0 = decltype(jc)::value;
 #pragma unroll
-          for (int t = 0; t < 16; ++t)
-            if (J0 + t < C::KS) rmax[(J0 + t) / WIN] = fmaxf(rmax[(J0 + t) / WIN], fmaf(z[t], c, rw[(J0 + t) % WIN]));
+          for (int t = 0; t < 16; ++t) {
+            // keys past the window in the upper half: their columns may hold stale TMEM
+            const bool tail = half && (J0 + t >= C::KS - C::K0);
+            if (!tail) rmax[(J0 + t) / WIN] = fmaxf(rmax[(J0 + t) / WIN], fmaf(z[t], c, rw[(J0 + t) % WIN]));
+          }
         });
 #pragma unroll
-        for (int r = 0; r < WIN; ++r) m = fmaxf(m, rmax[r] + rh[r]);
+        for (int r = 0; r < C::R0; ++r) m = fmaxf(m, rmax[r] + rhl[r]);
+        m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 16));
       }
       // ---- D = dout . out of this query
       float Dq = 0.f;
@@ -455,31 +504,35 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
       // ---- pass B: p' = 2^(c S + c rel_w + (c rel_h - m)) into the P buffer, row sum
-      float brow[WIN];
+      float brow[C::R0];
 #pragma unroll
-      for (int r = 0; r < WIN; ++r) brow[r] = rh[r] - m;
+      for (int r = 0; r < C::R0; ++r) brow[r] = rhl[r] - m;
+      // this half's first 8-key chunk of the P / dS rows; chunks past the
+      // buffer (keys beyond MT * 128, all outside the window) are not stored
+      const int u0 = half * (C::K0 / 8);
       float l = 0.f;
-      sweep16<C::NS>(ts, [&](const float (&z)[16], auto jc) {
+      sweep_half<C::NP, C::K0>(ts, [&](const float (&z)[16], auto jc) {
         constexpr int J0 = decltype(jc)::value;
         uint32_t pk[8];
 #pragma unroll
         for (int t = 0; t < 16; t += 2) {
-          float e0 = 0.f, e1 = 0.f;
-          if (J0 + t < C::KS) e0 = exp2_mufu(fmaf(z[t], c, rw[(J0 + t) % WIN]) + brow[(J0 + t) / WIN]);
-          if (J0 + t + 1 < C::KS)
-            e1 = exp2_mufu(fmaf(z[t + 1], c, rw[(J0 + t + 1) % WIN]) + brow[(J0 + t + 1) / WIN]);
+          const bool tail0 = half && (J0 + t >= C::KS - C::K0), tail1 = half && (J0 + t + 1 >= C::KS - C::K0);
+          const float e0 = tail0 ? 0.f : exp2_mufu(fmaf(z[t], c, rw[(J0 + t) % WIN]) + brow[(J0 + t) / WIN]);
+          const float e1 =
+              tail1 ? 0.f : exp2_mufu(fmaf(z[t + 1], c, rw[(J0 + t + 1) % WIN]) + brow[(J0 + t + 1) / WIN]);
           l += e0 + e1;
           pk[t / 2] = pack_bf16x2(e0, e1);
         }
-        if (act) {
-          if (!live) {
+        if (!rowlive) {
 #pragma unroll
-            for (int t = 0; t < 8; ++t) pk[t] = 0u;
-          }
-          *reinterpret_cast<uint4*>(sP + pofs(row, J0 / 8)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
-          *reinterpret_cast<uint4*>(sP + pofs(row, J0 / 8 + 1)) = make_uint4(pk[4], pk[5], pk[6], pk[7]);
+          for (int t = 0; t < 8; ++t) pk[t] = 0u;
+        }
+        if (u0 + J0 / 8 < C::MT * 16) {
+          *reinterpret_cast<uint4*>(sP + pofs(row, u0 + J0 / 8)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+          *reinterpret_cast<uint4*>(sP + pofs(row, u0 + J0 / 8 + 1)) = make_uint4(pk[4], pk[5], pk[6], pk[7]);
         }
       });
+      l += __shfl_xor_sync(0xffffffffu, l, 16);
       const float inv_l = 1.0f / l;
       // ---- R2: dP = dout V^T over the S columns
       tc_fence_before();
@@ -497,56 +550,70 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (!ok) break;
       tc_fence_after();
       // ---- pass C: p = p' / l, dS = p (dP - D); bf16 P and dS; row / column sums of dS
-      float rs[WIN], cs[WIN];
+      // (keys past the window have p = 0, hence dS = 0)
+      float rs[C::R0], cs[WIN];
 #pragma unroll
-      for (int i = 0; i < WIN; ++i) rs[i] = cs[i] = 0.f;
-      sweep16<C::NS>(ts, [&](const float (&dp)[16], auto jc) {
+      for (int i = 0; i < C::R0; ++i) rs[i] = 0.f;
+#pragma unroll
+      for (int i = 0; i < WIN; ++i) cs[i] = 0.f;
+      sweep_half<C::NP, C::K0>(ts, [&](const float (&dp)[16], auto jc) {
         constexpr int J0 = decltype(jc)::value;
-        uint4 pv[2];
-        pv[0] = *reinterpret_cast<const uint4*>(sP + pofs(row, J0 / 8));
-        pv[1] = *reinterpret_cast<const uint4*>(sP + pofs(row, J0 / 8 + 1));
+        const bool stored = u0 + J0 / 8 < C::MT * 16;
+        uint4 pv[2] = {make_uint4(0, 0, 0, 0), make_uint4(0, 0, 0, 0)};
+        if (stored) {
+          pv[0] = *reinterpret_cast<const uint4*>(sP + pofs(row, u0 + J0 / 8));
+          pv[1] = *reinterpret_cast<const uint4*>(sP + pofs(row, u0 + J0 / 8 + 1));
+        }
         const __nv_bfloat162* p2 = reinterpret_cast<const __nv_bfloat162*>(pv);
         uint32_t pk[8], dk[8];
 #pragma unroll
         for (int t = 0; t < 16; t += 2) {
           const float2 pp = __bfloat1622float2(p2[t / 2]);
           const float p0 = pp.x * inv_l, p1 = pp.y * inv_l;
-          float d0 = 0.f, d1 = 0.f;
-          if (J0 + t < C::KS) {
-            d0 = p0 * (dp[t] - Dq);
-            rs[(J0 + t) / WIN] += d0;
-            cs[(J0 + t) % WIN] += d0;
-          }
-          if (J0 + t + 1 < C::KS) {
-            d1 = p1 * (dp[t + 1] - Dq);
-            rs[(J0 + t + 1) / WIN] += d1;
-            cs[(J0 + t + 1) % WIN] += d1;
-          }
+          const bool tail0 = half && (J0 + t >= C::KS - C::K0), tail1 = half && (J0 + t + 1 >= C::KS - C::K0);
+          const float d0 = tail0 ? 0.f : p0 * (dp[t] - Dq), d1 = tail1 ? 0.f : p1 * (dp[t + 1] - Dq);
+          rs[(J0 + t) / WIN] += d0;
+          cs[(J0 + t) % WIN] += d0;
+          rs[(J0 + t + 1) / WIN] += d1;
+          cs[(J0 + t + 1) % WIN] += d1;
           pk[t / 2] = pack_bf16x2(p0, p1);
           dk[t / 2] = pack_bf16x2(d0, d1);
         }
-        if (act) {
-          if (!live) {
+        if (!rowlive) {
 #pragma unroll
-            for (int t = 0; t < 8; ++t) pk[t] = dk[t] = 0u;
-          }
-          *reinterpret_cast<uint4*>(sP + pofs(row, J0 / 8)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
-          *reinterpret_cast<uint4*>(sP + pofs(row, J0 / 8 + 1)) = make_uint4(pk[4], pk[5], pk[6], pk[7]);
-          *reinterpret_cast<uint4*>(sDS + pofs(row, J0 / 8)) = make_uint4(dk[0], dk[1], dk[2], dk[3]);
-          *reinterpret_cast<uint4*>(sDS + pofs(row, J0 / 8 + 1)) = make_uint4(dk[4], dk[5], dk[6], dk[7]);
+          for (int t = 0; t < 8; ++t) pk[t] = dk[t] = 0u;
+        }
+        if (stored) {
+          *reinterpret_cast<uint4*>(sP + pofs(row, u0 + J0 / 8)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+          *reinterpret_cast<uint4*>(sP + pofs(row, u0 + J0 / 8 + 1)) = make_uint4(pk[4], pk[5], pk[6], pk[7]);
+          *reinterpret_cast<uint4*>(sDS + pofs(row, u0 + J0 / 8)) = make_uint4(dk[0], dk[1], dk[2], dk[3]);
+          *reinterpret_cast<uint4*>(sDS + pofs(row, u0 + J0 / 8 + 1)) = make_uint4(dk[4], dk[5], dk[6], dk[7]);
         }
       });
-      // T row: rel_h entries kr - qy + w - 1, rel_w entries 28 + kc - qx + w - 1
+#pragma unroll
+      for (int i = 0; i < WIN; ++i) cs[i] += __shfl_xor_sync(0xffffffffu, cs[i], 16);
+      // T row: rel_h entries kr - qy + w - 1 (each half its window rows),
+      // rel_w entries 28 + kc - qx + w - 1 (lanes 0-15)
       if (act) {
 #pragma unroll
         for (int u = 0; u < 8; ++u) *reinterpret_cast<uint4*>(sT + swz<128>(row, u)) = make_uint4(0, 0, 0, 0);
       }
-      if (live) {
+      __syncwarp();
+      if (rowlive) {
 #pragma unroll
-        for (int i = 0; i < WIN; ++i) {
-          const int ah = i - qy + WIN - 1, aw = kRelW + i - qx + WIN - 1;
-          *reinterpret_cast<__nv_bfloat16*>(sT + swz<128>(row, ah >> 3) + (ah & 7) * 2) = __float2bfloat16_rn(rs[i]);
-          *reinterpret_cast<__nv_bfloat16*>(sT + swz<128>(row, aw >> 3) + (aw & 7) * 2) = __float2bfloat16_rn(cs[i]);
+        for (int i = 0; i < C::R0; ++i) {
+          const int kr = i + C::R0 * half;
+          if (kr < WIN) {
+            const int ah = kr - qy + WIN - 1;
+            *reinterpret_cast<__nv_bfloat16*>(sT + swz<128>(row, ah >> 3) + (ah & 7) * 2) = __float2bfloat16_rn(rs[i]);
+          }
+        }
+        if (act) {
+#pragma unroll
+          for (int i = 0; i < WIN; ++i) {
+            const int aw = kRelW + i - qx + WIN - 1;
+            *reinterpret_cast<__nv_bfloat16*>(sT + swz<128>(row, aw >> 3) + (aw & 7) * 2) = __float2bfloat16_rn(cs[i]);
+          }
         }
       }
       fence_proxy_async_smem();
