@@ -164,6 +164,9 @@ CASES += [
 for d in (16, 32):
     for halo in (0, 1, 2, 3):
         CASES.append(dict(N=16, H=32, W=48, heads=8, dim_head=d, block=8, halo=halo, stride=2))
+# four heads (one tile per block), more items than CTAs
+CASES.append(dict(N=8, H=32, W=48, heads=4, dim_head=32, block=8, halo=3, stride=2))
+CASES.append(dict(N=8, H=32, W=48, heads=4, dim_head=16, block=8, halo=2, stride=2))
 
 
 @pytest.mark.parametrize("case", CASES, ids=lambda c: "d{dim_head}_h{halo}_s{stride}_{H}x{W}_n{N}_heads{heads}".format(**c))
