@@ -23,8 +23,11 @@
 //     relative dot products of every query); after the softmax, warps
 //     q < NST of the owning warpgroup each issue a share of O = P V (window
 //     rows of one head) into their own accumulator, summed in the epilogue
-//     (for d = 16 the row sums come from a ones tile appended to V); with
-//     four heads of d = 32 per tile, one chain over all four V tiles.
+//     (for d = 16 the row sums come from a ones tile appended to V).
+//   * four heads of d = 32 per tile (stride 2) go in pairs: q, k, v boxes of
+//     two heads (128-byte rows), Q/K barriers per pair, one A.V chain over
+//     both pair tiles, P in TMEM (A operand of a TMEM-A MMA) and the shared
+//     memory of the P tiles used as a second V buffer.
 //   * warps 0-3 and 4-7 are two softmax warpgroups that take alternate items;
 //     each owns one half of every TMEM lane quadrant (lanes 0-15 or 16-31), so
 //     the MMAs of one item overlap the softmax of the other.  A query row is
@@ -32,8 +35,8 @@
 //     takes the even window rows, its partner the odd ones.
 //   * per row: gather the relative logits that apply to this query from G,
 //     add them, mask out-of-image keys, exact row max, exponentials (part on
-//     the MUFU unit, part as a cubic polynomial on the FMA pipe), bf16 P into
-//     shared memory, then normalise O and store bf16 NHWC directly.
+//     the MUFU unit), bf16 P into shared memory (or TMEM), then normalise O
+//     and store bf16 NHWC directly.
 //   Nothing but q, k, v, the tables and out touches global memory.
 #pragma once
 
