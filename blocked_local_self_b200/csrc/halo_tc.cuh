@@ -173,6 +173,9 @@ struct Cfg {
   static constexpr bool AV_ONE_CHAIN = PAIRED;
   static_assert(!PAIRED || (SPP == 1 && !SUM_BY_MMA), "paired heads: one stream per head");
   static constexpr int NIS = AV_ONE_CHAIN ? 1 : NST;      // A.V issuers (commits per item)
+  // the one chain is issued by warp 11 (otherwise idle), not by a softmax
+  // warp, which would stall on a full MMA queue instead of moving on
+  static constexpr bool AV_WARP = AV_ONE_CHAIN;
   // first O column of a slot: paired, P (8 columns per window row) sits at
   // [0, 8w) and O at [128, 256), over S's tail and G, both read by then
   static constexpr int O_BASE = PAIRED ? 128 : 0;
@@ -262,7 +265,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   __shared__ __align__(8) uint64_t bar_pfull[4];
   __shared__ __align__(8) uint64_t bar_ofull[4];
   __shared__ __align__(8) uint64_t bar_tfree[4];
-  __shared__ __align__(8) uint64_t bar_done[2];
+  __shared__ __align__(8) uint64_t bar_done[3];
   __shared__ uint32_t tmem_base_sh;
   __shared__ int abort_flag;
 
@@ -297,6 +300,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     mbar_init(&bar_done[0], 1);
     mbar_init(&bar_done[1], 1);
+    mbar_init(&bar_done[2], 1);
     abort_flag = 0;
     fence_mbar_init();
   }
@@ -481,6 +485,32 @@ __global__ void __launch_bounds__(kThreads, 1)
       // all issued MMAs complete before the CTA frees TMEM
       mma_commit(&bar_done[is_g ? 1 : 0]);
       mbar_wait(&bar_done[is_g ? 1 : 0], 0, kWaitNs);
+    }
+  } else if (C::AV_WARP && warp == kMmaWarp + 2) {
+    // ------------------------------------------------------------ A.V issue (warp 11)
+    // item k: once its warpgroup has stored P (pfull) and its V has landed,
+    // O = P V as one chain over both pair tiles into the slot's O columns
+    if (lane == 0) {
+      const uint32_t idO = idesc_bf16_f32(64, C::PARTS * D, true);
+      for (int k = 0; k < my_items; ++k) {
+        const int g = k & 1, jj = k >> 1, sl = jj & 1, b = 2 * g + sl;
+        if (!mbar_wait(&bar_pfull[b], (jj >> 1) & 1, kWaitNs, &abort_flag) ||
+            !mbar_wait(&bar_fv[k % (2 * SVB)], (k / (2 * SVB)) & 1, kWaitNs, &abort_flag)) {
+          if (!abort_flag) record_timeout(&abort_flag);
+          break;
+        }
+        tc_fence_after();
+        const uint32_t slot = tmem + (static_cast<uint32_t>(g * 16) << 16) + sl * kSlotCols;
+        const uint32_t va = smem_addr(vbuf(k));
+#pragma unroll 1
+        for (int kk = 0; kk < WIN; ++kk)
+          mma_f16_ts(slot + C::O_BASE, slot + 8 * kk,
+                     smem_desc(va + kk * kRowKeys * C::BROWB, C::V_TILE, C::BSBO, C::BSW), idO, kk != 0);
+        mma_commit(&bar_ofull[b]);
+        mma_commit(&bar_ev[k % SVB]);
+      }
+      mma_commit(&bar_done[2]);
+      mbar_wait(&bar_done[2], 0, kWaitNs);
     }
   }
   __syncwarp();  // reconverge lane 0 with its warp before the aligned barrier
@@ -705,9 +735,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       __syncwarp();
       if (lane == 0) mbar_arrive(&bar_pfull[b]);
-      // ---- A.V: warp wq < NIS issues its share once the whole P tile is written
+      // ---- A.V: warp wq < NIS issues its share once the whole P tile is
+      // written (with AV_WARP, warp 11 does)
       bool issued = true;
-      if (wq < C::NIS && lane == 0) {
+      if (!C::AV_WARP && wq < C::NIS && lane == 0) {
         issued = mbar_wait(&bar_pfull[b], (j >> 1) & 1, kWaitNs, &abort_flag) &&
                  mbar_wait(&bar_fv[k % (2 * SVB)], (k / (2 * SVB)) & 1, kWaitNs, &abort_flag);
         if (issued) {
